@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Hybrid-head layer prefill throughput on B200 (tokens/s) and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+A step is one forward pass of the whole hybrid-head layer (in_proj with the meta
+prepend, x_proj, dt_proj, attention heads, selective scan + gate, branch
+RMSNorm + beta, out_proj) over one batch of the seeded synthetic workload,
+through the C ABI (hymba_layer_fwd).  Default workload: the Hymba-350M-shaped
+layer (B=8, L=2048 + 32 meta tokens, d=1024, bf16).  W untimed warm-up steps,
+then exactly K timed steps, each bracketed by CUDA events on the launching
+stream with an L2 flush (256 MiB memset) between steps outside the events; a
+barrier and a device synchronise on both sides of the timed loop; the time is
+the max over ranks.  Under torchrun every rank runs its own batch (weak
+scaling, no collective on the data path).  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (each
+step a bounded sample of the same workload), as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hybrid_attention_ssm_hymba_b200 import synth  # noqa: E402
+
+METRIC = "hybrid-head layer prefill tokens/s at 1 B200; % of HBM/tensor roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _workload_config(wl: synth.Workload, extra=None):
+    s = wl.first
+    cfg = {"workload": wl.name, "description": wl.description, "batch": s.batch, "seq_len": s.seq_len,
+           "n_meta": s.n_meta, "d_model": s.d_model, "n_q_heads": s.n_q_heads, "n_kv_heads": s.n_kv_heads,
+           "head_dim": s.head_dim, "window": s.window, "d_inner": s.d_inner, "d_state": s.d_state,
+           "dt_rank": s.dt_rank, "n_layers": len(wl.layers), "ffn_dim": s.ffn_dim, "seed": wl.seed}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def _in_proj_flops(s: synth.LayerShape) -> float:
+    return 2.0 * s.d_model * s.n_in * s.batch * s.T
+
+
+# --------------------------------------------------------------------------- clocks (NVML)
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons of one GPU on a thread while active."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x100: "display_clock_setting", 0x10: "sync_boost"}
+
+    def __init__(self, device):
+        self.samples, self.reasons, self.ok = [], set(), False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            try:   # NVML enumerates every GPU; match the CUDA device by UUID
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(torch.cuda.get_device_properties(device).uuid))
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device.index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples), "source": "nvml unavailable" if not self.ok else "nvml"}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+# --------------------------------------------------------------------------- CPU oracle legs
+
+def _oracle_sample(wl: synth.Workload, x, meta, ps, b: int, L: int):
+    """Run the oracle on sequence b, first L tokens, through every layer of the workload."""
+    import dataclasses
+
+    import oracle as O
+    xb = x[b:b + 1, :L]
+    shapes = [dataclasses.replace(s, batch=1, seq_len=L) for s in wl.layers]
+    if wl.first.ffn_dim:
+        return O.stack_forward(xb, meta, ps, shapes)
+    h, kv = O.layer_forward(xb, meta, ps[0], shapes[0])
+    for i in range(1, len(shapes)):
+        h, _ = O.layer_forward(h, None, ps[i], shapes[i], kv_in=kv)
+    return h
+
+
+def _sample_len(wl: synth.Workload) -> int:
+    s = wl.first
+    if s.ffn_dim:
+        return min(s.seq_len, 256)
+    return min(s.seq_len, 2048)
+
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, x, meta, ps, budget_s=12.0):
+    L = _sample_len(wl)
+    done, t0 = 0, time.perf_counter()
+    seqs = []
+    for b in range(wl.first.batch):
+        _oracle_sample(wl, x, meta, ps, b, L)
+        done += L
+        seqs.append(b)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle on sequences {seqs} of the workload, first {L} of "
+                      f"{wl.first.seq_len} user tokens each ({dt:.1f} s wall)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    wl = synth.workload(args.workload)
+    x, meta = synth.layer_inputs(wl)
+    ps = [synth.layer_params(wl, i) for i in range(len(wl.layers))]
+    L = _sample_len(wl)
+    B = wl.first.batch
+    for i in range(args.warmup):
+        _oracle_sample(wl, x, meta, ps, i % B, L)
+    times = []
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_sample(wl, x, meta, ps, i % B, L)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.steps * L / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _workload_config(wl, {"sample_tokens_per_step": L}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
+                             "sample": f"each step: one sequence (rotating), first {L} user tokens, "
+                                       "all layers of the workload, fp64 numpy oracle"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- native (CUDA) leg
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import hybrid_attention_ssm_hymba_b200 as H
+    from hybrid_attention_ssm_hymba_b200 import host
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    wl = synth.workload(args.workload)
+    s0 = wl.first
+    dtype = s0.dtype
+    x_np, meta_np = synth.layer_inputs(wl)
+    ps_np = [synth.layer_params(wl, i) for i in range(len(wl.layers))]
+    dps = [host.params_to_device(p, dtype, dev) for p in ps_np]
+    cfgs = [H.make_cfg(s) for s in wl.layers]
+    weights = [H.make_weights(d) for d in dps]
+    T = s0.T
+    x = host.to_device(x_np, dtype, dev)
+    meta = host.to_device(meta_np, dtype, dev)
+    stack = bool(s0.ffn_dim)
+    ws_bytes = H.hymba_stack_workspace_size(cfgs) if stack else max(H.hymba_workspace_size(c) for c in cfgs)
+    ws = host.workspace(ws_bytes, dev)
+    outs = [torch.empty((s0.batch, T, s0.d_model), dtype=x.dtype, device=dev) for _ in wl.layers]
+    kv = torch.empty((2, s0.batch * T, s0.kv_width), dtype=x.dtype, device=dev) if len(wl.layers) > 1 \
+        and not stack else None
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n_launch_per_step = 7 * len(wl.layers) + (3 * len(wl.layers) + 1 if stack else 0)
+
+    def step(xin, stage_events=None):
+        if stack:
+            H.check(H.hymba_stack_fwd(xin, meta, weights, cfgs, outs[0], ws, stream=stream), "stack")
+            return outs[0]
+        if stage_events is not None:
+            H.check(H.hymba_layer_fwd_events(xin, meta, weights[0], cfgs[0], None, kv, outs[0], ws,
+                                             stage_events, stream=stream), "layer")
+        else:
+            H.check(H.hymba_layer_fwd(xin, meta, weights[0], cfgs[0], None, kv, outs[0], ws, stream=stream),
+                    "layer")
+        for i in range(1, len(wl.layers)):
+            H.check(H.hymba_layer_fwd(outs[i - 1], None, weights[i], cfgs[i], kv, None, outs[i], ws,
+                                      stream=stream), f"layer {i}")
+        return outs[-1]
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(x)
+    torch.cuda.synchronize(dev)
+    assert H.hymba_workspace_status(ws, stream) == H.HYMBA_OK
+
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)] if not stack else None
+    sampler = ClockSampler(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        for k in range(K):
+            flush.zero_()
+            ev_s[k].record(stream)
+            step(x, stage_ev[k] if stage_ev else None)
+            ev_e[k].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    step_ms = [ev_s[k].elapsed_time(ev_e[k]) for k in range(K)]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    status = H.hymba_workspace_status(ws, stream)
+    tokens_per_step = s0.batch * s0.seq_len
+    value = world * K * tokens_per_step / (total_ms * 1e-3)
+
+    peaks, peak_src = _peaks()
+    roofline, stages = None, None
+    if stage_ev:
+        per_stage = {name: float(np.mean([stage_ev[k][i].elapsed_time(stage_ev[k][i + 1]) for k in range(K)]))
+                     for i, name in enumerate(H.STAGES)}
+        stages = {n: round(v * 1e3, 2) for n, v in per_stage.items()}  # microseconds
+        t_in = per_stage["in_proj"] * 1e-3
+        ach = _in_proj_flops(s0) / t_in / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roofline = {"kernel": "in_proj gemm_bf16_tc (tcgen05)", "bound": "tensor", "achieved": round(ach, 1),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                    "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a continuous loop)",
+                    "in_proj_us": round(per_stage["in_proj"] * 1e3, 2),
+                    "algorithmic_flops_per_launch": _in_proj_flops(s0)}
+
+    e2e = None
+    if not args.no_e2e:
+        xh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+        xh.copy_(x.cpu())
+        oh = torch.empty(outs[-1].shape, dtype=x.dtype).pin_memory()
+        xd = torch.empty_like(x)
+        n_e2e = max(3, min(K, 50))
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e + 1)]
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e + 1)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        for k in range(n_e2e + 1):   # the first iteration warms the copy path, untimed
+            flush.zero_()
+            es[k].record(stream)
+            xd.copy_(xh, non_blocking=True)
+            o = step(xd)
+            oh.copy_(o, non_blocking=True)
+            ee[k].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = float(sum(es[k].elapsed_time(ee[k]) for k in range(1, n_e2e + 1)))
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * n_e2e * tokens_per_step / (e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+               "d2h_bytes_per_step": oh.numel() * oh.element_size(), "steps": n_e2e,
+               "path": "pinned host x -> device, hymba_layer_fwd, device out -> pinned host"}
+
+    line = None
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+                "config": _workload_config(wl, {
+                    "parallelism": f"replicas x{world} (batch per rank, no collective)" if world > 1 else "1 GPU",
+                    "tokens_per_step_per_gpu": tokens_per_step, "rows_per_step_per_gpu": s0.batch * T,
+                    "l2": "flushed between timed steps (256 MiB memset outside the events)"}),
+                "roofline": roofline, "stages_us": stages, "e2e": e2e,
+                "gpu_launches": n_launch_per_step * K, "clocks": sampler.summary(),
+                "device_status": H.hymba_status_string(status)}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, x_np, meta_np, ps_np)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="hymba350m_layer", choices=synth.WORKLOAD_ORDER)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        print("note: fewer than 3 warm-up steps requested", file=sys.stderr)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_native(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

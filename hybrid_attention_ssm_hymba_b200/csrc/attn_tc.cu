@@ -1,0 +1,398 @@
+// attn_tc.cu -- attention heads of the hybrid-head layer on the sm_100a tensor cores
+// (blog.outta.ai Hymba review, "Design formulation": Y_attn = softmax(Q K^T) V;
+// "Combine global and local attention": sliding-window attention in most layers;
+// "Meta Tokens": the meta tokens stay visible to every query).  A query i of a
+// sequence sees key j iff j <= i and (window < 0 or i - j <= window or j < n_meta);
+// query head h reads K/V head h / (Hq / Hkv) (GQA).  Scale 1/sqrt(head_dim).
+//
+// One CTA per (128-query tile, query head, sequence); 192 threads:
+//   warp 0      TMA producer: Q once, then K_j and V_j into two 2-deep rings
+//   warp 1      TMEM allocator + UMMA issuer: S_j = Q K_j^T into one of two TMEM
+//               S buffers (issued two blocks ahead), O_j = P_j V_j into TMEM
+//   warps 2..5  softmax: one query row per thread; fp32 row max and sum; P_j in bf16
+//               into swizzled smem (the A operand of P V); O accumulated in registers
+//               with the online-softmax rescale; final O / l stored as bf16.
+// K/V blocks with no visible pair are never loaded: the block list is the meta
+// blocks plus the window blocks.  Only blocks that straddle the mask boundary pay
+// for the elementwise mask.
+#include "hy_common.cuh"
+#include "hy_kernels.h"
+
+namespace hy {
+namespace {
+
+constexpr int BQ = 128, BKV = 128, DH = 128;
+constexpr int TILE_BYTES = 128 * DH * 2;  // 32 KB: a [128 x 128] bf16 tile = 2 swizzled 64-column halves
+constexpr int HALF = 128 * 64 * 2;        // 16 KB
+constexpr int SMEM_BYTES = 6 * TILE_BYTES + 1024 + 256;
+constexpr uint32_t IDESC_QK = idesc_bf16(BQ, BKV, false, false);  // A=Q (K-major), B=K (K-major)
+constexpr uint32_t IDESC_PV = idesc_bf16(BQ, DH, false, true);    // A=P (K-major), B=V (MN-major)
+
+struct AttnParams {
+  int T, Hq, Hkv, n_meta, window;
+  int q_tiles;
+  __nv_bfloat16* out;
+  long long out_ld;
+  float scale_log2;  // log2(e) / sqrt(dh)
+  unsigned* status;
+};
+
+struct BlockList {
+  int first, wlo, n;  // blocks [0, first) then [wlo, wlo + n - first)
+  __device__ __forceinline__ int block(int idx) const { return idx < first ? idx : wlo + (idx - first); }
+};
+
+__device__ __forceinline__ BlockList make_blocks(const AttnParams& p, int q0) {
+  BlockList bl;
+  const int last_row = min(q0 + BQ - 1, p.T - 1);
+  const int hi = last_row / BKV;
+  if (p.window < 0) {
+    bl.first = 0;
+    bl.wlo = 0;
+  } else {
+    const int mb = (p.n_meta + BKV - 1) / BKV;
+    bl.wlo = max(0, q0 - p.window) / BKV;
+    bl.first = min(mb, bl.wlo);
+  }
+  bl.n = bl.first + (hi - bl.wlo + 1);
+  return bl;
+}
+
+__device__ __forceinline__ bool visible(int i, int j, int n_meta, int window) {
+  return j <= i && (window < 0 || i - j <= window || j < n_meta);
+}
+
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* sQ = smem_raw + pad;
+  uint8_t* sK = sQ + TILE_BYTES;            // 2 stages
+  uint8_t* sV = sK + 2 * TILE_BYTES;        // 2 stages
+  uint8_t* sP = sV + 2 * TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + TILE_BYTES);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* k_empty = bars + 3;  // [2]
+  uint64_t* v_full = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;  // [2]
+  uint64_t* s_full = bars + 9;   // [2]
+  uint64_t* s_free = bars + 11;  // [2]
+  uint64_t* p_full = bars + 13;
+  uint64_t* o_full = bars + 14;
+  uint64_t* mma_done = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = p.q_tiles - 1 - static_cast<int>(blockIdx.x);  // longest tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (p.Hq / p.Hkv);
+  const int q0 = qt * BQ;
+  const BlockList bl = make_blocks(p, q0);
+  const int n = bl.n;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(o_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch(&tmQ);
+    tma_prefetch(&tmK);
+    tma_prefetch(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tS = tmem_base, tO = tmem_base + 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- producer
+      uint32_t k_iss = 0, v_iss = 0, k_par = 0, v_par = 0;
+      bool ok = true;
+      mbar_arrive_expect_tx(q_full, TILE_BYTES);
+      tma_load_3d(sQ, &tmQ, q_full, h * DH, q0, b);
+      tma_load_3d(sQ + HALF, &tmQ, q_full, h * DH + 64, q0, b);
+      auto issue_k = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&k_empty[s], ((j >> 1) & 1) ^ 1u, p.status, abort_flag)) return false;
+        mbar_arrive_expect_tx(&k_full[s], TILE_BYTES);
+        const int k0 = bl.block(j) * BKV;
+        tma_load_3d(sK + s * TILE_BYTES, &tmK, &k_full[s], kvh * DH, k0, b);
+        tma_load_3d(sK + s * TILE_BYTES + HALF, &tmK, &k_full[s], kvh * DH + 64, k0, b);
+        k_iss |= 1u << s;
+        k_par = (k_par & ~(1u << s)) | (static_cast<uint32_t>((j >> 1) & 1) << s);
+        return true;
+      };
+      auto issue_v = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&v_empty[s], ((j >> 1) & 1) ^ 1u, p.status, abort_flag)) return false;
+        mbar_arrive_expect_tx(&v_full[s], TILE_BYTES);
+        const int k0 = bl.block(j) * BKV;
+        tma_load_3d(sV + s * TILE_BYTES, &tmV, &v_full[s], kvh * DH, k0, b);
+        tma_load_3d(sV + s * TILE_BYTES + HALF, &tmV, &v_full[s], kvh * DH + 64, k0, b);
+        v_iss |= 1u << s;
+        v_par = (v_par & ~(1u << s)) | (static_cast<uint32_t>((j >> 1) & 1) << s);
+        return true;
+      };
+      // consumption order of the UMMA issuer: K0 K1 V0 K2 V1 K3 V2 ...
+      int kj = 0, vj = 0;
+      while (ok && kj < n && kj < 2) ok = issue_k(kj++);
+      while (ok && vj < n) {
+        ok = issue_v(vj++);
+        if (ok && kj < n) ok = issue_k(kj++);
+      }
+      int never = 0;
+      // drain: every issued copy lands before the CTA may exit
+      for (int s = 0; s < 2; ++s) {
+        if (k_iss & (1u << s)) mbar_wait(&k_full[s], (k_par >> s) & 1u, nullptr, &never, 100000000ull);
+        if (v_iss & (1u << s)) mbar_wait(&v_full[s], (v_par >> s) & 1u, nullptr, &never, 100000000ull);
+      }
+      mbar_wait(q_full, 0, nullptr, &never, 100000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- UMMA issuer
+      bool ok = mbar_wait(q_full, 0, p.status, abort_flag);
+      const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        if (!mbar_wait(&k_full[s], par, p.status, abort_flag)) return false;
+        if (!mbar_wait(&s_free[s], par ^ 1u, p.status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sK + s * TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
+          umma_bf16_ss(tS + s * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
+                       IDESC_QK, k != 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[s]);
+        umma_commit(&k_empty[s]);
+        return true;
+      };
+      if (ok && n > 0) ok = issue_s(0);
+      if (ok && n > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < n; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(p_full, j & 1, p.status, abort_flag)) break;
+        if (!mbar_wait(&v_full[s], (j >> 1) & 1, p.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sV + s * TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < BKV / 16; ++k) {
+          const uint32_t a_off = (k >> 2) * HALF + (k & 3) * 32;  // P: K-major, keys 16k..16k+15
+          const uint32_t b_off = k * 16 * 128;                      // V: MN-major, key rows 16k..
+          umma_bf16_ss(tO, sdesc_sw128(p_addr + a_off, 16, 1024), sdesc_sw128(v_addr + b_off, HALF, 1024), IDESC_PV,
+                       k != 0 ? 1u : 0u);
+        }
+        umma_commit(o_full);
+        umma_commit(&v_empty[s]);
+        if (j + 2 < n) ok = issue_s(j + 2);
+      }
+      umma_commit(mma_done);
+      int never = 0;
+      mbar_wait(mma_done, 0, nullptr, &never, 100000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int i = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    float o_acc[DH];
+#pragma unroll
+    for (int d = 0; d < DH; ++d) o_acc[d] = 0.f;
+    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+    bool ok = true;
+    uint8_t* prow = sP + r * 128;
+    for (int j = 0; j < n; ++j) {
+      const int s = j & 1;
+      const int k0 = bl.block(j) * BKV;
+      const bool need_mask =
+          !((k0 + BKV - 1 <= q0) && (p.window < 0 || q0 + BQ - 1 - k0 <= p.window || k0 + BKV - 1 < p.n_meta));
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[s], (j >> 1) & 1, p.status, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sbase = tS + s * 128 + lane_off;
+      // pass 1: row max over the visible keys of this block
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(sbase + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float sv = __uint_as_float(v[e]);
+          const bool vis = !need_mask || visible(i, k0 + c * 32 + e, p.n_meta, p.window);
+          mx = vis ? fmaxf(mx, sv) : mx;
+        }
+      }
+      const float m_new = fmaxf(m, mx * p.scale_log2);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = exp2f(m - m_use);
+      // fold in the previous block's P V (its smem P and TMEM O are then free)
+      if (j > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(o_full, (j - 1) & 1, p.status, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tO + lane_off + c * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o_acc[c * 32 + e] = fmaf(o_acc[c * 32 + e], alpha_prev, __uint_as_float(v[e]));
+        }
+      }
+      // pass 2: P = exp2(s * scale_log2 - m) in bf16 into the swizzled P tile
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(sbase + c * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const bool v0 = !need_mask || visible(i, k0 + c * 32 + e, p.n_meta, p.window);
+          const bool v1 = !need_mask || visible(i, k0 + c * 32 + e + 1, p.n_meta, p.window);
+          const float p0 = v0 ? exp2f(fmaf(__uint_as_float(v[e]), p.scale_log2, -m_use)) : 0.f;
+          const float p1 = v1 ? exp2f(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -m_use)) : 0.f;
+          sum += p0 + p1;
+          pk[e >> 1] = pack_bf16(p0, p1);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = c * 4 + q;  // 16-byte chunk = keys 8*chunk .. 8*chunk+7
+          uint8_t* dst = prow + (chunk >> 3) * HALF + (((chunk & 7) ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[s]);
+      fence_proxy_async_smem();
+      mbar_arrive(p_full);
+      l = fmaf(l, alpha, sum);
+      m = m_new;
+      alpha_prev = alpha;
+    }
+    if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(o_full, (n - 1) & 1, p.status, abort_flag))) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + lane_off + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o_acc[c * 32 + e] = fmaf(o_acc[c * 32 + e], alpha_prev, __uint_as_float(v[e]));
+      }
+      if (i < p.T) {
+        const float inv = 1.f / l;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(b) * p.T + i) * p.out_ld + h * DH);
+#pragma unroll
+        for (int q = 0; q < DH / 8; ++q)
+          dst[q] = make_uint4(pack_bf16(o_acc[8 * q] * inv, o_acc[8 * q + 1] * inv),
+                              pack_bf16(o_acc[8 * q + 2] * inv, o_acc[8 * q + 3] * inv),
+                              pack_bf16(o_acc[8 * q + 4] * inv, o_acc[8 * q + 5] * inv),
+                              pack_bf16(o_acc[8 * q + 6] * inv, o_acc[8 * q + 7] * inv));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn attn_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D bf16 map over [batch][T][cols] with row stride ld elements; box = 64 cols x 128 rows x 1.
+bool map_rows(CUtensorMap* m, const void* base, long long cols, long long ld, int T, int batch) {
+  EncodeTiledFn fn = attn_encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(batch)};
+  cuuint64_t gs[2] = {static_cast<cuuint64_t>(ld) * 2, static_cast<cuuint64_t>(ld) * 2 * T};
+  cuuint32_t bx[3] = {64, 128, 1}, es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gd, gs, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_attention_f32(const AttnDesc& a, cudaStream_t st);
+
+cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st) {
+  if (!a.bf16) return launch_attention_f32(a, st);
+  if (a.batch <= 0 || a.T <= 0) return cudaSuccess;
+  static int attr_dev_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 31 && !(attr_dev_mask & (1 << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_dev_mask |= 1 << dev;
+  }
+  CUtensorMap tq, tk, tv;
+  if (!map_rows(&tq, a.q, static_cast<long long>(a.n_q_heads) * DH, a.q_ld, a.T, a.batch)) return cudaErrorInvalidValue;
+  if (!map_rows(&tk, a.k, static_cast<long long>(a.n_kv_heads) * DH, a.kv_ld, a.T, a.batch))
+    return cudaErrorInvalidValue;
+  if (!map_rows(&tv, a.v, static_cast<long long>(a.n_kv_heads) * DH, a.kv_ld, a.T, a.batch))
+    return cudaErrorInvalidValue;
+  AttnParams p{};
+  p.T = a.T;
+  p.Hq = a.n_q_heads;
+  p.Hkv = a.n_kv_heads;
+  p.n_meta = a.n_meta;
+  p.window = a.window;
+  p.q_tiles = (a.T + BQ - 1) / BQ;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.out_ld = a.out_ld;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(DH));
+  p.status = a.status;
+  dim3 grid(p.q_tiles, a.n_q_heads, a.batch);
+  attn_fwd_tc<<<grid, 192, SMEM_BYTES, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace hy

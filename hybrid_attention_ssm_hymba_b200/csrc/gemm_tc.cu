@@ -1,0 +1,478 @@
+// gemm_tc.cu -- bf16 GEMM C = A W^T on the sm_100a tensor cores (tcgen05.mma, fp32
+// accumulators in TMEM), operands staged by TMA with 128-byte swizzle, no cluster
+// multicast.  Used for the fused in_proj W_in_proj = [W_Q, W_K, W_V, W_SSM, W_G],
+// x_proj, dt_proj and out_proj of the hybrid-head layer, and the SwiGLU FFN of the
+// stacked blocks (blog.outta.ai Hymba review, "Design formulation"; metaphor-xennon
+// page, "层配置": intermediate_size).
+//
+// Kernel shape: persistent, one CTA per SM, 192 threads:
+//   warp 0      TMA producer (one thread) -> STAGES-deep smem ring (full/empty mbarriers)
+//   warp 1      TMEM allocator + UMMA issuer (one thread), 128 x BN x 16 per instruction
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows, fused elementwise op,
+//               vector stores.  Two TMEM accumulators so the epilogue of tile i
+//               overlaps the mainloop of tile i+1.
+//
+// "Meta mode" reads the rows of X~_b = [meta; x_b] for each sequence b straight from
+// the meta tokens [M, K] and the user tokens x [B, L, K]: a 128-row tile that holds
+// meta rows gets them from the meta tensor map and the rest from x, into the same
+// swizzled smem tile, so the meta prepend costs no copy.
+#include <cstdio>
+#include <mutex>
+
+#include "hy_common.cuh"
+#include "hy_kernels.h"
+
+namespace hy {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int A_STAGE = BM * BK * 2;  // 16 KB
+
+struct GemmParams {
+  int meta_mode;
+  long long a_rows;  // plain mode: rows of A
+  int batch, T, n_meta;
+  int m_tiles;  // per sequence (meta mode) or in total (plain mode)
+  int n_tiles, k_blocks, N;
+  int epi;
+  int nseg;
+  Seg seg[kMaxSegs];
+  const __nv_bfloat16* resid;
+  long long resid_ld;
+  __nv_bfloat16* out;
+  long long out_ld;
+  int swiglu_F;
+  unsigned* status;
+};
+
+template <int BN>
+struct Cfg {
+  static constexpr int B_STAGE = BN * BK * 2;
+  static constexpr int STAGE = A_STAGE + B_STAGE;
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static constexpr uint32_t IDESC = idesc_bf16(BM, BN, false, false);
+};
+
+struct TileCoord {
+  int b, m, n;
+};
+__device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int tile) {
+  TileCoord c;
+  const int per_b = p.m_tiles * p.n_tiles;
+  c.b = p.meta_mode ? tile / per_b : 0;
+  const int r = p.meta_mode ? tile - c.b * per_b : tile;
+  c.m = r / p.n_tiles;
+  c.n = r - c.m * p.n_tiles;
+  return c;
+}
+
+// Store 16 consecutive accumulator columns [c0, c0 + 16) of one output row.
+__device__ __forceinline__ void store16(const GemmParams& p, long long row, int c0, const uint32_t* v) {
+  int s = 0;
+  while (s + 1 < p.nseg && c0 >= p.seg[s].col1) ++s;
+  const Seg& sg = p.seg[s];
+  if (c0 < sg.col0 || c0 >= sg.col1) return;
+  float f[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]);
+  if (sg.op == SEG_SILU) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) f[i] = silu_f(f[i]);
+  } else if (sg.op == SEG_SOFTPLUS_BIAS) {
+    const float4* bb = reinterpret_cast<const float4*>(sg.bias + (c0 - sg.col0));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 b4 = bb[j];
+      f[4 * j + 0] = softplus_f(f[4 * j + 0] + b4.x);
+      f[4 * j + 1] = softplus_f(f[4 * j + 1] + b4.y);
+      f[4 * j + 2] = softplus_f(f[4 * j + 2] + b4.z);
+      f[4 * j + 3] = softplus_f(f[4 * j + 3] + b4.w);
+    }
+  }
+  const long long off = row * sg.ld + (c0 - sg.col0);
+  if (sg.out_f32) {
+    float4* d = reinterpret_cast<float4*>(static_cast<float*>(sg.ptr) + off);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) d[j] = make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(sg.ptr) + off);
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      d[j] = make_uint4(pack_bf16(f[8 * j], f[8 * j + 1]), pack_bf16(f[8 * j + 2], f[8 * j + 3]),
+                        pack_bf16(f[8 * j + 4], f[8 * j + 5]), pack_bf16(f[8 * j + 6], f[8 * j + 7]));
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAx2,
+                 const __grid_constant__ CUtensorMap tmM1, const __grid_constant__ CUtensorMap tmM2,
+                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ GemmParams p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* sA = smem_raw + pad;
+  uint8_t* sB = sA + C::STAGES * A_STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_STAGE);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmB);
+    if (p.meta_mode) {
+      tma_prefetch(&tmAx2);
+      tma_prefetch(&tmM1);
+      tma_prefetch(&tmM2);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int total = (p.meta_mode ? p.batch : 1) * p.m_tiles * p.n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const TileCoord tc = decode_tile(p, tile);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint64_t* fb = &full[stage];
+          mbar_arrive_expect_tx(fb, C::STAGE);
+          const int kx = kb * BK;
+          uint8_t* a_dst = sA + stage * A_STAGE;
+          if (p.meta_mode) {
+            const int r0 = tc.m * BM;
+            int mc = p.n_meta - r0;
+            mc = mc < 0 ? 0 : (mc > BM ? BM : mc);
+            if (mc == BM) {
+              tma_load_2d(a_dst, &tmM1, fb, kx, r0);
+            } else if (mc > 0) {
+              tma_load_2d(a_dst, &tmM2, fb, kx, r0);
+              tma_load_3d(a_dst + mc * 128, &tmAx2, fb, kx, 0, tc.b);
+            } else {
+              tma_load_3d(a_dst, &tmA, fb, kx, r0 - p.n_meta, tc.b);
+            }
+          } else {
+            tma_load_2d(a_dst, &tmA, fb, kx, tc.m * BM);
+          }
+          uint8_t* b_dst = sB + stage * C::B_STAGE;
+          if (p.epi == EPI_SWIGLU) {
+            tma_load_2d(b_dst, &tmB, fb, kx, tc.n * 128);
+            tma_load_2d(b_dst + 128 * 128, &tmB, fb, kx, p.swiglu_F + tc.n * 128);
+          } else {
+            tma_load_2d(b_dst, &tmB, fb, kx, tc.n * BN);
+          }
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {  // let our own bulk copies land before the CTA's smem goes away
+        int never = 0;
+        for (int s = 0; s < C::STAGES; ++s)
+          if (issued & (1u << s)) mbar_wait(&full[s], (last_par >> s) & 1u, nullptr, &never, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ UMMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const uint32_t use = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], use ^ 1u, p.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16_ss(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024), sdesc_sw128(b0 + k * 32, 16, 1024), C::IDESC,
+                         (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[buf]);
+      }
+      umma_commit(mma_done);  // all our MMAs finished before TMEM is freed
+      int never = 0;
+      mbar_wait(mma_done, 0, nullptr, &never, 100000000ull);
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int r = quad * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t use = (it >> 1) & 1;
+      // warp-uniform exit: tcgen05.ld below is a warp-collective instruction
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], use, p.status, abort_flag))) break;
+      tc_fence_after();
+      const TileCoord tc = decode_tile(p, tile);
+      long long grow;
+      bool valid;
+      if (p.meta_mode) {
+        const int t = tc.m * BM + r;
+        valid = t < p.T;
+        grow = static_cast<long long>(tc.b) * p.T + t;
+      } else {
+        grow = static_cast<long long>(tc.m) * BM + r;
+        valid = grow < p.a_rows;
+      }
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * BN;
+      if (p.epi == EPI_SEGMENTS) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tb + c * 32, v);
+          tmem_wait_ld();
+          const int col = tc.n * BN + c * 32;
+          if (valid) {
+            if (col < p.N) store16(p, grow, col, v);
+            if (col + 16 < p.N) store16(p, grow, col + 16, v + 16);
+          }
+        }
+      } else if (p.epi == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tb + c * 32, g);
+          tmem_ld32(tb + 128 + c * 32, u);
+          tmem_wait_ld();
+          if (valid) {
+            uint4* d = reinterpret_cast<uint4*>(p.out + grow * p.out_ld + tc.n * 128 + c * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float f[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) f[i] = silu_f(__uint_as_float(g[8 * j + i])) * __uint_as_float(u[8 * j + i]);
+              d[j] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                                pack_bf16(f[6], f[7]));
+            }
+          }
+        }
+      } else {  // EPI_RESIDUAL
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tb + c * 32, v);
+          tmem_wait_ld();
+          const int col = tc.n * BN + c * 32;
+          if (valid && col < p.N) {
+            const uint4* rs = reinterpret_cast<const uint4*>(p.resid + grow * p.resid_ld + col);
+            uint4* d = reinterpret_cast<uint4*>(p.out + grow * p.out_ld + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 q = rs[j];
+              const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+              uint32_t o[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                o[i] = pack_bf16(bf16lo(qq[i]) + __uint_as_float(v[8 * j + 2 * i]),
+                                 bf16hi(qq[i]) + __uint_as_float(v[8 * j + 2 * i + 1]));
+              d[j] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor map, innermost dimension first; 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+              const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
+  using C = Cfg<BN>;
+  static bool attr_done = false;  // per process; all B200s share the attribute value
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  CUtensorMap tmA, tmAx2, tmM1, tmM2, tmB;
+  const uint64_t K = static_cast<uint64_t>(g.K);
+  GemmParams p{};
+  if (g.meta_mode) {
+    const int M = g.n_meta, r = M % BM;
+    uint64_t dx[3] = {K, static_cast<uint64_t>(g.L), static_cast<uint64_t>(g.batch)};
+    uint64_t sx[2] = {K * 2, K * 2 * static_cast<uint64_t>(g.L)};
+    uint32_t bx[3] = {BK, BM, 1};
+    if (!make_map(&tmA, g.x, 3, dx, sx, bx)) return cudaErrorInvalidValue;
+    tmAx2 = tmA;
+    tmM1 = tmA;
+    tmM2 = tmA;
+    if (r != 0) {
+      uint32_t bx2[3] = {BK, static_cast<uint32_t>(BM - r), 1};
+      if (!make_map(&tmAx2, g.x, 3, dx, sx, bx2)) return cudaErrorInvalidValue;
+    }
+    if (M > 0) {
+      uint64_t dm[2] = {K, static_cast<uint64_t>(M)};
+      uint64_t sm[1] = {K * 2};
+      uint32_t bm1[2] = {BK, BM};
+      if (!make_map(&tmM1, g.meta, 2, dm, sm, bm1)) return cudaErrorInvalidValue;
+      if (r != 0) {
+        uint32_t bm2[2] = {BK, static_cast<uint32_t>(r)};
+        if (!make_map(&tmM2, g.meta, 2, dm, sm, bm2)) return cudaErrorInvalidValue;
+      }
+    }
+    p.meta_mode = 1;
+    p.batch = g.batch;
+    p.T = g.L + g.n_meta;
+    p.n_meta = g.n_meta;
+    p.m_tiles = (p.T + BM - 1) / BM;
+    p.a_rows = static_cast<long long>(g.batch) * p.T;
+  } else {
+    uint64_t da[2] = {K, static_cast<uint64_t>(g.a_rows)};
+    uint64_t sa[1] = {K * 2};
+    uint32_t ba[2] = {BK, BM};
+    if (!make_map(&tmA, g.a, 2, da, sa, ba)) return cudaErrorInvalidValue;
+    tmAx2 = tmA;
+    tmM1 = tmA;
+    tmM2 = tmA;
+    p.meta_mode = 0;
+    p.batch = 1;
+    p.a_rows = g.a_rows;
+    p.m_tiles = static_cast<int>((g.a_rows + BM - 1) / BM);
+  }
+  {
+    uint64_t dw[2] = {K, static_cast<uint64_t>(g.N)};
+    uint64_t sw[1] = {K * 2};
+    uint32_t bw[2] = {BK, static_cast<uint32_t>(g.epi == EPI_SWIGLU ? 128 : BN)};
+    if (!make_map(&tmB, g.w, 2, dw, sw, bw)) return cudaErrorInvalidValue;
+  }
+  p.N = g.N;
+  p.n_tiles = (g.epi == EPI_SWIGLU) ? g.swiglu_F / 128 : (g.N + BN - 1) / BN;
+  p.k_blocks = (g.K + BK - 1) / BK;
+  p.epi = g.epi;
+  p.nseg = g.nseg;
+  for (int i = 0; i < g.nseg; ++i) p.seg[i] = g.seg[i];
+  p.resid = static_cast<const __nv_bfloat16*>(g.resid);
+  p.resid_ld = g.resid_ld;
+  p.out = static_cast<__nv_bfloat16*>(g.out);
+  p.out_ld = g.out_ld;
+  p.swiglu_F = g.swiglu_F;
+  p.status = g.status;
+  const long long total = static_cast<long long>(p.meta_mode ? p.batch : 1) * p.m_tiles * p.n_tiles;
+  if (total <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(total < num_sms() ? total : num_sms());
+  gemm_bf16_tc<BN><<<grid, 192, C::SMEM, st>>>(tmA, tmAx2, tmM1, tmM2, tmB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_bf16(const GemmDesc& g, cudaStream_t st) {
+  if (g.epi == EPI_SWIGLU || g.N > 128) return launch_bn<256>(g, st);
+  return launch_bn<128>(g, st);
+}
+
+int num_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+}  // namespace hy

@@ -1,0 +1,85 @@
+// hy_kernels.h -- host-side launchers of the library's kernels (internal; the public
+// C ABI is include/hymba.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hy {
+
+// One column segment of a GEMM output: columns [col0, col1) of the product go to
+// ptr + row * ld + (col - col0), optionally through an elementwise op.
+enum SegOp : int { SEG_STORE = 0, SEG_SILU = 1, SEG_SOFTPLUS_BIAS = 2 };
+struct Seg {
+  int col0, col1;
+  void* ptr;
+  long long ld;
+  int out_f32;         // 1: fp32 output, 0: the GEMM's dtype
+  int op;              // SegOp
+  const float* bias;   // SEG_SOFTPLUS_BIAS: bias[col - col0]
+};
+constexpr int kMaxSegs = 6;
+
+enum EpiKind : int {
+  EPI_SEGMENTS = 0,  // column segments (in_proj, x_proj, dt_proj, plain GEMMs)
+  EPI_SWIGLU = 1,    // out[:, j] = SiLU(acc[:, j]) * acc[:, F + j]   (W rows: gate then up)
+  EPI_RESIDUAL = 2   // out = resid + acc  (resid may alias out)
+};
+
+struct GemmDesc {
+  // A operand: plain [a_rows, K] row-major, or "meta mode": the rows of
+  // X~_b = [meta; x_b] for every sequence b, read straight from meta [M, K] and
+  // x [batch, L, K] (the meta tokens are never copied).
+  bool meta_mode = false;
+  const void* a = nullptr;
+  long long a_rows = 0;
+  const void* x = nullptr;
+  const void* meta = nullptr;
+  int batch = 0, L = 0, n_meta = 0;
+  int K = 0;
+  // B operand W [N, K] row-major
+  const void* w = nullptr;
+  int N = 0;
+  // epilogue
+  int epi = EPI_SEGMENTS;
+  int nseg = 0;
+  Seg seg[kMaxSegs];
+  const void* resid = nullptr;
+  long long resid_ld = 0;
+  void* out = nullptr;
+  long long out_ld = 0;
+  int swiglu_F = 0;
+  unsigned* status = nullptr;
+};
+
+cudaError_t launch_gemm_bf16(const GemmDesc& g, cudaStream_t st);
+cudaError_t launch_gemm_f32(const GemmDesc& g, cudaStream_t st);
+
+struct ScanDesc {
+  const void* x; const void* dt; const float* bc; const void* gate; const float* a_log;
+  void* y; long long y_ld;
+  int batch, T, d_inner, d_state;
+  bool bf16;
+  unsigned* status;
+};
+cudaError_t launch_scan(const ScanDesc& s, cudaStream_t st);
+
+struct AttnDesc {
+  const void* q; long long q_ld;     // [batch*T, q_ld], head h at column h*dh
+  const void* k; const void* v; long long kv_ld;  // [batch*T, kv_ld]
+  void* out; long long out_ld;
+  int batch, T, n_q_heads, n_kv_heads, head_dim, n_meta, window;
+  bool bf16;
+  unsigned* status;
+};
+cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st);
+
+cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, long long rows, int w_attn,
+                               int w_ssm, float eps, bool bf16, cudaStream_t st);
+cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float eps, bool bf16,
+                           cudaStream_t st);
+
+int num_sms();
+
+}  // namespace hy

@@ -1,0 +1,140 @@
+// norm.cu -- row-wise RMS normalisation kernels.
+//
+//   branch_norm: z = [beta1 * rms(z_attn) || beta2 * rms(z_ssm)] in place, the
+//     per-branch norm and learnable rescale before out_proj (blog.outta.ai Hymba
+//     review, "Design formulation", total fusion formulation; metaphor-xennon
+//     "PyTorch伪代码": one RMSNorm per branch).
+//   rmsnorm:     y = x / sqrt(mean(x^2) + eps), unit gain (pre-norm of the
+//     stacked blocks).
+// One CTA per row; fp32 sums; 16-byte vector loads and stores.  HBM-bound: one
+// read for the sums (the second read of the row hits L1/L2) and one write.
+#include "hy_common.cuh"
+#include "hy_kernels.h"
+
+namespace hy {
+namespace {
+
+constexpr int NT = 256;
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  if (threadIdx.x < 32) {
+    s = (l < NT / 32) ? red[l] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (l == 0) red[NT / 32] = s;
+  }
+  __syncthreads();
+  return red[NT / 32];
+}
+
+// vector of 8 elements
+template <typename T> struct Vec8;
+template <> struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&f)[8]) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = bf16lo(u[i]);
+      f[2 * i + 1] = bf16hi(u[i]);
+    }
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&f)[8]) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                                              pack_bf16(f[6], f[7]));
+  }
+};
+template <> struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&f)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&f)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+};
+
+template <typename T>
+__device__ __forceinline__ float sumsq(const T* row, int w) {
+  float s = 0.f;
+  for (int i = threadIdx.x * 8; i < w; i += NT * 8) {
+    float f[8];
+    Vec8<T>::load(row + i, f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s = fmaf(f[j], f[j], s);
+  }
+  return s;
+}
+
+template <typename T>
+__device__ __forceinline__ void scale_row(const T* src, T* dst, int w, float r, const float* beta) {
+  for (int i = threadIdx.x * 8; i < w; i += NT * 8) {
+    float f[8];
+    Vec8<T>::load(src + i, f);
+    if (beta) {
+      const float4 b0 = *reinterpret_cast<const float4*>(beta + i), b1 = *reinterpret_cast<const float4*>(beta + i + 4);
+      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] = f[j] * r * bb[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] *= r;
+    }
+    Vec8<T>::store(dst + i, f);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(NT) branch_norm_kernel(T* z, const float* __restrict__ beta1,
+                                                         const float* __restrict__ beta2, int wa, int ws, float eps) {
+  __shared__ float red[NT / 32 + 1];
+  T* row = z + static_cast<long long>(blockIdx.x) * (wa + ws);
+  const float sa = block_sum(sumsq(row, wa), red);
+  const float ss = block_sum(sumsq(row + wa, ws), red);
+  const float ra = rsqrtf(sa / wa + eps), rs = rsqrtf(ss / ws + eps);
+  scale_row(row, row, wa, ra, beta1);
+  scale_row(row + wa, row + wa, ws, rs, beta2);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(NT) rmsnorm_kernel(const T* x, T* y, int d, float eps) {
+  __shared__ float red[NT / 32 + 1];
+  const long long off = static_cast<long long>(blockIdx.x) * d;
+  const float s = block_sum(sumsq(x + off, d), red);
+  scale_row(x + off, y + off, d, rsqrtf(s / d + eps), nullptr);
+}
+
+}  // namespace
+
+cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, long long rows, int w_attn, int w_ssm,
+                               float eps, bool bf16, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (bf16)
+    branch_norm_kernel<__nv_bfloat16><<<static_cast<unsigned>(rows), NT, 0, st>>>(
+        static_cast<__nv_bfloat16*>(z), beta1, beta2, w_attn, w_ssm, eps);
+  else
+    branch_norm_kernel<float><<<static_cast<unsigned>(rows), NT, 0, st>>>(static_cast<float*>(z), beta1, beta2,
+                                                                           w_attn, w_ssm, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float eps, bool bf16, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (bf16)
+    rmsnorm_kernel<__nv_bfloat16><<<static_cast<unsigned>(rows), NT, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), d, eps);
+  else
+    rmsnorm_kernel<float><<<static_cast<unsigned>(rows), NT, 0, st>>>(static_cast<const float*>(x),
+                                                                       static_cast<float*>(y), d, eps);
+  return cudaGetLastError();
+}
+
+}  // namespace hy

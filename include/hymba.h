@@ -1,0 +1,210 @@
+/*
+ * hymba.h -- C ABI of the B200 (sm_100a) library for the forward (prefill) pass
+ * of Hymba's fused hybrid-head layer.
+ *
+ * What the layer computes (sources: the blog.outta.ai review of arXiv
+ * 2411.13676 "Hymba: A Hybrid-head Architecture for Small Language Models",
+ * section "Design formulation"; the metaphor-xennon page, sections
+ * "混合头模块" and "PyTorch伪代码"; the networkstorageforum summary, section
+ * "Key Components of Hymba"):
+ *
+ *   X~      = [meta; X]                                  (meta tokens prepended)
+ *   [Q K V X_ssm G_raw] = X~ W_in^T                      (one fused in_proj)
+ *   Y_attn  = softmax(Q K^T / sqrt(dh) + mask) V         (causal / SWA, meta always visible, GQA)
+ *   [dt_low B C] = X_ssm W_x^T,  dt = softplus(dt_low W_dt^T + b_dt),  A = -exp(A_log)
+ *   h_t     = exp(A dt_t) h_{t-1} + dt_t B_t x_t,  y_t = C_t . h_t     (selective scan)
+ *   Y_ssm   = SiLU(G_raw) * y
+ *   out     = W_out [ beta1 * rms(Y_attn) || beta2 * rms(Y_ssm) ]
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; row-major;
+ *     the library allocates no memory.  Calls are asynchronous on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - "dtype" tensors (activations and projection weights) are bf16 when
+ *     cfg.dtype == HYMBA_BF16 (fp32 accumulation, fp32 scan state) and fp32
+ *     when cfg.dtype == HYMBA_F32.  a_log, b_dt, beta1, beta2 are always fp32.
+ *   - Arguments are validated before anything is launched; a bad argument
+ *     returns an error status with no side effect.  HYMBA_ERR_CUDA is returned
+ *     only for a failed launch or CUDA call.
+ *   - Every kernel bounds its internal waits.  A wait that runs out records
+ *     HYMBA_ERR_TIMEOUT in the status word at the start of the workspace and
+ *     the kernel returns early; hymba_workspace_status() reads it.
+ */
+#ifndef HYMBA_H_
+#define HYMBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HYMBA_API __attribute__((visibility("default")))
+#else
+#define HYMBA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HYMBA_OK = 0,
+  HYMBA_ERR_INVALID_ARG = 1,  /* null pointer, negative or inconsistent size */
+  HYMBA_ERR_UNSUPPORTED = 2,  /* well-formed but outside what the kernels implement */
+  HYMBA_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than hymba_*workspace_size() */
+  HYMBA_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+  HYMBA_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (reported by hymba_workspace_status) */
+} hymba_status_t;
+
+typedef enum { HYMBA_F32 = 0, HYMBA_BF16 = 1 } hymba_dtype_t;
+
+/* Cross-layer KV sharing ("Cross-layer KV sharing" in the blog.outta.ai
+ * review: two consecutive layers share one KV cache).  The even layer of a
+ * pair produces K/V, the odd one consumes it and has no W_K / W_V rows. */
+typedef enum {
+  HYMBA_KV_OWN = 0,      /* compute K/V for this layer only (kept in the workspace) */
+  HYMBA_KV_PRODUCE = 1,  /* compute K/V and write them to kv_out for the partner layer */
+  HYMBA_KV_CONSUME = 2   /* no K/V projection: read the partner's K/V from kv_in */
+} hymba_kv_mode_t;
+
+typedef struct {
+  int batch;        /* B >= 1 */
+  int seq_len;      /* L >= 1: user tokens per sequence */
+  int n_meta;       /* M >= 0: meta tokens; T = L + M rows per sequence */
+  int d_model;      /* d */
+  int n_q_heads;    /* Hq */
+  int n_kv_heads;   /* Hkv, divides Hq (GQA) */
+  int head_dim;     /* dh: 128 for bf16; <= 128 for fp32 */
+  int window;       /* W: -1 = global causal; >= 0: query i sees key j iff j <= i and
+                       (i - j <= W or j < M) -- meta tokens always visible */
+  int d_inner;      /* Di: SSM channels */
+  int d_state;      /* N: 16, 32, 64, 128 or 256 */
+  int n_ssm_heads;  /* recorded only: the per-channel scan does not depend on it */
+  int dt_rank;      /* R: width of dt_low */
+  int a_per_state;  /* 0: A_log [Di] (supported); 1: A_log [Di, N] (HYMBA_ERR_UNSUPPORTED) */
+  int kv_mode;      /* hymba_kv_mode_t */
+  int ffn_dim;      /* F: SwiGLU FFN width for hymba_stack_fwd; 0 = no FFN */
+  float rms_eps;    /* RMSNorm epsilon (1e-6) */
+  hymba_dtype_t dtype;
+} hymba_cfg_t;
+
+/* Weights of one layer; device pointers, nn.Linear layout [out_features, in_features]. */
+typedef struct {
+  const void* w_in;       /* [Hq*dh + 2*Hkv*dh + 2*Di, d] rows W_Q, W_K, W_V, W_SSM, W_G
+                             (a HYMBA_KV_CONSUME layer has no W_K, W_V rows) */
+  const void* w_x;        /* [R + 2N, Di]   rows dt_low, B, C */
+  const void* w_dt;       /* [Di, R] */
+  const void* w_out;      /* [d, Hq*dh + Di] */
+  const float* a_log;     /* [Di]   A = -exp(A_log) */
+  const float* b_dt;      /* [Di] */
+  const float* beta1;     /* [Hq*dh] */
+  const float* beta2;     /* [Di] */
+  const void* w_gate_up;  /* [2F, d] gate rows then up rows (stack with ffn_dim > 0), else NULL */
+  const void* w_down;     /* [d, F] (stack with ffn_dim > 0), else NULL */
+} hymba_weights_t;
+
+/* Human-readable name of a status code (static string). */
+HYMBA_API const char* hymba_status_string(hymba_status_t s);
+
+/* Workspace bytes needed by hymba_layer_fwd for `cfg` (0 if cfg is invalid). */
+HYMBA_API size_t hymba_workspace_size(const hymba_cfg_t* cfg);
+
+/* Workspace bytes needed by hymba_stack_fwd for `n_layers` configs (0 if invalid). */
+HYMBA_API size_t hymba_stack_workspace_size(const hymba_cfg_t* cfgs, int n_layers);
+
+/*
+ * One hybrid-head layer, forward (prefill).
+ *   x       [B, L, d] dtype when meta != NULL; [B, T, d] (rows already X~) when meta == NULL
+ *   meta    [M, d] dtype, the learnable meta tokens shared by the batch, or NULL
+ *   kv_in   [2, B, T, Hkv*dh] dtype (K then V, token-major, head h at columns
+ *           [h*dh, (h+1)*dh)) -- required iff kv_mode == HYMBA_KV_CONSUME
+ *   kv_out  same layout -- required iff kv_mode == HYMBA_KV_PRODUCE
+ *   out     [B, T, d] dtype; meta rows are kept so the next layer sees [meta; X] state
+ *   workspace >= hymba_workspace_size(cfg) bytes, 256-byte aligned; its first 256
+ *           bytes hold the status word (reset by this call)
+ */
+HYMBA_API hymba_status_t hymba_layer_fwd(const void* x, const void* meta, const hymba_weights_t* w,
+                               const hymba_cfg_t* cfg, const void* kv_in, void* kv_out,
+                               void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * A stack of hybrid-head blocks ("Key Components of Hymba", networkstorageforum:
+ * blocks stacked with SWA and cross-layer KV sharing).  For each block i:
+ *   h += layer_i(RMSNorm(h));  if cfgs[i].ffn_dim: h += W_down(SiLU(W_gate u) * W_up u), u = RMSNorm(h)
+ * with unit RMSNorm gains; h starts as [meta; x].  K/V flow from a
+ * HYMBA_KV_PRODUCE block to the HYMBA_KV_CONSUME block after it through the
+ * workspace.  x, meta as in hymba_layer_fwd; out [B, T, d] = final h.
+ * All cfgs must share batch, seq_len, n_meta, d_model, dtype.
+ */
+HYMBA_API hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weights_t* w,
+                               const hymba_cfg_t* cfgs, int n_layers, void* out,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * hymba_layer_fwd with stage timing (tracing hook).  `events` holds 8 cudaEvent_t
+ * (created by the caller, passed as void*): events[i] is recorded on `stream`
+ * right before stage i and events[7] after the last one.  Stages:
+ * 0 in_proj, 1 x_proj, 2 dt_proj, 3 attention, 4 selective scan, 5 branch
+ * norm, 6 out_proj.  events == NULL behaves exactly like hymba_layer_fwd.
+ */
+HYMBA_API hymba_status_t hymba_layer_fwd_events(const void* x, const void* meta, const hymba_weights_t* w,
+                               const hymba_cfg_t* cfg, const void* kv_in, void* kv_out,
+                               void* out, void* workspace, size_t ws_bytes, void* stream,
+                               void* const* events);
+
+/* Synchronises `stream`, reads and clears the status word at the start of
+ * `workspace`: HYMBA_OK, or HYMBA_ERR_TIMEOUT if a kernel's bounded wait ran out. */
+HYMBA_API hymba_status_t hymba_workspace_status(void* workspace, void* stream);
+
+/* ---------------- stage entry points (each one kernel family) ---------------- */
+
+/* C[M, N] = A[M, K] W[N, K]^T (dtype in and out, fp32 accumulation); bf16 runs on the
+ * tcgen05 tensor-core GEMM.  workspace: >= 256 bytes (status word). */
+HYMBA_API hymba_status_t hymba_gemm(const void* a, const void* w, void* c, int M, int N, int K,
+                          hymba_dtype_t dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Selective scan fused with the output gate ("Design formulation": SSM head
+ * alpha_ij and Y_ssm = G . alpha W_SSM X~):
+ *   for each sequence b and channel c, from h = 0:
+ *     h_t = exp(A_c dt_t) h_{t-1} + dt_t x_t B_t,   y_t = gate_t * (C_t . h_t),   A_c = -exp(a_log[c])
+ *   x, dt, gate [batch*T, d_inner] dtype (dt > 0 already discretised; gate = SiLU(G_raw))
+ *   bc   [batch*T, 2*d_state] fp32, B_t then C_t
+ *   y    written at y + row*y_ld, dtype
+ *   workspace >= 256 bytes (status word)
+ */
+HYMBA_API hymba_status_t hymba_selective_scan(const void* x, const void* dt, const float* bc,
+                                    const void* gate, const float* a_log, void* y, int y_ld,
+                                    int batch, int T, int d_inner, int d_state,
+                                    hymba_dtype_t dtype, void* workspace, size_t ws_bytes,
+                                    void* stream);
+
+/*
+ * Attention heads ("Design formulation", attention head; "Combine global and local
+ * attention"): per sequence and query head h (KV head h / (Hq/Hkv)),
+ *   out_i = sum_j softmax_j(q_i . k_j / sqrt(dh)) v_j  over visible j (see hymba_cfg_t.window)
+ *   q   [batch*T, Hq*dh] dtype;  kv [2, batch*T, Hkv*dh] dtype (K then V)
+ *   out written at out + row*out_ld + h*dh, dtype
+ */
+HYMBA_API hymba_status_t hymba_attention(const void* q, const void* kv, void* out, int out_ld, int batch,
+                               int T, int n_q_heads, int n_kv_heads, int head_dim, int n_meta,
+                               int window, hymba_dtype_t dtype, void* workspace,
+                               size_t ws_bytes, void* stream);
+
+/*
+ * Per-branch RMSNorm and beta scale, in place ("Design formulation", total fusion):
+ *   z [rows, w_attn + w_ssm] dtype;  z[:, :w_attn] = beta1 * rms(z[:, :w_attn]),
+ *   z[:, w_attn:] = beta2 * rms(z[:, w_attn:]),   rms(v) = v / sqrt(mean(v^2) + eps)
+ */
+HYMBA_API hymba_status_t hymba_branch_norm(void* z, const float* beta1, const float* beta2, int rows,
+                                 int w_attn, int w_ssm, float eps, hymba_dtype_t dtype,
+                                 void* stream);
+
+/* y[rows, d] = x / sqrt(mean(x^2) + eps) row-wise (unit gain); x and y may alias. */
+HYMBA_API hymba_status_t hymba_rmsnorm(const void* x, void* y, int rows, int d, float eps,
+                             hymba_dtype_t dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYMBA_H_ */

@@ -1,0 +1,130 @@
+"""CPU-side checks of the C ABI: the library loads, exports every entry point
+declared in include/hymba.h, and validates arguments without touching a GPU."""
+import os
+import re
+
+import pytest
+
+import hybrid_attention_ssm_hymba_b200 as H
+from hybrid_attention_ssm_hymba_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "hymba.h")).read()
+    return sorted(set(re.findall(r"HYMBA_API\s+[\w\s\*]+?\b(hymba_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_entry_point():
+    lib = H.load()
+    declared = _declared()
+    assert len(declared) >= 11
+    assert set(declared) == set(H.ENTRY_POINTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    for s in range(6):
+        assert H.hymba_status_string(s)
+    assert "timed out" in H.hymba_status_string(H.HYMBA_ERR_TIMEOUT)
+
+
+@pytest.mark.parametrize("name", synth.WORKLOAD_ORDER)
+def test_every_workload_is_supported(name):
+    wl = synth.workload(name)
+    cfgs = [H.make_cfg(s) for s in wl.layers]
+    for c in cfgs:
+        assert H.hymba_workspace_size(c) > 0
+    assert H.hymba_stack_workspace_size(cfgs) > 0
+
+
+def _cfg(**kw):
+    return H.make_cfg(synth.workload("hymba350m_layer").first, **kw)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(batch=0), H.HYMBA_ERR_INVALID_ARG),
+    (dict(seq_len=0), H.HYMBA_ERR_INVALID_ARG),
+    (dict(n_meta=-1), H.HYMBA_ERR_INVALID_ARG),
+    (dict(window=-2), H.HYMBA_ERR_INVALID_ARG),
+    (dict(n_q_heads=3, n_kv_heads=2), H.HYMBA_ERR_INVALID_ARG),
+    (dict(kv_mode=3), H.HYMBA_ERR_INVALID_ARG),
+    (dict(head_dim=64), H.HYMBA_ERR_UNSUPPORTED),
+    (dict(d_state=24), H.HYMBA_ERR_UNSUPPORTED),
+    (dict(n_meta=12), H.HYMBA_ERR_UNSUPPORTED),
+    (dict(a_per_state=1), H.HYMBA_ERR_UNSUPPORTED),
+    (dict(dt_rank=40), H.HYMBA_ERR_UNSUPPORTED),
+    (dict(dtype=7), H.HYMBA_ERR_INVALID_ARG),
+])
+def test_layer_validation_rejects_before_launch(kw, expect):
+    """Bad configs return their status without any CUDA call (this runs on a CPU machine)."""
+    c = _cfg(**kw)
+    assert H.hymba_workspace_size(c) == 0
+    w = H.make_weights({k: 1 << 20 for k in ("w_in", "w_x", "w_dt", "w_out", "a_log", "b_dt",
+                                             "beta1", "beta2")})
+    st = H.hymba_layer_fwd(1 << 20, 1 << 20, w, c, None, None, 1 << 20, 1 << 20, ws_bytes=1 << 40,
+                           stream=0)
+    assert st == expect
+
+
+def test_layer_rejects_missing_pointers_and_small_workspace():
+    c = _cfg()
+    full = {k: 1 << 20 for k in ("w_in", "w_x", "w_dt", "w_out", "a_log", "b_dt", "beta1", "beta2")}
+    need = H.hymba_workspace_size(c)
+    assert H.hymba_layer_fwd(None, 1 << 20, H.make_weights(full), c, None, None, 1 << 20, 1 << 20,
+                             ws_bytes=need, stream=0) == H.HYMBA_ERR_INVALID_ARG
+    partial = dict(full, w_out=None)
+    assert H.hymba_layer_fwd(1 << 20, 1 << 20, H.make_weights(partial), c, None, None, 1 << 20,
+                             1 << 20, ws_bytes=need, stream=0) == H.HYMBA_ERR_INVALID_ARG
+    assert H.hymba_layer_fwd(1 << 20, 1 << 20, H.make_weights(full), c, None, None, 1 << 20, 1 << 20,
+                             ws_bytes=need - 1, stream=0) == H.HYMBA_ERR_WORKSPACE
+    # a consuming layer needs kv_in, a producing one kv_out
+    for mode in (H.HYMBA_KV_CONSUME, H.HYMBA_KV_PRODUCE):
+        cm = _cfg(kv_mode=mode)
+        assert H.hymba_layer_fwd(1 << 20, 1 << 20, H.make_weights(full), cm, None, None, 1 << 20,
+                                 1 << 20, ws_bytes=1 << 40, stream=0) == H.HYMBA_ERR_INVALID_ARG
+    # misaligned workspace
+    assert H.hymba_layer_fwd(1 << 20, 1 << 20, H.make_weights(full), c, None, None, 1 << 20,
+                             (1 << 20) + 8, ws_bytes=1 << 40, stream=0) == H.HYMBA_ERR_INVALID_ARG
+
+
+def test_stack_validation():
+    wl = synth.workload("hymba1p5b_stack24", n_layers=2)
+    cfgs = [H.make_cfg(s) for s in wl.layers]
+    full = {k: 1 << 20 for k in ("w_in", "w_x", "w_dt", "w_out", "a_log", "b_dt", "beta1", "beta2",
+                                 "w_gate_up", "w_down")}
+    ws = [H.make_weights(full)] * 2
+    # consumer first is invalid
+    bad = [cfgs[1], cfgs[0]]
+    assert H.hymba_stack_fwd(1 << 20, 1 << 20, ws, bad, 1 << 20, 1 << 20, ws_bytes=1 << 40,
+                             stream=0) == H.HYMBA_ERR_INVALID_ARG
+    # FFN weights required when ffn_dim > 0
+    ws2 = [H.make_weights(dict(full, w_down=None))] * 2
+    assert H.hymba_stack_fwd(1 << 20, 1 << 20, ws2, cfgs, 1 << 20, 1 << 20, ws_bytes=1 << 40,
+                             stream=0) == H.HYMBA_ERR_INVALID_ARG
+    need = H.hymba_stack_workspace_size(cfgs)
+    assert H.hymba_stack_fwd(1 << 20, 1 << 20, ws, cfgs, 1 << 20, 1 << 20, ws_bytes=need - 1,
+                             stream=0) == H.HYMBA_ERR_WORKSPACE
+
+
+def test_stage_validation():
+    assert H.load().hymba_gemm(None, 1, 1, 8, 16, 8, 1, 1, 256, None) == H.HYMBA_ERR_INVALID_ARG
+    assert H.load().hymba_gemm(1, 1, 1, 8, 24, 8, 1, 1, 256, None) == H.HYMBA_ERR_UNSUPPORTED
+    assert H.load().hymba_gemm(1, 1, 1, 8, 16, 8, 1, 1, 16, None) == H.HYMBA_ERR_WORKSPACE
+    assert H.load().hymba_selective_scan(1, 1, 1, 1, 1, 1, 64, 1, 10, 64, 24, 1, 1, 256,
+                                         None) == H.HYMBA_ERR_UNSUPPORTED
+    assert H.load().hymba_attention(1, 1, 1, 256, 1, 10, 2, 1, 64, 0, -1, 1, 1, 256,
+                                    None) == H.HYMBA_ERR_UNSUPPORTED
+    assert H.load().hymba_attention(1, 1, 1, 256, 1, 10, 3, 2, 128, 0, -1, 1, 1, 256,
+                                    None) == H.HYMBA_ERR_INVALID_ARG
+    assert H.load().hymba_branch_norm(1, 1, 1, 4, 12, 16, 1e-6, 1, None) == H.HYMBA_ERR_UNSUPPORTED
+    assert H.load().hymba_rmsnorm(1, 1, 4, 0, 1e-6, 1, None) == H.HYMBA_ERR_INVALID_ARG
+
+
+def test_no_cpu_fallback_when_library_missing(tmp_path, monkeypatch):
+    from hybrid_attention_ssm_hymba_b200 import _abi
+    monkeypatch.setattr(_abi, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        _abi.load(str(tmp_path / "libhymba.so"))

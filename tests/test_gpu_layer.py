@@ -1,0 +1,193 @@
+"""Whole-layer and whole-stack parity on the GPU against the fp64 oracle, through
+the C ABI, on the five seeded workloads.
+
+The GPU always runs the full workload (the launch configuration the bench
+times).  The oracle runs the full batch where it finishes in seconds and
+otherwise a causal prefix of chosen sequences: output rows [0, t) depend only
+on input rows [0, t), so the oracle on the truncated input gives those rows
+exactly.  Prefixes are longer than window + meta, so the sliding window and the
+always-visible meta tokens are exercised."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import hybrid_attention_ssm_hymba_b200 as H
+import oracle as O
+from hybrid_attention_ssm_hymba_b200 import host, synth
+from gpu_util import assert_close, dev, requires_cuda, status_ok, to_np
+
+pytestmark = [pytest.mark.gpu, requires_cuda]
+
+
+def _upload(wl, layers=None):
+    layers = range(len(wl.layers)) if layers is None else layers
+    ps = [synth.layer_params(wl, i) for i in layers]
+    return ps, [host.params_to_device(p, wl.layers[i].dtype) for i, p in zip(layers, ps)]
+
+
+def _oracle_layer(wl, ps, x, meta, batch_ids, L):
+    """Oracle output rows [0, M + L) of the listed sequences (layer pairs chained)."""
+    outs = []
+    for b in batch_ids:
+        xb = x[b:b + 1, :L]
+        kv = None
+        h = None
+        for i, s in enumerate(wl.layers):
+            si = dataclasses.replace(s, batch=1, seq_len=L)
+            if i == 0:
+                h, kv = O.layer_forward(xb, meta, ps[i], si)
+            else:   # the consumer reads the producer's output and K/V
+                h, _ = O.layer_forward(h, None, ps[i], si, kv_in=kv)
+        outs.append(h[0])
+    return outs
+
+
+def _gpu_layers(wl, dps, x, meta):
+    s0 = wl.first
+    T = s0.T
+    dtype = s0.dtype
+    cfgs = [H.make_cfg(s) for s in wl.layers]
+    ws = host.workspace(max(H.hymba_workspace_size(c) for c in cfgs))
+    kv = host.empty((2, s0.batch * T, s0.kv_width), dtype) if len(wl.layers) > 1 else None
+    tx, tm = dev(x, dtype), dev(meta, dtype)
+    out = host.empty((s0.batch, T, s0.d_model), dtype)
+    H.check(H.hymba_layer_fwd(tx, tm, H.make_weights(dps[0]), cfgs[0], None, kv, out, ws), "layer 0")
+    outs = [out]
+    for i in range(1, len(wl.layers)):
+        o2 = host.empty((s0.batch, T, s0.d_model), dtype)
+        H.check(H.hymba_layer_fwd(outs[-1], None, H.make_weights(dps[i]), cfgs[i], kv, None, o2, ws),
+                f"layer {i}")
+        outs.append(o2)
+    status_ok(ws)
+    return to_np(outs[-1])
+
+
+def test_tiny_fp32_layer_full():
+    wl = synth.workload("tiny_fp32")
+    x, meta = synth.layer_inputs(wl)
+    ps, dps = _upload(wl)
+    g = _gpu_layers(wl, dps, x, meta)
+    ref, _ = O.layer_forward(x, meta, ps[0], wl.first)
+    assert_close(g, ref, "f32", "tiny fp32 layer")
+
+
+def test_hymba350m_layer_full_batch():
+    wl = synth.workload("hymba350m_layer")
+    x, meta = synth.layer_inputs(wl)
+    ps, dps = _upload(wl)
+    g = _gpu_layers(wl, dps, x, meta)
+    ref, _ = O.layer_forward(x, meta, ps[0], wl.first)
+    for b in range(wl.first.batch):
+        assert_close(g[b], ref[b], "bf16", f"350M layer, sequence {b}")
+
+
+@pytest.mark.parametrize("name,prefixes", [
+    ("hymba1p5b_kvpair", {0: 1300, 3: 200}),
+    ("longctx_32k", {0: 1420}),
+])
+def test_large_layers_prefix(name, prefixes):
+    wl = synth.workload(name)
+    x, meta = synth.layer_inputs(wl)
+    ps, dps = _upload(wl)
+    g = _gpu_layers(wl, dps, x, meta)
+    M = wl.first.n_meta
+    for b, L in prefixes.items():
+        ref = _oracle_layer(wl, ps, x, meta, [b], L)[0]
+        assert_close(g[b, :M + L], ref, "bf16", f"{name} sequence {b} rows [0, {M + L})")
+
+
+def test_meta_rows_identical_across_batch_and_meta_mode_equals_explicit_xtilde():
+    """Meta output rows are the same for every sequence; passing meta separately
+    equals passing X~ = [meta; X] with meta = NULL."""
+    wl = synth.workload("hymba350m_layer", batch=3, seq_len=500)
+    x, meta = synth.layer_inputs(wl)
+    ps, dps = _upload(wl)
+    g = _gpu_layers(wl, dps, x, meta)
+    M = wl.first.n_meta
+    for b in range(1, 3):
+        np.testing.assert_array_equal(g[b, :M], g[0, :M])
+    xt = np.concatenate([np.broadcast_to(meta, (3,) + meta.shape), x], axis=1)
+    cfg = H.make_cfg(wl.first)
+    out = host.empty((3, wl.first.T, wl.first.d_model), "bf16")
+    ws = host.workspace(H.hymba_workspace_size(cfg))
+    H.check(H.hymba_layer_fwd(dev(xt, "bf16"), None, H.make_weights(dps[0]), cfg, None, None, out, ws), "X~")
+    np.testing.assert_array_equal(to_np(out), g)
+
+
+@pytest.mark.parametrize("kw", [dict(n_meta=0, window=0), dict(n_meta=8, window=0), dict(window=300),
+                                dict(seq_len=1), dict(n_meta=136, window=64)])
+def test_layer_edge_configs(kw):
+    """No meta / self-only window / meta + zero window / one token / meta not a
+    multiple of the 128-row tile."""
+    wl = synth.workload("hymba350m_layer", batch=2, seq_len=kw.pop("seq_len", 333), **kw)
+    x, meta = synth.layer_inputs(wl)
+    ps, dps = _upload(wl)
+    g = _gpu_layers(wl, dps, x, meta if wl.first.n_meta else np.zeros((0, wl.first.d_model), np.float32))
+    ref, _ = O.layer_forward(x, meta if wl.first.n_meta else None, ps[0], wl.first)
+    assert_close(g, ref, "bf16", f"edge {kw}")
+
+
+def test_kv_sharing_consumer_equals_standalone_layer():
+    """A consumer fed the producer's K/V equals a standalone layer whose W_K, W_V
+    rows would produce that K/V (same Q, SSM and output weights)."""
+    wl = synth.workload("hymba1p5b_kvpair", batch=1, seq_len=700)
+    x, meta = synth.layer_inputs(wl)
+    ps, dps = _upload(wl)
+    s0 = wl.first
+    T, wa, wkv = s0.T, s0.attn_width, s0.kv_width
+    kv = host.empty((2, T, wkv), "bf16")
+    cfg_p = H.make_cfg(s0)
+    ws = host.workspace(H.hymba_workspace_size(cfg_p))
+    out_p = host.empty((1, T, s0.d_model), "bf16")
+    tx, tm = dev(x, "bf16"), dev(meta, "bf16")
+    H.check(H.hymba_layer_fwd(tx, tm, H.make_weights(dps[0]), cfg_p, None, kv, out_p, ws), "producer")
+    # consumer weights = producer's weights without the W_K, W_V rows
+    w_in_c = torch.cat([dps[0]["w_in"][:wa], dps[0]["w_in"][wa + 2 * wkv:]]).contiguous()
+    dpc = dict(dps[0], w_in=w_in_c)
+    cfg_c = H.make_cfg(dataclasses.replace(s0, kv_mode=H.HYMBA_KV_CONSUME))
+    out_c = host.empty((1, T, s0.d_model), "bf16")
+    H.check(H.hymba_layer_fwd(tx, tm, H.make_weights(dpc), cfg_c, kv, None, out_c, ws), "consumer")
+    status_ok(ws)
+    np.testing.assert_array_equal(to_np(out_c), to_np(out_p))
+
+
+def test_stack24_prefix_and_per_block():
+    """The 24-block stack at full size on the GPU; the oracle runs the causal
+    prefix of sequence 0 through all 24 blocks (global blocks 0, 11, 23, SWA 1024
+    elsewhere, K/V shared by block pairs, SwiGLU FFN)."""
+    wl = synth.workload("hymba1p5b_stack24")
+    s0 = wl.first
+    x, meta = synth.layer_inputs(wl)
+    ps, dps = _upload(wl)
+    cfgs = [H.make_cfg(s) for s in wl.layers]
+    ws = host.workspace(H.hymba_stack_workspace_size(cfgs))
+    out = host.empty((s0.batch, s0.T, s0.d_model), "bf16")
+    H.check(H.hymba_stack_fwd(dev(x, "bf16"), dev(meta, "bf16"), [H.make_weights(d) for d in dps], cfgs, out,
+                              ws), "stack")
+    status_ok(ws)
+    g = to_np(out)
+    L = 1100
+    shapes = [dataclasses.replace(s, batch=1, seq_len=L) for s in wl.layers]
+    ref = O.stack_forward(x[:1, :L], meta, ps, shapes)
+    assert_close(g[0, :s0.n_meta + L], ref[0], "bf16", "24-block stack, sequence 0 prefix")
+
+
+def test_stack_small_full_parity():
+    """Four blocks (global, SWA, SWA, global), ragged T, every row checked."""
+    wl = synth.workload("hymba1p5b_stack24", n_layers=4, batch=2, seq_len=1300, d_state=16)
+    wl.layers[3] = dataclasses.replace(wl.layers[3], window=-1)
+    wl.layers[1] = dataclasses.replace(wl.layers[1], window=200)
+    wl.layers[2] = dataclasses.replace(wl.layers[2], window=1024)
+    s0 = wl.first
+    x, meta = synth.layer_inputs(wl)
+    ps, dps = _upload(wl)
+    cfgs = [H.make_cfg(s) for s in wl.layers]
+    ws = host.workspace(H.hymba_stack_workspace_size(cfgs))
+    out = host.empty((s0.batch, s0.T, s0.d_model), "bf16")
+    H.check(H.hymba_stack_fwd(dev(x, "bf16"), dev(meta, "bf16"), [H.make_weights(d) for d in dps], cfgs, out,
+                              ws), "stack")
+    status_ok(ws)
+    ref = O.stack_forward(x, meta, ps, wl.layers)
+    assert_close(to_np(out), ref, "bf16", "4-block stack")
