@@ -262,6 +262,11 @@ def run_native(args, rank, world, local_rank):
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)] if not stack else None
+    if stage_ev:   # torch creates the CUDA event lazily, at its first record
+        for evs in stage_ev:
+            for e in evs:
+                e.record(stream)
+        torch.cuda.synchronize(dev)
     sampler = ClockSampler(dev)
     barrier()
     torch.cuda.synchronize(dev)

@@ -102,8 +102,9 @@ bool weights_ok(const hymba_weights_t* w, const hymba_cfg_t& c, bool need_ffn) {
 hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t& w, const hymba_cfg_t& c,
                          const void* kv_in, void* kv_out, void* out, bool resid_out, uint8_t* ws, unsigned* status,
                          cudaStream_t st, void* const* events = nullptr) {
+  bool marks_ok = true;
   auto mark = [&](int i) {
-    if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+    if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) != cudaSuccess) marks_ok = false;
   };
   const LayerWs L = layer_ws(c, 0);
   const int T = c.seq_len + c.n_meta;
@@ -247,7 +248,7 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   go.status = status;
   if ((e = gemm(go, c.dtype, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
   mark(7);
-  return HYMBA_OK;
+  return marks_ok ? HYMBA_OK : HYMBA_ERR_CUDA;
 }
 
 // h[b] = [meta; x[b]] (stack input), vectorised 16-byte copy.
@@ -320,6 +321,9 @@ hymba_status_t hymba_layer_fwd_events(const void* x, const void* meta, const hym
   if (cfg->kv_mode == HYMBA_KV_PRODUCE && !kv_out) return HYMBA_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < hymba_workspace_size(cfg)) return HYMBA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255) return HYMBA_ERR_INVALID_ARG;
+  if (events)
+    for (int i = 0; i < 8; ++i)
+      if (!events[i]) return HYMBA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned* status = static_cast<unsigned*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;

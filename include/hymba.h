@@ -144,7 +144,8 @@ HYMBA_API hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const 
  * (created by the caller, passed as void*): events[i] is recorded on `stream`
  * right before stage i and events[7] after the last one.  Stages:
  * 0 in_proj, 1 x_proj, 2 dt_proj, 3 attention, 4 selective scan, 5 branch
- * norm, 6 out_proj.  events == NULL behaves exactly like hymba_layer_fwd.
+ * norm, 6 out_proj.  events == NULL behaves exactly like hymba_layer_fwd; a NULL
+ * entry in a non-NULL `events` returns HYMBA_ERR_INVALID_ARG before any launch.
  */
 HYMBA_API hymba_status_t hymba_layer_fwd_events(const void* x, const void* meta, const hymba_weights_t* w,
                                const hymba_cfg_t* cfg, const void* kv_in, void* kv_out,
