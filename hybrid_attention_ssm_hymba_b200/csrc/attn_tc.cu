@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       const float m_new = fmaxf(m, mx * p.scale_log2);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = exp2f(m - m_use);
+      const float alpha = ex2_approx(m - m_use);
       // fold in the previous block's P V (its smem P and TMEM O are then free)
       if (j > 0) {
         if (!__all_sync(0xffffffffu, mbar_wait(o_full, (j - 1) & 1, p.status, abort_flag))) {
@@ -280,8 +280,8 @@ __global__ void __launch_bounds__(192, 1)
         for (int e = 0; e < 32; e += 2) {
           const bool v0 = !need_mask || visible(i, k0 + c * 32 + e, p.n_meta, p.window);
           const bool v1 = !need_mask || visible(i, k0 + c * 32 + e + 1, p.n_meta, p.window);
-          const float p0 = v0 ? exp2f(fmaf(__uint_as_float(v[e]), p.scale_log2, -m_use)) : 0.f;
-          const float p1 = v1 ? exp2f(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -m_use)) : 0.f;
+          const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(v[e]), p.scale_log2, -m_use)) : 0.f;
+          const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -m_use)) : 0.f;
           sum += p0 + p1;
           pk[e >> 1] = pack_bf16(p0, p1);
         }

@@ -5,11 +5,12 @@
 // stacked blocks (blog.outta.ai Hymba review, "Design formulation"; metaphor-xennon
 // page, "层配置": intermediate_size).
 //
-// Kernel shape: persistent, one CTA per SM, 192 threads:
+// Kernel shape: persistent, one CTA per SM, 320 threads:
 //   warp 0      TMA producer (one thread) -> STAGES-deep smem ring (full/empty mbarriers)
 //   warp 1      TMEM allocator + UMMA issuer (one thread), 128 x BN x 16 per instruction
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows, fused elementwise op,
-//               vector stores.  Two TMEM accumulators so the epilogue of tile i
+//   warps 2..9  epilogue: two warps per TMEM lane quadrant, each taking every other
+//               32-column chunk: tcgen05.ld of the accumulator rows, fused elementwise
+//               op, vector stores.  Two TMEM accumulators so the epilogue of tile i
 //               overlaps the mainloop of tile i+1.
 //
 // "Meta mode" reads the rows of X~_b = [meta; x_b] for each sequence b straight from
@@ -27,6 +28,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
+constexpr int NTHREADS = 320;       // producer warp, MMA warp, 8 epilogue warps
+constexpr int EPI_THREADS = 256;
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 
 struct GemmParams {
@@ -107,7 +110,7 @@ __device__ __forceinline__ void store16(const GemmParams& p, long long row, int 
 }
 
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(NTHREADS, 1)
     gemm_bf16_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAx2,
                  const __grid_constant__ CUtensorMap tmM1, const __grid_constant__ CUtensorMap tmM2,
                  const __grid_constant__ CUtensorMap tmB, const __grid_constant__ GemmParams p) {
@@ -132,7 +135,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], EPI_THREADS);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -250,8 +253,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(mma_done, 0, nullptr, &never, 100000000ull);
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 2..5)
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    // ------------------------------------------------ epilogue (warps 2..9)
+    const int quad = warp & 3;         // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;  // which alternate 32-column chunks it takes
     const int r = quad * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * BN;
       if (p.epi == EPI_SEGMENTS) {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half; c < BN / 32; c += 2) {
           uint32_t v[32];
           tmem_ld32(tb + c * 32, v);
           tmem_wait_ld();
@@ -286,7 +290,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       } else if (p.epi == EPI_SWIGLU) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = half; c < 4; c += 2) {
           uint32_t g[32], u[32];
           tmem_ld32(tb + c * 32, g);
           tmem_ld32(tb + 128 + c * 32, u);
@@ -305,7 +309,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       } else {  // EPI_RESIDUAL
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half; c < BN / 32; c += 2) {
           uint32_t v[32];
           tmem_ld32(tb + c * 32, v);
           tmem_wait_ld();
@@ -451,7 +455,7 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
   const long long total = static_cast<long long>(p.meta_mode ? p.batch : 1) * p.m_tiles * p.n_tiles;
   if (total <= 0) return cudaSuccess;
   const int grid = static_cast<int>(total < num_sms() ? total : num_sms());
-  gemm_bf16_tc<BN><<<grid, 192, C::SMEM, st>>>(tmA, tmAx2, tmM1, tmM2, tmB, p);
+  gemm_bf16_tc<BN><<<grid, NTHREADS, C::SMEM, st>>>(tmA, tmAx2, tmM1, tmM2, tmB, p);
   return cudaGetLastError();
 }
 

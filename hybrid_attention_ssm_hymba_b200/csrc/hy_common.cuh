@@ -169,8 +169,29 @@ HY_DEV uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-HY_DEV float silu_f(float x) { return x / (1.0f + __expf(-x)); }
-HY_DEV float softplus_f(float z) { return z > 20.0f ? z : log1pf(__expf(z)); }
+// tanh.approx: the SFU's hyperbolic tangent (max relative error ~2^-11)
+HY_DEV float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// ex2.approx: the SFU's base-2 exponential
+HY_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// SiLU(x) = x * sigmoid(x), with sigmoid(x) = (1 + tanh(x / 2)) / 2: one SFU op.
+HY_DEV float silu_f(float x) { return x * fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
+// softplus(z) = log(1 + e^z).  For e^z < 1/64 the series e - e^2/2 + e^3/3 (next
+// term below 1e-6 relative) avoids the cancellation of log(1 + e) near 1; above
+// 20 softplus(z) = z to fp32 precision.
+HY_DEV float softplus_f(float z) {
+  const float e = __expf(z);
+  const float series = e * fmaf(e, fmaf(e, 0.33333333f, -0.5f), 1.0f);
+  const float direct = __logf(1.0f + e);
+  return z > 20.0f ? z : (e < 0.015625f ? series : direct);
+}
 
 template <typename T> HY_DEV float to_f(T v);
 template <> HY_DEV float to_f<float>(float v) { return v; }
