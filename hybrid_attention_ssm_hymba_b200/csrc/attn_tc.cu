@@ -9,9 +9,10 @@
 //   warp 0      TMA producer: Q once, then K_j and V_j into two 2-deep rings
 //   warp 1      TMEM allocator + UMMA issuer: S_j = Q K_j^T into one of two TMEM
 //               S buffers (issued two blocks ahead), O_j = P_j V_j into TMEM
-//   warps 2..5  softmax: one query row per thread; fp32 row max and sum; P_j in bf16
-//               into swizzled smem (the A operand of P V); O accumulated in registers
-//               with the online-softmax rescale; final O / l stored as bf16.
+//   warps 2..5  softmax: one query row per thread; S_j read from TMEM once; fp32 row
+//               max and sum; P_j in bf16 into one of two swizzled smem tiles (the A
+//               operand of P V); O accumulates in TMEM across blocks, rescaled in place
+//               only when the running max grows by more than 2^8; final O / l as bf16.
 // K/V blocks with no visible pair are never loaded: the block list is the meta
 // blocks plus the window blocks.  Only blocks that straddle the mask boundary pay
 // for the elementwise mask.
@@ -24,7 +25,7 @@ namespace {
 constexpr int BQ = 128, BKV = 128, DH = 128;
 constexpr int TILE_BYTES = 128 * DH * 2;  // 32 KB: a [128 x 128] bf16 tile = 2 swizzled 64-column halves
 constexpr int HALF = 128 * 64 * 2;        // 16 KB
-constexpr int SMEM_BYTES = 6 * TILE_BYTES + 1024 + 256;
+constexpr int SMEM_BYTES = 7 * TILE_BYTES + 1024 + 256;
 constexpr uint32_t IDESC_QK = idesc_bf16(BQ, BKV, false, false);  // A=Q (K-major), B=K (K-major)
 constexpr uint32_t IDESC_PV = idesc_bf16(BQ, DH, false, true);    // A=P (K-major), B=V (MN-major)
 
@@ -68,10 +69,10 @@ __global__ void __launch_bounds__(192, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* sQ = smem_raw + pad;
-  uint8_t* sK = sQ + TILE_BYTES;            // 2 stages
-  uint8_t* sV = sK + 2 * TILE_BYTES;        // 2 stages
-  uint8_t* sP = sV + 2 * TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + TILE_BYTES);
+  uint8_t* sK = sQ + TILE_BYTES;      // 2 stages
+  uint8_t* sV = sK + 2 * TILE_BYTES;  // 2 stages
+  uint8_t* sP = sV + 2 * TILE_BYTES;  // 2 buffers
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * TILE_BYTES);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;   // [2]
   uint64_t* k_empty = bars + 3;  // [2]
@@ -79,10 +80,11 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* v_empty = bars + 7;  // [2]
   uint64_t* s_full = bars + 9;   // [2]
   uint64_t* s_free = bars + 11;  // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* o_full = bars + 14;
-  uint64_t* mma_done = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* p_full = bars + 13;  // [2]
+  uint64_t* p_free = bars + 15;  // [2]
+  uint64_t* o_done = bars + 17;  // completes once per P V
+  uint64_t* mma_done = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,9 +104,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 128);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&p_free[s], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_full, 1);
+    mbar_init(o_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -120,7 +123,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tS = tmem_base, tO = tmem_base + 256;
+  const uint32_t tS = tmem_base, tO = tmem_base + 256;  // S: 2 x 128 columns, O: 128 columns
 
   if (warp == 0) {
     if (lane == 0) {
@@ -130,34 +133,24 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive_expect_tx(q_full, TILE_BYTES);
       tma_load_3d(sQ, &tmQ, q_full, h * DH, q0, b);
       tma_load_3d(sQ + HALF, &tmQ, q_full, h * DH + 64, q0, b);
-      auto issue_k = [&](int j) -> bool {
+      auto issue_kv = [&](uint8_t* ring, const CUtensorMap* map, uint64_t* full, uint64_t* empty, int j,
+                          uint32_t& iss, uint32_t& par) -> bool {
         const int s = j & 1;
-        if (!mbar_wait(&k_empty[s], ((j >> 1) & 1) ^ 1u, p.status, abort_flag)) return false;
-        mbar_arrive_expect_tx(&k_full[s], TILE_BYTES);
+        if (!mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1u, p.status, abort_flag)) return false;
+        mbar_arrive_expect_tx(&full[s], TILE_BYTES);
         const int k0 = bl.block(j) * BKV;
-        tma_load_3d(sK + s * TILE_BYTES, &tmK, &k_full[s], kvh * DH, k0, b);
-        tma_load_3d(sK + s * TILE_BYTES + HALF, &tmK, &k_full[s], kvh * DH + 64, k0, b);
-        k_iss |= 1u << s;
-        k_par = (k_par & ~(1u << s)) | (static_cast<uint32_t>((j >> 1) & 1) << s);
-        return true;
-      };
-      auto issue_v = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(&v_empty[s], ((j >> 1) & 1) ^ 1u, p.status, abort_flag)) return false;
-        mbar_arrive_expect_tx(&v_full[s], TILE_BYTES);
-        const int k0 = bl.block(j) * BKV;
-        tma_load_3d(sV + s * TILE_BYTES, &tmV, &v_full[s], kvh * DH, k0, b);
-        tma_load_3d(sV + s * TILE_BYTES + HALF, &tmV, &v_full[s], kvh * DH + 64, k0, b);
-        v_iss |= 1u << s;
-        v_par = (v_par & ~(1u << s)) | (static_cast<uint32_t>((j >> 1) & 1) << s);
+        tma_load_3d(ring + s * TILE_BYTES, map, &full[s], kvh * DH, k0, b);
+        tma_load_3d(ring + s * TILE_BYTES + HALF, map, &full[s], kvh * DH + 64, k0, b);
+        iss |= 1u << s;
+        par = (par & ~(1u << s)) | (static_cast<uint32_t>((j >> 1) & 1) << s);
         return true;
       };
       // consumption order of the UMMA issuer: K0 K1 V0 K2 V1 K3 V2 ...
       int kj = 0, vj = 0;
-      while (ok && kj < n && kj < 2) ok = issue_k(kj++);
+      while (ok && kj < n && kj < 2) ok = issue_kv(sK, &tmK, k_full, k_empty, kj++, k_iss, k_par);
       while (ok && vj < n) {
-        ok = issue_v(vj++);
-        if (ok && kj < n) ok = issue_k(kj++);
+        ok = issue_kv(sV, &tmV, v_full, v_empty, vj++, v_iss, v_par);
+        if (ok && kj < n) ok = issue_kv(sK, &tmK, k_full, k_empty, kj++, k_iss, k_par);
       }
       int never = 0;
       // drain: every issued copy lands before the CTA may exit
@@ -171,7 +164,7 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       // ---------------------------------------------------------------- UMMA issuer
       bool ok = mbar_wait(q_full, 0, p.status, abort_flag);
-      const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
+      const uint32_t q_addr = smem_u32(sQ);
       auto issue_s = [&](int j) -> bool {
         const int s = j & 1;
         const uint32_t par = (j >> 1) & 1;
@@ -193,18 +186,21 @@ __global__ void __launch_bounds__(192, 1)
       if (ok && n > 1) ok = issue_s(1);
       for (int j = 0; ok && j < n; ++j) {
         const int s = j & 1;
-        if (!mbar_wait(p_full, j & 1, p.status, abort_flag)) break;
-        if (!mbar_wait(&v_full[s], (j >> 1) & 1, p.status, abort_flag)) break;
+        const uint32_t par = (j >> 1) & 1;
+        if (!mbar_wait(&p_full[s], par, p.status, abort_flag)) break;
+        if (!mbar_wait(&v_full[s], par, p.status, abort_flag)) break;
         tc_fence_after();
+        const uint32_t p_addr = smem_u32(sP + s * TILE_BYTES);
         const uint32_t v_addr = smem_u32(sV + s * TILE_BYTES);
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k) {
           const uint32_t a_off = (k >> 2) * HALF + (k & 3) * 32;  // P: K-major, keys 16k..16k+15
           const uint32_t b_off = k * 16 * 128;                      // V: MN-major, key rows 16k..
           umma_bf16_ss(tO, sdesc_sw128(p_addr + a_off, 16, 1024), sdesc_sw128(v_addr + b_off, HALF, 1024), IDESC_PV,
-                       k != 0 ? 1u : 0u);
+                       (j | k) != 0 ? 1u : 0u);
         }
-        umma_commit(o_full);
+        umma_commit(o_done);
+        umma_commit(&p_free[s]);
         umma_commit(&v_empty[s]);
         if (j + 2 < n) ok = issue_s(j + 2);
       }
@@ -214,111 +210,119 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax
+    // One query row per thread.  O accumulates in TMEM across KV blocks with a lazy
+    // rescale: P is taken relative to the running max m_used, which moves (and O, l
+    // are rescaled by exp2(m_old - m_new)) only when a block raises the row max by
+    // more than 2^8, so P stays below 256 and the rescale is rare.
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int i = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    float o_acc[DH];
-#pragma unroll
-    for (int d = 0; d < DH; ++d) o_acc[d] = 0.f;
-    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+    constexpr float kRescaleLog2 = 8.0f;
+    float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* prow = sP + r * 128;
     for (int j = 0; j < n; ++j) {
       const int s = j & 1;
+      const uint32_t par = (j >> 1) & 1;
       const int k0 = bl.block(j) * BKV;
       const bool need_mask =
           !((k0 + BKV - 1 <= q0) && (p.window < 0 || q0 + BQ - 1 - k0 <= p.window || k0 + BKV - 1 < p.n_meta));
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[s], (j >> 1) & 1, p.status, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[s], par, p.status, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t sbase = tS + s * 128 + lane_off;
-      // pass 1: row max over the visible keys of this block
+      uint32_t sv[128];
+      {
+        uint32_t (&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
+        uint32_t (&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
+        uint32_t (&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[64]);
+        uint32_t (&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[96]);
+        const uint32_t sb = tS + s * 128 + lane_off;
+        tmem_ld32(sb, c0);
+        tmem_ld32(sb + 32, c1);
+        tmem_ld32(sb + 64, c2);
+        tmem_ld32(sb + 96, c3);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[s]);
+      if (need_mask) {
+#pragma unroll
+        for (int e = 0; e < 128; ++e)
+          if (!visible(i, k0 + e, p.n_meta, p.window)) sv[e] = __float_as_uint(-INFINITY);
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(sbase + c * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float sv = __uint_as_float(v[e]);
-          const bool vis = !need_mask || visible(i, k0 + c * 32 + e, p.n_meta, p.window);
-          mx = vis ? fmaxf(mx, sv) : mx;
-        }
+      for (int e = 0; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
+      const float m_cand = mx * p.scale_log2;
+      const bool need = m_cand > m_used + kRescaleLog2;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2_approx(m_used - m_cand);  // 0 when m_used is -inf
+        m_used = m_cand;
       }
-      const float m_new = fmaxf(m, mx * p.scale_log2);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2_approx(m - m_use);
-      // fold in the previous block's P V (its smem P and TMEM O are then free)
-      if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(o_full, (j - 1) & 1, p.status, abort_flag))) {
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // rescale the O rows accumulated so far (all earlier P V must have landed)
+        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, p.status, abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tO + lane_off + c * 32, v);
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o_acc[c * 32 + e] = fmaf(o_acc[c * 32 + e], alpha_prev, __uint_as_float(v[e]));
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + lane_off + c * 32, o);
         }
+        tmem_wait_st();
       }
-      // pass 2: P = exp2(s * scale_log2 - m) in bf16 into the swizzled P tile
+      const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
       float sum = 0.f;
+      if (!__all_sync(0xffffffffu, mbar_wait(&p_free[s], par ^ 1u, p.status, abort_flag))) {
+        ok = false;
+        break;
+      }
+      uint8_t* prow = sP + s * TILE_BYTES + r * 128;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(sbase + c * 32, v);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const bool v0 = !need_mask || visible(i, k0 + c * 32 + e, p.n_meta, p.window);
-          const bool v1 = !need_mask || visible(i, k0 + c * 32 + e + 1, p.n_meta, p.window);
-          const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(v[e]), p.scale_log2, -m_use)) : 0.f;
-          const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -m_use)) : 0.f;
-          sum += p0 + p1;
-          pk[e >> 1] = pack_bf16(p0, p1);
-        }
+      for (int chunk = 0; chunk < 16; ++chunk) {  // 16-byte chunk = keys 8*chunk .. 8*chunk+7
+        uint32_t pk[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int chunk = c * 4 + q;  // 16-byte chunk = keys 8*chunk .. 8*chunk+7
-          uint8_t* dst = prow + (chunk >> 3) * HALF + (((chunk & 7) ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[8 * chunk + 2 * q]), p.scale_log2, -m_ref));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[8 * chunk + 2 * q + 1]), p.scale_log2, -m_ref));
+          sum += p0 + p1;
+          pk[q] = pack_bf16(p0, p1);
         }
+        uint8_t* dst = prow + (chunk >> 3) * HALF + (((chunk & 7) ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[s]);
-      fence_proxy_async_smem();
-      mbar_arrive(p_full);
       l = fmaf(l, alpha, sum);
-      m = m_new;
-      alpha_prev = alpha;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[s]);
     }
-    if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(o_full, (n - 1) & 1, p.status, abort_flag))) {
+    if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(o_done, (n - 1) & 1, p.status, abort_flag))) {
       tc_fence_after();
+      const float inv = 1.f / l;
+      __nv_bfloat16* orow = p.out + (static_cast<long long>(b) * p.T + i) * p.out_ld + h * DH;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tO + lane_off + c * 32, v);
+        uint32_t o[32];
+        tmem_ld32(tO + lane_off + c * 32, o);
         tmem_wait_ld();
+        if (i < p.T) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o_acc[c * 32 + e] = fmaf(o_acc[c * 32 + e], alpha_prev, __uint_as_float(v[e]));
-      }
-      if (i < p.T) {
-        const float inv = 1.f / l;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(b) * p.T + i) * p.out_ld + h * DH);
-#pragma unroll
-        for (int q = 0; q < DH / 8; ++q)
-          dst[q] = make_uint4(pack_bf16(o_acc[8 * q] * inv, o_acc[8 * q + 1] * inv),
-                              pack_bf16(o_acc[8 * q + 2] * inv, o_acc[8 * q + 3] * inv),
-                              pack_bf16(o_acc[8 * q + 4] * inv, o_acc[8 * q + 5] * inv),
-                              pack_bf16(o_acc[8 * q + 6] * inv, o_acc[8 * q + 7] * inv));
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16(__uint_as_float(o[8 * q]) * inv, __uint_as_float(o[8 * q + 1]) * inv),
+                                pack_bf16(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv),
+                                pack_bf16(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv),
+                                pack_bf16(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv));
+        }
       }
     }
   }

@@ -188,6 +188,285 @@ __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------------
+// N <= 32: TMA-staged variant.  Each lane owns two adjacent channels with all N state
+// components (packed fp32x2 pairs), a warp owns 64 channels (one 128-byte row segment
+// per time step for bf16), and each warp streams its own time chunk through a
+// private STAGES-deep ring of ROWS-step tiles (x, dt, gate, B|C) loaded by TMA, so
+// the sequential recurrence never waits on a global load.  The chunk-combine buffer
+// aliases the ring (used only between the two passes, when no copy is in flight).
+template <typename TI, int N>
+struct PairCfg {
+  static constexpr int NWT = 8;    // time-chunk warps per CTA
+  static constexpr int ROWS = 8;   // time steps per staged tile
+  static constexpr int STAGES = 3;
+  static constexpr int CPW = 64;   // channels per warp (2 per lane)
+  static constexpr int XB = ROWS * CPW * (int)sizeof(TI);  // bytes of one x / dt / gate tile
+  static constexpr int BCB = ROWS * 2 * N * 4;              // bytes of one B|C tile
+  static constexpr int STAGE_B = 3 * XB + BCB;
+  static constexpr int WARP_B = STAGES * STAGE_B;
+  static constexpr int RING_B = NWT * WARP_B;
+  static constexpr int COMBINE_B = NWT * CPW * N * 4 + NWT * CPW * 4;
+  static constexpr int SMEM = (RING_B > COMBINE_B ? RING_B : COMBINE_B) + NWT * STAGES * 8 + 16 + 128;
+};
+
+template <typename TI> struct Pair2;
+template <> struct Pair2<__nv_bfloat16> {
+  static HY_DEV float2 ld(const uint8_t* p) {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    return make_float2(bf16lo(u), bf16hi(u));
+  }
+  static HY_DEV void st(__nv_bfloat16* p, float a, float b) { *reinterpret_cast<uint32_t*>(p) = pack_bf16(a, b); }
+};
+template <> struct Pair2<float> {
+  static HY_DEV float2 ld(const uint8_t* p) { return *reinterpret_cast<const float2*>(p); }
+  static HY_DEV void st(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+};
+
+template <typename TI, int N>
+__global__ void __launch_bounds__(256) scan_pair_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                        const __grid_constant__ CUtensorMap tmDT,
+                                                        const __grid_constant__ CUtensorMap tmG,
+                                                        const __grid_constant__ CUtensorMap tmBC,
+                                                        const ScanParams p, unsigned* status) {
+  using C = PairCfg<TI, N>;
+  constexpr int NP = N / 2;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (C::RING_B > C::COMBINE_B ? C::RING_B : C::COMBINE_B));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + C::NWT * C::STAGES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int c0 = blockIdx.x * C::CPW + 2 * lane;  // this lane's first channel
+  const int Lc = (p.T + C::NWT - 1) / C::NWT;
+  const int t0 = min(p.T, warp * Lc), t1 = min(p.T, t0 + Lc);
+  const int n_tiles = (t1 - t0 + C::ROWS - 1) / C::ROWS;
+  const int grow0 = b * p.T + t0;  // global row of the chunk start
+  uint8_t* ring = smem + warp * C::WARP_B;
+  uint64_t* my_full = full + warp * C::STAGES;
+
+  if (threadIdx.x == 0) *abort_flag = 0;
+  if (lane == 0)
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(&my_full[s], 1);
+  fence_mbar_init();
+  __syncthreads();
+
+  float A2[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) A2[q] = c0 + q < p.Di ? -expf(p.a_log[c0 + q]) * 1.4426950408889634f : 0.f;
+
+  // Ring bookkeeping shared by both passes: the i-th tile issued by this warp goes to
+  // slot i % STAGES and completes phase (i / STAGES) & 1 of that slot's mbarrier;
+  // tiles are consumed in issue order.
+  uint32_t issued = 0;
+  auto issue = [&](int k, bool with_gate) {  // tile k of this warp's chunk
+    if (lane == 0) {
+      const int slot = issued % C::STAGES;
+      uint8_t* st = ring + slot * C::STAGE_B;
+      uint64_t* bar = &my_full[slot];
+      mbar_arrive_expect_tx(bar, (with_gate ? 3 : 2) * C::XB + C::BCB);
+      const int row = grow0 + k * C::ROWS, col = blockIdx.x * C::CPW;
+      tma_load_2d(st, &tmX, bar, col, row);
+      tma_load_2d(st + C::XB, &tmDT, bar, col, row);
+      if (with_gate) tma_load_2d(st + 2 * C::XB, &tmG, bar, col, row);
+      tma_load_2d(st + 3 * C::XB, &tmBC, bar, 0, row);
+    }
+    ++issued;
+  };
+  uint32_t consumed = 0;
+  auto wait_tile = [&](int slot) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(&my_full[slot], (consumed / C::STAGES) & 1u, status, abort_flag));
+  };
+  auto drain = [&]() {  // after an abort: let this warp's copies in flight land
+    int never = 0;
+    if (lane == 0)
+      for (uint32_t i = consumed; i < issued; ++i)
+        mbar_wait(&my_full[i % C::STAGES], (i / C::STAGES) & 1u, nullptr, &never, 100000000ull);
+    __syncwarp();
+  };
+
+  float2 h[2][NP];
+#pragma unroll
+  for (int q = 0; q < 2; ++q)
+#pragma unroll
+    for (int i = 0; i < NP; ++i) h[q][i] = make_float2(0.f, 0.f);
+  float logdec[2] = {0.f, 0.f};
+  bool ok = true;
+
+  // ---------------- pass 1: local scan from h = 0 (end state and total log-decay)
+  for (int k = 0; k < C::STAGES - 1 && k < n_tiles; ++k) issue(k, false);
+  for (int k = 0; k < n_tiles; ++k) {
+    __syncwarp();
+    if (k + C::STAGES - 1 < n_tiles) issue(k + C::STAGES - 1, false);
+    const int slot = consumed % C::STAGES;
+    if (!wait_tile(slot)) {
+      ok = false;
+      break;
+    }
+    ++consumed;
+    const uint8_t* st = ring + slot * C::STAGE_B;
+    const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
+    for (int r = 0; r < rows; ++r) {
+      const float2 xv = Pair2<TI>::ld(st + (r * C::CPW + 2 * lane) * sizeof(TI));
+      const float2 dv = Pair2<TI>::ld(st + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+      const float4* B4 = reinterpret_cast<const float4*>(st + 3 * C::XB + r * 2 * N * 4);
+      const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
+      float2 a2[2], u2[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const float a = ex2_approx(A2[q] * dq[q]), u = dq[q] * xq[q];
+        a2[q] = make_float2(a, a);
+        u2[q] = make_float2(u, u);
+        logdec[q] = fmaf(A2[q], dq[q], logdec[q]);
+      }
+#pragma unroll
+      for (int j = 0; j < N / 4; ++j) {
+        const float4 bb = B4[j];
+        const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          h[q][2 * j] = __ffma2_rn(a2[q], h[q][2 * j], __fmul2_rn(u2[q], b01));
+          h[q][2 * j + 1] = __ffma2_rn(a2[q], h[q][2 * j + 1], __fmul2_rn(u2[q], b23));
+        }
+      }
+    }
+  }
+  // every issued copy has been consumed (or, after an abort, has landed): the ring is free
+  if (!ok) drain();
+  __syncthreads();
+  float* s_hend = reinterpret_cast<float*>(smem);              // [NWT][CPW][N]
+  float* s_logdec = s_hend + C::NWT * C::CPW * N;              // [NWT][CPW]
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    float2* dst = reinterpret_cast<float2*>(s_hend + (warp * C::CPW + 2 * lane + q) * N);
+#pragma unroll
+    for (int i = 0; i < NP; ++i) dst[i] = h[q][i];
+    s_logdec[warp * C::CPW + 2 * lane + q] = logdec[q];
+  }
+  __syncthreads();
+  // ---------------- combine: state entering this warp's chunk
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+#pragma unroll
+    for (int i = 0; i < NP; ++i) h[q][i] = make_float2(0.f, 0.f);
+    for (int k = 0; k < warp; ++k) {
+      const float dec = ex2_approx(s_logdec[k * C::CPW + 2 * lane + q]);
+      const float2 dec2 = make_float2(dec, dec);
+      const float2* hk = reinterpret_cast<const float2*>(s_hend + (k * C::CPW + 2 * lane + q) * N);
+#pragma unroll
+      for (int i = 0; i < NP; ++i) h[q][i] = __ffma2_rn(dec2, h[q][i], hk[i]);
+    }
+  }
+  fence_proxy_async_smem();  // generic accesses to the ring area before the copies below
+  __syncthreads();           // the ring is reused below
+
+  // ---------------- pass 2: rescan with the carried state, emit gated output
+  TI* Y = static_cast<TI*>(p.y);
+  const bool w0 = c0 < p.Di, w1 = c0 + 1 < p.Di;
+  for (int k = 0; ok && k < C::STAGES - 1 && k < n_tiles; ++k) issue(k, true);
+  for (int k = 0; ok && k < n_tiles; ++k) {
+    __syncwarp();
+    if (k + C::STAGES - 1 < n_tiles) issue(k + C::STAGES - 1, true);
+    const int slot = consumed % C::STAGES;
+    if (!wait_tile(slot)) {
+      ok = false;
+      break;
+    }
+    ++consumed;
+    const uint8_t* st = ring + slot * C::STAGE_B;
+    const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
+    for (int r = 0; r < rows; ++r) {
+      const float2 xv = Pair2<TI>::ld(st + (r * C::CPW + 2 * lane) * sizeof(TI));
+      const float2 dv = Pair2<TI>::ld(st + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+      const float2 gv = Pair2<TI>::ld(st + 2 * C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+      const float4* B4 = reinterpret_cast<const float4*>(st + 3 * C::XB + r * 2 * N * 4);
+      const float4* C4 = B4 + N / 4;
+      const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
+      float2 a2[2], u2[2], y2[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const float a = ex2_approx(A2[q] * dq[q]), u = dq[q] * xq[q];
+        a2[q] = make_float2(a, a);
+        u2[q] = make_float2(u, u);
+        y2[q] = make_float2(0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < N / 4; ++j) {
+        const float4 bb = B4[j], cv = C4[j];
+        const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
+        const float2 c01 = make_float2(cv.x, cv.y), c23 = make_float2(cv.z, cv.w);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          h[q][2 * j] = __ffma2_rn(a2[q], h[q][2 * j], __fmul2_rn(u2[q], b01));
+          h[q][2 * j + 1] = __ffma2_rn(a2[q], h[q][2 * j + 1], __fmul2_rn(u2[q], b23));
+          y2[q] = __ffma2_rn(c01, h[q][2 * j], y2[q]);
+          y2[q] = __ffma2_rn(c23, h[q][2 * j + 1], y2[q]);
+        }
+      }
+      const long long row = static_cast<long long>(grow0) + k * C::ROWS + r;
+      TI* yrow = Y + row * p.y_ld + c0;
+      const float ya = gv.x * (y2[0].x + y2[0].y), yb = gv.y * (y2[1].x + y2[1].y);
+      if (w0 && w1) Pair2<TI>::st(yrow, ya, yb);
+      else if (w0) yrow[0] = from_f<TI>(ya);
+    }
+  }
+  if (!ok) drain();
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn scan_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over [rows, cols] (row stride ld elements), box = bc x br, no swizzle.
+bool map2d(CUtensorMap* m, const void* base, bool f32, long long rows, long long cols, long long ld, int bc, int br) {
+  EncodeTiledFn fn = scan_encode_fn();
+  if (!fn) return false;
+  const int es = f32 ? 4 : 2;
+  cuuint64_t gd[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t gs[1] = {static_cast<cuuint64_t>(ld) * es};
+  cuuint32_t bx[2] = {static_cast<cuuint32_t>(bc), static_cast<cuuint32_t>(br)}, el[2] = {1, 1};
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+            gd, gs, bx, el, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename TI, int N>
+cudaError_t launch_pair(const ScanDesc& s, cudaStream_t st) {
+  using C = PairCfg<TI, N>;
+  const bool f32 = sizeof(TI) == 4;
+  const long long rows = static_cast<long long>(s.batch) * s.T;
+  CUtensorMap tx, td, tg, tb;
+  if (!map2d(&tx, s.x, f32, rows, s.d_inner, s.d_inner, C::CPW, C::ROWS) ||
+      !map2d(&td, s.dt, f32, rows, s.d_inner, s.d_inner, C::CPW, C::ROWS) ||
+      !map2d(&tg, s.gate, f32, rows, s.d_inner, s.d_inner, C::CPW, C::ROWS) ||
+      !map2d(&tb, s.bc, true, rows, 2 * N, 2 * N, 2 * N, C::ROWS))
+    return cudaErrorInvalidValue;
+  static int attr_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 31 && !(attr_mask & (1 << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(scan_pair_kernel<TI, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_mask |= 1 << dev;
+  }
+  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
+  dim3 grid((s.d_inner + C::CPW - 1) / C::CPW, s.batch);
+  scan_pair_kernel<TI, N><<<grid, 32 * C::NWT, C::SMEM, st>>>(tx, td, tg, tb, p, s.status);
+  return cudaGetLastError();
+}
+
 template <typename TI, int NS, int TPC, int NWT>
 cudaError_t launch_one(const ScanDesc& s, cudaStream_t st) {
   constexpr int CPW = 32 / TPC;
@@ -199,9 +478,15 @@ cudaError_t launch_one(const ScanDesc& s, cudaStream_t st) {
 
 template <typename TI>
 cudaError_t launch_t(const ScanDesc& s, cudaStream_t st) {
+  // The TMA-staged pair kernel needs 16-byte aligned bases and row strides for x, dt,
+  // gate, B|C, and 2-channel aligned output stores; otherwise the per-channel kernel runs.
+  auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  const bool pair_ok = (s.d_inner * static_cast<int>(sizeof(TI))) % 16 == 0 && a16(s.x) && a16(s.dt) &&
+                       a16(s.gate) && a16(s.bc) && (s.y_ld % 2) == 0 &&
+                       (reinterpret_cast<uintptr_t>(s.y) % (2 * sizeof(TI))) == 0;
   switch (s.d_state) {
-    case 16: return launch_one<TI, 16, 1, 16>(s, st);
-    case 32: return launch_one<TI, 32, 1, 8>(s, st);
+    case 16: return pair_ok ? launch_pair<TI, 16>(s, st) : launch_one<TI, 16, 1, 16>(s, st);
+    case 32: return pair_ok ? launch_pair<TI, 32>(s, st) : launch_one<TI, 32, 1, 8>(s, st);
     case 64: return launch_one<TI, 32, 2, 8>(s, st);
     case 128: return launch_one<TI, 32, 4, 8>(s, st);
     case 256: return launch_one<TI, 32, 8, 8>(s, st);
