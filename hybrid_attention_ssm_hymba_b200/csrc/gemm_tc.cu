@@ -30,6 +30,7 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int NTHREADS = 320;       // producer warp, MMA warp, 8 epilogue warps
 constexpr int EPI_THREADS = 256;
+constexpr int kMaxBiasSmem = 4096;  // a bias vector up to this length is staged in smem once
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 
 struct GemmParams {
@@ -46,6 +47,8 @@ struct GemmParams {
   __nv_bfloat16* out;
   long long out_ld;
   int swiglu_F;
+  int bias_len;             // > 0: the (single) bias segment's vector is staged in smem
+  const float* bias_src;
   unsigned* status;
 };
 
@@ -55,7 +58,7 @@ struct Cfg {
   static constexpr int STAGE = A_STAGE + B_STAGE;
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;  // + bias_len * 4 when the bias is staged
   static constexpr uint32_t IDESC = idesc_bf16(BM, BN, false, false);
 };
 
@@ -73,7 +76,8 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int tile) 
 }
 
 // Store 16 consecutive accumulator columns [c0, c0 + 16) of one output row.
-__device__ __forceinline__ void store16(const GemmParams& p, long long row, int c0, const uint32_t* v) {
+__device__ __forceinline__ void store16(const GemmParams& p, long long row, int c0, const uint32_t* v,
+                                        const float* tile_bias) {
   int s = 0;
   while (s + 1 < p.nseg && c0 >= p.seg[s].col1) ++s;
   const Seg& sg = p.seg[s];
@@ -85,7 +89,7 @@ __device__ __forceinline__ void store16(const GemmParams& p, long long row, int 
 #pragma unroll
     for (int i = 0; i < 16; ++i) f[i] = silu_f(f[i]);
   } else if (sg.op == SEG_SOFTPLUS_BIAS) {
-    const float4* bb = reinterpret_cast<const float4*>(sg.bias + (c0 - sg.col0));
+    const float4* bb = reinterpret_cast<const float4*>((tile_bias ? tile_bias : sg.bias) + (c0 - sg.col0));
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float4 b4 = bb[j];
@@ -126,6 +130,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_bias = reinterpret_cast<float*>(sB + C::STAGES * C::B_STAGE + 256);  // [bias_len]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -145,6 +150,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  for (int i = threadIdx.x; i < p.bias_len; i += blockDim.x) s_bias[i] = p.bias_src[i];
   if (threadIdx.x == 0) {
     tma_prefetch(&tmA);
     tma_prefetch(&tmB);
@@ -284,8 +290,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_wait_ld();
           const int col = tc.n * BN + c * 32;
           if (valid) {
-            if (col < p.N) store16(p, grow, col, v);
-            if (col + 16 < p.N) store16(p, grow, col + 16, v + 16);
+            const float* tb_bias = p.bias_len ? s_bias : nullptr;
+            if (col < p.N) store16(p, grow, col, v, tb_bias);
+            if (col + 16 < p.N) store16(p, grow, col + 16, v + 16, tb_bias);
           }
         }
       } else if (p.epi == EPI_SWIGLU) {
@@ -383,11 +390,14 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
 template <int BN>
 cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
   using C = Cfg<BN>;
-  static bool attr_done = false;  // per process; all B200s share the attribute value
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  static int attr_mask = 0;  // the attribute is per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 31 && !(attr_mask & (1 << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM + kMaxBiasSmem * 4);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    attr_mask |= 1 << dev;
   }
   CUtensorMap tmA, tmAx2, tmM1, tmM2, tmB;
   const uint64_t K = static_cast<uint64_t>(g.K);
@@ -445,7 +455,18 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
   p.k_blocks = (g.K + BK - 1) / BK;
   p.epi = g.epi;
   p.nseg = g.nseg;
-  for (int i = 0; i < g.nseg; ++i) p.seg[i] = g.seg[i];
+  p.bias_len = 0;
+  p.bias_src = nullptr;
+  int n_bias = 0;
+  for (int i = 0; i < g.nseg; ++i) {
+    p.seg[i] = g.seg[i];
+    if (g.seg[i].op == SEG_SOFTPLUS_BIAS) {
+      ++n_bias;
+      p.bias_len = g.seg[i].col1 - g.seg[i].col0;
+      p.bias_src = g.seg[i].bias;
+    }
+  }
+  if (n_bias != 1 || p.bias_len > kMaxBiasSmem) p.bias_len = 0;  // read from global instead
   p.resid = static_cast<const __nv_bfloat16*>(g.resid);
   p.resid_ld = g.resid_ld;
   p.out = static_cast<__nv_bfloat16*>(g.out);
@@ -455,7 +476,7 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
   const long long total = static_cast<long long>(p.meta_mode ? p.batch : 1) * p.m_tiles * p.n_tiles;
   if (total <= 0) return cudaSuccess;
   const int grid = static_cast<int>(total < num_sms() ? total : num_sms());
-  gemm_bf16_tc<BN><<<grid, NTHREADS, C::SMEM, st>>>(tmA, tmAx2, tmM1, tmM2, tmB, p);
+  gemm_bf16_tc<BN><<<grid, NTHREADS, C::SMEM + p.bias_len * 4, st>>>(tmA, tmAx2, tmM1, tmM2, tmB, p);
   return cudaGetLastError();
 }
 

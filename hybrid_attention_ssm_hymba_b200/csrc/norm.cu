@@ -6,8 +6,9 @@
 //     "PyTorch伪代码": one RMSNorm per branch).
 //   rmsnorm:     y = x / sqrt(mean(x^2) + eps), unit gain (pre-norm of the
 //     stacked blocks).
-// One CTA per row; fp32 sums; 16-byte vector loads and stores.  HBM-bound: one
-// read for the sums (the second read of the row hits L1/L2) and one write.
+// bf16 rows up to 6144 elements: one warp per row with the row held in registers
+// (one HBM read, one write).  Wider rows and fp32: one CTA per row (the second read
+// of the row hits L1/L2).  fp32 sums; 16-byte vector loads and stores.
 #include "hy_common.cuh"
 #include "hy_kernels.h"
 
@@ -112,11 +113,98 @@ __global__ void __launch_bounds__(NT) rmsnorm_kernel(const T* x, T* y, int d, fl
   scale_row(x + off, y + off, d, rsqrtf(s / d + eps), nullptr);
 }
 
+// bf16 rows up to 32 * 8 * MAXV elements: one warp per row, the row held in
+// registers (16-byte vectors, lane-interleaved), one read and one write of HBM,
+// warp-shuffle sums.  `wa` (the first branch's width) is a multiple of 8, so no
+// vector straddles the two branches; wa = 0 gives a plain unit-gain RMSNorm.
+template <int MAXV>
+__global__ void __launch_bounds__(256) rownorm_warp_kernel(const __nv_bfloat16* x,  // x and y may alias
+                                                           __nv_bfloat16* y, long long rows, int wa,
+                                                           int ws, const float* __restrict__ beta1,
+                                                           const float* __restrict__ beta2, float eps) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int W = wa + ws;
+  const int nv = W / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(x + row * W);
+  uint4 v[MAXV];
+  float sa = 0.f, ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int vi = lane + 32 * k;
+    if (vi < nv) {
+      v[k] = src[vi];
+      const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a = bf16lo(u[q]), bb = bf16hi(u[q]);
+        acc = fmaf(a, a, fmaf(bb, bb, acc));
+      }
+      if (vi * 8 < wa) sa += acc;
+      else ss += acc;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sa += __shfl_xor_sync(0xffffffffu, sa, o);
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  }
+  const float ra = wa > 0 ? rsqrtf(sa / wa + eps) : 0.f, rs = rsqrtf(ss / ws + eps);
+  uint4* dst = reinterpret_cast<uint4*>(y + row * W);
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int vi = lane + 32 * k;
+    if (vi < nv) {
+      const int col = vi * 8;
+      const bool first = col < wa;
+      const float r = first ? ra : rs;
+      const float* beta = first ? beta1 + col : (beta2 ? beta2 + (col - wa) : nullptr);
+      const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+      float f[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        f[2 * q] = bf16lo(u[q]) * r;
+        f[2 * q + 1] = bf16hi(u[q]) * r;
+      }
+      if (beta) {
+        const float4 b0 = *reinterpret_cast<const float4*>(beta), b1 = *reinterpret_cast<const float4*>(beta + 4);
+        f[0] *= b0.x; f[1] *= b0.y; f[2] *= b0.z; f[3] *= b0.w;
+        f[4] *= b1.x; f[5] *= b1.y; f[6] *= b1.z; f[7] *= b1.w;
+      }
+      dst[vi] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
+    }
+  }
+}
+
+template <int MAXV>
+void launch_rownorm(const void* x, void* y, long long rows, int wa, int ws, const float* b1, const float* b2,
+                    float eps, cudaStream_t st) {
+  rownorm_warp_kernel<MAXV><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), rows, wa, ws, b1, b2, eps);
+}
+
+// picks the smallest register footprint that holds a row; false if the row is too wide
+bool rownorm_bf16(const void* x, void* y, long long rows, int wa, int ws, const float* b1, const float* b2, float eps,
+                  cudaStream_t st) {
+  const int nv = (wa + ws) / 8;
+  const int per_lane = (nv + 31) / 32;
+  if (per_lane <= 4) launch_rownorm<4>(x, y, rows, wa, ws, b1, b2, eps, st);
+  else if (per_lane <= 8) launch_rownorm<8>(x, y, rows, wa, ws, b1, b2, eps, st);
+  else if (per_lane <= 12) launch_rownorm<12>(x, y, rows, wa, ws, b1, b2, eps, st);
+  else if (per_lane <= 16) launch_rownorm<16>(x, y, rows, wa, ws, b1, b2, eps, st);
+  else if (per_lane <= 24) launch_rownorm<24>(x, y, rows, wa, ws, b1, b2, eps, st);
+  else return false;
+  return true;
+}
+
 }  // namespace
 
 cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, long long rows, int w_attn, int w_ssm,
                                float eps, bool bf16, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
+  if (bf16 && rownorm_bf16(z, z, rows, w_attn, w_ssm, beta1, beta2, eps, st)) return cudaGetLastError();
   if (bf16)
     branch_norm_kernel<__nv_bfloat16><<<static_cast<unsigned>(rows), NT, 0, st>>>(
         static_cast<__nv_bfloat16*>(z), beta1, beta2, w_attn, w_ssm, eps);
@@ -128,6 +216,7 @@ cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, 
 
 cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float eps, bool bf16, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
+  if (bf16 && rownorm_bf16(x, y, rows, 0, d, nullptr, nullptr, eps, st)) return cudaGetLastError();
   if (bf16)
     rmsnorm_kernel<__nv_bfloat16><<<static_cast<unsigned>(rows), NT, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), d, eps);

@@ -189,15 +189,26 @@ __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
 }
 
 // ---------------------------------------------------------------------------------
-// N <= 32: TMA-staged variant.  Each lane owns two adjacent channels with all N state
-// components (packed fp32x2 pairs), a warp owns 64 channels (one 128-byte row segment
-// per time step for bf16), and each warp streams its own time chunk through a
-// private STAGES-deep ring of ROWS-step tiles (x, dt, gate, B|C) loaded by TMA, so
-// the sequential recurrence never waits on a global load.  The chunk-combine buffer
-// aliases the ring (used only between the two passes, when no copy is in flight).
+// N <= 32: TMA-staged, scaled-state variant.
+//
+// Each lane owns two adjacent channels with all N state components (packed fp32x2
+// pairs); a warp owns 64 channels (one 128-byte row segment per time step for bf16).
+// A CTA walks T in segments of NWT * SUB steps; inside a segment warp w owns SUB
+// consecutive steps and streams them through a private STAGES-deep ring of ROWS-step
+// TMA tiles (x, dt, gate, B|C), so the recurrence never waits on a global load and
+// the second pass re-reads data that is still in L2.
+//
+// Scaled state: with P_t = prod_{s<=t} exp(A dt_s) (since the last rescale) and
+// g_t = h_t / P_t, the recurrence becomes g_t = g_{t-1} + (dt_t x_t / P_t) B_t and
+// y_t = P_t (C_t . g_t): one FMA per state component per step instead of two.
+// P is kept as its log2 (cl); when it would fall below 2^-60 the scale is folded
+// back into g (g <- P g, cl <- 0), and a single step that decays by more than 2^-60
+// simply restarts the state (its contribution from h_{t-1} is below 2^-60).
 template <typename TI, int N>
 struct PairCfg {
-  static constexpr int NWT = 8;    // time-chunk warps per CTA
+  static constexpr int NWT = 8;    // warps per CTA
+  static constexpr int SUB = 64;   // steps per warp per segment
+  static constexpr int SEG = NWT * SUB;
   static constexpr int ROWS = 8;   // time steps per staged tile
   static constexpr int STAGES = 3;
   static constexpr int CPW = 64;   // channels per warp (2 per lane)
@@ -207,7 +218,9 @@ struct PairCfg {
   static constexpr int WARP_B = STAGES * STAGE_B;
   static constexpr int RING_B = NWT * WARP_B;
   static constexpr int COMBINE_B = NWT * CPW * N * 4 + NWT * CPW * 4;
-  static constexpr int SMEM = (RING_B > COMBINE_B ? RING_B : COMBINE_B) + NWT * STAGES * 8 + 16 + 128;
+  static constexpr int AREA_B = RING_B > COMBINE_B ? RING_B : COMBINE_B;
+  static constexpr int CARRY_B = 2 * CPW * N * 4;
+  static constexpr int SMEM = AREA_B + CARRY_B + NWT * STAGES * 8 + 16 + 128;
 };
 
 template <typename TI> struct Pair2;
@@ -223,6 +236,42 @@ template <> struct Pair2<float> {
   static HY_DEV void st(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
 };
 
+HY_DEV float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int NP>
+struct ScaledState {
+  float2 g[NP];
+  float cl;  // log2 of the scale P
+  HY_DEV void zero() {
+#pragma unroll
+    for (int i = 0; i < NP; ++i) g[i] = make_float2(0.f, 0.f);
+    cl = 0.f;
+  }
+  // advance the scale by one step of log2-decay l2a; returns 1 / P_t
+  HY_DEV float advance(float l2a) {
+    float c = cl + l2a;
+    if (c < -60.f) {  // rare: fold the scale into g
+      const float P = ex2_approx(cl);
+      const float2 P2 = make_float2(P, P);
+#pragma unroll
+      for (int i = 0; i < NP; ++i) g[i] = __fmul2_rn(g[i], P2);
+      if (l2a < -60.f) {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) g[i] = make_float2(0.f, 0.f);
+        c = 0.f;
+      } else {
+        c = l2a;
+      }
+    }
+    cl = c;
+    return ex2_approx(-c);
+  }
+};
+
 template <typename TI, int N>
 __global__ void __launch_bounds__(256) scan_pair_kernel(const __grid_constant__ CUtensorMap tmX,
                                                         const __grid_constant__ CUtensorMap tmDT,
@@ -232,50 +281,52 @@ __global__ void __launch_bounds__(256) scan_pair_kernel(const __grid_constant__ 
   using C = PairCfg<TI, N>;
   constexpr int NP = N / 2;
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (C::RING_B > C::COMBINE_B ? C::RING_B : C::COMBINE_B));
+  float* s_carry = reinterpret_cast<float*>(smem + C::AREA_B);  // [2][CPW][N]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::AREA_B + C::CARRY_B);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(full + C::NWT * C::STAGES);
+  float* s_hend = reinterpret_cast<float*>(smem);       // [NWT][CPW][N]  (aliases the ring)
+  float* s_logdec = s_hend + C::NWT * C::CPW * N;       // [NWT][CPW]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int c0 = blockIdx.x * C::CPW + 2 * lane;  // this lane's first channel
-  const int Lc = (p.T + C::NWT - 1) / C::NWT;
-  const int t0 = min(p.T, warp * Lc), t1 = min(p.T, t0 + Lc);
-  const int n_tiles = (t1 - t0 + C::ROWS - 1) / C::ROWS;
-  const int grow0 = b * p.T + t0;  // global row of the chunk start
   uint8_t* ring = smem + warp * C::WARP_B;
   uint64_t* my_full = full + warp * C::STAGES;
 
   if (threadIdx.x == 0) *abort_flag = 0;
   if (lane == 0)
     for (int s = 0; s < C::STAGES; ++s) mbar_init(&my_full[s], 1);
+  for (int i = threadIdx.x; i < C::CPW * N; i += blockDim.x) s_carry[i] = 0.f;  // h = 0 before the first row
   fence_mbar_init();
   __syncthreads();
 
   float A2[2];
 #pragma unroll
   for (int q = 0; q < 2; ++q) A2[q] = c0 + q < p.Di ? -expf(p.a_log[c0 + q]) * 1.4426950408889634f : 0.f;
+  const bool w0 = c0 < p.Di, w1 = c0 + 1 < p.Di;
+  TI* Y = static_cast<TI*>(p.y);
 
-  // Ring bookkeeping shared by both passes: the i-th tile issued by this warp goes to
-  // slot i % STAGES and completes phase (i / STAGES) & 1 of that slot's mbarrier;
-  // tiles are consumed in issue order.
-  uint32_t issued = 0;
-  auto issue = [&](int k, bool with_gate) {  // tile k of this warp's chunk
+  // Ring bookkeeping across segments and passes: the i-th tile issued by this warp
+  // goes to slot i % STAGES and completes phase (i / STAGES) & 1 of that slot's
+  // mbarrier; tiles are consumed in issue order.
+  uint32_t issued = 0, consumed = 0;
+  auto issue = [&](int grow, bool with_gate) {
     if (lane == 0) {
       const int slot = issued % C::STAGES;
       uint8_t* st = ring + slot * C::STAGE_B;
       uint64_t* bar = &my_full[slot];
       mbar_arrive_expect_tx(bar, (with_gate ? 3 : 2) * C::XB + C::BCB);
-      const int row = grow0 + k * C::ROWS, col = blockIdx.x * C::CPW;
-      tma_load_2d(st, &tmX, bar, col, row);
-      tma_load_2d(st + C::XB, &tmDT, bar, col, row);
-      if (with_gate) tma_load_2d(st + 2 * C::XB, &tmG, bar, col, row);
-      tma_load_2d(st + 3 * C::XB, &tmBC, bar, 0, row);
+      const int col = blockIdx.x * C::CPW;
+      tma_load_2d(st, &tmX, bar, col, grow);
+      tma_load_2d(st + C::XB, &tmDT, bar, col, grow);
+      if (with_gate) tma_load_2d(st + 2 * C::XB, &tmG, bar, col, grow);
+      tma_load_2d(st + 3 * C::XB, &tmBC, bar, 0, grow);
     }
     ++issued;
   };
-  uint32_t consumed = 0;
-  auto wait_tile = [&](int slot) -> bool {
-    return __all_sync(0xffffffffu, mbar_wait(&my_full[slot], (consumed / C::STAGES) & 1u, status, abort_flag));
+  auto wait_tile = [&]() -> bool {
+    return __all_sync(0xffffffffu,
+                      mbar_wait(&my_full[consumed % C::STAGES], (consumed / C::STAGES) & 1u, status, abort_flag));
   };
   auto drain = [&]() {  // after an abort: let this warp's copies in flight land
     int never = 0;
@@ -285,132 +336,152 @@ __global__ void __launch_bounds__(256) scan_pair_kernel(const __grid_constant__ 
     __syncwarp();
   };
 
-  float2 h[2][NP];
-#pragma unroll
-  for (int q = 0; q < 2; ++q)
-#pragma unroll
-    for (int i = 0; i < NP; ++i) h[q][i] = make_float2(0.f, 0.f);
-  float logdec[2] = {0.f, 0.f};
   bool ok = true;
-
-  // ---------------- pass 1: local scan from h = 0 (end state and total log-decay)
-  for (int k = 0; k < C::STAGES - 1 && k < n_tiles; ++k) issue(k, false);
-  for (int k = 0; k < n_tiles; ++k) {
-    __syncwarp();
-    if (k + C::STAGES - 1 < n_tiles) issue(k + C::STAGES - 1, false);
-    const int slot = consumed % C::STAGES;
-    if (!wait_tile(slot)) {
-      ok = false;
-      break;
-    }
-    ++consumed;
-    const uint8_t* st = ring + slot * C::STAGE_B;
-    const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
-    for (int r = 0; r < rows; ++r) {
-      const float2 xv = Pair2<TI>::ld(st + (r * C::CPW + 2 * lane) * sizeof(TI));
-      const float2 dv = Pair2<TI>::ld(st + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-      const float4* B4 = reinterpret_cast<const float4*>(st + 3 * C::XB + r * 2 * N * 4);
-      const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
-      float2 a2[2], u2[2];
+  ScaledState<NP> st[2];
+  int seg_id = 0;
+  for (int seg0 = 0; seg0 < p.T; seg0 += C::SEG, ++seg_id) {
+    const int t0 = min(p.T, seg0 + warp * C::SUB), t1 = min(p.T, min(seg0 + C::SEG, t0 + C::SUB));
+    const int n_tiles = (t1 - t0 + C::ROWS - 1) / C::ROWS;
+    const int grow0 = b * p.T + t0;
+    // ---------------- pass 1: local scan from h = 0 -> end state and total log2-decay
+    float logdec[2] = {0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const float a = ex2_approx(A2[q] * dq[q]), u = dq[q] * xq[q];
-        a2[q] = make_float2(a, a);
-        u2[q] = make_float2(u, u);
-        logdec[q] = fmaf(A2[q], dq[q], logdec[q]);
+    for (int q = 0; q < 2; ++q) st[q].zero();
+    for (int k = 0; ok && k < C::STAGES - 1 && k < n_tiles; ++k) issue(grow0 + k * C::ROWS, false);
+    for (int k = 0; ok && k < n_tiles; ++k) {
+      __syncwarp();
+      if (k + C::STAGES - 1 < n_tiles) issue(grow0 + (k + C::STAGES - 1) * C::ROWS, false);
+      const uint8_t* tile = ring + (consumed % C::STAGES) * C::STAGE_B;
+      if (!wait_tile()) {
+        ok = false;
+        break;
       }
-#pragma unroll
-      for (int j = 0; j < N / 4; ++j) {
-        const float4 bb = B4[j];
-        const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
+      ++consumed;
+      const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
+      for (int r = 0; r < rows; ++r) {
+        const float2 xv = Pair2<TI>::ld(tile + (r * C::CPW + 2 * lane) * sizeof(TI));
+        const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+        const float4* B4 = reinterpret_cast<const float4*>(tile + 3 * C::XB + r * 2 * N * 4);
+        const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
+        float2 q2[2];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          h[q][2 * j] = __ffma2_rn(a2[q], h[q][2 * j], __fmul2_rn(u2[q], b01));
-          h[q][2 * j + 1] = __ffma2_rn(a2[q], h[q][2 * j + 1], __fmul2_rn(u2[q], b23));
+          const float l2a = A2[q] * dq[q];
+          logdec[q] += l2a;
+          const float v = dq[q] * xq[q] * st[q].advance(l2a);
+          q2[q] = make_float2(v, v);
+        }
+#pragma unroll
+        for (int j = 0; j < N / 4; ++j) {
+          const float4 bb = B4[j];
+          const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            st[q].g[2 * j] = __ffma2_rn(q2[q], b01, st[q].g[2 * j]);
+            st[q].g[2 * j + 1] = __ffma2_rn(q2[q], b23, st[q].g[2 * j + 1]);
+          }
         }
       }
     }
-  }
-  // every issued copy has been consumed (or, after an abort, has landed): the ring is free
-  if (!ok) drain();
-  __syncthreads();
-  float* s_hend = reinterpret_cast<float*>(smem);              // [NWT][CPW][N]
-  float* s_logdec = s_hend + C::NWT * C::CPW * N;              // [NWT][CPW]
+    if (!ok) drain();
+    __syncthreads();  // the ring area becomes the combine area
+    // local end state h_end = P g
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    float2* dst = reinterpret_cast<float2*>(s_hend + (warp * C::CPW + 2 * lane + q) * N);
+    for (int q = 0; q < 2; ++q) {
+      const float P = ex2_approx(st[q].cl);
+      const float2 P2 = make_float2(P, P);
+      float2* dst = reinterpret_cast<float2*>(s_hend + (warp * C::CPW + 2 * lane + q) * N);
 #pragma unroll
-    for (int i = 0; i < NP; ++i) dst[i] = h[q][i];
-    s_logdec[warp * C::CPW + 2 * lane + q] = logdec[q];
-  }
-  __syncthreads();
-  // ---------------- combine: state entering this warp's chunk
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-#pragma unroll
-    for (int i = 0; i < NP; ++i) h[q][i] = make_float2(0.f, 0.f);
-    for (int k = 0; k < warp; ++k) {
-      const float dec = ex2_approx(s_logdec[k * C::CPW + 2 * lane + q]);
-      const float2 dec2 = make_float2(dec, dec);
-      const float2* hk = reinterpret_cast<const float2*>(s_hend + (k * C::CPW + 2 * lane + q) * N);
-#pragma unroll
-      for (int i = 0; i < NP; ++i) h[q][i] = __ffma2_rn(dec2, h[q][i], hk[i]);
+      for (int i = 0; i < NP; ++i) dst[i] = __fmul2_rn(st[q].g[i], P2);
+      s_logdec[warp * C::CPW + 2 * lane + q] = logdec[q];
     }
-  }
-  fence_proxy_async_smem();  // generic accesses to the ring area before the copies below
-  __syncthreads();           // the ring is reused below
-
-  // ---------------- pass 2: rescan with the carried state, emit gated output
-  TI* Y = static_cast<TI*>(p.y);
-  const bool w0 = c0 < p.Di, w1 = c0 + 1 < p.Di;
-  for (int k = 0; ok && k < C::STAGES - 1 && k < n_tiles; ++k) issue(k, true);
-  for (int k = 0; ok && k < n_tiles; ++k) {
-    __syncwarp();
-    if (k + C::STAGES - 1 < n_tiles) issue(k + C::STAGES - 1, true);
-    const int slot = consumed % C::STAGES;
-    if (!wait_tile(slot)) {
-      ok = false;
-      break;
-    }
-    ++consumed;
-    const uint8_t* st = ring + slot * C::STAGE_B;
-    const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
-    for (int r = 0; r < rows; ++r) {
-      const float2 xv = Pair2<TI>::ld(st + (r * C::CPW + 2 * lane) * sizeof(TI));
-      const float2 dv = Pair2<TI>::ld(st + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-      const float2 gv = Pair2<TI>::ld(st + 2 * C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-      const float4* B4 = reinterpret_cast<const float4*>(st + 3 * C::XB + r * 2 * N * 4);
-      const float4* C4 = B4 + N / 4;
-      const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
-      float2 a2[2], u2[2], y2[2];
+    __syncthreads();
+    // ---------------- combine: state entering this warp's steps (chained from the
+    // segment's carry-in), and the last warp also forms the next segment's carry-in
+    const float* carry_in = s_carry + (seg_id & 1) * C::CPW * N;
+    float* carry_out = s_carry + ((seg_id + 1) & 1) * C::CPW * N;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const float a = ex2_approx(A2[q] * dq[q]), u = dq[q] * xq[q];
-        a2[q] = make_float2(a, a);
-        u2[q] = make_float2(u, u);
-        y2[q] = make_float2(0.f, 0.f);
+    for (int q = 0; q < 2; ++q) {
+      const int ch = 2 * lane + q;
+      const float2* cin = reinterpret_cast<const float2*>(carry_in + ch * N);
+#pragma unroll
+      for (int i = 0; i < NP; ++i) st[q].g[i] = cin[i];
+      st[q].cl = 0.f;
+      const int kmax = (warp == C::NWT - 1) ? C::NWT : warp;
+      for (int k = 0; k < kmax; ++k) {
+        if (k == warp) {  // last warp: its own entry state is complete; store it, then go on
+          float2* tmp = reinterpret_cast<float2*>(carry_out + ch * N);
+#pragma unroll
+          for (int i = 0; i < NP; ++i) tmp[i] = st[q].g[i];
+        }
+        const float dec = ex2_approx(s_logdec[k * C::CPW + ch]);
+        const float2 dec2 = make_float2(dec, dec);
+        const float2* hk = reinterpret_cast<const float2*>(s_hend + (k * C::CPW + ch) * N);
+#pragma unroll
+        for (int i = 0; i < NP; ++i) st[q].g[i] = __ffma2_rn(dec2, st[q].g[i], hk[i]);
       }
+      if (warp == C::NWT - 1) {  // g = carry-out (end of segment); restore own entry state
+        float2* co = reinterpret_cast<float2*>(carry_out + ch * N);
 #pragma unroll
-      for (int j = 0; j < N / 4; ++j) {
-        const float4 bb = B4[j], cv = C4[j];
-        const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
-        const float2 c01 = make_float2(cv.x, cv.y), c23 = make_float2(cv.z, cv.w);
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          h[q][2 * j] = __ffma2_rn(a2[q], h[q][2 * j], __fmul2_rn(u2[q], b01));
-          h[q][2 * j + 1] = __ffma2_rn(a2[q], h[q][2 * j + 1], __fmul2_rn(u2[q], b23));
-          y2[q] = __ffma2_rn(c01, h[q][2 * j], y2[q]);
-          y2[q] = __ffma2_rn(c23, h[q][2 * j + 1], y2[q]);
+        for (int i = 0; i < NP; ++i) {
+          const float2 own = co[i];
+          co[i] = st[q].g[i];
+          st[q].g[i] = own;
         }
       }
-      const long long row = static_cast<long long>(grow0) + k * C::ROWS + r;
-      TI* yrow = Y + row * p.y_ld + c0;
-      const float ya = gv.x * (y2[0].x + y2[0].y), yb = gv.y * (y2[1].x + y2[1].y);
-      if (w0 && w1) Pair2<TI>::st(yrow, ya, yb);
-      else if (w0) yrow[0] = from_f<TI>(ya);
     }
+    fence_proxy_async_smem();  // generic accesses to the ring area before the copies below
+    __syncthreads();
+    // ---------------- pass 2: rescan from the carried state, emit y = gate (C . h)
+    for (int k = 0; ok && k < C::STAGES - 1 && k < n_tiles; ++k) issue(grow0 + k * C::ROWS, true);
+    for (int k = 0; ok && k < n_tiles; ++k) {
+      __syncwarp();
+      if (k + C::STAGES - 1 < n_tiles) issue(grow0 + (k + C::STAGES - 1) * C::ROWS, true);
+      const uint8_t* tile = ring + (consumed % C::STAGES) * C::STAGE_B;
+      if (!wait_tile()) {
+        ok = false;
+        break;
+      }
+      ++consumed;
+      const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
+      for (int r = 0; r < rows; ++r) {
+        const float2 xv = Pair2<TI>::ld(tile + (r * C::CPW + 2 * lane) * sizeof(TI));
+        const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+        const float2 gv = Pair2<TI>::ld(tile + 2 * C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+        const float4* B4 = reinterpret_cast<const float4*>(tile + 3 * C::XB + r * 2 * N * 4);
+        const float4* C4 = B4 + N / 4;
+        const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
+        float2 q2[2], y2[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float v = dq[q] * xq[q] * st[q].advance(A2[q] * dq[q]);
+          q2[q] = make_float2(v, v);
+          y2[q] = make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < N / 4; ++j) {
+          const float4 bb = B4[j], cv = C4[j];
+          const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
+          const float2 c01 = make_float2(cv.x, cv.y), c23 = make_float2(cv.z, cv.w);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            st[q].g[2 * j] = __ffma2_rn(q2[q], b01, st[q].g[2 * j]);
+            st[q].g[2 * j + 1] = __ffma2_rn(q2[q], b23, st[q].g[2 * j + 1]);
+            y2[q] = __ffma2_rn(c01, st[q].g[2 * j], y2[q]);
+            y2[q] = __ffma2_rn(c23, st[q].g[2 * j + 1], y2[q]);
+          }
+        }
+        const long long row = static_cast<long long>(grow0) + k * C::ROWS + r;
+        TI* yrow = Y + row * p.y_ld + c0;
+        const float ya = gv.x * ex2_approx(st[0].cl) * (y2[0].x + y2[0].y);
+        const float yb = gv.y * ex2_approx(st[1].cl) * (y2[1].x + y2[1].y);
+        if (w0 && w1) Pair2<TI>::st(yrow, ya, yb);
+        else if (w0) yrow[0] = from_f<TI>(ya);
+      }
+    }
+    if (!ok) drain();
+    __syncthreads();  // carry-out visible; the ring area is reused by the next segment's pass 1
   }
-  if (!ok) drain();
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

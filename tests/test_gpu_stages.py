@@ -83,6 +83,20 @@ def test_scan_parity(dtype, B, T, Di, N):
     assert_close(_run_scan(inp, B, T, Di, N, dtype), _scan_ref(inp, B, T, Di, N), dtype, "scan")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("N,T", [(16, 1100), (32, 1500)])
+def test_scan_extreme_decay_and_segments(dtype, N, T):
+    """dt up to 6 with |A| up to 16: single steps decaying by more than 2^-60 and long
+    runs of strong decay (the scaled-state fold and restart paths), over several
+    512-step segments; plus a channel count that is not a multiple of 64."""
+    B, Di = 2, 96
+    inp = synth.scan_inputs(24, B, T, Di, N, dtype=dtype)
+    g = np.random.default_rng(5)
+    dt = np.exp(g.uniform(np.log(1e-3), np.log(6.0), size=(B * T, Di))).astype(np.float32)
+    inp["dt"] = synth.round_bf16(dt) if dtype == "bf16" else dt
+    assert_close(_run_scan(inp, B, T, Di, N, dtype), _scan_ref(inp, B, T, Di, N), dtype, "scan extreme decay")
+
+
 def test_scan_long_decay_small_dt():
     """dt down to 1e-4 over 32K steps: fp32 state keeps the long decay products."""
     B, T, Di, N = 1, 32896, 16, 128
