@@ -334,6 +334,271 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ---------------------------------------------------------------------------------
+// Two query heads of one KV head per CTA (GQA groups of even size): the two softmax
+// warpgroups ping-pong against the tensor core and share every K/V tile.
+//   warp 0      TMA producer: Q of both heads once, then K_j / V_j (2-deep rings)
+//   warp 1      UMMA issuer, per block j: P_a V_j, S_a(j+1), P_b V_j, S_b(j+1)
+//   warps 2..5  softmax of head a, warps 6..9 softmax of head b (one row per thread)
+// TMEM (512 columns): S_a | S_b | O_a | O_b, 128 fp32 columns each.  P_x(j) (bf16,
+// two keys per 32-bit column) is written over the consumed S_x(j) columns and read
+// by the P V instruction straight from TMEM, so P never touches shared memory; S_x(j+1)
+// is issued only after P_x V_j has completed.  O accumulates in TMEM with the same
+// lazy rescale as the one-head kernel.
+constexpr int SMEM2_BYTES = 6 * TILE_BYTES + 1024 + 256;
+
+__global__ void __launch_bounds__(320, 1)
+    attn_fwd_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* sQ = smem_raw + pad;       // 2 heads
+  uint8_t* sK = sQ + 2 * TILE_BYTES;  // 2 stages
+  uint8_t* sV = sK + 2 * TILE_BYTES;  // 2 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * TILE_BYTES);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* k_empty = bars + 3;  // [2]
+  uint64_t* v_full = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;  // [2]
+  uint64_t* s_full = bars + 9;   // [head]
+  uint64_t* p_full = bars + 11;  // [head]
+  uint64_t* o_done = bars + 13;  // [head], completes once per P V
+  uint64_t* mma_done = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = p.q_tiles - 1 - static_cast<int>(blockIdx.x);  // longest tiles first
+  const int h0 = 2 * blockIdx.y, b = blockIdx.z;                // heads h0, h0 + 1
+  const int kvh = h0 / (p.Hq / p.Hkv);
+  const int q0 = qt * BQ;
+  const BlockList bl = make_blocks(p, q0);
+  const int n = bl.n;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&o_done[s], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch(&tmQ);
+    tma_prefetch(&tmK);
+    tma_prefetch(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- producer
+      uint32_t k_iss = 0, v_iss = 0, k_par = 0, v_par = 0;
+      bool ok = true;
+      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_3d(sQ + x * TILE_BYTES, &tmQ, q_full, (h0 + x) * DH, q0, b);
+        tma_load_3d(sQ + x * TILE_BYTES + HALF, &tmQ, q_full, (h0 + x) * DH + 64, q0, b);
+      }
+      auto issue_kv = [&](uint8_t* ring, const CUtensorMap* map, uint64_t* full, uint64_t* empty, int j,
+                          uint32_t& iss, uint32_t& par) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1u, p.status, abort_flag)) return false;
+        mbar_arrive_expect_tx(&full[s], TILE_BYTES);
+        const int k0 = bl.block(j) * BKV;
+        tma_load_3d(ring + s * TILE_BYTES, map, &full[s], kvh * DH, k0, b);
+        tma_load_3d(ring + s * TILE_BYTES + HALF, map, &full[s], kvh * DH + 64, k0, b);
+        iss |= 1u << s;
+        par = (par & ~(1u << s)) | (static_cast<uint32_t>((j >> 1) & 1) << s);
+        return true;
+      };
+      // first-use order of the UMMA issuer: K0 V0 K1 V1 K2 V2 ...
+      for (int j = 0; ok && j < n; ++j) {
+        ok = issue_kv(sK, &tmK, k_full, k_empty, j, k_iss, k_par);
+        if (ok) ok = issue_kv(sV, &tmV, v_full, v_empty, j, v_iss, v_par);
+      }
+      int never = 0;
+      for (int s = 0; s < 2; ++s) {
+        if (k_iss & (1u << s)) mbar_wait(&k_full[s], (k_par >> s) & 1u, nullptr, &never, 100000000ull);
+        if (v_iss & (1u << s)) mbar_wait(&v_full[s], (v_par >> s) & 1u, nullptr, &never, 100000000ull);
+      }
+      mbar_wait(q_full, 0, nullptr, &never, 100000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- UMMA issuer
+      bool ok = mbar_wait(q_full, 0, p.status, abort_flag);
+      auto issue_s = [&](int x, int j) {  // S_x(j) = Q_x K_j^T into TMEM columns [128 x, 128 x + 128)
+        const uint32_t q_addr = smem_u32(sQ + x * TILE_BYTES), k_addr = smem_u32(sK + (j & 1) * TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
+          umma_bf16_ss(tmem_base + x * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
+                       IDESC_QK, k != 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[x]);
+      };
+      auto issue_pv = [&](int x, int j) {  // O_x (+)= P_x(j) V_j, P_x from TMEM over S_x
+        const uint32_t v_addr = smem_u32(sV + (j & 1) * TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < BKV / 16; ++k)
+          umma_bf16_ts(tmem_base + 256 + x * 128, tmem_base + x * 128 + k * 8,
+                       sdesc_sw128(v_addr + k * 16 * 128, HALF, 1024), IDESC_PV, (j | k) != 0 ? 1u : 0u);
+        umma_commit(&o_done[x]);
+      };
+      if (ok && n > 0) {
+        ok = mbar_wait(&k_full[0], 0, p.status, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          issue_s(1, 0);
+          umma_commit(&k_empty[0]);
+        }
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const uint32_t par = j & 1;
+        for (int x = 0; ok && x < 2; ++x) {
+          if (!mbar_wait(&p_full[x], par, p.status, abort_flag)) { ok = false; break; }
+          if (x == 0 && !mbar_wait(&v_full[j & 1], (j >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(x, j);
+          if (x == 1) umma_commit(&v_empty[j & 1]);
+          if (j + 1 < n) {
+            // S_x(j+1) overwrites the TMEM columns P_x(j) V_j reads: wait for that MMA
+            if (!mbar_wait(&o_done[x], par, p.status, abort_flag)) { ok = false; break; }
+            if (x == 0 && !mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, p.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(x, j + 1);
+            if (x == 1) umma_commit(&k_empty[(j + 1) & 1]);
+          }
+        }
+      }
+      umma_commit(mma_done);
+      int never = 0;
+      mbar_wait(mma_done, 0, nullptr, &never, 100000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax (two warpgroups)
+    const int x = (warp - 2) >> 2;  // head of this warpgroup
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int i = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tSx = tmem_base + x * 128 + lane_off, tOx = tmem_base + 256 + x * 128 + lane_off;
+    constexpr float kRescaleLog2 = 8.0f;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int k0 = bl.block(j) * BKV;
+      const bool need_mask =
+          !((k0 + BKV - 1 <= q0) && (p.window < 0 || q0 + BQ - 1 - k0 <= p.window || k0 + BKV - 1 < p.n_meta));
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1, p.status, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[128];
+      {
+        uint32_t (&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
+        uint32_t (&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
+        uint32_t (&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[64]);
+        uint32_t (&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[96]);
+        tmem_ld32(tSx, c0);
+        tmem_ld32(tSx + 32, c1);
+        tmem_ld32(tSx + 64, c2);
+        tmem_ld32(tSx + 96, c3);
+        tmem_wait_ld();
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int e = 0; e < 128; ++e)
+          if (!visible(i, k0 + e, p.n_meta, p.window)) sv[e] = __float_as_uint(-INFINITY);
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
+      const float m_cand = mx * p.scale_log2;
+      const bool need = m_cand > m_used + kRescaleLog2;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2_approx(m_used - m_cand);  // 0 when m_used is -inf
+        m_used = m_cand;
+      }
+      const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
+      float sum = 0.f;
+      // P in bf16, packed in place: sv[q] <- (p[2q], p[2q+1]) (reads index >= q first)
+#pragma unroll
+      for (int q = 0; q < 64; ++q) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * q]), p.scale_log2, -m_ref));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * q + 1]), p.scale_log2, -m_ref));
+        sum += p0 + p1;
+        sv[q] = pack_bf16(p0, p1);
+      }
+      tmem_st32(tSx, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_st32(tSx + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // rescale O (every earlier P V of this head has completed: S_x(j) was issued
+        // after it, and P_x V_j cannot start before p_full below)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tOx + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tOx + c * 32, o);
+        }
+      }
+      tmem_wait_st();
+      l = fmaf(l, alpha, sum);
+      tc_fence_before();
+      mbar_arrive(&p_full[x]);
+    }
+    if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(&o_done[x], (n - 1) & 1, p.status, abort_flag))) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      __nv_bfloat16* orow = p.out + (static_cast<long long>(b) * p.T + i) * p.out_ld + (h0 + x) * DH;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tOx + c * 32, o);
+        tmem_wait_ld();
+        if (i < p.T) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16(__uint_as_float(o[8 * q]) * inv, __uint_as_float(o[8 * q + 1]) * inv),
+                                pack_bf16(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv),
+                                pack_bf16(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv),
+                                pack_bf16(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -369,7 +634,7 @@ cudaError_t launch_attention_f32(const AttnDesc& a, cudaStream_t st);
 cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st) {
   if (!a.bf16) return launch_attention_f32(a, st);
   if (a.batch <= 0 || a.T <= 0) return cudaSuccess;
-  static int attr_dev_mask = 0;
+  static int attr_dev_mask = 0, attr2_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 31 && !(attr_dev_mask & (1 << dev))) {
@@ -394,6 +659,16 @@ cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st) {
   p.out_ld = a.out_ld;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(DH));
   p.status = a.status;
+  if ((a.n_q_heads / a.n_kv_heads) % 2 == 0) {  // pairs of query heads share each K/V tile
+    if (dev < 31 && !(attr2_mask & (1 << dev))) {
+      cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+      if (e != cudaSuccess) return e;
+      attr2_mask |= 1 << dev;
+    }
+    dim3 grid(p.q_tiles, a.n_q_heads / 2, a.batch);
+    attn_fwd_tc2<<<grid, 320, SMEM2_BYTES, st>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+  }
   dim3 grid(p.q_tiles, a.n_q_heads, a.batch);
   attn_fwd_tc<<<grid, 192, SMEM_BYTES, st>>>(tq, tk, tv, p);
   return cudaGetLastError();

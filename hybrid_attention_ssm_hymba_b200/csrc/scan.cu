@@ -272,6 +272,103 @@ struct ScaledState {
   }
 };
 
+// Fast path of one full ROWS-step tile.  First folds the running scale into g for
+// every lane (g <- P g, P <- 1), then checks (warp-uniformly) that no lane's decay
+// over the tile passes 2^-60, so that the scales of all its steps can be formed
+// independently; returns false (slow, per-step guarded path) for a partial tile or
+// an extreme decay.
+template <typename TI, int N>
+HY_DEV bool fast_tile(const uint8_t* tile, int lane, int rows, const float (&A2)[2], ScaledState<N / 2> (&st)[2]) {
+  using C = PairCfg<TI, N>;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const float P = ex2_approx(st[q].cl);
+    const float2 P2 = make_float2(P, P);
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) st[q].g[i] = __fmul2_rn(st[q].g[i], P2);
+    st[q].cl = 0.f;
+  }
+  bool ok = rows == C::ROWS;
+  if (ok) {
+    float c[2] = {0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < C::ROWS; ++r) {
+      const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+      c[0] = fmaf(A2[0], dv.x, c[0]);
+      c[1] = fmaf(A2[1], dv.y, c[1]);
+    }
+    ok = c[0] >= -60.f && c[1] >= -60.f;
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Four steps (rows h2 .. h2+3 of a staged tile) of the scaled-state recurrence with
+// no fold needed: the four scales are formed up front (independent SFU ops), then the
+// state chain runs; with EMIT the gated outputs y = gate P (C . g) are stored.
+template <typename TI, int N, bool EMIT>
+HY_DEV void step4(const uint8_t* tile, int lane, int h2, const float (&A2)[2], ScaledState<N / 2> (&st)[2],
+                  float (&logdec)[2], TI* ybase, long long y_ld, int, bool w0, bool w1) {
+  using C = PairCfg<TI, N>;
+  float v[4][2], P[4][2], gate[4][2];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = h2 + k;
+    const float2 xv = Pair2<TI>::ld(tile + (r * C::CPW + 2 * lane) * sizeof(TI));
+    const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+    const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
+    if (EMIT) {
+      const float2 gv = Pair2<TI>::ld(tile + 2 * C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+      gate[k][0] = gv.x;
+      gate[k][1] = gv.y;
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const float l2a = A2[q] * dq[q];
+      if (!EMIT) logdec[q] += l2a;
+      st[q].cl += l2a;
+      v[k][q] = dq[q] * xq[q] * ex2_approx(-st[q].cl);
+      if (EMIT) P[k][q] = ex2_approx(st[q].cl);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = h2 + k;
+    const float4* B4 = reinterpret_cast<const float4*>(tile + 3 * C::XB + r * 2 * N * 4);
+    float2 q2[2], y2[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      q2[q] = make_float2(v[k][q], v[k][q]);
+      y2[q] = make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < N / 4; ++j) {
+      const float4 bb = B4[j];
+      const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        st[q].g[2 * j] = __ffma2_rn(q2[q], b01, st[q].g[2 * j]);
+        st[q].g[2 * j + 1] = __ffma2_rn(q2[q], b23, st[q].g[2 * j + 1]);
+      }
+      if (EMIT) {
+        const float4 cv = B4[N / 4 + j];
+        const float2 c01 = make_float2(cv.x, cv.y), c23 = make_float2(cv.z, cv.w);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          y2[q] = __ffma2_rn(c01, st[q].g[2 * j], y2[q]);
+          y2[q] = __ffma2_rn(c23, st[q].g[2 * j + 1], y2[q]);
+        }
+      }
+    }
+    if (EMIT) {
+      TI* yrow = ybase + r * y_ld;
+      const float ya = gate[k][0] * P[k][0] * (y2[0].x + y2[0].y);
+      const float yb = gate[k][1] * P[k][1] * (y2[1].x + y2[1].y);
+      if (w0 && w1) Pair2<TI>::st(yrow, ya, yb);
+      else if (w0) yrow[0] = from_f<TI>(ya);
+    }
+  }
+}
+
 template <typename TI, int N>
 __global__ void __launch_bounds__(256) scan_pair_kernel(const __grid_constant__ CUtensorMap tmX,
                                                         const __grid_constant__ CUtensorMap tmDT,
@@ -358,27 +455,32 @@ __global__ void __launch_bounds__(256) scan_pair_kernel(const __grid_constant__ 
       }
       ++consumed;
       const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
-      for (int r = 0; r < rows; ++r) {
-        const float2 xv = Pair2<TI>::ld(tile + (r * C::CPW + 2 * lane) * sizeof(TI));
-        const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-        const float4* B4 = reinterpret_cast<const float4*>(tile + 3 * C::XB + r * 2 * N * 4);
-        const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
-        float2 q2[2];
+      if (fast_tile<TI, N>(tile, lane, rows, A2, st)) {
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const float l2a = A2[q] * dq[q];
-          logdec[q] += l2a;
-          const float v = dq[q] * xq[q] * st[q].advance(l2a);
-          q2[q] = make_float2(v, v);
-        }
-#pragma unroll
-        for (int j = 0; j < N / 4; ++j) {
-          const float4 bb = B4[j];
-          const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
+        for (int h2 = 0; h2 < C::ROWS; h2 += 4) step4<TI, N, false>(tile, lane, h2, A2, st, logdec, nullptr, 0, 0, false, false);
+      } else {
+        for (int r = 0; r < rows; ++r) {
+          const float2 xv = Pair2<TI>::ld(tile + (r * C::CPW + 2 * lane) * sizeof(TI));
+          const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
+          const float4* B4 = reinterpret_cast<const float4*>(tile + 3 * C::XB + r * 2 * N * 4);
+          const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
+          float2 q2[2];
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
-            st[q].g[2 * j] = __ffma2_rn(q2[q], b01, st[q].g[2 * j]);
-            st[q].g[2 * j + 1] = __ffma2_rn(q2[q], b23, st[q].g[2 * j + 1]);
+            const float l2a = A2[q] * dq[q];
+            logdec[q] += l2a;
+            const float v = dq[q] * xq[q] * st[q].advance(l2a);
+            q2[q] = make_float2(v, v);
+          }
+#pragma unroll
+          for (int j = 0; j < N / 4; ++j) {
+            const float4 bb = B4[j];
+            const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              st[q].g[2 * j] = __ffma2_rn(q2[q], b01, st[q].g[2 * j]);
+              st[q].g[2 * j + 1] = __ffma2_rn(q2[q], b23, st[q].g[2 * j + 1]);
+            }
           }
         }
       }
@@ -444,6 +546,14 @@ __global__ void __launch_bounds__(256) scan_pair_kernel(const __grid_constant__ 
       }
       ++consumed;
       const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
+      if (fast_tile<TI, N>(tile, lane, rows, A2, st)) {
+        float ld_unused[2] = {0.f, 0.f};
+        TI* ybase = Y + (static_cast<long long>(grow0) + k * C::ROWS) * p.y_ld + c0;
+#pragma unroll
+        for (int h2 = 0; h2 < C::ROWS; h2 += 4)
+          step4<TI, N, true>(tile, lane, h2, A2, st, ld_unused, ybase, p.y_ld, 0, w0, w1);
+        continue;
+      }
       for (int r = 0; r < rows; ++r) {
         const float2 xv = Pair2<TI>::ld(tile + (r * C::CPW + 2 * lane) * sizeof(TI));
         const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
