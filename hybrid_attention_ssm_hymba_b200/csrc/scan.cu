@@ -189,59 +189,23 @@ __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
 }
 
 // ---------------------------------------------------------------------------------
-// N <= 32: TMA-staged, scaled-state variant.
+// Single-pass TMA-staged scan (the main path).
 //
-// Each lane owns two adjacent channels with all N state components (packed fp32x2
-// pairs); a warp owns 64 channels (one 128-byte row segment per time step for bf16).
-// A CTA walks T in segments of NWT * SUB steps; inside a segment warp w owns SUB
-// consecutive steps and streams them through a private STAGES-deep ring of ROWS-step
-// TMA tiles (x, dt, gate, B|C), so the recurrence never waits on a global load and
-// the second pass re-reads data that is still in L2.
+// Each channel is scanned once, sequentially over all T steps (the critical path is
+// T short steps; parallelism comes from channels x state slices).  A channel's N
+// state components are split over TPC lanes (NS each, packed fp32x2 updates) and
+// y = C . h is reduced with shuffles.  A CTA of NWARP warps (CPB channels) shares one
+// STAGES-deep ring of ROWS-step TMA tiles -- x, dt, gate for its channels and the
+// full B|C rows -- filled by one thread and released by the warps through an
+// mbarrier; y goes out through a per-warp smem tile and a TMA store.  Tensor maps
+// are 3-D ([batch][T][cols]), so no tile reads or writes across a sequence end.
 //
-// Scaled state: with P_t = prod_{s<=t} exp(A dt_s) (since the last rescale) and
-// g_t = h_t / P_t, the recurrence becomes g_t = g_{t-1} + (dt_t x_t / P_t) B_t and
-// y_t = P_t (C_t . g_t): one FMA per state component per step instead of two.
-// P is kept as its log2 (cl); when it would fall below 2^-60 the scale is folded
-// back into g (g <- P g, cl <- 0), and a single step that decays by more than 2^-60
-// simply restarts the state (its contribution from h_{t-1} is below 2^-60).
-template <typename TI, int N>
-struct PairCfg {
-  static constexpr int NWT = 8;    // warps per CTA
-  static constexpr int SUB = 64;   // steps per warp per segment
-  static constexpr int SEG = NWT * SUB;
-  static constexpr int ROWS = 8;   // time steps per staged tile
-  static constexpr int STAGES = 3;
-  static constexpr int CPW = 64;   // channels per warp (2 per lane)
-  static constexpr int XB = ROWS * CPW * (int)sizeof(TI);  // bytes of one x / dt / gate tile
-  static constexpr int BCB = ROWS * 2 * N * 4;              // bytes of one B|C tile
-  static constexpr int STAGE_B = 3 * XB + BCB;
-  static constexpr int WARP_B = STAGES * STAGE_B;
-  static constexpr int RING_B = NWT * WARP_B;
-  static constexpr int COMBINE_B = NWT * CPW * N * 4 + NWT * CPW * 4;
-  static constexpr int AREA_B = RING_B > COMBINE_B ? RING_B : COMBINE_B;
-  static constexpr int CARRY_B = 2 * CPW * N * 4;
-  static constexpr int SMEM = AREA_B + CARRY_B + NWT * STAGES * 8 + 16 + 128;
-};
-
-template <typename TI> struct Pair2;
-template <> struct Pair2<__nv_bfloat16> {
-  static HY_DEV float2 ld(const uint8_t* p) {
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
-    return make_float2(bf16lo(u), bf16hi(u));
-  }
-  static HY_DEV void st(__nv_bfloat16* p, float a, float b) { *reinterpret_cast<uint32_t*>(p) = pack_bf16(a, b); }
-};
-template <> struct Pair2<float> {
-  static HY_DEV float2 ld(const uint8_t* p) { return *reinterpret_cast<const float2*>(p); }
-  static HY_DEV void st(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
-};
-
-HY_DEV float rcp_approx(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
+// Scaled state: with P_t = prod exp(A dt_s) since the last rescale and g = h / P,
+// g_t = g_{t-1} + (dt_t x_t / P_t) B_t and y_t = P_t (C_t . g_t).  P is kept as its
+// log2 (cl) and folded back into g (g <- P g) at every tile start; when no lane's
+// decay over the tile passes 2^-60 (checked warp-uniformly) the tile runs the
+// unrolled fast path, otherwise the per-step path that folds on demand and restarts
+// the state after a single step decaying by more than 2^-60.
 template <int NP>
 struct ScaledState {
   float2 g[NP];
@@ -251,14 +215,18 @@ struct ScaledState {
     for (int i = 0; i < NP; ++i) g[i] = make_float2(0.f, 0.f);
     cl = 0.f;
   }
+  HY_DEV void fold() {
+    const float P = ex2_approx(cl);
+    const float2 P2 = make_float2(P, P);
+#pragma unroll
+    for (int i = 0; i < NP; ++i) g[i] = __fmul2_rn(g[i], P2);
+    cl = 0.f;
+  }
   // advance the scale by one step of log2-decay l2a; returns 1 / P_t
   HY_DEV float advance(float l2a) {
     float c = cl + l2a;
     if (c < -60.f) {  // rare: fold the scale into g
-      const float P = ex2_approx(cl);
-      const float2 P2 = make_float2(P, P);
-#pragma unroll
-      for (int i = 0; i < NP; ++i) g[i] = __fmul2_rn(g[i], P2);
+      fold();
       if (l2a < -60.f) {
 #pragma unroll
         for (int i = 0; i < NP; ++i) g[i] = make_float2(0.f, 0.f);
@@ -272,325 +240,181 @@ struct ScaledState {
   }
 };
 
-// Fast path of one full ROWS-step tile.  First folds the running scale into g for
-// every lane (g <- P g, P <- 1), then checks (warp-uniformly) that no lane's decay
-// over the tile passes 2^-60, so that the scales of all its steps can be formed
-// independently; returns false (slow, per-step guarded path) for a partial tile or
-// an extreme decay.
-template <typename TI, int N>
-HY_DEV bool fast_tile(const uint8_t* tile, int lane, int rows, const float (&A2)[2], ScaledState<N / 2> (&st)[2]) {
-  using C = PairCfg<TI, N>;
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const float P = ex2_approx(st[q].cl);
-    const float2 P2 = make_float2(P, P);
-#pragma unroll
-    for (int i = 0; i < N / 2; ++i) st[q].g[i] = __fmul2_rn(st[q].g[i], P2);
-    st[q].cl = 0.f;
-  }
-  bool ok = rows == C::ROWS;
-  if (ok) {
-    float c[2] = {0.f, 0.f};
-#pragma unroll
-    for (int r = 0; r < C::ROWS; ++r) {
-      const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-      c[0] = fmaf(A2[0], dv.x, c[0]);
-      c[1] = fmaf(A2[1], dv.y, c[1]);
-    }
-    ok = c[0] >= -60.f && c[1] >= -60.f;
-  }
-  return __all_sync(0xffffffffu, ok);
-}
+template <typename TI, int NS, int TPC>
+struct V5Cfg {
+  static constexpr int N = NS * TPC;
+  static constexpr int NWARP = 4;
+  static constexpr int CPW = 32 / TPC;        // channels per warp
+  static constexpr int CPB = NWARP * CPW;     // channels per CTA
+  static constexpr int ROWS = N <= 32 ? 16 : 8;  // steps per tile (B|C rows grow with N)
+  static constexpr int STAGES = 4;
+  static constexpr int XB = ROWS * CPB * (int)sizeof(TI);  // one x / dt / gate tile
+  static constexpr int BCB = ROWS * 2 * N * 4;              // one B|C tile
+  static constexpr int STAGE_B = 3 * XB + BCB;
+  static constexpr int YB = ROWS * CPW * (int)sizeof(TI);   // one warp's y tile
+  static constexpr int SMEM = STAGES * STAGE_B + NWARP * 2 * YB + 2 * STAGES * 8 + 16 + 128;
+};
 
-// Four steps (rows h2 .. h2+3 of a staged tile) of the scaled-state recurrence with
-// no fold needed: the four scales are formed up front (independent SFU ops), then the
-// state chain runs; with EMIT the gated outputs y = gate P (C . g) are stored.
-template <typename TI, int N, bool EMIT>
-HY_DEV void step4(const uint8_t* tile, int lane, int h2, const float (&A2)[2], ScaledState<N / 2> (&st)[2],
-                  float (&logdec)[2], TI* ybase, long long y_ld, int, bool w0, bool w1) {
-  using C = PairCfg<TI, N>;
-  float v[4][2], P[4][2], gate[4][2];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = h2 + k;
-    const float2 xv = Pair2<TI>::ld(tile + (r * C::CPW + 2 * lane) * sizeof(TI));
-    const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-    const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
-    if (EMIT) {
-      const float2 gv = Pair2<TI>::ld(tile + 2 * C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-      gate[k][0] = gv.x;
-      gate[k][1] = gv.y;
-    }
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const float l2a = A2[q] * dq[q];
-      if (!EMIT) logdec[q] += l2a;
-      st[q].cl += l2a;
-      v[k][q] = dq[q] * xq[q] * ex2_approx(-st[q].cl);
-      if (EMIT) P[k][q] = ex2_approx(st[q].cl);
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = h2 + k;
-    const float4* B4 = reinterpret_cast<const float4*>(tile + 3 * C::XB + r * 2 * N * 4);
-    float2 q2[2], y2[2];
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      q2[q] = make_float2(v[k][q], v[k][q]);
-      y2[q] = make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int j = 0; j < N / 4; ++j) {
-      const float4 bb = B4[j];
-      const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        st[q].g[2 * j] = __ffma2_rn(q2[q], b01, st[q].g[2 * j]);
-        st[q].g[2 * j + 1] = __ffma2_rn(q2[q], b23, st[q].g[2 * j + 1]);
-      }
-      if (EMIT) {
-        const float4 cv = B4[N / 4 + j];
-        const float2 c01 = make_float2(cv.x, cv.y), c23 = make_float2(cv.z, cv.w);
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          y2[q] = __ffma2_rn(c01, st[q].g[2 * j], y2[q]);
-          y2[q] = __ffma2_rn(c23, st[q].g[2 * j + 1], y2[q]);
-        }
-      }
-    }
-    if (EMIT) {
-      TI* yrow = ybase + r * y_ld;
-      const float ya = gate[k][0] * P[k][0] * (y2[0].x + y2[0].y);
-      const float yb = gate[k][1] * P[k][1] * (y2[1].x + y2[1].y);
-      if (w0 && w1) Pair2<TI>::st(yrow, ya, yb);
-      else if (w0) yrow[0] = from_f<TI>(ya);
-    }
-  }
-}
-
-template <typename TI, int N>
-__global__ void __launch_bounds__(256) scan_pair_kernel(const __grid_constant__ CUtensorMap tmX,
-                                                        const __grid_constant__ CUtensorMap tmDT,
-                                                        const __grid_constant__ CUtensorMap tmG,
-                                                        const __grid_constant__ CUtensorMap tmBC,
-                                                        const ScanParams p, unsigned* status) {
-  using C = PairCfg<TI, N>;
-  constexpr int NP = N / 2;
+template <typename TI, int NS, int TPC>
+__global__ void __launch_bounds__(128) scan_v5_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                      const __grid_constant__ CUtensorMap tmDT,
+                                                      const __grid_constant__ CUtensorMap tmG,
+                                                      const __grid_constant__ CUtensorMap tmBC,
+                                                      const __grid_constant__ CUtensorMap tmY, const ScanParams p,
+                                                      unsigned* status) {
+  using C = V5Cfg<TI, NS, TPC>;
+  constexpr int N = C::N;
+  constexpr int NP = NS / 2;
   extern __shared__ __align__(128) uint8_t smem[];
-  float* s_carry = reinterpret_cast<float*>(smem + C::AREA_B);  // [2][CPW][N]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::AREA_B + C::CARRY_B);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + C::NWT * C::STAGES);
-  float* s_hend = reinterpret_cast<float*>(smem);       // [NWT][CPW][N]  (aliases the ring)
-  float* s_logdec = s_hend + C::NWT * C::CPW * N;       // [NWT][CPW]
+  uint8_t* ybuf = smem + C::STAGES * C::STAGE_B;  // [NWARP][2][ROWS][CPW]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ybuf + C::NWARP * 2 * C::YB);
+  uint64_t* empty = full + C::STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::STAGES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chw = lane / TPC, slice = lane % TPC;  // channel within the warp, state slice
+  const int cl_cta = warp * C::CPW + chw;          // channel within the CTA
+  const int c = blockIdx.x * C::CPB + cl_cta;
   const int b = blockIdx.y;
-  const int c0 = blockIdx.x * C::CPW + 2 * lane;  // this lane's first channel
-  uint8_t* ring = smem + warp * C::WARP_B;
-  uint64_t* my_full = full + warp * C::STAGES;
+  const int n0 = slice * NS;
+  const int n_tiles = (p.T + C::ROWS - 1) / C::ROWS;
 
-  if (threadIdx.x == 0) *abort_flag = 0;
-  if (lane == 0)
-    for (int s = 0; s < C::STAGES; ++s) mbar_init(&my_full[s], 1);
-  for (int i = threadIdx.x; i < C::CPW * N; i += blockDim.x) s_carry[i] = 0.f;  // h = 0 before the first row
-  fence_mbar_init();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::NWARP);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
   __syncthreads();
 
-  float A2[2];
-#pragma unroll
-  for (int q = 0; q < 2; ++q) A2[q] = c0 + q < p.Di ? -expf(p.a_log[c0 + q]) * 1.4426950408889634f : 0.f;
-  const bool w0 = c0 < p.Di, w1 = c0 + 1 < p.Di;
-  TI* Y = static_cast<TI*>(p.y);
-
-  // Ring bookkeeping across segments and passes: the i-th tile issued by this warp
-  // goes to slot i % STAGES and completes phase (i / STAGES) & 1 of that slot's
-  // mbarrier; tiles are consumed in issue order.
-  uint32_t issued = 0, consumed = 0;
-  auto issue = [&](int grow, bool with_gate) {
-    if (lane == 0) {
-      const int slot = issued % C::STAGES;
-      uint8_t* st = ring + slot * C::STAGE_B;
-      uint64_t* bar = &my_full[slot];
-      mbar_arrive_expect_tx(bar, (with_gate ? 3 : 2) * C::XB + C::BCB);
-      const int col = blockIdx.x * C::CPW;
-      tma_load_2d(st, &tmX, bar, col, grow);
-      tma_load_2d(st + C::XB, &tmDT, bar, col, grow);
-      if (with_gate) tma_load_2d(st + 2 * C::XB, &tmG, bar, col, grow);
-      tma_load_2d(st + 3 * C::XB, &tmBC, bar, 0, grow);
-    }
+  const float A2 = c < p.Di ? -expf(p.a_log[c]) * 1.4426950408889634f : 0.f;
+  const bool producer = threadIdx.x == 0;
+  uint32_t issued = 0;
+  auto issue = [&](int k) {  // tile k -> slot k % STAGES (tiles are issued in order)
+    const int slot = k % C::STAGES;
+    if (k >= C::STAGES && !mbar_wait(&empty[slot], ((k / C::STAGES) & 1) ^ 1u, status, abort_flag)) return false;
+    uint8_t* st = smem + slot * C::STAGE_B;
+    mbar_arrive_expect_tx(&full[slot], C::STAGE_B);
+    const int col = blockIdx.x * C::CPB, t = k * C::ROWS;
+    tma_load_3d(st, &tmX, &full[slot], col, t, b);
+    tma_load_3d(st + C::XB, &tmDT, &full[slot], col, t, b);
+    tma_load_3d(st + 2 * C::XB, &tmG, &full[slot], col, t, b);
+    tma_load_3d(st + 3 * C::XB, &tmBC, &full[slot], 0, t, b);
     ++issued;
+    return true;
   };
-  auto wait_tile = [&]() -> bool {
-    return __all_sync(0xffffffffu,
-                      mbar_wait(&my_full[consumed % C::STAGES], (consumed / C::STAGES) & 1u, status, abort_flag));
-  };
-  auto drain = [&]() {  // after an abort: let this warp's copies in flight land
-    int never = 0;
-    if (lane == 0)
-      for (uint32_t i = consumed; i < issued; ++i)
-        mbar_wait(&my_full[i % C::STAGES], (i / C::STAGES) & 1u, nullptr, &never, 100000000ull);
-    __syncwarp();
-  };
-
   bool ok = true;
-  ScaledState<NP> st[2];
-  int seg_id = 0;
-  for (int seg0 = 0; seg0 < p.T; seg0 += C::SEG, ++seg_id) {
-    const int t0 = min(p.T, seg0 + warp * C::SUB), t1 = min(p.T, min(seg0 + C::SEG, t0 + C::SUB));
-    const int n_tiles = (t1 - t0 + C::ROWS - 1) / C::ROWS;
-    const int grow0 = b * p.T + t0;
-    // ---------------- pass 1: local scan from h = 0 -> end state and total log2-decay
-    float logdec[2] = {0.f, 0.f};
+  if (producer)
+    for (int k = 0; ok && k < C::STAGES - 1 && k < n_tiles; ++k) ok = issue(k);
+
+  ScaledState<NP> st;
+  st.zero();
+  uint8_t* my_y = ybuf + warp * 2 * C::YB;
+  const size_t es = sizeof(TI);
+  int k = 0;
+  for (; k < n_tiles; ++k) {
+    if (producer && ok && k + C::STAGES - 1 < n_tiles) ok = issue(k + C::STAGES - 1);
+    const int slot = k % C::STAGES;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], (k / C::STAGES) & 1, status, abort_flag))) {
+      ok = false;
+      break;
+    }
+    const uint8_t* tile = smem + slot * C::STAGE_B;
+    const uint8_t* tx = tile + cl_cta * es;
+    const uint8_t* td = tile + C::XB + cl_cta * es;
+    const uint8_t* tg = tile + 2 * C::XB + cl_cta * es;
+    const float* tbc = reinterpret_cast<const float*>(tile + 3 * C::XB) + n0;
+    const int rows = min(C::ROWS, p.T - k * C::ROWS);
+    // y tile of this warp (double-buffered; the TMA store of tile k-2 must have read it)
+    TI* yt = reinterpret_cast<TI*>(my_y + (k & 1) * C::YB);
+    if (lane == 0) bulk_wait_read1();
+    __syncwarp();
+
+    st.fold();
+    bool fast = rows == C::ROWS;
+    if (fast) {
+      float cum = 0.f;
 #pragma unroll
-    for (int q = 0; q < 2; ++q) st[q].zero();
-    for (int k = 0; ok && k < C::STAGES - 1 && k < n_tiles; ++k) issue(grow0 + k * C::ROWS, false);
-    for (int k = 0; ok && k < n_tiles; ++k) {
-      __syncwarp();
-      if (k + C::STAGES - 1 < n_tiles) issue(grow0 + (k + C::STAGES - 1) * C::ROWS, false);
-      const uint8_t* tile = ring + (consumed % C::STAGES) * C::STAGE_B;
-      if (!wait_tile()) {
-        ok = false;
-        break;
-      }
-      ++consumed;
-      const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
-      if (fast_tile<TI, N>(tile, lane, rows, A2, st)) {
+      for (int r = 0; r < C::ROWS; ++r) cum = fmaf(A2, to_f<TI>(*reinterpret_cast<const TI*>(td + r * C::CPB * es)), cum);
+      fast = cum >= -60.f;
+    }
+    if (__all_sync(0xffffffffu, fast)) {
 #pragma unroll
-        for (int h2 = 0; h2 < C::ROWS; h2 += 4) step4<TI, N, false>(tile, lane, h2, A2, st, logdec, nullptr, 0, 0, false, false);
-      } else {
-        for (int r = 0; r < rows; ++r) {
-          const float2 xv = Pair2<TI>::ld(tile + (r * C::CPW + 2 * lane) * sizeof(TI));
-          const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-          const float4* B4 = reinterpret_cast<const float4*>(tile + 3 * C::XB + r * 2 * N * 4);
-          const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
-          float2 q2[2];
+      for (int r0 = 0; r0 < C::ROWS; r0 += 4) {  // four steps: scales first (independent SFU ops), then the chain
+        float v[4], P[4], gt[4];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const float l2a = A2[q] * dq[q];
-            logdec[q] += l2a;
-            const float v = dq[q] * xq[q] * st[q].advance(l2a);
-            q2[q] = make_float2(v, v);
+        for (int q = 0; q < 4; ++q) {
+          const int r = r0 + q;
+          const float d = to_f<TI>(*reinterpret_cast<const TI*>(td + r * C::CPB * es));
+          const float xv = to_f<TI>(*reinterpret_cast<const TI*>(tx + r * C::CPB * es));
+          gt[q] = to_f<TI>(*reinterpret_cast<const TI*>(tg + r * C::CPB * es));
+          st.cl = fmaf(A2, d, st.cl);
+          v[q] = d * xv * ex2_approx(-st.cl);
+          P[q] = ex2_approx(st.cl);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int r = r0 + q;
+          const float4* B4 = reinterpret_cast<const float4*>(tbc + r * 2 * N);
+          const float4* C4 = reinterpret_cast<const float4*>(tbc + r * 2 * N + N);
+          const float2 v2 = make_float2(v[q], v[q]);
+          float2 ya = make_float2(0.f, 0.f), yb = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < NS / 4; ++j) {
+            const float4 bb = B4[j], cv = C4[j];
+            st.g[2 * j] = __ffma2_rn(v2, make_float2(bb.x, bb.y), st.g[2 * j]);
+            st.g[2 * j + 1] = __ffma2_rn(v2, make_float2(bb.z, bb.w), st.g[2 * j + 1]);
+            ya = __ffma2_rn(make_float2(cv.x, cv.y), st.g[2 * j], ya);
+            yb = __ffma2_rn(make_float2(cv.z, cv.w), st.g[2 * j + 1], yb);
           }
+          float y = (ya.x + ya.y) + (yb.x + yb.y);
 #pragma unroll
-          for (int j = 0; j < N / 4; ++j) {
-            const float4 bb = B4[j];
-            const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              st[q].g[2 * j] = __ffma2_rn(q2[q], b01, st[q].g[2 * j]);
-              st[q].g[2 * j + 1] = __ffma2_rn(q2[q], b23, st[q].g[2 * j + 1]);
-            }
-          }
+          for (int off = 1; off < TPC; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
+          if (slice == 0) yt[r * C::CPW + chw] = from_f<TI>(gt[q] * P[q] * y);
         }
       }
-    }
-    if (!ok) drain();
-    __syncthreads();  // the ring area becomes the combine area
-    // local end state h_end = P g
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const float P = ex2_approx(st[q].cl);
-      const float2 P2 = make_float2(P, P);
-      float2* dst = reinterpret_cast<float2*>(s_hend + (warp * C::CPW + 2 * lane + q) * N);
-#pragma unroll
-      for (int i = 0; i < NP; ++i) dst[i] = __fmul2_rn(st[q].g[i], P2);
-      s_logdec[warp * C::CPW + 2 * lane + q] = logdec[q];
-    }
-    __syncthreads();
-    // ---------------- combine: state entering this warp's steps (chained from the
-    // segment's carry-in), and the last warp also forms the next segment's carry-in
-    const float* carry_in = s_carry + (seg_id & 1) * C::CPW * N;
-    float* carry_out = s_carry + ((seg_id + 1) & 1) * C::CPW * N;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int ch = 2 * lane + q;
-      const float2* cin = reinterpret_cast<const float2*>(carry_in + ch * N);
-#pragma unroll
-      for (int i = 0; i < NP; ++i) st[q].g[i] = cin[i];
-      st[q].cl = 0.f;
-      const int kmax = (warp == C::NWT - 1) ? C::NWT : warp;
-      for (int k = 0; k < kmax; ++k) {
-        if (k == warp) {  // last warp: its own entry state is complete; store it, then go on
-          float2* tmp = reinterpret_cast<float2*>(carry_out + ch * N);
-#pragma unroll
-          for (int i = 0; i < NP; ++i) tmp[i] = st[q].g[i];
-        }
-        const float dec = ex2_approx(s_logdec[k * C::CPW + ch]);
-        const float2 dec2 = make_float2(dec, dec);
-        const float2* hk = reinterpret_cast<const float2*>(s_hend + (k * C::CPW + ch) * N);
-#pragma unroll
-        for (int i = 0; i < NP; ++i) st[q].g[i] = __ffma2_rn(dec2, st[q].g[i], hk[i]);
-      }
-      if (warp == C::NWT - 1) {  // g = carry-out (end of segment); restore own entry state
-        float2* co = reinterpret_cast<float2*>(carry_out + ch * N);
-#pragma unroll
-        for (int i = 0; i < NP; ++i) {
-          const float2 own = co[i];
-          co[i] = st[q].g[i];
-          st[q].g[i] = own;
-        }
-      }
-    }
-    fence_proxy_async_smem();  // generic accesses to the ring area before the copies below
-    __syncthreads();
-    // ---------------- pass 2: rescan from the carried state, emit y = gate (C . h)
-    for (int k = 0; ok && k < C::STAGES - 1 && k < n_tiles; ++k) issue(grow0 + k * C::ROWS, true);
-    for (int k = 0; ok && k < n_tiles; ++k) {
-      __syncwarp();
-      if (k + C::STAGES - 1 < n_tiles) issue(grow0 + (k + C::STAGES - 1) * C::ROWS, true);
-      const uint8_t* tile = ring + (consumed % C::STAGES) * C::STAGE_B;
-      if (!wait_tile()) {
-        ok = false;
-        break;
-      }
-      ++consumed;
-      const int rows = min(C::ROWS, t1 - t0 - k * C::ROWS);
-      if (fast_tile<TI, N>(tile, lane, rows, A2, st)) {
-        float ld_unused[2] = {0.f, 0.f};
-        TI* ybase = Y + (static_cast<long long>(grow0) + k * C::ROWS) * p.y_ld + c0;
-#pragma unroll
-        for (int h2 = 0; h2 < C::ROWS; h2 += 4)
-          step4<TI, N, true>(tile, lane, h2, A2, st, ld_unused, ybase, p.y_ld, 0, w0, w1);
-        continue;
-      }
+    } else {
       for (int r = 0; r < rows; ++r) {
-        const float2 xv = Pair2<TI>::ld(tile + (r * C::CPW + 2 * lane) * sizeof(TI));
-        const float2 dv = Pair2<TI>::ld(tile + C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-        const float2 gv = Pair2<TI>::ld(tile + 2 * C::XB + (r * C::CPW + 2 * lane) * sizeof(TI));
-        const float4* B4 = reinterpret_cast<const float4*>(tile + 3 * C::XB + r * 2 * N * 4);
-        const float4* C4 = B4 + N / 4;
-        const float dq[2] = {dv.x, dv.y}, xq[2] = {xv.x, xv.y};
-        float2 q2[2], y2[2];
+        const float d = to_f<TI>(*reinterpret_cast<const TI*>(td + r * C::CPB * es));
+        const float xv = to_f<TI>(*reinterpret_cast<const TI*>(tx + r * C::CPB * es));
+        const float gv = to_f<TI>(*reinterpret_cast<const TI*>(tg + r * C::CPB * es));
+        const float v = d * xv * st.advance(A2 * d);
+        const float2 v2 = make_float2(v, v);
+        const float4* B4 = reinterpret_cast<const float4*>(tbc + r * 2 * N);
+        const float4* C4 = reinterpret_cast<const float4*>(tbc + r * 2 * N + N);
+        float2 ya = make_float2(0.f, 0.f), yb = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const float v = dq[q] * xq[q] * st[q].advance(A2[q] * dq[q]);
-          q2[q] = make_float2(v, v);
-          y2[q] = make_float2(0.f, 0.f);
-        }
-#pragma unroll
-        for (int j = 0; j < N / 4; ++j) {
+        for (int j = 0; j < NS / 4; ++j) {
           const float4 bb = B4[j], cv = C4[j];
-          const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
-          const float2 c01 = make_float2(cv.x, cv.y), c23 = make_float2(cv.z, cv.w);
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            st[q].g[2 * j] = __ffma2_rn(q2[q], b01, st[q].g[2 * j]);
-            st[q].g[2 * j + 1] = __ffma2_rn(q2[q], b23, st[q].g[2 * j + 1]);
-            y2[q] = __ffma2_rn(c01, st[q].g[2 * j], y2[q]);
-            y2[q] = __ffma2_rn(c23, st[q].g[2 * j + 1], y2[q]);
-          }
+          st.g[2 * j] = __ffma2_rn(v2, make_float2(bb.x, bb.y), st.g[2 * j]);
+          st.g[2 * j + 1] = __ffma2_rn(v2, make_float2(bb.z, bb.w), st.g[2 * j + 1]);
+          ya = __ffma2_rn(make_float2(cv.x, cv.y), st.g[2 * j], ya);
+          yb = __ffma2_rn(make_float2(cv.z, cv.w), st.g[2 * j + 1], yb);
         }
-        const long long row = static_cast<long long>(grow0) + k * C::ROWS + r;
-        TI* yrow = Y + row * p.y_ld + c0;
-        const float ya = gv.x * ex2_approx(st[0].cl) * (y2[0].x + y2[0].y);
-        const float yb = gv.y * ex2_approx(st[1].cl) * (y2[1].x + y2[1].y);
-        if (w0 && w1) Pair2<TI>::st(yrow, ya, yb);
-        else if (w0) yrow[0] = from_f<TI>(ya);
+        float y = (ya.x + ya.y) + (yb.x + yb.y);
+#pragma unroll
+        for (int off = 1; off < TPC; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
+        if (slice == 0) yt[r * C::CPW + chw] = from_f<TI>(gv * ex2_approx(st.cl) * y);
       }
     }
-    if (!ok) drain();
-    __syncthreads();  // carry-out visible; the ring area is reused by the next segment's pass 1
+    // release the input tile, then store this warp's y tile
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    const int ycol = blockIdx.x * C::CPB + warp * C::CPW;
+    if (lane == 0 && ycol < p.Di) {  // a warp whose channels all lie past Di stores nothing
+      tma_store_3d(&tmY, yt, ycol, k * C::ROWS, b);
+      bulk_commit();
+    }
+  }
+  if (lane == 0) bulk_wait_all();
+  if (!ok && producer) {  // let the copies this warp has not consumed land before the CTA exits
+    int never = 0;
+    for (int t = k; t < static_cast<int>(issued); ++t)
+      mbar_wait(&full[t % C::STAGES], (t / C::STAGES) & 1u, nullptr, &never, 100000000ull);
   }
 }
 
@@ -623,28 +447,42 @@ bool map2d(CUtensorMap* m, const void* base, bool f32, long long rows, long long
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename TI, int N>
-cudaError_t launch_pair(const ScanDesc& s, cudaStream_t st) {
-  using C = PairCfg<TI, N>;
+// 3-D map over [batch][T][cols] (row stride ld elements), box = bc x br x 1, no swizzle.
+bool map3d(CUtensorMap* m, const void* base, bool f32, int batch, int T, long long cols, long long ld, int bc,
+           int br) {
+  EncodeTiledFn fn = scan_encode_fn();
+  if (!fn) return false;
+  const int es = f32 ? 4 : 2;
+  cuuint64_t gd[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(batch)};
+  cuuint64_t gs[2] = {static_cast<cuuint64_t>(ld) * es, static_cast<cuuint64_t>(ld) * es * T};
+  cuuint32_t bx[3] = {static_cast<cuuint32_t>(bc), static_cast<cuuint32_t>(br), 1}, el[3] = {1, 1, 1};
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+            gd, gs, bx, el, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename TI, int NS, int TPC>
+cudaError_t launch_v5(const ScanDesc& s, cudaStream_t st) {
+  using C = V5Cfg<TI, NS, TPC>;
   const bool f32 = sizeof(TI) == 4;
-  const long long rows = static_cast<long long>(s.batch) * s.T;
-  CUtensorMap tx, td, tg, tb;
-  if (!map2d(&tx, s.x, f32, rows, s.d_inner, s.d_inner, C::CPW, C::ROWS) ||
-      !map2d(&td, s.dt, f32, rows, s.d_inner, s.d_inner, C::CPW, C::ROWS) ||
-      !map2d(&tg, s.gate, f32, rows, s.d_inner, s.d_inner, C::CPW, C::ROWS) ||
-      !map2d(&tb, s.bc, true, rows, 2 * N, 2 * N, 2 * N, C::ROWS))
+  CUtensorMap tx, td, tg, tb, ty;
+  if (!map3d(&tx, s.x, f32, s.batch, s.T, s.d_inner, s.d_inner, C::CPB, C::ROWS) ||
+      !map3d(&td, s.dt, f32, s.batch, s.T, s.d_inner, s.d_inner, C::CPB, C::ROWS) ||
+      !map3d(&tg, s.gate, f32, s.batch, s.T, s.d_inner, s.d_inner, C::CPB, C::ROWS) ||
+      !map3d(&tb, s.bc, true, s.batch, s.T, 2 * C::N, 2 * C::N, 2 * C::N, C::ROWS) ||
+      !map3d(&ty, s.y, f32, s.batch, s.T, s.d_inner, s.y_ld, C::CPW, C::ROWS))
     return cudaErrorInvalidValue;
   static int attr_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 31 && !(attr_mask & (1 << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(scan_pair_kernel<TI, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(scan_v5_kernel<TI, NS, TPC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_mask |= 1 << dev;
   }
   ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
-  dim3 grid((s.d_inner + C::CPW - 1) / C::CPW, s.batch);
-  scan_pair_kernel<TI, N><<<grid, 32 * C::NWT, C::SMEM, st>>>(tx, td, tg, tb, p, s.status);
+  dim3 grid((s.d_inner + C::CPB - 1) / C::CPB, s.batch);
+  scan_v5_kernel<TI, NS, TPC><<<grid, 32 * C::NWARP, C::SMEM, st>>>(tx, td, tg, tb, ty, p, s.status);
   return cudaGetLastError();
 }
 
@@ -659,15 +497,24 @@ cudaError_t launch_one(const ScanDesc& s, cudaStream_t st) {
 
 template <typename TI>
 cudaError_t launch_t(const ScanDesc& s, cudaStream_t st) {
-  // The TMA-staged pair kernel needs 16-byte aligned bases and row strides for x, dt,
-  // gate, B|C, and 2-channel aligned output stores; otherwise the per-channel kernel runs.
+  // The TMA-staged single-pass kernel needs 16-byte aligned bases and row strides for
+  // x, dt, gate, B|C and y; otherwise the per-channel kernel runs.
   auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
-  const bool pair_ok = (s.d_inner * static_cast<int>(sizeof(TI))) % 16 == 0 && a16(s.x) && a16(s.dt) &&
-                       a16(s.gate) && a16(s.bc) && (s.y_ld % 2) == 0 &&
-                       (reinterpret_cast<uintptr_t>(s.y) % (2 * sizeof(TI))) == 0;
+  const long long es = static_cast<long long>(sizeof(TI));
+  const bool v5_ok = (s.d_inner * es) % 16 == 0 && (s.y_ld * es) % 16 == 0 && a16(s.x) && a16(s.dt) &&
+                     a16(s.gate) && a16(s.bc) && a16(s.y);
+  if (v5_ok) {
+    switch (s.d_state) {
+      case 16: return launch_v5<TI, 8, 2>(s, st);
+      case 32: return launch_v5<TI, 16, 2>(s, st);
+      case 64: return launch_v5<TI, 16, 4>(s, st);
+      case 128: return launch_v5<TI, 32, 4>(s, st);
+      default: break;  // N = 256: a B|C row exceeds one TMA box; per-channel kernel below
+    }
+  }
   switch (s.d_state) {
-    case 16: return pair_ok ? launch_pair<TI, 16>(s, st) : launch_one<TI, 16, 1, 16>(s, st);
-    case 32: return pair_ok ? launch_pair<TI, 32>(s, st) : launch_one<TI, 32, 1, 8>(s, st);
+    case 16: return launch_one<TI, 16, 1, 16>(s, st);
+    case 32: return launch_one<TI, 32, 1, 8>(s, st);
     case 64: return launch_one<TI, 32, 2, 8>(s, st);
     case 128: return launch_one<TI, 32, 4, 8>(s, st);
     case 256: return launch_one<TI, 32, 8, 8>(s, st);
