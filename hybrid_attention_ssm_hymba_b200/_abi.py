@@ -23,8 +23,11 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhymba.so
 ENTRY_POINTS = (
     "hymba_status_string", "hymba_workspace_size", "hymba_stack_workspace_size", "hymba_layer_fwd",
     "hymba_stack_fwd", "hymba_workspace_status", "hymba_layer_fwd_events", "hymba_gemm", "hymba_selective_scan",
-    "hymba_attention", "hymba_branch_norm", "hymba_rmsnorm",
+    "hymba_attention", "hymba_branch_norm", "hymba_rmsnorm", "hymba_layer_fwd_noalloc",
 )
+
+# size of the library-owned scratch block behind hymba_layer_fwd_noalloc (HYMBA_NOALLOC_SCRATCH_BYTES)
+HYMBA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class HymbaError(RuntimeError):
@@ -55,6 +58,8 @@ _SIGS = {
                              _VP, _VP, _VP, _VP, _SZ, _VP]),
     "hymba_layer_fwd_events": (_I, [_VP, _VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t),
                                     _VP, _VP, _VP, _VP, _SZ, _VP, ctypes.POINTER(_VP)]),
+    "hymba_layer_fwd_noalloc": (_I, [_VP, _VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t),
+                                     _VP, _VP, _VP, _VP]),
     "hymba_stack_fwd": (_I, [_VP, _VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t),
                              _I, _VP, _VP, _SZ, _VP]),
     "hymba_workspace_status": (_I, [_VP, _VP]),
@@ -151,6 +156,15 @@ def hymba_layer_fwd(x, meta, weights: hymba_weights_t, cfg: hymba_cfg_t, kv_in, 
     return load().hymba_layer_fwd(_ptr(x), _ptr(meta), ctypes.byref(weights), ctypes.byref(cfg),
                                   _ptr(kv_in), _ptr(kv_out), _ptr(out), _ptr(workspace), wsb,
                                   _stream(stream))
+
+
+def hymba_layer_fwd_noalloc(x, meta, weights: hymba_weights_t, cfg: hymba_cfg_t, kv_in, kv_out, out,
+                            stream=None) -> int:
+    """hymba_layer_fwd with the intermediates in the library's own static scratch block
+    (no workspace argument; configs needing more than HYMBA_NOALLOC_SCRATCH_BYTES are
+    rejected with HYMBA_ERR_WORKSPACE)."""
+    return load().hymba_layer_fwd_noalloc(_ptr(x), _ptr(meta), ctypes.byref(weights), ctypes.byref(cfg),
+                                          _ptr(kv_in), _ptr(kv_out), _ptr(out), _stream(stream))
 
 
 STAGES = ("in_proj", "x_proj", "dt_proj", "attention", "scan", "branch_norm", "out_proj")

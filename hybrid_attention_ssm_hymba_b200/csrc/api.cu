@@ -11,6 +11,7 @@
 //   6 norm      Z <- [beta1 rms(Z_attn) || beta2 rms(Z_ssm)]   (in place)
 //   7 out_proj  Z W_out^T -> out   (+ residual inside a stack)
 #include <cstring>
+#include <mutex>
 
 #include "hy_kernels.h"
 #include "hymba.h"
@@ -264,6 +265,37 @@ __global__ void prepend_kernel(const uint4* __restrict__ x, const uint4* __restr
   }
 }
 
+// ---- library-owned scratch for hymba_layer_fwd_noalloc
+//
+// One fixed block of device memory per GPU, reserved when the module loads on that
+// device and held until the process exits.  Host code must not use the symbol's name
+// as a pointer (on the host it names a stand-in object, not device memory): the device
+// address comes from cudaGetSymbolAddress, looked up once per device with that device
+// current and cached.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[HYMBA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxNoallocDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxNoallocDevices] = {};
+
+// Device address of the scratch block on the current device (set up on first use).
+cudaError_t noalloc_scratch(uint8_t** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxNoallocDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    if (!ptr) return cudaErrorInvalidSymbol;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = static_cast<uint8_t*>(g_noalloc_addr[dev]);
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -329,6 +361,27 @@ hymba_status_t hymba_layer_fwd_events(const void* x, const void* meta, const hym
   if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;
   return run_layer(x, cfg->n_meta > 0 ? meta : nullptr, *w, *cfg, kv_in, kv_out, out, false,
                    static_cast<uint8_t*>(workspace) + 256, status, st, events);
+}
+
+hymba_status_t hymba_layer_fwd_noalloc(const void* x, const void* meta, const hymba_weights_t* w,
+                                       const hymba_cfg_t* cfg, const void* kv_in, void* kv_out, void* out,
+                                       void* stream) {
+  hymba_status_t s = validate_cfg(cfg);
+  if (s != HYMBA_OK) return s;
+  if (!x || !out || !weights_ok(w, *cfg, false)) return HYMBA_ERR_INVALID_ARG;
+  if (cfg->kv_mode == HYMBA_KV_CONSUME && !kv_in) return HYMBA_ERR_INVALID_ARG;
+  if (cfg->kv_mode == HYMBA_KV_PRODUCE && !kv_out) return HYMBA_ERR_INVALID_ARG;
+  // the same layout hymba_layer_fwd uses: status word, then the layer's intermediates
+  if (hymba_workspace_size(cfg) > HYMBA_NOALLOC_SCRATCH_BYTES) return HYMBA_ERR_WORKSPACE;
+  uint8_t* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return HYMBA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* status = reinterpret_cast<unsigned*>(scratch);
+  // the block keeps the previous call's contents: the status word must start at zero
+  // (every intermediate is written before it is read)
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  return run_layer(x, cfg->n_meta > 0 ? meta : nullptr, *w, *cfg, kv_in, kv_out, out, false, scratch + 256, status,
+                   st);
 }
 
 hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weights_t* w, const hymba_cfg_t* cfgs,

@@ -152,6 +152,37 @@ HYMBA_API hymba_status_t hymba_layer_fwd_events(const void* x, const void* meta,
                                void* out, void* workspace, size_t ws_bytes, void* stream,
                                void* const* events);
 
+/*
+ * hymba_layer_fwd without a caller-provided workspace.  The paper has no
+ * counterpart to this entry point: it exists for callers that cannot allocate
+ * device memory when they run the layer -- code inside a host framework that owns
+ * every device allocation (a plugin or custom-op execute step that must not call
+ * cudaMalloc), or latency-critical paths where cudaMalloc/cudaFree would
+ * synchronise the device.  Such a caller passes only inputs and outputs.
+ *
+ * Scratch: the layer's intermediates live in one block of HYMBA_NOALLOC_SCRATCH_BYTES
+ * bytes that the library reserves statically on every GPU that loads it; the
+ * block is held until the process exits.  Nothing is allocated by this call (no
+ * cudaMalloc, cudaFree or allocating library routine).
+ *   - A cfg whose hymba_workspace_size(cfg) exceeds HYMBA_NOALLOC_SCRATCH_BYTES
+ *     returns HYMBA_ERR_WORKSPACE before anything runs; use hymba_layer_fwd there.
+ *   - The first call on a device looks up the block's device address (once per
+ *     device, with that device current).  Make that first call before any stream
+ *     capture on the device.
+ *   - Every call on a device shares the block, which keeps the last call's
+ *     contents; the call clears its status word and overwrites every intermediate
+ *     before reading it.  Calls whose execution overlaps on the GPU (different
+ *     streams, or several host threads) race on the block: serialise them.
+ *   - A kernel wait that runs out is recorded in the block's status word, which
+ *     the caller cannot read; callers that need HYMBA_ERR_TIMEOUT reports use
+ *     hymba_layer_fwd with their own workspace.
+ * Arguments, layouts, validation and results are those of hymba_layer_fwd.
+ */
+#define HYMBA_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB per GPU */
+HYMBA_API hymba_status_t hymba_layer_fwd_noalloc(const void* x, const void* meta, const hymba_weights_t* w,
+                               const hymba_cfg_t* cfg, const void* kv_in, void* kv_out,
+                               void* out, void* stream);
+
 /* Synchronises `stream`, reads and clears the status word at the start of
  * `workspace`: HYMBA_OK, or HYMBA_ERR_TIMEOUT if a kernel's bounded wait ran out. */
 HYMBA_API hymba_status_t hymba_workspace_status(void* workspace, void* stream);

@@ -128,3 +128,12 @@ def test_no_cpu_fallback_when_library_missing(tmp_path, monkeypatch):
     monkeypatch.setattr(_abi, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         _abi.load(str(tmp_path / "libhymba.so"))
+
+
+def test_noalloc_rejects_oversized_config_before_touching_a_gpu():
+    """The allocation-free layer entry point validates its size limit on the host."""
+    cfg = _cfg()   # the full 350M-shaped layer needs ~300 MB of intermediates
+    assert H.hymba_workspace_size(cfg) > H.HYMBA_NOALLOC_SCRATCH_BYTES
+    w = H.make_weights({k: 16 for k in ("w_in", "w_x", "w_dt", "w_out", "a_log", "b_dt", "beta1", "beta2")})
+    assert H.hymba_layer_fwd_noalloc(16, 16, w, cfg, None, None, 16, stream=0) == H.HYMBA_ERR_WORKSPACE
+    assert H.hymba_layer_fwd_noalloc(16, 16, w, _cfg(batch=0), None, None, 16, stream=0) == H.HYMBA_ERR_INVALID_ARG

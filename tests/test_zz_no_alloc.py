@@ -1,0 +1,67 @@
+"""hymba_layer_fwd_noalloc: the layer forward for callers that cannot allocate device
+memory (for example a plugin whose execute step runs inside a framework that owns
+every allocation, or a latency-critical path where cudaMalloc would synchronise the
+device).  It keeps the intermediates in the library's own static scratch block
+instead of a caller workspace.
+
+Checked here through the C ABI: two calls in a row, each on fresh inputs, give the
+same output as hymba_layer_fwd with a caller workspace, within the tolerances of the
+other parity tests; the second call must not see anything the first one left in the
+shared block.  This file is collected last on purpose."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import hybrid_attention_ssm_hymba_b200 as H
+from hybrid_attention_ssm_hymba_b200 import host, synth
+from gpu_util import assert_close, dev, requires_cuda, status_ok, to_np
+
+pytestmark = [pytest.mark.gpu, requires_cuda]
+
+
+def _with_workspace(x, meta, w, cfg, out_shape, dtype):
+    out = host.empty(out_shape, dtype)
+    ws = host.workspace(H.hymba_workspace_size(cfg))
+    H.check(H.hymba_layer_fwd(x, meta, w, cfg, None, None, out, ws), "hymba_layer_fwd")
+    status_ok(ws)
+    return to_np(out)
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_fp32", {}),
+    ("hymba350m_layer", dict(batch=1, seq_len=224)),
+    ("hymba1p5b_kvpair", dict(n_layers=1, batch=1, seq_len=120, window=48, d_model=512, n_q_heads=4,
+                              n_kv_heads=2, d_inner=512, dt_rank=32)),
+])
+def test_noalloc_matches_workspace_entry_point_two_calls(name, kw):
+    wl = synth.workload(name, **kw)
+    s = dataclasses.replace(wl.first, kv_mode=H.HYMBA_KV_OWN)
+    cfg = H.make_cfg(s)
+    assert 0 < H.hymba_workspace_size(cfg) <= H.HYMBA_NOALLOC_SCRATCH_BYTES
+    dps = host.params_to_device(synth.layer_params(wl, 0), s.dtype)   # kept alive for the calls
+    w = H.make_weights(dps)
+    x1, meta = synth.layer_inputs(wl)
+    x2 = synth.normal(wl.seed, 1, "x", x1.shape, 1.0, s.dtype)   # another stream of the same recipe
+    tm = dev(meta, s.dtype)
+    shape = (s.batch, s.T, s.d_model)
+    outs = []
+    for x in (x1, x2):   # two calls in a row on the shared block, different inputs
+        out = host.empty(shape, s.dtype)
+        out.fill_(float("nan"))
+        H.check(H.hymba_layer_fwd_noalloc(dev(x, s.dtype), tm, w, cfg, None, None, out), "noalloc")
+        outs.append(to_np(out))
+    for i, x in enumerate((x1, x2)):
+        ref = _with_workspace(dev(x, s.dtype), tm, w, cfg, shape, s.dtype)
+        assert_close(outs[i], ref, s.dtype, f"{name} noalloc call {i + 1}")
+    assert not np.allclose(outs[0], outs[1]), "the two calls must see their own inputs"
+
+
+def test_noalloc_rejects_configs_beyond_the_scratch_block():
+    wl = synth.workload("hymba350m_layer")   # B=8, L=2048: ~300 MB of intermediates
+    cfg = H.make_cfg(wl.first)
+    assert H.hymba_workspace_size(cfg) > H.HYMBA_NOALLOC_SCRATCH_BYTES
+    dps = host.params_to_device(synth.layer_params(synth.workload("tiny_fp32"), 0), "f32")
+    w = H.make_weights(dps)
+    out = host.empty((1, 1, 8), "bf16")
+    assert H.hymba_layer_fwd_noalloc(out, out, w, cfg, None, None, out) == H.HYMBA_ERR_WORKSPACE
