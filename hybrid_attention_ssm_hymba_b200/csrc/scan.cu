@@ -20,6 +20,17 @@
 #include "hy_common.cuh"
 #include "hy_kernels.h"
 
+// Launch shapes of the main kernel (lanes per channel, channels per lane) for the two
+// state sizes of the workloads.
+#ifndef HY_SCAN16_TPC
+#define HY_SCAN16_TPC 1
+#define HY_SCAN16_CPL 1
+#endif
+#ifndef HY_SCAN128_TPC
+#define HY_SCAN128_TPC 4
+#define HY_SCAN128_CPL 2
+#endif
+
 namespace hy {
 namespace {
 
@@ -189,232 +200,338 @@ __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
 }
 
 // ---------------------------------------------------------------------------------
-// Single-pass TMA-staged scan (the main path).
+// Single-pass scan with warp-private pipelines (the main path).
 //
-// Each channel is scanned once, sequentially over all T steps (the critical path is
-// T short steps; parallelism comes from channels x state slices).  A channel's N
-// state components are split over TPC lanes (NS each, packed fp32x2 updates) and
-// y = C . h is reduced with shuffles.  A CTA of NWARP warps (CPB channels) shares one
-// STAGES-deep ring of ROWS-step TMA tiles -- x, dt, gate for its channels and the
-// full B|C rows -- filled by one thread and released by the warps through an
-// mbarrier; y goes out through a per-warp smem tile and a TMA store.  Tensor maps
-// are 3-D ([batch][T][cols]), so no tile reads or writes across a sequence end.
+// Each channel is scanned once, sequentially over all T steps; parallelism comes from
+// channels x state slices.  A lane owns CPL adjacent channels and NS = N / TPC of
+// their state components (TPC lanes per channel); the partial dot products of y are
+// reduced over the TPC lanes with shuffles.  Every warp of a CTA is an independent
+// worker on CPW channels of one sequence with its own STAGES-deep ring of ROWS-step
+// TMA tiles (x, dt, gate of its channels and the full B|C rows), refilled by its own
+// lane 0 as soon as the warp has consumed a tile, and its own double-buffered y tile
+// stored with TMA.  CTAs are four warps, one per SM sub-partition, so the warps of
+// an SM share its issue slots evenly.  Tensor maps are 3-D ([batch][T][cols]): no
+// tile crosses a sequence end, rows past T load as zeros (dt = 0 leaves the state
+// unchanged) and are clipped on store.
 //
 // Scaled state: with P_t = prod exp(A dt_s) since the last rescale and g = h / P,
-// g_t = g_{t-1} + (dt_t x_t / P_t) B_t and y_t = P_t (C_t . g_t).  P is kept as its
-// log2 (cl) and folded back into g (g <- P g) at every tile start; when no lane's
-// decay over the tile passes 2^-60 (checked warp-uniformly) the tile runs the
-// unrolled fast path, otherwise the per-step path that folds on demand and restarts
-// the state after a single step decaying by more than 2^-60.
-template <int NP>
-struct ScaledState {
-  float2 g[NP];
-  float cl;  // log2 of the scale P
-  HY_DEV void zero() {
-#pragma unroll
-    for (int i = 0; i < NP; ++i) g[i] = make_float2(0.f, 0.f);
-    cl = 0.f;
-  }
-  HY_DEV void fold() {
-    const float P = ex2_approx(cl);
-    const float2 P2 = make_float2(P, P);
-#pragma unroll
-    for (int i = 0; i < NP; ++i) g[i] = __fmul2_rn(g[i], P2);
-    cl = 0.f;
-  }
-  // advance the scale by one step of log2-decay l2a; returns 1 / P_t
-  HY_DEV float advance(float l2a) {
-    float c = cl + l2a;
-    if (c < -60.f) {  // rare: fold the scale into g
-      fold();
-      if (l2a < -60.f) {
-#pragma unroll
-        for (int i = 0; i < NP; ++i) g[i] = make_float2(0.f, 0.f);
-        c = 0.f;
-      } else {
-        c = l2a;
-      }
-    }
-    cl = c;
-    return ex2_approx(-c);
-  }
-};
-
-template <typename TI, int NS, int TPC>
-struct V5Cfg {
-  static constexpr int N = NS * TPC;
-  static constexpr int NWARP = 4;
-  static constexpr int CPW = 32 / TPC;        // channels per warp
-  static constexpr int CPB = NWARP * CPW;     // channels per CTA
-  static constexpr int ROWS = N <= 32 ? 16 : 8;  // steps per tile (B|C rows grow with N)
-  static constexpr int STAGES = 4;
-  static constexpr int XB = ROWS * CPB * (int)sizeof(TI);  // one x / dt / gate tile
+// g_t = g_{t-1} + (dt_t x_t / P_t) B_t and y_t = P_t (C_t . g_t).  The output is
+// formed as y_t = P_t (C_t . g_{t-1} + v_t (C_t . B_t)), v_t = dt_t x_t / P_t, so
+// that it reads only the previous state and never waits on this step's update; the
+// row dot product C_t . B_t is shared by all channels and computed once per tile row.
+// -log2 P is kept per channel (ncl) and folded back into g every block of BLK steps;
+// a block whose decay would take P below 2^-60 runs the per-step path that folds on
+// demand and restarts the state after a single step decaying by more than 2^-60.
+//
+// B|C reads: lanes of different slices read different 16-byte chunks of the same row;
+// slice s visits its chunks in an order rotated by (s * NS / 32), which puts the
+// slices' chunks in distinct shared-memory banks.
+template <typename TI, int N, int TPC, int CPL>
+struct WCfg {
+  static constexpr int NS = N / TPC;            // state components per lane and channel
+  static constexpr int NP = NS / 2;             // packed fp32x2 pairs
+  static constexpr int NQ = NS / 4;             // 16-byte chunks of B (and of C) per lane
+  static constexpr int CPW = (32 / TPC) * CPL;  // channels per warp
+  static constexpr int WPC = 4;                 // warps per CTA
+  static constexpr int CPB = WPC * CPW;         // channels per CTA
+  static constexpr int BLK = NQ * CPL <= 4 ? 16 : 8;  // steps per unrolled block (registers)
+  static constexpr int ROWS = (N == 16 && sizeof(TI) == 2) ? 32 : (N <= 32 ? 16 : 8);  // a multiple of BLK
+  static constexpr int STAGES = (N <= 32 && TPC == 1) ? 4 : 3;
+  static constexpr int LPR = 32 / ROWS;               // lanes per row for C . B
+  static constexpr int XB = ROWS * CPW * (int)sizeof(TI);  // one x / dt / gate tile
   static constexpr int BCB = ROWS * 2 * N * 4;              // one B|C tile
   static constexpr int STAGE_B = 3 * XB + BCB;
-  static constexpr int YB = ROWS * CPW * (int)sizeof(TI);   // one warp's y tile
-  static constexpr int SMEM = STAGES * STAGE_B + NWARP * 2 * YB + 2 * STAGES * 8 + 16 + 128;
+  static constexpr int YB = ROWS * CPW * (int)sizeof(TI);   // one y tile
+  static constexpr int WARP_B = (STAGES * STAGE_B + 2 * YB + STAGES * 8 + 16 + 127) / 128 * 128;
+  static constexpr int SMEM = WPC * WARP_B + 128;
+  static constexpr int THREADS = 32 * WPC;
+  static_assert(ROWS % BLK == 0 && 32 % ROWS == 0, "tile rows");
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
-template <typename TI, int NS, int TPC>
-__global__ void __launch_bounds__(128) scan_v5_kernel(const __grid_constant__ CUtensorMap tmX,
-                                                      const __grid_constant__ CUtensorMap tmDT,
-                                                      const __grid_constant__ CUtensorMap tmG,
-                                                      const __grid_constant__ CUtensorMap tmBC,
-                                                      const __grid_constant__ CUtensorMap tmY, const ScanParams p,
-                                                      unsigned* status) {
-  using C = V5Cfg<TI, NS, TPC>;
-  constexpr int N = C::N;
-  constexpr int NP = NS / 2;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* ybuf = smem + C::STAGES * C::STAGE_B;  // [NWARP][2][ROWS][CPW]
-  uint64_t* full = reinterpret_cast<uint64_t*>(ybuf + C::NWARP * 2 * C::YB);
-  uint64_t* empty = full + C::STAGES;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::STAGES);
+// CPL adjacent channels of one row: load from a shared address, store to a pointer.
+template <typename TI, int CPL> struct ChanLd;
+template <> struct ChanLd<__nv_bfloat16, 1> {
+  static HY_DEV void ld(uint32_t a, float (&v)[1]) { v[0] = __uint_as_float(lds_u16(a) << 16); }
+  static HY_DEV void st(uint8_t* p, const float (&v)[1]) { *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v[0]); }
+};
+template <> struct ChanLd<__nv_bfloat16, 2> {
+  static HY_DEV void ld(uint32_t a, float (&v)[2]) {
+    const uint32_t u = lds_u32(a);
+    v[0] = bf16lo(u);
+    v[1] = bf16hi(u);
+  }
+  static HY_DEV void st(uint8_t* p, const float (&v)[2]) { *reinterpret_cast<uint32_t*>(p) = pack_bf16(v[0], v[1]); }
+};
+template <> struct ChanLd<float, 1> {
+  static HY_DEV void ld(uint32_t a, float (&v)[1]) { v[0] = lds_f32(a); }
+  static HY_DEV void st(uint8_t* p, const float (&v)[1]) { *reinterpret_cast<float*>(p) = v[0]; }
+};
+template <> struct ChanLd<float, 2> {
+  static HY_DEV void ld(uint32_t a, float (&v)[2]) {
+    const float2 f = lds_f2(a);
+    v[0] = f.x;
+    v[1] = f.y;
+  }
+  static HY_DEV void st(uint8_t* p, const float (&v)[2]) { *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]); }
+};
 
+template <typename TI, int N, int TPC, int CPL>
+__global__ void __launch_bounds__(128) scan_w_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                     const __grid_constant__ CUtensorMap tmDT,
+                                                     const __grid_constant__ CUtensorMap tmG,
+                                                     const __grid_constant__ CUtensorMap tmBC,
+                                                     const __grid_constant__ CUtensorMap tmY, const ScanParams p,
+                                                     unsigned* status) {
+  using C = WCfg<TI, N, TPC, CPL>;
+  constexpr int NS = C::NS, NP = C::NP, NQ = C::NQ, CPW = C::CPW;
+  constexpr uint32_t es = sizeof(TI);
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chw = lane / TPC, slice = lane % TPC;  // channel within the warp, state slice
-  const int cl_cta = warp * C::CPW + chw;          // channel within the CTA
-  const int c = blockIdx.x * C::CPB + cl_cta;
   const int b = blockIdx.y;
-  const int n0 = slice * NS;
+  const int wcol = (blockIdx.x * C::WPC + warp) * CPW;  // first channel of this warp
+  if (wcol >= p.Di) return;                             // (no CTA-wide synchronisation below)
   const int n_tiles = (p.T + C::ROWS - 1) / C::ROWS;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C::NWARP);
-    }
+  uint8_t* wsm = smem_raw + warp * C::WARP_B;
+  const uint32_t ring = smem_u32(wsm);
+  uint8_t* ybuf = wsm + C::STAGES * C::STAGE_B;  // [2][ROWS][CPW]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ybuf + 2 * C::YB);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + C::STAGES);
+
+  if (lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(&full[s], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  __syncthreads();
-
-  const float A2 = c < p.Di ? -expf(p.a_log[c]) * 1.4426950408889634f : 0.f;
-  const bool producer = threadIdx.x == 0;
-  uint32_t issued = 0;
-  auto issue = [&](int k) {  // tile k -> slot k % STAGES (tiles are issued in order)
-    const int slot = k % C::STAGES;
-    if (k >= C::STAGES && !mbar_wait(&empty[slot], ((k / C::STAGES) & 1) ^ 1u, status, abort_flag)) return false;
-    uint8_t* st = smem + slot * C::STAGE_B;
+  __syncwarp();
+  int issued = 0;  // meaningful on lane 0
+  auto issue = [&](int t_idx) {  // lane 0: tile t_idx into slot t_idx % STAGES
+    const int slot = t_idx % C::STAGES;
+    uint8_t* st = wsm + slot * C::STAGE_B;
     mbar_arrive_expect_tx(&full[slot], C::STAGE_B);
-    const int col = blockIdx.x * C::CPB, t = k * C::ROWS;
-    tma_load_3d(st, &tmX, &full[slot], col, t, b);
-    tma_load_3d(st + C::XB, &tmDT, &full[slot], col, t, b);
-    tma_load_3d(st + 2 * C::XB, &tmG, &full[slot], col, t, b);
+    const int t = t_idx * C::ROWS;
+    tma_load_3d(st, &tmX, &full[slot], wcol, t, b);
+    tma_load_3d(st + C::XB, &tmDT, &full[slot], wcol, t, b);
+    tma_load_3d(st + 2 * C::XB, &tmG, &full[slot], wcol, t, b);
     tma_load_3d(st + 3 * C::XB, &tmBC, &full[slot], 0, t, b);
     ++issued;
-    return true;
   };
-  bool ok = true;
-  if (producer)
-    for (int k = 0; ok && k < C::STAGES - 1 && k < n_tiles; ++k) ok = issue(k);
+  if (lane == 0)
+    for (int t_idx = 0; t_idx < C::STAGES && t_idx < n_tiles; ++t_idx) issue(t_idx);
 
-  ScaledState<NP> st;
-  st.zero();
-  uint8_t* my_y = ybuf + warp * 2 * C::YB;
-  const size_t es = sizeof(TI);
+  const int cg = lane / TPC, slice = lane % TPC;
+  const int ccol = cg * CPL;  // first channel of this lane within the warp
+  const int c0 = wcol + ccol;
+  const int n0 = slice * NS;
+  const int rot = (slice * NS / 32) & (NQ - 1);
+  float A2[CPL];  // A in log2 units: exp(A dt) = exp2(A2 dt)
+#pragma unroll
+  for (int q = 0; q < CPL; ++q) A2[q] = c0 + q < p.Di ? -expf(p.a_log[c0 + q]) * 1.4426950408889634f : 0.f;
+
+  float2 g[CPL][NP];
+  float ncl[CPL];  // -log2 of the running scale P
+#pragma unroll
+  for (int q = 0; q < CPL; ++q) {
+#pragma unroll
+    for (int i = 0; i < NP; ++i) g[q][i] = make_float2(0.f, 0.f);
+    ncl[q] = 0.f;
+  }
+  const bool ywriter = slice == 0;
+
+  // B and C chunks of this lane for one row (rotated chunk order, see above)
+  auto load_bc = [&](uint32_t row_addr, float4 (&bq)[NQ], float4 (&cq)[NQ]) {
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      const uint32_t off = (n0 + ((j + rot) & (NQ - 1)) * 4) * 4;
+      bq[j] = lds_f4(row_addr + off);
+      cq[j] = lds_f4(row_addr + N * 4 + off);
+    }
+  };
+  // one step: y = C_t . g_{t-1} + v_t (C_t . B_t) (the partial dot reduced over the
+  // slices), then g_t = g_{t-1} + v_t B_t.  Both read only the previous state.
+  auto step_core = [&](const float4 (&bq)[NQ], const float4 (&cq)[NQ], const float (&v)[CPL], float cb,
+                       float (&y)[CPL]) {
+    float2 ya[CPL], yb[CPL];
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) {
+      ya[q] = make_float2(0.f, 0.f);
+      yb[q] = make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      const float2 b01 = make_float2(bq[j].x, bq[j].y), b23 = make_float2(bq[j].z, bq[j].w);
+      const float2 c01 = make_float2(cq[j].x, cq[j].y), c23 = make_float2(cq[j].z, cq[j].w);
+#pragma unroll
+      for (int q = 0; q < CPL; ++q) {
+        const float2 v2 = make_float2(v[q], v[q]);
+        ya[q] = __ffma2_rn(c01, g[q][2 * j], ya[q]);
+        yb[q] = __ffma2_rn(c23, g[q][2 * j + 1], yb[q]);
+        g[q][2 * j] = __ffma2_rn(v2, b01, g[q][2 * j]);
+        g[q][2 * j + 1] = __ffma2_rn(v2, b23, g[q][2 * j + 1]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) {
+      float sum = (ya[q].x + ya[q].y) + (yb[q].x + yb[q].y);
+#pragma unroll
+      for (int off = 1; off < TPC; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      y[q] = fmaf(v[q], cb, sum);
+    }
+  };
+  // B|C rows are prefetched one step ahead when the registers allow it
+  constexpr bool kPrefetch = NQ * CPL <= 4;
+
+  bool ok = true;
   int k = 0;
   for (; k < n_tiles; ++k) {
-    if (producer && ok && k + C::STAGES - 1 < n_tiles) ok = issue(k + C::STAGES - 1);
     const int slot = k % C::STAGES;
     if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], (k / C::STAGES) & 1, status, abort_flag))) {
       ok = false;
       break;
     }
-    const uint8_t* tile = smem + slot * C::STAGE_B;
-    const uint8_t* tx = tile + cl_cta * es;
-    const uint8_t* td = tile + C::XB + cl_cta * es;
-    const uint8_t* tg = tile + 2 * C::XB + cl_cta * es;
-    const float* tbc = reinterpret_cast<const float*>(tile + 3 * C::XB) + n0;
-    const int rows = min(C::ROWS, p.T - k * C::ROWS);
-    // y tile of this warp (double-buffered; the TMA store of tile k-2 must have read it)
-    TI* yt = reinterpret_cast<TI*>(my_y + (k & 1) * C::YB);
-    if (lane == 0) bulk_wait_read1();
+    const uint32_t tile = ring + slot * C::STAGE_B;
+    const uint32_t tx = tile + ccol * es;
+    const uint32_t td = tile + C::XB + ccol * es;
+    const uint32_t tg = tile + 2 * C::XB + ccol * es;
+    const uint32_t tbc = tile + 3 * C::XB;
+    uint8_t* yt = ybuf + (k & 1) * C::YB;  // this warp's y tile [ROWS][CPW]
+    if (lane == 0) bulk_wait_read1();      // the store of tile k-2 has read this buffer
     __syncwarp();
 
-    st.fold();
-    bool fast = rows == C::ROWS;
-    if (fast) {
-      float cum = 0.f;
+    // C_t . B_t of the tile's rows: LPR lanes per row, chunks rotated by row (banks)
+    float cb_row;
+    {
+      constexpr int CPP = (N / 4) / C::LPR;  // 16-byte chunks per lane
+      const int row = lane / C::LPR, part = lane % C::LPR;
+      const uint32_t ra = tbc + row * 2 * N * 4;
+      float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int r = 0; r < C::ROWS; ++r) cum = fmaf(A2, to_f<TI>(*reinterpret_cast<const TI*>(td + r * C::CPB * es)), cum);
-      fast = cum >= -60.f;
+      for (int j = 0; j < CPP; ++j) {
+        const uint32_t off = (part * CPP + ((j + row) & (CPP - 1))) * 16;
+        const float4 bb = lds_f4(ra + off), cc = lds_f4(ra + N * 4 + off);
+        a0 = __ffma2_rn(make_float2(bb.x, bb.y), make_float2(cc.x, cc.y), a0);
+        a1 = __ffma2_rn(make_float2(bb.z, bb.w), make_float2(cc.z, cc.w), a1);
+      }
+      cb_row = (a0.x + a0.y) + (a1.x + a1.y);
+#pragma unroll
+      for (int off = 1; off < C::LPR; off <<= 1) cb_row += __shfl_xor_sync(0xffffffffu, cb_row, off);
     }
-    if (__all_sync(0xffffffffu, fast)) {
+
+    // blocks of BLK steps: fold the scale into g, then either the unrolled fast block
+    // (every scalar of the block's steps first -- loads, decay chain, SFU -- then the
+    // state chain with B|C prefetched one step ahead) or, when some channel's decay
+    // over the block passes 2^-60, the per-step path.
+#pragma unroll 1
+    for (int r0 = 0; r0 < C::ROWS; r0 += C::BLK) {
 #pragma unroll
-      for (int r0 = 0; r0 < C::ROWS; r0 += 4) {  // four steps: scales first (independent SFU ops), then the chain
-        float v[4], P[4], gt[4];
+      for (int q = 0; q < CPL; ++q) {
+        const float P = ex2_approx(-ncl[q]);
+        const float2 P2 = make_float2(P, P);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int r = r0 + q;
-          const float d = to_f<TI>(*reinterpret_cast<const TI*>(td + r * C::CPB * es));
-          const float xv = to_f<TI>(*reinterpret_cast<const TI*>(tx + r * C::CPB * es));
-          gt[q] = to_f<TI>(*reinterpret_cast<const TI*>(tg + r * C::CPB * es));
-          st.cl = fmaf(A2, d, st.cl);
-          v[q] = d * xv * ex2_approx(-st.cl);
-          P[q] = ex2_approx(st.cl);
-        }
+        for (int i = 0; i < NP; ++i) g[q][i] = __fmul2_rn(g[q][i], P2);
+        ncl[q] = 0.f;
+      }
+      float v[C::BLK][CPL], P[C::BLK][CPL], gv[C::BLK][CPL];
+      bool fast = true;
+      {
+        float nc[CPL];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int r = r0 + q;
-          const float4* B4 = reinterpret_cast<const float4*>(tbc + r * 2 * N);
-          const float4* C4 = reinterpret_cast<const float4*>(tbc + r * 2 * N + N);
-          const float2 v2 = make_float2(v[q], v[q]);
-          float2 ya = make_float2(0.f, 0.f), yb = make_float2(0.f, 0.f);
+        for (int q = 0; q < CPL; ++q) nc[q] = 0.f;
 #pragma unroll
-          for (int j = 0; j < NS / 4; ++j) {
-            const float4 bb = B4[j], cv = C4[j];
-            st.g[2 * j] = __ffma2_rn(v2, make_float2(bb.x, bb.y), st.g[2 * j]);
-            st.g[2 * j + 1] = __ffma2_rn(v2, make_float2(bb.z, bb.w), st.g[2 * j + 1]);
-            ya = __ffma2_rn(make_float2(cv.x, cv.y), st.g[2 * j], ya);
-            yb = __ffma2_rn(make_float2(cv.z, cv.w), st.g[2 * j + 1], yb);
+        for (int s = 0; s < C::BLK; ++s) {
+          float dv[CPL], xv[CPL];
+          const uint32_t ro = (r0 + s) * CPW * es;
+          ChanLd<TI, CPL>::ld(td + ro, dv);
+          ChanLd<TI, CPL>::ld(tx + ro, xv);
+          ChanLd<TI, CPL>::ld(tg + ro, gv[s]);
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) {
+            nc[q] = fmaf(-A2[q], dv[q], nc[q]);
+            v[s][q] = dv[q] * xv[q] * ex2_approx(nc[q]);
+            P[s][q] = ex2_approx(-nc[q]);
           }
-          float y = (ya.x + ya.y) + (yb.x + yb.y);
+        }
 #pragma unroll
-          for (int off = 1; off < TPC; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
-          if (slice == 0) yt[r * C::CPW + chw] = from_f<TI>(gt[q] * P[q] * y);
+        for (int q = 0; q < CPL; ++q) {
+          fast = fast && nc[q] <= 60.f;
+          ncl[q] = nc[q];
         }
       }
-    } else {
-      for (int r = 0; r < rows; ++r) {
-        const float d = to_f<TI>(*reinterpret_cast<const TI*>(td + r * C::CPB * es));
-        const float xv = to_f<TI>(*reinterpret_cast<const TI*>(tx + r * C::CPB * es));
-        const float gv = to_f<TI>(*reinterpret_cast<const TI*>(tg + r * C::CPB * es));
-        const float v = d * xv * st.advance(A2 * d);
-        const float2 v2 = make_float2(v, v);
-        const float4* B4 = reinterpret_cast<const float4*>(tbc + r * 2 * N);
-        const float4* C4 = reinterpret_cast<const float4*>(tbc + r * 2 * N + N);
-        float2 ya = make_float2(0.f, 0.f), yb = make_float2(0.f, 0.f);
+      if (__all_sync(0xffffffffu, fast)) {
+        float4 bq[2][NQ], cq[2][NQ];
+        if (kPrefetch) load_bc(tbc + r0 * 2 * N * 4, bq[0], cq[0]);
 #pragma unroll
-        for (int j = 0; j < NS / 4; ++j) {
-          const float4 bb = B4[j], cv = C4[j];
-          st.g[2 * j] = __ffma2_rn(v2, make_float2(bb.x, bb.y), st.g[2 * j]);
-          st.g[2 * j + 1] = __ffma2_rn(v2, make_float2(bb.z, bb.w), st.g[2 * j + 1]);
-          ya = __ffma2_rn(make_float2(cv.x, cv.y), st.g[2 * j], ya);
-          yb = __ffma2_rn(make_float2(cv.z, cv.w), st.g[2 * j + 1], yb);
+        for (int s = 0; s < C::BLK; ++s) {
+          float y[CPL], o[CPL];
+          if (kPrefetch) {
+            if (s + 1 < C::BLK) load_bc(tbc + (r0 + s + 1) * 2 * N * 4, bq[(s + 1) & 1], cq[(s + 1) & 1]);
+          } else {
+            load_bc(tbc + (r0 + s) * 2 * N * 4, bq[s & 1], cq[s & 1]);
+          }
+          const float cb = __shfl_sync(0xffffffffu, cb_row, (r0 + s) * C::LPR);
+          step_core(bq[s & 1], cq[s & 1], v[s], cb, y);
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) o[q] = gv[s][q] * P[s][q] * y[q];
+          if (ywriter) ChanLd<TI, CPL>::st(yt + ((r0 + s) * CPW + ccol) * es, o);
         }
-        float y = (ya.x + ya.y) + (yb.x + yb.y);
+      } else {
+        // per-step path: fold on demand, restart after a single step decaying past 2^-60
 #pragma unroll
-        for (int off = 1; off < TPC; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
-        if (slice == 0) yt[r * C::CPW + chw] = from_f<TI>(gv * ex2_approx(st.cl) * y);
+        for (int q = 0; q < CPL; ++q) ncl[q] = 0.f;
+#pragma unroll 1
+        for (int s = 0; s < C::BLK; ++s) {
+          float dv[CPL], xv[CPL], gt[CPL], vv[CPL], y[CPL], o[CPL];
+          const uint32_t ro = (r0 + s) * CPW * es;
+          ChanLd<TI, CPL>::ld(td + ro, dv);
+          ChanLd<TI, CPL>::ld(tx + ro, xv);
+          ChanLd<TI, CPL>::ld(tg + ro, gt);
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) {
+            const float l = -A2[q] * dv[q];  // >= 0
+            float c = ncl[q] + l;
+            if (c > 60.f) {
+              const float Pf = ex2_approx(-ncl[q]);
+              const float2 P2 = make_float2(Pf, Pf);
+#pragma unroll
+              for (int i = 0; i < NP; ++i) g[q][i] = __fmul2_rn(g[q][i], P2);
+              if (l > 60.f) {
+#pragma unroll
+                for (int i = 0; i < NP; ++i) g[q][i] = make_float2(0.f, 0.f);
+                c = 0.f;
+              } else {
+                c = l;
+              }
+            }
+            ncl[q] = c;
+            vv[q] = dv[q] * xv[q] * ex2_approx(c);
+          }
+          float4 bq[NQ], cq[NQ];
+          load_bc(tbc + (r0 + s) * 2 * N * 4, bq, cq);
+          const float cb = __shfl_sync(0xffffffffu, cb_row, (r0 + s) * C::LPR);
+          step_core(bq, cq, vv, cb, y);
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) o[q] = gt[q] * ex2_approx(-ncl[q]) * y[q];
+          if (ywriter) ChanLd<TI, CPL>::st(yt + ((r0 + s) * CPW + ccol) * es, o);
+        }
       }
     }
-    // release the input tile, then store this warp's y tile
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
+    // every lane is done with the slot and the y tile: refill the slot, store y
     fence_proxy_async_smem();
     __syncwarp();
-    const int ycol = blockIdx.x * C::CPB + warp * C::CPW;
-    if (lane == 0 && ycol < p.Di) {  // a warp whose channels all lie past Di stores nothing
-      tma_store_3d(&tmY, yt, ycol, k * C::ROWS, b);
+    if (lane == 0) {
+      if (k + C::STAGES < n_tiles) issue(k + C::STAGES);
+      tma_store_3d(&tmY, yt, wcol, k * C::ROWS, b);
       bulk_commit();
     }
   }
-  if (lane == 0) bulk_wait_all();
-  if (!ok && producer) {  // let the copies this warp has not consumed land before the CTA exits
-    int never = 0;
-    for (int t = k; t < static_cast<int>(issued); ++t)
-      mbar_wait(&full[t % C::STAGES], (t / C::STAGES) & 1u, nullptr, &never, 100000000ull);
+  if (lane == 0) {
+    bulk_wait_all();
+    if (!ok) {  // let the copies this warp issued but did not consume land before it exits
+      int never = 0;
+      for (int j = k; j < issued; ++j)
+        mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1u, nullptr, &never, 100000000ull);
+    }
   }
 }
 
@@ -434,18 +551,6 @@ EncodeTiledFn scan_encode_fn() {
   return fn;
 }
 
-// 2-D map over [rows, cols] (row stride ld elements), box = bc x br, no swizzle.
-bool map2d(CUtensorMap* m, const void* base, bool f32, long long rows, long long cols, long long ld, int bc, int br) {
-  EncodeTiledFn fn = scan_encode_fn();
-  if (!fn) return false;
-  const int es = f32 ? 4 : 2;
-  cuuint64_t gd[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t gs[1] = {static_cast<cuuint64_t>(ld) * es};
-  cuuint32_t bx[2] = {static_cast<cuuint32_t>(bc), static_cast<cuuint32_t>(br)}, el[2] = {1, 1};
-  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
-            gd, gs, bx, el, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 // 3-D map over [batch][T][cols] (row stride ld elements), box = bc x br x 1, no swizzle.
 bool map3d(CUtensorMap* m, const void* base, bool f32, int batch, int T, long long cols, long long ld, int bc,
@@ -461,28 +566,30 @@ bool map3d(CUtensorMap* m, const void* base, bool f32, int batch, int T, long lo
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename TI, int NS, int TPC>
-cudaError_t launch_v5(const ScanDesc& s, cudaStream_t st) {
-  using C = V5Cfg<TI, NS, TPC>;
+template <typename TI, int N, int TPC, int CPL>
+cudaError_t launch_w(const ScanDesc& s, cudaStream_t st) {
+  using C = WCfg<TI, N, TPC, CPL>;
+  static_assert(C::CPW * sizeof(TI) % 16 == 0, "tile rows must be whole 16-byte units");
   const bool f32 = sizeof(TI) == 4;
   CUtensorMap tx, td, tg, tb, ty;
-  if (!map3d(&tx, s.x, f32, s.batch, s.T, s.d_inner, s.d_inner, C::CPB, C::ROWS) ||
-      !map3d(&td, s.dt, f32, s.batch, s.T, s.d_inner, s.d_inner, C::CPB, C::ROWS) ||
-      !map3d(&tg, s.gate, f32, s.batch, s.T, s.d_inner, s.d_inner, C::CPB, C::ROWS) ||
-      !map3d(&tb, s.bc, true, s.batch, s.T, 2 * C::N, 2 * C::N, 2 * C::N, C::ROWS) ||
+  if (!map3d(&tx, s.x, f32, s.batch, s.T, s.d_inner, s.d_inner, C::CPW, C::ROWS) ||
+      !map3d(&td, s.dt, f32, s.batch, s.T, s.d_inner, s.d_inner, C::CPW, C::ROWS) ||
+      !map3d(&tg, s.gate, f32, s.batch, s.T, s.d_inner, s.d_inner, C::CPW, C::ROWS) ||
+      !map3d(&tb, s.bc, true, s.batch, s.T, 2 * N, 2 * N, 2 * N, C::ROWS) ||
       !map3d(&ty, s.y, f32, s.batch, s.T, s.d_inner, s.y_ld, C::CPW, C::ROWS))
     return cudaErrorInvalidValue;
   static int attr_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 31 && !(attr_mask & (1 << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(scan_v5_kernel<TI, NS, TPC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e =
+        cudaFuncSetAttribute(scan_w_kernel<TI, N, TPC, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_mask |= 1 << dev;
   }
   ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
   dim3 grid((s.d_inner + C::CPB - 1) / C::CPB, s.batch);
-  scan_v5_kernel<TI, NS, TPC><<<grid, 32 * C::NWARP, C::SMEM, st>>>(tx, td, tg, tb, ty, p, s.status);
+  scan_w_kernel<TI, N, TPC, CPL><<<grid, C::THREADS, C::SMEM, st>>>(tx, td, tg, tb, ty, p, s.status);
   return cudaGetLastError();
 }
 
@@ -501,14 +608,14 @@ cudaError_t launch_t(const ScanDesc& s, cudaStream_t st) {
   // x, dt, gate, B|C and y; otherwise the per-channel kernel runs.
   auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
   const long long es = static_cast<long long>(sizeof(TI));
-  const bool v5_ok = (s.d_inner * es) % 16 == 0 && (s.y_ld * es) % 16 == 0 && a16(s.x) && a16(s.dt) &&
+  const bool tma_ok = (s.d_inner * es) % 16 == 0 && (s.y_ld * es) % 16 == 0 && a16(s.x) && a16(s.dt) &&
                      a16(s.gate) && a16(s.bc) && a16(s.y);
-  if (v5_ok) {
+  if (tma_ok) {
     switch (s.d_state) {
-      case 16: return launch_v5<TI, 8, 2>(s, st);
-      case 32: return launch_v5<TI, 16, 2>(s, st);
-      case 64: return launch_v5<TI, 16, 4>(s, st);
-      case 128: return launch_v5<TI, 32, 4>(s, st);
+      case 16: return launch_w<TI, 16, HY_SCAN16_TPC, HY_SCAN16_CPL>(s, st);
+      case 32: return launch_w<TI, 32, 1, 1>(s, st);
+      case 64: return launch_w<TI, 64, 4, 2>(s, st);
+      case 128: return launch_w<TI, 128, HY_SCAN128_TPC, HY_SCAN128_CPL>(s, st);
       default: break;  // N = 256: a B|C row exceeds one TMA box; per-channel kernel below
     }
   }
