@@ -170,7 +170,13 @@ def test_stack24_block_pair_full_size(pair):
     """Every block pair (2k, 2k+1) of the 24-block workload -- producer and consumer
     of one shared K/V, global or SWA as scheduled, SwiGLU FFN -- run as a 2-block
     stack on the full batch; sequence 0 checked over a causal prefix longer than
-    window + meta, sequence 7 over a short prefix, both at the 2e-2 bound."""
+    window + meta, sequence 7 over a short prefix.  Bound per (pair, sequence): 2e-2,
+    or 1.5x the pair's bf16-storage deviation where that is larger (two layers and two
+    FFNs compose; derived by tests/golden/make_stack_tolerance.py from the oracle)."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "stack24_tolerance.json")) as f:
+        bounds = json.load(f)["block_pairs"]
     full = synth.workload("hymba1p5b_stack24")
     wl = synth.workload("hymba1p5b_stack24")
     wl.layers = full.layers[2 * pair:2 * pair + 2]
@@ -182,7 +188,10 @@ def test_stack24_block_pair_full_size(pair):
     for b, L in ((0, 1100), (7, 160)):
         shapes = [dataclasses.replace(s, batch=1, seq_len=L) for s in wl.layers]
         ref = O.stack_forward(x[b:b + 1, :L], meta, ps, shapes)
-        assert_close(g[b, :s0.n_meta + L], ref[0], "bf16", f"blocks {2 * pair},{2 * pair + 1} sequence {b}")
+        bound = bounds[f"{pair}/{b}"]
+        assert bound["prefix_user_tokens"] == L
+        assert_close(g[b, :s0.n_meta + L], ref[0], "bf16", f"blocks {2 * pair},{2 * pair + 1} sequence {b}",
+                     tol=bound["tolerance"])
 
 
 def test_stack24_full_depth_prefix():
