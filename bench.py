@@ -59,8 +59,84 @@ def _workload_config(wl: synth.Workload, extra=None):
     return cfg
 
 
-def _in_proj_flops(s: synth.LayerShape) -> float:
-    return 2.0 * s.d_model * s.n_in * s.batch * s.T
+def _visible_pairs(T: int, M: int, W: int) -> int:
+    """(query, key) pairs the attention mask admits in one sequence of T rows:
+    key j <= query i and (i - j <= W or j < M); W = -1 is global causal."""
+    if W < 0:
+        return T * (T + 1) // 2
+    i = np.arange(T, dtype=np.int64)
+    return int((np.minimum(i + 1, W + 1) + np.maximum(0, np.minimum(M, i - W))).sum())
+
+
+def stage_work(s: synth.LayerShape):
+    """Algorithmic work of each stage of one layer launch: (FLOPs, HBM bytes).
+
+    FLOPs count the dense contractions only (2 per multiply-add; attention 4 dh per
+    visible pair per query head).  Bytes are the compulsory traffic: every operand read
+    once and every result written once (weights included), in the layer's dtype, with
+    B|C in fp32."""
+    es = 2 if s.dtype == "bf16" else 4
+    rows = s.batch * s.T
+    wa, di, n, r, d = s.attn_width, s.d_inner, s.d_state, s.dt_rank, s.d_model
+    kv_out = 0 if s.kv_mode == synth.KV_CONSUME else 2 * s.kv_width
+    pairs = s.batch * _visible_pairs(s.T, s.n_meta, s.window)
+    return {
+        "in_proj": (2.0 * d * s.n_in * rows, es * (rows * d + s.n_in * d + rows * (wa + kv_out + 2 * di))),
+        "x_proj": (2.0 * di * s.xproj_width * rows, es * (rows * di + s.xproj_width * di + rows * r) + 4 * rows * 2 * n),
+        "dt_proj": (2.0 * r * di * rows, es * (rows * r + di * r + rows * di) + 4 * di),
+        "attention": (4.0 * s.head_dim * s.n_q_heads * pairs,
+                      es * (rows * wa + 2 * rows * s.kv_width + rows * wa)),
+        "scan": (4.0 * n * di * rows, es * 4 * rows * di + 4 * rows * 2 * n + 4 * di),
+        "branch_norm": (0.0, es * 2 * rows * (wa + di) + 4 * (wa + di)),
+        "out_proj": (2.0 * (wa + di) * d * rows, es * (rows * (wa + di) + d * (wa + di) + rows * d)),
+    }
+
+
+KERNEL_NAMES = {"in_proj": "gemm_bf16_tc, tcgen05", "x_proj": "gemm_bf16_tc, tcgen05",
+                "dt_proj": "gemm_bf16_tc, tcgen05", "attention": "attn_fwd_tc, tcgen05",
+                "scan": "scan_w_kernel", "branch_norm": "rownorm_warp_kernel", "out_proj": "gemm_bf16_tc, tcgen05"}
+
+# dominant bound of each stage: a dense contraction on the tensor cores or HBM traffic
+STAGE_BOUND = {"in_proj": "tensor", "x_proj": "hbm", "dt_proj": "hbm", "attention": "tensor",
+               "scan": "hbm", "branch_norm": "hbm", "out_proj": "tensor"}
+
+
+def _traffic(stage: str):
+    """DRAM bytes per launch from the committed ncu capture of this stage's kernel,
+    or None when there is none or the kernel's source changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(stage)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
+        return None
+    return rec["dram_bytes_per_launch"]
+
+
+def stage_rooflines(s: synth.LayerShape, stage_us, peaks):
+    """Per stage: achieved work rate against its peak (measured peaks), and the layer's
+    roofline time (sum over stages of the slower of its FLOP and byte times)."""
+    out, t_roof = {}, 0.0
+    hbm = peaks["hbm_gbs"] * 1e9
+    tc = peaks["bf16_tflops_sustained"] * 1e12
+    for name, (fl, by) in stage_work(s).items():
+        t = stage_us[name] * 1e-6
+        t_roof += max(fl / tc, by / hbm)
+        if STAGE_BOUND[name] == "tensor":
+            ach = fl / t / 1e12
+            out[name] = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops_sustained"], 4),
+                         "work_per_launch": fl, "us": stage_us[name]}
+        else:
+            ach = by / t / 1e9
+            out[name] = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(ach / peaks["hbm_gbs"], 4), "work_per_launch": by, "us": stage_us[name]}
+    return out, t_roof * 1e6
 
 
 # --------------------------------------------------------------------------- clocks (NVML)
@@ -289,19 +365,22 @@ def run_native(args, rank, world, local_rank):
     value = world * K * tokens_per_step / (total_ms * 1e-3)
 
     peaks, peak_src = _peaks()
-    roofline, stages = None, None
+    roofline, stages, stage_roof, layer_roof = None, None, None, None
     if stage_ev:
         per_stage = {name: float(np.mean([stage_ev[k][i].elapsed_time(stage_ev[k][i + 1]) for k in range(K)]))
                      for i, name in enumerate(H.STAGES)}
         stages = {n: round(v * 1e3, 2) for n, v in per_stage.items()}  # microseconds
-        t_in = per_stage["in_proj"] * 1e-3
-        ach = _in_proj_flops(s0) / t_in / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roofline = {"kernel": "in_proj gemm_bf16_tc (tcgen05)", "bound": "tensor", "achieved": round(ach, 1),
-                    "peak": peak, "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
-                    "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a continuous loop)",
-                    "in_proj_us": round(per_stage["in_proj"] * 1e3, 2),
-                    "algorithmic_flops_per_launch": _in_proj_flops(s0)}
+        stage_roof, t_roof_us = stage_rooflines(s0, stages, peaks)
+        top = max(stages, key=stages.get)   # the dominant kernel of the step
+        r = stage_roof[top]
+        roofline = {"kernel": f"{top} ({KERNEL_NAMES[top]})", "bound": r["bound"], "achieved": r["achieved"],
+                    "peak": r["peak"], "unit": r["unit"], "frac": r["frac"], "traffic": _traffic(top),
+                    "peak_source": (f"{peak_src} bf16_tflops_sustained (kernel timed inside a continuous loop)"
+                                    if r["bound"] == "tensor" else f"{peak_src} hbm_gbs (STREAM-style copy)"),
+                    "us_per_launch": stages[top], "algorithmic_work_per_launch": r["work_per_launch"]}
+        layer_roof = {"roofline_us": round(t_roof_us, 2), "measured_us": round(sum(stages.values()), 2),
+                      "frac": round(t_roof_us / sum(stages.values()), 4),
+                      "definition": "sum over stages of max(FLOPs / bf16 sustained peak, bytes / HBM peak)"}
 
     e2e = None
     if not args.no_e2e:
@@ -342,7 +421,8 @@ def run_native(args, rank, world, local_rank):
                     "parallelism": f"replicas x{world} (batch per rank, no collective)" if world > 1 else "1 GPU",
                     "tokens_per_step_per_gpu": tokens_per_step, "rows_per_step_per_gpu": s0.batch * T,
                     "l2": "flushed between timed steps (256 MiB memset outside the events)"}),
-                "roofline": roofline, "stages_us": stages, "e2e": e2e,
+                "roofline": roofline, "stages_us": stages, "stage_roofline": stage_roof,
+                "layer_roofline": layer_roof, "e2e": e2e,
                 "gpu_launches": n_launch_per_step * K, "clocks": sampler.summary(),
                 "device_status": H.hymba_status_string(status)}
         if world == 1 and not args.no_cpu_baseline:
