@@ -8,8 +8,11 @@
 //   3 dt_proj   softplus(dt_low W_dt^T + b_dt) -> dt
 //   4 attention Q, K/V (own or kv_in) -> Z[:, :Hq*dh]
 //   5 scan      x = X_ssm, dt, B, C, gate = SiLU(G) -> Z[:, Hq*dh:]
-//   6 norm      Z <- [beta1 rms(Z_attn) || beta2 rms(Z_ssm)]   (in place)
+//   6 norm      Z <- [beta1 rms(Z_attn) || beta2 rms(Z_ssm)]   (in place; fp32 only)
 //   7 out_proj  Z W_out^T -> out   (+ residual inside a stack)
+// bf16 fuses the rewrite of step 6 away: each row's two sums of squares are read from
+// Z, beta is folded into W_out's columns, and out_proj accumulates the attention and
+// SSM columns apart and scales each by its row's 1 / rms.
 #include <cstring>
 #include <mutex>
 
@@ -25,8 +28,14 @@ inline size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 inline size_t esize(hymba_dtype_t t) { return t == HYMBA_BF16 ? 2 : 4; }
 
 struct LayerWs {
-  size_t q, kv, xs, g, dtlow, bc, dt, z, total;
+  size_t q, kv, xs, g, dtlow, bc, dt, z, ssq, wsc, total;
 };
+
+// bf16 layers fuse the branch norm into out_proj (the row-sum kernel holds a row of up
+// to 6144 bf16 in one warp's registers); fp32 layers run the separate norm kernel.
+bool fused_branch_norm(const hymba_cfg_t& c) {
+  return c.dtype == HYMBA_BF16 && c.n_q_heads * c.head_dim + c.d_inner <= 6144;
+}
 
 LayerWs layer_ws(const hymba_cfg_t& c, size_t base) {
   const size_t es = esize(c.dtype);
@@ -43,6 +52,11 @@ LayerWs layer_ws(const hymba_cfg_t& c, size_t base) {
   w.bc = o; o = al256(o + rows * 2 * c.d_state * 4);
   w.dt = o; o = al256(o + rows * c.d_inner * es);
   w.z = o; o = al256(o + rows * (wa + c.d_inner) * es);
+  // fused branch norm (bf16): per row, the sums of squares of Y_attn and Y_ssm; and
+  // W_out with beta1 | beta2 folded into its columns
+  const bool fused = fused_branch_norm(c);
+  w.ssq = o; o = al256(o + (fused ? rows * 2 * sizeof(float) : 0));
+  w.wsc = o; o = al256(o + (fused ? static_cast<size_t>(c.d_model) * (wa + c.d_inner) * es : 0));
   w.total = o;
   return w;
 }
@@ -120,6 +134,27 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   float* bc = reinterpret_cast<float*>(ws + L.bc);
   void* dt = ws + L.dt;
   void* z = ws + L.z;
+
+  hy::ScanDesc sd;
+  sd.x = xs;
+  sd.dt = dt;
+  sd.bc = bc;
+  sd.gate = g;
+  sd.a_log = w.a_log;
+  sd.y = static_cast<uint8_t*>(z) + wa * es;
+  sd.y_ld = wa + di;
+  sd.batch = c.batch;
+  sd.T = T;
+  sd.d_inner = di;
+  sd.d_state = c.d_state;
+  sd.bf16 = c.dtype == HYMBA_BF16;
+  sd.status = status;
+  // bf16: the branch norm is fused into out_proj -- the rows of Z are not rewritten;
+  // their two sums of squares are read once, beta is folded into W_out's columns, and
+  // out_proj applies the two 1 / rms row scales to its two accumulators
+  const bool fused_norm = fused_branch_norm(c);
+  float2* ssq = reinterpret_cast<float2*>(ws + L.ssq);
+  void* w_out_scaled = ws + L.wsc;
   void* kvbuf = c.kv_mode == HYMBA_KV_PRODUCE ? kv_out : (c.kv_mode == HYMBA_KV_OWN ? ws + L.kv : nullptr);
   const void* kv_k = c.kv_mode == HYMBA_KV_CONSUME ? kv_in : kvbuf;
   const void* kv_v = static_cast<const uint8_t*>(kv_k) + static_cast<size_t>(rows) * wkv * es;
@@ -207,27 +242,18 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
 
   // 5 selective scan + gate -> Z[:, wa:]
   mark(4);
-  hy::ScanDesc sd;
-  sd.x = xs;
-  sd.dt = dt;
-  sd.bc = bc;
-  sd.gate = g;
-  sd.a_log = w.a_log;
-  sd.y = static_cast<uint8_t*>(z) + wa * es;
-  sd.y_ld = wa + di;
-  sd.batch = c.batch;
-  sd.T = T;
-  sd.d_inner = di;
-  sd.d_state = c.d_state;
-  sd.bf16 = c.dtype == HYMBA_BF16;
-  sd.status = status;
   if ((e = hy::launch_scan(sd, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
 
   // 6 per-branch RMSNorm and beta
   mark(5);
-  if ((e = hy::launch_branch_norm(z, w.beta1, w.beta2, rows, wa, di, c.rms_eps, c.dtype == HYMBA_BF16, st)) !=
-      cudaSuccess)
+  if (fused_norm) {
+    if ((e = hy::launch_scale_cols(w.w_out, w_out_scaled, c.d_model, wa, di, w.beta1, w.beta2, st)) != cudaSuccess ||
+        (e = hy::launch_row_ssq(z, rows, wa, di, ssq, st)) != cudaSuccess)
+      return HYMBA_ERR_CUDA;
+  } else if ((e = hy::launch_branch_norm(z, w.beta1, w.beta2, rows, wa, di, c.rms_eps, c.dtype == HYMBA_BF16,
+                                         st)) != cudaSuccess) {
     return HYMBA_ERR_CUDA;
+  }
 
   // 7 out_proj
   mark(6);
@@ -235,8 +261,17 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   go.a = z;
   go.a_rows = rows;
   go.K = wa + di;
-  go.w = w.w_out;
+  go.w = fused_norm ? w_out_scaled : w.w_out;
   go.N = c.d_model;
+  if (fused_norm) {
+    go.dual_k_blocks = wa / 64;
+    go.row_ssq = ssq;
+    go.inv_wa = 1.f / static_cast<float>(wa);
+    go.inv_ws = 1.f / static_cast<float>(di);
+    go.eps = c.rms_eps;
+    go.out = out;
+    go.out_ld = c.d_model;
+  }
   if (resid_out) {
     go.epi = hy::EPI_RESIDUAL;
     go.resid = out;

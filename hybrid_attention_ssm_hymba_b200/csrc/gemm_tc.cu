@@ -5,13 +5,15 @@
 // stacked blocks (blog.outta.ai Hymba review, "Design formulation"; metaphor-xennon
 // page, "层配置": intermediate_size).
 //
-// Kernel shape: persistent, one CTA per SM, 320 threads:
-//   warp 0      TMA producer (one thread) -> STAGES-deep smem ring (full/empty mbarriers)
-//   warp 1      TMEM allocator + UMMA issuer (one thread), 128 x BN x 16 per instruction
-//   warps 2..9  epilogue: two warps per TMEM lane quadrant, each taking every other
-//               32-column chunk: tcgen05.ld of the accumulator rows, fused elementwise
-//               op, vector stores.  Two TMEM accumulators so the epilogue of tile i
-//               overlaps the mainloop of tile i+1.
+// Kernel shape: persistent, one CTA per SM, 576 threads:
+//   warp 0       TMA producer (one thread) -> STAGES-deep smem ring (full/empty mbarriers)
+//   warp 1       TMEM allocator + UMMA issuer (one thread), 128 x BN x 16 per instruction
+//   warps 2..17  epilogue: four warps per TMEM lane quadrant, each taking every fourth
+//                32-column chunk: tcgen05.ld of its chunks (all issued before the wait),
+//                fused elementwise op, vector stores.  Two TMEM accumulators so the
+//                epilogue of tile i overlaps the mainloop of tile i+1; sixteen warps so
+//                that short-K GEMMs (dt_proj), whose time is all epilogue, keep enough
+//                independent work in flight.
 //
 // "Meta mode" reads the rows of X~_b = [meta; x_b] for each sequence b straight from
 // the meta tokens [M, K] and the user tokens x [B, L, K]: a 128-row tile that holds
@@ -28,8 +30,9 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int NTHREADS = 320;       // producer warp, MMA warp, 8 epilogue warps
-constexpr int EPI_THREADS = 256;
+constexpr int NTHREADS = 576;       // producer warp, MMA warp, 16 epilogue warps
+constexpr int EPI_THREADS = 512;
+constexpr int EPI_GROUPS = 4;       // epilogue warps per TMEM lane quadrant
 constexpr int kMaxBiasSmem = 4096;  // a bias vector up to this length is staged in smem once
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 
@@ -49,6 +52,9 @@ struct GemmParams {
   int swiglu_F;
   int bias_len;             // > 0: the (single) bias segment's vector is staged in smem
   const float* bias_src;
+  int dual_k;               // > 0: fused branch norm, two accumulators split at this K block
+  const float2* row_ssq;
+  float inv_wa, inv_ws, eps;
   unsigned* status;
 };
 
@@ -228,12 +234,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
-        const int buf = it & 1;
-        const uint32_t use = (it >> 1) & 1;
+        // dual mode: one buffer holding both accumulators (attention K blocks, then SSM)
+        const int buf = p.dual_k ? 0 : (it & 1);
+        const uint32_t use = p.dual_k ? (it & 1) : ((it >> 1) & 1);
         if (!mbar_wait(&tempty[buf], use ^ 1u, p.status, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * BN;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
+          const bool second = p.dual_k && kb >= p.dual_k;
+          const uint32_t d_tmem = tmem_base + (p.dual_k ? (second ? BN : 0) : buf * BN);
+          const int kfirst = second ? p.dual_k : 0;  // first K block of this accumulator
           if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) {
             ok = false;
             break;
@@ -244,7 +253,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             umma_bf16_ss(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024), sdesc_sw128(b0 + k * 32, 16, 1024), C::IDESC,
-                         (kb | k) != 0 ? 1u : 0u);
+                         (kb != kfirst || k != 0) ? 1u : 0u);
           umma_commit(&empty[stage]);
           if (++stage == C::STAGES) {
             stage = 0;
@@ -259,14 +268,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_wait(mma_done, 0, nullptr, &never, 100000000ull);
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 2..9)
-    const int quad = warp & 3;         // TMEM lane quadrant this warp may access
-    const int half = (warp - 2) >> 2;  // which alternate 32-column chunks it takes
+    // ------------------------------------------------ epilogue (warps 2..17)
+    const int quad = warp & 3;          // TMEM lane quadrant this warp may access
+    const int grp = (warp - 2) >> 2;    // which every-fourth 32-column chunks it takes
     const int r = quad * 32 + lane;
+    constexpr int CPT = BN / 32 / EPI_GROUPS;  // chunks per thread (BN = 256: 2, BN = 128: 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-      const int buf = it & 1;
-      const uint32_t use = (it >> 1) & 1;
+      const int buf = p.dual_k ? 0 : (it & 1);
+      const uint32_t use = p.dual_k ? (it & 1) : ((it >> 1) & 1);
       // warp-uniform exit: tcgen05.ld below is a warp-collective instruction
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], use, p.status, abort_flag))) break;
       tc_fence_after();
@@ -282,64 +292,117 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         valid = grow < p.a_rows;
       }
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * BN;
-      if (p.epi == EPI_SEGMENTS) {
-#pragma unroll 1
-        for (int c = half; c < BN / 32; c += 2) {
-          uint32_t v[32];
-          tmem_ld32(tb + c * 32, v);
-          tmem_wait_ld();
-          const int col = tc.n * BN + c * 32;
-          if (valid) {
-            const float* tb_bias = p.bias_len ? s_bias : nullptr;
-            if (col < p.N) store16(p, grow, col, v, tb_bias);
-            if (col + 16 < p.N) store16(p, grow, col + 16, v + 16, tb_bias);
-          }
+      if (p.dual_k) {
+        // fused branch norm: out (+ resid) = rsqrt(ssq_a / wa + eps) acc_a + rsqrt(ssq_s / ws + eps) acc_s
+        float sa = 0.f, ss = 0.f;
+        if (valid) {
+          const float2 q2 = p.row_ssq[grow];
+          sa = rsqrtf(fmaf(q2.x, p.inv_wa, p.eps));
+          ss = rsqrtf(fmaf(q2.y, p.inv_ws, p.eps));
         }
-      } else if (p.epi == EPI_SWIGLU) {
-#pragma unroll 1
-        for (int c = half; c < 4; c += 2) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tb + c * 32, g);
-          tmem_ld32(tb + 128 + c * 32, u);
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) {
+          const int cc = (grp + q * EPI_GROUPS) * 32;
+          uint32_t va[32], vs[32];
+          tmem_ld32(tb + cc, va);
+          tmem_ld32(tb + BN + cc, vs);
           tmem_wait_ld();
-          if (valid) {
-            uint4* d = reinterpret_cast<uint4*>(p.out + grow * p.out_ld + tc.n * 128 + c * 32);
+          if (q == CPT - 1) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          const int col = tc.n * BN + cc;
+          if (valid && col < p.N) {
+            float f[32];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float f[8];
+            for (int e = 0; e < 32; ++e) f[e] = fmaf(sa, __uint_as_float(va[e]), ss * __uint_as_float(vs[e]));
+            if (p.epi == EPI_RESIDUAL) {
+              const uint4* rs = reinterpret_cast<const uint4*>(p.resid + grow * p.resid_ld + col);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) f[i] = silu_f(__uint_as_float(g[8 * j + i])) * __uint_as_float(u[8 * j + i]);
-              d[j] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                                pack_bf16(f[6], f[7]));
+              for (int j = 0; j < 4; ++j) {
+                const uint4 qv = rs[j];
+                const uint32_t qq[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  f[8 * j + 2 * i] += bf16lo(qq[i]);
+                  f[8 * j + 2 * i + 1] += bf16hi(qq[i]);
+                }
+              }
             }
+            uint4* d = reinterpret_cast<uint4*>(p.out + grow * p.out_ld + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              d[j] = make_uint4(pack_bf16(f[8 * j], f[8 * j + 1]), pack_bf16(f[8 * j + 2], f[8 * j + 3]),
+                                pack_bf16(f[8 * j + 4], f[8 * j + 5]), pack_bf16(f[8 * j + 6], f[8 * j + 7]));
           }
         }
+        continue;
+      }
+      if (p.epi == EPI_SEGMENTS) {
+        uint32_t v[CPT][32];
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) tmem_ld32(tb + (grp + q * EPI_GROUPS) * 32, v[q]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);  // the accumulator is in registers: free it for tile i+2
+        if (valid) {
+          const float* tb_bias = p.bias_len ? s_bias : nullptr;
+#pragma unroll
+          for (int q = 0; q < CPT; ++q) {
+            const int col = tc.n * BN + (grp + q * EPI_GROUPS) * 32;
+            if (col < p.N) store16(p, grow, col, v[q], tb_bias);
+            if (col + 16 < p.N) store16(p, grow, col + 16, v[q] + 16, tb_bias);
+          }
+        }
+        continue;
+      } else if (p.epi == EPI_SWIGLU) {
+        uint32_t g[32], u[32];
+        const int c = grp;  // one 32-column chunk of the 128 gate / 128 up columns
+        tmem_ld32(tb + c * 32, g);
+        tmem_ld32(tb + 128 + c * 32, u);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);
+        if (valid) {
+          uint4* d = reinterpret_cast<uint4*>(p.out + grow * p.out_ld + tc.n * 128 + c * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = silu_f(__uint_as_float(g[8 * j + i])) * __uint_as_float(u[8 * j + i]);
+            d[j] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                              pack_bf16(f[6], f[7]));
+          }
+        }
+        continue;
       } else {  // EPI_RESIDUAL
-#pragma unroll 1
-        for (int c = half; c < BN / 32; c += 2) {
-          uint32_t v[32];
-          tmem_ld32(tb + c * 32, v);
-          tmem_wait_ld();
-          const int col = tc.n * BN + c * 32;
+        uint32_t v[CPT][32];
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) tmem_ld32(tb + (grp + q * EPI_GROUPS) * 32, v[q]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) {
+          const int col = tc.n * BN + (grp + q * EPI_GROUPS) * 32;
           if (valid && col < p.N) {
             const uint4* rs = reinterpret_cast<const uint4*>(p.resid + grow * p.resid_ld + col);
             uint4* d = reinterpret_cast<uint4*>(p.out + grow * p.out_ld + col);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const uint4 q = rs[j];
-              const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+              const uint4 qv = rs[j];
+              const uint32_t qq[4] = {qv.x, qv.y, qv.z, qv.w};
               uint32_t o[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i)
-                o[i] = pack_bf16(bf16lo(qq[i]) + __uint_as_float(v[8 * j + 2 * i]),
-                                 bf16hi(qq[i]) + __uint_as_float(v[8 * j + 2 * i + 1]));
+                o[i] = pack_bf16(bf16lo(qq[i]) + __uint_as_float(v[q][8 * j + 2 * i]),
+                                 bf16hi(qq[i]) + __uint_as_float(v[q][8 * j + 2 * i + 1]));
               d[j] = make_uint4(o[0], o[1], o[2], o[3]);
             }
           }
         }
+        continue;
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[buf]);
     }
   }
   tc_fence_before();
@@ -467,6 +530,11 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
     }
   }
   if (n_bias != 1 || p.bias_len > kMaxBiasSmem) p.bias_len = 0;  // read from global instead
+  p.dual_k = g.dual_k_blocks;
+  p.row_ssq = g.row_ssq;
+  p.inv_wa = g.inv_wa;
+  p.inv_ws = g.inv_ws;
+  p.eps = g.eps;
   p.resid = static_cast<const __nv_bfloat16*>(g.resid);
   p.resid_ld = g.resid_ld;
   p.out = static_cast<__nv_bfloat16*>(g.out);
@@ -483,7 +551,7 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_gemm_bf16(const GemmDesc& g, cudaStream_t st) {
-  if (g.epi == EPI_SWIGLU || g.N > 128) return launch_bn<256>(g, st);
+  if (g.epi == EPI_SWIGLU || g.N > 128 || g.dual_k_blocks > 0) return launch_bn<256>(g, st);
   return launch_bn<128>(g, st);
 }
 

@@ -50,6 +50,12 @@ struct GemmDesc {
   void* out = nullptr;
   long long out_ld = 0;
   int swiglu_F = 0;
+  // Fused branch norm (bf16 out_proj): the first dual_k_blocks 64-wide K blocks (the
+  // attention columns of Z) accumulate apart from the rest (the SSM columns), and the
+  // epilogue forms rsqrt(row_ssq.x * inv_wa + eps) acc_a + rsqrt(row_ssq.y * inv_ws + eps) acc_s.
+  int dual_k_blocks = 0;
+  const float2* row_ssq = nullptr;
+  float inv_wa = 0.f, inv_ws = 0.f, eps = 0.f;
   unsigned* status = nullptr;
 };
 
@@ -79,6 +85,12 @@ cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, 
                                int w_ssm, float eps, bool bf16, cudaStream_t st);
 cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float eps, bool bf16,
                            cudaStream_t st);
+// Fused branch norm (bf16).  row_ssq: ssq[row] = (sum of z[row, :w_attn]^2, sum of
+// z[row, w_attn:]^2).  scale_cols: w_out[n, k] = w[n, k] * (k < w_attn ? beta1[k] :
+// beta2[k - w_attn]) for a [N, w_attn + w_ssm] weight.
+cudaError_t launch_row_ssq(const void* z, long long rows, int w_attn, int w_ssm, float2* ssq, cudaStream_t st);
+cudaError_t launch_scale_cols(const void* w, void* w_out, int N, int w_attn, int w_ssm, const float* beta1,
+                              const float* beta2, cudaStream_t st);
 
 int num_sms();
 

@@ -6,6 +6,9 @@
 //     "PyTorch伪代码": one RMSNorm per branch).
 //   rmsnorm:     y = x / sqrt(mean(x^2) + eps), unit gain (pre-norm of the
 //     stacked blocks).
+//   row_ssq, scale_cols: the two pieces of the branch norm fused into out_proj (bf16):
+//     per-row sums of squares of both branches, and W_out with beta folded into its
+//     columns.
 // bf16 rows up to 6144 elements: one warp per row with the row held in registers
 // (one HBM read, one write).  Wider rows and fp32: one CTA per row (the second read
 // of the row hits L1/L2).  fp32 sums; 16-byte vector loads and stores.
@@ -199,7 +202,84 @@ bool rownorm_bf16(const void* x, void* y, long long rows, int wa, int ws, const 
   return true;
 }
 
+// Row sums of squares of the two branches of Z (bf16), one warp per row, the row held
+// in registers (16-byte vectors): ssq[row] = (sum over [0, wa), sum over [wa, wa + ws)).
+// wa is a multiple of 8, so no vector straddles the branches.
+template <int MAXV>
+__global__ void __launch_bounds__(256) row_ssq_kernel(const __nv_bfloat16* __restrict__ z, long long rows, int wa,
+                                                      int ws, float2* __restrict__ ssq) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int nv = (wa + ws) / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(z + row * (wa + ws));
+  uint4 v[MAXV];
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k)
+    if (lane + 32 * k < nv) v[k] = src[lane + 32 * k];
+  float sa = 0.f, ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int vi = lane + 32 * k;
+    if (vi < nv) {
+      const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc = fmaf(bf16lo(u[q]), bf16lo(u[q]), fmaf(bf16hi(u[q]), bf16hi(u[q]), acc));
+      if (vi * 8 < wa) sa += acc;
+      else ss += acc;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sa += __shfl_xor_sync(0xffffffffu, sa, o);
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  }
+  if (lane == 0) ssq[row] = make_float2(sa, ss);
+}
+
+// w_out[n, k] = w[n, k] * beta(k), 8 bf16 per thread, grid-stride.
+__global__ void __launch_bounds__(256) scale_cols_kernel(const uint4* __restrict__ w, uint4* __restrict__ w_out,
+                                                         long long n_vec, int row_vecs, int wa,
+                                                         const float* __restrict__ beta1,
+                                                         const float* __restrict__ beta2) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n_vec;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int k0 = static_cast<int>(i % row_vecs) * 8;
+    const float* bb = k0 < wa ? beta1 + k0 : beta2 + (k0 - wa);
+    const float4 b0 = __ldg(reinterpret_cast<const float4*>(bb)), b1 = __ldg(reinterpret_cast<const float4*>(bb + 4));
+    const uint4 q = w[i];
+    w_out[i] = make_uint4(pack_bf16(bf16lo(q.x) * b0.x, bf16hi(q.x) * b0.y), pack_bf16(bf16lo(q.y) * b0.z, bf16hi(q.y) * b0.w),
+                          pack_bf16(bf16lo(q.z) * b1.x, bf16hi(q.z) * b1.y), pack_bf16(bf16lo(q.w) * b1.z, bf16hi(q.w) * b1.w));
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_row_ssq(const void* z, long long rows, int w_attn, int w_ssm, float2* ssq, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const int per_lane = ((w_attn + w_ssm) / 8 + 31) / 32;
+  const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+  const __nv_bfloat16* zz = static_cast<const __nv_bfloat16*>(z);
+  if (per_lane <= 4) row_ssq_kernel<4><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
+  else if (per_lane <= 8) row_ssq_kernel<8><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
+  else if (per_lane <= 12) row_ssq_kernel<12><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
+  else if (per_lane <= 16) row_ssq_kernel<16><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
+  else if (per_lane <= 24) row_ssq_kernel<24><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scale_cols(const void* w, void* w_out, int N, int w_attn, int w_ssm, const float* beta1,
+                              const float* beta2, cudaStream_t st) {
+  const int row_vecs = (w_attn + w_ssm) / 8;
+  const long long n_vec = static_cast<long long>(N) * row_vecs;
+  if (n_vec <= 0) return cudaSuccess;
+  const long long blocks = (n_vec + 255) / 256;
+  scale_cols_kernel<<<static_cast<unsigned>(blocks < 4 * num_sms() ? blocks : 4 * num_sms()), 256, 0, st>>>(
+      static_cast<const uint4*>(w), static_cast<uint4*>(w_out), n_vec, row_vecs, w_attn, beta1, beta2);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, long long rows, int w_attn, int w_ssm,
                                float eps, bool bf16, cudaStream_t st) {
