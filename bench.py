@@ -87,14 +87,18 @@ def stage_work(s: synth.LayerShape):
         "attention": (4.0 * s.head_dim * s.n_q_heads * pairs,
                       es * (rows * wa + 2 * rows * s.kv_width + rows * wa)),
         "scan": (4.0 * n * di * rows, es * 4 * rows * di + 4 * rows * 2 * n + 4 * di),
-        "branch_norm": (0.0, es * 2 * rows * (wa + di) + 4 * (wa + di)),
+        # bf16: the norm is fused into out_proj -- this stage reads Z once for the row sums of
+        # squares and folds beta into a copy of W_out; fp32: Z is normalised in place
+        "branch_norm": (0.0, (es * rows * (wa + di) + 8 * rows + 2 * es * d * (wa + di) + 4 * (wa + di))
+                        if s.dtype == "bf16" else es * 2 * rows * (wa + di) + 4 * (wa + di)),
         "out_proj": (2.0 * (wa + di) * d * rows, es * (rows * (wa + di) + d * (wa + di) + rows * d)),
     }
 
 
 KERNEL_NAMES = {"in_proj": "gemm_bf16_tc, tcgen05", "x_proj": "gemm_bf16_tc, tcgen05",
                 "dt_proj": "gemm_bf16_tc, tcgen05", "attention": "attn_fwd_tc, tcgen05",
-                "scan": "scan_w_kernel", "branch_norm": "rownorm_warp_kernel", "out_proj": "gemm_bf16_tc, tcgen05"}
+                "scan": "scan_w_kernel", "branch_norm": "row_ssq_kernel + scale_cols_kernel",
+                "out_proj": "gemm_bf16_tc, tcgen05, two accumulators"}
 
 # dominant bound of each stage: a dense contraction on the tensor cores or HBM traffic
 STAGE_BOUND = {"in_proj": "tensor", "x_proj": "hbm", "dt_proj": "hbm", "attention": "tensor",
