@@ -24,7 +24,7 @@
 // state sizes of the workloads.
 #ifndef HY_SCAN16_TPC
 #define HY_SCAN16_TPC 1
-#define HY_SCAN16_CPL 1
+#define HY_SCAN16_CPL 2
 #endif
 #ifndef HY_SCAN128_TPC
 #define HY_SCAN128_TPC 4
@@ -200,25 +200,28 @@ __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
 }
 
 // ---------------------------------------------------------------------------------
-// Single-pass scan with warp-private pipelines (the main path).
+// Main scan kernel: warp-private pipelines, optional split of T into chunks.
 //
-// Each channel is scanned once, sequentially over all T steps; parallelism comes from
-// channels x state slices.  A lane owns CPL adjacent channels and NS = N / TPC of
-// their state components (TPC lanes per channel); the partial dot products of y are
-// reduced over the TPC lanes with shuffles.  Every warp of a CTA is an independent
-// worker on CPW channels of one sequence with its own STAGES-deep ring of ROWS-step
-// TMA tiles (x, dt, gate of its channels and the full B|C rows), refilled by its own
-// lane 0 as soon as the warp has consumed a tile, and its own double-buffered y tile
-// stored with TMA.  CTAs are four warps, one per SM sub-partition, so the warps of
-// an SM share its issue slots evenly.  Tensor maps are 3-D ([batch][T][cols]): no
-// tile crosses a sequence end, rows past T load as zeros (dt = 0 leaves the state
-// unchanged) and are clipped on store.
+// A lane owns CPL adjacent channels and NS = N / TPC of their state components (TPC
+// lanes per channel); partial dot products are reduced over the TPC lanes with
+// shuffles.  Every warp streams its own STAGES-deep ring of ROWS-step TMA tiles (x, dt,
+// gate of its CPW channels and the full B|C rows), refilled by its own lane 0, and
+// writes y through a double-buffered smem tile and TMA stores.  A CTA holds G channel
+// groups x S time chunks of one sequence (G * S warps).  With S = 1 each warp scans all
+// T steps of its channels once.  With S > 1 the warps of a group take consecutive
+// chunks: pass 1 scans each chunk but the last from h = 0 for its end state only
+// (state update, no output, no gate or C reads); the end states meet in shared
+// memory, where chunk k forms its entry state c_k = D_{k-1} c_{k-1} + h_end_{k-1}
+// (D = the chunk's total decay); pass 2 rescans every chunk from its entry state and
+// emits y.  S is chosen per launch so that the SM sub-partitions have enough warps.
+// Tensor maps are 3-D ([batch][T][cols]): no tile crosses a sequence end, rows past T
+// load as zeros (dt = 0 leaves the state unchanged) and are clipped on store.
 //
 // Scaled state: with P_t = prod exp(A dt_s) since the last rescale and g = h / P,
 // g_t = g_{t-1} + (dt_t x_t / P_t) B_t and y_t = P_t (C_t . g_t).  The output is
-// formed as y_t = P_t (C_t . g_{t-1} + v_t (C_t . B_t)), v_t = dt_t x_t / P_t, so
-// that it reads only the previous state and never waits on this step's update; the
-// row dot product C_t . B_t is shared by all channels and computed once per tile row.
+// formed as y_t = P_t (C_t . g_{t-1} + v_t (C_t . B_t)), v_t = dt_t x_t / P_t, so that it
+// reads only the previous state and never waits on this step's update; the row dot
+// product C_t . B_t is shared by all channels and computed once per tile row.
 // -log2 P is kept per channel (ncl) and folded back into g every block of BLK steps;
 // a block whose decay would take P below 2^-60 runs the per-step path that folds on
 // demand and restarts the state after a single step decaying by more than 2^-60.
@@ -232,21 +235,20 @@ struct WCfg {
   static constexpr int NP = NS / 2;             // packed fp32x2 pairs
   static constexpr int NQ = NS / 4;             // 16-byte chunks of B (and of C) per lane
   static constexpr int CPW = (32 / TPC) * CPL;  // channels per warp
-  static constexpr int WPC = 4;                 // warps per CTA
-  static constexpr int CPB = WPC * CPW;         // channels per CTA
   static constexpr int BLK = NQ * CPL <= 4 ? 16 : 8;  // steps per unrolled block (registers)
-  static constexpr int ROWS = (N == 16 && sizeof(TI) == 2) ? 32 : (N <= 32 ? 16 : 8);  // a multiple of BLK
-  static constexpr int STAGES = (N <= 32 && TPC == 1) ? 4 : 3;
+  static constexpr int ROWS = (N == 16 && sizeof(TI) == 2 && CPL == 1) ? 32 : (N <= 32 ? 16 : 8);
+  static constexpr int STAGES = (N <= 32 && TPC == 1) ? (CPL == 1 ? 4 : 2) : 3;
   static constexpr int LPR = 32 / ROWS;               // lanes per row for C . B
   static constexpr int XB = ROWS * CPW * (int)sizeof(TI);  // one x / dt / gate tile
   static constexpr int BCB = ROWS * 2 * N * 4;              // one B|C tile
   static constexpr int STAGE_B = 3 * XB + BCB;
   static constexpr int YB = ROWS * CPW * (int)sizeof(TI);   // one y tile
   static constexpr int WARP_B = (STAGES * STAGE_B + 2 * YB + STAGES * 8 + 16 + 127) / 128 * 128;
-  static constexpr int SMEM = WPC * WARP_B + 128;
-  static constexpr int THREADS = 32 * WPC;
+  static constexpr int MAX_WARPS = 8;
+  static constexpr int HEND_B = 32 * CPL * (NS + 1) * 4;    // a warp's end state + log-decay
   static_assert(ROWS % BLK == 0 && 32 % ROWS == 0, "tile rows");
-  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  static_assert(HEND_B <= STAGE_B, "the end state is published in ring slot 0");
+  static_assert(4 * WARP_B + 128 <= 227 * 1024, "shared memory per CTA");
 };
 
 // CPL adjacent channels of one row: load from a shared address, store to a pointer.
@@ -276,22 +278,30 @@ template <> struct ChanLd<float, 2> {
   static HY_DEV void st(uint8_t* p, const float (&v)[2]) { *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]); }
 };
 
+struct SplitParams {
+  int S;       // time chunks per channel group (warps per group)
+  int G;       // channel groups per CTA
+  int ctiles;  // tiles per chunk
+};
+
 template <typename TI, int N, int TPC, int CPL>
-__global__ void __launch_bounds__(128) scan_w_kernel(const __grid_constant__ CUtensorMap tmX,
+__global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUtensorMap tmX,
                                                      const __grid_constant__ CUtensorMap tmDT,
                                                      const __grid_constant__ CUtensorMap tmG,
                                                      const __grid_constant__ CUtensorMap tmBC,
                                                      const __grid_constant__ CUtensorMap tmY, const ScanParams p,
-                                                     unsigned* status) {
+                                                     const SplitParams sp, unsigned* status) {
   using C = WCfg<TI, N, TPC, CPL>;
   constexpr int NS = C::NS, NP = C::NP, NQ = C::NQ, CPW = C::CPW;
   constexpr uint32_t es = sizeof(TI);
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
-  const int wcol = (blockIdx.x * C::WPC + warp) * CPW;  // first channel of this warp
-  if (wcol >= p.Di) return;                             // (no CTA-wide synchronisation below)
+  const int grp = warp / sp.S, chunk = warp % sp.S;
+  const int wcol = (blockIdx.x * sp.G + grp) * CPW;  // first channel of this warp
+  const bool active = wcol < p.Di;                   // inactive warps still meet the CTA barriers
   const int n_tiles = (p.T + C::ROWS - 1) / C::ROWS;
+  const int k_begin = min(n_tiles, chunk * sp.ctiles), k_end = min(n_tiles, k_begin + sp.ctiles);
 
   uint8_t* wsm = smem_raw + warp * C::WARP_B;
   const uint32_t ring = smem_u32(wsm);
@@ -305,20 +315,27 @@ __global__ void __launch_bounds__(128) scan_w_kernel(const __grid_constant__ CUt
     fence_mbar_init();
   }
   __syncwarp();
-  int issued = 0;  // meaningful on lane 0
-  auto issue = [&](int t_idx) {  // lane 0: tile t_idx into slot t_idx % STAGES
-    const int slot = t_idx % C::STAGES;
+  // Ring bookkeeping across both passes: the i-th tile this warp issues goes to slot
+  // i % STAGES and completes phase (i / STAGES) & 1 there; tiles are consumed in order.
+  uint32_t issued = 0, consumed = 0;  // (issued is meaningful on lane 0)
+  auto issue = [&](int k, bool with_gate) {  // lane 0: time tile k
+    const int slot = issued % C::STAGES;
     uint8_t* st = wsm + slot * C::STAGE_B;
-    mbar_arrive_expect_tx(&full[slot], C::STAGE_B);
-    const int t = t_idx * C::ROWS;
+    mbar_arrive_expect_tx(&full[slot], (with_gate ? 3 : 2) * C::XB + C::BCB);
+    const int t = k * C::ROWS;
     tma_load_3d(st, &tmX, &full[slot], wcol, t, b);
     tma_load_3d(st + C::XB, &tmDT, &full[slot], wcol, t, b);
-    tma_load_3d(st + 2 * C::XB, &tmG, &full[slot], wcol, t, b);
+    if (with_gate) tma_load_3d(st + 2 * C::XB, &tmG, &full[slot], wcol, t, b);
     tma_load_3d(st + 3 * C::XB, &tmBC, &full[slot], 0, t, b);
     ++issued;
   };
-  if (lane == 0)
-    for (int t_idx = 0; t_idx < C::STAGES && t_idx < n_tiles; ++t_idx) issue(t_idx);
+  bool ok = true;
+  auto wait_tile = [&]() -> bool {
+    const bool r = __all_sync(0xffffffffu, mbar_wait(&full[consumed % C::STAGES], (consumed / C::STAGES) & 1u,
+                                                     status, abort_flag));
+    ++consumed;
+    return r;
+  };
 
   const int cg = lane / TPC, slice = lane % TPC;
   const int ccol = cg * CPL;  // first channel of this lane within the warp
@@ -327,7 +344,7 @@ __global__ void __launch_bounds__(128) scan_w_kernel(const __grid_constant__ CUt
   const int rot = (slice * NS / 32) & (NQ - 1);
   float A2[CPL];  // A in log2 units: exp(A dt) = exp2(A2 dt)
 #pragma unroll
-  for (int q = 0; q < CPL; ++q) A2[q] = c0 + q < p.Di ? -expf(p.a_log[c0 + q]) * 1.4426950408889634f : 0.f;
+  for (int q = 0; q < CPL; ++q) A2[q] = (active && c0 + q < p.Di) ? -expf(p.a_log[c0 + q]) * 1.4426950408889634f : 0.f;
 
   float2 g[CPL][NP];
   float ncl[CPL];  // -log2 of the running scale P
@@ -339,7 +356,10 @@ __global__ void __launch_bounds__(128) scan_w_kernel(const __grid_constant__ CUt
   }
   const bool ywriter = slice == 0;
 
-  // B and C chunks of this lane for one row (rotated chunk order, see above)
+  auto load_b = [&](uint32_t row_addr, float4 (&bq)[NQ]) {
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) bq[j] = lds_f4(row_addr + (n0 + ((j + rot) & (NQ - 1)) * 4) * 4);
+  };
   auto load_bc = [&](uint32_t row_addr, float4 (&bq)[NQ], float4 (&cq)[NQ]) {
 #pragma unroll
     for (int j = 0; j < NQ; ++j) {
@@ -348,8 +368,21 @@ __global__ void __launch_bounds__(128) scan_w_kernel(const __grid_constant__ CUt
       cq[j] = lds_f4(row_addr + N * 4 + off);
     }
   };
-  // one step: y = C_t . g_{t-1} + v_t (C_t . B_t) (the partial dot reduced over the
-  // slices), then g_t = g_{t-1} + v_t B_t.  Both read only the previous state.
+  // g_t = g_{t-1} + v_t B_t
+  auto update = [&](const float4 (&bq)[NQ], const float (&v)[CPL]) {
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      const float2 b01 = make_float2(bq[j].x, bq[j].y), b23 = make_float2(bq[j].z, bq[j].w);
+#pragma unroll
+      for (int q = 0; q < CPL; ++q) {
+        const float2 v2 = make_float2(v[q], v[q]);
+        g[q][2 * j] = __ffma2_rn(v2, b01, g[q][2 * j]);
+        g[q][2 * j + 1] = __ffma2_rn(v2, b23, g[q][2 * j + 1]);
+      }
+    }
+  };
+  // y = C_t . g_{t-1} + v_t (C_t . B_t) (the partial dot reduced over the slices), then
+  // g_t = g_{t-1} + v_t B_t.  Both read only the previous state.
   auto step_core = [&](const float4 (&bq)[NQ], const float4 (&cq)[NQ], const float (&v)[CPL], float cb,
                        float (&y)[CPL]) {
     float2 ya[CPL], yb[CPL];
@@ -360,17 +393,14 @@ __global__ void __launch_bounds__(128) scan_w_kernel(const __grid_constant__ CUt
     }
 #pragma unroll
     for (int j = 0; j < NQ; ++j) {
-      const float2 b01 = make_float2(bq[j].x, bq[j].y), b23 = make_float2(bq[j].z, bq[j].w);
       const float2 c01 = make_float2(cq[j].x, cq[j].y), c23 = make_float2(cq[j].z, cq[j].w);
 #pragma unroll
       for (int q = 0; q < CPL; ++q) {
-        const float2 v2 = make_float2(v[q], v[q]);
         ya[q] = __ffma2_rn(c01, g[q][2 * j], ya[q]);
         yb[q] = __ffma2_rn(c23, g[q][2 * j + 1], yb[q]);
-        g[q][2 * j] = __ffma2_rn(v2, b01, g[q][2 * j]);
-        g[q][2 * j + 1] = __ffma2_rn(v2, b23, g[q][2 * j + 1]);
       }
     }
+    update(bq, v);
 #pragma unroll
     for (int q = 0; q < CPL; ++q) {
       float sum = (ya[q].x + ya[q].y) + (yb[q].x + yb[q].y);
@@ -379,157 +409,281 @@ __global__ void __launch_bounds__(128) scan_w_kernel(const __grid_constant__ CUt
       y[q] = fmaf(v[q], cb, sum);
     }
   };
+  // one step of the per-step (extreme decay) path: fold on demand, restart after a single
+  // step decaying past 2^-60; returns v and keeps ncl
+  auto slow_scalars = [&](const float (&dv)[CPL], const float (&xv)[CPL], float (&vv)[CPL], float (&lsum)[CPL]) {
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) {
+      const float l = -A2[q] * dv[q];  // >= 0
+      lsum[q] += l;
+      float c = ncl[q] + l;
+      if (c > 60.f) {
+        const float Pf = ex2_approx(-ncl[q]);
+        const float2 P2 = make_float2(Pf, Pf);
+#pragma unroll
+        for (int i = 0; i < NP; ++i) g[q][i] = __fmul2_rn(g[q][i], P2);
+        if (l > 60.f) {
+#pragma unroll
+          for (int i = 0; i < NP; ++i) g[q][i] = make_float2(0.f, 0.f);
+          c = 0.f;
+        } else {
+          c = l;
+        }
+      }
+      ncl[q] = c;
+      vv[q] = dv[q] * xv[q] * ex2_approx(c);
+    }
+  };
+  auto fold = [&]() {
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) {
+      const float P = ex2_approx(-ncl[q]);
+      const float2 P2 = make_float2(P, P);
+#pragma unroll
+      for (int i = 0; i < NP; ++i) g[q][i] = __fmul2_rn(g[q][i], P2);
+      ncl[q] = 0.f;
+    }
+  };
   // B|C rows are prefetched one step ahead when the registers allow it
   constexpr bool kPrefetch = NQ * CPL <= 4;
 
-  bool ok = true;
-  int k = 0;
-  for (; k < n_tiles; ++k) {
-    const int slot = k % C::STAGES;
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], (k / C::STAGES) & 1, status, abort_flag))) {
-      ok = false;
-      break;
-    }
-    const uint32_t tile = ring + slot * C::STAGE_B;
-    const uint32_t tx = tile + ccol * es;
-    const uint32_t td = tile + C::XB + ccol * es;
-    const uint32_t tg = tile + 2 * C::XB + ccol * es;
-    const uint32_t tbc = tile + 3 * C::XB;
-    uint8_t* yt = ybuf + (k & 1) * C::YB;  // this warp's y tile [ROWS][CPW]
-    if (lane == 0) bulk_wait_read1();      // the store of tile k-2 has read this buffer
-    __syncwarp();
-
-    // C_t . B_t of the tile's rows: LPR lanes per row, chunks rotated by row (banks)
-    float cb_row;
-    {
-      constexpr int CPP = (N / 4) / C::LPR;  // 16-byte chunks per lane
-      const int row = lane / C::LPR, part = lane % C::LPR;
-      const uint32_t ra = tbc + row * 2 * N * 4;
-      float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+  // ======================== pass 1: end state of this chunk (every chunk but the last)
+  float ltot[CPL];  // the chunk's total decay, -log2 D
 #pragma unroll
-      for (int j = 0; j < CPP; ++j) {
-        const uint32_t off = (part * CPP + ((j + row) & (CPP - 1))) * 16;
-        const float4 bb = lds_f4(ra + off), cc = lds_f4(ra + N * 4 + off);
-        a0 = __ffma2_rn(make_float2(bb.x, bb.y), make_float2(cc.x, cc.y), a0);
-        a1 = __ffma2_rn(make_float2(bb.z, bb.w), make_float2(cc.z, cc.w), a1);
+  for (int q = 0; q < CPL; ++q) ltot[q] = 0.f;
+  const bool pass1 = active && sp.S > 1 && chunk < sp.S - 1;
+  if (pass1) {
+    if (lane == 0)
+      for (int k = k_begin; k < k_end && k < k_begin + C::STAGES; ++k) issue(k, false);
+    for (int k = k_begin; k < k_end; ++k) {
+      if (!wait_tile()) {
+        ok = false;
+        break;
       }
-      cb_row = (a0.x + a0.y) + (a1.x + a1.y);
-#pragma unroll
-      for (int off = 1; off < C::LPR; off <<= 1) cb_row += __shfl_xor_sync(0xffffffffu, cb_row, off);
-    }
-
-    // blocks of BLK steps: fold the scale into g, then either the unrolled fast block
-    // (every scalar of the block's steps first -- loads, decay chain, SFU -- then the
-    // state chain with B|C prefetched one step ahead) or, when some channel's decay
-    // over the block passes 2^-60, the per-step path.
+      const uint32_t tile = ring + ((consumed - 1) % C::STAGES) * C::STAGE_B;
+      const uint32_t tx = tile + ccol * es, td = tile + C::XB + ccol * es, tbc = tile + 3 * C::XB;
 #pragma unroll 1
-    for (int r0 = 0; r0 < C::ROWS; r0 += C::BLK) {
+      for (int r0 = 0; r0 < C::ROWS; r0 += C::BLK) {
+        fold();
+        float v[C::BLK][CPL];
+        bool fast = true;
+        {
+          float nc[CPL];
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) nc[q] = 0.f;
+#pragma unroll
+          for (int s = 0; s < C::BLK; ++s) {
+            float dv[CPL], xv[CPL];
+            const uint32_t ro = (r0 + s) * CPW * es;
+            ChanLd<TI, CPL>::ld(td + ro, dv);
+            ChanLd<TI, CPL>::ld(tx + ro, xv);
+#pragma unroll
+            for (int q = 0; q < CPL; ++q) {
+              nc[q] = fmaf(-A2[q], dv[q], nc[q]);
+              v[s][q] = dv[q] * xv[q] * ex2_approx(nc[q]);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) {
+            fast = fast && nc[q] <= 60.f;
+            ncl[q] = nc[q];
+          }
+        }
+        if (__all_sync(0xffffffffu, fast)) {
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) ltot[q] += ncl[q];
+          float4 bq[2][NQ];
+          load_b(tbc + r0 * 2 * N * 4, bq[0]);
+#pragma unroll
+          for (int s = 0; s < C::BLK; ++s) {
+            if (s + 1 < C::BLK) load_b(tbc + (r0 + s + 1) * 2 * N * 4, bq[(s + 1) & 1]);
+            update(bq[s & 1], v[s]);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) ncl[q] = 0.f;
+#pragma unroll 1
+          for (int s = 0; s < C::BLK; ++s) {
+            float dv[CPL], xv[CPL], vv[CPL];
+            const uint32_t ro = (r0 + s) * CPW * es;
+            ChanLd<TI, CPL>::ld(td + ro, dv);
+            ChanLd<TI, CPL>::ld(tx + ro, xv);
+            slow_scalars(dv, xv, vv, ltot);
+            float4 bq[NQ];
+            load_b(tbc + (r0 + s) * 2 * N * 4, bq);
+            update(bq, vv);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && k + C::STAGES < k_end) issue(k + C::STAGES, false);
+    }
+  }
+  // ======================== combine: entry state of every chunk
+  if (sp.S > 1) {
+    // the end state h = P g and -log2 D, published in ring slot 0 (no copy in flight now)
+    float* pub = reinterpret_cast<float*>(wsm) + lane * CPL * (NS + 1);
+    if (pass1) {
 #pragma unroll
       for (int q = 0; q < CPL; ++q) {
         const float P = ex2_approx(-ncl[q]);
-        const float2 P2 = make_float2(P, P);
 #pragma unroll
-        for (int i = 0; i < NP; ++i) g[q][i] = __fmul2_rn(g[q][i], P2);
-        ncl[q] = 0.f;
-      }
-      float v[C::BLK][CPL], P[C::BLK][CPL], gv[C::BLK][CPL];
-      bool fast = true;
-      {
-        float nc[CPL];
-#pragma unroll
-        for (int q = 0; q < CPL; ++q) nc[q] = 0.f;
-#pragma unroll
-        for (int s = 0; s < C::BLK; ++s) {
-          float dv[CPL], xv[CPL];
-          const uint32_t ro = (r0 + s) * CPW * es;
-          ChanLd<TI, CPL>::ld(td + ro, dv);
-          ChanLd<TI, CPL>::ld(tx + ro, xv);
-          ChanLd<TI, CPL>::ld(tg + ro, gv[s]);
-#pragma unroll
-          for (int q = 0; q < CPL; ++q) {
-            nc[q] = fmaf(-A2[q], dv[q], nc[q]);
-            v[s][q] = dv[q] * xv[q] * ex2_approx(nc[q]);
-            P[s][q] = ex2_approx(-nc[q]);
-          }
+        for (int i = 0; i < NP; ++i) {
+          pub[q * (NS + 1) + 2 * i] = g[q][i].x * P;
+          pub[q * (NS + 1) + 2 * i + 1] = g[q][i].y * P;
         }
-#pragma unroll
-        for (int q = 0; q < CPL; ++q) {
-          fast = fast && nc[q] <= 60.f;
-          ncl[q] = nc[q];
-        }
-      }
-      if (__all_sync(0xffffffffu, fast)) {
-        float4 bq[2][NQ], cq[2][NQ];
-        if (kPrefetch) load_bc(tbc + r0 * 2 * N * 4, bq[0], cq[0]);
-#pragma unroll
-        for (int s = 0; s < C::BLK; ++s) {
-          float y[CPL], o[CPL];
-          if (kPrefetch) {
-            if (s + 1 < C::BLK) load_bc(tbc + (r0 + s + 1) * 2 * N * 4, bq[(s + 1) & 1], cq[(s + 1) & 1]);
-          } else {
-            load_bc(tbc + (r0 + s) * 2 * N * 4, bq[s & 1], cq[s & 1]);
-          }
-          const float cb = __shfl_sync(0xffffffffu, cb_row, (r0 + s) * C::LPR);
-          step_core(bq[s & 1], cq[s & 1], v[s], cb, y);
-#pragma unroll
-          for (int q = 0; q < CPL; ++q) o[q] = gv[s][q] * P[s][q] * y[q];
-          if (ywriter) ChanLd<TI, CPL>::st(yt + ((r0 + s) * CPW + ccol) * es, o);
-        }
-      } else {
-        // per-step path: fold on demand, restart after a single step decaying past 2^-60
-#pragma unroll
-        for (int q = 0; q < CPL; ++q) ncl[q] = 0.f;
-#pragma unroll 1
-        for (int s = 0; s < C::BLK; ++s) {
-          float dv[CPL], xv[CPL], gt[CPL], vv[CPL], y[CPL], o[CPL];
-          const uint32_t ro = (r0 + s) * CPW * es;
-          ChanLd<TI, CPL>::ld(td + ro, dv);
-          ChanLd<TI, CPL>::ld(tx + ro, xv);
-          ChanLd<TI, CPL>::ld(tg + ro, gt);
-#pragma unroll
-          for (int q = 0; q < CPL; ++q) {
-            const float l = -A2[q] * dv[q];  // >= 0
-            float c = ncl[q] + l;
-            if (c > 60.f) {
-              const float Pf = ex2_approx(-ncl[q]);
-              const float2 P2 = make_float2(Pf, Pf);
-#pragma unroll
-              for (int i = 0; i < NP; ++i) g[q][i] = __fmul2_rn(g[q][i], P2);
-              if (l > 60.f) {
-#pragma unroll
-                for (int i = 0; i < NP; ++i) g[q][i] = make_float2(0.f, 0.f);
-                c = 0.f;
-              } else {
-                c = l;
-              }
-            }
-            ncl[q] = c;
-            vv[q] = dv[q] * xv[q] * ex2_approx(c);
-          }
-          float4 bq[NQ], cq[NQ];
-          load_bc(tbc + (r0 + s) * 2 * N * 4, bq, cq);
-          const float cb = __shfl_sync(0xffffffffu, cb_row, (r0 + s) * C::LPR);
-          step_core(bq, cq, vv, cb, y);
-#pragma unroll
-          for (int q = 0; q < CPL; ++q) o[q] = gt[q] * ex2_approx(-ncl[q]) * y[q];
-          if (ywriter) ChanLd<TI, CPL>::st(yt + ((r0 + s) * CPW + ccol) * es, o);
-        }
+        pub[q * (NS + 1) + NS] = ltot[q];
       }
     }
-    // every lane is done with the slot and the y tile: refill the slot, store y
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      if (k + C::STAGES < n_tiles) issue(k + C::STAGES);
-      tma_store_3d(&tmY, yt, wcol, k * C::ROWS, b);
-      bulk_commit();
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) {
+#pragma unroll
+      for (int i = 0; i < NP; ++i) g[q][i] = make_float2(0.f, 0.f);
+      ncl[q] = 0.f;
+    }
+    for (int j = 0; j < chunk; ++j) {  // c_{j+1} = D_j c_j + h_end_j
+      const float* src = reinterpret_cast<const float*>(smem_raw + (grp * sp.S + j) * C::WARP_B) +
+                         lane * CPL * (NS + 1);
+#pragma unroll
+      for (int q = 0; q < CPL; ++q) {
+        const float D = ex2_approx(-src[q * (NS + 1) + NS]);
+        const float2 D2 = make_float2(D, D);
+#pragma unroll
+        for (int i = 0; i < NP; ++i)
+          g[q][i] = __ffma2_rn(D2, g[q][i], make_float2(src[q * (NS + 1) + 2 * i], src[q * (NS + 1) + 2 * i + 1]));
+      }
+    }
+    fence_proxy_async_smem();  // the published values are read before copies overwrite slot 0
+    __syncthreads();
+  }
+
+  // ======================== pass 2: scan the chunk from its entry state, emit y
+  if (active && ok) {
+    if (lane == 0)
+      for (int k = k_begin; k < k_end && k < k_begin + C::STAGES; ++k) issue(k, true);
+    for (int k = k_begin; k < k_end; ++k) {
+      if (!wait_tile()) {
+        ok = false;
+        break;
+      }
+      const int slot = (consumed - 1) % C::STAGES;
+      const uint32_t tile = ring + slot * C::STAGE_B;
+      const uint32_t tx = tile + ccol * es;
+      const uint32_t td = tile + C::XB + ccol * es;
+      const uint32_t tg = tile + 2 * C::XB + ccol * es;
+      const uint32_t tbc = tile + 3 * C::XB;
+      uint8_t* yt = ybuf + (k & 1) * C::YB;  // this warp's y tile [ROWS][CPW]
+      if (lane == 0) bulk_wait_read1();      // the store of tile k-2 has read this buffer
+      __syncwarp();
+
+      // C_t . B_t of the tile's rows: LPR lanes per row, chunks rotated by row (banks)
+      float cb_row;
+      {
+        constexpr int CPP = (N / 4) / C::LPR;  // 16-byte chunks per lane
+        const int row = lane / C::LPR, part = lane % C::LPR;
+        const uint32_t ra = tbc + row * 2 * N * 4;
+        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < CPP; ++j) {
+          const uint32_t off = (part * CPP + ((j + row) & (CPP - 1))) * 16;
+          const float4 bb = lds_f4(ra + off), cc = lds_f4(ra + N * 4 + off);
+          a0 = __ffma2_rn(make_float2(bb.x, bb.y), make_float2(cc.x, cc.y), a0);
+          a1 = __ffma2_rn(make_float2(bb.z, bb.w), make_float2(cc.z, cc.w), a1);
+        }
+        cb_row = (a0.x + a0.y) + (a1.x + a1.y);
+#pragma unroll
+        for (int off = 1; off < C::LPR; off <<= 1) cb_row += __shfl_xor_sync(0xffffffffu, cb_row, off);
+      }
+
+      // blocks of BLK steps: fold the scale into g, then either the unrolled fast block
+      // (every scalar of the block's steps first -- loads, decay chain, SFU -- then the
+      // state chain with B|C prefetched one step ahead) or, when some channel's decay
+      // over the block passes 2^-60, the per-step path.
+#pragma unroll 1
+      for (int r0 = 0; r0 < C::ROWS; r0 += C::BLK) {
+        fold();
+        float v[C::BLK][CPL], P[C::BLK][CPL], gv[C::BLK][CPL];
+        bool fast = true;
+        {
+          float nc[CPL];
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) nc[q] = 0.f;
+#pragma unroll
+          for (int s = 0; s < C::BLK; ++s) {
+            float dv[CPL], xv[CPL];
+            const uint32_t ro = (r0 + s) * CPW * es;
+            ChanLd<TI, CPL>::ld(td + ro, dv);
+            ChanLd<TI, CPL>::ld(tx + ro, xv);
+            ChanLd<TI, CPL>::ld(tg + ro, gv[s]);
+#pragma unroll
+            for (int q = 0; q < CPL; ++q) {
+              nc[q] = fmaf(-A2[q], dv[q], nc[q]);
+              v[s][q] = dv[q] * xv[q] * ex2_approx(nc[q]);
+              P[s][q] = ex2_approx(-nc[q]);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) {
+            fast = fast && nc[q] <= 60.f;
+            ncl[q] = nc[q];
+          }
+        }
+        if (__all_sync(0xffffffffu, fast)) {
+          float4 bq[2][NQ], cq[2][NQ];
+          if (kPrefetch) load_bc(tbc + r0 * 2 * N * 4, bq[0], cq[0]);
+#pragma unroll
+          for (int s = 0; s < C::BLK; ++s) {
+            float y[CPL], o[CPL];
+            if (kPrefetch) {
+              if (s + 1 < C::BLK) load_bc(tbc + (r0 + s + 1) * 2 * N * 4, bq[(s + 1) & 1], cq[(s + 1) & 1]);
+            } else {
+              load_bc(tbc + (r0 + s) * 2 * N * 4, bq[s & 1], cq[s & 1]);
+            }
+            const float cb = __shfl_sync(0xffffffffu, cb_row, (r0 + s) * C::LPR);
+            step_core(bq[s & 1], cq[s & 1], v[s], cb, y);
+#pragma unroll
+            for (int q = 0; q < CPL; ++q) o[q] = gv[s][q] * P[s][q] * y[q];
+            if (ywriter) ChanLd<TI, CPL>::st(yt + ((r0 + s) * CPW + ccol) * es, o);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) ncl[q] = 0.f;
+          float unused[CPL];
+#pragma unroll 1
+          for (int s = 0; s < C::BLK; ++s) {
+            float dv[CPL], xv[CPL], gt[CPL], vv[CPL], y[CPL], o[CPL];
+            const uint32_t ro = (r0 + s) * CPW * es;
+            ChanLd<TI, CPL>::ld(td + ro, dv);
+            ChanLd<TI, CPL>::ld(tx + ro, xv);
+            ChanLd<TI, CPL>::ld(tg + ro, gt);
+            slow_scalars(dv, xv, vv, unused);
+            float4 bq[NQ], cq[NQ];
+            load_bc(tbc + (r0 + s) * 2 * N * 4, bq, cq);
+            const float cb = __shfl_sync(0xffffffffu, cb_row, (r0 + s) * C::LPR);
+            step_core(bq, cq, vv, cb, y);
+#pragma unroll
+            for (int q = 0; q < CPL; ++q) o[q] = gt[q] * ex2_approx(-ncl[q]) * y[q];
+            if (ywriter) ChanLd<TI, CPL>::st(yt + ((r0 + s) * CPW + ccol) * es, o);
+          }
+        }
+      }
+      // every lane is done with the slot and the y tile: refill the slot, store y
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (k + C::STAGES < k_end) issue(k + C::STAGES, true);
+        tma_store_3d(&tmY, yt, wcol, k * C::ROWS, b);
+        bulk_commit();
+      }
     }
   }
   if (lane == 0) {
     bulk_wait_all();
     if (!ok) {  // let the copies this warp issued but did not consume land before it exits
       int never = 0;
-      for (int j = k; j < issued; ++j)
+      for (uint32_t j = consumed; j < issued; ++j)
         mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1u, nullptr, &never, 100000000ull);
     }
   }
@@ -578,18 +732,38 @@ cudaError_t launch_w(const ScanDesc& s, cudaStream_t st) {
       !map3d(&tb, s.bc, true, s.batch, s.T, 2 * N, 2 * N, 2 * N, C::ROWS) ||
       !map3d(&ty, s.y, f32, s.batch, s.T, s.d_inner, s.y_ld, C::CPW, C::ROWS))
     return cudaErrorInvalidValue;
+  const int groups = (s.d_inner + C::CPW - 1) / C::CPW;
+  const int n_tiles = (s.T + C::ROWS - 1) / C::ROWS;
+  const int max_warps = (227 * 1024 - 128) / C::WARP_B < C::MAX_WARPS ? (227 * 1024 - 128) / C::WARP_B : C::MAX_WARPS;
   static int attr_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 31 && !(attr_mask & (1 << dev))) {
-    cudaError_t e =
-        cudaFuncSetAttribute(scan_w_kernel<TI, N, TPC, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(scan_w_kernel<TI, N, TPC, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         max_warps * C::WARP_B + 128);
     if (e != cudaSuccess) return e;
     attr_mask |= 1 << dev;
   }
+  // Time chunks S: the smallest split that gives about two warps per SM sub-partition,
+  // else the largest whose grid still fits in one wave; chunks of at least 8 tiles.
+  SplitParams sp{1, 4, n_tiles};
+  for (int S = 1; S <= C::MAX_WARPS; S *= 2) {
+    const int G = S >= 4 ? 1 : 4 / S, warps = G * S;
+    if (warps > max_warps || (S > 1 && n_tiles < 8 * S)) break;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_w_kernel<TI, N, TPC, CPL>, 32 * warps,
+                                                      warps * C::WARP_B + 128) != cudaSuccess)
+      per_sm = 0;
+    const long long ctas = static_cast<long long>((groups + G - 1) / G) * s.batch;
+    if (S > 1 && ctas > static_cast<long long>(per_sm) * num_sms()) break;
+    sp = SplitParams{S, G, (n_tiles + S - 1) / S};
+    if (ctas * warps >= 2LL * 4 * num_sms()) break;
+  }
+  const int warps = sp.G * sp.S;
+  const int smem = warps * C::WARP_B + 128;
   ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
-  dim3 grid((s.d_inner + C::CPB - 1) / C::CPB, s.batch);
-  scan_w_kernel<TI, N, TPC, CPL><<<grid, C::THREADS, C::SMEM, st>>>(tx, td, tg, tb, ty, p, s.status);
+  dim3 grid((groups + sp.G - 1) / sp.G, s.batch);
+  scan_w_kernel<TI, N, TPC, CPL><<<grid, 32 * warps, smem, st>>>(tx, td, tg, tb, ty, p, sp, s.status);
   return cudaGetLastError();
 }
 
