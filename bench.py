@@ -277,24 +277,60 @@ def run_reference(args, rank, world):
     return 0
 
 
+# --------------------------------------------------------------------------- multi-process plumbing
+
+class Ranks:
+    """One process per GPU: the process group, its barrier and the max over ranks.
+    World 1 needs no process group; the data path has no collective (each rank runs
+    its own batch), so the only cross-rank traffic is timing."""
+
+    def __init__(self, world: int, local_rank: int, backend: str, device, timeout_s: float = 180.0):
+        import torch.distributed as dist
+        self.world, self.local_rank, self.backend, self.device = world, local_rank, backend, device
+        self.dist = dist
+        if world > 1:
+            from datetime import timedelta
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            if self.backend == "nccl":
+                self.dist.barrier(device_ids=[self.local_rank])
+            else:
+                self.dist.barrier()
+
+    def max(self, value: float) -> float:
+        """The largest value over the ranks (every rank gets it)."""
+        if self.world == 1:
+            return float(value)
+        import torch
+        t = torch.tensor([float(value)], device=self.device, dtype=torch.float64)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+def weak_scaling_rate(world: int, steps: int, units_per_step_per_rank: float, max_total_ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * steps * units_per_step_per_rank / (max_total_ms * 1e-3)
+
+
 # --------------------------------------------------------------------------- native (CUDA) leg
 
 def run_native(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
 
     import hybrid_attention_ssm_hymba_b200 as H
     from hybrid_attention_ssm_hymba_b200 import host
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local_rank])
+    ranks = Ranks(world, local_rank, "nccl", dev)
+    barrier = ranks.barrier
 
     wl = synth.workload(args.workload)
     s0 = wl.first
@@ -359,14 +395,10 @@ def run_native(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
     barrier()
     step_ms = [ev_s[k].elapsed_time(ev_e[k]) for k in range(K)]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = ranks.max(float(sum(step_ms)))
     status = H.hymba_workspace_status(ws, stream)
     tokens_per_step = s0.batch * s0.seq_len
-    value = world * K * tokens_per_step / (total_ms * 1e-3)
+    value = weak_scaling_rate(world, K, tokens_per_step, total_ms)
 
     peaks, peak_src = _peaks()
     roofline, stages, stage_roof, layer_roof = None, None, None, None
@@ -406,12 +438,8 @@ def run_native(args, rank, world, local_rank):
             ee[k].record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e_ms = float(sum(es[k].elapsed_time(ee[k]) for k in range(1, n_e2e + 1)))
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * n_e2e * tokens_per_step / (e_ms * 1e-3), "unit": UNIT,
+        e_ms = ranks.max(float(sum(es[k].elapsed_time(ee[k]) for k in range(1, n_e2e + 1))))
+        e2e = {"value": weak_scaling_rate(world, n_e2e, tokens_per_step, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": xh.numel() * xh.element_size(),
                "d2h_bytes_per_step": oh.numel() * oh.element_size(), "steps": n_e2e,
                "path": "pinned host x -> device, hymba_layer_fwd, device out -> pinned host"}
@@ -432,8 +460,7 @@ def run_native(args, rank, world, local_rank):
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, x_np, meta_np, ps_np)
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
