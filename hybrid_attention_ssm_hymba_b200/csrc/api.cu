@@ -16,6 +16,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "hy_common.cuh"
 #include "hy_kernels.h"
 #include "hymba.h"
 
@@ -290,6 +291,8 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
 // h[b] = [meta; x[b]] (stack input), vectorised 16-byte copy.
 __global__ void prepend_kernel(const uint4* __restrict__ x, const uint4* __restrict__ meta, uint4* __restrict__ h,
                                long long row_vecs, int L, int M, long long total) {
+  hy::pdl_trigger();
+  hy::pdl_wait();
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long row = i / row_vecs, e = i - row * row_vecs;
@@ -466,9 +469,10 @@ hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weig
     const long long total = rows * row_vecs;
     if (c0.d_model * es % 16) return HYMBA_ERR_UNSUPPORTED;
     const int blocks = static_cast<int>(total / 256 + 1 < 4096 ? total / 256 + 1 : 4096);
-    prepend_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(x), static_cast<const uint4*>(meta),
-                                           static_cast<uint4*>(out), row_vecs, c0.seq_len, c0.n_meta, total);
-    if (cudaGetLastError() != cudaSuccess) return HYMBA_ERR_CUDA;
+    if (hy::launch(prepend_kernel, dim3(blocks), dim3(256), 0, st, static_cast<const uint4*>(x),
+                   static_cast<const uint4*>(meta), static_cast<uint4*>(out), row_vecs, c0.seq_len, c0.n_meta,
+                   total) != cudaSuccess)
+      return HYMBA_ERR_CUDA;
   }
   for (int i = 0; i < n_layers; ++i) {
     const hymba_cfg_t& c = cfgs[i];

@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = p.q_tiles - 1 - static_cast<int>(blockIdx.x);  // longest tiles first
   const int h = blockIdx.y, b = blockIdx.z;
@@ -368,6 +370,8 @@ __global__ void __launch_bounds__(320, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = p.q_tiles - 1 - static_cast<int>(blockIdx.x);  // longest tiles first
   const int h0 = 2 * blockIdx.y, b = blockIdx.z;                // heads h0, h0 + 1
@@ -666,12 +670,10 @@ cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st) {
       attr2_mask |= 1 << dev;
     }
     dim3 grid(p.q_tiles, a.n_q_heads / 2, a.batch);
-    attn_fwd_tc2<<<grid, 320, SMEM2_BYTES, st>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    return launch(attn_fwd_tc2, grid, dim3(320), SMEM2_BYTES, st, tq, tk, tv, p);
   }
   dim3 grid(p.q_tiles, a.n_q_heads, a.batch);
-  attn_fwd_tc<<<grid, 192, SMEM_BYTES, st>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  return launch(attn_fwd_tc, grid, dim3(192), SMEM_BYTES, st, tq, tk, tv, p);
 }
 
 }  // namespace hy

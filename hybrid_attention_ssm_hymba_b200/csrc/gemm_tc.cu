@@ -156,6 +156,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_trigger();
+  pdl_wait();  // barriers and TMEM are set up; from here on global memory is touched
   for (int i = threadIdx.x; i < p.bias_len; i += blockDim.x) s_bias[i] = p.bias_src[i];
   if (threadIdx.x == 0) {
     tma_prefetch(&tmA);
@@ -544,8 +546,8 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
   const long long total = static_cast<long long>(p.meta_mode ? p.batch : 1) * p.m_tiles * p.n_tiles;
   if (total <= 0) return cudaSuccess;
   const int grid = static_cast<int>(total < num_sms() ? total : num_sms());
-  gemm_bf16_tc<BN><<<grid, NTHREADS, C::SMEM + p.bias_len * 4, st>>>(tmA, tmAx2, tmM1, tmM2, tmB, p);
-  return cudaGetLastError();
+  return launch(gemm_bf16_tc<BN>, dim3(grid), dim3(NTHREADS), C::SMEM + p.bias_len * 4, st, tmA, tmAx2, tmM1, tmM2,
+                tmB, p);
 }
 
 }  // namespace

@@ -101,6 +101,16 @@ HY_DEV uint32_t lds_u16(uint32_t a) {
   return v;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Kernels are launched with programmatic stream serialization (hy::launch): the next
+// kernel of the stream may be scheduled while this one still runs.  Every kernel calls
+// pdl_wait() after its on-chip setup and before its first access to global memory
+// (it returns once the preceding kernel has completed and its writes are visible), and
+// pdl_trigger() at its start, which lets the next kernel be scheduled once every CTA of
+// this one is resident (so a waiting dependent never holds an SM this kernel needs).
+HY_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+HY_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ fences
 HY_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 HY_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }

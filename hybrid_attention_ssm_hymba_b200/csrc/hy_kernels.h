@@ -8,6 +8,22 @@
 
 namespace hy {
 
+// Launch with programmatic stream serialization (see pdl_wait in hy_common.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // One column segment of a GEMM output: columns [col0, col1) of the product go to
 // ptr + row * ld + (col - col0), optionally through an elementwise op.
 enum SegOp : int { SEG_STORE = 0, SEG_SILU = 1, SEG_SOFTPLUS_BIAS = 2 };

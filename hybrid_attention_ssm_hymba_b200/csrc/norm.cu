@@ -99,6 +99,8 @@ __device__ __forceinline__ void scale_row(const T* src, T* dst, int w, float r, 
 template <typename T>
 __global__ void __launch_bounds__(NT) branch_norm_kernel(T* z, const float* __restrict__ beta1,
                                                          const float* __restrict__ beta2, int wa, int ws, float eps) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[NT / 32 + 1];
   T* row = z + static_cast<long long>(blockIdx.x) * (wa + ws);
   const float sa = block_sum(sumsq(row, wa), red);
@@ -110,6 +112,8 @@ __global__ void __launch_bounds__(NT) branch_norm_kernel(T* z, const float* __re
 
 template <typename T>
 __global__ void __launch_bounds__(NT) rmsnorm_kernel(const T* x, T* y, int d, float eps) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[NT / 32 + 1];
   const long long off = static_cast<long long>(blockIdx.x) * d;
   const float s = block_sum(sumsq(x + off, d), red);
@@ -125,6 +129,8 @@ __global__ void __launch_bounds__(256) rownorm_warp_kernel(const __nv_bfloat16* 
                                                            __nv_bfloat16* y, long long rows, int wa,
                                                            int ws, const float* __restrict__ beta1,
                                                            const float* __restrict__ beta2, float eps) {
+  pdl_trigger();
+  pdl_wait();
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -184,8 +190,8 @@ __global__ void __launch_bounds__(256) rownorm_warp_kernel(const __nv_bfloat16* 
 template <int MAXV>
 void launch_rownorm(const void* x, void* y, long long rows, int wa, int ws, const float* b1, const float* b2,
                     float eps, cudaStream_t st) {
-  rownorm_warp_kernel<MAXV><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), rows, wa, ws, b1, b2, eps);
+  launch(rownorm_warp_kernel<MAXV>, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, st,
+         static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), rows, wa, ws, b1, b2, eps);
 }
 
 // picks the smallest register footprint that holds a row; false if the row is too wide
@@ -208,6 +214,8 @@ bool rownorm_bf16(const void* x, void* y, long long rows, int wa, int ws, const 
 template <int MAXV>
 __global__ void __launch_bounds__(256) row_ssq_kernel(const __nv_bfloat16* __restrict__ z, long long rows, int wa,
                                                       int ws, float2* __restrict__ ssq) {
+  pdl_trigger();
+  pdl_wait();
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -243,6 +251,8 @@ __global__ void __launch_bounds__(256) scale_cols_kernel(const uint4* __restrict
                                                          long long n_vec, int row_vecs, int wa,
                                                          const float* __restrict__ beta1,
                                                          const float* __restrict__ beta2) {
+  pdl_trigger();
+  pdl_wait();
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n_vec;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int k0 = static_cast<int>(i % row_vecs) * 8;
@@ -261,11 +271,11 @@ cudaError_t launch_row_ssq(const void* z, long long rows, int w_attn, int w_ssm,
   const int per_lane = ((w_attn + w_ssm) / 8 + 31) / 32;
   const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
   const __nv_bfloat16* zz = static_cast<const __nv_bfloat16*>(z);
-  if (per_lane <= 4) row_ssq_kernel<4><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
-  else if (per_lane <= 8) row_ssq_kernel<8><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
-  else if (per_lane <= 12) row_ssq_kernel<12><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
-  else if (per_lane <= 16) row_ssq_kernel<16><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
-  else if (per_lane <= 24) row_ssq_kernel<24><<<grid, 256, 0, st>>>(zz, rows, w_attn, w_ssm, ssq);
+  if (per_lane <= 4) launch(row_ssq_kernel<4>, dim3(grid), dim3(256), 0, st, zz, rows, w_attn, w_ssm, ssq);
+  else if (per_lane <= 8) launch(row_ssq_kernel<8>, dim3(grid), dim3(256), 0, st, zz, rows, w_attn, w_ssm, ssq);
+  else if (per_lane <= 12) launch(row_ssq_kernel<12>, dim3(grid), dim3(256), 0, st, zz, rows, w_attn, w_ssm, ssq);
+  else if (per_lane <= 16) launch(row_ssq_kernel<16>, dim3(grid), dim3(256), 0, st, zz, rows, w_attn, w_ssm, ssq);
+  else if (per_lane <= 24) launch(row_ssq_kernel<24>, dim3(grid), dim3(256), 0, st, zz, rows, w_attn, w_ssm, ssq);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
@@ -276,9 +286,9 @@ cudaError_t launch_scale_cols(const void* w, void* w_out, int N, int w_attn, int
   const long long n_vec = static_cast<long long>(N) * row_vecs;
   if (n_vec <= 0) return cudaSuccess;
   const long long blocks = (n_vec + 255) / 256;
-  scale_cols_kernel<<<static_cast<unsigned>(blocks < 4 * num_sms() ? blocks : 4 * num_sms()), 256, 0, st>>>(
-      static_cast<const uint4*>(w), static_cast<uint4*>(w_out), n_vec, row_vecs, w_attn, beta1, beta2);
-  return cudaGetLastError();
+  return launch(scale_cols_kernel, dim3(static_cast<unsigned>(blocks < 4 * num_sms() ? blocks : 4 * num_sms())),
+                dim3(256), 0, st, static_cast<const uint4*>(w), static_cast<uint4*>(w_out), n_vec, row_vecs, w_attn,
+                beta1, beta2);
 }
 
 cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, long long rows, int w_attn, int w_ssm,
@@ -286,24 +296,20 @@ cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, 
   if (rows <= 0) return cudaSuccess;
   if (bf16 && rownorm_bf16(z, z, rows, w_attn, w_ssm, beta1, beta2, eps, st)) return cudaGetLastError();
   if (bf16)
-    branch_norm_kernel<__nv_bfloat16><<<static_cast<unsigned>(rows), NT, 0, st>>>(
-        static_cast<__nv_bfloat16*>(z), beta1, beta2, w_attn, w_ssm, eps);
-  else
-    branch_norm_kernel<float><<<static_cast<unsigned>(rows), NT, 0, st>>>(static_cast<float*>(z), beta1, beta2,
-                                                                           w_attn, w_ssm, eps);
-  return cudaGetLastError();
+    return launch(branch_norm_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(rows)), dim3(NT), 0, st,
+                  static_cast<__nv_bfloat16*>(z), beta1, beta2, w_attn, w_ssm, eps);
+  return launch(branch_norm_kernel<float>, dim3(static_cast<unsigned>(rows)), dim3(NT), 0, st, static_cast<float*>(z),
+                beta1, beta2, w_attn, w_ssm, eps);
 }
 
 cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float eps, bool bf16, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   if (bf16 && rownorm_bf16(x, y, rows, 0, d, nullptr, nullptr, eps, st)) return cudaGetLastError();
   if (bf16)
-    rmsnorm_kernel<__nv_bfloat16><<<static_cast<unsigned>(rows), NT, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), d, eps);
-  else
-    rmsnorm_kernel<float><<<static_cast<unsigned>(rows), NT, 0, st>>>(static_cast<const float*>(x),
-                                                                       static_cast<float*>(y), d, eps);
-  return cudaGetLastError();
+    return launch(rmsnorm_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(rows)), dim3(NT), 0, st,
+                  static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), d, eps);
+  return launch(rmsnorm_kernel<float>, dim3(static_cast<unsigned>(rows)), dim3(NT), 0, st,
+                static_cast<const float*>(x), static_cast<float*>(y), d, eps);
 }
 
 }  // namespace hy

@@ -47,6 +47,8 @@ struct ScanParams {
 
 template <typename TI, int NS, int TPC, int NWT>
 __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int CPW = 32 / TPC;  // channels per warp (= per CTA)
   constexpr int N = NS * TPC;
   constexpr int NP = NS / 2;     // state pairs per thread (packed fp32x2 updates)
@@ -295,6 +297,8 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
   constexpr int NS = C::NS, NP = C::NP, NQ = C::NQ, CPW = C::CPW;
   constexpr uint32_t es = sizeof(TI);
   extern __shared__ __align__(128) uint8_t smem_raw[];
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int grp = warp / sp.S, chunk = warp % sp.S;
@@ -763,8 +767,7 @@ cudaError_t launch_w(const ScanDesc& s, cudaStream_t st) {
   const int smem = warps * C::WARP_B + 128;
   ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
   dim3 grid((groups + sp.G - 1) / sp.G, s.batch);
-  scan_w_kernel<TI, N, TPC, CPL><<<grid, 32 * warps, smem, st>>>(tx, td, tg, tb, ty, p, sp, s.status);
-  return cudaGetLastError();
+  return launch(scan_w_kernel<TI, N, TPC, CPL>, grid, dim3(32 * warps), smem, st, tx, td, tg, tb, ty, p, sp, s.status);
 }
 
 template <typename TI, int NS, int TPC, int NWT>
@@ -772,8 +775,7 @@ cudaError_t launch_one(const ScanDesc& s, cudaStream_t st) {
   constexpr int CPW = 32 / TPC;
   ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
   dim3 grid((s.d_inner + CPW - 1) / CPW, s.batch);
-  scan_kernel<TI, NS, TPC, NWT><<<grid, 32 * NWT, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch(scan_kernel<TI, NS, TPC, NWT>, grid, dim3(32 * NWT), 0, st, p);
 }
 
 template <typename TI>

@@ -53,6 +53,8 @@ __device__ __forceinline__ void store_elem(const F32GemmParams& p, long long row
 // C tile 64 x 64, 256 threads x (4 x 4); SWIGLU computes gate and up tiles together.
 template <bool SWIGLU>
 __global__ void __launch_bounds__(256) gemm_f32_kernel(const __grid_constant__ F32GemmParams p) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float As[TK][TB + 1];
   __shared__ float Ws[TK][TB + 1];
   __shared__ float Us[SWIGLU ? TK : 1][TB + 1];
@@ -121,6 +123,8 @@ __global__ void __launch_bounds__(128) attention_f32_kernel(const float* __restr
                                                             const float* __restrict__ v, long long kv_ld,
                                                             float* __restrict__ out, long long out_ld, int T, int Hq,
                                                             int Hkv, int dh, int n_meta, int window, int batch) {
+  pdl_trigger();
+  pdl_wait();
   const long long wid = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const long long total = static_cast<long long>(batch) * Hq * T;
@@ -194,21 +198,17 @@ cudaError_t launch_gemm_f32(const GemmDesc& g, cudaStream_t st) {
   if (p.rows <= 0) return cudaSuccess;
   const int ncols = g.epi == EPI_SWIGLU ? g.swiglu_F : g.N;
   dim3 grid((ncols + TB - 1) / TB, static_cast<unsigned>((p.rows + TB - 1) / TB));
-  if (g.epi == EPI_SWIGLU)
-    gemm_f32_kernel<true><<<grid, 256, 0, st>>>(p);
-  else
-    gemm_f32_kernel<false><<<grid, 256, 0, st>>>(p);
-  return cudaGetLastError();
+  if (g.epi == EPI_SWIGLU) return launch(gemm_f32_kernel<true>, grid, dim3(256), 0, st, p);
+  return launch(gemm_f32_kernel<false>, grid, dim3(256), 0, st, p);
 }
 
 cudaError_t launch_attention_f32(const AttnDesc& a, cudaStream_t st) {
   const long long total = static_cast<long long>(a.batch) * a.n_q_heads * a.T;
   if (total <= 0) return cudaSuccess;
-  attention_f32_kernel<<<static_cast<unsigned>((total + 3) / 4), 128, 0, st>>>(
-      static_cast<const float*>(a.q), a.q_ld, static_cast<const float*>(a.k), static_cast<const float*>(a.v), a.kv_ld,
-      static_cast<float*>(a.out), a.out_ld, a.T, a.n_q_heads, a.n_kv_heads, a.head_dim, a.n_meta, a.window,
-      a.batch);
-  return cudaGetLastError();
+  return launch(attention_f32_kernel, dim3(static_cast<unsigned>((total + 3) / 4)), dim3(128), 0, st,
+                static_cast<const float*>(a.q), a.q_ld, static_cast<const float*>(a.k),
+                static_cast<const float*>(a.v), a.kv_ld, static_cast<float*>(a.out), a.out_ld, a.T, a.n_q_heads,
+                a.n_kv_heads, a.head_dim, a.n_meta, a.window, a.batch);
 }
 
 }  // namespace hy
