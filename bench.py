@@ -97,7 +97,7 @@ def stage_work(s: synth.LayerShape):
 
 KERNEL_NAMES = {"in_proj": "gemm_bf16_tc, tcgen05", "x_proj": "gemm_bf16_tc, tcgen05",
                 "dt_proj": "gemm_bf16_tc, tcgen05", "attention": "attn_fwd_tc, tcgen05",
-                "scan": "scan_w_kernel", "branch_norm": "row_ssq_kernel + scale_cols_kernel",
+                "scan": "scan_tc_kernel, tcgen05 tf32", "branch_norm": "row_ssq_kernel + scale_cols_kernel",
                 "out_proj": "gemm_bf16_tc, tcgen05, two accumulators"}
 
 # dominant bound of each stage: a dense contraction on the tensor cores or HBM traffic

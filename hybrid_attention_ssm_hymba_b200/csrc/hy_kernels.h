@@ -86,6 +86,9 @@ struct ScanDesc {
   unsigned* status;
 };
 cudaError_t launch_scan(const ScanDesc& s, cudaStream_t st);
+// The tensor-core form of the scan (bf16, d_state = 16, 16-byte aligned operands);
+// cudaErrorNotSupported for any other configuration.
+cudaError_t launch_scan_tc(const ScanDesc& s, cudaStream_t st);
 
 struct AttnDesc {
   const void* q; long long q_ld;     // [batch*T, q_ld], head h at column h*dh

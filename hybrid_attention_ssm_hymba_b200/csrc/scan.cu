@@ -26,6 +26,10 @@
 #define HY_SCAN16_TPC 1
 #define HY_SCAN16_CPL 2
 #endif
+// bf16 with d_state = 16 runs the tensor-core block form (scan_tc.cu) by default.
+#ifndef HY_SCAN_TC
+#define HY_SCAN_TC 1
+#endif
 #ifndef HY_SCAN128_TPC
 #define HY_SCAN128_TPC 4
 #define HY_SCAN128_CPL 2
@@ -787,6 +791,12 @@ cudaError_t launch_t(const ScanDesc& s, cudaStream_t st) {
   const bool tma_ok = (s.d_inner * es) % 16 == 0 && (s.y_ld * es) % 16 == 0 && a16(s.x) && a16(s.dt) &&
                      a16(s.gate) && a16(s.bc) && a16(s.y);
   if (tma_ok) {
+#if HY_SCAN_TC
+    if (sizeof(TI) == 2 && s.d_state == 16) {
+      const cudaError_t e = launch_scan_tc(s, st);
+      if (e != cudaErrorNotSupported) return e;
+    }
+#endif
     switch (s.d_state) {
       case 16: return launch_w<TI, 16, HY_SCAN16_TPC, HY_SCAN16_CPL>(s, st);
       case 32: return launch_w<TI, 32, 1, 1>(s, st);

@@ -1,0 +1,475 @@
+// scan_tc.cu -- the selective scan of the SSM heads as block matrix products on the
+// 5th-generation tensor cores (bf16 layers, d_state = 16).
+//
+// Hymba writes its SSM head as a mixing matrix (blog.outta.ai Hymba review, "Design
+// formulation"): y_i = G_i . sum_{j<=i} alpha_ij x_j with
+//   alpha_ij = C_i (prod_{k=j+1..i} exp(A dt_k)) B_j dt_j.
+// With A one scalar per channel the decay product factors: write
+// lambda_t = sum_{k<=t} |A| dt_k / ln 2 within a block of Q = 64 steps and a reference
+// r (the block's lambda after its first 32 steps).  Then for s <= t in the block
+//   prod_{k=s+1..t} exp(A dt_k) = 2^(r - lambda_t) * 2^(lambda_s - r)
+// and the block's output is, per channel c (h_in the state entering the block),
+//   y[c,t] = W[c,t] * ( sum_s V[c,s] M[t,s] + sum_n G'[c,n] C[t,n] )
+//   V[c,s] = dt x 2^(lambda_s - r),  W[c,t] = gate 2^(r - lambda_t),
+//   M[t,s] = (C_t . B_s) [s <= t],   G'[c,n] = h_in[c,n] 2^(-r).
+// The state leaving the block is h_out = 2^(-lambda_63) h_in + 2^(r - lambda_63) V B.
+// So each block is four small tensor-core products that every channel shares the
+// operands of: M = C B^T (once per block for all channels), Y = V M^T + G' C^T, and
+// dG = V B.  Only the prefix sums, the exponentials and the 16-element state update
+// per channel and block run on the CUDA cores.
+//
+// Ranges: |lambda_s - r| stays below 2^100 when both half-block decay sums stay
+// below 100 (log2 units), which keeps every factor a normal fp32 number.  A block
+// where some channel of the CTA exceeds that (very large dt) is run on the CUDA
+// cores by the plain recurrence instead, for every channel of the CTA.
+//
+// CTA = 128 channels of one sequence, all T steps, 384 threads:
+//   warps 0-7   channel warps: warp w owns TMEM lane quadrant w % 4 (channel
+//               32 (w % 4) + lane) and half w / 4 of each block's 64 steps; half 1
+//               also carries the state chain and the large-decay path.
+//   warps 8-9   mask C B^T (TMEM lanes 0-63 = t) into M, transpose B into B^T.
+//   warp 10     TMA producer (x, dt, gate [64 t][128 c] bf16; B|C [64 t][32] fp32).
+//   warp 11     TMEM owner and MMA issuer.
+// Operands: V, G' in TMEM (A from TMEM); M, B^T, C in shared memory, 128-byte
+// swizzled K-major; accumulators Y (64 columns), dG (16), C B^T (64) in TMEM; all
+// products kind::tf32 with fp32 accumulation.  y goes out through a double-buffered
+// shared tile and TMA stores.
+#include "hy_common.cuh"
+#include "hy_kernels.h"
+
+namespace hy {
+namespace {
+
+constexpr int Q = 64;         // steps per block
+constexpr int CH = 128;       // channels per CTA (TMEM lanes)
+constexpr int NST = 16;       // state size handled here
+constexpr int STAGES = 3;
+constexpr int NTHR = 384;
+constexpr int NCHT = 256;     // channel threads (named barrier 1)
+constexpr float kRange = 100.f;  // max half-block decay sum (log2 units) for the product form
+
+constexpr int TILE_B = Q * CH * 2;       // [64 t][128 c] bf16
+constexpr int BC_B = Q * 2 * NST * 4;    // [64 t][B 16 | C 16] fp32, 128-byte rows
+constexpr int MT_B = Q * Q * 4;          // M [t][s] tf32: two K chunks of [64 rows][128 B]
+constexpr int BT_B = NST * Q * 4;        // B^T [n][s] tf32: two K chunks of [16 rows][128 B]
+
+constexpr int OFF_X = 0;
+constexpr int OFF_DT = OFF_X + STAGES * TILE_B;
+constexpr int OFF_G = OFF_DT + STAGES * TILE_B;
+constexpr int OFF_BC = OFF_G + STAGES * TILE_B;
+constexpr int OFF_MT = OFF_BC + STAGES * BC_B;   // also the rows C B^T reads past the last B|C tile
+constexpr int OFF_BT = OFF_MT + MT_B;
+constexpr int OFF_Y = OFF_BT + BT_B;
+constexpr int OFF_S = OFF_Y + 2 * TILE_B;        // float [2][128]: half-block decay sums
+constexpr int OFF_BAR = OFF_S + 2 * CH * 4;
+constexpr int NBAR = 2 * STAGES + 4 * 2 + 3;
+constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
+constexpr int SMEM_TOTAL = SMEM_USED + 1024;     // + alignment of the base to 1024
+static_assert(OFF_BC % 1024 == 0 && OFF_MT % 1024 == 0 && OFF_BT % 1024 == 0, "swizzled tiles 1024-aligned");
+static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
+
+// TMEM columns (512 allocated)
+constexpr uint32_t COL_Y = 0;      // [2][64]
+constexpr uint32_t COL_V = 128;    // [2][64]
+constexpr uint32_t COL_W = 256;    // [2][64]
+constexpr uint32_t COL_MR = 384;   // [64]: C B^T (lanes 0-63)
+constexpr uint32_t COL_DG = 448;   // [2][16]
+constexpr uint32_t COL_GP = 480;   // [2][16]
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr uint32_t IDESC_N64 = idesc_tf32(128, 64);
+constexpr uint32_t IDESC_N16 = idesc_tf32(128, 16);
+
+HY_DEV float bf2f(uint16_t u) { return __uint_as_float(static_cast<uint32_t>(u) << 16); }
+
+__global__ void __launch_bounds__(NTHR, 1)
+    scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDT,
+                   const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmBC,
+                   const __grid_constant__ CUtensorMap tmY, const float* __restrict__ a_log, int T, int Di,
+                   unsigned* status) {
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* full = bars;                    // [STAGES] TMA landed
+  uint64_t* empty = full + STAGES;          // [STAGES] last MMA reading the stage done
+  uint64_t* vready = empty + STAGES;        // [2] V, W in TMEM (256 arrivals)
+  uint64_t* dgready = vready + 2;           // [2] Y = V M^T and dG = V B done
+  uint64_t* gready = dgready + 2;           // [2] G' in TMEM (128 arrivals)
+  uint64_t* yready = gready + 2;            // [2] Y complete
+  uint64_t* mraw = yready + 2;              // C B^T in TMEM
+  uint64_t* mready = mraw + 1;              // M and B^T in shared memory (64 arrivals)
+  uint64_t* mma_done = mready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sS = reinterpret_cast<float*>(sm + OFF_S);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c0 = blockIdx.x * CH, b = blockIdx.y;
+  const int nblk = (T + Q - 1) / Q;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&vready[i], NCHT);
+      mbar_init(&dgready[i], 1);
+      mbar_init(&gready[i], NCHT / 2);
+      mbar_init(&yready[i], 1);
+    }
+    mbar_init(mraw, 1);
+    mbar_init(mready, 64);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 11) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  pdl_wait();
+  if (threadIdx.x == 320) {
+    tma_prefetch(&tmX);
+    tma_prefetch(&tmDT);
+    tma_prefetch(&tmG);
+    tma_prefetch(&tmBC);
+    tma_prefetch(&tmY);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(sm);
+
+  if (warp == 10) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int k = 0;
+      for (; k < nblk; ++k) {
+        const int s = k % STAGES;
+        if (k >= STAGES && !mbar_wait(&empty[s], ((k / STAGES) - 1) & 1u, status, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[s], 3 * TILE_B + BC_B);
+        tma_load_3d(sm + OFF_X + s * TILE_B, &tmX, &full[s], c0, k * Q, b);
+        tma_load_3d(sm + OFF_DT + s * TILE_B, &tmDT, &full[s], c0, k * Q, b);
+        tma_load_3d(sm + OFF_G + s * TILE_B, &tmG, &full[s], c0, k * Q, b);
+        tma_load_3d(sm + OFF_BC + s * BC_B, &tmBC, &full[s], 0, k * Q, b);
+      }
+      if (k < nblk) {  // aborted: let the copies already issued land before smem goes away
+        int never = 0;
+        for (int j = (k > STAGES ? k - STAGES : 0); j < k; ++j)
+          mbar_wait(&full[j % STAGES], (j / STAGES) & 1u, nullptr, &never, 100000000ull);
+      }
+    }
+  } else if (warp == 11) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t mt = sbase + OFF_MT, bt = sbase + OFF_BT;
+      auto issue_mraw = [&](int k) -> bool {
+        const int s = k % STAGES;
+        if (!mbar_wait(&full[s], (k / STAGES) & 1u, status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t bc = sbase + OFF_BC + s * BC_B;
+        // C B^T: A = C rows (128 rows read; rows 64..127 are whatever follows the tile and
+        // land in TMEM lanes nobody reads), B = B rows; K = 16 = two tf32 steps.
+        for (int j = 0; j < 2; ++j)
+          umma_tf32_ss(tmem + COL_MR, sdesc_sw128(bc + 64 + 32 * j, 16, 1024), sdesc_sw128(bc + 32 * j, 16, 1024),
+                       IDESC_N64, j);
+        umma_commit(mraw);
+        return true;
+      };
+      bool ok = nblk > 0 && issue_mraw(0);
+      for (int k = 0; ok && k < nblk; ++k) {
+        const int i = k & 1, s = k % STAGES;
+        const uint32_t par = (k >> 1) & 1u;
+        if (!mbar_wait(&vready[i], par, status, abort_flag) || !mbar_wait(mready, k & 1u, status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t vcol = tmem + COL_V + 64 * i;
+        // Y = V M^T (K = s, 64 = 8 steps) and dG = V B (B^T tile)
+        for (int j = 0; j < 8; ++j)
+          umma_tf32_ts(tmem + COL_Y + 64 * i, vcol + 8 * j, sdesc_sw128(mt + (j >> 2) * 8192 + (j & 3) * 32, 16, 1024),
+                       IDESC_N64, j);
+        for (int j = 0; j < 8; ++j)
+          umma_tf32_ts(tmem + COL_DG + 16 * i, vcol + 8 * j, sdesc_sw128(bt + (j >> 2) * 2048 + (j & 3) * 32, 16, 1024),
+                       IDESC_N16, j);
+        umma_commit(&dgready[i]);
+        if (!mbar_wait(&gready[i], par, status, abort_flag)) break;
+        tc_fence_after();
+        // Y += G' C^T (K = n = 16)
+        const uint32_t bc = sbase + OFF_BC + s * BC_B;
+        for (int j = 0; j < 2; ++j)
+          umma_tf32_ts(tmem + COL_Y + 64 * i, tmem + COL_GP + 16 * i + 8 * j, sdesc_sw128(bc + 64 + 32 * j, 16, 1024),
+                       IDESC_N64, 1);
+        umma_commit(&yready[i]);
+        umma_commit(&empty[s]);
+        if (k + 1 < nblk && !issue_mraw(k + 1)) break;
+      }
+      umma_commit(mma_done);
+      int never = 0;
+      mbar_wait(mma_done, 0, nullptr, &never, 100000000ull);
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ M = mask(C B^T), B^T
+    const int t = (warp - 8) * 32 + lane;  // TMEM lane = step within the block
+    const uint32_t tl = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    uint8_t* mt = sm + OFF_MT;
+    uint8_t* bt = sm + OFF_BT;
+    for (int k = 0; k < nblk; ++k) {
+      const int s = k % STAGES;
+      bool ok = mbar_wait(mraw, k & 1u, status, abort_flag) && mbar_wait(&full[s], (k / STAGES) & 1u, status, abort_flag);
+      if (ok && k > 0) ok = mbar_wait(&dgready[(k - 1) & 1], ((k - 1) >> 1) & 1u, status, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t r[2][32];
+      tmem_ld32(tl + COL_MR, r[0]);
+      tmem_ld32(tl + COL_MR + 32, r[1]);
+      tmem_wait_ld();
+      // row t of M (K-major, 128-byte swizzle): s in [32 h, 32 h + 32) -> chunk h
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint8_t* row = mt + h * 8192 + (t >> 3) * 1024 + (t & 7) * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint32_t v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int si = 32 * h + 4 * j + e;
+            v[e] = si <= t ? tf32_rna(__uint_as_float(r[h][4 * j + e])) : 0u;
+          }
+          *reinterpret_cast<uint4*>(row + ((j ^ (t & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+        }
+      }
+      // B^T [n][s]: element (n, s = t)
+      const uint8_t* bcrow = sm + OFF_BC + s * BC_B + t * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 q = *reinterpret_cast<const float4*>(bcrow + ((j ^ (t & 7)) << 4));
+        const float qv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int n = 4 * j + e;
+          uint8_t* dst = bt + (t >> 5) * 2048 + (n >> 3) * 1024 + (n & 7) * 128 + ((((t & 31) >> 2) ^ (n & 7)) << 4) +
+                         (t & 3) * 4;
+          *reinterpret_cast<uint32_t*>(dst) = tf32_rna(qv[e]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(mready);
+    }
+  } else {
+    // ------------------------------------------------------------ channel warps
+    const int qd = warp & 3, half = warp >> 2;
+    const int cl = qd * 32 + lane, c = c0 + cl;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const float A2 = c < Di ? expf(a_log[c]) * 1.4426950408889634f : 0.f;  // |A| / ln 2
+    float h[NST];
+#pragma unroll
+    for (int n = 0; n < NST; ++n) h[n] = 0.f;
+    float pS0 = 0.f, pS1 = 0.f;  // previous block's half sums (chain)
+    bool prev_any = false;
+    for (int k = 0; k <= nblk; ++k) {
+      bool fail = false;
+      bool any = false;
+      if (k < nblk) {
+        const int s = k % STAGES, i = k & 1;
+        const uint8_t* xt = sm + OFF_X + s * TILE_B + cl * 2;
+        const uint8_t* dtt = sm + OFF_DT + s * TILE_B + cl * 2;
+        const uint8_t* gt = sm + OFF_G + s * TILE_B + cl * 2;
+        fail = !__all_sync(0xffffffffu, mbar_wait(&full[s], (k / STAGES) & 1u, status, abort_flag));
+        // ---- half-block decay sum
+        float dtv[32];
+        float S = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          dtv[j] = bf2f(*reinterpret_cast<const uint16_t*>(dtt + (32 * half + j) * 256));
+          S = fmaf(A2, dtv[j], S);
+        }
+        sS[half * CH + cl] = S;
+        any = bar_red_or(1, NCHT, fail || !(S <= kRange));
+        // ---- V = dt x 2^(lambda - r), W = gate 2^(r - lambda) into TMEM
+        if (!fail) {
+          uint32_t vr[32], wr[32];
+          if (!any) {
+            float mu = half ? 0.f : -S;  // lambda - r
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              mu = fmaf(A2, dtv[j], mu);
+              const int row = (32 * half + j) * 256;
+              const float xv = bf2f(*reinterpret_cast<const uint16_t*>(xt + row));
+              const float gv = bf2f(*reinterpret_cast<const uint16_t*>(gt + row));
+              vr[j] = tf32_rna(dtv[j] * xv * ex2_approx(mu));
+              wr[j] = __float_as_uint(gv * ex2_approx(-mu));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) vr[j] = wr[j] = 0u;
+          }
+          tmem_st32(tl + COL_V + 64 * i + 32 * half, vr);
+          tmem_st32(tl + COL_W + 64 * i + 32 * half, wr);
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        mbar_arrive(&vready[i]);
+        // ---- state chain: h entering block k, G' = h 2^(-r)  (half 1)
+        if (half == 1 && !fail) {
+          const float S0 = sS[cl], S1 = S;
+          if (k > 0 && !prev_any) {
+            if (__all_sync(0xffffffffu, mbar_wait(&dgready[(k - 1) & 1], ((k - 1) >> 1) & 1u, status, abort_flag))) {
+              tc_fence_after();
+              uint32_t d[16];
+              tmem_ld16(tl + COL_DG + 16 * ((k - 1) & 1), d);
+              tmem_wait_ld();
+              const float a = ex2_approx(-(pS0 + pS1)), bs = ex2_approx(-pS1);
+#pragma unroll
+              for (int n = 0; n < NST; ++n) h[n] = fmaf(a, h[n], bs * __uint_as_float(d[n]));
+            } else {
+              fail = true;
+            }
+          }
+          if (!fail) {
+            uint32_t gp[16];
+            const float sc = ex2_approx(-S0);
+#pragma unroll
+            for (int n = 0; n < NST; ++n) gp[n] = any ? 0u : tf32_rna(h[n] * sc);
+            tmem_st16(tl + COL_GP + 16 * i, gp);
+            tmem_wait_st();
+            tc_fence_before();
+          }
+          pS0 = S0;
+          pS1 = S1;
+        }
+        // ---- large decays: the plain recurrence over the block, y into the y tile.  G' is
+        // announced only after it, since the MMA that waits for G' frees the stage.
+        if (any) {
+          if (threadIdx.x == 0) bulk_wait_all();  // the store that last read this y tile is done
+          bar_sync_n(1, NCHT);
+          if (half == 1 && !fail) {
+            uint8_t* yt = sm + OFF_Y + i * TILE_B + cl * 2;
+            const uint8_t* bct = sm + OFF_BC + s * BC_B;
+#pragma unroll 1
+            for (int t = 0; t < Q; ++t) {
+              const float dt = bf2f(*reinterpret_cast<const uint16_t*>(dtt + t * 256));
+              const float xv = bf2f(*reinterpret_cast<const uint16_t*>(xt + t * 256));
+              const float gv = bf2f(*reinterpret_cast<const uint16_t*>(gt + t * 256));
+              const float a = ex2_approx(-A2 * dt), u = dt * xv;
+              const uint8_t* row = bct + t * 128;
+              float y = 0.f;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float4 bq = *reinterpret_cast<const float4*>(row + ((j ^ (t & 7)) << 4));
+                const float4 cq = *reinterpret_cast<const float4*>(row + (((j + 4) ^ (t & 7)) << 4));
+                h[4 * j + 0] = fmaf(a, h[4 * j + 0], u * bq.x);
+                h[4 * j + 1] = fmaf(a, h[4 * j + 1], u * bq.y);
+                h[4 * j + 2] = fmaf(a, h[4 * j + 2], u * bq.z);
+                h[4 * j + 3] = fmaf(a, h[4 * j + 3], u * bq.w);
+                y = fmaf(cq.x, h[4 * j + 0], y);
+                y = fmaf(cq.y, h[4 * j + 1], y);
+                y = fmaf(cq.z, h[4 * j + 2], y);
+                y = fmaf(cq.w, h[4 * j + 3], y);
+              }
+              *reinterpret_cast<uint16_t*>(yt + t * 256) = bf16_bits(gv * y);
+            }
+          }
+        }
+        if (half == 1) mbar_arrive(&gready[i]);
+      }
+      // ---- output of block k - 1: y = W * Y into the y tile, TMA store
+      if (k > 0) {
+        const int jb = k - 1, i = jb & 1;
+        if (!fail) {
+          fail = !__all_sync(0xffffffffu, mbar_wait(&yready[i], (jb >> 1) & 1u, status, abort_flag));
+          if (!fail && !prev_any) {
+            tc_fence_after();
+            uint32_t yv[32], wv[32];
+            tmem_ld32(tl + COL_Y + 64 * i + 32 * half, yv);
+            tmem_ld32(tl + COL_W + 64 * i + 32 * half, wv);
+            tmem_wait_ld();
+            uint8_t* yt = sm + OFF_Y + i * TILE_B + cl * 2 + 32 * half * 256;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              *reinterpret_cast<uint16_t*>(yt + j * 256) = bf16_bits(__uint_as_float(yv[j]) * __uint_as_float(wv[j]));
+          }
+        }
+        fence_proxy_async_smem();
+        if (bar_red_or(1, NCHT, fail || *abort_flag)) break;
+        if (threadIdx.x == 0) {
+          tma_store_3d(&tmY, sm + OFF_Y + i * TILE_B, c0, jb * Q, b);
+          bulk_commit();
+          bulk_wait_read1();  // the store before it has read its tile: that tile may be rewritten
+        }
+      } else if (fail) {
+        if (bar_red_or(1, NCHT, true)) break;
+      } else {
+        if (bar_red_or(1, NCHT, *abort_flag != 0)) break;
+      }
+      if (k < nblk) prev_any = any;
+    }
+    if (threadIdx.x == 0) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 11) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D map over [batch][T][cols] (row stride ld elements), box = bc x br x 1.
+bool map3d(CUtensorMap* m, const void* base, bool f32, int batch, int T, long long cols, long long ld, int bc,
+           int br, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const int es = f32 ? 4 : 2;
+  cuuint64_t gd[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(batch)};
+  cuuint64_t gs[2] = {static_cast<cuuint64_t>(ld) * es, static_cast<cuuint64_t>(ld) * es * T};
+  cuuint32_t bx[3] = {static_cast<cuuint32_t>(bc), static_cast<cuuint32_t>(br), 1}, el[3] = {1, 1, 1};
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+            gd, gs, bx, el, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// bf16, d_state = 16, 16-byte aligned operands and row strides (checked by the caller).
+// Returns cudaErrorNotSupported when the configuration is not this kernel's.
+cudaError_t launch_scan_tc(const ScanDesc& s, cudaStream_t st) {
+  if (!s.bf16 || s.d_state != NST) return cudaErrorNotSupported;
+  CUtensorMap tx, td, tg, tb, ty;
+  if (!map3d(&tx, s.x, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !map3d(&td, s.dt, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !map3d(&tg, s.gate, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !map3d(&tb, s.bc, true, s.batch, s.T, 2 * NST, 2 * NST, 2 * NST, Q, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3d(&ty, s.y, false, s.batch, s.T, s.d_inner, s.y_ld, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorNotSupported;
+  static int attr_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 31 && !(attr_mask & (1 << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TOTAL);
+    if (e != cudaSuccess) return e;
+    attr_mask |= 1 << dev;
+  }
+  dim3 grid((s.d_inner + CH - 1) / CH, s.batch);
+  return launch(scan_tc_kernel, grid, dim3(NTHR), SMEM_TOTAL, st, tx, td, tg, tb, ty, s.a_log, s.T, s.d_inner,
+                s.status);
+}
+
+}  // namespace hy
