@@ -37,6 +37,16 @@
 #include "hy_common.cuh"
 #include "hy_kernels.h"
 
+// W = gate 2^(r - lambda) as gate / 2^(lambda - r) with a Newton reciprocal on the FMA
+// pipe (1) or a second SFU exp2 (0).
+#ifndef HY_SCANTC_W_NEWTON
+#define HY_SCANTC_W_NEWTON 0
+#endif
+// Paired fp32 arithmetic (fma/mul.rn.f32x2) for two steps at a time.
+#ifndef HY_SCANTC_PACK
+#define HY_SCANTC_PACK 1
+#endif
+
 namespace hy {
 namespace {
 
@@ -81,6 +91,17 @@ constexpr uint32_t IDESC_N64 = idesc_tf32(128, 64);
 constexpr uint32_t IDESC_N16 = idesc_tf32(128, 16);
 
 HY_DEV float bf2f(uint16_t u) { return __uint_as_float(static_cast<uint32_t>(u) << 16); }
+// fp32 -> tf32 bit pattern, magnitude rounded to nearest (ties away from zero), on the
+// integer pipe: add half of the dropped 13-bit field and clear it.
+HY_DEV uint32_t tf32_round(float x) { return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u; }
+// 1/e for e > 0 on the FMA pipe: exponent-negating initial guess (relative error below
+// 1/8) and three Newton steps r <- r (2 - e r), each squaring the error (below 1e-7).
+HY_DEV float recip_newton(float e) {
+  float r = __uint_as_float(0x7EF311C3u - __float_as_uint(e));
+#pragma unroll
+  for (int i = 0; i < 3; ++i) r = r * fmaf(-e, r, 2.f);
+  return r;
+}
 
 __global__ void __launch_bounds__(NTHR, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDT,
@@ -235,7 +256,7 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int si = 32 * h + 4 * j + e;
-            v[e] = si <= t ? tf32_rna(__uint_as_float(r[h][4 * j + e])) : 0u;
+            v[e] = si <= t ? tf32_round(__uint_as_float(r[h][4 * j + e])) : 0u;
           }
           *reinterpret_cast<uint4*>(row + ((j ^ (t & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
         }
@@ -251,7 +272,7 @@ __global__ void __launch_bounds__(NTHR, 1)
           const int n = 4 * j + e;
           uint8_t* dst = bt + (t >> 5) * 2048 + (n >> 3) * 1024 + (n & 7) * 128 + ((((t & 31) >> 2) ^ (n & 7)) << 4) +
                          (t & 3) * 4;
-          *reinterpret_cast<uint32_t*>(dst) = tf32_rna(qv[e]);
+          *reinterpret_cast<uint32_t*>(dst) = tf32_round(qv[e]);
         }
       }
       fence_proxy_async_smem();
@@ -280,12 +301,23 @@ __global__ void __launch_bounds__(NTHR, 1)
         fail = !__all_sync(0xffffffffu, mbar_wait(&full[s], (k / STAGES) & 1u, status, abort_flag));
         // ---- half-block decay sum
         float dtv[32];
+#if HY_SCANTC_PACK
+        float2 S2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          dtv[j] = bf2f(*reinterpret_cast<const uint16_t*>(dtt + (32 * half + j) * 256));
+          dtv[j + 1] = bf2f(*reinterpret_cast<const uint16_t*>(dtt + (32 * half + j + 1) * 256));
+          S2 = __ffma2_rn(make_float2(A2, A2), make_float2(dtv[j], dtv[j + 1]), S2);
+        }
+        const float S = S2.x + S2.y;
+#else
         float S = 0.f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           dtv[j] = bf2f(*reinterpret_cast<const uint16_t*>(dtt + (32 * half + j) * 256));
           S = fmaf(A2, dtv[j], S);
         }
+#endif
         sS[half * CH + cl] = S;
         any = bar_red_or(1, NCHT, fail || !(S <= kRange));
         // ---- V = dt x 2^(lambda - r), W = gate 2^(r - lambda) into TMEM
@@ -293,15 +325,40 @@ __global__ void __launch_bounds__(NTHR, 1)
           uint32_t vr[32], wr[32];
           if (!any) {
             float mu = half ? 0.f : -S;  // lambda - r
+#if HY_SCANTC_PACK
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float mu0 = fmaf(A2, dtv[j], mu);
+              mu = fmaf(A2, dtv[j + 1], mu0);
+              const int row = (32 * half + j) * 256;
+              const float2 xv = make_float2(bf2f(*reinterpret_cast<const uint16_t*>(xt + row)),
+                                            bf2f(*reinterpret_cast<const uint16_t*>(xt + row + 256)));
+              const float2 gv = make_float2(bf2f(*reinterpret_cast<const uint16_t*>(gt + row)),
+                                            bf2f(*reinterpret_cast<const uint16_t*>(gt + row + 256)));
+              const float2 e = make_float2(ex2_approx(mu0), ex2_approx(mu));
+              const float2 v = __fmul2_rn(__fmul2_rn(make_float2(dtv[j], dtv[j + 1]), xv), e);
+              const float2 w = __fmul2_rn(gv, make_float2(ex2_approx(-mu0), ex2_approx(-mu)));
+              vr[j] = tf32_round(v.x);
+              vr[j + 1] = tf32_round(v.y);
+              wr[j] = __float_as_uint(w.x);
+              wr[j + 1] = __float_as_uint(w.y);
+            }
+#else
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               mu = fmaf(A2, dtv[j], mu);
               const int row = (32 * half + j) * 256;
               const float xv = bf2f(*reinterpret_cast<const uint16_t*>(xt + row));
               const float gv = bf2f(*reinterpret_cast<const uint16_t*>(gt + row));
-              vr[j] = tf32_rna(dtv[j] * xv * ex2_approx(mu));
+              const float e = ex2_approx(mu);
+              vr[j] = tf32_round(dtv[j] * xv * e);
+#if HY_SCANTC_W_NEWTON
+              wr[j] = __float_as_uint(gv * recip_newton(e));
+#else
               wr[j] = __float_as_uint(gv * ex2_approx(-mu));
+#endif
             }
+#endif
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) vr[j] = wr[j] = 0u;
@@ -332,7 +389,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             uint32_t gp[16];
             const float sc = ex2_approx(-S0);
 #pragma unroll
-            for (int n = 0; n < NST; ++n) gp[n] = any ? 0u : tf32_rna(h[n] * sc);
+            for (int n = 0; n < NST; ++n) gp[n] = any ? 0u : tf32_round(h[n] * sc);
             tmem_st16(tl + COL_GP + 16 * i, gp);
             tmem_wait_st();
             tc_fence_before();
@@ -388,8 +445,18 @@ __global__ void __launch_bounds__(NTHR, 1)
             tmem_wait_ld();
             uint8_t* yt = sm + OFF_Y + i * TILE_B + cl * 2 + 32 * half * 256;
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              *reinterpret_cast<uint16_t*>(yt + j * 256) = bf16_bits(__uint_as_float(yv[j]) * __uint_as_float(wv[j]));
+            for (int j = 0; j < 32; j += 2) {
+#if HY_SCANTC_PACK
+              const float2 o = __fmul2_rn(make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])),
+                                          make_float2(__uint_as_float(wv[j]), __uint_as_float(wv[j + 1])));
+              const uint32_t p2 = pack_bf16(o.x, o.y);
+#else
+              const uint32_t p2 = pack_bf16(__uint_as_float(yv[j]) * __uint_as_float(wv[j]),
+                                            __uint_as_float(yv[j + 1]) * __uint_as_float(wv[j + 1]));
+#endif
+              *reinterpret_cast<uint16_t*>(yt + j * 256) = static_cast<uint16_t>(p2);
+              *reinterpret_cast<uint16_t*>(yt + (j + 1) * 256) = static_cast<uint16_t>(p2 >> 16);
+            }
           }
         }
         fence_proxy_async_smem();

@@ -97,6 +97,22 @@ def test_scan_extreme_decay_and_segments(dtype, N, T):
     assert_close(_run_scan(inp, B, T, Di, N, dtype), _scan_ref(inp, B, T, Di, N), dtype, "scan extreme decay")
 
 
+def test_scan_block_form_hands_large_decay_blocks_to_the_recurrence():
+    """bf16, d_state 16 (the tensor-core block form): a 64-step block in which some
+    channel's half-block decay sum leaves the range of the factored form runs the plain
+    recurrence for every channel of its 128-channel tile, and the state chain resumes
+    after it.  Such blocks here sit between ordinary ones, in the first and in the second
+    half of a block, in the second (partial) channel tile and in the ragged last block."""
+    B, T, Di, N = 2, 700, 192, 16
+    inp = synth.scan_inputs(25, B, T, Di, N)
+    dt = inp["dt"].reshape(B, T, Di).astype(np.float32).copy()
+    dt[0, 130:150, 7] = 6.0      # block 2, first half, tile 0
+    dt[0, 360:380, 150] = 6.0    # block 5, second half, tile 1
+    dt[1, 650:670, 100] = 6.0    # block 10 (60 steps), tile 0
+    inp["dt"] = synth.round_bf16(dt.reshape(B * T, Di))
+    assert_close(_run_scan(inp, B, T, Di, N, "bf16"), _scan_ref(inp, B, T, Di, N), "bf16", "scan mixed blocks")
+
+
 def test_scan_long_decay_small_dt():
     """dt down to 1e-4 over 32K steps: fp32 state keeps the long decay products."""
     B, T, Di, N = 1, 32896, 16, 128
