@@ -5,24 +5,32 @@ next, and the random-init stack amplifies a perturbation of its input (in exact
 fp64 arithmetic a 1e-3 relative perturbation of X~ grows to ~7e-3 relative L2
 after 8 blocks).  A bf16 pipeline rounds its activations to bf16 (2^-9 relative)
 at every storage point of every block, so the end-of-stack deviation from the
-exact oracle grows with depth: every single hybrid-head layer and block pair
-meets the 2e-2 bound, the 24-block output cannot.
+exact oracle grows with depth: every single hybrid-head layer meets the 2e-2
+bound; a block pair (two layers and two FFNs) may not, the 24-block output cannot.
 
 This script measures that growth with the oracle alone: it runs the exact fp64
 oracle and the same oracle functions with each stored activation rounded to bf16
 at the storage points the bf16 path uses (the normalised block input, the fused
 in_proj outputs Q|K|V|X_ssm|SiLU(G), dt_low, dt, the attention output, the gated
-SSM output, the fused Z, the residual stream, the SwiGLU product), on the test's
+SSM output, W_out with beta folded in (the branch norm is fused into out_proj, so
+the normalised Z itself is never stored), the residual stream, the SwiGLU product)
+and the SSM output at tf32 precision (the scan's block products take tf32
+operands), on the test's
 input (sequence 0 of the 24-block workload, first 1100 user tokens), and writes
 the deviation at every depth and the tolerance 1.5x that deviation to
 ``stack24_tolerance.json``; and the same deviation for every block pair run as a
 2-block stack (the block-pair check), with its bound max(2e-2, 1.5x deviation).
+Every deviation is the largest over four placements of the rounding errors (round
+to nearest, and three seeds of round to nearest on a randomly scaled grid, at the same
+points): the max-norm deviation of one placement is heavy-tailed.
 It imports nothing from the CUDA path.
 
     python tests/golden/make_stack_tolerance.py
 """
+import concurrent.futures as cf
 import dataclasses
 import json
+import multiprocessing as mp
 import os
 import sys
 
@@ -36,10 +44,38 @@ from hybrid_attention_ssm_hymba_b200 import synth  # noqa: E402
 
 PREFIX = 1100
 HEADROOM = 1.5
+REALIZATIONS = 4   # round to nearest; then three seeds of the same rounding on a shifted grid
+
+_GRID = None       # numpy Generator: round x*s (s uniform in [1, 2) per element) and divide by s
+
+
+def _rne_bits(a, drop):
+    """Keep the top 32 - drop bits of each fp32 value, rounding to nearest (ties to even
+    for bf16, ties away for tf32, as the path rounds)."""
+    u = np.asarray(a, np.float32).view(np.uint32).astype(np.uint64)
+    u = u + (0x7FFF + ((u >> 16) & 1) if drop == 16 else (1 << (drop - 1)))
+    return (u & ((1 << 32) - (1 << drop))).astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def _round_bits(a, drop):
+    """Round to nearest at the path's precision.  In a shifted-grid realization each value
+    is rounded as x*s and divided back by s: the error keeps the round-to-nearest
+    distribution (half an ulp of the value's own binade position, now random) but lands
+    on every element independently of the first realization."""
+    if _GRID is None:
+        return _rne_bits(a, drop)
+    a = np.asarray(a, np.float64)
+    sc = 1.0 + _GRID.random(a.shape)
+    return _rne_bits(a * sc, drop) / sc
 
 
 def _bf16(a):
-    return synth.round_bf16(np.asarray(a, np.float32)).astype(np.float64)
+    return _round_bits(a, 16)
+
+
+def _tf32(a):
+    """Round to the tf32 significand (10 explicit bits)."""
+    return _round_bits(a, 13)
 
 
 def _layer_bf16_storage(x, p, s, kv_in=None):
@@ -57,9 +93,15 @@ def _layer_bf16_storage(x, p, s, kv_in=None):
         Bm, Cm = xdbc[:, s.dt_rank:s.dt_rank + s.d_state], xdbc[:, s.dt_rank + s.d_state:]
         dt = _bf16(O.softplus(O.linear(dt_low, p["w_dt"]) + p["b_dt"]))
         y = O.selective_scan(parts["x_ssm"][b], dt, O.ssm_decay_rate(p["a_log"]), Bm, Cm)
+        if s.d_state == 16:   # the scan's products take tf32 operands: y at tf32 precision
+            y = _tf32(y)
         ys.append(_bf16(parts["g"][b] * y))
-    z = _bf16(O.branch_fusion(ya, np.stack(ys), p["beta1"], p["beta2"], s.rms_eps))
-    return O.linear(z, p["w_out"]), (k, v)
+    # fused branch norm: the normalised Z is never stored; beta is folded into W_out,
+    # which is stored in bf16, and out_proj scales each row by its 1/rms in fp32
+    ones1, ones2 = np.ones_like(p["beta1"]), np.ones_like(p["beta2"])
+    zn = O.branch_fusion(ya, np.stack(ys), ones1, ones2, s.rms_eps)
+    w_scaled = _bf16(p["w_out"] * np.concatenate([p["beta1"], p["beta2"]])[None, :])
+    return O.linear(zn, w_scaled), (k, v)
 
 
 def stack_bf16_storage(x, meta, params, shapes):
@@ -78,7 +120,11 @@ def stack_bf16_storage(x, meta, params, shapes):
     return hidden
 
 
-def main():
+def realization(r):
+    """Deviations of one rounding realization (r = 0: nearest; r > 0: nearest on a shifted grid, seed r):
+    the 24-block stack by depth, and every block pair."""
+    global _GRID
+    _GRID = None if r == 0 else np.random.default_rng(9000 + r)
     wl = synth.workload("hymba1p5b_stack24")
     x, meta = synth.layer_inputs(wl, batch=1, seq_len=PREFIX)
     params = [synth.layer_params(wl, i) for i in range(len(wl.layers))]
@@ -86,16 +132,37 @@ def main():
     _, exact = O.stack_forward(x, meta, params, shapes, return_hidden=True)
     model = stack_bf16_storage(x, meta, params, shapes)
     dev = [float(np.abs(m - e).max() / np.abs(e).max()) for m, e in zip(model, exact)]
+    return dev, block_pair_deviations(full=wl)
+
+
+def main():
+    """The max-norm deviation of one realization is heavy-tailed (a few rows with small
+    branch RMS carry the largest relative error after the norm), so each bound is taken
+    over REALIZATIONS placements of the rounding errors: the maximum deviation, times
+    HEADROOM."""
+    os.environ.setdefault("OMP_NUM_THREADS", "2")
+    with cf.ProcessPoolExecutor(REALIZATIONS, mp_context=mp.get_context("spawn")) as ex:
+        runs = list(ex.map(realization, range(REALIZATIONS)))
+    dev = [max(r[0][i] for r in runs) for i in range(len(runs[0][0]))]
+    wl = synth.workload("hymba1p5b_stack24")
     out = {
         "workload": wl.name, "sequence": 0, "prefix_user_tokens": PREFIX,
         "metric": "max|g-o| / max|o| of the block output h",
+        "realizations": "round to nearest, and 3 seeds of round to nearest on a randomly scaled grid, at the same points",
         "bf16_storage_deviation_by_depth": dev,
+        "deviation_24_blocks_by_realization": [r[0][-1] for r in runs],
         "headroom": HEADROOM,
         "tolerance_24_blocks": HEADROOM * dev[-1],
-        "derivation": "deviation of the oracle with bf16 rounding at the bf16 path's storage points "
-                      "from the exact fp64 oracle (this script; oracle functions only)",
+        "derivation": "largest deviation over the realizations of the oracle with rounding at the bf16 "
+                      "path's rounding points from the exact fp64 oracle (this script; oracle functions "
+                      "only), times the headroom",
     }
-    out["block_pairs"] = block_pair_bounds(full=wl)
+    pairs = {}
+    for key in runs[0][1]:
+        ds = [r[1][key][1] for r in runs]
+        pairs[key] = {"prefix_user_tokens": runs[0][1][key][0], "bf16_storage_deviation": max(ds),
+                      "by_realization": ds, "tolerance": max(2e-2, HEADROOM * max(ds))}
+    out["block_pairs"] = pairs
     with open(os.path.join(HERE, "stack24_tolerance.json"), "w") as f:
         json.dump(out, f, indent=1)
     print(json.dumps({k: out[k] for k in ("tolerance_24_blocks",)}), [round(d, 4) for d in dev])
@@ -105,12 +172,12 @@ def main():
 PAIR_CASES = ((0, 1100), (7, 160))
 
 
-def block_pair_bounds(full):
+def block_pair_deviations(full):
     """Every block pair (2k, 2k+1) run as a 2-block stack from X, as the block-pair GPU
-    test runs it: the bf16-storage deviation of the pair's output for each checked
-    (sequence, prefix), and the bound max(2e-2, HEADROOM x deviation).  One hybrid-head
-    layer meets 2e-2; a pair composes two layers and two SwiGLU FFNs, and its
-    bf16-storage deviation alone can exceed 2e-2."""
+    test runs it: the deviation of the pair's output for each checked (sequence,
+    prefix).  The bound is max(2e-2, HEADROOM x deviation): one hybrid-head layer meets
+    2e-2; a pair composes two layers and two SwiGLU FFNs, and its rounding deviation
+    alone can exceed 2e-2."""
     res = {}
     for pair in range(len(full.layers) // 2):
         wl = synth.workload(full.name)
@@ -121,9 +188,7 @@ def block_pair_bounds(full):
             shapes = [dataclasses.replace(s, batch=1, seq_len=L) for s in wl.layers]
             exact = O.stack_forward(x[b:b + 1, :L], meta, params, shapes)
             model = stack_bf16_storage(x[b:b + 1, :L], meta, params, shapes)[-1]
-            d = float(np.abs(model - exact).max() / np.abs(exact).max())
-            res[f"{pair}/{b}"] = {"prefix_user_tokens": L, "bf16_storage_deviation": d,
-                                  "tolerance": max(2e-2, HEADROOM * d)}
+            res[f"{pair}/{b}"] = (L, float(np.abs(model - exact).max() / np.abs(exact).max()))
     return res
 
 
