@@ -68,19 +68,20 @@ def _visible_pairs(T: int, M: int, W: int) -> int:
     return int((np.minimum(i + 1, W + 1) + np.maximum(0, np.minimum(M, i - W))).sum())
 
 
-def stage_work(s: synth.LayerShape):
+def stage_work(s: synth.LayerShape, dt_in_scan: bool = False):
     """Algorithmic work of each stage of one layer launch: (FLOPs, HBM bytes).
 
     FLOPs count the dense contractions only (2 per multiply-add; attention 4 dh per
     visible pair per query head).  Bytes are the compulsory traffic: every operand read
     once and every result written once (weights included), in the layer's dtype, with
-    B|C in fp32."""
+    B|C in fp32.  dt_in_scan: the scan computes dt from dt_low itself (no dt_proj stage;
+    the scan reads dt_low and W_dt instead of dt)."""
     es = 2 if s.dtype == "bf16" else 4
     rows = s.batch * s.T
     wa, di, n, r, d = s.attn_width, s.d_inner, s.d_state, s.dt_rank, s.d_model
     kv_out = 0 if s.kv_mode == synth.KV_CONSUME else 2 * s.kv_width
     pairs = s.batch * _visible_pairs(s.T, s.n_meta, s.window)
-    return {
+    work = {
         "in_proj": (2.0 * d * s.n_in * rows, es * (rows * d + s.n_in * d + rows * (wa + kv_out + 2 * di))),
         "x_proj": (2.0 * di * s.xproj_width * rows, es * (rows * di + s.xproj_width * di + rows * r) + 4 * rows * 2 * n),
         "dt_proj": (2.0 * r * di * rows, es * (rows * r + di * r + rows * di) + 4 * di),
@@ -93,11 +94,16 @@ def stage_work(s: synth.LayerShape):
                         if s.dtype == "bf16" else es * 2 * rows * (wa + di) + 4 * (wa + di)),
         "out_proj": (2.0 * (wa + di) * d * rows, es * (rows * (wa + di) + d * (wa + di) + rows * d)),
     }
+    if dt_in_scan:
+        fl_dt, _ = work.pop("dt_proj")
+        fl, by = work["scan"]
+        work["scan"] = (fl + fl_dt, by - es * rows * di + es * (rows * r + di * r) + 4 * di)
+    return work
 
 
 KERNEL_NAMES = {"in_proj": "gemm_bf16_tc, tcgen05", "x_proj": "gemm_bf16_tc, tcgen05",
                 "dt_proj": "gemm_bf16_tc, tcgen05", "attention": "attn_fwd_tc, tcgen05",
-                "scan": "scan_tc_kernel, tcgen05 tf32", "branch_norm": "row_ssq_kernel + scale_cols_kernel",
+                "scan": "scan_tc_kernel, tcgen05 tf32 (+ dt projection, bf16)", "branch_norm": "row_ssq_kernel + scale_cols_kernel",
                 "out_proj": "gemm_bf16_tc, tcgen05, two accumulators"}
 
 # dominant bound of each stage: a dense contraction on the tensor cores or HBM traffic
@@ -122,13 +128,13 @@ def _traffic(stage: str):
     return rec["dram_bytes_per_launch"]
 
 
-def stage_rooflines(s: synth.LayerShape, stage_us, peaks):
+def stage_rooflines(s: synth.LayerShape, stage_us, peaks, dt_in_scan=False):
     """Per stage: achieved work rate against its peak (measured peaks), and the layer's
     roofline time (sum over stages of the slower of its FLOP and byte times)."""
     out, t_roof = {}, 0.0
     hbm = peaks["hbm_gbs"] * 1e9
     tc = peaks["bf16_tflops_sustained"] * 1e12
-    for name, (fl, by) in stage_work(s).items():
+    for name, (fl, by) in stage_work(s, dt_in_scan).items():
         t = stage_us[name] * 1e-6
         t_roof += max(fl / tc, by / hbm)
         if STAGE_BOUND[name] == "tensor":
@@ -351,11 +357,13 @@ def run_native(args, rank, world, local_rank):
         and not stack else None
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    # this library's kernels per step: in_proj, x_proj, dt_proj, attention, scan, out_proj and
-    # the norm stage (bf16: row sums + beta-scaled W_out; fp32: in-place norm); a stack adds
-    # two pre-norms and the two FFN GEMMs per block, and the meta prepend
-    per_layer = 8 if dtype == "bf16" else 7
-    n_launch_per_step = per_layer * len(wl.layers) + (4 * len(wl.layers) + 1 if stack else 0)
+    # this library's kernels per step: in_proj, x_proj, dt_proj (unless the scan computes dt),
+    # attention, scan, out_proj and the norm stage (bf16: row sums + beta-scaled W_out; fp32:
+    # in-place norm); a stack adds two pre-norms and the two FFN GEMMs per block, and the
+    # meta prepend
+    dt_in_scan = [H.hymba_layer_fuses_dt_proj(c) for c in cfgs]
+    n_launch_per_step = sum((8 if dtype == "bf16" else 7) - int(f) for f in dt_in_scan) + \
+        (4 * len(wl.layers) + 1 if stack else 0)
 
     def step(xin, stage_events=None):
         if stack:
@@ -418,7 +426,9 @@ def run_native(args, rank, world, local_rank):
         per_stage = {name: float(np.mean([stage_ev[k][i].elapsed_time(stage_ev[k][i + 1]) for k in range(n_stage)]))
                      for i, name in enumerate(H.STAGES)}
         stages = {n: round(v * 1e3, 2) for n, v in per_stage.items()}  # microseconds
-        stage_roof, t_roof_us = stage_rooflines(s0, stages, peaks)
+        if dt_in_scan[0]:   # stage 2 launches nothing: dt is computed inside the scan
+            stages.pop("dt_proj")
+        stage_roof, t_roof_us = stage_rooflines(s0, stages, peaks, dt_in_scan[0])
         top = max(stages, key=stages.get)   # the dominant kernel of the step
         r = stage_roof[top]
         roofline = {"kernel": f"{top} ({KERNEL_NAMES[top]})", "bound": r["bound"], "achieved": r["achieved"],

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhymba.so
 ENTRY_POINTS = (
     "hymba_status_string", "hymba_workspace_size", "hymba_stack_workspace_size", "hymba_layer_fwd",
     "hymba_stack_fwd", "hymba_workspace_status", "hymba_layer_fwd_events", "hymba_gemm", "hymba_selective_scan",
-    "hymba_attention", "hymba_branch_norm", "hymba_rmsnorm", "hymba_layer_fwd_noalloc",
+    "hymba_attention", "hymba_branch_norm", "hymba_rmsnorm", "hymba_layer_fwd_noalloc", "hymba_layer_fuses_dt_proj",
 )
 
 # size of the library-owned scratch block behind hymba_layer_fwd_noalloc (HYMBA_NOALLOC_SCRATCH_BYTES)
@@ -53,6 +53,7 @@ _VP, _SZ, _I, _F = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_floa
 _SIGS = {
     "hymba_status_string": (ctypes.c_char_p, [_I]),
     "hymba_workspace_size": (_SZ, [ctypes.POINTER(hymba_cfg_t)]),
+    "hymba_layer_fuses_dt_proj": (ctypes.c_int, [ctypes.POINTER(hymba_cfg_t)]),
     "hymba_stack_workspace_size": (_SZ, [ctypes.POINTER(hymba_cfg_t), _I]),
     "hymba_layer_fwd": (_I, [_VP, _VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t),
                              _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -143,6 +144,10 @@ def hymba_status_string(status: int) -> str:
 
 def hymba_workspace_size(cfg: hymba_cfg_t) -> int:
     return load().hymba_workspace_size(ctypes.byref(cfg))
+
+
+def hymba_layer_fuses_dt_proj(cfg: hymba_cfg_t) -> bool:
+    return bool(load().hymba_layer_fuses_dt_proj(ctypes.byref(cfg)))
 
 
 def hymba_stack_workspace_size(cfgs: Sequence[hymba_cfg_t]) -> int:

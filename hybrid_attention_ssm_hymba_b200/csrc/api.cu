@@ -150,6 +150,17 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   sd.d_state = c.d_state;
   sd.bf16 = c.dtype == HYMBA_BF16;
   sd.status = status;
+  // bf16 with d_state 16 and dt_rank <= 64: dt_proj runs inside the tensor-core scan
+  // (dt = softplus(dt_low W_dt^T + b_dt) per block, never stored)
+  {
+    hy::ScanDesc f = sd;
+    f.dt_low = dtlow;
+    f.w_dt = w.w_dt;
+    f.b_dt = w.b_dt;
+    f.dt_rank = c.dt_rank;
+    if (hy::scan_tc_fuses_dt(f)) sd = f;
+  }
+  const bool fused_dt = sd.dt_low != nullptr;
   // bf16: the branch norm is fused into out_proj -- the rows of Z are not rewritten;
   // their two sums of squares are read once, beta is folded into W_out's columns, and
   // out_proj applies the two 1 / rms row scales to its two accumulators
@@ -208,17 +219,19 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   gx.status = status;
   if ((e = gemm(gx, c.dtype, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
 
-  // 3 dt_proj with softplus(. + b_dt)
+  // 3 dt_proj with softplus(. + b_dt) (in the scan when fused_dt)
   mark(2);
-  GemmDesc gd;
-  gd.a = dtlow;
-  gd.a_rows = rows;
-  gd.K = c.dt_rank;
-  gd.w = w.w_dt;
-  gd.N = di;
-  gd.seg[gd.nseg++] = seg(0, di, dt, di, f32out, hy::SEG_SOFTPLUS_BIAS, w.b_dt);
-  gd.status = status;
-  if ((e = gemm(gd, c.dtype, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
+  if (!fused_dt) {
+    GemmDesc gd;
+    gd.a = dtlow;
+    gd.a_rows = rows;
+    gd.K = c.dt_rank;
+    gd.w = w.w_dt;
+    gd.N = di;
+    gd.seg[gd.nseg++] = seg(0, di, dt, di, f32out, hy::SEG_SOFTPLUS_BIAS, w.b_dt);
+    gd.status = status;
+    if ((e = gemm(gd, c.dtype, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
+  }
 
   // 4 attention heads -> Z[:, :wa]
   mark(3);
@@ -348,6 +361,22 @@ const char* hymba_status_string(hymba_status_t s) {
     case HYMBA_ERR_TIMEOUT: return "a kernel's bounded wait timed out";
   }
   return "unknown status";
+}
+
+int hymba_layer_fuses_dt_proj(const hymba_cfg_t* cfg) {
+  if (validate_cfg(cfg) != HYMBA_OK) return 0;
+  // the same test run_layer makes, on 256-byte aligned workspace buffers and weights
+  hy::ScanDesc f;
+  f.x = f.gate = f.dt_low = f.w_dt = reinterpret_cast<const void*>(256);
+  f.y = reinterpret_cast<void*>(256);
+  f.bc = reinterpret_cast<const float*>(256);
+  f.b_dt = reinterpret_cast<const float*>(256);
+  f.y_ld = static_cast<long long>(cfg->n_q_heads) * cfg->head_dim + cfg->d_inner;
+  f.d_inner = cfg->d_inner;
+  f.d_state = cfg->d_state;
+  f.dt_rank = cfg->dt_rank;
+  f.bf16 = cfg->dtype == HYMBA_BF16;
+  return hy::scan_tc_fuses_dt(f) ? 1 : 0;
 }
 
 size_t hymba_workspace_size(const hymba_cfg_t* cfg) {

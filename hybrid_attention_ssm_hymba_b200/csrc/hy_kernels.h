@@ -84,11 +84,19 @@ struct ScanDesc {
   int batch, T, d_inner, d_state;
   bool bf16;
   unsigned* status;
+  // Fused dt projection (tensor-core scan only): when dt_low is set, dt is not read but
+  // computed as softplus(dt_low w_dt^T + b_dt); dt_low [batch*T, dt_rank] bf16 (row
+  // stride dt_rank), w_dt [d_inner, dt_rank] bf16, b_dt [d_inner] fp32.
+  const void* dt_low = nullptr; const void* w_dt = nullptr; const float* b_dt = nullptr;
+  int dt_rank = 0;
 };
 cudaError_t launch_scan(const ScanDesc& s, cudaStream_t st);
 // The tensor-core form of the scan (bf16, d_state = 16, 16-byte aligned operands);
 // cudaErrorNotSupported for any other configuration.
 cudaError_t launch_scan_tc(const ScanDesc& s, cudaStream_t st);
+// Whether launch_scan_tc takes this configuration with the dt projection fused
+// (bf16, d_state 16, dt_rank a multiple of 8 up to 64, 16-byte aligned operands).
+bool scan_tc_fuses_dt(const ScanDesc& s);
 
 struct AttnDesc {
   const void* q; long long q_ld;     // [batch*T, q_ld], head h at column h*dh

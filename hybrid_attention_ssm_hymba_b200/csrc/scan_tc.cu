@@ -23,29 +23,25 @@
 // where some channel of the CTA exceeds that (very large dt) is run on the CUDA
 // cores by the plain recurrence instead, for every channel of the CTA.
 //
+// dt itself can come in two ways: read from memory, or computed here from the
+// low-rank projection (the layer's dt_proj, softplus(dt_low W_dt^T + b_dt)) as a fifth
+// product per block, W_dt[c,:] . dt_low[t,:] with the CTA's 128 rows of W_dt resident
+// in shared memory, so dt never goes through HBM.
+//
 // CTA = 128 channels of one sequence, all T steps, 384 threads:
 //   warps 0-7   channel warps: warp w owns TMEM lane quadrant w % 4 (channel
 //               32 (w % 4) + lane) and half w / 4 of each block's 64 steps; half 1
 //               also carries the state chain and the large-decay path.
 //   warps 8-9   mask C B^T (TMEM lanes 0-63 = t) into M, transpose B into B^T.
-//   warp 10     TMA producer (x, dt, gate [64 t][128 c] bf16; B|C [64 t][32] fp32).
+//   warp 10     TMA producer (x, dt, gate [64 t][128 c] bf16 or dt_low [64 t][64] bf16;
+//               B|C [64 t][32] fp32).
 //   warp 11     TMEM owner and MMA issuer.
 // Operands: V, G' in TMEM (A from TMEM); M, B^T, C in shared memory, 128-byte
-// swizzled K-major; accumulators Y (64 columns), dG (16), C B^T (64) in TMEM; all
-// products kind::tf32 with fp32 accumulation.  y goes out through a double-buffered
-// shared tile and TMA stores.
+// swizzled K-major; accumulators Y (64 columns), dG (16), C B^T (64), W_dt dt_low^T (64)
+// in TMEM; the scan's products kind::tf32, the dt projection kind::f16 (bf16), all with
+// fp32 accumulation.  y goes out through a double-buffered shared tile and TMA stores.
 #include "hy_common.cuh"
 #include "hy_kernels.h"
-
-// W = gate 2^(r - lambda) as gate / 2^(lambda - r) with a Newton reciprocal on the FMA
-// pipe (1) or a second SFU exp2 (0).
-#ifndef HY_SCANTC_W_NEWTON
-#define HY_SCANTC_W_NEWTON 0
-#endif
-// Paired fp32 arithmetic (fma/mul.rn.f32x2) for two steps at a time.
-#ifndef HY_SCANTC_PACK
-#define HY_SCANTC_PACK 1
-#endif
 
 namespace hy {
 namespace {
@@ -62,26 +58,38 @@ constexpr int TILE_B = Q * CH * 2;       // [64 t][128 c] bf16
 constexpr int BC_B = Q * 2 * NST * 4;    // [64 t][B 16 | C 16] fp32, 128-byte rows
 constexpr int MT_B = Q * Q * 4;          // M [t][s] tf32: two K chunks of [64 rows][128 B]
 constexpr int BT_B = NST * Q * 4;        // B^T [n][s] tf32: two K chunks of [16 rows][128 B]
+constexpr int KR = 64;                   // dt_rank capacity of the fused dt projection
+constexpr int DL_B = Q * KR * 2;         // dt_low [64 t][64 r] bf16, 128-byte swizzle
+constexpr int WD_B = CH * KR * 2;        // W_dt rows of the CTA [128 c][64 r] bf16, 128-byte swizzle
 
-constexpr int OFF_X = 0;
-constexpr int OFF_DT = OFF_X + STAGES * TILE_B;
-constexpr int OFF_G = OFF_DT + STAGES * TILE_B;
-constexpr int OFF_BC = OFF_G + STAGES * TILE_B;
-constexpr int OFF_MT = OFF_BC + STAGES * BC_B;   // also the rows C B^T reads past the last B|C tile
-constexpr int OFF_BT = OFF_MT + MT_B;
-constexpr int OFF_Y = OFF_BT + BT_B;
-constexpr int OFF_S = OFF_Y + 2 * TILE_B;        // float [2][128]: half-block decay sums
-constexpr int OFF_BAR = OFF_S + 2 * CH * 4;
-constexpr int NBAR = 2 * STAGES + 4 * 2 + 3;
-constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
-constexpr int SMEM_TOTAL = SMEM_USED + 1024;     // + alignment of the base to 1024
-static_assert(OFF_BC % 1024 == 0 && OFF_MT % 1024 == 0 && OFF_BT % 1024 == 0, "swizzled tiles 1024-aligned");
-static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
+// Shared-memory layout (offsets from a 1024-aligned base).  Stage s holds x, gate, the
+// dt tile (dt, or dt_low when FUSED) and B|C of one 64-step block.
+template <bool FUSED>
+struct Lay {
+  static constexpr int D_B = FUSED ? DL_B : TILE_B;
+  static constexpr int OFF_X = 0;
+  static constexpr int OFF_G = OFF_X + STAGES * TILE_B;
+  static constexpr int OFF_BC = OFF_G + STAGES * TILE_B;
+  static constexpr int OFF_MT = OFF_BC + STAGES * BC_B;   // also the rows C B^T reads past the last B|C tile
+  static constexpr int OFF_BT = OFF_MT + MT_B;
+  static constexpr int OFF_D = OFF_BT + BT_B;
+  static constexpr int OFF_WD = OFF_D + STAGES * D_B;     // FUSED only
+  static constexpr int OFF_Y = OFF_WD + (FUSED ? WD_B : 0);
+  static constexpr int OFF_S = OFF_Y + 2 * TILE_B;        // float [2][128]: half-block decay sums
+  static constexpr int OFF_BAR = OFF_S + 2 * CH * 4;
+  static constexpr int NBAR = 2 * STAGES + 4 * 2 + 4;
+  static constexpr int SMEM_TOTAL = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment of the base
+  static_assert(OFF_BC % 1024 == 0 && OFF_MT % 1024 == 0 && OFF_BT % 1024 == 0 && OFF_D % 1024 == 0 &&
+                    OFF_WD % 1024 == 0 && D_B % 1024 == 0,
+                "swizzled tiles 1024-aligned");
+  static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
+};
 
 // TMEM columns (512 allocated)
 constexpr uint32_t COL_Y = 0;      // [2][64]
-constexpr uint32_t COL_V = 128;    // [2][64]
-constexpr uint32_t COL_W = 256;    // [2][64]
+constexpr uint32_t COL_W = 128;    // [2][64]; dt of a block that runs the plain recurrence
+constexpr uint32_t COL_V = 256;    // [64]
+constexpr uint32_t COL_DT = 320;   // [64]: W_dt dt_low^T (FUSED)
 constexpr uint32_t COL_MR = 384;   // [64]: C B^T (lanes 0-63)
 constexpr uint32_t COL_DG = 448;   // [2][16]
 constexpr uint32_t COL_GP = 480;   // [2][16]
@@ -89,41 +97,51 @@ constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_N64 = idesc_tf32(128, 64);
 constexpr uint32_t IDESC_N16 = idesc_tf32(128, 16);
+constexpr uint32_t IDESC_DT = idesc_bf16(128, 64, false, false);
 
 HY_DEV float bf2f(uint16_t u) { return __uint_as_float(static_cast<uint32_t>(u) << 16); }
 // fp32 -> tf32 bit pattern, magnitude rounded to nearest (ties away from zero), on the
 // integer pipe: add half of the dropped 13-bit field and clear it.
 HY_DEV uint32_t tf32_round(float x) { return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u; }
-// 1/e for e > 0 on the FMA pipe: exponent-negating initial guess (relative error below
-// 1/8) and three Newton steps r <- r (2 - e r), each squaring the error (below 1e-7).
-HY_DEV float recip_newton(float e) {
-  float r = __uint_as_float(0x7EF311C3u - __float_as_uint(e));
-#pragma unroll
-  for (int i = 0; i < 3; ++i) r = r * fmaf(-e, r, 2.f);
-  return r;
+// Two lanes of softplus(z) = max(z, 0) + log1p(e^-|z|), the log1p as u q(u) with the
+// same degree-5 polynomial as softplus_f, on paired fp32 operations.
+HY_DEV float2 softplus2(float2 z) {
+  const float2 a = __fmul2_rn(make_float2(fabsf(z.x), fabsf(z.y)),
+                              make_float2(-1.4426950408889634f, -1.4426950408889634f));
+  const float2 u = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+  float2 q = __ffma2_rn(make_float2(-0.02386615f, -0.02386615f), u, make_float2(0.10121477f, 0.10121477f));
+  q = __ffma2_rn(q, u, make_float2(-0.21004209f, -0.21004209f));
+  q = __ffma2_rn(q, u, make_float2(0.32520431f, 0.32520431f));
+  q = __ffma2_rn(q, u, make_float2(-0.49936107f, -0.49936107f));
+  q = __ffma2_rn(q, u, make_float2(0.99999160f, 0.99999160f));
+  return __ffma2_rn(u, q, make_float2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
 }
 
+template <bool FUSED>
 __global__ void __launch_bounds__(NTHR, 1)
-    scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDT,
+    scan_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmD,
                    const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmBC,
-                   const __grid_constant__ CUtensorMap tmY, const float* __restrict__ a_log, int T, int Di,
+                   const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmWD,
+                   const float* __restrict__ a_log, const float* __restrict__ b_dt, int T, int Di,
                    unsigned* status) {
+  using L = Lay<FUSED>;
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
   uint64_t* full = bars;                    // [STAGES] TMA landed
   uint64_t* empty = full + STAGES;          // [STAGES] last MMA reading the stage done
   uint64_t* vready = empty + STAGES;        // [2] V, W in TMEM (256 arrivals)
-  uint64_t* dgready = vready + 2;           // [2] Y = V M^T and dG = V B done
+  uint64_t* dgready = vready + 2;           // [2] Y = V M^T and dG = V B done (V free)
   uint64_t* gready = dgready + 2;           // [2] G' in TMEM (128 arrivals)
   uint64_t* yready = gready + 2;            // [2] Y complete
   uint64_t* mraw = yready + 2;              // C B^T in TMEM
   uint64_t* mready = mraw + 1;              // M and B^T in shared memory (64 arrivals)
-  uint64_t* mma_done = mready + 1;
+  uint64_t* dtready = mready + 1;           // W_dt dt_low^T in TMEM (FUSED)
+  uint64_t* mma_done = dtready + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* sS = reinterpret_cast<float*>(sm + OFF_S);
+  float* sS = reinterpret_cast<float*>(sm + L::OFF_S);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c0 = blockIdx.x * CH, b = blockIdx.y;
@@ -142,6 +160,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     mbar_init(mraw, 1);
     mbar_init(mready, 64);
+    mbar_init(dtready, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -153,10 +172,11 @@ __global__ void __launch_bounds__(NTHR, 1)
   pdl_wait();
   if (threadIdx.x == 320) {
     tma_prefetch(&tmX);
-    tma_prefetch(&tmDT);
+    tma_prefetch(&tmD);
     tma_prefetch(&tmG);
     tma_prefetch(&tmBC);
     tma_prefetch(&tmY);
+    if (FUSED) tma_prefetch(&tmWD);
   }
   tc_fence_before();
   __syncthreads();
@@ -171,11 +191,12 @@ __global__ void __launch_bounds__(NTHR, 1)
       for (; k < nblk; ++k) {
         const int s = k % STAGES;
         if (k >= STAGES && !mbar_wait(&empty[s], ((k / STAGES) - 1) & 1u, status, abort_flag)) break;
-        mbar_arrive_expect_tx(&full[s], 3 * TILE_B + BC_B);
-        tma_load_3d(sm + OFF_X + s * TILE_B, &tmX, &full[s], c0, k * Q, b);
-        tma_load_3d(sm + OFF_DT + s * TILE_B, &tmDT, &full[s], c0, k * Q, b);
-        tma_load_3d(sm + OFF_G + s * TILE_B, &tmG, &full[s], c0, k * Q, b);
-        tma_load_3d(sm + OFF_BC + s * BC_B, &tmBC, &full[s], 0, k * Q, b);
+        mbar_arrive_expect_tx(&full[s], 2 * TILE_B + L::D_B + BC_B + (FUSED && k == 0 ? WD_B : 0));
+        if (FUSED && k == 0) tma_load_2d(sm + L::OFF_WD, &tmWD, &full[s], 0, c0);
+        tma_load_3d(sm + L::OFF_X + s * TILE_B, &tmX, &full[s], c0, k * Q, b);
+        tma_load_3d(sm + L::OFF_D + s * L::D_B, &tmD, &full[s], FUSED ? 0 : c0, k * Q, b);
+        tma_load_3d(sm + L::OFF_G + s * TILE_B, &tmG, &full[s], c0, k * Q, b);
+        tma_load_3d(sm + L::OFF_BC + s * BC_B, &tmBC, &full[s], 0, k * Q, b);
       }
       if (k < nblk) {  // aborted: let the copies already issued land before smem goes away
         int never = 0;
@@ -186,12 +207,20 @@ __global__ void __launch_bounds__(NTHR, 1)
   } else if (warp == 11) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t mt = sbase + OFF_MT, bt = sbase + OFF_BT;
-      auto issue_mraw = [&](int k) -> bool {
+      const uint32_t mt = sbase + L::OFF_MT, bt = sbase + L::OFF_BT;
+      // Block k's stage has landed: W_dt dt_low^T (FUSED) and C B^T.
+      auto issue_stage = [&](int k) -> bool {
         const int s = k % STAGES;
         if (!mbar_wait(&full[s], (k / STAGES) & 1u, status, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t bc = sbase + OFF_BC + s * BC_B;
+        if (FUSED) {
+          const uint32_t dl = sbase + L::OFF_D + s * L::D_B, wd = sbase + L::OFF_WD;
+          for (int j = 0; j < KR / 16; ++j)
+            umma_bf16_ss(tmem + COL_DT, sdesc_sw128(wd + 32 * j, 16, 1024), sdesc_sw128(dl + 32 * j, 16, 1024),
+                         IDESC_DT, j);
+          umma_commit(dtready);
+        }
+        const uint32_t bc = sbase + L::OFF_BC + s * BC_B;
         // C B^T: A = C rows (128 rows read; rows 64..127 are whatever follows the tile and
         // land in TMEM lanes nobody reads), B = B rows; K = 16 = two tf32 steps.
         for (int j = 0; j < 2; ++j)
@@ -200,31 +229,31 @@ __global__ void __launch_bounds__(NTHR, 1)
         umma_commit(mraw);
         return true;
       };
-      bool ok = nblk > 0 && issue_mraw(0);
+      bool ok = nblk > 0 && issue_stage(0);
       for (int k = 0; ok && k < nblk; ++k) {
         const int i = k & 1, s = k % STAGES;
         const uint32_t par = (k >> 1) & 1u;
         if (!mbar_wait(&vready[i], par, status, abort_flag) || !mbar_wait(mready, k & 1u, status, abort_flag)) break;
         tc_fence_after();
-        const uint32_t vcol = tmem + COL_V + 64 * i;
         // Y = V M^T (K = s, 64 = 8 steps) and dG = V B (B^T tile)
         for (int j = 0; j < 8; ++j)
-          umma_tf32_ts(tmem + COL_Y + 64 * i, vcol + 8 * j, sdesc_sw128(mt + (j >> 2) * 8192 + (j & 3) * 32, 16, 1024),
-                       IDESC_N64, j);
+          umma_tf32_ts(tmem + COL_Y + 64 * i, tmem + COL_V + 8 * j,
+                       sdesc_sw128(mt + (j >> 2) * 8192 + (j & 3) * 32, 16, 1024), IDESC_N64, j);
         for (int j = 0; j < 8; ++j)
-          umma_tf32_ts(tmem + COL_DG + 16 * i, vcol + 8 * j, sdesc_sw128(bt + (j >> 2) * 2048 + (j & 3) * 32, 16, 1024),
-                       IDESC_N16, j);
+          umma_tf32_ts(tmem + COL_DG + 16 * i, tmem + COL_V + 8 * j,
+                       sdesc_sw128(bt + (j >> 2) * 2048 + (j & 3) * 32, 16, 1024), IDESC_N16, j);
         umma_commit(&dgready[i]);
+        // the next block's dt projection and C B^T (their TMEM was read before vready / mready)
+        if (k + 1 < nblk && !issue_stage(k + 1)) break;
         if (!mbar_wait(&gready[i], par, status, abort_flag)) break;
         tc_fence_after();
         // Y += G' C^T (K = n = 16)
-        const uint32_t bc = sbase + OFF_BC + s * BC_B;
+        const uint32_t bc = sbase + L::OFF_BC + s * BC_B;
         for (int j = 0; j < 2; ++j)
           umma_tf32_ts(tmem + COL_Y + 64 * i, tmem + COL_GP + 16 * i + 8 * j, sdesc_sw128(bc + 64 + 32 * j, 16, 1024),
                        IDESC_N64, 1);
         umma_commit(&yready[i]);
         umma_commit(&empty[s]);
-        if (k + 1 < nblk && !issue_mraw(k + 1)) break;
       }
       umma_commit(mma_done);
       int never = 0;
@@ -234,8 +263,8 @@ __global__ void __launch_bounds__(NTHR, 1)
     // ------------------------------------------------------------ M = mask(C B^T), B^T
     const int t = (warp - 8) * 32 + lane;  // TMEM lane = step within the block
     const uint32_t tl = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    uint8_t* mt = sm + OFF_MT;
-    uint8_t* bt = sm + OFF_BT;
+    uint8_t* mt = sm + L::OFF_MT;
+    uint8_t* bt = sm + L::OFF_BT;
     for (int k = 0; k < nblk; ++k) {
       const int s = k % STAGES;
       bool ok = mbar_wait(mraw, k & 1u, status, abort_flag) && mbar_wait(&full[s], (k / STAGES) & 1u, status, abort_flag);
@@ -262,7 +291,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
       }
       // B^T [n][s]: element (n, s = t)
-      const uint8_t* bcrow = sm + OFF_BC + s * BC_B + t * 128;
+      const uint8_t* bcrow = sm + L::OFF_BC + s * BC_B + t * 128;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float4 q = *reinterpret_cast<const float4*>(bcrow + ((j ^ (t & 7)) << 4));
@@ -285,6 +314,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     const int cl = qd * 32 + lane, c = c0 + cl;
     const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const float A2 = c < Di ? expf(a_log[c]) * 1.4426950408889634f : 0.f;  // |A| / ln 2
+    const float bdt = FUSED && c < Di ? b_dt[c] : 0.f;
     float h[NST];
 #pragma unroll
     for (int n = 0; n < NST; ++n) h[n] = 0.f;
@@ -295,37 +325,48 @@ __global__ void __launch_bounds__(NTHR, 1)
       bool any = false;
       if (k < nblk) {
         const int s = k % STAGES, i = k & 1;
-        const uint8_t* xt = sm + OFF_X + s * TILE_B + cl * 2;
-        const uint8_t* dtt = sm + OFF_DT + s * TILE_B + cl * 2;
-        const uint8_t* gt = sm + OFF_G + s * TILE_B + cl * 2;
+        const uint8_t* xt = sm + L::OFF_X + s * TILE_B + cl * 2;
+        const uint8_t* gt = sm + L::OFF_G + s * TILE_B + cl * 2;
         fail = !__all_sync(0xffffffffu, mbar_wait(&full[s], (k / STAGES) & 1u, status, abort_flag));
-        // ---- half-block decay sum
+        // ---- dt of this half block, and its decay sum
         float dtv[32];
-#if HY_SCANTC_PACK
         float2 S2 = make_float2(0.f, 0.f);
+        if (FUSED) {
+          if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(dtready, k & 1u, status, abort_flag));
+          uint32_t z[32];
+          if (!fail) {
+            tc_fence_after();
+            tmem_ld32(tl + COL_DT + 32 * half, z);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          dtv[j] = bf2f(*reinterpret_cast<const uint16_t*>(dtt + (32 * half + j) * 256));
-          dtv[j + 1] = bf2f(*reinterpret_cast<const uint16_t*>(dtt + (32 * half + j + 1) * 256));
-          S2 = __ffma2_rn(make_float2(A2, A2), make_float2(dtv[j], dtv[j + 1]), S2);
+            for (int j = 0; j < 32; ++j) z[j] = 0u;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 d = softplus2(make_float2(__uint_as_float(z[j]) + bdt, __uint_as_float(z[j + 1]) + bdt));
+            dtv[j] = d.x;
+            dtv[j + 1] = d.y;
+            S2 = __ffma2_rn(make_float2(A2, A2), d, S2);
+          }
+        } else {
+          const uint8_t* dtt = sm + L::OFF_D + s * L::D_B + cl * 2;
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            dtv[j] = bf2f(*reinterpret_cast<const uint16_t*>(dtt + (32 * half + j) * 256));
+            dtv[j + 1] = bf2f(*reinterpret_cast<const uint16_t*>(dtt + (32 * half + j + 1) * 256));
+            S2 = __ffma2_rn(make_float2(A2, A2), make_float2(dtv[j], dtv[j + 1]), S2);
+          }
         }
         const float S = S2.x + S2.y;
-#else
-        float S = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          dtv[j] = bf2f(*reinterpret_cast<const uint16_t*>(dtt + (32 * half + j) * 256));
-          S = fmaf(A2, dtv[j], S);
-        }
-#endif
         sS[half * CH + cl] = S;
         any = bar_red_or(1, NCHT, fail || !(S <= kRange));
-        // ---- V = dt x 2^(lambda - r), W = gate 2^(r - lambda) into TMEM
+        // ---- V = dt x 2^(lambda - r), W = gate 2^(r - lambda) into TMEM.  In a block that
+        // runs the plain recurrence V is zero and the W columns carry dt instead.
         if (!fail) {
           uint32_t vr[32], wr[32];
           if (!any) {
             float mu = half ? 0.f : -S;  // lambda - r
-#if HY_SCANTC_PACK
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               const float mu0 = fmaf(A2, dtv[j], mu);
@@ -343,57 +384,43 @@ __global__ void __launch_bounds__(NTHR, 1)
               wr[j] = __float_as_uint(w.x);
               wr[j + 1] = __float_as_uint(w.y);
             }
-#else
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              mu = fmaf(A2, dtv[j], mu);
-              const int row = (32 * half + j) * 256;
-              const float xv = bf2f(*reinterpret_cast<const uint16_t*>(xt + row));
-              const float gv = bf2f(*reinterpret_cast<const uint16_t*>(gt + row));
-              const float e = ex2_approx(mu);
-              vr[j] = tf32_round(dtv[j] * xv * e);
-#if HY_SCANTC_W_NEWTON
-              wr[j] = __float_as_uint(gv * recip_newton(e));
-#else
-              wr[j] = __float_as_uint(gv * ex2_approx(-mu));
-#endif
-            }
-#endif
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) vr[j] = wr[j] = 0u;
+            for (int j = 0; j < 32; ++j) {
+              vr[j] = 0u;
+              wr[j] = __float_as_uint(dtv[j]);
+            }
           }
-          tmem_st32(tl + COL_V + 64 * i + 32 * half, vr);
-          tmem_st32(tl + COL_W + 64 * i + 32 * half, wr);
-          tmem_wait_st();
-          tc_fence_before();
+          // V has one buffer: the products of block k - 1 must have read it
+          if (k > 0) fail = !__all_sync(0xffffffffu, mbar_wait(&dgready[(k - 1) & 1], ((k - 1) >> 1) & 1u, status,
+                                                                 abort_flag));
+          if (!fail) {
+            tc_fence_after();
+            tmem_st32(tl + COL_V + 32 * half, vr);
+            tmem_st32(tl + COL_W + 64 * i + 32 * half, wr);
+            tmem_wait_st();
+            tc_fence_before();
+          }
         }
         mbar_arrive(&vready[i]);
         // ---- state chain: h entering block k, G' = h 2^(-r)  (half 1)
         if (half == 1 && !fail) {
           const float S0 = sS[cl], S1 = S;
-          if (k > 0 && !prev_any) {
-            if (__all_sync(0xffffffffu, mbar_wait(&dgready[(k - 1) & 1], ((k - 1) >> 1) & 1u, status, abort_flag))) {
-              tc_fence_after();
-              uint32_t d[16];
-              tmem_ld16(tl + COL_DG + 16 * ((k - 1) & 1), d);
-              tmem_wait_ld();
-              const float a = ex2_approx(-(pS0 + pS1)), bs = ex2_approx(-pS1);
+          if (k > 0 && !prev_any) {  // dG of block k - 1 is complete (waited above)
+            uint32_t d[16];
+            tmem_ld16(tl + COL_DG + 16 * ((k - 1) & 1), d);
+            tmem_wait_ld();
+            const float a = ex2_approx(-(pS0 + pS1)), bs = ex2_approx(-pS1);
 #pragma unroll
-              for (int n = 0; n < NST; ++n) h[n] = fmaf(a, h[n], bs * __uint_as_float(d[n]));
-            } else {
-              fail = true;
-            }
+            for (int n = 0; n < NST; ++n) h[n] = fmaf(a, h[n], bs * __uint_as_float(d[n]));
           }
-          if (!fail) {
-            uint32_t gp[16];
-            const float sc = ex2_approx(-S0);
+          uint32_t gp[16];
+          const float sc = ex2_approx(-S0);
 #pragma unroll
-            for (int n = 0; n < NST; ++n) gp[n] = any ? 0u : tf32_round(h[n] * sc);
-            tmem_st16(tl + COL_GP + 16 * i, gp);
-            tmem_wait_st();
-            tc_fence_before();
-          }
+          for (int n = 0; n < NST; ++n) gp[n] = any ? 0u : tf32_round(h[n] * sc);
+          tmem_st16(tl + COL_GP + 16 * i, gp);
+          tmem_wait_st();
+          tc_fence_before();
           pS0 = S0;
           pS1 = S1;
         }
@@ -401,32 +428,40 @@ __global__ void __launch_bounds__(NTHR, 1)
         // announced only after it, since the MMA that waits for G' frees the stage.
         if (any) {
           if (threadIdx.x == 0) bulk_wait_all();  // the store that last read this y tile is done
-          bar_sync_n(1, NCHT);
+          bar_sync_n(1, NCHT);                    // and every half's dt is in the W columns
           if (half == 1 && !fail) {
-            uint8_t* yt = sm + OFF_Y + i * TILE_B + cl * 2;
-            const uint8_t* bct = sm + OFF_BC + s * BC_B;
+            tc_fence_after();
+            uint8_t* yt = sm + L::OFF_Y + i * TILE_B + cl * 2;
+            const uint8_t* bct = sm + L::OFF_BC + s * BC_B;
 #pragma unroll 1
-            for (int t = 0; t < Q; ++t) {
-              const float dt = bf2f(*reinterpret_cast<const uint16_t*>(dtt + t * 256));
-              const float xv = bf2f(*reinterpret_cast<const uint16_t*>(xt + t * 256));
-              const float gv = bf2f(*reinterpret_cast<const uint16_t*>(gt + t * 256));
-              const float a = ex2_approx(-A2 * dt), u = dt * xv;
-              const uint8_t* row = bct + t * 128;
-              float y = 0.f;
+            for (int t0 = 0; t0 < Q; t0 += 16) {
+              uint32_t dq[16];
+              tmem_ld16(tl + COL_W + 64 * i + t0, dq);
+              tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float4 bq = *reinterpret_cast<const float4*>(row + ((j ^ (t & 7)) << 4));
-                const float4 cq = *reinterpret_cast<const float4*>(row + (((j + 4) ^ (t & 7)) << 4));
-                h[4 * j + 0] = fmaf(a, h[4 * j + 0], u * bq.x);
-                h[4 * j + 1] = fmaf(a, h[4 * j + 1], u * bq.y);
-                h[4 * j + 2] = fmaf(a, h[4 * j + 2], u * bq.z);
-                h[4 * j + 3] = fmaf(a, h[4 * j + 3], u * bq.w);
-                y = fmaf(cq.x, h[4 * j + 0], y);
-                y = fmaf(cq.y, h[4 * j + 1], y);
-                y = fmaf(cq.z, h[4 * j + 2], y);
-                y = fmaf(cq.w, h[4 * j + 3], y);
+              for (int tt = 0; tt < 16; ++tt) {
+                const int t = t0 + tt;
+                const float dt = __uint_as_float(dq[tt]);
+                const float xv = bf2f(*reinterpret_cast<const uint16_t*>(xt + t * 256));
+                const float gv = bf2f(*reinterpret_cast<const uint16_t*>(gt + t * 256));
+                const float a = ex2_approx(-A2 * dt), u = dt * xv;
+                const uint8_t* row = bct + t * 128;
+                float y = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const float4 bq = *reinterpret_cast<const float4*>(row + ((j ^ (t & 7)) << 4));
+                  const float4 cq = *reinterpret_cast<const float4*>(row + (((j + 4) ^ (t & 7)) << 4));
+                  h[4 * j + 0] = fmaf(a, h[4 * j + 0], u * bq.x);
+                  h[4 * j + 1] = fmaf(a, h[4 * j + 1], u * bq.y);
+                  h[4 * j + 2] = fmaf(a, h[4 * j + 2], u * bq.z);
+                  h[4 * j + 3] = fmaf(a, h[4 * j + 3], u * bq.w);
+                  y = fmaf(cq.x, h[4 * j + 0], y);
+                  y = fmaf(cq.y, h[4 * j + 1], y);
+                  y = fmaf(cq.z, h[4 * j + 2], y);
+                  y = fmaf(cq.w, h[4 * j + 3], y);
+                }
+                *reinterpret_cast<uint16_t*>(yt + t * 256) = bf16_bits(gv * y);
               }
-              *reinterpret_cast<uint16_t*>(yt + t * 256) = bf16_bits(gv * y);
             }
           }
         }
@@ -443,17 +478,12 @@ __global__ void __launch_bounds__(NTHR, 1)
             tmem_ld32(tl + COL_Y + 64 * i + 32 * half, yv);
             tmem_ld32(tl + COL_W + 64 * i + 32 * half, wv);
             tmem_wait_ld();
-            uint8_t* yt = sm + OFF_Y + i * TILE_B + cl * 2 + 32 * half * 256;
+            uint8_t* yt = sm + L::OFF_Y + i * TILE_B + cl * 2 + 32 * half * 256;
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-#if HY_SCANTC_PACK
               const float2 o = __fmul2_rn(make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])),
                                           make_float2(__uint_as_float(wv[j]), __uint_as_float(wv[j + 1])));
               const uint32_t p2 = pack_bf16(o.x, o.y);
-#else
-              const uint32_t p2 = pack_bf16(__uint_as_float(yv[j]) * __uint_as_float(wv[j]),
-                                            __uint_as_float(yv[j + 1]) * __uint_as_float(wv[j + 1]));
-#endif
               *reinterpret_cast<uint16_t*>(yt + j * 256) = static_cast<uint16_t>(p2);
               *reinterpret_cast<uint16_t*>(yt + (j + 1) * 256) = static_cast<uint16_t>(p2 >> 16);
             }
@@ -462,7 +492,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         fence_proxy_async_smem();
         if (bar_red_or(1, NCHT, fail || *abort_flag)) break;
         if (threadIdx.x == 0) {
-          tma_store_3d(&tmY, sm + OFF_Y + i * TILE_B, c0, jb * Q, b);
+          tma_store_3d(&tmY, sm + L::OFF_Y + i * TILE_B, c0, jb * Q, b);
           bulk_commit();
           bulk_wait_read1();  // the store before it has read its tile: that tile may be rewritten
         }
@@ -513,30 +543,66 @@ bool map3d(CUtensorMap* m, const void* base, bool f32, int batch, int T, long lo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
+// 2-D map over [rows][cols] (row stride ld elements), box = bc x br, 128-byte swizzle.
+bool map2d_sw128(CUtensorMap* m, const void* base, long long rows, long long cols, long long ld, int bc, int br) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t gs[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t bx[2] = {static_cast<cuuint32_t>(bc), static_cast<cuuint32_t>(br)}, el[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gd, gs, bx, el,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
-// bf16, d_state = 16, 16-byte aligned operands and row strides (checked by the caller).
-// Returns cudaErrorNotSupported when the configuration is not this kernel's.
-cudaError_t launch_scan_tc(const ScanDesc& s, cudaStream_t st) {
-  if (!s.bf16 || s.d_state != NST) return cudaErrorNotSupported;
-  CUtensorMap tx, td, tg, tb, ty;
-  if (!map3d(&tx, s.x, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !map3d(&td, s.dt, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !map3d(&tg, s.gate, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !map3d(&tb, s.bc, true, s.batch, s.T, 2 * NST, 2 * NST, 2 * NST, Q, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map3d(&ty, s.y, false, s.batch, s.T, s.d_inner, s.y_ld, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorNotSupported;
+bool a16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
+
+template <bool FUSED>
+cudaError_t launch_tc(const ScanDesc& s, cudaStream_t st) {
+  using L = Lay<FUSED>;
+  CUtensorMap tx, td, tg, tb, ty, tw;
+  bool ok = map3d(&tx, s.x, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+            map3d(&tg, s.gate, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+            map3d(&tb, s.bc, true, s.batch, s.T, 2 * NST, 2 * NST, 2 * NST, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            map3d(&ty, s.y, false, s.batch, s.T, s.d_inner, s.y_ld, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (FUSED) {
+    // dt_low tiles [64 t][KR r] (columns past dt_rank read as zero) and the CTA's W_dt rows
+    ok = ok && map3d(&td, s.dt_low, false, s.batch, s.T, s.dt_rank, s.dt_rank, KR, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         map2d_sw128(&tw, s.w_dt, s.d_inner, s.dt_rank, s.dt_rank, KR, CH);
+  } else {
+    ok = ok && map3d(&td, s.dt, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE);
+    tw = tx;  // unused
+  }
+  if (!ok) return cudaErrorNotSupported;
   static int attr_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 31 && !(attr_mask & (1 << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TOTAL);
+    cudaError_t e =
+        cudaFuncSetAttribute(scan_tc_kernel<FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_TOTAL);
     if (e != cudaSuccess) return e;
     attr_mask |= 1 << dev;
   }
   dim3 grid((s.d_inner + CH - 1) / CH, s.batch);
-  return launch(scan_tc_kernel, grid, dim3(NTHR), SMEM_TOTAL, st, tx, td, tg, tb, ty, s.a_log, s.T, s.d_inner,
-                s.status);
+  return launch(scan_tc_kernel<FUSED>, grid, dim3(NTHR), L::SMEM_TOTAL, st, tx, td, tg, tb, ty, tw, s.a_log, s.b_dt,
+                s.T, s.d_inner, s.status);
+}
+
+}  // namespace
+
+bool scan_tc_fuses_dt(const ScanDesc& s) {
+  return s.bf16 && s.d_state == NST && s.dt_rank > 0 && s.dt_rank <= KR && s.dt_rank % 8 == 0 &&
+         (s.d_inner * 2) % 16 == 0 && (s.y_ld * 2) % 16 == 0 && a16(s.x) && a16(s.gate) && a16(s.bc) && a16(s.y) &&
+         a16(s.dt_low) && a16(s.w_dt) && s.b_dt != nullptr;
+}
+
+// bf16, d_state = 16, 16-byte aligned operands and row strides (checked by the caller;
+// with dt_low set, scan_tc_fuses_dt).  cudaErrorNotSupported when the configuration is
+// not this kernel's.
+cudaError_t launch_scan_tc(const ScanDesc& s, cudaStream_t st) {
+  if (!s.bf16 || s.d_state != NST) return cudaErrorNotSupported;
+  if (s.dt_low) return scan_tc_fuses_dt(s) ? launch_tc<true>(s, st) : cudaErrorNotSupported;
+  return launch_tc<false>(s, st);
 }
 
 }  // namespace hy

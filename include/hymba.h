@@ -140,6 +140,16 @@ HYMBA_API hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const 
                                void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Whether the layer of `cfg` computes its dt projection ("Design formulation", the
+ * SSM head's dt = softplus(dt_low W_dt^T + b_dt)) inside the selective-scan kernel
+ * instead of as a separate GEMM: 1 for bf16 with d_state 16 and dt_rank a multiple of
+ * 8 up to 64, given 16-byte aligned weights; 0 otherwise (also for an invalid cfg).
+ * With 1, stage 2 of hymba_layer_fwd_events launches nothing and its work is part of
+ * stage 4.
+ */
+HYMBA_API int hymba_layer_fuses_dt_proj(const hymba_cfg_t* cfg);
+
+/*
  * hymba_layer_fwd with stage timing (tracing hook).  `events` holds 8 cudaEvent_t
  * (created by the caller, passed as void*): events[i] is recorded on `stream`
  * right before stage i and events[7] after the last one.  Stages:

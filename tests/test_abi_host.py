@@ -137,3 +137,15 @@ def test_noalloc_rejects_oversized_config_before_touching_a_gpu():
     w = H.make_weights({k: 16 for k in ("w_in", "w_x", "w_dt", "w_out", "a_log", "b_dt", "beta1", "beta2")})
     assert H.hymba_layer_fwd_noalloc(16, 16, w, cfg, None, None, 16, stream=0) == H.HYMBA_ERR_WORKSPACE
     assert H.hymba_layer_fwd_noalloc(16, 16, w, _cfg(batch=0), None, None, 16, stream=0) == H.HYMBA_ERR_INVALID_ARG
+
+
+def test_layer_fuses_dt_proj_only_where_the_scan_computes_dt():
+    """bf16 with d_state 16 and dt_rank <= 64 (the 350M-shaped layer) runs its dt
+    projection inside the scan; fp32, dt_rank 128 and invalid configs do not."""
+    from hybrid_attention_ssm_hymba_b200 import synth
+    assert H.hymba_layer_fuses_dt_proj(H.make_cfg(synth.workload("hymba350m_layer").first))
+    assert not H.hymba_layer_fuses_dt_proj(H.make_cfg(synth.workload("hymba1p5b_stack24").first))
+    assert not H.hymba_layer_fuses_dt_proj(H.make_cfg(synth.workload("tiny_fp32").first))
+    bad = H.make_cfg(synth.workload("hymba350m_layer").first)
+    bad.batch = 0
+    assert not H.hymba_layer_fuses_dt_proj(bad)
