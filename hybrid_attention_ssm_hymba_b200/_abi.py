@@ -65,7 +65,7 @@ _SIGS = {
                              _I, _VP, _VP, _SZ, _VP]),
     "hymba_workspace_status": (_I, [_VP, _VP]),
     "hymba_gemm": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _VP, _SZ, _VP]),
-    "hymba_selective_scan": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
+    "hymba_selective_scan": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "hymba_attention": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "hymba_branch_norm": (_I, [_VP, _VP, _VP, _I, _I, _I, _F, _I, _VP]),
     "hymba_rmsnorm": (_I, [_VP, _VP, _I, _I, _F, _I, _VP]),
@@ -207,10 +207,10 @@ def hymba_gemm(a, w, c, M: int, N: int, K: int, dtype: int, workspace, stream=No
 
 
 def hymba_selective_scan(x, dt, bc, gate, a_log, y, y_ld: int, batch: int, T: int, d_inner: int,
-                         d_state: int, dtype: int, workspace, stream=None) -> int:
+                         d_state: int, dtype: int, workspace, stream=None, a_per_state: int = 0) -> int:
     return load().hymba_selective_scan(_ptr(x), _ptr(dt), _ptr(bc), _ptr(gate), _ptr(a_log), _ptr(y),
-                                       y_ld, batch, T, d_inner, d_state, dtype, _ptr(workspace),
-                                       _nbytes(workspace), _stream(stream))
+                                       y_ld, batch, T, d_inner, d_state, int(a_per_state), dtype,
+                                       _ptr(workspace), _nbytes(workspace), _stream(stream))
 
 
 def hymba_attention(q, kv, out, out_ld: int, batch: int, T: int, n_q_heads: int, n_kv_heads: int,

@@ -72,7 +72,7 @@ hymba_status_t validate_cfg(const hymba_cfg_t* c) {
       c->dt_rank < 1 || c->ffn_dim < 0 || c->kv_mode < 0 || c->kv_mode > 2 || !(c->rms_eps >= 0.f))
     return HYMBA_ERR_INVALID_ARG;
   if (c->n_q_heads % c->n_kv_heads != 0) return HYMBA_ERR_INVALID_ARG;
-  if (c->a_per_state != 0) return HYMBA_ERR_UNSUPPORTED;
+  if (c->a_per_state != 0 && c->a_per_state != 1) return HYMBA_ERR_INVALID_ARG;
   if (!valid_state(c->d_state)) return HYMBA_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(c->batch) * (c->seq_len + c->n_meta);
   if (rows > (1ll << 31) - 1) return HYMBA_ERR_UNSUPPORTED;
@@ -150,6 +150,7 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   sd.d_state = c.d_state;
   sd.bf16 = c.dtype == HYMBA_BF16;
   sd.status = status;
+  sd.a_per_state = c.a_per_state != 0;
   // bf16 with d_state 16 and dt_rank <= 64: dt_proj runs inside the tensor-core scan
   // (dt = softplus(dt_low W_dt^T + b_dt) per block, never stored)
   {
@@ -376,6 +377,7 @@ int hymba_layer_fuses_dt_proj(const hymba_cfg_t* cfg) {
   f.d_state = cfg->d_state;
   f.dt_rank = cfg->dt_rank;
   f.bf16 = cfg->dtype == HYMBA_BF16;
+  f.a_per_state = cfg->a_per_state != 0;
   return hy::scan_tc_fuses_dt(f) ? 1 : 0;
 }
 
@@ -576,9 +578,10 @@ hymba_status_t hymba_gemm(const void* a, const void* w, void* c, int M, int N, i
 
 hymba_status_t hymba_selective_scan(const void* x, const void* dt, const float* bc, const void* gate,
                                     const float* a_log, void* y, int y_ld, int batch, int T, int d_inner,
-                                    int d_state, hymba_dtype_t dtype, void* workspace, size_t ws_bytes,
-                                    void* stream) {
-  if (!x || !dt || !bc || !gate || !a_log || !y || batch < 1 || T < 1 || d_inner < 1 || y_ld < d_inner)
+                                    int d_state, int a_per_state, hymba_dtype_t dtype, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  if (!x || !dt || !bc || !gate || !a_log || !y || batch < 1 || T < 1 || d_inner < 1 || y_ld < d_inner ||
+      (a_per_state != 0 && a_per_state != 1))
     return HYMBA_ERR_INVALID_ARG;
   if (dtype != HYMBA_BF16 && dtype != HYMBA_F32) return HYMBA_ERR_INVALID_ARG;
   if (!valid_state(d_state)) return HYMBA_ERR_UNSUPPORTED;
@@ -596,6 +599,7 @@ hymba_status_t hymba_selective_scan(const void* x, const void* dt, const float* 
   s.d_inner = d_inner;
   s.d_state = d_state;
   s.bf16 = dtype == HYMBA_BF16;
+  s.a_per_state = a_per_state != 0;
   s.status = static_cast<unsigned*>(workspace);
   return cuda_status(hy::launch_scan(s, static_cast<cudaStream_t>(stream)));
 }

@@ -84,6 +84,7 @@ struct ScanDesc {
   int batch, T, d_inner, d_state;
   bool bf16;
   unsigned* status;
+  bool a_per_state = false;  // a_log [d_inner, d_state] instead of [d_inner]
   // Fused dt projection (tensor-core scan only): when dt_low is set, dt is not read but
   // computed as softplus(dt_low w_dt^T + b_dt); dt_low [batch*T, dt_rank] bf16 (row
   // stride dt_rank), w_dt [d_inner, dt_rank] bf16, b_dt [d_inner] fp32.

@@ -697,6 +697,81 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
   }
 }
 
+// Per-state decay, A[c, n] = -exp(a_log[c, n]): the recurrence with one exp2 per state
+// and step (the block forms above need one decay per channel).  TPC = N / NS lanes share
+// a channel, each holding NS of its states; C_t . h_t is summed over those lanes by
+// shuffles.  One pass over T per channel.
+template <typename TI, int N>
+__global__ void __launch_bounds__(128) scan_ps_kernel(const ScanParams p) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int NS = N < 8 ? N : 8;
+  constexpr int TPC = N / NS;          // lanes per channel
+  constexpr int CPW = 32 / TPC;        // channels per warp
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ch = lane / TPC, slice = lane % TPC;
+  const int c = (blockIdx.x * 4 + warp) * CPW + ch;
+  const int b = blockIdx.y;
+  const bool valid = c < p.Di;
+  const int cc = valid ? c : 0;
+  const int n0 = slice * NS;
+  float A2[NS], h[NS];
+#pragma unroll
+  for (int n = 0; n < NS; ++n) {
+    A2[n] = -expf(p.a_log[static_cast<long long>(cc) * N + n0 + n]) * 1.4426950408889634f;
+    h[n] = 0.f;
+  }
+  const long long row0 = static_cast<long long>(b) * p.T;
+  const TI* xp = static_cast<const TI*>(p.x) + row0 * p.Di + cc;
+  const TI* dp = static_cast<const TI*>(p.dt) + row0 * p.Di + cc;
+  const TI* gp = static_cast<const TI*>(p.gate) + row0 * p.Di + cc;
+  const float* bp = p.bc + row0 * 2 * N + n0;
+  TI* yp = static_cast<TI*>(p.y) + row0 * p.y_ld + cc;
+#pragma unroll 1
+  for (int t = 0; t < p.T; ++t) {
+    const float d = to_f<TI>(dp[static_cast<long long>(t) * p.Di]);
+    const float u = d * to_f<TI>(xp[static_cast<long long>(t) * p.Di]);
+    const float* brow = bp + static_cast<long long>(t) * 2 * N;
+    float y = 0.f;
+#pragma unroll
+    for (int j = 0; j < NS; j += 4) {
+      const float4 bb = __ldg(reinterpret_cast<const float4*>(brow + j));
+      const float4 cq = __ldg(reinterpret_cast<const float4*>(brow + N + j));
+      const float bv[4] = {bb.x, bb.y, bb.z, bb.w}, cv[4] = {cq.x, cq.y, cq.z, cq.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        h[j + e] = fmaf(ex2_approx(A2[j + e] * d), h[j + e], u * bv[e]);
+        y = fmaf(cv[e], h[j + e], y);
+      }
+    }
+#pragma unroll
+    for (int off = 1; off < TPC; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
+    if (valid && slice == 0)
+      yp[static_cast<long long>(t) * p.y_ld] = from_f<TI>(to_f<TI>(gp[static_cast<long long>(t) * p.Di]) * y);
+  }
+}
+
+template <typename TI, int N>
+cudaError_t launch_ps(const ScanDesc& s, cudaStream_t st) {
+  constexpr int NS = N < 8 ? N : 8;
+  constexpr int CPB = 4 * (32 / (N / NS));  // channels per block
+  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
+  dim3 grid((s.d_inner + CPB - 1) / CPB, s.batch);
+  return launch(scan_ps_kernel<TI, N>, grid, dim3(128), 0, st, p);
+}
+
+template <typename TI>
+cudaError_t launch_ps_t(const ScanDesc& s, cudaStream_t st) {
+  switch (s.d_state) {
+    case 16: return launch_ps<TI, 16>(s, st);
+    case 32: return launch_ps<TI, 32>(s, st);
+    case 64: return launch_ps<TI, 64>(s, st);
+    case 128: return launch_ps<TI, 128>(s, st);
+    case 256: return launch_ps<TI, 256>(s, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -819,6 +894,10 @@ cudaError_t launch_t(const ScanDesc& s, cudaStream_t st) {
 
 cudaError_t launch_scan(const ScanDesc& s, cudaStream_t st) {
   if (s.batch <= 0 || s.T <= 0 || s.d_inner <= 0) return cudaSuccess;
+  if (s.a_per_state) {
+    if (s.dt_low) return cudaErrorNotSupported;  // the fused dt projection is the block form's
+    return s.bf16 ? launch_ps_t<__nv_bfloat16>(s, st) : launch_ps_t<float>(s, st);
+  }
   return s.bf16 ? launch_t<__nv_bfloat16>(s, st) : launch_t<float>(s, st);
 }
 

@@ -80,7 +80,7 @@ typedef struct {
   int d_state;      /* N: 16, 32, 64, 128 or 256 */
   int n_ssm_heads;  /* recorded only: the per-channel scan does not depend on it */
   int dt_rank;      /* R: width of dt_low */
-  int a_per_state;  /* 0: A_log [Di] (supported); 1: A_log [Di, N] (HYMBA_ERR_UNSUPPORTED) */
+  int a_per_state;  /* 0: A_log [Di] (one decay per channel); 1: A_log [Di, N] (one per channel and state) */
   int kv_mode;      /* hymba_kv_mode_t */
   int ffn_dim;      /* F: SwiGLU FFN width for hymba_stack_fwd; 0 = no FFN */
   float rms_eps;    /* RMSNorm epsilon (1e-6) */
@@ -143,7 +143,8 @@ HYMBA_API hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const 
  * Whether the layer of `cfg` computes its dt projection ("Design formulation", the
  * SSM head's dt = softplus(dt_low W_dt^T + b_dt)) inside the selective-scan kernel
  * instead of as a separate GEMM: 1 for bf16 with d_state 16 and dt_rank a multiple of
- * 8 up to 64, given 16-byte aligned weights; 0 otherwise (also for an invalid cfg).
+ * 8 up to 64 and one decay per channel (a_per_state 0), given 16-byte aligned weights;
+ * 0 otherwise (also for an invalid cfg).
  * With 1, stage 2 of hymba_layer_fwd_events launches nothing and its work is part of
  * stage 4.
  */
@@ -209,6 +210,9 @@ HYMBA_API hymba_status_t hymba_gemm(const void* a, const void* w, void* c, int M
  * alpha_ij and Y_ssm = G . alpha W_SSM X~):
  *   for each sequence b and channel c, from h = 0:
  *     h_t = exp(A_c dt_t) h_{t-1} + dt_t x_t B_t,   y_t = gate_t * (C_t . h_t),   A_c = -exp(a_log[c])
+ *   a_per_state = 0: a_log [d_inner];  1: a_log [d_inner, d_state] and the state component n
+ *     decays by exp(A_{c,n} dt_t), A_{c,n} = -exp(a_log[c, n]) (the Mamba variant with a
+ *     diagonal A per channel)
  *   x, dt, gate [batch*T, d_inner] dtype (dt > 0 already discretised; gate = SiLU(G_raw))
  *   bc   [batch*T, 2*d_state] fp32, B_t then C_t
  *   y    written at y + row*y_ld, dtype
@@ -216,7 +220,7 @@ HYMBA_API hymba_status_t hymba_gemm(const void* a, const void* w, void* c, int M
  */
 HYMBA_API hymba_status_t hymba_selective_scan(const void* x, const void* dt, const float* bc,
                                     const void* gate, const float* a_log, void* y, int y_ld,
-                                    int batch, int T, int d_inner, int d_state,
+                                    int batch, int T, int d_inner, int d_state, int a_per_state,
                                     hymba_dtype_t dtype, void* workspace, size_t ws_bytes,
                                     void* stream);
 

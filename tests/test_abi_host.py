@@ -54,7 +54,7 @@ def _cfg(**kw):
     (dict(head_dim=64), H.HYMBA_ERR_UNSUPPORTED),
     (dict(d_state=24), H.HYMBA_ERR_UNSUPPORTED),
     (dict(n_meta=12), H.HYMBA_ERR_UNSUPPORTED),
-    (dict(a_per_state=1), H.HYMBA_ERR_UNSUPPORTED),
+    (dict(a_per_state=2), H.HYMBA_ERR_INVALID_ARG),
     (dict(dt_rank=40), H.HYMBA_ERR_UNSUPPORTED),
     (dict(dtype=7), H.HYMBA_ERR_INVALID_ARG),
 ])
@@ -113,8 +113,10 @@ def test_stage_validation():
     assert H.load().hymba_gemm(None, 1, 1, 8, 16, 8, 1, 1, 256, None) == H.HYMBA_ERR_INVALID_ARG
     assert H.load().hymba_gemm(1, 1, 1, 8, 24, 8, 1, 1, 256, None) == H.HYMBA_ERR_UNSUPPORTED
     assert H.load().hymba_gemm(1, 1, 1, 8, 16, 8, 1, 1, 16, None) == H.HYMBA_ERR_WORKSPACE
-    assert H.load().hymba_selective_scan(1, 1, 1, 1, 1, 1, 64, 1, 10, 64, 24, 1, 1, 256,
+    assert H.load().hymba_selective_scan(1, 1, 1, 1, 1, 1, 64, 1, 10, 64, 24, 0, 1, 1, 256,
                                          None) == H.HYMBA_ERR_UNSUPPORTED
+    assert H.load().hymba_selective_scan(1, 1, 1, 1, 1, 1, 64, 1, 10, 64, 16, 2, 1, 1, 256,
+                                         None) == H.HYMBA_ERR_INVALID_ARG
     assert H.load().hymba_attention(1, 1, 1, 256, 1, 10, 2, 1, 64, 0, -1, 1, 1, 256,
                                     None) == H.HYMBA_ERR_UNSUPPORTED
     assert H.load().hymba_attention(1, 1, 1, 256, 1, 10, 3, 2, 128, 0, -1, 1, 1, 256,
@@ -149,3 +151,13 @@ def test_layer_fuses_dt_proj_only_where_the_scan_computes_dt():
     bad = H.make_cfg(synth.workload("hymba350m_layer").first)
     bad.batch = 0
     assert not H.hymba_layer_fuses_dt_proj(bad)
+
+
+def test_per_state_decay_layer_is_accepted():
+    """a_per_state = 1 (A_log [d_inner, d_state]) is a supported layer configuration: it has a
+    workspace size and does not fold the dt projection into the scan."""
+    from hybrid_attention_ssm_hymba_b200 import synth
+    import dataclasses
+    c = H.make_cfg(dataclasses.replace(synth.workload("hymba350m_layer").first, a_per_state=1))
+    assert H.hymba_workspace_size(c) > 0
+    assert not H.hymba_layer_fuses_dt_proj(c)

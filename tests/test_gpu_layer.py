@@ -130,6 +130,20 @@ def test_layer_edge_configs(kw):
     assert_close(g, ref, "bf16", f"edge {kw}")
 
 
+@pytest.mark.parametrize("name,kw", [("tiny_fp32", {}), ("hymba350m_layer", dict(batch=2, seq_len=300))])
+def test_layer_per_state_decay(name, kw):
+    """a_per_state = 1: A_log [d_inner, d_state], the SSM head with one decay per channel and
+    state, through the whole layer."""
+    wl = synth.workload(name, a_per_state=1, **kw)
+    assert wl.first.a_per_state == 1
+    x, meta = synth.layer_inputs(wl)
+    ps, dps = _upload(wl)
+    assert ps[0]["a_log"].shape == (wl.first.d_inner, wl.first.d_state)
+    g = _gpu_layers(wl, dps, x, meta)
+    ref, _ = O.layer_forward(x, meta, ps[0], wl.first)
+    assert_close(g, ref, wl.first.dtype, f"{name} per-state A")
+
+
 def test_kv_sharing_consumer_equals_standalone_layer():
     """A consumer fed the producer's K/V equals a standalone layer whose W_K, W_V
     rows would produce that K/V (same Q, SSM and output weights)."""

@@ -56,6 +56,7 @@ def test_gemm_full_size_sampled_rows(M, N, K):
 
 def _scan_ref(inp, B, T, Di, N, chans=None):
     chans = np.arange(Di) if chans is None else np.asarray(chans)
+    # a_log is [Di] or [Di, N] (per-state decay); ssm_decay_rate keeps the shape
     x = inp["x"].reshape(B, T, Di)[:, :, chans]
     dt = inp["dt"].reshape(B, T, Di)[:, :, chans]
     g = inp["g"].reshape(B, T, Di)[:, :, chans]
@@ -69,7 +70,7 @@ def _run_scan(inp, B, T, Di, N, dtype):
     ws = host.workspace(256)
     H.check(H.hymba_selective_scan(dev(inp["x"], dtype), dev(inp["dt"], dtype), fp32(inp["bc"]),
                                    dev(inp["g"], dtype), fp32(inp["a_log"]), y, Di, B, T, Di, N,
-                                   DT[dtype], ws), "scan")
+                                   DT[dtype], ws, a_per_state=int(inp["a_log"].ndim == 2)), "scan")
     status_ok(ws)
     return to_np(y)
 
@@ -111,6 +112,16 @@ def test_scan_block_form_hands_large_decay_blocks_to_the_recurrence():
     dt[1, 650:670, 100] = 6.0    # block 10 (60 steps), tile 0
     inp["dt"] = synth.round_bf16(dt.reshape(B * T, Di))
     assert_close(_run_scan(inp, B, T, Di, N, "bf16"), _scan_ref(inp, B, T, Di, N), "bf16", "scan mixed blocks")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,T,Di,N", [(2, 300, 64, 16), (1, 200, 40, 32), (1, 130, 24, 128), (1, 33, 16, 256)])
+def test_scan_per_state_decay(dtype, B, T, Di, N):
+    """A_log [Di, N]: every state component decays at its own rate (the recurrence kernel),
+    including channel counts that are not a multiple of the channels per block."""
+    inp = synth.scan_inputs(26, B, T, Di, N, dtype=dtype, a_per_state=True)
+    assert inp["a_log"].shape == (Di, N)
+    assert_close(_run_scan(inp, B, T, Di, N, dtype), _scan_ref(inp, B, T, Di, N), dtype, "scan per-state A")
 
 
 def test_scan_long_decay_small_dt():
