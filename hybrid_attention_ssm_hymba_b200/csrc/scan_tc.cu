@@ -320,14 +320,11 @@ __global__ void __launch_bounds__(NTHR, 1)
     for (int n = 0; n < NST; ++n) h[n] = 0.f;
     float pS0 = 0.f, pS1 = 0.f;  // previous block's half sums (chain)
     bool prev_any = false;
-    uint32_t z[32];            // W_dt dt_low^T of the next block, loaded ahead (FUSED)
-    bool z_loaded = false;
     for (int k = 0; k <= nblk; ++k) {
       bool fail = false;
       bool any = false;
-      const int i = k & 1, s = k % STAGES;
-      float S = 0.f;
       if (k < nblk) {
+        const int s = k % STAGES, i = k & 1;
         const uint8_t* xt = sm + L::OFF_X + s * TILE_B + cl * 2;
         const uint8_t* gt = sm + L::OFF_G + s * TILE_B + cl * 2;
         fail = !__all_sync(0xffffffffu, mbar_wait(&full[s], (k / STAGES) & 1u, status, abort_flag));
@@ -335,20 +332,16 @@ __global__ void __launch_bounds__(NTHR, 1)
         float dtv[32];
         float2 S2 = make_float2(0.f, 0.f);
         if (FUSED) {
-          if (!fail && !z_loaded) {
-            fail = !__all_sync(0xffffffffu, mbar_wait(dtready, k & 1u, status, abort_flag));
-            if (!fail) {
-              tc_fence_after();
-              tmem_ld32(tl + COL_DT + 32 * half, z);
-            }
-          }
+          if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(dtready, k & 1u, status, abort_flag));
+          uint32_t z[32];
           if (!fail) {
+            tc_fence_after();
+            tmem_ld32(tl + COL_DT + 32 * half, z);
             tmem_wait_ld();
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) z[j] = 0u;
           }
-          z_loaded = false;
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
             const float2 d = softplus2(make_float2(__uint_as_float(z[j]) + bdt, __uint_as_float(z[j + 1]) + bdt));
@@ -365,7 +358,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             S2 = __ffma2_rn(make_float2(A2, A2), make_float2(dtv[j], dtv[j + 1]), S2);
           }
         }
-        S = S2.x + S2.y;
+        const float S = S2.x + S2.y;
         sS[half * CH + cl] = S;
         any = bar_red_or(1, NCHT, fail || !(S <= kRange));
         // ---- V = dt x 2^(lambda - r), W = gate 2^(r - lambda) into TMEM.  In a block that
@@ -405,52 +398,18 @@ __global__ void __launch_bounds__(NTHR, 1)
             tc_fence_after();
             tmem_st32(tl + COL_V + 32 * half, vr);
             tmem_st32(tl + COL_W + 64 * i + 32 * half, wr);
+            tmem_wait_st();
+            tc_fence_before();
           }
         }
-      }
-      // ---- TMEM reads while the stores drain: block k - 1's Y and W rows (its output)
-      // and dG (the chain)
-      uint32_t yv[32], wv[32], d[16];
-      const int jb = k - 1, ib = jb & 1;
-      bool have_y = false;
-      if (k > 0 && !fail) {
-        fail = !__all_sync(0xffffffffu, mbar_wait(&yready[ib], (jb >> 1) & 1u, status, abort_flag));
-        if (!fail && !prev_any) {
-          tc_fence_after();
-          tmem_ld32(tl + COL_Y + 64 * ib + 32 * half, yv);
-          tmem_ld32(tl + COL_W + 64 * ib + 32 * half, wv);
-          have_y = true;
-        }
-      }
-      const bool chain_dg = k < nblk && half == 1 && k > 0 && !prev_any && !fail;
-      if (chain_dg) tmem_ld16(tl + COL_DG + 16 * ((k - 1) & 1), d);  // complete: dgready waited above
-      if (k < nblk) {
-        if (!fail) {
-          tmem_wait_st();
-          tc_fence_before();
-        }
         mbar_arrive(&vready[i]);
-      }
-      tmem_wait_ld();
-      // ---- output of block k - 1: y = W * Y into its y tile (stored after the barrier)
-      if (have_y) {
-        uint8_t* yt = sm + L::OFF_Y + ib * TILE_B + cl * 2 + 32 * half * 256;
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float2 o = __fmul2_rn(make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])),
-                                      make_float2(__uint_as_float(wv[j]), __uint_as_float(wv[j + 1])));
-          const uint32_t p2 = pack_bf16(o.x, o.y);
-          *reinterpret_cast<uint16_t*>(yt + j * 256) = static_cast<uint16_t>(p2);
-          *reinterpret_cast<uint16_t*>(yt + (j + 1) * 256) = static_cast<uint16_t>(p2 >> 16);
-        }
-      }
-      if (k < nblk) {
-        const uint8_t* xt = sm + L::OFF_X + s * TILE_B + cl * 2;
-        const uint8_t* gt = sm + L::OFF_G + s * TILE_B + cl * 2;
         // ---- state chain: h entering block k, G' = h 2^(-r)  (half 1)
         if (half == 1 && !fail) {
           const float S0 = sS[cl], S1 = S;
-          if (chain_dg) {
+          if (k > 0 && !prev_any) {  // dG of block k - 1 is complete (waited above)
+            uint32_t d[16];
+            tmem_ld16(tl + COL_DG + 16 * ((k - 1) & 1), d);
+            tmem_wait_ld();
             const float a = ex2_approx(-(pS0 + pS1)), bs = ex2_approx(-pS1);
 #pragma unroll
             for (int n = 0; n < NST; ++n) h[n] = fmaf(a, h[n], bs * __uint_as_float(d[n]));
@@ -508,26 +467,42 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
         if (half == 1) mbar_arrive(&gready[i]);
       }
-      if (k > 0) fence_proxy_async_smem();  // the y tile of block k - 1 is complete
-      // the next block's dt projection, read ahead of the barrier (issued after vready)
-      if (FUSED && k + 1 < nblk && !fail) {
-        if (__all_sync(0xffffffffu, mbar_wait(dtready, (k + 1) & 1u, status, abort_flag))) {
-          tc_fence_after();
-          tmem_ld32(tl + COL_DT + 32 * half, z);
-          z_loaded = true;
-        } else {
-          fail = true;
+      // ---- output of block k - 1: y = W * Y into the y tile, TMA store
+      if (k > 0) {
+        const int jb = k - 1, i = jb & 1;
+        if (!fail) {
+          fail = !__all_sync(0xffffffffu, mbar_wait(&yready[i], (jb >> 1) & 1u, status, abort_flag));
+          if (!fail && !prev_any) {
+            tc_fence_after();
+            uint32_t yv[32], wv[32];
+            tmem_ld32(tl + COL_Y + 64 * i + 32 * half, yv);
+            tmem_ld32(tl + COL_W + 64 * i + 32 * half, wv);
+            tmem_wait_ld();
+            uint8_t* yt = sm + L::OFF_Y + i * TILE_B + cl * 2 + 32 * half * 256;
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float2 o = __fmul2_rn(make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])),
+                                          make_float2(__uint_as_float(wv[j]), __uint_as_float(wv[j + 1])));
+              const uint32_t p2 = pack_bf16(o.x, o.y);
+              *reinterpret_cast<uint16_t*>(yt + j * 256) = static_cast<uint16_t>(p2);
+              *reinterpret_cast<uint16_t*>(yt + (j + 1) * 256) = static_cast<uint16_t>(p2 >> 16);
+            }
+          }
         }
-      }
-      if (bar_red_or(1, NCHT, fail || *abort_flag)) break;
-      if (k > 0 && threadIdx.x == 0) {
-        tma_store_3d(&tmY, sm + L::OFF_Y + ib * TILE_B, c0, jb * Q, b);
-        bulk_commit();
-        bulk_wait_read1();  // the store before it has read its tile: that tile may be rewritten
+        fence_proxy_async_smem();
+        if (bar_red_or(1, NCHT, fail || *abort_flag)) break;
+        if (threadIdx.x == 0) {
+          tma_store_3d(&tmY, sm + L::OFF_Y + i * TILE_B, c0, jb * Q, b);
+          bulk_commit();
+          bulk_wait_read1();  // the store before it has read its tile: that tile may be rewritten
+        }
+      } else if (fail) {
+        if (bar_red_or(1, NCHT, true)) break;
+      } else {
+        if (bar_red_or(1, NCHT, *abort_flag != 0)) break;
       }
       if (k < nblk) prev_any = any;
     }
-    tmem_wait_ld();
     if (threadIdx.x == 0) bulk_wait_all();
   }
   tc_fence_before();
