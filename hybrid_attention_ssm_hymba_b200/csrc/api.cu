@@ -113,6 +113,35 @@ bool weights_ok(const hymba_weights_t* w, const hymba_cfg_t& c, bool need_ffn) {
   return true;
 }
 
+// The attention heads and the SSM heads of a layer are independent until the branch
+// norm: the attention runs on a second stream of the library's (one per device, made on
+// first use), forked from the caller's stream after in_proj and joined back before the
+// norm, so that its CTAs and the scan's fill the SMs together.
+cudaStream_t side_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev] = nullptr;
+  return streams[dev];
+}
+
+// Joins the side stream back into the caller's stream once (at join() or on any return).
+struct SideJoin {
+  cudaStream_t st = nullptr;
+  cudaEvent_t done = nullptr;
+  cudaError_t join() {
+    if (!done) return cudaSuccess;
+    const cudaError_t e = cudaStreamWaitEvent(st, done, 0);
+    cudaEventDestroy(done);
+    done = nullptr;
+    return e;
+  }
+  ~SideJoin() { join(); }
+};
+
 // One layer.  x: meta mode when meta != nullptr, else [rows, d] holding X~.
 // resid_out: when true the out_proj adds into `out` (out = out + Z W_out^T).
 hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t& w, const hymba_cfg_t& c,
@@ -207,6 +236,43 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   cudaError_t e = gemm(gi, c.dtype, st);
   if (e != cudaSuccess) return HYMBA_ERR_CUDA;
 
+  // 4 attention heads -> Z[:, :wa], on the side stream unless stage events are recorded
+  // (then every stage runs in order on st)
+  hy::AttnDesc ad;
+  ad.q = q;
+  ad.q_ld = wa;
+  ad.k = kv_k;
+  ad.v = kv_v;
+  ad.kv_ld = wkv;
+  ad.out = z;
+  ad.out_ld = wa + di;
+  ad.batch = c.batch;
+  ad.T = T;
+  ad.n_q_heads = c.n_q_heads;
+  ad.n_kv_heads = c.n_kv_heads;
+  ad.head_dim = c.head_dim;
+  ad.n_meta = c.n_meta;
+  ad.window = c.window;
+  ad.bf16 = c.dtype == HYMBA_BF16;
+  ad.status = status;
+  cudaStream_t side = events ? nullptr : side_stream();
+  SideJoin joiner;
+  joiner.st = st;
+  if (side) {
+    cudaEvent_t forked = nullptr, done = nullptr;
+    if (cudaEventCreateWithFlags(&forked, cudaEventDisableTiming) != cudaSuccess) return HYMBA_ERR_CUDA;
+    const bool ok = cudaEventRecord(forked, st) == cudaSuccess && cudaStreamWaitEvent(side, forked, 0) == cudaSuccess;
+    cudaEventDestroy(forked);
+    if (!ok || cudaEventCreateWithFlags(&done, cudaEventDisableTiming) != cudaSuccess) return HYMBA_ERR_CUDA;
+    const cudaError_t ea = hy::launch_attention(ad, side);
+    if (cudaEventRecord(done, side) != cudaSuccess) {
+      cudaEventDestroy(done);
+      return HYMBA_ERR_CUDA;
+    }
+    joiner.done = done;
+    if (ea != cudaSuccess) return HYMBA_ERR_CUDA;
+  }
+
   // 2 x_proj
   mark(1);
   GemmDesc gx;
@@ -234,30 +300,13 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
     if ((e = gemm(gd, c.dtype, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
   }
 
-  // 4 attention heads -> Z[:, :wa]
   mark(3);
-  hy::AttnDesc ad;
-  ad.q = q;
-  ad.q_ld = wa;
-  ad.k = kv_k;
-  ad.v = kv_v;
-  ad.kv_ld = wkv;
-  ad.out = z;
-  ad.out_ld = wa + di;
-  ad.batch = c.batch;
-  ad.T = T;
-  ad.n_q_heads = c.n_q_heads;
-  ad.n_kv_heads = c.n_kv_heads;
-  ad.head_dim = c.head_dim;
-  ad.n_meta = c.n_meta;
-  ad.window = c.window;
-  ad.bf16 = c.dtype == HYMBA_BF16;
-  ad.status = status;
-  if ((e = hy::launch_attention(ad, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
+  if (!side && (e = hy::launch_attention(ad, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
 
   // 5 selective scan + gate -> Z[:, wa:]
   mark(4);
-  if ((e = hy::launch_scan(sd, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
+  e = hy::launch_scan(sd, st);
+  if (joiner.join() != cudaSuccess || e != cudaSuccess) return HYMBA_ERR_CUDA;  // the norm reads all of Z
 
   // 6 per-branch RMSNorm and beta
   mark(5);
