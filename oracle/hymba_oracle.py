@@ -40,7 +40,9 @@ blocks are pre-norm residual around the mixer and a SwiGLU FFN.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 against closed forms, brute force, special cases that reduce to library
-routines and the invariants the pages imply.  No function is "parity unpinned".
+routines and the invariants the pages imply, and the generation step
+(``layer_prefill_state``, ``layer_decode_step``) by ``tests/test_oracle_decode.py``
+against the longer prefill it must reproduce.  No function is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -287,6 +289,64 @@ def layer_forward(x, meta, p: Dict[str, np.ndarray], s, kv_in: Optional[Tuple] =
     if return_parts:
         return out, (k, v), dict(parts, y_attn=y_attn, y_ssm=y_ssm, z=z)
     return out, (k, v)
+
+
+# ---------------------------------------------------------------------------
+# generation: one new token from the KV cache and the SSM state
+
+def layer_prefill_state(x, meta, p: Dict[str, np.ndarray], s, kv_in: Optional[Tuple] = None):
+    """layer_forward plus what generating the next token needs afterwards: the layer's
+    K/V over all T rows (the attention heads' cache, [B, T, Hkv*dh] each) and the SSM
+    heads' state after the last row, h_T [B, Di, N] -- the fixed-size state the SSM
+    heads carry where attention keeps a growing cache ([R] "Efficiency and KV cache
+    optimization").  Returns (out [B, T, d], (K, V), h_T)."""
+    out, (k, v), parts = layer_forward(x, meta, p, s, kv_in=kv_in, return_parts=True)
+    hs = []
+    for b in range(out.shape[0]):
+        xdbc = linear(parts["x_ssm"][b], p["w_x"])
+        dt = softplus(linear(xdbc[:, :s.dt_rank], p["w_dt"]) + f64(p["b_dt"]))
+        _, h = selective_scan(parts["x_ssm"][b], dt, ssm_decay_rate(p["a_log"]),
+                              xdbc[:, s.dt_rank:s.dt_rank + s.d_state],
+                              xdbc[:, s.dt_rank + s.d_state:s.dt_rank + 2 * s.d_state], return_state=True)
+        hs.append(h)
+    return out, (k, v), np.stack(hs)
+
+
+def layer_decode_step(x_t, p: Dict[str, np.ndarray], s, kv_cache: Tuple, h, pos: int):
+    """One new token per sequence at row ``pos`` (the number of rows already in the
+    cache, meta rows included): x_t [B, d] -> out_t [B, d].  The same definitions as
+    layer_forward applied to row ``pos`` of a (pos + 1)-row sequence: the token's query
+    attends over the cached keys and its own under the visibility rule (causal, window
+    W, meta always visible); the SSM heads advance their state one step,
+    h <- exp(A dt) h + dt x B, y = C . h ([R] "Design formulation").
+
+    kv_cache = (K, V) [B, pos, Hkv*dh] for a layer with its own K/V (the new row is
+    appended), or the producer's (K, V) [B, pos + 1, Hkv*dh] already holding the new row
+    for a consuming layer.  h [B, Di, N].  Returns (out_t, (K, V) with pos + 1 rows,
+    h_new)."""
+    xt = f64(x_t)[:, None, :]
+    B = xt.shape[0]
+    parts = split_in_proj(linear(xt, p["w_in"]), s)
+    if s.kv_mode == KV_CONSUME:
+        k, v = f64(kv_cache[0]), f64(kv_cache[1])
+    else:
+        k = np.concatenate([f64(kv_cache[0]), parts["k"]], axis=1)
+        v = np.concatenate([f64(kv_cache[1]), parts["v"]], axis=1)
+    assert k.shape[1] == pos + 1, "the cache must hold rows [0, pos]"
+    y_attn = np.stack([attention(parts["q"][b], k[b], v[b], s.n_q_heads, s.n_kv_heads,
+                                 s.n_meta, s.window, rows=np.array([pos])) for b in range(B)])
+    A = ssm_decay_rate(p["a_log"])
+    xdbc = linear(parts["x_ssm"], p["w_x"])
+    dt = softplus(linear(xdbc[..., :s.dt_rank], p["w_dt"]) + f64(p["b_dt"]))
+    ys, hs = [], []
+    for b in range(B):
+        y, hb = selective_scan(parts["x_ssm"][b], dt[b], A, xdbc[b, :, s.dt_rank:s.dt_rank + s.d_state],
+                               xdbc[b, :, s.dt_rank + s.d_state:s.dt_rank + 2 * s.d_state], h0=h[b],
+                               return_state=True)
+        ys.append(silu(parts["g_raw"][b]) * y)
+        hs.append(hb)
+    z = branch_fusion(y_attn, np.stack(ys), p["beta1"], p["beta2"], s.rms_eps)
+    return linear(z, p["w_out"])[:, 0], (k, v), np.stack(hs)
 
 
 def swiglu_ffn(x, w_gate_up, w_down):
