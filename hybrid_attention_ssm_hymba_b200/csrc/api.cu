@@ -180,7 +180,7 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   sd.bf16 = c.dtype == HYMBA_BF16;
   sd.status = status;
   sd.a_per_state = c.a_per_state != 0;
-  // bf16 with d_state 16 and dt_rank <= 64: dt_proj runs inside the tensor-core scan
+  // bf16 with d_state 16 and dt_rank 64: dt_proj runs inside the tensor-core scan
   // (dt = softplus(dt_low W_dt^T + b_dt) per block, never stored)
   {
     hy::ScanDesc f = sd;

@@ -96,7 +96,7 @@ cudaError_t launch_scan(const ScanDesc& s, cudaStream_t st);
 // cudaErrorNotSupported for any other configuration.
 cudaError_t launch_scan_tc(const ScanDesc& s, cudaStream_t st);
 // Whether launch_scan_tc takes this configuration with the dt projection fused
-// (bf16, d_state 16, dt_rank a multiple of 8 up to 64, 16-byte aligned operands).
+// (bf16, d_state 16, dt_rank 64, one decay per channel, 16-byte aligned operands).
 bool scan_tc_fuses_dt(const ScanDesc& s);
 
 struct AttnDesc {

@@ -591,7 +591,7 @@ cudaError_t launch_tc(const ScanDesc& s, cudaStream_t st) {
 }  // namespace
 
 bool scan_tc_fuses_dt(const ScanDesc& s) {
-  return s.bf16 && s.d_state == NST && !s.a_per_state && s.dt_rank > 0 && s.dt_rank <= KR && s.dt_rank % 8 == 0 &&
+  return s.bf16 && s.d_state == NST && !s.a_per_state && s.dt_rank == KR &&
          (s.d_inner * 2) % 16 == 0 && (s.y_ld * 2) % 16 == 0 && a16(s.x) && a16(s.gate) && a16(s.bc) && a16(s.y) &&
          a16(s.dt_low) && a16(s.w_dt) && s.b_dt != nullptr;
 }

@@ -142,9 +142,9 @@ HYMBA_API hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const 
 /*
  * Whether the layer of `cfg` computes its dt projection ("Design formulation", the
  * SSM head's dt = softplus(dt_low W_dt^T + b_dt)) inside the selective-scan kernel
- * instead of as a separate GEMM: 1 for bf16 with d_state 16 and dt_rank a multiple of
- * 8 up to 64 and one decay per channel (a_per_state 0), given 16-byte aligned weights;
- * 0 otherwise (also for an invalid cfg).
+ * instead of as a separate GEMM: 1 for bf16 with d_state 16, dt_rank 64 and one decay
+ * per channel (a_per_state 0), given 16-byte aligned weights; 0 otherwise (also for an
+ * invalid cfg).
  * With 1, stage 2 of hymba_layer_fwd_events launches nothing and its work is part of
  * stage 4.
  */
