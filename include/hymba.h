@@ -121,6 +121,12 @@ HYMBA_API size_t hymba_stack_workspace_size(const hymba_cfg_t* cfgs, int n_layer
  *   out     [B, T, d] dtype; meta rows are kept so the next layer sees [meta; X] state
  *   workspace >= hymba_workspace_size(cfg) bytes, 256-byte aligned; its first 256
  *           bytes hold the status word (reset by this call)
+ * Streams: all work is ordered on `stream`.  The attention heads run on a second,
+ * non-blocking stream the library creates on its first call on each device (forked
+ * from `stream` after the input projection with an event and joined back before the
+ * branch norm), so the call behaves as one stream-ordered operation and can be
+ * captured into a CUDA graph once the first call on the device has been made
+ * outside the capture.
  */
 HYMBA_API hymba_status_t hymba_layer_fwd(const void* x, const void* meta, const hymba_weights_t* w,
                                const hymba_cfg_t* cfg, const void* kv_in, void* kv_out,
@@ -178,8 +184,8 @@ HYMBA_API hymba_status_t hymba_layer_fwd_events(const void* x, const void* meta,
  *   - A cfg whose hymba_workspace_size(cfg) exceeds HYMBA_NOALLOC_SCRATCH_BYTES
  *     returns HYMBA_ERR_WORKSPACE before anything runs; use hymba_layer_fwd there.
  *   - The first call on a device looks up the block's device address (once per
- *     device, with that device current).  Make that first call before any stream
- *     capture on the device.
+ *     device, with that device current) and creates the layer's second stream (see
+ *     hymba_layer_fwd).  Make that first call before any stream capture on the device.
  *   - Every call on a device shares the block, which keeps the last call's
  *     contents; the call clears its status word and overwrites every intermediate
  *     before reading it.  Calls whose execution overlaps on the GPU (different
