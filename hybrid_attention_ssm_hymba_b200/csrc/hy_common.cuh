@@ -73,31 +73,32 @@ HY_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status, volatile
 }
 
 // ------------------------------------------------------------------ shared-memory loads
-// Explicit ld.shared (32-bit shared addresses).  Not volatile: they may be scheduled
-// freely; callers order them against other agents' writes through mbarriers.
+// Explicit ld.shared (32-bit shared addresses).  Volatile: an asm statement without
+// memory operands would otherwise count as reading no memory and could be moved across
+// the (volatile) mbarrier waits that order these loads after other agents' writes.
 HY_DEV float4 lds_f4(uint32_t a) {
   float4 v;
-  asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
   return v;
 }
 HY_DEV float2 lds_f2(uint32_t a) {
   float2 v;
-  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
   return v;
 }
 HY_DEV float lds_f32(uint32_t a) {
   float v;
-  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
   return v;
 }
 HY_DEV uint32_t lds_u32(uint32_t a) {
   uint32_t v;
-  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 HY_DEV uint32_t lds_u16(uint32_t a) {
   unsigned short v;
-  asm("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
   return v;
 }
 
