@@ -38,7 +38,7 @@ import numpy as np
 _STREAM = {
     "x": 1, "meta": 2,
     "w_in": 10, "w_x": 11, "w_dt": 12, "w_out": 13, "a_log": 14, "dt0": 15,
-    "beta1": 16, "beta2": 17, "w_gate_up": 18, "w_down": 19,
+    "beta1": 16, "beta2": 17, "w_gate_up": 18, "w_down": 19, "norm1": 20, "norm2": 21,
     # free-standing stage inputs used by the per-kernel tests
     "s_x": 40, "s_dt": 41, "s_bc": 42, "s_g": 43, "s_q": 44, "s_kv": 45,
     "s_z": 46, "s_a": 47, "s_w": 48,
@@ -232,7 +232,7 @@ def layer_inputs(wl: Workload, batch: Optional[int] = None, seq_len: Optional[in
     return full, meta
 
 
-def layer_params(wl: Workload, layer: int) -> Dict[str, np.ndarray]:
+def layer_params(wl: Workload, layer: int, norm_gains: bool = False) -> Dict[str, np.ndarray]:
     """Weights of one layer, as float32 arrays (bf16-exact for bf16 workloads).
 
     Layouts (row-major, nn.Linear convention [out_features, in_features]):
@@ -243,6 +243,8 @@ def layer_params(wl: Workload, layer: int) -> Dict[str, np.ndarray]:
       w_out [d, Hq*dh + Di]
       a_log [Di] (or [Di, N] when a_per_state), b_dt [Di], beta1 [Hq*dh], beta2 [Di]: fp32
       w_gate_up [2F, d] (gate rows then up rows), w_down [d, F]   (ffn_dim > 0)
+      norm1, norm2 [d] fp32 ~ U(0.5, 1.5): the stacked block's pre-norm gains, only with
+                        norm_gains (the workloads use unit gains, their initial value)
     """
     s = wl.layers[layer]
     sd, dt = wl.seed, s.dtype
@@ -265,6 +267,9 @@ def layer_params(wl: Workload, layer: int) -> Dict[str, np.ndarray]:
     if s.ffn_dim:
         p["w_gate_up"] = normal(sd, layer, "w_gate_up", (2 * s.ffn_dim, s.d_model), 0.02, dt)
         p["w_down"] = normal(sd, layer, "w_down", (s.d_model, s.ffn_dim), 0.02, dt)
+    if norm_gains:
+        p["norm1"] = uniform(sd, layer, "norm1", (s.d_model,), 0.5, 1.5)
+        p["norm2"] = uniform(sd, layer, "norm2", (s.d_model,), 0.5, 1.5)
     return p
 
 

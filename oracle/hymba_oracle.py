@@ -83,6 +83,13 @@ def rms_normalize(v, eps: float):
     return v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
 
 
+def rms_norm(v, eps: float, gain=None):
+    """RMSNorm with a learnable per-feature gain (the pre-norms of the stacked blocks;
+    gain None = unit gain): gain * v / sqrt(mean(v^2) + eps)."""
+    y = rms_normalize(v, eps)
+    return y if gain is None else y * f64(gain)
+
+
 # ---------------------------------------------------------------------------
 # meta tokens and projections
 
@@ -291,6 +298,26 @@ def layer_forward(x, meta, p: Dict[str, np.ndarray], s, kv_in: Optional[Tuple] =
     return out, (k, v)
 
 
+def layer_forward_rows(x, meta, p: Dict[str, np.ndarray], s, rows, kv_in: Optional[Tuple] = None):
+    """Output rows ``rows`` of layer_forward for one sequence (x [1, L, d] or, with meta
+    None, [1, T, d]): the projections and the SSM scan run over every row (each output row
+    depends on all rows before it), the attention and out_proj only for the listed rows.
+    kv_in = (K, V) [1, T, Hkv*dh] for a consuming layer.  Returns [len(rows), d]."""
+    rows = np.asarray(rows)
+    xt = meta_prepend(x, meta)
+    parts = split_in_proj(linear(xt, p["w_in"]), s)
+    if s.kv_mode == KV_CONSUME:
+        assert kv_in is not None, "a consuming layer needs the producer's K/V"
+        k, v = f64(kv_in[0]), f64(kv_in[1])
+    else:
+        k, v = parts["k"], parts["v"]
+    y_attn = attention(parts["q"][0][rows], k[0], v[0], s.n_q_heads, s.n_kv_heads, s.n_meta, s.window,
+                       rows=rows)
+    y_ssm = ssm_branch(parts["x_ssm"][0], parts["g_raw"][0], p["w_x"], p["w_dt"], p["b_dt"], p["a_log"],
+                       s.d_state, s.dt_rank)[rows]
+    return linear(branch_fusion(y_attn, y_ssm, p["beta1"], p["beta2"], s.rms_eps), p["w_out"])
+
+
 # ---------------------------------------------------------------------------
 # generation: one new token from the KV cache and the SSM state
 
@@ -362,18 +389,19 @@ def stack_forward(x, meta, params: Sequence[Dict[str, np.ndarray]], shapes: Sequ
     """Stacked hybrid-head blocks ([S] "Key Components of Hymba": blocks stacked
     with sliding-window attention and cross-layer KV sharing; [R] "Cross-layer
     KV sharing": two consecutive layers share one KV cache).  Each block is
-    h += mixer(RMSNorm(h)); h += SwiGLU(RMSNorm(h)), unit RMSNorm gains.
+    h += mixer(RMSNorm_1(h)); h += SwiGLU(RMSNorm_2(h)), with the gains
+    p["norm1"], p["norm2"] (unit gains when absent).
     Returns h [B, T, d] (and the list of per-block outputs if asked)."""
     h = meta_prepend(x, meta)
     kv = None
     hidden = []
     for p, s in zip(params, shapes):
-        xn = rms_normalize(h, s.rms_eps)
+        xn = rms_norm(h, s.rms_eps, p.get("norm1"))
         out, kv_l = layer_forward(xn, None, p, s, kv_in=kv if s.kv_mode == KV_CONSUME else None)
         if s.kv_mode != KV_CONSUME:
             kv = kv_l
         h = h + out
         if s.ffn_dim:
-            h = h + swiglu_ffn(rms_normalize(h, s.rms_eps), p["w_gate_up"], p["w_down"])
+            h = h + swiglu_ffn(rms_norm(h, s.rms_eps, p.get("norm2")), p["w_gate_up"], p["w_down"])
         hidden.append(h)
     return (h, hidden) if return_hidden else h

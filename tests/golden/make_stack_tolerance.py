@@ -1,29 +1,30 @@
-"""Derive the parity tolerance of the full-depth (24-block) bf16 stack check.
+"""Derive the parity bound of the full-depth (24-block) bf16 stack check, and report
+the expected deviation of every block pair, from the oracle alone.
 
-Why a derived tolerance: the stacked blocks feed each block's output into the
-next, and the random-init stack amplifies a perturbation of its input (in exact
-fp64 arithmetic a 1e-3 relative perturbation of X~ grows to ~7e-3 relative L2
-after 8 blocks).  A bf16 pipeline rounds its activations to bf16 (2^-9 relative)
-at every storage point of every block, so the end-of-stack deviation from the
-exact oracle grows with depth: every single hybrid-head layer meets the 2e-2
-bound; a block pair (two layers and two FFNs) may not, the 24-block output cannot.
+Procedure (fixed before any GPU run of the stack path it models):
 
-This script measures that growth with the oracle alone: it runs the exact fp64
-oracle and the same oracle functions with each stored activation rounded to bf16
-at the storage points the bf16 path uses (the normalised block input, the fused
-in_proj outputs Q|K|V|X_ssm|SiLU(G), dt_low, dt, the attention output, the gated
-SSM output, W_out with beta folded in (the branch norm is fused into out_proj, so
-the normalised Z itself is never stored), the residual stream, the SwiGLU product)
-and the SSM output at tf32 precision (the scan's block products take tf32
-operands), on the test's
-input (sequence 0 of the 24-block workload, first 1100 user tokens), and writes
-the deviation at every depth and the tolerance 1.5x that deviation to
-``stack24_tolerance.json``; and the same deviation for every block pair run as a
-2-block stack (the block-pair check), with its bound max(2e-2, 1.5x deviation).
-Every deviation is the largest over four placements of the rounding errors (round
-to nearest, and three seeds of round to nearest on a randomly scaled grid, at the same
-points): the max-norm deviation of one placement is heavy-tailed.
-It imports nothing from the CUDA path.
+* The model: the oracle's own functions, with each value the bf16 path stores rounded
+  at the point where the path stores it -- the residual stream h in fp32; each
+  pre-norm's output in bf16 (the GEMM operand) and, for the mixer's pre-norm, the fp32
+  remainder that this rounding drops, itself in bf16, carried into [dt_low | B | C]
+  through W_eff = W_x W_SSM (in bf16); the fused in_proj outputs Q | K | V | X_ssm |
+  SiLU(G) in bf16; dt_low and dt in bf16; B and C in fp32; the SSM output at tf32
+  precision (d_state 16: the scan's block products take tf32 operands); the attention
+  and gated SSM outputs in bf16; W_out with beta folded in, in bf16 (the branch norm is
+  fused into out_proj); the SwiGLU product in bf16; the block output in bf16.
+* REALIZATIONS = 8 placements of the rounding errors: round to nearest, and seven seeds
+  of round to nearest on a randomly scaled grid (each value x rounded as x*s, s uniform
+  in [1, 2), then divided by s), which keeps the error distribution and moves where it
+  lands.  One placement understates a max-norm deviation, which is heavy-tailed (a few
+  early rows whose SSM output is a near-cancelling sum carry the largest error after the
+  branch norm); the count is fixed here, not tuned to any result.
+* Depth 24: the bound is HEADROOM x the largest deviation over the realizations.
+* Block pairs: the bound is the pages' 2e-2 for every pair (not derived); this script
+  only reports the model's deviation for each (pair, sequence) beside it.
+
+Metric: max|g - o| / max|o| of the block output.  Inputs: sequence 0 of the 24-block
+workload, first PREFIX user tokens (depth check); for the pairs, the (sequence, prefix)
+cases of PAIR_CASES.  It imports nothing from the CUDA path.
 
     python tests/golden/make_stack_tolerance.py
 """
@@ -44,7 +45,10 @@ from hybrid_attention_ssm_hymba_b200 import synth  # noqa: E402
 
 PREFIX = 1100
 HEADROOM = 1.5
-REALIZATIONS = 4   # round to nearest; then three seeds of the same rounding on a shifted grid
+REALIZATIONS = 8
+PAIR_BOUND = 2e-2
+# (sequence, user-token prefix) pairs the block-pair GPU test checks
+PAIR_CASES = ((0, 1100), (7, 160))
 
 _GRID = None       # numpy Generator: round x*s (s uniform in [1, 2) per element) and divide by s
 
@@ -58,10 +62,6 @@ def _rne_bits(a, drop):
 
 
 def _round_bits(a, drop):
-    """Round to nearest at the path's precision.  In a shifted-grid realization each value
-    is rounded as x*s and divided back by s: the error keeps the round-to-nearest
-    distribution (half an ulp of the value's own binade position, now random) but lands
-    on every element independently of the first realization."""
     if _GRID is None:
         return _rne_bits(a, drop)
     a = np.asarray(a, np.float64)
@@ -78,17 +78,25 @@ def _tf32(a):
     return _round_bits(a, 13)
 
 
-def _layer_bf16_storage(x, p, s, kv_in=None):
-    B = x.shape[0]
-    parts = O.split_in_proj(O.linear(x, p["w_in"]), s)
+def _f32(a):
+    return np.asarray(a, np.float32).astype(np.float64)
+
+
+def _layer_model(xn, xlo, p, s, kv_in=None):
+    """One hybrid-head layer of a stacked block as the bf16 path stores it."""
+    B = xn.shape[0]
+    parts = O.split_in_proj(O.linear(xn, p["w_in"]), s)
     parts["g"] = _bf16(O.silu(parts.pop("g_raw")))
     parts = {k: _bf16(v) for k, v in parts.items()}
     k, v = kv_in if s.kv_mode == O.KV_CONSUME else (parts["k"], parts["v"])
+    wa, wkv = s.n_q_heads * s.head_dim, s.n_kv_heads * s.head_dim
+    r0 = wa + (0 if s.kv_mode == O.KV_CONSUME else 2 * wkv)
+    w_eff = _bf16(O.linear(p["w_x"], O.f64(p["w_in"][r0:r0 + s.d_inner]).T))   # W_x W_SSM [R + 2N, d]
     ya = np.stack([_bf16(O.attention(parts["q"][b], k[b], v[b], s.n_q_heads, s.n_kv_heads, s.n_meta,
                                      s.window)) for b in range(B)])
     ys = []
     for b in range(B):
-        xdbc = O.linear(parts["x_ssm"][b], p["w_x"])
+        xdbc = O.linear(parts["x_ssm"][b], p["w_x"]) + O.linear(xlo[b], w_eff)
         dt_low = _bf16(xdbc[:, :s.dt_rank])
         Bm, Cm = xdbc[:, s.dt_rank:s.dt_rank + s.d_state], xdbc[:, s.dt_rank + s.d_state:]
         dt = _bf16(O.softplus(O.linear(dt_low, p["w_dt"]) + p["b_dt"]))
@@ -96,88 +104,39 @@ def _layer_bf16_storage(x, p, s, kv_in=None):
         if s.d_state == 16:   # the scan's products take tf32 operands: y at tf32 precision
             y = _tf32(y)
         ys.append(_bf16(parts["g"][b] * y))
-    # fused branch norm: the normalised Z is never stored; beta is folded into W_out,
-    # which is stored in bf16, and out_proj scales each row by its 1/rms in fp32
     ones1, ones2 = np.ones_like(p["beta1"]), np.ones_like(p["beta2"])
     zn = O.branch_fusion(ya, np.stack(ys), ones1, ones2, s.rms_eps)
     w_scaled = _bf16(p["w_out"] * np.concatenate([p["beta1"], p["beta2"]])[None, :])
     return O.linear(zn, w_scaled), (k, v)
 
 
-def stack_bf16_storage(x, meta, params, shapes):
-    h = _bf16(O.meta_prepend(x, meta))
+def stack_model(x, meta, params, shapes):
+    """Block outputs of the stack as the bf16 path stores them (the last one rounded to
+    bf16, the others as the fp32 residual stream)."""
+    h = _f32(O.meta_prepend(x, meta))
     kv, hidden = None, []
     for p, s in zip(params, shapes):
-        out, kv_l = _layer_bf16_storage(_bf16(O.rms_normalize(h, s.rms_eps)), p, s,
-                                        kv if s.kv_mode == O.KV_CONSUME else None)
+        v = _f32(O.rms_norm(h, s.rms_eps, p.get("norm1")))
+        xn = _bf16(v)
+        out, kv_l = _layer_model(xn, _bf16(v - xn), p, s, kv if s.kv_mode == O.KV_CONSUME else None)
         if s.kv_mode != O.KV_CONSUME:
             kv = kv_l
-        h = _bf16(h + out)
+        h = _f32(h + out)
         F = s.ffn_dim
-        gu = O.linear(_bf16(O.rms_normalize(h, s.rms_eps)), p["w_gate_up"])
-        h = _bf16(h + O.linear(_bf16(O.silu(gu[..., :F]) * gu[..., F:]), p["w_down"]))
+        gu = O.linear(_bf16(O.rms_norm(h, s.rms_eps, p.get("norm2"))), p["w_gate_up"])
+        h = _f32(h + O.linear(_bf16(O.silu(gu[..., :F]) * gu[..., F:]), p["w_down"]))
         hidden.append(h)
+    hidden[-1] = _bf16(hidden[-1])
     return hidden
 
 
-def realization(r):
-    """Deviations of one rounding realization (r = 0: nearest; r > 0: nearest on a shifted grid, seed r):
-    the 24-block stack by depth, and every block pair."""
-    global _GRID
-    _GRID = None if r == 0 else np.random.default_rng(9000 + r)
-    wl = synth.workload("hymba1p5b_stack24")
-    x, meta = synth.layer_inputs(wl, batch=1, seq_len=PREFIX)
-    params = [synth.layer_params(wl, i) for i in range(len(wl.layers))]
-    shapes = [dataclasses.replace(s, batch=1, seq_len=PREFIX) for s in wl.layers]
-    _, exact = O.stack_forward(x, meta, params, shapes, return_hidden=True)
-    model = stack_bf16_storage(x, meta, params, shapes)
-    dev = [float(np.abs(m - e).max() / np.abs(e).max()) for m, e in zip(model, exact)]
-    return dev, block_pair_deviations(full=wl)
-
-
-def main():
-    """The max-norm deviation of one realization is heavy-tailed (a few rows with small
-    branch RMS carry the largest relative error after the norm), so each bound is taken
-    over REALIZATIONS placements of the rounding errors: the maximum deviation, times
-    HEADROOM."""
-    os.environ.setdefault("OMP_NUM_THREADS", "2")
-    with cf.ProcessPoolExecutor(REALIZATIONS, mp_context=mp.get_context("spawn")) as ex:
-        runs = list(ex.map(realization, range(REALIZATIONS)))
-    dev = [max(r[0][i] for r in runs) for i in range(len(runs[0][0]))]
-    wl = synth.workload("hymba1p5b_stack24")
-    out = {
-        "workload": wl.name, "sequence": 0, "prefix_user_tokens": PREFIX,
-        "metric": "max|g-o| / max|o| of the block output h",
-        "realizations": "round to nearest, and 3 seeds of round to nearest on a randomly scaled grid, at the same points",
-        "bf16_storage_deviation_by_depth": dev,
-        "deviation_24_blocks_by_realization": [r[0][-1] for r in runs],
-        "headroom": HEADROOM,
-        "tolerance_24_blocks": HEADROOM * dev[-1],
-        "derivation": "largest deviation over the realizations of the oracle with rounding at the bf16 "
-                      "path's rounding points from the exact fp64 oracle (this script; oracle functions "
-                      "only), times the headroom",
-    }
-    pairs = {}
-    for key in runs[0][1]:
-        ds = [r[1][key][1] for r in runs]
-        pairs[key] = {"prefix_user_tokens": runs[0][1][key][0], "bf16_storage_deviation": max(ds),
-                      "by_realization": ds, "tolerance": max(2e-2, HEADROOM * max(ds))}
-    out["block_pairs"] = pairs
-    with open(os.path.join(HERE, "stack24_tolerance.json"), "w") as f:
-        json.dump(out, f, indent=1)
-    print(json.dumps({k: out[k] for k in ("tolerance_24_blocks",)}), [round(d, 4) for d in dev])
-
-
-# (sequence, user-token prefix) pairs the block-pair GPU test checks
-PAIR_CASES = ((0, 1100), (7, 160))
+def _dev(model, exact):
+    return float(np.abs(model - exact).max() / np.abs(exact).max())
 
 
 def block_pair_deviations(full):
     """Every block pair (2k, 2k+1) run as a 2-block stack from X, as the block-pair GPU
-    test runs it: the deviation of the pair's output for each checked (sequence,
-    prefix).  The bound is max(2e-2, HEADROOM x deviation): one hybrid-head layer meets
-    2e-2; a pair composes two layers and two SwiGLU FFNs, and its rounding deviation
-    alone can exceed 2e-2."""
+    test runs it: the model's deviation for each checked (sequence, prefix)."""
     res = {}
     for pair in range(len(full.layers) // 2):
         wl = synth.workload(full.name)
@@ -187,9 +146,55 @@ def block_pair_deviations(full):
         for b, L in PAIR_CASES:
             shapes = [dataclasses.replace(s, batch=1, seq_len=L) for s in wl.layers]
             exact = O.stack_forward(x[b:b + 1, :L], meta, params, shapes)
-            model = stack_bf16_storage(x[b:b + 1, :L], meta, params, shapes)[-1]
-            res[f"{pair}/{b}"] = (L, float(np.abs(model - exact).max() / np.abs(exact).max()))
+            res[f"{pair}/{b}"] = (L, _dev(stack_model(x[b:b + 1, :L], meta, params, shapes)[-1], exact))
     return res
+
+
+def realization(r):
+    """Deviations of one rounding realization (r = 0: nearest; r > 0: nearest on a scaled
+    grid, seed r): the 24-block stack by depth, and every block pair."""
+    global _GRID
+    _GRID = None if r == 0 else np.random.default_rng(9000 + r)
+    wl = synth.workload("hymba1p5b_stack24")
+    x, meta = synth.layer_inputs(wl, batch=1, seq_len=PREFIX)
+    params = [synth.layer_params(wl, i) for i in range(len(wl.layers))]
+    shapes = [dataclasses.replace(s, batch=1, seq_len=PREFIX) for s in wl.layers]
+    _, exact = O.stack_forward(x, meta, params, shapes, return_hidden=True)
+    model = stack_model(x, meta, params, shapes)
+    return [_dev(m, e) for m, e in zip(model, exact)], block_pair_deviations(full=wl)
+
+
+def main():
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    workers = min(REALIZATIONS, os.cpu_count() or 1)
+    with cf.ProcessPoolExecutor(workers, mp_context=mp.get_context("spawn")) as ex:
+        runs = list(ex.map(realization, range(REALIZATIONS)))
+    dev = [max(r[0][i] for r in runs) for i in range(len(runs[0][0]))]
+    wl = synth.workload("hymba1p5b_stack24")
+    out = {
+        "workload": wl.name, "sequence": 0, "prefix_user_tokens": PREFIX,
+        "metric": "max|g-o| / max|o| of the block output h",
+        "realizations": f"{REALIZATIONS}: round to nearest, and {REALIZATIONS - 1} seeds of round to nearest on "
+                        "a randomly scaled grid, at the same points",
+        "model_deviation_by_depth": dev,
+        "deviation_24_blocks_by_realization": [r[0][-1] for r in runs],
+        "headroom": HEADROOM,
+        "tolerance_24_blocks": HEADROOM * dev[-1],
+        "derivation": "largest deviation over the realizations of the oracle with rounding at the bf16 "
+                      "path's storage points from the exact fp64 oracle (this script; oracle functions "
+                      "only), times the headroom",
+    }
+    pairs = {}
+    for key in runs[0][1]:
+        ds = [r[1][key][1] for r in runs]
+        pairs[key] = {"prefix_user_tokens": runs[0][1][key][0], "model_deviation": max(ds),
+                      "by_realization": ds, "tolerance": PAIR_BOUND}
+    out["block_pairs"] = pairs
+    with open(os.path.join(HERE, "stack24_tolerance.json"), "w") as f:
+        json.dump(out, f, indent=1)
+    print(json.dumps({"tolerance_24_blocks": out["tolerance_24_blocks"],
+                      "worst_pair": max((v["model_deviation"], k) for k, v in pairs.items())}),
+          [round(d, 4) for d in dev])
 
 
 if __name__ == "__main__":

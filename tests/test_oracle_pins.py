@@ -403,3 +403,48 @@ def test_stack_kv_pairing_uses_producer_kv():
     a = O.stack_forward(x, meta, ps2, layers)
     b = O.stack_forward(x, meta, ps3, layers)
     assert np.abs(a - b).max() > 1e-6
+
+
+def test_stack_prenorm_gains_fold_into_the_following_weights():
+    """Gains g1, g2 of the two pre-norms of a block equal unit gains with g1 folded into the
+    columns of W_in and g2 into the columns of W_gate_up (W (g * u) = (W diag g) u): two
+    stacks that differ only in where the gain sits give the same output; a gain of c * 1
+    on a block's pre-norm is not a no-op (the norm's output is rescaled, not re-normalised)."""
+    s = _tiny_shape(window=3, ffn_dim=10)
+    layers = [dataclasses.replace(s, kv_mode=O.KV_PRODUCE), dataclasses.replace(s, kv_mode=O.KV_CONSUME)]
+    wl = synth.Workload("t", layers, 6, 1e-3, False, "t")
+    x, meta = synth.layer_inputs(wl)
+    ps = [synth.layer_params(wl, i, norm_gains=True) for i in range(2)]
+    assert ps[0]["norm1"].shape == (s.d_model,) and not np.allclose(ps[0]["norm1"], 1.0)
+    folded = []
+    for p in ps:
+        q = {k: v for k, v in p.items() if k not in ("norm1", "norm2")}
+        q["w_in"] = p["w_in"].astype(float) * p["norm1"][None, :]
+        q["w_gate_up"] = p["w_gate_up"].astype(float) * p["norm2"][None, :]
+        folded.append(q)
+    np.testing.assert_allclose(O.stack_forward(x, meta, ps, layers), O.stack_forward(x, meta, folded, layers),
+                               rtol=1e-11, atol=1e-12)
+    unit = [{k: v for k, v in p.items() if k not in ("norm1", "norm2")} for p in ps]
+    scaled = [dict(u, norm1=np.full(s.d_model, 2.0)) for u in unit]
+    assert np.abs(O.stack_forward(x, meta, scaled, layers) - O.stack_forward(x, meta, unit, layers)).max() > 1e-3
+    np.testing.assert_allclose(O.rms_norm(np.full((1, 4), -3.0), 0.0, np.array([1.0, 2.0, 3.0, 4.0])),
+                               [[-1.0, -2.0, -3.0, -4.0]], rtol=1e-15)
+
+
+@pytest.mark.parametrize("window,kv", [(-1, O.KV_OWN), (3, O.KV_PRODUCE), (2, O.KV_CONSUME)])
+def test_layer_forward_rows_equals_the_full_layer_rows(window, kv):
+    """The row-subset layer (projections and scan over every row, attention and out_proj
+    for the listed rows only) returns exactly those rows of the full layer, including
+    rows past window + meta and the last row."""
+    s = dataclasses.replace(_tiny_shape(window=window, batch=1), kv_mode=kv)
+    wl = synth.Workload("t", [s], 7, 1e-3, False, "t")
+    x, meta = synth.layer_inputs(wl)
+    p = synth.layer_params(wl, 0)
+    kv_in = None
+    if kv == O.KV_CONSUME:
+        T = s.T
+        kv_in = (RNG.standard_normal((1, T, s.kv_width)), RNG.standard_normal((1, T, s.kv_width)))
+    full, _ = O.layer_forward(x, meta, p, s, kv_in=kv_in)
+    rows = np.array([0, 1, s.n_meta, s.T // 2, s.T - 1])
+    np.testing.assert_allclose(O.layer_forward_rows(x, meta, p, s, rows, kv_in=kv_in), full[0][rows],
+                               rtol=1e-12, atol=1e-13)
