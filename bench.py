@@ -3,19 +3,22 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
 
-A step is one forward pass of the whole hybrid-head layer (in_proj with the meta
-prepend, x_proj, dt_proj, attention heads, selective scan + gate, branch
-RMSNorm + beta, out_proj) over one batch of the seeded synthetic workload,
-through the C ABI (hymba_layer_fwd).  Default workload: the Hymba-350M-shaped
-layer (B=8, L=2048 + 32 meta tokens, d=1024, bf16).  W untimed warm-up steps,
-then exactly K timed steps, each bracketed by CUDA events on the launching
-stream with an L2 flush (256 MiB memset) between steps outside the events; a
-barrier and a device synchronise on both sides of the timed loop; the time is
-the max over ranks.  Under torchrun every rank runs its own batch (weak
-scaling, no collective on the data path).  Rank 0 prints one JSON line.
+A step is one forward pass of every layer of the workload (in_proj with the meta
+prepend, x_proj, dt_proj, attention heads, selective scan + gate, branch RMSNorm +
+beta, out_proj; the stacked workload adds the pre-norms and the SwiGLU FFN) over one
+batch of the seeded synthetic workload, through the C ABI.  Default workload: the
+Hymba-1.5B-shaped producer + consumer layer pair sharing K/V (B=4, L=8192 + 128 meta
+tokens, d=2048, SWA 1024, d_state 128, bf16) -- the largest single-GPU layer
+configuration.  W untimed warm-up steps, then exactly K timed steps, each bracketed
+by CUDA events on the launching stream with an L2 flush (256 MiB memset) between
+steps outside the events; a barrier and a device synchronise on both sides of the
+timed loop; the time is the max over ranks.  Under torchrun every rank runs its own
+batch (weak scaling, no collective on the data path).  Rank 0 prints one JSON line;
+at N = 1 it also carries `per_workload` (every other workload measured the same way
+with fewer steps) and `decode` (the generation step of the layer pair).
 
---impl reference times the fp64 CPU oracle on the host cores instead (each
-step a bounded sample of the same workload), as the reference arm.
+--impl reference times the fp64 CPU oracle on the host cores instead (each step a
+bounded sample of the same workload), as the reference arm.
 """
 from __future__ import annotations
 
@@ -101,52 +104,127 @@ def stage_work(s: synth.LayerShape, dt_in_scan: bool = False):
     return work
 
 
+def ffn_work(s: synth.LayerShape):
+    """SwiGLU FFN and the two pre-norms of a stacked block: (FLOPs, HBM bytes)."""
+    es = 2 if s.dtype == "bf16" else 4
+    rows, d, F = s.batch * s.T, s.d_model, s.ffn_dim
+    fl = 6.0 * d * F * rows
+    by = es * (rows * d + 2 * F * d + rows * F) + es * (rows * F + F * d) + 4 * rows * d * 2
+    by += 2 * (4 * rows * d + es * rows * d)          # pre-norms: read h (fp32), write the bf16 operand
+    return fl, by
+
+
+def scan_kernel_name(s: synth.LayerShape) -> str:
+    if s.dtype == "bf16" and s.d_state == 16 and not s.a_per_state:
+        return "scan_tc_kernel, tcgen05 tf32"
+    return "scan_w_kernel, fp32 FMA"
+
+
+def stage_bound(stage: str, s: synth.LayerShape) -> str:
+    """The bound that binds each stage: a dense contraction on the tensor cores, HBM
+    traffic, or (the CUDA-core scan at d_state > 16) the fp32 FMA rate."""
+    if stage in ("in_proj", "out_proj", "attention"):
+        return "tensor"
+    if stage == "scan" and not scan_kernel_name(s).startswith("scan_tc"):
+        return "alu"
+    return "hbm"
+
+
 KERNEL_NAMES = {"in_proj": "gemm_bf16_tc, tcgen05", "x_proj": "gemm_bf16_tc, tcgen05",
-                "dt_proj": "gemm_bf16_tc, tcgen05", "attention": "attn_fwd_tc, tcgen05",
-                "scan": "scan_tc_kernel, tcgen05 tf32 (+ dt projection, bf16)", "branch_norm": "row_ssq_kernel + scale_cols_kernel",
+                "dt_proj": "gemm_bf16_tc, tcgen05", "attention": "attn_fwd_tc2, tcgen05",
+                "branch_norm": "row_ssq_kernel + scale_cols_kernel",
                 "out_proj": "gemm_bf16_tc, tcgen05, two accumulators"}
 
-# dominant bound of each stage: a dense contraction on the tensor cores or HBM traffic
-STAGE_BOUND = {"in_proj": "tensor", "x_proj": "hbm", "dt_proj": "hbm", "attention": "tensor",
-               "scan": "hbm", "branch_norm": "hbm", "out_proj": "tensor"}
+PROFILE_COMMON = ("hybrid_attention_ssm_hymba_b200/csrc/hy_common.cuh",
+                  "hybrid_attention_ssm_hymba_b200/csrc/hy_kernels.h")
 
 
-def _traffic(stage: str):
-    """DRAM bytes per launch from the committed ncu capture of this stage's kernel,
-    or None when there is none or the kernel's source changed since it was taken."""
+def source_hash(sources) -> str:
+    """sha256 over a kernel's source file and the headers every kernel includes."""
     import hashlib
+    h = hashlib.sha256()
+    for rel in list(sources) + list(PROFILE_COMMON):
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()
+
+
+def _traffic(workload: str, stage: str):
+    """DRAM bytes per launch from the committed ncu capture of this stage's kernel on this
+    workload, or None when there is none or the kernel's sources (its file and the common
+    headers) changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f).get(stage)
+        rec = json.load(f).get(workload, {}).get(stage)
     if not rec:
         return None
-    src = os.path.join(ROOT, rec["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
+    try:
+        if source_hash(rec["sources"]) != rec["sha256"]:
+            return None
+    except OSError:
         return None
     return rec["dram_bytes_per_launch"]
 
 
-def stage_rooflines(s: synth.LayerShape, stage_us, peaks, dt_in_scan=False):
-    """Per stage: achieved work rate against its peak (measured peaks), and the layer's
-    roofline time (sum over stages of the slower of its FLOP and byte times)."""
-    out, t_roof = {}, 0.0
+def alu_peak_tflops(peaks, sm_mhz=None):
+    """fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP per clock at the SM clock (the sampled
+    maximum, else 1965 MHz)."""
+    return 148 * 128 * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12
+
+
+def stage_rooflines(layers, stage_us, peaks, dt_in_scan, sm_max_mhz=None):
+    """Per stage, summed over the layers of the workload: the achieved rate of its binding
+    resource against that resource's measured peak (tensor: burst bf16 -- the layers run
+    in sub-second steps; HBM: the measured copy bandwidth; fp32 FMA: derived), and the
+    workload's roofline time (sum over stages of the slowest of its FLOP, byte and ALU
+    times)."""
     hbm = peaks["hbm_gbs"] * 1e9
-    tc = peaks["bf16_tflops_sustained"] * 1e12
-    for name, (fl, by) in stage_work(s, dt_in_scan).items():
+    tc = peaks["bf16_tflops"] * 1e12
+    alu = alu_peak_tflops(peaks, sm_max_mhz) * 1e12
+    tot = {}
+    t_roof = 0.0
+    for s, fused in zip(layers, dt_in_scan):
+        for name, (fl, by) in stage_work(s, fused).items():
+            b = stage_bound(name, s)
+            t_roof += max(fl / tc if b == "tensor" else 0.0, by / hbm, fl / alu if b == "alu" else 0.0)
+            f0, b0, _ = tot.get(name, (0.0, 0.0, b))
+            tot[name] = (f0 + fl, b0 + by, b)
+    out = {}
+    for name, (fl, by, b) in tot.items():
         t = stage_us[name] * 1e-6
-        t_roof += max(fl / tc, by / hbm)
-        if STAGE_BOUND[name] == "tensor":
+        if b == "tensor":
             ach = fl / t / 1e12
-            out[name] = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops_sustained"],
-                         "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops_sustained"], 4),
-                         "work_per_launch": fl, "us": stage_us[name]}
+            out[name] = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4), "work": fl,
+                         "us": stage_us[name]}
+        elif b == "alu":
+            ach = fl / t / 1e12
+            pk = alu / 1e12
+            out[name] = {"bound": "alu", "achieved": round(ach, 2), "peak": round(pk, 2), "unit": "TFLOP/s",
+                         "frac": round(ach / pk, 4), "work": fl, "us": stage_us[name],
+                         "hbm_frac": round(by / t / hbm, 4)}
         else:
             ach = by / t / 1e9
             out[name] = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(ach / peaks["hbm_gbs"], 4), "work_per_launch": by, "us": stage_us[name]}
+                         "frac": round(ach / peaks["hbm_gbs"], 4), "work": by, "us": stage_us[name]}
     return out, t_roof * 1e6
+
+
+def stack_roofline_us(layers, peaks, dt_in_scan):
+    """Roofline time of a stacked workload: every layer's stages plus its FFN and pre-norms."""
+    hbm = peaks["hbm_gbs"] * 1e9
+    tc = peaks["bf16_tflops"] * 1e12
+    alu = alu_peak_tflops(peaks) * 1e12
+    t = 0.0
+    for s, fused in zip(layers, dt_in_scan):
+        for name, (fl, by) in stage_work(s, fused).items():
+            b = stage_bound(name, s)
+            t += max(fl / tc if b == "tensor" else 0.0, by / hbm, fl / alu if b == "alu" else 0.0)
+        if s.ffn_dim:
+            fl, by = ffn_work(s)
+            t += max(fl / tc, by / hbm)
+    return t * 1e6
 
 
 # --------------------------------------------------------------------------- clocks (NVML)
@@ -327,191 +405,330 @@ def weak_scaling_rate(world: int, steps: int, units_per_step_per_rank: float, ma
 
 # --------------------------------------------------------------------------- native (CUDA) leg
 
-def run_native(args, rank, world, local_rank):
-    import torch
+class Workbench:
+    """Device-resident inputs, weights and buffers of one workload, and its step."""
 
-    import hybrid_attention_ssm_hymba_b200 as H
-    from hybrid_attention_ssm_hymba_b200 import host
+    def __init__(self, name, dev):
+        import torch
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    ranks = Ranks(world, local_rank, "nccl", dev)
-    barrier = ranks.barrier
-
-    wl = synth.workload(args.workload)
-    s0 = wl.first
-    dtype = s0.dtype
-    x_np, meta_np = synth.layer_inputs(wl)
-    ps_np = [synth.layer_params(wl, i) for i in range(len(wl.layers))]
-    dps = [host.params_to_device(p, dtype, dev) for p in ps_np]
-    cfgs = [H.make_cfg(s) for s in wl.layers]
-    weights = [H.make_weights(d) for d in dps]
-    T = s0.T
-    x = host.to_device(x_np, dtype, dev)
-    meta = host.to_device(meta_np, dtype, dev)
-    stack = bool(s0.ffn_dim)
-    ws_bytes = H.hymba_stack_workspace_size(cfgs) if stack else max(H.hymba_workspace_size(c) for c in cfgs)
-    ws = host.workspace(ws_bytes, dev)
-    outs = [torch.empty((s0.batch, T, s0.d_model), dtype=x.dtype, device=dev) for _ in wl.layers]
-    kv = torch.empty((2, s0.batch * T, s0.kv_width), dtype=x.dtype, device=dev) if len(wl.layers) > 1 \
-        and not stack else None
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    # this library's kernels per step: in_proj, x_proj, dt_proj (unless the scan computes dt),
-    # attention, scan, out_proj and the norm stage (bf16: row sums + beta-scaled W_out; fp32:
-    # in-place norm); a stack adds two pre-norms and the two FFN GEMMs per block, and the
-    # meta prepend
-    dt_in_scan = [H.hymba_layer_fuses_dt_proj(c) for c in cfgs]
-    n_launch_per_step = sum((8 if dtype == "bf16" else 7) - int(f) for f in dt_in_scan) + \
-        (4 * len(wl.layers) + 1 if stack else 0)
-
-    def step(xin, stage_events=None, out_list=None):
-        o = outs if out_list is None else out_list
-        if stack:
-            H.check(H.hymba_stack_fwd(xin, meta, weights, cfgs, o[0], ws, stream=stream), "stack")
-            return o[0]
-        if stage_events is not None:
-            H.check(H.hymba_layer_fwd_events(xin, meta, weights[0], cfgs[0], None, kv, o[0], ws,
-                                             stage_events, stream=stream), "layer")
+        import hybrid_attention_ssm_hymba_b200 as H
+        from hybrid_attention_ssm_hymba_b200 import host
+        self.H, self.torch = H, torch
+        self.wl = wl = synth.workload(name)
+        self.s0 = s0 = wl.first
+        self.dtype = s0.dtype
+        self.x_np, self.meta_np = synth.layer_inputs(wl)
+        self.ps_np = [synth.layer_params(wl, i) for i in range(len(wl.layers))]
+        self.dps = [host.params_to_device(p, self.dtype, dev) for p in self.ps_np]
+        self.cfgs = [H.make_cfg(s) for s in wl.layers]
+        self.weights = [H.make_weights(d) for d in self.dps]
+        self.x = host.to_device(self.x_np, self.dtype, dev)
+        self.meta = host.to_device(self.meta_np, self.dtype, dev)
+        self.stack = bool(s0.ffn_dim)
+        ws_bytes = H.hymba_stack_workspace_size(self.cfgs) if self.stack else \
+            max(H.hymba_workspace_size(c) for c in self.cfgs)
+        self.ws = host.workspace(ws_bytes, dev)
+        T = s0.T
+        self.outs = [torch.empty((s0.batch, T, s0.d_model), dtype=self.x.dtype, device=dev) for _ in wl.layers]
+        self.kv = torch.empty((2, s0.batch * T, s0.kv_width), dtype=self.x.dtype, device=dev) \
+            if len(wl.layers) > 1 and not self.stack else None
+        self.stream = torch.cuda.current_stream(dev)
+        self.dt_in_scan = [H.hymba_layer_fuses_dt_proj(c) for c in self.cfgs]
+        bf16 = self.dtype == "bf16"
+        per_layer = [(8 if bf16 else 7) - int(f) for f in self.dt_in_scan]
+        if self.stack:   # the prepend; per block: the mixer's pre-norm (bf16: + W_SSM transpose and the
+            # W_eff GEMM), the layer, and with an FFN its pre-norm and two GEMMs
+            self.launches = 1 + sum(n + (3 if bf16 else 1) + (3 if s.ffn_dim else 0)
+                                    for n, s in zip(per_layer, wl.layers))
         else:
-            H.check(H.hymba_layer_fwd(xin, meta, weights[0], cfgs[0], None, kv, o[0], ws, stream=stream),
-                    "layer")
-        for i in range(1, len(wl.layers)):
-            H.check(H.hymba_layer_fwd(o[i - 1], None, weights[i], cfgs[i], kv, None, o[i], ws,
-                                      stream=stream), f"layer {i}")
+            self.launches = sum(per_layer)
+        self.tokens = s0.batch * s0.seq_len
+
+    def step(self, xin, stage_events=None, out_list=None):
+        H = self.H
+        o = self.outs if out_list is None else out_list
+        st = self.stream
+        if self.stack:
+            H.check(H.hymba_stack_fwd(xin, self.meta, self.weights, self.cfgs, o[0], self.ws, stream=st), "stack")
+            return o[0]
+        meta = self.meta
+        for i in range(len(self.cfgs)):
+            kv_in = self.kv if i > 0 else None
+            kv_out = self.kv if i == 0 else None
+            if stage_events is not None:
+                H.check(H.hymba_layer_fwd_events(xin, meta, self.weights[i], self.cfgs[i], kv_in, kv_out, o[i],
+                                                 self.ws, stage_events[i], stream=st), f"layer {i}")
+            else:
+                H.check(H.hymba_layer_fwd(xin, meta, self.weights[i], self.cfgs[i], kv_in, kv_out, o[i], self.ws,
+                                          stream=st), f"layer {i}")
+            xin, meta = o[i], None
         return o[-1]
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step(x)
-    torch.cuda.synchronize(dev)
-    assert H.hymba_workspace_status(ws, stream) == H.HYMBA_OK
 
-    K = args.steps
+def measure(bench: Workbench, K: int, W: int, ranks, dev, flush, stages=True, e2e=False):
+    """Time K steps of the workload (after W warm-up steps), then optionally the stage
+    breakdown and the end-to-end path.  Returns (record, total_ms)."""
+    import torch
+    H = bench.H
+    stream = bench.stream
+    for _ in range(W):
+        flush.zero_()
+        bench.step(bench.x)
+    torch.cuda.synchronize(dev)
+    assert H.hymba_workspace_status(bench.ws, stream) == H.HYMBA_OK
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     sampler = ClockSampler(dev)
-    barrier()
+    ranks.barrier()
     torch.cuda.synchronize(dev)
     with sampler:
         for k in range(K):
             flush.zero_()
             ev_s[k].record(stream)
-            step(x)
+            bench.step(bench.x)
             ev_e[k].record(stream)
         torch.cuda.synchronize(dev)
-    barrier()
-    # Stage breakdown in a separate pass: events between the kernels of a step order
-    # them fully (no programmatic overlap), so they are kept out of the timed steps.
-    n_stage = max(3, min(K, 50))
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(n_stage)] \
-        if not stack else None
-    if stage_ev:
-        for evs in stage_ev:   # torch creates the CUDA event lazily, at its first record
-            for e in evs:
-                e.record(stream)
-        torch.cuda.synchronize(dev)
-        for k in range(n_stage):
-            flush.zero_()
-            step(x, stage_ev[k])
+        ranks.barrier()
+        # clocks under load: keep stepping (untimed) until the sampler has a few hundred ms
+        t_end = time.perf_counter() + 0.3
+        while time.perf_counter() < t_end:
+            bench.step(bench.x)
         torch.cuda.synchronize(dev)
     step_ms = [ev_s[k].elapsed_time(ev_e[k]) for k in range(K)]
     total_ms = ranks.max(float(sum(step_ms)))
-    status = H.hymba_workspace_status(ws, stream)
-    tokens_per_step = s0.batch * s0.seq_len
-    value = weak_scaling_rate(world, K, tokens_per_step, total_ms)
-
+    rec = {"ms_per_step": total_ms / K, "steps": K, "warmup": W, "clocks": sampler.summary(),
+           "gpu_launches": bench.launches * K}
     peaks, peak_src = _peaks()
-    roofline, stages, stage_roof, layer_roof = None, None, None, None
-    if stage_ev:
-        per_stage = {name: float(np.mean([stage_ev[k][i].elapsed_time(stage_ev[k][i + 1]) for k in range(n_stage)]))
-                     for i, name in enumerate(H.STAGES)}
-        stages = {n: round(v * 1e3, 2) for n, v in per_stage.items()}  # microseconds
-        if dt_in_scan[0]:   # stage 2 launches nothing: dt is computed inside the scan
-            stages.pop("dt_proj")
-        stage_roof, t_roof_us = stage_rooflines(s0, stages, peaks, dt_in_scan[0])
-        top = max(stages, key=stages.get)   # the dominant kernel of the step
-        r = stage_roof[top]
-        roofline = {"kernel": f"{top} ({KERNEL_NAMES[top]})", "bound": r["bound"], "achieved": r["achieved"],
-                    "peak": r["peak"], "unit": r["unit"], "frac": r["frac"], "traffic": _traffic(top),
-                    "peak_source": (f"{peak_src} bf16_tflops_sustained (kernel timed inside a continuous loop)"
-                                    if r["bound"] == "tensor" else f"{peak_src} hbm_gbs (STREAM-style copy)"),
-                    "us_per_launch": stages[top], "algorithmic_work_per_launch": r["work_per_launch"]}
-        layer_roof = {"roofline_us": round(t_roof_us, 2), "measured_us": round(1e3 * total_ms / K, 2),
-                      "frac": round(t_roof_us / (1e3 * total_ms / K), 4),
-                      "definition": "sum over stages of max(FLOPs / bf16 sustained peak, bytes / HBM peak), "
-                                    "against the timed step"}
-
-    e2e = None
-    if not args.no_e2e:
-        # Through the public entry point with host buffers, as a serving loop runs it: each
-        # step copies its input from pinned host memory and its output back, double-buffered
-        # over three streams so that step k's input copy (host -> device), step k-1's layer
-        # (the compute stream, with the same L2 flush before it) and step k-2's output copy
-        # (device -> host) overlap.  Timed from the first timed input copy to the last output
-        # copy, on the device.
-        xh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
-        xh.copy_(x.cpu())
-        ohs = [torch.empty(outs[-1].shape, dtype=x.dtype).pin_memory() for _ in range(2)]
-        xds = [torch.empty_like(x) for _ in range(2)]
-        out_sets = [outs, [torch.empty_like(o) for o in outs]]
-        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        n_e2e, n_warm = max(3, min(K, 50)), 3
-        total = n_warm + n_e2e
-        h2d = [torch.cuda.Event() for _ in range(total)]
-        comp = [torch.cuda.Event() for _ in range(total)]
-        d2h = [torch.cuda.Event() for _ in range(total)]
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
+    wl = bench.wl
+    if stages and not bench.stack:
+        # Stage breakdown in a separate pass: events between the kernels of a step order them
+        # fully (no programmatic overlap, the attention on the caller's stream), so they are
+        # kept out of the timed steps.
+        n_stage = max(3, min(K, 20))
+        nl = len(bench.cfgs)
+        ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(nl)] for _ in range(n_stage)]
+        for per_step in ev:   # torch creates the CUDA event lazily, at its first record
+            for evs in per_step:
+                for e in evs:
+                    e.record(stream)
         torch.cuda.synchronize(dev)
-        for k in range(total):
-            j = k % 2
-            if k == n_warm:
-                torch.cuda.synchronize(dev)   # warm-up steps done; the timed pipeline starts empty
-                t0.record(s_in)
-            if k >= 2:
-                s_in.wait_event(comp[k - 2])   # the layer that read xds[j] is done
-            with torch.cuda.stream(s_in):
-                xds[j].copy_(xh, non_blocking=True)
-            h2d[k].record(s_in)
-            stream.wait_event(h2d[k])
-            if k >= 2:
-                stream.wait_event(d2h[k - 2])  # out_sets[j] has been copied out
+        for k in range(n_stage):
             flush.zero_()
-            o = step(xds[j], out_list=out_sets[j])
-            comp[k].record(stream)
-            s_out.wait_event(comp[k])
-            with torch.cuda.stream(s_out):
-                ohs[j].copy_(o, non_blocking=True)
-            d2h[k].record(s_out)
-        t1.record(s_out)
+            bench.step(bench.x, ev[k])
         torch.cuda.synchronize(dev)
-        barrier()
-        e_ms = ranks.max(float(t0.elapsed_time(t1)))
-        e2e = {"value": weak_scaling_rate(world, n_e2e, tokens_per_step, e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": xh.numel() * xh.element_size(),
-               "d2h_bytes_per_step": ohs[0].numel() * ohs[0].element_size(), "steps": n_e2e,
-               "path": "pinned host x -> device (copy stream), hymba_layer_fwd / hymba_stack_fwd (compute "
-                       "stream, L2 flushed before each step), device out -> pinned host (copy stream); two "
-                       "buffers each, so consecutive steps' copies and layers overlap"}
+        stages_us = {}
+        by_layer = []
+        for li in range(nl):
+            per = {name: 1e3 * float(np.mean([ev[k][li][i].elapsed_time(ev[k][li][i + 1]) for k in range(n_stage)]))
+                   for i, name in enumerate(H.STAGES)}
+            if bench.dt_in_scan[li]:   # stage 2 launches nothing: dt is computed inside the scan
+                per.pop("dt_proj")
+            by_layer.append({k: round(v, 2) for k, v in per.items()})
+            for k, v in per.items():
+                stages_us[k] = stages_us.get(k, 0.0) + v
+        stages_us = {k: round(v, 2) for k, v in stages_us.items()}
+        stage_roof, t_roof_us = stage_rooflines(wl.layers, stages_us, peaks, bench.dt_in_scan,
+                                                rec["clocks"].get("sm_max_mhz"))
+        top = max(stages_us, key=stages_us.get)
+        r = stage_roof[top]
+        kname = KERNEL_NAMES.get(top) or scan_kernel_name(wl.first)
+        n_launch = nl
+        peak_note = {"tensor": f"{peak_src} bf16_tflops (burst: the kernel runs inside a sub-second step)",
+                     "hbm": f"{peak_src} hbm_gbs (STREAM-style copy)",
+                     "alu": "fp32 FMA peak derived from 148 SMs x 128 lanes x 2 FLOP x the SM clock"}[r["bound"]]
+        traffic = _traffic(wl.name, top)
+        rec["roofline"] = {"kernel": f"{top} ({kname})", "bound": r["bound"], "achieved": r["achieved"],
+                           "peak": r["peak"], "unit": r["unit"], "frac": r["frac"],
+                           "traffic": traffic if traffic is None else traffic,
+                           "peak_source": peak_note, "launches_per_step": n_launch,
+                           "us_per_launch": round(stages_us[top] / n_launch, 2),
+                           "algorithmic_work_per_launch": r["work"] / n_launch}
+        rec["stages_us"] = stages_us
+        if nl > 1:
+            rec["stages_us_by_layer"] = by_layer
+        rec["stages_note"] = (f"stage events in a separate {n_stage}-step pass (events between kernels disable "
+                              "their programmatic overlap and the second stream)")
+        rec["stage_roofline"] = stage_roof
+        rec["layer_roofline"] = {"roofline_us": round(t_roof_us, 2), "measured_us": round(1e3 * rec["ms_per_step"], 2),
+                                 "frac": round(t_roof_us / (1e3 * rec["ms_per_step"]), 4),
+                                 "definition": "sum over stages and layers of max(tensor FLOPs / burst bf16 peak, "
+                                               "bytes / HBM peak, scan FMA FLOPs / fp32 peak where the CUDA-core "
+                                               "scan runs), against the timed step"}
+    elif bench.stack:
+        t_roof_us = stack_roofline_us(wl.layers, peaks, bench.dt_in_scan)
+        rec["layer_roofline"] = {"roofline_us": round(t_roof_us, 2), "measured_us": round(1e3 * rec["ms_per_step"], 2),
+                                 "frac": round(t_roof_us / (1e3 * rec["ms_per_step"]), 4),
+                                 "definition": "sum over the blocks of their stages' bounds plus the SwiGLU FFN and "
+                                               "pre-norms (max of tensor FLOPs / burst bf16 peak and bytes / HBM "
+                                               "peak), against the timed step"}
+    if e2e:
+        rec["e2e"] = measure_e2e(bench, ranks, dev, flush, K)
+    return rec, total_ms
+
+
+def measure_e2e(bench: Workbench, ranks, dev, flush, K):
+    """Through the public entry point with host buffers, as a serving loop runs it: each step
+    copies its input from pinned host memory and its output back, double-buffered over three
+    streams so that step k's input copy (host -> device), step k-1's layers (the compute
+    stream, with the same L2 flush before it) and step k-2's output copy (device -> host)
+    overlap.  Timed from the first timed input copy to the last output copy, on the device."""
+    import torch
+    x, outs, stream = bench.x, bench.outs, bench.stream
+    xh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    xh.copy_(x.cpu())
+    ohs = [torch.empty(outs[-1].shape, dtype=x.dtype).pin_memory() for _ in range(2)]
+    xds = [torch.empty_like(x) for _ in range(2)]
+    out_sets = [outs, [torch.empty_like(o) for o in outs]]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    n_e2e, n_warm = max(3, min(K, 50)), 3
+    total = n_warm + n_e2e
+    h2d = [torch.cuda.Event() for _ in range(total)]
+    comp = [torch.cuda.Event() for _ in range(total)]
+    d2h = [torch.cuda.Event() for _ in range(total)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    for k in range(total):
+        j = k % 2
+        if k == n_warm:
+            torch.cuda.synchronize(dev)   # warm-up steps done; the timed pipeline starts empty
+            t0.record(s_in)
+        if k >= 2:
+            s_in.wait_event(comp[k - 2])   # the layers that read xds[j] are done
+        with torch.cuda.stream(s_in):
+            xds[j].copy_(xh, non_blocking=True)
+        h2d[k].record(s_in)
+        stream.wait_event(h2d[k])
+        if k >= 2:
+            stream.wait_event(d2h[k - 2])  # out_sets[j] has been copied out
+        flush.zero_()
+        o = bench.step(xds[j], out_list=out_sets[j])
+        comp[k].record(stream)
+        s_out.wait_event(comp[k])
+        with torch.cuda.stream(s_out):
+            ohs[j].copy_(o, non_blocking=True)
+        d2h[k].record(s_out)
+    t1.record(s_out)
+    torch.cuda.synchronize(dev)
+    ranks.barrier()
+    e_ms = ranks.max(float(t0.elapsed_time(t1)))
+    return {"value": weak_scaling_rate(ranks.world, n_e2e, bench.tokens, e_ms), "unit": UNIT,
+            "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+            "d2h_bytes_per_step": ohs[0].numel() * ohs[0].element_size(), "steps": n_e2e,
+            "path": "pinned host x -> device (copy stream), hymba_layer_fwd / hymba_stack_fwd (compute "
+                    "stream, L2 flushed before each step), device out -> pinned host (copy stream); two "
+                    "buffers each, so consecutive steps' copies and layers overlap"}
+
+
+def measure_decode(name: str, dev, flush, steps: int = 64, warmup: int = 8):
+    """Generation steps of a layer workload after its full prompt: hymba_layer_prefill of every
+    layer (untimed), then one new token per sequence per step through every layer
+    (hymba_layer_decode), timed with CUDA events over `steps` steps."""
+    import torch
+
+    import hybrid_attention_ssm_hymba_b200 as H
+    from hybrid_attention_ssm_hymba_b200 import host
+    wl = synth.workload(name)
+    s0 = wl.first
+    dt = s0.dtype
+    x_np, meta_np = synth.layer_inputs(wl)
+    dps = [host.params_to_device(synth.layer_params(wl, i), dt, dev) for i in range(len(wl.layers))]
+    cfgs = [H.make_cfg(s) for s in wl.layers]
+    T = s0.T
+    cap = T + warmup + steps
+    ws = host.workspace(max(H.hymba_decode_workspace_size(c) for c in cfgs), dev)
+    cache = torch.zeros((2, s0.batch, cap, s0.kv_width), dtype=host.torch_dtype(dt), device=dev)
+    states = [torch.zeros((s0.batch, s.d_inner, s.d_state), dtype=torch.float32, device=dev) for s in wl.layers]
+    weights = [H.make_weights(d) for d in dps]
+    xin, meta = host.to_device(x_np, dt, dev), host.to_device(meta_np, dt, dev)
+    for i, c in enumerate(cfgs):
+        out = torch.empty((s0.batch, T, s0.d_model), dtype=host.torch_dtype(dt), device=dev)
+        H.check(H.hymba_layer_prefill(xin, meta, weights[i], c, cache, cap, states[i], out, ws), "prefill")
+        xin, meta = out, None
+    toks = torch.randn((warmup + steps, s0.batch, s0.d_model), device=dev).to(host.torch_dtype(dt))
+    bufs = [torch.empty((s0.batch, s0.d_model), dtype=host.torch_dtype(dt), device=dev) for _ in wl.layers]
+
+    def one(k):
+        xi = toks[k]
+        for i, c in enumerate(cfgs):
+            H.check(H.hymba_layer_decode(xi, weights[i], c, cache, cap, T + k, states[i], bufs[i], ws), "decode")
+            xi = bufs[i]
+
+    for k in range(warmup):
+        one(k)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for k in range(warmup, warmup + steps):
+        one(k)
+    t1.record()
+    torch.cuda.synchronize(dev)
+    assert H.hymba_workspace_status(ws) == H.HYMBA_OK
+    ms = t0.elapsed_time(t1)
+    return {"workload": name, "tokens_per_s": s0.batch * steps / (ms * 1e-3), "unit": "tokens/s",
+            "us_per_step": round(1e3 * ms / steps, 2), "steps": steps, "batch": s0.batch,
+            "context_rows": [T + warmup, T + warmup + steps], "layers": len(cfgs),
+            "launches_per_step": 8 * len(cfgs),
+            "note": "one new token per sequence per step through every layer of the workload, after the "
+                    "full prompt; K/V cache and SSM state resident; no L2 flush between steps (a generation "
+                    "loop re-reads the same weights)"}
+
+
+def run_native(args, rank, world, local_rank):
+    import torch
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    ranks = Ranks(world, local_rank, "nccl", dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    bench = Workbench(args.workload, dev)
+    K = args.steps
+    rec, total_ms = measure(bench, K, args.warmup, ranks, dev, flush, stages=True, e2e=not args.no_e2e)
+    value = weak_scaling_rate(world, K, bench.tokens, total_ms)
+    status = bench.H.hymba_workspace_status(bench.ws, bench.stream)
+    wl, s0 = bench.wl, bench.s0
 
     line = None
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+                "scaling": "weak", "vs_baseline": None, "dtype": bench.dtype, "data": "synthetic",
                 "config": _workload_config(wl, {
                     "parallelism": f"replicas x{world} (batch per rank, no collective)" if world > 1 else "1 GPU",
-                    "tokens_per_step_per_gpu": tokens_per_step, "rows_per_step_per_gpu": s0.batch * T,
-                    "l2": "flushed between timed steps (256 MiB memset outside the events)"}),
-                "roofline": roofline, "stages_us": stages, "stages_note": "stage events in a separate "
-                f"{n_stage}-step pass (events between kernels disable their programmatic overlap)" if stages else None,
-                "stage_roofline": stage_roof,
-                "layer_roofline": layer_roof, "e2e": e2e,
-                "gpu_launches": n_launch_per_step * K, "clocks": sampler.summary(),
-                "device_status": H.hymba_status_string(status)}
+                    "tokens_per_step_per_gpu": bench.tokens, "rows_per_step_per_gpu": s0.batch * s0.T,
+                    "l2": "flushed between timed steps (256 MiB memset outside the events)"})}
+        for k in ("roofline", "stages_us", "stages_us_by_layer", "stages_note", "stage_roofline", "layer_roofline",
+                  "e2e", "gpu_launches", "clocks"):
+            if k in rec:
+                line[k] = rec[k]
+        line["device_status"] = bench.H.hymba_status_string(status)
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl, x_np, meta_np, ps_np)
+            line["cpu_baseline"] = cpu_baseline(wl, bench.x_np, bench.meta_np, bench.ps_np)
+    del bench
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_per_workload:
+        per = {}
+        for name in synth.WORKLOAD_ORDER:
+            if name == args.workload:
+                continue
+            b = Workbench(name, dev)
+            k = min(K, 10 if not b.stack else 3)
+            r, t_ms = measure(b, k, 3, ranks, dev, flush, stages=True, e2e=False)
+            r["value"] = weak_scaling_rate(1, k, b.tokens, t_ms)
+            r["unit"] = UNIT
+            r["dtype"] = b.dtype
+            r["config"] = _workload_config(b.wl)
+            if rank == 0 and not args.no_cpu_baseline:
+                r["cpu_baseline"] = cpu_baseline(b.wl, b.x_np, b.meta_np, b.ps_np, budget_s=6.0)
+            per[name] = r
+            del b
+            torch.cuda.empty_cache()
+        if line is not None:
+            line["per_workload"] = per
+    if world == 1 and not args.no_decode and line is not None:
+        line["decode"] = measure_decode("hymba1p5b_kvpair", dev, flush)
+    if line is not None:
         print(json.dumps(line), flush=True)
     ranks.close()
     return 0
@@ -520,10 +737,12 @@ def run_native(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="hymba350m_layer", choices=synth.WORKLOAD_ORDER)
+    ap.add_argument("--workload", default="hymba1p5b_kvpair", choices=synth.WORKLOAD_ORDER)
+    ap.add_argument("--no-per-workload", action="store_true", help="skip the other workloads' lines")
+    ap.add_argument("--no-decode", action="store_true", help="skip the generation-step measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()

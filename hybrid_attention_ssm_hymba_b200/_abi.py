@@ -24,6 +24,7 @@ ENTRY_POINTS = (
     "hymba_status_string", "hymba_workspace_size", "hymba_stack_workspace_size", "hymba_layer_fwd",
     "hymba_stack_fwd", "hymba_workspace_status", "hymba_layer_fwd_events", "hymba_gemm", "hymba_selective_scan",
     "hymba_attention", "hymba_branch_norm", "hymba_rmsnorm", "hymba_layer_fwd_noalloc", "hymba_layer_fuses_dt_proj",
+    "hymba_check_wait_timeout", "hymba_decode_workspace_size", "hymba_layer_prefill", "hymba_layer_decode",
 )
 
 # size of the library-owned scratch block behind hymba_layer_fwd_noalloc (HYMBA_NOALLOC_SCRATCH_BYTES)
@@ -46,7 +47,8 @@ class hymba_cfg_t(ctypes.Structure):
 
 class hymba_weights_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
-        "w_in", "w_x", "w_dt", "w_out", "a_log", "b_dt", "beta1", "beta2", "w_gate_up", "w_down")]
+        "w_in", "w_x", "w_dt", "w_out", "a_log", "b_dt", "beta1", "beta2", "w_gate_up", "w_down",
+        "norm1", "norm2")]
 
 
 _VP, _SZ, _I, _F = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
@@ -69,6 +71,12 @@ _SIGS = {
     "hymba_attention": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "hymba_branch_norm": (_I, [_VP, _VP, _VP, _I, _I, _I, _F, _I, _VP]),
     "hymba_rmsnorm": (_I, [_VP, _VP, _I, _I, _F, _I, _VP]),
+    "hymba_check_wait_timeout": (_I, [_VP, _SZ, ctypes.c_uint, _VP]),
+    "hymba_decode_workspace_size": (_SZ, [ctypes.POINTER(hymba_cfg_t)]),
+    "hymba_layer_prefill": (_I, [_VP, _VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t),
+                                 _VP, _I, _VP, _VP, _VP, _SZ, _VP]),
+    "hymba_layer_decode": (_I, [_VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t),
+                                _VP, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
 }
 
 _lib = None
@@ -228,6 +236,30 @@ def hymba_branch_norm(z, beta1, beta2, rows: int, w_attn: int, w_ssm: int, eps: 
 
 def hymba_rmsnorm(x, y, rows: int, d: int, eps: float, dtype: int, stream=None) -> int:
     return load().hymba_rmsnorm(_ptr(x), _ptr(y), rows, d, eps, dtype, _stream(stream))
+
+
+def hymba_decode_workspace_size(cfg: hymba_cfg_t) -> int:
+    return load().hymba_decode_workspace_size(ctypes.byref(cfg))
+
+
+def hymba_layer_prefill(x, meta, weights: hymba_weights_t, cfg: hymba_cfg_t, kv_cache, cache_rows: int,
+                        ssm_state, out, workspace, stream=None) -> int:
+    return load().hymba_layer_prefill(_ptr(x), _ptr(meta), ctypes.byref(weights), ctypes.byref(cfg),
+                                      _ptr(kv_cache), int(cache_rows), _ptr(ssm_state), _ptr(out),
+                                      _ptr(workspace), _nbytes(workspace), _stream(stream))
+
+
+def hymba_layer_decode(x_t, weights: hymba_weights_t, cfg: hymba_cfg_t, kv_cache, cache_rows: int, pos: int,
+                       ssm_state, out_t, workspace, stream=None) -> int:
+    return load().hymba_layer_decode(_ptr(x_t), ctypes.byref(weights), ctypes.byref(cfg), _ptr(kv_cache),
+                                     int(cache_rows), int(pos), _ptr(ssm_state), _ptr(out_t), _ptr(workspace),
+                                     _nbytes(workspace), _stream(stream))
+
+
+def hymba_check_wait_timeout(workspace, limit_us: int, stream=None) -> int:
+    """Runs the bounded-wait failure path once (a wait that nothing ends, limited to
+    limit_us); the workspace's status word then reads HYMBA_ERR_TIMEOUT."""
+    return load().hymba_check_wait_timeout(_ptr(workspace), _nbytes(workspace), int(limit_us), _stream(stream))
 
 
 def check(status: int, what: str = "") -> None:

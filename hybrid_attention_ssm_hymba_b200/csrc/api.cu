@@ -14,7 +14,9 @@
 // Z, beta is folded into W_out's columns, and out_proj accumulates the attention and
 // SSM columns apart and scales each by its row's 1 / rms.
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "hy_common.cuh"
 #include "hy_kernels.h"
@@ -58,6 +60,45 @@ LayerWs layer_ws(const hymba_cfg_t& c, size_t base) {
   const bool fused = fused_branch_norm(c);
   w.ssq = o; o = al256(o + (fused ? rows * 2 * sizeof(float) : 0));
   w.wsc = o; o = al256(o + (fused ? static_cast<size_t>(c.d_model) * (wa + c.d_inner) * es : 0));
+  w.total = o;
+  return w;
+}
+
+// Workspace of hymba_stack_fwd (after the 256-byte status word): the largest layer's
+// workspace, the normalised block input xn (dtype) and, for bf16, its rounding remainder
+// xlo and the fp32 residual stream h; K/V of the current pair; the FFN activation; for
+// bf16 the transposed W_SSM and W_eff = W_x W_SSM of the current block.
+struct StackWs {
+  size_t layer, xn, xlo, h, kv, act, wssm_t, weff, total;
+};
+
+StackWs stack_ws(const hymba_cfg_t* cfgs, int n) {
+  const hymba_cfg_t& c = cfgs[0];
+  const size_t es = esize(c.dtype);
+  const bool bf16 = c.dtype == HYMBA_BF16;
+  const size_t rows = static_cast<size_t>(c.batch) * (c.seq_len + c.n_meta);
+  const size_t d = static_cast<size_t>(c.d_model);
+  size_t layer_max = 0, kvw = 0, ffn = 0, di = 0, xw = 0;
+  for (int i = 0; i < n; ++i) {
+    const size_t t = layer_ws(cfgs[i], 0).total;
+    layer_max = t > layer_max ? t : layer_max;
+    const size_t k = static_cast<size_t>(cfgs[i].n_kv_heads) * cfgs[i].head_dim;
+    kvw = k > kvw ? k : kvw;
+    ffn = static_cast<size_t>(cfgs[i].ffn_dim) > ffn ? cfgs[i].ffn_dim : ffn;
+    di = static_cast<size_t>(cfgs[i].d_inner) > di ? cfgs[i].d_inner : di;
+    const size_t x = static_cast<size_t>(cfgs[i].dt_rank) + 2 * cfgs[i].d_state;
+    xw = x > xw ? x : xw;
+  }
+  StackWs w;
+  size_t o = 0;
+  w.layer = o; o = al256(o + layer_max);
+  w.xn = o; o = al256(o + rows * d * es);
+  w.xlo = o; o = al256(o + (bf16 ? rows * d * 2 : 0));
+  w.h = o; o = al256(o + (bf16 ? rows * d * 4 : 0));
+  w.kv = o; o = al256(o + 2 * rows * kvw * es);
+  w.act = o; o = al256(o + rows * ffn * es);
+  w.wssm_t = o; o = al256(o + (bf16 ? d * di * 2 : 0));
+  w.weff = o; o = al256(o + (bf16 ? xw * d * 2 : 0));
   w.total = o;
   return w;
 }
@@ -114,18 +155,37 @@ bool weights_ok(const hymba_weights_t* w, const hymba_cfg_t& c, bool need_ffn) {
 }
 
 // The attention heads and the SSM heads of a layer are independent until the branch
-// norm: the attention runs on a second stream of the library's (one per device, made on
-// first use), forked from the caller's stream after in_proj and joined back before the
-// norm, so that its CTAs and the scan's fill the SMs together.
-cudaStream_t side_stream() {
-  static std::mutex mu;
-  static cudaStream_t streams[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
-    streams[dev] = nullptr;
-  return streams[dev];
+// norm: the attention runs on a second stream of the library's, forked from the caller's
+// stream after in_proj and joined back before the norm, so that its CTAs and the scan's
+// fill the SMs together.  One second stream (with its fork and join events) per host
+// thread, device and stream priority: calls from different threads never share one, and
+// the attention keeps the caller stream's priority.  Calls made on several streams from
+// the same thread do share it (their attention launches are ordered on it).
+struct SideStream {
+  cudaStream_t st = nullptr;
+  cudaEvent_t forked = nullptr, done = nullptr;
+};
+
+bool side_stream(cudaStream_t caller, SideStream* out) {
+  thread_local std::map<std::pair<int, int>, SideStream> cache;
+  int dev = 0, prio = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaStreamGetPriority(caller, &prio) != cudaSuccess) return false;
+  SideStream& e = cache[std::make_pair(dev, prio)];
+  if (!e.st) {
+    if (cudaStreamCreateWithPriority(&e.st, cudaStreamNonBlocking, prio) != cudaSuccess) {
+      e.st = nullptr;
+      return false;
+    }
+    if (cudaEventCreateWithFlags(&e.forked, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&e.done, cudaEventDisableTiming) != cudaSuccess) {
+      cudaStreamDestroy(e.st);
+      e = SideStream();
+      return false;
+    }
+  }
+  *out = e;
+  return true;
 }
 
 // Joins the side stream back into the caller's stream once (at join() or on any return).
@@ -135,18 +195,33 @@ struct SideJoin {
   cudaError_t join() {
     if (!done) return cudaSuccess;
     const cudaError_t e = cudaStreamWaitEvent(st, done, 0);
-    cudaEventDestroy(done);
     done = nullptr;
     return e;
   }
   ~SideJoin() { join(); }
 };
 
+// Where a layer's out_proj writes: out = Z W_out^T, or out = resid + Z W_out^T (resid may
+// alias out), each in the layer's dtype or in fp32 (a stack's fp32 residual stream).
+// xlo / weff: the x_proj of a stacked block adds xlo W_eff^T (xlo the bf16 rounding
+// remainder of the block's normalised input, W_eff = W_x W_SSM) to [dt_low | B | C].
+// h_out: the SSM heads' state after the last row [B, Di, N] fp32 (a prefill that a
+// generation step continues); kv_rows: rows per sequence of a consumed K/V buffer (a cache).
+struct LayerOut {
+  void* out = nullptr;
+  const void* resid = nullptr;
+  bool resid_f32 = false, out_f32 = false;
+  const void* xlo = nullptr;
+  const void* weff = nullptr;
+  float* h_out = nullptr;
+  long long kv_rows = 0;
+};
+
 // One layer.  x: meta mode when meta != nullptr, else [rows, d] holding X~.
-// resid_out: when true the out_proj adds into `out` (out = out + Z W_out^T).
 hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t& w, const hymba_cfg_t& c,
-                         const void* kv_in, void* kv_out, void* out, bool resid_out, uint8_t* ws, unsigned* status,
+                         const void* kv_in, void* kv_out, const LayerOut& lo, uint8_t* ws, unsigned* status,
                          cudaStream_t st, void* const* events = nullptr) {
+  void* out = lo.out;
   bool marks_ok = true;
   auto mark = [&](int i) {
     if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) != cudaSuccess) marks_ok = false;
@@ -180,6 +255,7 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   sd.bf16 = c.dtype == HYMBA_BF16;
   sd.status = status;
   sd.a_per_state = c.a_per_state != 0;
+  sd.h_out = lo.h_out;
   // bf16 with d_state 16 and dt_rank 64: dt_proj runs inside the tensor-core scan
   // (dt = softplus(dt_low W_dt^T + b_dt) per block, never stored)
   {
@@ -199,7 +275,8 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   void* w_out_scaled = ws + L.wsc;
   void* kvbuf = c.kv_mode == HYMBA_KV_PRODUCE ? kv_out : (c.kv_mode == HYMBA_KV_OWN ? ws + L.kv : nullptr);
   const void* kv_k = c.kv_mode == HYMBA_KV_CONSUME ? kv_in : kvbuf;
-  const void* kv_v = static_cast<const uint8_t*>(kv_k) + static_cast<size_t>(rows) * wkv * es;
+  const long long kv_seq_rows = (c.kv_mode == HYMBA_KV_CONSUME && lo.kv_rows > 0) ? lo.kv_rows : T;
+  const void* kv_v = static_cast<const uint8_t*>(kv_k) + static_cast<size_t>(c.batch) * kv_seq_rows * wkv * es;
 
   // 1 in_proj
   mark(0);
@@ -255,21 +332,21 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   ad.window = c.window;
   ad.bf16 = c.dtype == HYMBA_BF16;
   ad.status = status;
-  cudaStream_t side = events ? nullptr : side_stream();
+  ad.kv_rows = c.kv_mode == HYMBA_KV_CONSUME ? lo.kv_rows : 0;
+  SideStream ss;
+  cudaStream_t side = nullptr;
+  if (!events) {
+    if (!side_stream(st, &ss)) return HYMBA_ERR_CUDA;
+    side = ss.st;
+  }
   SideJoin joiner;
   joiner.st = st;
   if (side) {
-    cudaEvent_t forked = nullptr, done = nullptr;
-    if (cudaEventCreateWithFlags(&forked, cudaEventDisableTiming) != cudaSuccess) return HYMBA_ERR_CUDA;
-    const bool ok = cudaEventRecord(forked, st) == cudaSuccess && cudaStreamWaitEvent(side, forked, 0) == cudaSuccess;
-    cudaEventDestroy(forked);
-    if (!ok || cudaEventCreateWithFlags(&done, cudaEventDisableTiming) != cudaSuccess) return HYMBA_ERR_CUDA;
-    const cudaError_t ea = hy::launch_attention(ad, side);
-    if (cudaEventRecord(done, side) != cudaSuccess) {
-      cudaEventDestroy(done);
+    if (cudaEventRecord(ss.forked, st) != cudaSuccess || cudaStreamWaitEvent(side, ss.forked, 0) != cudaSuccess)
       return HYMBA_ERR_CUDA;
-    }
-    joiner.done = done;
+    const cudaError_t ea = hy::launch_attention(ad, side);
+    if (cudaEventRecord(ss.done, side) != cudaSuccess) return HYMBA_ERR_CUDA;
+    joiner.done = ss.done;
     if (ea != cudaSuccess) return HYMBA_ERR_CUDA;
   }
 
@@ -283,6 +360,11 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   gx.N = c.dt_rank + 2 * c.d_state;
   gx.seg[gx.nseg++] = seg(0, c.dt_rank, dtlow, c.dt_rank, f32out, hy::SEG_STORE);
   gx.seg[gx.nseg++] = seg(c.dt_rank, gx.N, bc, 2 * c.d_state, 1, hy::SEG_STORE);
+  if (lo.xlo && c.dtype == HYMBA_BF16) {
+    gx.a2 = lo.xlo;
+    gx.w2 = lo.weff;
+    gx.K2 = c.d_model;
+  }
   gx.status = status;
   if ((e = gemm(gx, c.dtype, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
 
@@ -336,12 +418,14 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
     go.out = out;
     go.out_ld = c.d_model;
   }
-  if (resid_out) {
+  if (lo.resid) {
     go.epi = hy::EPI_RESIDUAL;
-    go.resid = out;
+    go.resid = lo.resid;
     go.resid_ld = c.d_model;
     go.out = out;
     go.out_ld = c.d_model;
+    go.resid_f32 = lo.resid_f32;
+    go.out_f32 = lo.out_f32;
   } else {
     go.seg[go.nseg++] = seg(0, c.d_model, out, c.d_model, f32out, hy::SEG_STORE);
   }
@@ -397,6 +481,47 @@ cudaError_t noalloc_scratch(uint8_t** out) {
   return cudaSuccess;
 }
 
+// ---- generation (prefill with state, decode step)
+
+constexpr int kMaxDecodeSplits = 256;
+
+struct DecodeWs {
+  size_t q, xs, g, dt, dtlow, bc, z, part, total;
+};
+
+DecodeWs decode_ws(const hymba_cfg_t& c) {
+  const size_t es = esize(c.dtype), B = static_cast<size_t>(c.batch);
+  const size_t wa = static_cast<size_t>(c.n_q_heads) * c.head_dim;
+  DecodeWs w;
+  size_t o = 0;
+  w.q = o; o = al256(o + B * wa * es);
+  w.xs = o; o = al256(o + B * c.d_inner * es);
+  w.g = o; o = al256(o + B * c.d_inner * es);
+  w.dt = o; o = al256(o + B * c.d_inner * es);
+  w.dtlow = o; o = al256(o + B * c.dt_rank * es);
+  w.bc = o; o = al256(o + B * 2 * c.d_state * 4);
+  w.z = o; o = al256(o + B * (wa + c.d_inner) * es);
+  w.part = o; o = al256(o + B * c.n_q_heads * kMaxDecodeSplits * (c.head_dim + 2) * 4);
+  w.total = o;
+  return w;
+}
+
+// the prefill runs the layer with its K/V in the workspace (own mode) and copies them into
+// the cache; a consuming layer reads the producer's cache in place
+hymba_cfg_t prefill_cfg(const hymba_cfg_t& c) {
+  hymba_cfg_t p = c;
+  if (p.kv_mode == HYMBA_KV_PRODUCE) p.kv_mode = HYMBA_KV_OWN;
+  return p;
+}
+
+hymba_status_t validate_generation(const hymba_cfg_t* cfg) {
+  hymba_status_t s = validate_cfg(cfg);
+  if (s != HYMBA_OK) return s;
+  if (cfg->head_dim % 32 || cfg->n_q_heads / cfg->n_kv_heads > 8 || cfg->d_state % 8)
+    return HYMBA_ERR_UNSUPPORTED;
+  return HYMBA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -437,22 +562,9 @@ size_t hymba_workspace_size(const hymba_cfg_t* cfg) {
 
 size_t hymba_stack_workspace_size(const hymba_cfg_t* cfgs, int n_layers) {
   if (!cfgs || n_layers < 1) return 0;
-  size_t layer_max = 0;
-  for (int i = 0; i < n_layers; ++i) {
+  for (int i = 0; i < n_layers; ++i)
     if (validate_cfg(&cfgs[i]) != HYMBA_OK) return 0;
-    const size_t t = layer_ws(cfgs[i], 0).total;
-    layer_max = t > layer_max ? t : layer_max;
-  }
-  const hymba_cfg_t& c = cfgs[0];
-  const size_t es = esize(c.dtype);
-  const size_t rows = static_cast<size_t>(c.batch) * (c.seq_len + c.n_meta);
-  size_t kvw = 0, ffn = 0;
-  for (int i = 0; i < n_layers; ++i) {
-    const size_t w = static_cast<size_t>(cfgs[i].n_kv_heads) * cfgs[i].head_dim;
-    kvw = w > kvw ? w : kvw;
-    ffn = static_cast<size_t>(cfgs[i].ffn_dim) > ffn ? cfgs[i].ffn_dim : ffn;
-  }
-  return 256 + al256(layer_max) + al256(rows * c.d_model * es) + al256(2 * rows * kvw * es) + al256(rows * ffn * es);
+  return 256 + stack_ws(cfgs, n_layers).total;
 }
 
 hymba_status_t hymba_layer_fwd(const void* x, const void* meta, const hymba_weights_t* w, const hymba_cfg_t* cfg,
@@ -477,7 +589,9 @@ hymba_status_t hymba_layer_fwd_events(const void* x, const void* meta, const hym
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned* status = static_cast<unsigned*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;
-  return run_layer(x, cfg->n_meta > 0 ? meta : nullptr, *w, *cfg, kv_in, kv_out, out, false,
+  LayerOut lo;
+  lo.out = out;
+  return run_layer(x, cfg->n_meta > 0 ? meta : nullptr, *w, *cfg, kv_in, kv_out, lo,
                    static_cast<uint8_t*>(workspace) + 256, status, st, events);
 }
 
@@ -498,8 +612,9 @@ hymba_status_t hymba_layer_fwd_noalloc(const void* x, const void* meta, const hy
   // the block keeps the previous call's contents: the status word must start at zero
   // (every intermediate is written before it is read)
   if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;
-  return run_layer(x, cfg->n_meta > 0 ? meta : nullptr, *w, *cfg, kv_in, kv_out, out, false, scratch + 256, status,
-                   st);
+  LayerOut lo;
+  lo.out = out;
+  return run_layer(x, cfg->n_meta > 0 ? meta : nullptr, *w, *cfg, kv_in, kv_out, lo, scratch + 256, status, st);
 }
 
 hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weights_t* w, const hymba_cfg_t* cfgs,
@@ -526,28 +641,30 @@ hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weig
   unsigned* status = static_cast<unsigned*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;
 
-  size_t layer_max = 0, kvw = 0;
-  for (int i = 0; i < n_layers; ++i) {
-    const size_t t = layer_ws(cfgs[i], 0).total;
-    layer_max = t > layer_max ? t : layer_max;
-    const size_t k = static_cast<size_t>(cfgs[i].n_kv_heads) * cfgs[i].head_dim;
-    kvw = k > kvw ? k : kvw;
-  }
-  const size_t es = esize(c0.dtype);
+  const StackWs S = stack_ws(cfgs, n_layers);
+  uint8_t* base = static_cast<uint8_t*>(workspace) + 256;
+  const bool bf16 = c0.dtype == HYMBA_BF16;
   const int T = c0.seq_len + c0.n_meta;
   const long long rows = static_cast<long long>(c0.batch) * T;
-  uint8_t* base = static_cast<uint8_t*>(workspace) + 256;
-  uint8_t* lws = base;
-  uint8_t* xn = lws + al256(layer_max);
-  uint8_t* kv = xn + al256(rows * c0.d_model * es);
-  uint8_t* act = kv + al256(2 * rows * kvw * es);
-  const bool bf16 = c0.dtype == HYMBA_BF16;
+  const int d = c0.d_model;
+  uint8_t* lws = base + S.layer;
+  void* xn = base + S.xn;
+  void* xlo = bf16 ? base + S.xlo : nullptr;
+  void* kv = base + S.kv;
+  void* act = base + S.act;
+  // the residual stream h: fp32 in the workspace (bf16), or `out` itself (fp32)
+  float* h = bf16 ? reinterpret_cast<float*>(base + S.h) : static_cast<float*>(out);
+  void* wssm_t = base + S.wssm_t;
+  void* weff = base + S.weff;
 
-  // h = [meta; x] lives in `out` and is updated in place
-  {
-    const long long row_vecs = static_cast<long long>(c0.d_model) * es / 16;
+  cudaError_t e;
+  if (bf16) {
+    if ((e = hy::launch_prepend_f32(x, meta, h, c0.batch, c0.seq_len, c0.n_meta, d, st)) != cudaSuccess)
+      return HYMBA_ERR_CUDA;
+  } else {
+    // h = [meta; x] lives in `out` and is updated in place
+    const long long row_vecs = static_cast<long long>(d) * 4 / 16;
     const long long total = rows * row_vecs;
-    if (c0.d_model * es % 16) return HYMBA_ERR_UNSUPPORTED;
     const int blocks = static_cast<int>(total / 256 + 1 < 4096 ? total / 256 + 1 : 4096);
     if (hy::launch(prepend_kernel, dim3(blocks), dim3(256), 0, st, static_cast<const uint4*>(x),
                    static_cast<const uint4*>(meta), static_cast<uint4*>(out), row_vecs, c0.seq_len, c0.n_meta,
@@ -556,17 +673,48 @@ hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weig
   }
   for (int i = 0; i < n_layers; ++i) {
     const hymba_cfg_t& c = cfgs[i];
-    cudaError_t e = hy::launch_rmsnorm(out, xn, rows, c.d_model, c.rms_eps, bf16, st);
-    if (e != cudaSuccess) return HYMBA_ERR_CUDA;
-    hymba_status_t s = run_layer(xn, nullptr, w[i], c, kv, kv, out, true, lws, status, st);
+    const bool last = i == n_layers - 1;
+    LayerOut lo;
+    lo.resid = h;
+    lo.resid_f32 = true;
+    // the last sub-block rounds h into `out` (bf16); every other one updates h in place
+    const bool mixer_last = last && c.ffn_dim == 0;
+    lo.out = (bf16 && mixer_last) ? out : static_cast<void*>(h);
+    lo.out_f32 = !(bf16 && mixer_last);
+    if (bf16) {
+      if ((e = hy::launch_prenorm_f32(h, w[i].norm1, xn, xlo, rows, d, c.rms_eps, st)) != cudaSuccess)
+        return HYMBA_ERR_CUDA;
+      // W_eff = W_x W_SSM [R + 2N, d]: x_proj adds xlo W_eff^T, the part of [dt_low | B | C]
+      // that the bf16 rounding of the normalised input dropped
+      const int wa = c.n_q_heads * c.head_dim, wkv = c.n_kv_heads * c.head_dim;
+      const int ssm_row0 = wa + (c.kv_mode == HYMBA_KV_CONSUME ? 0 : 2 * wkv);
+      const uint8_t* wssm = static_cast<const uint8_t*>(w[i].w_in) + static_cast<size_t>(ssm_row0) * d * 2;
+      if ((e = hy::launch_transpose_bf16(wssm, d, wssm_t, c.d_inner, d, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
+      GemmDesc ge;
+      ge.a = w[i].w_x;
+      ge.a_rows = c.dt_rank + 2 * c.d_state;
+      ge.K = c.d_inner;
+      ge.w = wssm_t;
+      ge.N = d;
+      ge.seg[ge.nseg++] = seg(0, d, weff, d, 0, hy::SEG_STORE);
+      ge.status = status;
+      if (gemm(ge, c.dtype, st) != cudaSuccess) return HYMBA_ERR_CUDA;
+      lo.xlo = xlo;
+      lo.weff = weff;
+    } else if ((e = hy::launch_prenorm_f32_out_f32(h, w[i].norm1, static_cast<float*>(xn), rows, d, c.rms_eps,
+                                                   st)) != cudaSuccess) {
+      return HYMBA_ERR_CUDA;
+    }
+    hymba_status_t s = run_layer(xn, nullptr, w[i], c, kv, kv, lo, lws, status, st);
     if (s != HYMBA_OK) return s;
     if (c.ffn_dim > 0) {
-      if ((e = hy::launch_rmsnorm(out, xn, rows, c.d_model, c.rms_eps, bf16, st)) != cudaSuccess)
-        return HYMBA_ERR_CUDA;
+      e = bf16 ? hy::launch_prenorm_f32(h, w[i].norm2, xn, nullptr, rows, d, c.rms_eps, st)
+               : hy::launch_prenorm_f32_out_f32(h, w[i].norm2, static_cast<float*>(xn), rows, d, c.rms_eps, st);
+      if (e != cudaSuccess) return HYMBA_ERR_CUDA;
       GemmDesc gu;
       gu.a = xn;
       gu.a_rows = rows;
-      gu.K = c.d_model;
+      gu.K = d;
       gu.w = w[i].w_gate_up;
       gu.N = 2 * c.ffn_dim;
       gu.epi = hy::EPI_SWIGLU;
@@ -580,17 +728,176 @@ hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weig
       gdn.a_rows = rows;
       gdn.K = c.ffn_dim;
       gdn.w = w[i].w_down;
-      gdn.N = c.d_model;
+      gdn.N = d;
       gdn.epi = hy::EPI_RESIDUAL;
-      gdn.resid = out;
-      gdn.resid_ld = c.d_model;
-      gdn.out = out;
-      gdn.out_ld = c.d_model;
+      gdn.resid = h;
+      gdn.resid_ld = d;
+      gdn.resid_f32 = true;
+      gdn.out = (bf16 && last) ? out : static_cast<void*>(h);
+      gdn.out_f32 = !(bf16 && last);
+      gdn.out_ld = d;
       gdn.status = status;
       if (gemm(gdn, c.dtype, st) != cudaSuccess) return HYMBA_ERR_CUDA;
     }
   }
   return HYMBA_OK;
+}
+
+// ---- generation: prefill that keeps the K/V cache and the SSM state, then one token per step
+
+size_t hymba_decode_workspace_size(const hymba_cfg_t* cfg) {
+  if (validate_generation(cfg) != HYMBA_OK) return 0;
+  const hymba_cfg_t p = prefill_cfg(*cfg);
+  const size_t a = layer_ws(p, 0).total, b = decode_ws(*cfg).total;
+  return 256 + (a > b ? a : b);
+}
+
+hymba_status_t hymba_layer_prefill(const void* x, const void* meta, const hymba_weights_t* w, const hymba_cfg_t* cfg,
+                                   void* kv_cache, int cache_rows, float* ssm_state, void* out, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  hymba_status_t s = validate_generation(cfg);
+  if (s != HYMBA_OK) return s;
+  const int T = cfg->seq_len + cfg->n_meta;
+  if (!x || !out || !kv_cache || !ssm_state || !weights_ok(w, *cfg, false) || cache_rows < T)
+    return HYMBA_ERR_INVALID_ARG;
+  if (cfg->n_meta > 0 && !meta) return HYMBA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < hymba_decode_workspace_size(cfg)) return HYMBA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return HYMBA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* status = static_cast<unsigned*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  const hymba_cfg_t p = prefill_cfg(*cfg);
+  uint8_t* ws = static_cast<uint8_t*>(workspace) + 256;
+  LayerOut lo;
+  lo.out = out;
+  lo.h_out = ssm_state;
+  lo.kv_rows = cache_rows;
+  s = run_layer(x, meta, *w, p, cfg->kv_mode == HYMBA_KV_CONSUME ? kv_cache : nullptr, nullptr, lo, ws, status, st);
+  if (s != HYMBA_OK || cfg->kv_mode == HYMBA_KV_CONSUME) return s;
+  // K, V [2][B*T][wkv] in the workspace -> the cache [2][B][cache_rows][wkv]
+  const size_t es = esize(cfg->dtype), wkv = static_cast<size_t>(cfg->n_kv_heads) * cfg->head_dim;
+  const LayerWs L = layer_ws(p, 0);
+  if (cudaMemcpy2DAsync(kv_cache, static_cast<size_t>(cache_rows) * wkv * es, ws + L.kv, T * wkv * es,
+                        T * wkv * es, 2 * static_cast<size_t>(cfg->batch), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return HYMBA_ERR_CUDA;
+  return HYMBA_OK;
+}
+
+hymba_status_t hymba_layer_decode(const void* x_t, const hymba_weights_t* w, const hymba_cfg_t* cfg, void* kv_cache,
+                                  int cache_rows, int pos, float* ssm_state, void* out_t, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+  hymba_status_t s = validate_generation(cfg);
+  if (s != HYMBA_OK) return s;
+  const hymba_cfg_t& c = *cfg;
+  if (!x_t || !out_t || !kv_cache || !ssm_state || !weights_ok(w, c, false) || pos < 0 || pos >= cache_rows)
+    return HYMBA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < hymba_decode_workspace_size(cfg)) return HYMBA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return HYMBA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* status = static_cast<unsigned*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace) + 256;
+  const DecodeWs D = decode_ws(c);
+  const size_t es = esize(c.dtype);
+  const int wa = c.n_q_heads * c.head_dim, wkv = c.n_kv_heads * c.head_dim, di = c.d_inner, B = c.batch;
+  const long long cache_ld = static_cast<long long>(cache_rows) * wkv;   // elements between sequences
+  uint8_t* kc = static_cast<uint8_t*>(kv_cache);
+  uint8_t* vc = kc + static_cast<size_t>(B) * cache_ld * es;
+  void* q = ws + D.q;
+  void* xs = ws + D.xs;
+  void* g = ws + D.g;
+  void* dt = ws + D.dt;
+  void* dtlow = ws + D.dtlow;
+  float* bc = reinterpret_cast<float*>(ws + D.bc);
+  void* z = ws + D.z;
+  // in_proj of the new rows; K, V go straight into the cache at row pos
+  GemmDesc gi;
+  gi.a = x_t;
+  gi.a_rows = B;
+  gi.K = c.d_model;
+  gi.w = w->w_in;
+  int col = 0;
+  gi.seg[gi.nseg++] = seg(col, col + wa, q, wa, 0, hy::SEG_STORE);
+  col += wa;
+  if (c.kv_mode != HYMBA_KV_CONSUME) {
+    gi.seg[gi.nseg++] = seg(col, col + wkv, kc + static_cast<size_t>(pos) * wkv * es, cache_ld, 0, hy::SEG_STORE);
+    col += wkv;
+    gi.seg[gi.nseg++] = seg(col, col + wkv, vc + static_cast<size_t>(pos) * wkv * es, cache_ld, 0, hy::SEG_STORE);
+    col += wkv;
+  }
+  gi.seg[gi.nseg++] = seg(col, col + di, xs, di, 0, hy::SEG_STORE);
+  col += di;
+  gi.seg[gi.nseg++] = seg(col, col + di, g, di, 0, hy::SEG_SILU);
+  col += di;
+  gi.N = col;
+  gi.status = status;
+  if (gemm(gi, c.dtype, st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  GemmDesc gx;
+  gx.a = xs;
+  gx.a_rows = B;
+  gx.K = di;
+  gx.w = w->w_x;
+  gx.N = c.dt_rank + 2 * c.d_state;
+  gx.seg[gx.nseg++] = seg(0, c.dt_rank, dtlow, c.dt_rank, 0, hy::SEG_STORE);
+  gx.seg[gx.nseg++] = seg(c.dt_rank, gx.N, bc, 2 * c.d_state, 1, hy::SEG_STORE);
+  gx.status = status;
+  if (gemm(gx, c.dtype, st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  GemmDesc gd;
+  gd.a = dtlow;
+  gd.a_rows = B;
+  gd.K = c.dt_rank;
+  gd.w = w->w_dt;
+  gd.N = di;
+  gd.seg[gd.nseg++] = seg(0, di, dt, di, 0, hy::SEG_SOFTPLUS_BIAS, w->b_dt);
+  gd.status = status;
+  if (gemm(gd, c.dtype, st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  // the token's query against the cached rows it sees
+  hy::DecodeAttnDesc ad;
+  ad.q = q;
+  ad.k = kc;
+  ad.v = vc;
+  ad.cap = cache_rows;
+  ad.kv_ld = wkv;
+  ad.out = z;
+  ad.out_ld = wa + di;
+  ad.part = reinterpret_cast<float*>(ws + D.part);
+  ad.max_splits = kMaxDecodeSplits;
+  ad.batch = B;
+  ad.n_q_heads = c.n_q_heads;
+  ad.n_kv_heads = c.n_kv_heads;
+  ad.head_dim = c.head_dim;
+  ad.pos = pos;
+  ad.n_meta = c.n_meta;
+  ad.window = c.window;
+  ad.bf16 = c.dtype == HYMBA_BF16;
+  if (hy::launch_attention_decode(ad, st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  // one step of every SSM channel from the carried state
+  hy::ScanStepDesc sd;
+  sd.x = xs;
+  sd.dt = dt;
+  sd.bc = bc;
+  sd.gate = g;
+  sd.a_log = w->a_log;
+  sd.a_per_state = c.a_per_state != 0;
+  sd.h = ssm_state;
+  sd.y = static_cast<uint8_t*>(z) + wa * es;
+  sd.y_ld = wa + di;
+  sd.batch = B;
+  sd.d_inner = di;
+  sd.d_state = c.d_state;
+  sd.bf16 = c.dtype == HYMBA_BF16;
+  if (hy::launch_scan_step(sd, st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  if (hy::launch_branch_norm(z, w->beta1, w->beta2, B, wa, di, c.rms_eps, c.dtype == HYMBA_BF16, st) != cudaSuccess)
+    return HYMBA_ERR_CUDA;
+  GemmDesc go;
+  go.a = z;
+  go.a_rows = B;
+  go.K = wa + di;
+  go.w = w->w_out;
+  go.N = c.d_model;
+  go.seg[go.nseg++] = seg(0, c.d_model, out_t, c.d_model, 0, hy::SEG_STORE);
+  go.status = status;
+  return gemm(go, c.dtype, st) == cudaSuccess ? HYMBA_OK : HYMBA_ERR_CUDA;
 }
 
 hymba_status_t hymba_workspace_status(void* workspace, void* stream) {

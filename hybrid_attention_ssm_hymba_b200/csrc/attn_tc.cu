@@ -620,11 +620,14 @@ EncodeTiledFn attn_encode_fn() {
 }
 
 // 3-D bf16 map over [batch][T][cols] with row stride ld elements; box = 64 cols x 128 rows x 1.
-bool map_rows(CUtensorMap* m, const void* base, long long cols, long long ld, int T, int batch) {
+// rows_per_seq: the buffer's rows per sequence (>= T; rows past T read as zeros).
+bool map_rows(CUtensorMap* m, const void* base, long long cols, long long ld, int T, int batch,
+              long long rows_per_seq = 0) {
   EncodeTiledFn fn = attn_encode_fn();
   if (!fn) return false;
+  if (rows_per_seq <= 0) rows_per_seq = T;
   cuuint64_t gd[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(batch)};
-  cuuint64_t gs[2] = {static_cast<cuuint64_t>(ld) * 2, static_cast<cuuint64_t>(ld) * 2 * T};
+  cuuint64_t gs[2] = {static_cast<cuuint64_t>(ld) * 2, static_cast<cuuint64_t>(ld) * 2 * rows_per_seq};
   cuuint32_t bx[3] = {64, 128, 1}, es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gd, gs, bx, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -638,19 +641,13 @@ cudaError_t launch_attention_f32(const AttnDesc& a, cudaStream_t st);
 cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st) {
   if (!a.bf16) return launch_attention_f32(a, st);
   if (a.batch <= 0 || a.T <= 0) return cudaSuccess;
-  static int attr_dev_mask = 0, attr2_mask = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 31 && !(attr_dev_mask & (1 << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_dev_mask |= 1 << dev;
-  }
+  static std::atomic<uint64_t> attr_done{0}, attr2_done{0};
+  if (cudaError_t e = smem_attr_once(attn_fwd_tc, SMEM_BYTES, attr_done)) return e;
   CUtensorMap tq, tk, tv;
   if (!map_rows(&tq, a.q, static_cast<long long>(a.n_q_heads) * DH, a.q_ld, a.T, a.batch)) return cudaErrorInvalidValue;
-  if (!map_rows(&tk, a.k, static_cast<long long>(a.n_kv_heads) * DH, a.kv_ld, a.T, a.batch))
+  if (!map_rows(&tk, a.k, static_cast<long long>(a.n_kv_heads) * DH, a.kv_ld, a.T, a.batch, a.kv_rows))
     return cudaErrorInvalidValue;
-  if (!map_rows(&tv, a.v, static_cast<long long>(a.n_kv_heads) * DH, a.kv_ld, a.T, a.batch))
+  if (!map_rows(&tv, a.v, static_cast<long long>(a.n_kv_heads) * DH, a.kv_ld, a.T, a.batch, a.kv_rows))
     return cudaErrorInvalidValue;
   AttnParams p{};
   p.T = a.T;
@@ -664,11 +661,7 @@ cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st) {
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(DH));
   p.status = a.status;
   if ((a.n_q_heads / a.n_kv_heads) % 2 == 0) {  // pairs of query heads share each K/V tile
-    if (dev < 31 && !(attr2_mask & (1 << dev))) {
-      cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
-      if (e != cudaSuccess) return e;
-      attr2_mask |= 1 << dev;
-    }
+    if (cudaError_t e = smem_attr_once(attn_fwd_tc2, SMEM2_BYTES, attr2_done)) return e;
     dim3 grid(p.q_tiles, a.n_q_heads / 2, a.batch);
     return launch(attn_fwd_tc2, grid, dim3(320), SMEM2_BYTES, st, tq, tk, tv, p);
   }

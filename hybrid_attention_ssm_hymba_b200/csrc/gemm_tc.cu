@@ -42,13 +42,15 @@ struct GemmParams {
   int batch, T, n_meta;
   int m_tiles;  // per sequence (meta mode) or in total (plain mode)
   int n_tiles, k_blocks, N;
+  int k_blocks1;            // > 0: concatenated K, blocks [k_blocks1, k_blocks) come from A2 / W2
   int epi;
   int nseg;
   Seg seg[kMaxSegs];
-  const __nv_bfloat16* resid;
+  const void* resid;
   long long resid_ld;
-  __nv_bfloat16* out;
+  void* out;
   long long out_ld;
+  int resid_f32, out_f32;   // residual / output element type of EPI_RESIDUAL and the dual epilogue
   int swiglu_F;
   int bias_len;             // > 0: the (single) bias segment's vector is staged in smem
   const float* bias_src;
@@ -116,6 +118,35 @@ __device__ __forceinline__ void store16(const GemmParams& p, long long row, int 
     for (int j = 0; j < 2; ++j)
       d[j] = make_uint4(pack_bf16(f[8 * j], f[8 * j + 1]), pack_bf16(f[8 * j + 2], f[8 * j + 3]),
                         pack_bf16(f[8 * j + 4], f[8 * j + 5]), pack_bf16(f[8 * j + 6], f[8 * j + 7]));
+  }
+}
+
+// Eight consecutive columns of a residual row (fp32 or bf16) added into f[0..8).
+__device__ __forceinline__ void add_resid8(const GemmParams& p, long long row, int col, float* f) {
+  if (p.resid_f32) {
+    const float4* rs = reinterpret_cast<const float4*>(static_cast<const float*>(p.resid) + row * p.resid_ld + col);
+    const float4 a = rs[0], b = rs[1];
+    f[0] += a.x; f[1] += a.y; f[2] += a.z; f[3] += a.w;
+    f[4] += b.x; f[5] += b.y; f[6] += b.z; f[7] += b.w;
+  } else {
+    const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.resid) + row * p.resid_ld + col);
+    const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] += bf16lo(qq[i]);
+      f[2 * i + 1] += bf16hi(qq[i]);
+    }
+  }
+}
+// Eight consecutive output columns (fp32 or bf16).
+__device__ __forceinline__ void store_out8(const GemmParams& p, long long row, int col, const float* f) {
+  if (p.out_f32) {
+    float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.out_ld + col);
+    d[0] = make_float4(f[0], f[1], f[2], f[3]);
+    d[1] = make_float4(f[4], f[5], f[6], f[7]);
+  } else {
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row * p.out_ld + col) =
+        make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
   }
 }
 
@@ -204,6 +235,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             } else {
               tma_load_3d(a_dst, &tmA, fb, kx, r0 - p.n_meta, tc.b);
             }
+          } else if (p.k_blocks1 > 0 && kb >= p.k_blocks1) {
+            // second K segment: A2 (map in the tmAx2 slot) and W2 (map in the tmM1 slot)
+            tma_load_2d(a_dst, &tmAx2, fb, (kb - p.k_blocks1) * BK, tc.m * BM);
           } else {
             tma_load_2d(a_dst, &tmA, fb, kx, tc.m * BM);
           }
@@ -211,6 +245,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (p.epi == EPI_SWIGLU) {
             tma_load_2d(b_dst, &tmB, fb, kx, tc.n * 128);
             tma_load_2d(b_dst + 128 * 128, &tmB, fb, kx, p.swiglu_F + tc.n * 128);
+          } else if (p.k_blocks1 > 0 && kb >= p.k_blocks1) {
+            tma_load_2d(b_dst, &tmM1, fb, (kb - p.k_blocks1) * BK, tc.n * BN);
           } else {
             tma_load_2d(b_dst, &tmB, fb, kx, tc.n * BN);
           }
@@ -315,27 +351,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           const int col = tc.n * BN + cc;
           if (valid && col < p.N) {
-            float f[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) f[e] = fmaf(sa, __uint_as_float(va[e]), ss * __uint_as_float(vs[e]));
-            if (p.epi == EPI_RESIDUAL) {
-              const uint4* rs = reinterpret_cast<const uint4*>(p.resid + grow * p.resid_ld + col);
+            for (int j = 0; j < 4; ++j) {
+              float f[8];
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint4 qv = rs[j];
-                const uint32_t qq[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  f[8 * j + 2 * i] += bf16lo(qq[i]);
-                  f[8 * j + 2 * i + 1] += bf16hi(qq[i]);
-                }
-              }
+              for (int e = 0; e < 8; ++e)
+                f[e] = fmaf(sa, __uint_as_float(va[8 * j + e]), ss * __uint_as_float(vs[8 * j + e]));
+              if (p.epi == EPI_RESIDUAL) add_resid8(p, grow, col + 8 * j, f);
+              store_out8(p, grow, col + 8 * j, f);
             }
-            uint4* d = reinterpret_cast<uint4*>(p.out + grow * p.out_ld + col);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              d[j] = make_uint4(pack_bf16(f[8 * j], f[8 * j + 1]), pack_bf16(f[8 * j + 2], f[8 * j + 3]),
-                                pack_bf16(f[8 * j + 4], f[8 * j + 5]), pack_bf16(f[8 * j + 6], f[8 * j + 7]));
           }
         }
         continue;
@@ -366,7 +390,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_before();
         mbar_arrive(&tempty[buf]);
         if (valid) {
-          uint4* d = reinterpret_cast<uint4*>(p.out + grow * p.out_ld + tc.n * 128 + c * 32);
+          uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + grow * p.out_ld + tc.n * 128 + c * 32);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             float f[8];
@@ -388,18 +412,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int q = 0; q < CPT; ++q) {
           const int col = tc.n * BN + (grp + q * EPI_GROUPS) * 32;
           if (valid && col < p.N) {
-            const uint4* rs = reinterpret_cast<const uint4*>(p.resid + grow * p.resid_ld + col);
-            uint4* d = reinterpret_cast<uint4*>(p.out + grow * p.out_ld + col);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const uint4 qv = rs[j];
-              const uint32_t qq[4] = {qv.x, qv.y, qv.z, qv.w};
-              uint32_t o[4];
+              float f[8];
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                o[i] = pack_bf16(bf16lo(qq[i]) + __uint_as_float(v[q][8 * j + 2 * i]),
-                                 bf16hi(qq[i]) + __uint_as_float(v[q][8 * j + 2 * i + 1]));
-              d[j] = make_uint4(o[0], o[1], o[2], o[3]);
+              for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[q][8 * j + e]);
+              add_resid8(p, grow, col + 8 * j, f);
+              store_out8(p, grow, col + 8 * j, f);
             }
           }
         }
@@ -455,15 +474,8 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
 template <int BN>
 cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
   using C = Cfg<BN>;
-  static int attr_mask = 0;  // the attribute is per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 31 && !(attr_mask & (1 << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM + kMaxBiasSmem * 4);
-    if (e != cudaSuccess) return e;
-    attr_mask |= 1 << dev;
-  }
+  static std::atomic<uint64_t> attr_done{0};  // the attribute is per device
+  if (cudaError_t e = smem_attr_once(gemm_bf16_tc<BN>, C::SMEM + kMaxBiasSmem * 4, attr_done)) return e;
   CUtensorMap tmA, tmAx2, tmM1, tmM2, tmB;
   const uint64_t K = static_cast<uint64_t>(g.K);
   GemmParams p{};
@@ -504,6 +516,15 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
     tmAx2 = tmA;
     tmM1 = tmA;
     tmM2 = tmA;
+    if (g.K2 > 0) {  // second K segment: A2 in the tmAx2 slot, W2 in the tmM1 slot
+      const uint64_t K2 = static_cast<uint64_t>(g.K2);
+      uint64_t da2[2] = {K2, static_cast<uint64_t>(g.a_rows)};
+      uint64_t sa2[1] = {K2 * 2};
+      if (!make_map(&tmAx2, g.a2, 2, da2, sa2, ba)) return cudaErrorInvalidValue;
+      uint64_t dw2[2] = {K2, static_cast<uint64_t>(g.N)};
+      uint32_t bw2[2] = {BK, static_cast<uint32_t>(BN)};
+      if (!make_map(&tmM1, g.w2, 2, dw2, sa2, bw2)) return cudaErrorInvalidValue;
+    }
     p.meta_mode = 0;
     p.batch = 1;
     p.a_rows = g.a_rows;
@@ -518,6 +539,11 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
   p.N = g.N;
   p.n_tiles = (g.epi == EPI_SWIGLU) ? g.swiglu_F / 128 : (g.N + BN - 1) / BN;
   p.k_blocks = (g.K + BK - 1) / BK;
+  p.k_blocks1 = 0;
+  if (g.K2 > 0 && !g.meta_mode && g.epi != EPI_SWIGLU && g.dual_k_blocks == 0) {
+    p.k_blocks1 = p.k_blocks;
+    p.k_blocks += (g.K2 + BK - 1) / BK;
+  }
   p.epi = g.epi;
   p.nseg = g.nseg;
   p.bias_len = 0;
@@ -537,10 +563,12 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
   p.inv_wa = g.inv_wa;
   p.inv_ws = g.inv_ws;
   p.eps = g.eps;
-  p.resid = static_cast<const __nv_bfloat16*>(g.resid);
+  p.resid = g.resid;
   p.resid_ld = g.resid_ld;
-  p.out = static_cast<__nv_bfloat16*>(g.out);
+  p.out = g.out;
   p.out_ld = g.out_ld;
+  p.resid_f32 = g.resid_f32 ? 1 : 0;
+  p.out_f32 = g.out_f32 ? 1 : 0;
   p.swiglu_F = g.swiglu_F;
   p.status = g.status;
   const long long total = static_cast<long long>(p.meta_mode ? p.batch : 1) * p.m_tiles * p.n_tiles;
@@ -553,6 +581,8 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_gemm_bf16(const GemmDesc& g, cudaStream_t st) {
+  if (g.K2 > 0 && (g.meta_mode || g.epi == EPI_SWIGLU || g.dual_k_blocks > 0 || !g.a2 || !g.w2))
+    return cudaErrorInvalidValue;  // the second K segment is a plain-mode option
   if (g.epi == EPI_SWIGLU || g.N > 128 || g.dual_k_blocks > 0) return launch_bn<256>(g, st);
   return launch_bn<128>(g, st);
 }

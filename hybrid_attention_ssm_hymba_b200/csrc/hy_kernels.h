@@ -6,7 +6,25 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace hy {
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` once per device (devices 0..63);
+// `done` is the kernel's own mask of devices already set.  Safe from several host threads
+// (a repeated cudaFuncSetAttribute is harmless).
+template <typename K>
+cudaError_t smem_attr_once(K* kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Launch with programmatic stream serialization (see pdl_wait in hy_common.cuh).
 template <typename... KArgs, typename... Args>
@@ -57,6 +75,12 @@ struct GemmDesc {
   // B operand W [N, K] row-major
   const void* w = nullptr;
   int N = 0;
+  // Concatenated K (plain mode, bf16 only): C = [A | A2] [W | W2]^T, i.e. the product over
+  // K columns of A and W followed by K2 columns of a2 [a_rows, K2] and w2 [N, K2] into the
+  // same accumulator.  K2 = 0: off.
+  const void* a2 = nullptr;
+  const void* w2 = nullptr;
+  int K2 = 0;
   // epilogue
   int epi = EPI_SEGMENTS;
   int nseg = 0;
@@ -65,6 +89,9 @@ struct GemmDesc {
   long long resid_ld = 0;
   void* out = nullptr;
   long long out_ld = 0;
+  // EPI_RESIDUAL and the fused branch-norm epilogue: resid and/or out in fp32 instead of
+  // the GEMM's dtype (a residual stream carried in fp32)
+  bool resid_f32 = false, out_f32 = false;
   int swiglu_F = 0;
   // Fused branch norm (bf16 out_proj): the first dual_k_blocks 64-wide K blocks (the
   // attention columns of Z) accumulate apart from the rest (the SSM columns), and the
@@ -90,6 +117,9 @@ struct ScanDesc {
   // stride dt_rank), w_dt [d_inner, dt_rank] bf16, b_dt [d_inner] fp32.
   const void* dt_low = nullptr; const void* w_dt = nullptr; const float* b_dt = nullptr;
   int dt_rank = 0;
+  // Final state: when set, h_out [batch, d_inner, d_state] fp32 receives each sequence's
+  // state after its last row (what the next row of a generation step starts from).
+  float* h_out = nullptr;
 };
 cudaError_t launch_scan(const ScanDesc& s, cudaStream_t st);
 // The tensor-core form of the scan (bf16, d_state = 16, 16-byte aligned operands);
@@ -106,13 +136,53 @@ struct AttnDesc {
   int batch, T, n_q_heads, n_kv_heads, head_dim, n_meta, window;
   bool bf16;
   unsigned* status;
+  long long kv_rows = 0;  // rows per sequence in the K/V buffers (0: T; a cache may hold more)
 };
 cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st);
+
+// Generation step (decode.cu).  One query row per sequence at row `pos`; K/V cache
+// rows of sequence b at (b * cap + row) * kv_ld; part: [batch, Hq, max_splits, dh + 2]
+// fp32 partials; out at out + b * out_ld + h * dh.
+struct DecodeAttnDesc {
+  const void* q; const void* k; const void* v;
+  long long cap, kv_ld;
+  void* out; long long out_ld;
+  float* part; int max_splits;
+  int batch, n_q_heads, n_kv_heads, head_dim, pos, n_meta, window;
+  bool bf16;
+};
+cudaError_t launch_attention_decode(const DecodeAttnDesc& a, cudaStream_t st);
+// Number of key splits (and keys per split) the decode attention uses.
+int decode_attn_splits(int batch, int n_kv_heads, int n_visible, int max_splits, int* keys_per_split);
+// One scan step: h [batch, Di, N] fp32 updated in place; x, dt, gate [batch, Di];
+// bc [batch, 2N] fp32; y at y + b * y_ld + c.
+struct ScanStepDesc {
+  const void* x; const void* dt; const float* bc; const void* gate; const float* a_log;
+  bool a_per_state;
+  float* h;
+  void* y; long long y_ld;
+  int batch, d_inner, d_state;
+  bool bf16;
+};
+cudaError_t launch_scan_step(const ScanStepDesc& s, cudaStream_t st);
 
 cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, long long rows, int w_attn,
                                int w_ssm, float eps, bool bf16, cudaStream_t st);
 cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float eps, bool bf16,
                            cudaStream_t st);
+// Pre-norm of a residual stream kept in fp32: y = bf16(gain * x / sqrt(mean(x^2) + eps)) per
+// row of x [rows, d] fp32 (gain [d] fp32, or NULL for unit gain); when y_lo is given it also
+// receives the part of the fp32 result that the bf16 rounding dropped, bf16(v - float(y)).
+cudaError_t launch_prenorm_f32(const float* x, const float* gain, void* y, void* y_lo, long long rows, int d,
+                               float eps, cudaStream_t st);
+cudaError_t launch_prenorm_f32_out_f32(const float* x, const float* gain, float* y, long long rows, int d, float eps,
+                                       cudaStream_t st);
+// h[b, t, :] = float([meta; x_b][t, :]) for a bf16 stack input (h fp32 [batch, L + M, d]).
+cudaError_t launch_prepend_f32(const void* x, const void* meta, float* h, int batch, int L, int M, int d,
+                               cudaStream_t st);
+// dst[c, r] = src[r, c] for a bf16 matrix src [rows, cols] with row stride src_ld.
+cudaError_t launch_transpose_bf16(const void* src, long long src_ld, void* dst, int rows, int cols,
+                                  cudaStream_t st);
 // Fused branch norm (bf16).  row_ssq: ssq[row] = (sum of z[row, :w_attn]^2, sum of
 // z[row, w_attn:]^2).  scale_cols: w_out[n, k] = w[n, k] * (k < w_attn ? beta1[k] :
 // beta2[k - w_attn]) for a [N, w_attn + w_ssm] weight.

@@ -313,3 +313,133 @@ cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float 
 }
 
 }  // namespace hy
+
+// ---------------------------------------------------------------------------------
+// Residual stream in fp32 (stacked blocks).
+
+namespace hy {
+namespace {
+
+// One warp per row of x [rows, d] fp32: y = gain * x / sqrt(mean(x^2) + eps) in TO (bf16 or
+// fp32); with y_lo, also the bf16 rounding remainder v - float(bf16(v)) (bf16 output only).
+// Two passes over the row: the second re-reads it from L1/L2.
+template <typename TO>
+__global__ void __launch_bounds__(256) prenorm_f32_kernel(const float* __restrict__ x, const float* __restrict__ gain,
+                                                          TO* __restrict__ y, __nv_bfloat16* __restrict__ y_lo,
+                                                          long long rows, int d, float eps) {
+  pdl_trigger();
+  pdl_wait();
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float* xr = x + row * d;
+  float s = 0.f;
+  for (int i = lane * 8; i < d; i += 256) {
+    float f[8];
+    Vec8<float>::load(xr + i, f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s = fmaf(f[j], f[j], s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float r = rsqrtf(s / d + eps);
+  for (int i = lane * 8; i < d; i += 256) {
+    float f[8];
+    Vec8<float>::load(xr + i, f);
+    if (gain) {
+      float g[8];
+      Vec8<float>::load(gain + i, g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] = f[j] * r * g[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] *= r;
+    }
+    Vec8<TO>::store(y + row * d + i, f);
+    if (y_lo) {
+      float lo[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) lo[j] = f[j] - __bfloat162float(__float2bfloat16_rn(f[j]));
+      Vec8<__nv_bfloat16>::store(y_lo + row * d + i, lo);
+    }
+  }
+}
+
+// h[b, t, :] = float(t < M ? meta[t, :] : x[b, t - M, :]), 8 elements per thread.
+__global__ void __launch_bounds__(256) prepend_f32_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const __nv_bfloat16* __restrict__ meta,
+                                                          float* __restrict__ h, int L, int M, int d,
+                                                          long long total_vec) {
+  pdl_trigger();
+  pdl_wait();
+  const int rv = d / 8;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total_vec;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = i / rv;
+    const int e = static_cast<int>(i - row * rv) * 8;
+    const long long T = L + M, b = row / T, t = row - b * T;
+    const __nv_bfloat16* src = t < M ? meta + t * d + e : x + (b * L + (t - M)) * d + e;
+    float f[8];
+    Vec8<__nv_bfloat16>::load(src, f);
+    Vec8<float>::store(h + row * d + e, f);
+  }
+}
+
+// dst [cols, rows] = src [rows, cols]^T through a 32 x 32 shared tile (bf16).
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src, long long src_ld,
+                                                             __nv_bfloat16* __restrict__ dst, int rows, int cols) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of 32 threads
+  for (int k = ty; k < 32; k += 8) {
+    const int r = r0 + k, c = c0 + tx;
+    if (r < rows && c < cols) tile[k][tx] = src[static_cast<long long>(r) * src_ld + c];
+  }
+  __syncthreads();
+  for (int k = ty; k < 32; k += 8) {
+    const int c = c0 + k, r = r0 + tx;
+    if (r < rows && c < cols) dst[static_cast<long long>(c) * rows + r] = tile[tx][k];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prenorm_f32(const float* x, const float* gain, void* y, void* y_lo, long long rows, int d,
+                               float eps, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (d % 8) return cudaErrorInvalidValue;
+  const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+  return launch(prenorm_f32_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, x, gain,
+                static_cast<__nv_bfloat16*>(y), static_cast<__nv_bfloat16*>(y_lo), rows, d, eps);
+}
+
+cudaError_t launch_prenorm_f32_out_f32(const float* x, const float* gain, float* y, long long rows, int d, float eps,
+                                       cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (d % 8) return cudaErrorInvalidValue;
+  const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+  return launch(prenorm_f32_kernel<float>, dim3(grid), dim3(256), 0, st, x, gain, y,
+                static_cast<__nv_bfloat16*>(nullptr), rows, d, eps);
+}
+
+cudaError_t launch_prepend_f32(const void* x, const void* meta, float* h, int batch, int L, int M, int d,
+                               cudaStream_t st) {
+  const long long total = static_cast<long long>(batch) * (L + M) * (d / 8);
+  if (total <= 0) return cudaSuccess;
+  if (d % 8) return cudaErrorInvalidValue;
+  const long long blocks = (total + 255) / 256;
+  return launch(prepend_f32_kernel, dim3(static_cast<unsigned>(blocks < 8 * num_sms() ? blocks : 8 * num_sms())),
+                dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(meta), h, L,
+                M, d, total);
+}
+
+cudaError_t launch_transpose_bf16(const void* src, long long src_ld, void* dst, int rows, int cols, cudaStream_t st) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32);
+  return launch(transpose_bf16_kernel, grid, dim3(256), 0, st, static_cast<const __nv_bfloat16*>(src), src_ld,
+                static_cast<__nv_bfloat16*>(dst), rows, cols);
+}
+
+}  // namespace hy

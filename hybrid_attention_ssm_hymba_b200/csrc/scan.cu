@@ -47,6 +47,7 @@ struct ScanParams {
   void* y;
   long long y_ld;
   int T, Di, N;
+  float* h_out;  // [batch, Di, N] state after the last row, or nullptr
 };
 
 template <typename TI, int NS, int TPC, int NWT>
@@ -201,6 +202,15 @@ __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
       gp += p.Di;
       bp += 2 * N;
       yp += p.y_ld;
+    }
+  }
+  // the last chunk's warp ends at row T - 1 (an empty chunk keeps its entry state)
+  if (p.h_out && valid && warp == NWT - 1) {
+    float* ho = p.h_out + (static_cast<long long>(b) * p.Di + c) * N + n0;
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      ho[2 * i] = h[i].x;
+      ho[2 * i + 1] = h[i].y;
     }
   }
 }
@@ -687,6 +697,22 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
       }
     }
   }
+  // state after the last row: the last chunk's warp, h = P g with -log2 P = ncl (rows past
+  // T loaded as zeros leave it unchanged)
+  if (p.h_out && active && ok && chunk == sp.S - 1) {
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) {
+      if (c0 + q < p.Di) {
+        const float P = ex2_approx(-ncl[q]);
+        float* ho = p.h_out + (static_cast<long long>(b) * p.Di + c0 + q) * N + n0;
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+          ho[2 * i] = g[q][i].x * P;
+          ho[2 * i + 1] = g[q][i].y * P;
+        }
+      }
+    }
+  }
   if (lane == 0) {
     bulk_wait_all();
     if (!ok) {  // let the copies this warp issued but did not consume land before it exits
@@ -749,13 +775,18 @@ __global__ void __launch_bounds__(128) scan_ps_kernel(const ScanParams p) {
     if (valid && slice == 0)
       yp[static_cast<long long>(t) * p.y_ld] = from_f<TI>(to_f<TI>(gp[static_cast<long long>(t) * p.Di]) * y);
   }
+  if (p.h_out && valid) {
+    float* ho = p.h_out + (static_cast<long long>(b) * p.Di + c) * N + n0;
+#pragma unroll
+    for (int n = 0; n < NS; ++n) ho[n] = h[n];
+  }
 }
 
 template <typename TI, int N>
 cudaError_t launch_ps(const ScanDesc& s, cudaStream_t st) {
   constexpr int NS = N < 8 ? N : 8;
   constexpr int CPB = 4 * (32 / (N / NS));  // channels per block
-  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
+  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state, s.h_out};
   dim3 grid((s.d_inner + CPB - 1) / CPB, s.batch);
   return launch(scan_ps_kernel<TI, N>, grid, dim3(128), 0, st, p);
 }
@@ -818,15 +849,9 @@ cudaError_t launch_w(const ScanDesc& s, cudaStream_t st) {
   const int groups = (s.d_inner + C::CPW - 1) / C::CPW;
   const int n_tiles = (s.T + C::ROWS - 1) / C::ROWS;
   const int max_warps = (227 * 1024 - 128) / C::WARP_B < C::MAX_WARPS ? (227 * 1024 - 128) / C::WARP_B : C::MAX_WARPS;
-  static int attr_mask = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 31 && !(attr_mask & (1 << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(scan_w_kernel<TI, N, TPC, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         max_warps * C::WARP_B + 128);
-    if (e != cudaSuccess) return e;
-    attr_mask |= 1 << dev;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (cudaError_t e = smem_attr_once(scan_w_kernel<TI, N, TPC, CPL>, max_warps * C::WARP_B + 128, attr_done))
+    return e;
   // Time chunks S: the smallest split that gives about two warps per SM sub-partition,
   // else the largest whose grid still fits in one wave; chunks of at least 8 tiles.
   SplitParams sp{1, 4, n_tiles};
@@ -844,7 +869,7 @@ cudaError_t launch_w(const ScanDesc& s, cudaStream_t st) {
   }
   const int warps = sp.G * sp.S;
   const int smem = warps * C::WARP_B + 128;
-  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
+  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state, s.h_out};
   dim3 grid((groups + sp.G - 1) / sp.G, s.batch);
   return launch(scan_w_kernel<TI, N, TPC, CPL>, grid, dim3(32 * warps), smem, st, tx, td, tg, tb, ty, p, sp, s.status);
 }
@@ -852,7 +877,7 @@ cudaError_t launch_w(const ScanDesc& s, cudaStream_t st) {
 template <typename TI, int NS, int TPC, int NWT>
 cudaError_t launch_one(const ScanDesc& s, cudaStream_t st) {
   constexpr int CPW = 32 / TPC;
-  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state};
+  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state, s.h_out};
   dim3 grid((s.d_inner + CPW - 1) / CPW, s.batch);
   return launch(scan_kernel<TI, NS, TPC, NWT>, grid, dim3(32 * NWT), 0, st, p);
 }

@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                    const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmBC,
                    const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmWD,
                    const float* __restrict__ a_log, const float* __restrict__ b_dt, int T, int Di,
-                   unsigned* status) {
+                   float* __restrict__ h_out, unsigned* status) {
   using L = Lay<FUSED>;
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
@@ -342,9 +342,13 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) z[j] = 0u;
           }
+          // steps past T (zero-filled dt_low) get dt = 0, so they leave the state alone
+          const int t_end = T - (k * Q + 32 * half);
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const float2 d = softplus2(make_float2(__uint_as_float(z[j]) + bdt, __uint_as_float(z[j + 1]) + bdt));
+            float2 d = softplus2(make_float2(__uint_as_float(z[j]) + bdt, __uint_as_float(z[j + 1]) + bdt));
+            if (j >= t_end) d.x = 0.f;
+            if (j + 1 >= t_end) d.y = 0.f;
             dtv[j] = d.x;
             dtv[j + 1] = d.y;
             S2 = __ffma2_rn(make_float2(A2, A2), d, S2);
@@ -502,6 +506,25 @@ __global__ void __launch_bounds__(NTHR, 1)
         if (bar_red_or(1, NCHT, *abort_flag != 0)) break;
       }
       if (k < nblk) prev_any = any;
+      if (k == nblk && h_out && half == 1) {  // warp-uniform (tcgen05.ld below is warp-collective)
+        // state after the last row: h entering the last block advanced by that block's dG
+        // (complete: its yready, waited above, was committed after it), unless the block
+        // ran the plain recurrence, which left h there already
+        if (!prev_any) {
+          tc_fence_after();
+          uint32_t d[16];
+          tmem_ld16(tl + COL_DG + 16 * ((nblk - 1) & 1), d);
+          tmem_wait_ld();
+          const float a = ex2_approx(-(pS0 + pS1)), bs = ex2_approx(-pS1);
+#pragma unroll
+          for (int n = 0; n < NST; ++n) h[n] = fmaf(a, h[n], bs * __uint_as_float(d[n]));
+        }
+        if (c < Di) {
+          float4* ho = reinterpret_cast<float4*>(h_out + (static_cast<long long>(b) * Di + c) * NST);
+#pragma unroll
+          for (int j = 0; j < NST / 4; ++j) ho[j] = make_float4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+        }
+      }
     }
     if (threadIdx.x == 0) bulk_wait_all();
   }
@@ -574,18 +597,11 @@ cudaError_t launch_tc(const ScanDesc& s, cudaStream_t st) {
     tw = tx;  // unused
   }
   if (!ok) return cudaErrorNotSupported;
-  static int attr_mask = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 31 && !(attr_mask & (1 << dev))) {
-    cudaError_t e =
-        cudaFuncSetAttribute(scan_tc_kernel<FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_TOTAL);
-    if (e != cudaSuccess) return e;
-    attr_mask |= 1 << dev;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (cudaError_t e = smem_attr_once(scan_tc_kernel<FUSED>, L::SMEM_TOTAL, attr_done)) return e;
   dim3 grid((s.d_inner + CH - 1) / CH, s.batch);
   return launch(scan_tc_kernel<FUSED>, grid, dim3(NTHR), L::SMEM_TOTAL, st, tx, td, tg, tb, ty, tw, s.a_log, s.b_dt,
-                s.T, s.d_inner, s.status);
+                s.T, s.d_inner, s.h_out, s.status);
 }
 
 }  // namespace

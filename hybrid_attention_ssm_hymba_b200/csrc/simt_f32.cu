@@ -122,7 +122,8 @@ __global__ void __launch_bounds__(128) attention_f32_kernel(const float* __restr
                                                             const float* __restrict__ k,
                                                             const float* __restrict__ v, long long kv_ld,
                                                             float* __restrict__ out, long long out_ld, int T, int Hq,
-                                                            int Hkv, int dh, int n_meta, int window, int batch) {
+                                                            int Hkv, int dh, int n_meta, int window, int batch,
+                                                            long long kv_rows) {
   pdl_trigger();
   pdl_wait();
   const long long wid = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(128) attention_f32_kernel(const float* __restr
   float m = -INFINITY, l = 0.f;
   for (int j = 0; j <= i; ++j) {
     if (!(window < 0 || i - j <= window || j < n_meta)) continue;
-    const long long krow = static_cast<long long>(b) * T + j;
+    const long long krow = static_cast<long long>(b) * kv_rows + j;
     float s = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -208,7 +209,7 @@ cudaError_t launch_attention_f32(const AttnDesc& a, cudaStream_t st) {
   return launch(attention_f32_kernel, dim3(static_cast<unsigned>((total + 3) / 4)), dim3(128), 0, st,
                 static_cast<const float*>(a.q), a.q_ld, static_cast<const float*>(a.k),
                 static_cast<const float*>(a.v), a.kv_ld, static_cast<float*>(a.out), a.out_ld, a.T, a.n_q_heads,
-                a.n_kv_heads, a.head_dim, a.n_meta, a.window, a.batch);
+                a.n_kv_heads, a.head_dim, a.n_meta, a.window, a.batch, a.kv_rows > 0 ? a.kv_rows : a.T);
 }
 
 }  // namespace hy

@@ -10,7 +10,7 @@ import torch
 
 from . import _abi
 
-FP32_KEYS = ("a_log", "b_dt", "beta1", "beta2")
+FP32_KEYS = ("a_log", "b_dt", "beta1", "beta2", "norm1", "norm2")
 
 
 def torch_dtype(dtype: str) -> torch.dtype:
@@ -25,7 +25,8 @@ def to_device(a: np.ndarray, dtype: str, device="cuda", pin: bool = False) -> to
 
 
 def params_to_device(p: Dict[str, np.ndarray], dtype: str, device="cuda") -> Dict[str, torch.Tensor]:
-    """Projection weights in the layer's dtype; a_log, b_dt, beta1, beta2 in fp32."""
+    """Projection weights in the layer's dtype; a_log, b_dt, beta1, beta2 (and the pre-norm
+    gains norm1, norm2) in fp32."""
     return {k: to_device(v, "f32" if k in FP32_KEYS else dtype, device) for k, v in p.items()}
 
 

@@ -100,6 +100,9 @@ typedef struct {
   const float* beta2;     /* [Di] */
   const void* w_gate_up;  /* [2F, d] gate rows then up rows (stack with ffn_dim > 0), else NULL */
   const void* w_down;     /* [d, F] (stack with ffn_dim > 0), else NULL */
+  const float* norm1;     /* [d] fp32 gain of the block's pre-norm before the mixer (stack only);
+                             NULL = unit gain; ignored by the single-layer entry points */
+  const float* norm2;     /* [d] fp32 gain of the pre-norm before the FFN (stack only); NULL = unit gain */
 } hymba_weights_t;
 
 /* Human-readable name of a status code (static string). */
@@ -134,12 +137,18 @@ HYMBA_API hymba_status_t hymba_layer_fwd(const void* x, const void* meta, const 
 
 /*
  * A stack of hybrid-head blocks ("Key Components of Hymba", networkstorageforum:
- * blocks stacked with SWA and cross-layer KV sharing).  For each block i:
- *   h += layer_i(RMSNorm(h));  if cfgs[i].ffn_dim: h += W_down(SiLU(W_gate u) * W_up u), u = RMSNorm(h)
- * with unit RMSNorm gains; h starts as [meta; x].  K/V flow from a
- * HYMBA_KV_PRODUCE block to the HYMBA_KV_CONSUME block after it through the
- * workspace.  x, meta as in hymba_layer_fwd; out [B, T, d] = final h.
- * All cfgs must share batch, seq_len, n_meta, d_model, dtype.
+ * blocks stacked with SWA and cross-layer KV sharing; the blog.outta.ai review,
+ * "Cross-layer KV sharing": two consecutive layers share one KV cache).  For each block i:
+ *   h += layer_i(RMSNorm_1(h));  if cfgs[i].ffn_dim: h += W_down(SiLU(W_gate u) * W_up u), u = RMSNorm_2(h)
+ * with RMSNorm_k(v) = norm_k * v / sqrt(mean(v^2) + eps) (w[i].norm1 / norm2; NULL = unit
+ * gain); h starts as [meta; x].  K/V flow from a HYMBA_KV_PRODUCE block to the
+ * HYMBA_KV_CONSUME block after it through the workspace.  x, meta as in hymba_layer_fwd;
+ * out [B, T, d] dtype = final h.  All cfgs must share batch, seq_len, n_meta, d_model, dtype.
+ * Precision (bf16): the residual stream h is carried in fp32 in the workspace and rounded
+ * to bf16 once, into `out`; each pre-norm's output is the bf16 operand of the next GEMM,
+ * and the part of it that the bf16 rounding drops is carried into the SSM heads' B and C
+ * (x_proj adds it through W_x W_SSM, formed per call in the workspace), because a block's
+ * output at early positions depends on those two projections with a large condition number.
  */
 HYMBA_API hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weights_t* w,
                                const hymba_cfg_t* cfgs, int n_layers, void* out,
@@ -203,6 +212,57 @@ HYMBA_API hymba_status_t hymba_layer_fwd_noalloc(const void* x, const void* meta
 /* Synchronises `stream`, reads and clears the status word at the start of
  * `workspace`: HYMBA_OK, or HYMBA_ERR_TIMEOUT if a kernel's bounded wait ran out. */
 HYMBA_API hymba_status_t hymba_workspace_status(void* workspace, void* stream);
+
+/* ---------------- generation: prefill with state, then one token per step ----------------
+ * The attention heads keep a K/V cache that grows with the sequence; the SSM heads keep a
+ * fixed-size state (the blog.outta.ai review, "Efficiency and KV cache optimization").
+ * A KV-sharing pair keeps one cache (the review, "Cross-layer KV sharing"): the producer's.
+ *
+ * Layouts (dtype unless noted):
+ *   kv_cache   [2, B, cache_rows, Hkv*dh]: K then V; sequence b's row t at (b*cache_rows + t)
+ *   ssm_state  [B, Di, N] fp32: the state after the last row processed
+ * Workspace for both calls: hymba_decode_workspace_size(cfg) bytes, 256-byte aligned, its
+ * first 256 bytes the status word.  Both calls are asynchronous on `stream`; the head_dim
+ * must be a multiple of 32, at most 8 query heads per KV head, d_state a multiple of 8.
+ */
+HYMBA_API size_t hymba_decode_workspace_size(const hymba_cfg_t* cfg);
+
+/*
+ * hymba_layer_fwd over the T = L + M prompt rows (cfg.seq_len = L) that also leaves what
+ * the next token needs: rows [0, T) of each sequence's K/V in kv_cache (cache_rows >= T;
+ * for a HYMBA_KV_CONSUME layer kv_cache is the producer's cache, read only) and the SSM
+ * state after row T - 1 in ssm_state.  x, meta, out as in hymba_layer_fwd.
+ */
+HYMBA_API hymba_status_t hymba_layer_prefill(const void* x, const void* meta, const hymba_weights_t* w,
+                                   const hymba_cfg_t* cfg, void* kv_cache, int cache_rows,
+                                   float* ssm_state, void* out, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/*
+ * One new token per sequence at row `pos` (rows [0, pos) are in the cache, meta rows
+ * included; 0 <= pos < cache_rows): x_t [B, d] -> out_t [B, d].  The same definitions as
+ * hymba_layer_fwd applied to row pos: its query attends over the cached rows it sees
+ * (causal, window W, meta rows always visible) and its own; the SSM heads advance one
+ * step, h <- exp(A dt) h + dt x B, y = C . h (the review, "Design formulation").  A layer
+ * with its own K/V (HYMBA_KV_OWN / HYMBA_KV_PRODUCE) writes the token's K, V into row pos
+ * of kv_cache first; a HYMBA_KV_CONSUME layer reads the producer's cache, which must
+ * already hold row pos.  ssm_state is read and updated in place.  cfg.seq_len is not used.
+ */
+HYMBA_API hymba_status_t hymba_layer_decode(const void* x_t, const hymba_weights_t* w, const hymba_cfg_t* cfg,
+                                  void* kv_cache, int cache_rows, int pos, float* ssm_state,
+                                  void* out_t, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Check of the failure-detection path (no counterpart in the pages).  Every kernel of this
+ * library bounds its waits on mbarriers; a wait that runs out records HYMBA_ERR_TIMEOUT
+ * in the status word and the kernel returns instead of hanging.  This call runs one
+ * kernel whose single waiting thread waits on an mbarrier that nothing arrives on, with
+ * a limit of limit_us microseconds (1 .. 1000000): the wait runs out, the status word at
+ * the start of `workspace` (>= 256 bytes; cleared first) becomes HYMBA_ERR_TIMEOUT, and
+ * the kernel returns.  Read it with hymba_workspace_status().
+ */
+HYMBA_API hymba_status_t hymba_check_wait_timeout(void* workspace, size_t ws_bytes, unsigned limit_us,
+                                                  void* stream);
 
 /* ---------------- stage entry points (each one kernel family) ---------------- */
 
