@@ -10,7 +10,7 @@ import torch
 
 from . import _abi
 
-FP32_KEYS = ("a_log", "b_dt", "beta1", "beta2", "norm1", "norm2")
+FP32_KEYS = ("a_log", "b_dt", "beta1", "beta2", "norm1", "norm2", "b_conv", "d_skip")
 
 
 def torch_dtype(dtype: str) -> torch.dtype:

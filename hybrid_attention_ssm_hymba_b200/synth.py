@@ -39,6 +39,7 @@ _STREAM = {
     "x": 1, "meta": 2,
     "w_in": 10, "w_x": 11, "w_dt": 12, "w_out": 13, "a_log": 14, "dt0": 15,
     "beta1": 16, "beta2": 17, "w_gate_up": 18, "w_down": 19, "norm1": 20, "norm2": 21,
+    "w_conv": 22, "b_conv": 23, "d_skip": 24,
     # free-standing stage inputs used by the per-kernel tests
     "s_x": 40, "s_dt": 41, "s_bc": 42, "s_g": 43, "s_q": 44, "s_kv": 45,
     "s_z": 46, "s_a": 47, "s_w": 48,
@@ -68,6 +69,10 @@ class LayerShape:
     a_per_state: int = 0
     rms_eps: float = 1e-6
     dtype: str = "bf16"   # "bf16" or "f32"
+    conv_width: int = 0   # Mamba option: causal depthwise conv of this width + SiLU on X_ssm
+    d_skip: int = 0       # Mamba option: 1 = the SSM output gets D * x before the gate
+    norm_group: int = 0   # branch norm per group of this many features (0: whole branch)
+    fusion: int = 0       # 0: sum of the branches; 1: difference (SSM branch subtracted)
 
     @property
     def T(self) -> int:
@@ -243,6 +248,8 @@ def layer_params(wl: Workload, layer: int, norm_gains: bool = False) -> Dict[str
       w_out [d, Hq*dh + Di]
       a_log [Di] (or [Di, N] when a_per_state), b_dt [Di], beta1 [Hq*dh], beta2 [Di]: fp32
       w_gate_up [2F, d] (gate rows then up rows), w_down [d, F]   (ffn_dim > 0)
+      w_conv [Di, K] (dtype), b_conv [Di] fp32 ~ U(+-1/sqrt(K)): with conv_width = K
+      d_skip [Di] fp32 ~ U(0.5, 1.5): with d_skip
       norm1, norm2 [d] fp32 ~ U(0.5, 1.5): the stacked block's pre-norm gains, only with
                         norm_gains (the workloads use unit gains, their initial value)
     """
@@ -267,6 +274,12 @@ def layer_params(wl: Workload, layer: int, norm_gains: bool = False) -> Dict[str
     if s.ffn_dim:
         p["w_gate_up"] = normal(sd, layer, "w_gate_up", (2 * s.ffn_dim, s.d_model), 0.02, dt)
         p["w_down"] = normal(sd, layer, "w_down", (s.d_model, s.ffn_dim), 0.02, dt)
+    if s.conv_width:   # the default init of a depthwise Conv1d: U(-1/sqrt(K), 1/sqrt(K))
+        bound = 1.0 / math.sqrt(s.conv_width)
+        p["w_conv"] = uniform(sd, layer, "w_conv", (s.d_inner, s.conv_width), -bound, bound, dt)
+        p["b_conv"] = uniform(sd, layer, "b_conv", (s.d_inner,), -bound, bound)
+    if s.d_skip:
+        p["d_skip"] = uniform(sd, layer, "d_skip", (s.d_inner,), 0.5, 1.5)
     if norm_gains:
         p["norm1"] = uniform(sd, layer, "norm1", (s.d_model,), 0.5, 1.5)
         p["norm2"] = uniform(sd, layer, "norm2", (s.d_model,), 0.5, 1.5)

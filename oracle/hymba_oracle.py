@@ -30,8 +30,10 @@ Sources (web pages on Hymba, arXiv 2411.13676), cited by page and section:
 Readings where the pages are silent or disagree (each also listed in the
 design notes): attention scale 1/sqrt(head_dim); no positional encoding;
 A = -exp(A_log) per channel (or per channel and state); [dt_low | B | C] =
-x_proj(X_ssm) and dt = softplus(dt_low W_dt^T + b_dt); no conv1d and no D skip;
-RMSNorm over each branch's full width with eps and no separate gain; the
+x_proj(X_ssm) and dt = softplus(dt_low W_dt^T + b_dt); no conv1d and no D skip by
+default (Mamba's causal depthwise conv + SiLU on X_ssm and its D skip are options);
+RMSNorm over each branch's full width with eps and no separate gain by default (per-group
+norm and difference fusion, from the intra-layer hybrid study, are options); the
 branches of unequal width are combined as out_proj of their concatenation;
 query i sees key j iff j <= i and (i - j <= W or j < M); meta rows are queries
 under the same mask, run through the SSM from h = 0, and kept in the output;
@@ -245,28 +247,74 @@ def ssm_from_alpha(x, alpha):
     return np.einsum("cij,jc->ic", f64(alpha), f64(x))
 
 
-def ssm_branch(x_ssm, g_raw, w_x, w_dt, b_dt, a_log, d_state: int, dt_rank: int):
+def causal_conv1d(x, w_conv, b_conv):
+    """Depthwise causal convolution along time, the short convolution of a Mamba head
+    ([R] "Design formulation" names the SSM head a Mamba head; the pages print no
+    convolution, so it is an option): out[t, c] = b[c] + sum_{k<K} w[c, k] x[t-(K-1)+k, c],
+    rows before the first one read as zero.  x [..., T, Di], w_conv [Di, K], b_conv [Di]."""
+    x, w = f64(x), f64(w_conv)
+    K, T = w.shape[1], x.shape[-2]
+    out = np.zeros_like(x) + f64(b_conv)
+    for k in range(K):
+        shift = K - 1 - k
+        out[..., shift:, :] += w[:, k] * x[..., :T - shift, :]
+    return out
+
+
+def ssm_branch(x_ssm, g_raw, w_x, w_dt, b_dt, a_log, d_state: int, dt_rank: int, w_conv=None, b_conv=None,
+               d_skip=None):
     """One sequence's SSM heads: x_proj -> (dt_low, B, C); dt = softplus(dt_low
-    W_dt^T + b_dt); scan; gate.  x_ssm, g_raw [T, Di] -> Y_ssm [T, Di]."""
-    xdbc = linear(x_ssm, w_x)
+    W_dt^T + b_dt); scan; gate.  x_ssm, g_raw [T, Di] -> Y_ssm [T, Di].
+    Mamba options (not in the pages' formula): with w_conv the head's input is
+    x = SiLU(conv(X_ssm) + b_conv) in place of X_ssm (for x_proj and the scan alike); with
+    d_skip the output before the gate is y + D * x."""
+    x = silu(causal_conv1d(x_ssm, w_conv, b_conv)) if w_conv is not None else f64(x_ssm)
+    xdbc = linear(x, w_x)
     dt_low = xdbc[..., :dt_rank]
     Bm = xdbc[..., dt_rank:dt_rank + d_state]
     Cm = xdbc[..., dt_rank + d_state:dt_rank + 2 * d_state]
     dt = softplus(linear(dt_low, w_dt) + f64(b_dt))
-    y = selective_scan(x_ssm, dt, ssm_decay_rate(a_log), Bm, Cm)
+    y = selective_scan(x, dt, ssm_decay_rate(a_log), Bm, Cm)
+    if d_skip is not None:
+        y = y + f64(d_skip) * x
     return silu(g_raw) * y
+
+
+def _ssm_opts(p):
+    return dict(w_conv=p.get("w_conv"), b_conv=p.get("b_conv"), d_skip=p.get("d_skip"))
 
 
 # ---------------------------------------------------------------------------
 # fusion, layer, stack
 
-def branch_fusion(y_attn, y_ssm, beta1, beta2, eps: float):
+def rms_normalize_groups(v, eps: float, group: int = 0):
+    """Group RMSNorm: each run of `group` consecutive features normalised on its own
+    (group 0: the whole last axis, rms_normalize).  The intra-layer hybrid study
+    summarised on the gist.science page finds group normalisation of the branch outputs
+    effective; a group is read as one head's width."""
+    v = f64(v)
+    if not group or group == v.shape[-1]:
+        return rms_normalize(v, eps)
+    assert v.shape[-1] % group == 0
+    g = v.reshape(v.shape[:-1] + (v.shape[-1] // group, group))
+    return rms_normalize(g, eps).reshape(v.shape)
+
+
+def branch_fusion(y_attn, y_ssm, beta1, beta2, eps: float, group: int = 0, difference: bool = False):
     """Z = [beta1 * norm(Y_attn) || beta2 * norm(Y_ssm)], the argument of W_out
     ([R] "Design formulation", total fusion formulation; the two branch widths
     differ, so the sum inside W_out(.) is taken as W_out applied to the
-    concatenation, i.e. the sum of each branch mapped by its slice of W_out)."""
-    return np.concatenate([f64(beta1) * rms_normalize(y_attn, eps),
-                           f64(beta2) * rms_normalize(y_ssm, eps)], axis=-1)
+    concatenation, i.e. the sum of each branch mapped by its slice of W_out).
+    Variants of the intra-layer hybrid study (gist.science page): norm per group of
+    `group` features, and difference fusion, the SSM branch subtracted instead of added
+    (its half of Z negated)."""
+    sign = -1.0 if difference else 1.0
+    return np.concatenate([f64(beta1) * rms_normalize_groups(y_attn, eps, group),
+                           sign * f64(beta2) * rms_normalize_groups(y_ssm, eps, group)], axis=-1)
+
+
+def _fusion_opts(s):
+    return dict(group=getattr(s, "norm_group", 0), difference=bool(getattr(s, "fusion", 0)))
 
 
 def layer_forward(x, meta, p: Dict[str, np.ndarray], s, kv_in: Optional[Tuple] = None,
@@ -289,9 +337,9 @@ def layer_forward(x, meta, p: Dict[str, np.ndarray], s, kv_in: Optional[Tuple] =
     y_attn = np.stack([attention(parts["q"][b], k[b], v[b], s.n_q_heads, s.n_kv_heads,
                                  s.n_meta, s.window) for b in range(B)])
     y_ssm = np.stack([ssm_branch(parts["x_ssm"][b], parts["g_raw"][b], p["w_x"], p["w_dt"],
-                                 p["b_dt"], p["a_log"], s.d_state, s.dt_rank)
+                                 p["b_dt"], p["a_log"], s.d_state, s.dt_rank, **_ssm_opts(p))
                       for b in range(B)])
-    z = branch_fusion(y_attn, y_ssm, p["beta1"], p["beta2"], s.rms_eps)
+    z = branch_fusion(y_attn, y_ssm, p["beta1"], p["beta2"], s.rms_eps, **_fusion_opts(s))
     out = linear(z, p["w_out"])
     if return_parts:
         return out, (k, v), dict(parts, y_attn=y_attn, y_ssm=y_ssm, z=z)
@@ -314,8 +362,8 @@ def layer_forward_rows(x, meta, p: Dict[str, np.ndarray], s, rows, kv_in: Option
     y_attn = attention(parts["q"][0][rows], k[0], v[0], s.n_q_heads, s.n_kv_heads, s.n_meta, s.window,
                        rows=rows)
     y_ssm = ssm_branch(parts["x_ssm"][0], parts["g_raw"][0], p["w_x"], p["w_dt"], p["b_dt"], p["a_log"],
-                       s.d_state, s.dt_rank)[rows]
-    return linear(branch_fusion(y_attn, y_ssm, p["beta1"], p["beta2"], s.rms_eps), p["w_out"])
+                       s.d_state, s.dt_rank, **_ssm_opts(p))[rows]
+    return linear(branch_fusion(y_attn, y_ssm, p["beta1"], p["beta2"], s.rms_eps, **_fusion_opts(s)), p["w_out"])
 
 
 # ---------------------------------------------------------------------------
@@ -327,6 +375,7 @@ def layer_prefill_state(x, meta, p: Dict[str, np.ndarray], s, kv_in: Optional[Tu
     heads' state after the last row, h_T [B, Di, N] -- the fixed-size state the SSM
     heads carry where attention keeps a growing cache ([R] "Efficiency and KV cache
     optimization").  Returns (out [B, T, d], (K, V), h_T)."""
+    assert p.get("w_conv") is None, "the generation step carries no convolution state"
     out, (k, v), parts = layer_forward(x, meta, p, s, kv_in=kv_in, return_parts=True)
     hs = []
     for b in range(out.shape[0]):
@@ -351,6 +400,7 @@ def layer_decode_step(x_t, p: Dict[str, np.ndarray], s, kv_cache: Tuple, h, pos:
     appended), or the producer's (K, V) [B, pos + 1, Hkv*dh] already holding the new row
     for a consuming layer.  h [B, Di, N].  Returns (out_t, (K, V) with pos + 1 rows,
     h_new)."""
+    assert p.get("w_conv") is None, "the generation step carries no convolution state"
     xt = f64(x_t)[:, None, :]
     B = xt.shape[0]
     parts = split_in_proj(linear(xt, p["w_in"]), s)
@@ -370,9 +420,11 @@ def layer_decode_step(x_t, p: Dict[str, np.ndarray], s, kv_cache: Tuple, h, pos:
         y, hb = selective_scan(parts["x_ssm"][b], dt[b], A, xdbc[b, :, s.dt_rank:s.dt_rank + s.d_state],
                                xdbc[b, :, s.dt_rank + s.d_state:s.dt_rank + 2 * s.d_state], h0=h[b],
                                return_state=True)
+        if p.get("d_skip") is not None:
+            y = y + f64(p["d_skip"]) * parts["x_ssm"][b]
         ys.append(silu(parts["g_raw"][b]) * y)
         hs.append(hb)
-    z = branch_fusion(y_attn, np.stack(ys), p["beta1"], p["beta2"], s.rms_eps)
+    z = branch_fusion(y_attn, np.stack(ys), p["beta1"], p["beta2"], s.rms_eps, **_fusion_opts(s))
     return linear(z, p["w_out"])[:, 0], (k, v), np.stack(hs)
 
 

@@ -448,3 +448,107 @@ def test_layer_forward_rows_equals_the_full_layer_rows(window, kv):
     rows = np.array([0, 1, s.n_meta, s.T // 2, s.T - 1])
     np.testing.assert_allclose(O.layer_forward_rows(x, meta, p, s, rows, kv_in=kv_in), full[0][rows],
                                rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Mamba options (causal conv + SiLU, D skip) and the fusion variants (group norm, difference)
+
+def test_causal_conv_equals_a_library_fir_filter_per_channel():
+    """out[:, c] = b[c] + FIR filter of x[:, c] with taps w[c, ::-1] (scipy.signal.lfilter),
+    i.e. a causal convolution whose rows before the first read as zero."""
+    import scipy.signal
+    T, Di, K = 19, 5, 4
+    x = RNG.standard_normal((T, Di))
+    w = RNG.standard_normal((Di, K))
+    b = RNG.standard_normal(Di)
+    out = O.causal_conv1d(x, w, b)
+    for c in range(Di):
+        np.testing.assert_allclose(out[:, c], b[c] + scipy.signal.lfilter(w[c, ::-1], [1.0], x[:, c]), rtol=1e-12,
+                                   atol=1e-13)
+
+
+def test_causal_conv_is_causal_and_width_one_identity():
+    T, Di, K = 12, 3, 4
+    x = RNG.standard_normal((2, T, Di))
+    w, b = RNG.standard_normal((Di, K)), RNG.standard_normal(Di)
+    a = O.causal_conv1d(x, w, b)
+    x2 = x.copy()
+    x2[:, 7] += 5.0
+    c2 = O.causal_conv1d(x2, w, b)
+    np.testing.assert_array_equal(a[:, :7], c2[:, :7])
+    assert np.abs(a[:, 7:7 + K] - c2[:, 7:7 + K]).min() > 0       # rows t..t+K-1 see row t
+    np.testing.assert_array_equal(a[:, 7 + K:], c2[:, 7 + K:])     # and no later row
+    np.testing.assert_allclose(O.causal_conv1d(x, np.ones((Di, 1)), np.zeros(Di)), x, rtol=0)
+
+
+def test_d_skip_alone_when_c_is_zero_and_conv_feeds_x_proj_and_scan():
+    """With W_x's C rows zero the scan output is 0, so Y = SiLU(G) * D * x with x the head's
+    input -- SiLU(conv(X_ssm) + b) when the conv is on; without D and conv the branch is
+    unchanged."""
+    T, Di, N, R = 9, 6, 3, 2
+    xs, g = RNG.standard_normal((T, Di)), RNG.standard_normal((T, Di))
+    w_x = RNG.standard_normal((R + 2 * N, Di))
+    w_x[R + N:] = 0.0
+    w_dt, b_dt, a_log = RNG.standard_normal((Di, R)), RNG.standard_normal(Di), RNG.uniform(0, 2, Di)
+    D = RNG.uniform(0.5, 1.5, Di)
+    w_c, b_c = RNG.standard_normal((Di, 4)), RNG.standard_normal(Di)
+    sig = lambda z: 1.0 / (1.0 + np.exp(-z))
+    y = O.ssm_branch(xs, g, w_x, w_dt, b_dt, a_log, N, R, d_skip=D)
+    np.testing.assert_allclose(y, g * sig(g) * D * xs, rtol=1e-12)
+    xc = O.causal_conv1d(xs, w_c, b_c)
+    y = O.ssm_branch(xs, g, w_x, w_dt, b_dt, a_log, N, R, w_conv=w_c, b_conv=b_c, d_skip=D)
+    np.testing.assert_allclose(y, g * sig(g) * D * xc * sig(xc), rtol=1e-12)
+    w_x2 = RNG.standard_normal((R + 2 * N, Di))
+    np.testing.assert_array_equal(O.ssm_branch(xs, g, w_x2, w_dt, b_dt, a_log, N, R),
+                                  O.ssm_branch(xs, g, w_x2, w_dt, b_dt, a_log, N, R, d_skip=None))
+
+
+def test_group_norm_closed_forms():
+    """Groups of constant values c_j normalise to sign(c_j) (eps 0); every group has unit RMS;
+    one group over the whole width is the plain RMSNorm."""
+    c = np.array([3.0, -0.5, 2.0, -7.0])
+    v = np.repeat(c, 4)[None, :]
+    np.testing.assert_allclose(O.rms_normalize_groups(v, 0.0, 4), np.repeat(np.sign(c), 4)[None, :], rtol=1e-15)
+    z = RNG.standard_normal((5, 24))
+    n = O.rms_normalize_groups(z, 0.0, 8).reshape(5, 3, 8)
+    np.testing.assert_allclose(np.sqrt((n * n).mean(-1)), 1.0, rtol=1e-13)
+    np.testing.assert_array_equal(O.rms_normalize_groups(z, 1e-6, 24), O.rms_normalize(z, 1e-6))
+    np.testing.assert_array_equal(O.rms_normalize_groups(z, 1e-6, 0), O.rms_normalize(z, 1e-6))
+
+
+def test_difference_fusion_identity():
+    """out(difference) + out(sum) = 2 out(beta2 = 0): the SSM branch enters with the opposite
+    sign and the attention branch is unchanged (eps tiny, so both branches normalise to
+    unit RMS)."""
+    s, x, meta, p = _tiny(rms_eps=1e-14)
+    sd = dataclasses.replace(s, fusion=1)
+    o_sum, _ = O.layer_forward(x, meta, p, s)
+    o_dif, _ = O.layer_forward(x, meta, p, sd)
+    o_att, _ = O.layer_forward(x, meta, dict(p, beta2=np.zeros_like(p["beta2"])), s)
+    np.testing.assert_allclose(o_sum + o_dif, 2.0 * o_att, rtol=1e-11, atol=1e-12)
+    assert np.abs(o_sum - o_dif).max() > 1e-3
+
+
+def test_layer_with_every_option_matches_its_hand_composition():
+    """Conv + D skip + group norm + difference through layer_forward equal the stages
+    composed by hand for one sequence."""
+    s = _tiny_shape(batch=1, conv_width=4, d_skip=1, norm_group=4, fusion=1, window=3)
+    wl = synth.Workload("t", [s], 8, 1e-3, False, "t")
+    x, meta = synth.layer_inputs(wl)
+    p = synth.layer_params(wl, 0)
+    assert p["w_conv"].shape == (s.d_inner, 4) and p["d_skip"].shape == (s.d_inner,)
+    out, _ = O.layer_forward(x, meta, p, s)
+    xt = O.meta_prepend(x, meta)[0]
+    parts = O.split_in_proj(xt @ p["w_in"].T.astype(float), s)
+    ya = O.attention(parts["q"], parts["k"], parts["v"], s.n_q_heads, s.n_kv_heads, s.n_meta, s.window)
+    xc = O.causal_conv1d(parts["x_ssm"], p["w_conv"], p["b_conv"])
+    xc = xc / (1.0 + np.exp(-xc))
+    xdbc = xc @ p["w_x"].T.astype(float)
+    dt = np.log1p(np.exp(xdbc[:, :s.dt_rank] @ p["w_dt"].T.astype(float) + p["b_dt"]))
+    y = O.selective_scan(xc, dt, -np.exp(p["a_log"].astype(float)), xdbc[:, s.dt_rank:s.dt_rank + s.d_state],
+                         xdbc[:, s.dt_rank + s.d_state:])
+    ys = parts["g_raw"] * scipy.special.expit(parts["g_raw"]) * (y + p["d_skip"] * xc)
+    grp = lambda v: (v.reshape(v.shape[0], -1, 4) / np.sqrt((v.reshape(v.shape[0], -1, 4) ** 2).mean(-1, keepdims=True)
+                                                                + 1e-6)).reshape(v.shape)
+    z = np.concatenate([p["beta1"] * grp(ya), -p["beta2"] * grp(ys)], 1)
+    np.testing.assert_allclose(out[0], z @ p["w_out"].T.astype(float), rtol=1e-11, atol=1e-12)
