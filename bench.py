@@ -408,13 +408,13 @@ def weak_scaling_rate(world: int, steps: int, units_per_step_per_rank: float, ma
 class Workbench:
     """Device-resident inputs, weights and buffers of one workload, and its step."""
 
-    def __init__(self, name, dev):
+    def __init__(self, name, dev, **overrides):
         import torch
 
         import hybrid_attention_ssm_hymba_b200 as H
         from hybrid_attention_ssm_hymba_b200 import host
         self.H, self.torch = H, torch
-        self.wl = wl = synth.workload(name)
+        self.wl = wl = synth.workload(name, **overrides)
         self.s0 = s0 = wl.first
         self.dtype = s0.dtype
         self.x_np, self.meta_np = synth.layer_inputs(wl)
@@ -435,7 +435,11 @@ class Workbench:
         self.stream = torch.cuda.current_stream(dev)
         self.dt_in_scan = [H.hymba_layer_fuses_dt_proj(c) for c in self.cfgs]
         bf16 = self.dtype == "bf16"
-        per_layer = [(8 if bf16 else 7) - int(f) for f in self.dt_in_scan]
+        # in_proj, x_proj, dt_proj (unless the scan computes dt), attention, scan, the branch norm
+        # (bf16 whole-branch: row sums + beta-scaled W_out; else one in-place norm), out_proj;
+        # the options add the conv and the D skip
+        per_layer = [(8 if bf16 and not s.norm_group else 7) - int(f) + int(s.conv_width > 0) + int(bool(s.d_skip))
+                     for f, s in zip(self.dt_in_scan, wl.layers)]
         if self.stack:   # the prepend; per block: the mixer's pre-norm (bf16: + W_SSM transpose and the
             # W_eff GEMM), the layer, and with an FFN its pre-norm and two GEMMs
             self.launches = 1 + sum(n + (3 if bf16 else 1) + (3 if s.ffn_dim else 0)
@@ -620,6 +624,57 @@ def measure_e2e(bench: Workbench, ranks, dev, flush, K):
                     "buffers each, so consecutive steps' copies and layers overlap"}
 
 
+def measure_prefixed(bench: Workbench, K: int, W: int, dev, flush):
+    """The workload's layers with their meta rows from records of hymba_meta_prefix (built
+    once, outside the timed region): hymba_layer_fwd_prefixed runs the user rows only.
+    Timed like the headline (K steps, L2 flushed between them)."""
+    import torch
+    H = bench.H
+    from hybrid_attention_ssm_hymba_b200 import host
+    s0, st = bench.s0, bench.stream
+    if bench.stack or s0.n_meta == 0:
+        return None
+    es = 2 if bench.dtype == "bf16" else 4
+    recs = [host.workspace(H.hymba_meta_prefix_size(c), dev) for c in bench.cfgs]
+    meta_in = bench.meta
+    for i, c in enumerate(bench.cfgs):
+        H.check(H.hymba_meta_prefix(meta_in, bench.weights[i], c, recs[0] if i > 0 else None, recs[i], bench.ws,
+                                    stream=st), "meta prefix")
+        meta_in = recs[i][:s0.n_meta * s0.d_model * es].view(bench.x.dtype).view(s0.n_meta, s0.d_model)
+    user_in = [None] + [o[:, s0.n_meta:] for o in bench.outs[:-1]]
+    # a consumer's input rows: the producer's user rows, in a contiguous buffer
+    user_bufs = [None] + [torch.empty((s0.batch, s0.seq_len, s0.d_model), dtype=bench.x.dtype, device=dev)
+                          for _ in bench.outs[:-1]]
+
+    def step():
+        xin = bench.x
+        for i, c in enumerate(bench.cfgs):
+            if i > 0:
+                user_bufs[i].copy_(user_in[i])
+                xin = user_bufs[i]
+            H.check(H.hymba_layer_fwd_prefixed(xin, recs[i], bench.weights[i], c, bench.kv if i > 0 else None,
+                                               bench.kv if i == 0 else None, bench.outs[i], bench.ws, stream=st),
+                    "prefixed")
+
+    for _ in range(W):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for k in range(K):
+        flush.zero_()
+        ev[k][0].record(st)
+        step()
+        ev[k][1].record(st)
+    torch.cuda.synchronize(dev)
+    assert H.hymba_workspace_status(bench.ws, st) == H.HYMBA_OK
+    ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    return {"ms_per_step": ms, "value": bench.tokens / (ms * 1e-3), "unit": UNIT,
+            "note": "meta rows from hymba_meta_prefix records built once per weight set; each step runs "
+                    "hymba_layer_fwd_prefixed on the user rows (a consumer's input copied out of the producer's "
+                    "output rows inside the step)"}
+
+
 def measure_decode(name: str, dev, flush, steps: int = 64, warmup: int = 8):
     """Generation steps of a layer workload after its full prompt: hymba_layer_prefill of every
     layer (untimed), then one new token per sequence per step through every layer
@@ -703,6 +758,10 @@ def run_native(args, rank, world, local_rank):
             if k in rec:
                 line[k] = rec[k]
         line["device_status"] = bench.H.hymba_status_string(status)
+        pre = measure_prefixed(bench, K, args.warmup, dev, flush)
+        if pre is not None:
+            pre["saving_frac"] = round(1.0 - pre["ms_per_step"] / line["ms_per_step"], 4)
+            line["meta_prefix"] = pre
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, bench.x_np, bench.meta_np, bench.ps_np)
     del bench
@@ -728,6 +787,21 @@ def run_native(args, rank, world, local_rank):
             line["per_workload"] = per
     if world == 1 and not args.no_decode and line is not None:
         line["decode"] = measure_decode("hymba1p5b_kvpair", dev, flush)
+    if world == 1 and not args.no_per_workload and line is not None:
+        # the option paths (Mamba conv + D skip, per-group branch norm, difference fusion) on
+        # the 350M-shaped layer, against the same layer without them
+        opts = dict(conv_width=4, d_skip=1, norm_group=128, fusion=1)
+        b = Workbench("hymba350m_layer", dev, **opts)
+        r, t_ms = measure(b, min(K, 10), 3, ranks, dev, flush, stages=True, e2e=False)
+        r["value"] = weak_scaling_rate(1, min(K, 10), b.tokens, t_ms)
+        r["unit"] = UNIT
+        r["options"] = opts
+        base = line.get("per_workload", {}).get("hymba350m_layer")
+        if base:
+            r["overhead_frac"] = round(r["ms_per_step"] / base["ms_per_step"] - 1.0, 4)
+        line["options"] = r
+        del b
+        torch.cuda.empty_cache()
     if line is not None:
         print(json.dumps(line), flush=True)
     ranks.close()

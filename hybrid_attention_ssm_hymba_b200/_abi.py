@@ -25,6 +25,7 @@ ENTRY_POINTS = (
     "hymba_stack_fwd", "hymba_workspace_status", "hymba_layer_fwd_events", "hymba_gemm", "hymba_selective_scan",
     "hymba_attention", "hymba_branch_norm", "hymba_rmsnorm", "hymba_layer_fwd_noalloc", "hymba_layer_fuses_dt_proj",
     "hymba_check_wait_timeout", "hymba_decode_workspace_size", "hymba_layer_prefill", "hymba_layer_decode",
+    "hymba_meta_prefix_size", "hymba_meta_prefix", "hymba_layer_fwd_prefixed",
 )
 
 # size of the library-owned scratch block behind hymba_layer_fwd_noalloc (HYMBA_NOALLOC_SCRATCH_BYTES)
@@ -42,13 +43,14 @@ class hymba_cfg_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "batch", "seq_len", "n_meta", "d_model", "n_q_heads", "n_kv_heads", "head_dim", "window",
         "d_inner", "d_state", "n_ssm_heads", "dt_rank", "a_per_state", "kv_mode", "ffn_dim")] + [
-        ("rms_eps", ctypes.c_float), ("dtype", ctypes.c_int)]
+        ("rms_eps", ctypes.c_float), ("dtype", ctypes.c_int), ("conv_width", ctypes.c_int),
+        ("norm_group", ctypes.c_int), ("fusion", ctypes.c_int)]
 
 
 class hymba_weights_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "w_in", "w_x", "w_dt", "w_out", "a_log", "b_dt", "beta1", "beta2", "w_gate_up", "w_down",
-        "norm1", "norm2")]
+        "norm1", "norm2", "w_conv", "b_conv", "d_skip")]
 
 
 _VP, _SZ, _I, _F = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
@@ -73,6 +75,11 @@ _SIGS = {
     "hymba_rmsnorm": (_I, [_VP, _VP, _I, _I, _F, _I, _VP]),
     "hymba_check_wait_timeout": (_I, [_VP, _SZ, ctypes.c_uint, _VP]),
     "hymba_decode_workspace_size": (_SZ, [ctypes.POINTER(hymba_cfg_t)]),
+    "hymba_meta_prefix_size": (_SZ, [ctypes.POINTER(hymba_cfg_t)]),
+    "hymba_meta_prefix": (_I, [_VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t), _VP, _VP, _VP,
+                               _SZ, _VP]),
+    "hymba_layer_fwd_prefixed": (_I, [_VP, _VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t),
+                                      _VP, _VP, _VP, _VP, _SZ, _VP]),
     "hymba_layer_prefill": (_I, [_VP, _VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t),
                                  _VP, _I, _VP, _VP, _VP, _SZ, _VP]),
     "hymba_layer_decode": (_I, [_VP, ctypes.POINTER(hymba_weights_t), ctypes.POINTER(hymba_cfg_t),
@@ -236,6 +243,23 @@ def hymba_branch_norm(z, beta1, beta2, rows: int, w_attn: int, w_ssm: int, eps: 
 
 def hymba_rmsnorm(x, y, rows: int, d: int, eps: float, dtype: int, stream=None) -> int:
     return load().hymba_rmsnorm(_ptr(x), _ptr(y), rows, d, eps, dtype, _stream(stream))
+
+
+def hymba_meta_prefix_size(cfg: hymba_cfg_t) -> int:
+    return load().hymba_meta_prefix_size(ctypes.byref(cfg))
+
+
+def hymba_meta_prefix(meta_in, weights: hymba_weights_t, cfg: hymba_cfg_t, kv_prefix_in, prefix, workspace,
+                      stream=None) -> int:
+    return load().hymba_meta_prefix(_ptr(meta_in), ctypes.byref(weights), ctypes.byref(cfg), _ptr(kv_prefix_in),
+                                    _ptr(prefix), _ptr(workspace), _nbytes(workspace), _stream(stream))
+
+
+def hymba_layer_fwd_prefixed(x, prefix, weights: hymba_weights_t, cfg: hymba_cfg_t, kv_in, kv_out, out,
+                             workspace, stream=None) -> int:
+    return load().hymba_layer_fwd_prefixed(_ptr(x), _ptr(prefix), ctypes.byref(weights), ctypes.byref(cfg),
+                                           _ptr(kv_in), _ptr(kv_out), _ptr(out), _ptr(workspace),
+                                           _nbytes(workspace), _stream(stream))
 
 
 def hymba_decode_workspace_size(cfg: hymba_cfg_t) -> int:

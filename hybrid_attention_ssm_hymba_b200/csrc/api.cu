@@ -31,13 +31,14 @@ inline size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 inline size_t esize(hymba_dtype_t t) { return t == HYMBA_BF16 ? 2 : 4; }
 
 struct LayerWs {
-  size_t q, kv, xs, g, dtlow, bc, dt, z, ssq, wsc, total;
+  size_t q, kv, xs, g, dtlow, bc, dt, z, ssq, wsc, xc, total;
 };
 
 // bf16 layers fuse the branch norm into out_proj (the row-sum kernel holds a row of up
-// to 6144 bf16 in one warp's registers); fp32 layers run the separate norm kernel.
+// to 6144 bf16 in one warp's registers); fp32 layers and per-group norms run a separate
+// norm kernel.
 bool fused_branch_norm(const hymba_cfg_t& c) {
-  return c.dtype == HYMBA_BF16 && c.n_q_heads * c.head_dim + c.d_inner <= 6144;
+  return c.dtype == HYMBA_BF16 && c.norm_group == 0 && c.n_q_heads * c.head_dim + c.d_inner <= 6144;
 }
 
 LayerWs layer_ws(const hymba_cfg_t& c, size_t base) {
@@ -60,6 +61,7 @@ LayerWs layer_ws(const hymba_cfg_t& c, size_t base) {
   const bool fused = fused_branch_norm(c);
   w.ssq = o; o = al256(o + (fused ? rows * 2 * sizeof(float) : 0));
   w.wsc = o; o = al256(o + (fused ? static_cast<size_t>(c.d_model) * (wa + c.d_inner) * es : 0));
+  w.xc = o; o = al256(o + (c.conv_width > 0 ? rows * c.d_inner * es : 0));   // SiLU(conv(X_ssm))
   w.total = o;
   return w;
 }
@@ -114,6 +116,11 @@ hymba_status_t validate_cfg(const hymba_cfg_t* c) {
     return HYMBA_ERR_INVALID_ARG;
   if (c->n_q_heads % c->n_kv_heads != 0) return HYMBA_ERR_INVALID_ARG;
   if (c->a_per_state != 0 && c->a_per_state != 1) return HYMBA_ERR_INVALID_ARG;
+  if (c->conv_width < 0 || c->conv_width > 4 || c->fusion < 0 || c->fusion > 1 || c->norm_group < 0)
+    return HYMBA_ERR_INVALID_ARG;
+  if (c->norm_group && ((c->norm_group != 64 && c->norm_group != 128 && c->norm_group != 256) ||
+                        (c->n_q_heads * c->head_dim) % c->norm_group || c->d_inner % c->norm_group))
+    return HYMBA_ERR_UNSUPPORTED;
   if (!valid_state(c->d_state)) return HYMBA_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(c->batch) * (c->seq_len + c->n_meta);
   if (rows > (1ll << 31) - 1) return HYMBA_ERR_UNSUPPORTED;
@@ -151,6 +158,7 @@ bool weights_ok(const hymba_weights_t* w, const hymba_cfg_t& c, bool need_ffn) {
   if (!w || !w->w_in || !w->w_x || !w->w_dt || !w->w_out || !w->a_log || !w->b_dt || !w->beta1 || !w->beta2)
     return false;
   if (need_ffn && c.ffn_dim > 0 && (!w->w_gate_up || !w->w_down)) return false;
+  if (c.conv_width > 0 && (!w->w_conv || !w->b_conv)) return false;
   return true;
 }
 
@@ -215,7 +223,28 @@ struct LayerOut {
   const void* weff = nullptr;
   float* h_out = nullptr;
   long long kv_rows = 0;
+  // Meta-prefix record (hymba_meta_prefix): x holds the user rows [B, L, d] only; the meta
+  // rows' K/V, SSM state and outputs come from the record instead of being recomputed.
+  const uint8_t* prefix = nullptr;
 };
+
+// Layout of a meta-prefix record (offsets in bytes): the M meta rows' layer output
+// [M, d] (dtype), their K then V [2, M, Hkv*dh] (dtype; none for a consuming layer) and
+// the SSM state after them [Di, N] fp32.
+struct PrefixLayout {
+  size_t out, kv, h, total;
+};
+PrefixLayout prefix_layout(const hymba_cfg_t& c) {
+  const size_t es = esize(c.dtype), M = static_cast<size_t>(c.n_meta);
+  const size_t wkv = static_cast<size_t>(c.n_kv_heads) * c.head_dim;
+  PrefixLayout p;
+  size_t o = 0;
+  p.out = o; o = al256(o + M * c.d_model * es);
+  p.kv = o; o = al256(o + (c.kv_mode == HYMBA_KV_CONSUME ? 0 : 2 * M * wkv * es));
+  p.h = o; o = al256(o + static_cast<size_t>(c.d_inner) * c.d_state * 4);
+  p.total = o;
+  return p;
+}
 
 // One layer.  x: meta mode when meta != nullptr, else [rows, d] holding X~.
 hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t& w, const hymba_cfg_t& c,
@@ -240,8 +269,11 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   void* dt = ws + L.dt;
   void* z = ws + L.z;
 
+  // the SSM heads' input: X_ssm, or SiLU(conv(X_ssm)) with the Mamba conv
+  void* xin_ssm = c.conv_width > 0 ? static_cast<void*>(ws + L.xc) : xs;
+  const float s2 = c.fusion ? -1.f : 1.f;   // difference fusion: the SSM branch subtracted
   hy::ScanDesc sd;
-  sd.x = xs;
+  sd.x = xin_ssm;
   sd.dt = dt;
   sd.bc = bc;
   sd.gate = g;
@@ -256,6 +288,12 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   sd.status = status;
   sd.a_per_state = c.a_per_state != 0;
   sd.h_out = lo.h_out;
+  const PrefixLayout PL = prefix_layout(c);
+  if (lo.prefix) {   // the scan starts after the meta rows, from their state
+    sd.t0 = c.n_meta;
+    sd.h0 = reinterpret_cast<const float*>(lo.prefix + PL.h);
+    sd.h0_bstride = 0;
+  }
   // bf16 with d_state 16 and dt_rank 64: dt_proj runs inside the tensor-core scan
   // (dt = softplus(dt_low W_dt^T + b_dt) per block, never stored)
   {
@@ -281,7 +319,13 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   // 1 in_proj
   mark(0);
   GemmDesc gi;
-  if (meta) {
+  if (lo.prefix) {   // user rows only, written at their places in the [B, T] layout
+    gi.a = x;
+    gi.a_rows = static_cast<long long>(c.batch) * c.seq_len;
+    gi.remap_L = c.seq_len;
+    gi.remap_T = T;
+    gi.remap_M = c.n_meta;
+  } else if (meta) {
     gi.meta_mode = true;
     gi.x = x;
     gi.meta = meta;
@@ -312,6 +356,13 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   gi.status = status;
   cudaError_t e = gemm(gi, c.dtype, st);
   if (e != cudaSuccess) return HYMBA_ERR_CUDA;
+  if (lo.prefix && c.kv_mode != HYMBA_KV_CONSUME) {   // the meta rows' K, V into every sequence
+    const size_t blk = static_cast<size_t>(c.n_meta) * wkv * es, seq = static_cast<size_t>(T) * wkv * es;
+    if (hy::launch_broadcast(lo.prefix + PL.kv, blk, kvbuf, seq, c.batch, st) != cudaSuccess ||
+        hy::launch_broadcast(lo.prefix + PL.kv + blk, blk, static_cast<uint8_t*>(kvbuf) + rows * wkv * es, seq,
+                             c.batch, st) != cudaSuccess)
+      return HYMBA_ERR_CUDA;
+  }
 
   // 4 attention heads -> Z[:, :wa], on the side stream unless stage events are recorded
   // (then every stage runs in order on st)
@@ -333,6 +384,7 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   ad.bf16 = c.dtype == HYMBA_BF16;
   ad.status = status;
   ad.kv_rows = c.kv_mode == HYMBA_KV_CONSUME ? lo.kv_rows : 0;
+  ad.q_row0 = lo.prefix ? c.n_meta : 0;
   SideStream ss;
   cudaStream_t side = nullptr;
   if (!events) {
@@ -350,10 +402,13 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
     if (ea != cudaSuccess) return HYMBA_ERR_CUDA;
   }
 
-  // 2 x_proj
+  // 2 x_proj (after the conv, when the layer has one)
   mark(1);
+  if (c.conv_width > 0 && hy::launch_conv_silu(xs, w.w_conv, w.b_conv, xin_ssm, c.batch, T, di, c.conv_width,
+                                               c.dtype == HYMBA_BF16, st) != cudaSuccess)
+    return HYMBA_ERR_CUDA;
   GemmDesc gx;
-  gx.a = xs;
+  gx.a = xin_ssm;
   gx.a_rows = rows;
   gx.K = di;
   gx.w = w.w_x;
@@ -388,16 +443,24 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   // 5 selective scan + gate -> Z[:, wa:]
   mark(4);
   e = hy::launch_scan(sd, st);
+  if (e == cudaSuccess && w.d_skip)   // Mamba's D skip on the scan's output columns
+    e = hy::launch_ssm_skip(static_cast<uint8_t*>(z) + wa * es, wa + di, g, xin_ssm, w.d_skip, rows, di,
+                            c.dtype == HYMBA_BF16, st);
   if (joiner.join() != cudaSuccess || e != cudaSuccess) return HYMBA_ERR_CUDA;  // the norm reads all of Z
 
   // 6 per-branch RMSNorm and beta
   mark(5);
   if (fused_norm) {
-    if ((e = hy::launch_scale_cols(w.w_out, w_out_scaled, c.d_model, wa, di, w.beta1, w.beta2, st)) != cudaSuccess ||
+    if ((e = hy::launch_scale_cols(w.w_out, w_out_scaled, c.d_model, wa, di, w.beta1, w.beta2, st, s2)) !=
+            cudaSuccess ||
         (e = hy::launch_row_ssq(z, rows, wa, di, ssq, st)) != cudaSuccess)
       return HYMBA_ERR_CUDA;
-  } else if ((e = hy::launch_branch_norm(z, w.beta1, w.beta2, rows, wa, di, c.rms_eps, c.dtype == HYMBA_BF16,
-                                         st)) != cudaSuccess) {
+  } else if (c.norm_group) {
+    if ((e = hy::launch_group_norm(z, rows, wa, di, c.norm_group, w.beta1, w.beta2, s2, c.rms_eps,
+                                   c.dtype == HYMBA_BF16, st)) != cudaSuccess)
+      return HYMBA_ERR_CUDA;
+  } else if ((e = hy::launch_branch_norm(z, w.beta1, w.beta2, rows, wa, di, c.rms_eps, c.dtype == HYMBA_BF16, st,
+                                         s2)) != cudaSuccess) {
     return HYMBA_ERR_CUDA;
   }
 
@@ -431,6 +494,9 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   }
   go.status = status;
   if ((e = gemm(go, c.dtype, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
+  if (lo.prefix && hy::launch_broadcast(lo.prefix + PL.out, static_cast<size_t>(c.n_meta) * c.d_model * es, out,
+                                        static_cast<size_t>(T) * c.d_model * es, c.batch, st) != cudaSuccess)
+    return HYMBA_ERR_CUDA;   // the meta rows' outputs
   mark(7);
   return marks_ok ? HYMBA_OK : HYMBA_ERR_CUDA;
 }
@@ -517,6 +583,7 @@ hymba_cfg_t prefill_cfg(const hymba_cfg_t& c) {
 hymba_status_t validate_generation(const hymba_cfg_t* cfg) {
   hymba_status_t s = validate_cfg(cfg);
   if (s != HYMBA_OK) return s;
+  if (cfg->conv_width > 0) return HYMBA_ERR_UNSUPPORTED;   // no convolution state is carried
   if (cfg->head_dim % 32 || cfg->n_q_heads / cfg->n_kv_heads > 8 || cfg->d_state % 8)
     return HYMBA_ERR_UNSUPPORTED;
   return HYMBA_OK;
@@ -681,9 +748,14 @@ hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weig
     const bool mixer_last = last && c.ffn_dim == 0;
     lo.out = (bf16 && mixer_last) ? out : static_cast<void*>(h);
     lo.out_f32 = !(bf16 && mixer_last);
+    // the B|C compensation is linear in the normalised input: not with the conv option
+    const bool compensate = bf16 && c.conv_width == 0;
     if (bf16) {
-      if ((e = hy::launch_prenorm_f32(h, w[i].norm1, xn, xlo, rows, d, c.rms_eps, st)) != cudaSuccess)
+      if ((e = hy::launch_prenorm_f32(h, w[i].norm1, xn, compensate ? xlo : nullptr, rows, d, c.rms_eps, st)) !=
+          cudaSuccess)
         return HYMBA_ERR_CUDA;
+    }
+    if (compensate) {
       // W_eff = W_x W_SSM [R + 2N, d]: x_proj adds xlo W_eff^T, the part of [dt_low | B | C]
       // that the bf16 rounding of the normalised input dropped
       const int wa = c.n_q_heads * c.head_dim, wkv = c.n_kv_heads * c.head_dim;
@@ -701,8 +773,8 @@ hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weig
       if (gemm(ge, c.dtype, st) != cudaSuccess) return HYMBA_ERR_CUDA;
       lo.xlo = xlo;
       lo.weff = weff;
-    } else if ((e = hy::launch_prenorm_f32_out_f32(h, w[i].norm1, static_cast<float*>(xn), rows, d, c.rms_eps,
-                                                   st)) != cudaSuccess) {
+    } else if (!bf16 && (e = hy::launch_prenorm_f32_out_f32(h, w[i].norm1, static_cast<float*>(xn), rows, d,
+                                                            c.rms_eps, st)) != cudaSuccess) {
       return HYMBA_ERR_CUDA;
     }
     hymba_status_t s = run_layer(xn, nullptr, w[i], c, kv, kv, lo, lws, status, st);
@@ -886,9 +958,14 @@ hymba_status_t hymba_layer_decode(const void* x_t, const hymba_weights_t* w, con
   sd.d_inner = di;
   sd.d_state = c.d_state;
   sd.bf16 = c.dtype == HYMBA_BF16;
+  sd.d_skip = w->d_skip;
   if (hy::launch_scan_step(sd, st) != cudaSuccess) return HYMBA_ERR_CUDA;
-  if (hy::launch_branch_norm(z, w->beta1, w->beta2, B, wa, di, c.rms_eps, c.dtype == HYMBA_BF16, st) != cudaSuccess)
-    return HYMBA_ERR_CUDA;
+  const float s2 = c.fusion ? -1.f : 1.f;
+  const cudaError_t en = c.norm_group ? hy::launch_group_norm(z, B, wa, di, c.norm_group, w->beta1, w->beta2, s2,
+                                                              c.rms_eps, c.dtype == HYMBA_BF16, st)
+                                      : hy::launch_branch_norm(z, w->beta1, w->beta2, B, wa, di, c.rms_eps,
+                                                               c.dtype == HYMBA_BF16, st, s2);
+  if (en != cudaSuccess) return HYMBA_ERR_CUDA;
   GemmDesc go;
   go.a = z;
   go.a_rows = B;
@@ -898,6 +975,73 @@ hymba_status_t hymba_layer_decode(const void* x_t, const hymba_weights_t* w, con
   go.seg[go.nseg++] = seg(0, c.d_model, out_t, c.d_model, 0, hy::SEG_STORE);
   go.status = status;
   return gemm(go, c.dtype, st) == cudaSuccess ? HYMBA_OK : HYMBA_ERR_CUDA;
+}
+
+// ---- meta-prefix precompute: the meta rows once per weight set, then only the user rows
+
+size_t hymba_meta_prefix_size(const hymba_cfg_t* cfg) {
+  if (validate_cfg(cfg) != HYMBA_OK || cfg->n_meta < 1) return 0;
+  return prefix_layout(*cfg).total;
+}
+
+hymba_status_t hymba_meta_prefix(const void* meta_in, const hymba_weights_t* w, const hymba_cfg_t* cfg,
+                                 const void* kv_prefix_in, void* prefix, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  hymba_status_t s = validate_cfg(cfg);
+  if (s != HYMBA_OK) return s;
+  if (cfg->conv_width > 0) return HYMBA_ERR_UNSUPPORTED;   // the conv would need the meta rows' X_ssm
+  if (cfg->n_meta < 1 || !meta_in || !prefix || !weights_ok(w, *cfg, false)) return HYMBA_ERR_INVALID_ARG;
+  if (cfg->kv_mode == HYMBA_KV_CONSUME && !kv_prefix_in) return HYMBA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(prefix) & 255) return HYMBA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < hymba_workspace_size(cfg)) return HYMBA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return HYMBA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* status = static_cast<unsigned*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  // The meta rows alone, as one sequence of M rows: every meta row sees every meta row
+  // before it whatever the window (all are meta tokens), so the prefix runs as global
+  // causal attention; a layer with its own K/V writes them into the record.
+  hymba_cfg_t p = *cfg;
+  p.batch = 1;
+  p.seq_len = cfg->n_meta;
+  p.n_meta = 0;
+  p.window = -1;
+  if (p.kv_mode == HYMBA_KV_OWN) p.kv_mode = HYMBA_KV_PRODUCE;
+  const PrefixLayout PL = prefix_layout(*cfg);
+  uint8_t* rec = static_cast<uint8_t*>(prefix);
+  LayerOut lo;
+  lo.out = rec + PL.out;
+  lo.h_out = reinterpret_cast<float*>(rec + PL.h);
+  lo.kv_rows = cfg->n_meta;
+  // a consuming layer's meta rows read the producer's meta K/V from the producer's record
+  hymba_cfg_t producer = *cfg;
+  producer.kv_mode = HYMBA_KV_PRODUCE;
+  const void* kv_in = cfg->kv_mode == HYMBA_KV_CONSUME
+                          ? static_cast<const uint8_t*>(kv_prefix_in) + prefix_layout(producer).kv
+                          : nullptr;
+  return run_layer(meta_in, nullptr, *w, p, kv_in, cfg->kv_mode == HYMBA_KV_CONSUME ? nullptr : rec + PL.kv, lo,
+                   static_cast<uint8_t*>(workspace) + 256, status, st);
+}
+
+hymba_status_t hymba_layer_fwd_prefixed(const void* x, const void* prefix, const hymba_weights_t* w,
+                                        const hymba_cfg_t* cfg, const void* kv_in, void* kv_out, void* out,
+                                        void* workspace, size_t ws_bytes, void* stream) {
+  hymba_status_t s = validate_cfg(cfg);
+  if (s != HYMBA_OK) return s;
+  if (cfg->conv_width > 0) return HYMBA_ERR_UNSUPPORTED;
+  if (cfg->n_meta < 1 || !x || !prefix || !out || !weights_ok(w, *cfg, false)) return HYMBA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(prefix) & 255) return HYMBA_ERR_INVALID_ARG;
+  if (cfg->kv_mode == HYMBA_KV_CONSUME && !kv_in) return HYMBA_ERR_INVALID_ARG;
+  if (cfg->kv_mode == HYMBA_KV_PRODUCE && !kv_out) return HYMBA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < hymba_workspace_size(cfg)) return HYMBA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return HYMBA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* status = static_cast<unsigned*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), st) != cudaSuccess) return HYMBA_ERR_CUDA;
+  LayerOut lo;
+  lo.out = out;
+  lo.prefix = static_cast<const uint8_t*>(prefix);
+  return run_layer(x, nullptr, *w, *cfg, kv_in, kv_out, lo, static_cast<uint8_t*>(workspace) + 256, status, st);
 }
 
 hymba_status_t hymba_workspace_status(void* workspace, void* stream) {

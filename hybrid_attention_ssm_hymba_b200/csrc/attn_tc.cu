@@ -640,7 +640,8 @@ cudaError_t launch_attention_f32(const AttnDesc& a, cudaStream_t st);
 
 cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st) {
   if (!a.bf16) return launch_attention_f32(a, st);
-  if (a.batch <= 0 || a.T <= 0) return cudaSuccess;
+  if (a.q_row0 < 0) return cudaErrorInvalidValue;
+  if (a.batch <= 0 || a.T <= 0 || a.q_row0 >= a.T) return cudaSuccess;
   static std::atomic<uint64_t> attr_done{0}, attr2_done{0};
   if (cudaError_t e = smem_attr_once(attn_fwd_tc, SMEM_BYTES, attr_done)) return e;
   CUtensorMap tq, tk, tv;
@@ -662,10 +663,10 @@ cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st) {
   p.status = a.status;
   if ((a.n_q_heads / a.n_kv_heads) % 2 == 0) {  // pairs of query heads share each K/V tile
     if (cudaError_t e = smem_attr_once(attn_fwd_tc2, SMEM2_BYTES, attr2_done)) return e;
-    dim3 grid(p.q_tiles, a.n_q_heads / 2, a.batch);
+    dim3 grid(p.q_tiles - a.q_row0 / BQ, a.n_q_heads / 2, a.batch);
     return launch(attn_fwd_tc2, grid, dim3(320), SMEM2_BYTES, st, tq, tk, tv, p);
   }
-  dim3 grid(p.q_tiles, a.n_q_heads, a.batch);
+  dim3 grid(p.q_tiles - a.q_row0 / BQ, a.n_q_heads, a.batch);
   return launch(attn_fwd_tc, grid, dim3(192), SMEM_BYTES, st, tq, tk, tv, p);
 }
 

@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(256) scan_step_kernel(const T* __restrict__ x,
                                                         const float* __restrict__ bc, const T* __restrict__ gate,
                                                         const float* __restrict__ a_log, int a_per_state,
                                                         float* __restrict__ h, T* __restrict__ y, long long y_ld,
-                                                        int B, int Di, int N) {
+                                                        int B, int Di, int N, const float* __restrict__ d_skip) {
   pdl_trigger();
   pdl_wait();
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -241,6 +241,7 @@ __global__ void __launch_bounds__(256) scan_step_kernel(const T* __restrict__ x,
   for (int off = 1; off < 8; off <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, off);
   if (valid && sl == 0) {
     const long long r = static_cast<long long>(b) * Di + c;
+    if (d_skip) yv = fmaf(d_skip[c], to_f<T>(x[r]), yv);
     y[static_cast<long long>(b) * y_ld + c] = from_f<T>(to_f<T>(gate[r]) * yv);
   }
 }
@@ -296,10 +297,11 @@ cudaError_t launch_scan_step(const ScanStepDesc& s, cudaStream_t st) {
     return launch(scan_step_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
                   static_cast<const __nv_bfloat16*>(s.x), static_cast<const __nv_bfloat16*>(s.dt), s.bc,
                   static_cast<const __nv_bfloat16*>(s.gate), s.a_log, s.a_per_state ? 1 : 0, s.h,
-                  static_cast<__nv_bfloat16*>(s.y), s.y_ld, s.batch, s.d_inner, s.d_state);
+                  static_cast<__nv_bfloat16*>(s.y), s.y_ld, s.batch, s.d_inner, s.d_state, s.d_skip);
   return launch(scan_step_kernel<float>, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(s.x),
                 static_cast<const float*>(s.dt), s.bc, static_cast<const float*>(s.gate), s.a_log,
-                s.a_per_state ? 1 : 0, s.h, static_cast<float*>(s.y), s.y_ld, s.batch, s.d_inner, s.d_state);
+                s.a_per_state ? 1 : 0, s.h, static_cast<float*>(s.y), s.y_ld, s.batch, s.d_inner, s.d_state,
+                s.d_skip);
 }
 
 }  // namespace hy

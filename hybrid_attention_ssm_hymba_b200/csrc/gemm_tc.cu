@@ -51,6 +51,7 @@ struct GemmParams {
   void* out;
   long long out_ld;
   int resid_f32, out_f32;   // residual / output element type of EPI_RESIDUAL and the dual epilogue
+  int remap_L, remap_T, remap_M;  // segment rows: r -> (r / L) T + M + r % L when remap_L > 0
   int swiglu_F;
   int bias_len;             // > 0: the (single) bias segment's vector is staged in smem
   const float* bias_src;
@@ -365,6 +366,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         continue;
       }
       if (p.epi == EPI_SEGMENTS) {
+        if (p.remap_L) grow = (grow / p.remap_L) * p.remap_T + p.remap_M + grow % p.remap_L;
         uint32_t v[CPT][32];
 #pragma unroll
         for (int q = 0; q < CPT; ++q) tmem_ld32(tb + (grp + q * EPI_GROUPS) * 32, v[q]);
@@ -569,6 +571,9 @@ cudaError_t launch_bn(const GemmDesc& g, cudaStream_t st) {
   p.out_ld = g.out_ld;
   p.resid_f32 = g.resid_f32 ? 1 : 0;
   p.out_f32 = g.out_f32 ? 1 : 0;
+  p.remap_L = g.meta_mode ? 0 : g.remap_L;
+  p.remap_T = g.remap_T;
+  p.remap_M = g.remap_M;
   p.swiglu_F = g.swiglu_F;
   p.status = g.status;
   const long long total = static_cast<long long>(p.meta_mode ? p.batch : 1) * p.m_tiles * p.n_tiles;

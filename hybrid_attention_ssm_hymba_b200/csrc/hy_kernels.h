@@ -92,6 +92,10 @@ struct GemmDesc {
   // EPI_RESIDUAL and the fused branch-norm epilogue: resid and/or out in fp32 instead of
   // the GEMM's dtype (a residual stream carried in fp32)
   bool resid_f32 = false, out_f32 = false;
+  // Output row remap (plain mode, segment epilogue): row r of A is written as row
+  // (r / remap_L) * remap_T + remap_M + r % remap_L -- the user rows of [batch, L] landing
+  // in a [batch, M + L] layout.  remap_L = 0: off.
+  int remap_L = 0, remap_T = 0, remap_M = 0;
   int swiglu_F = 0;
   // Fused branch norm (bf16 out_proj): the first dual_k_blocks 64-wide K blocks (the
   // attention columns of Z) accumulate apart from the rest (the SSM columns), and the
@@ -120,6 +124,12 @@ struct ScanDesc {
   // Final state: when set, h_out [batch, d_inner, d_state] fp32 receives each sequence's
   // state after its last row (what the next row of a generation step starts from).
   float* h_out = nullptr;
+  // Start row: rows [t0, T) of each sequence are scanned (rows below t0 are neither read
+  // nor written), from the state h0 [d_inner, d_state] fp32 of sequence b at
+  // h0 + b * h0_bstride (h0_bstride 0: one state for every sequence); h0 NULL = zeros.
+  int t0 = 0;
+  const float* h0 = nullptr;
+  long long h0_bstride = 0;
 };
 cudaError_t launch_scan(const ScanDesc& s, cudaStream_t st);
 // The tensor-core form of the scan (bf16, d_state = 16, 16-byte aligned operands);
@@ -137,6 +147,7 @@ struct AttnDesc {
   bool bf16;
   unsigned* status;
   long long kv_rows = 0;  // rows per sequence in the K/V buffers (0: T; a cache may hold more)
+  int q_row0 = 0;         // query rows below q_row0 need no output (their 128-row tiles are skipped)
 };
 cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st);
 
@@ -163,11 +174,22 @@ struct ScanStepDesc {
   void* y; long long y_ld;
   int batch, d_inner, d_state;
   bool bf16;
+  const float* d_skip = nullptr;   // [Di]: y += D x before the gate, or nullptr
 };
 cudaError_t launch_scan_step(const ScanStepDesc& s, cudaStream_t st);
 
+// z = [beta1 rms(z_a) || s2 beta2 rms(z_s)] in place (s2 = -1: difference fusion).
 cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, long long rows, int w_attn,
-                               int w_ssm, float eps, bool bf16, cudaStream_t st);
+                               int w_ssm, float eps, bool bf16, cudaStream_t st, float s2 = 1.f);
+// The same per group of `group` (64, 128 or 256) features of each branch.
+cudaError_t launch_group_norm(void* z, long long rows, int wa, int ws, int group, const float* beta1,
+                              const float* beta2, float s2, float eps, bool bf16, cudaStream_t st);
+// y = SiLU(bias + causal depthwise conv of width K of x) over [batch, Tseq, Di] rows.
+cudaError_t launch_conv_silu(const void* x, const void* w, const float* bias, void* y, int batch, int Tseq, int Di,
+                             int K, bool bf16, cudaStream_t st);
+// z[r, c] += gate[r, c] * D[c] * x[r, c] for the SSM columns z (row stride z_ld).
+cudaError_t launch_ssm_skip(void* z, long long z_ld, const void* gate, const void* x, const float* D, long long rows,
+                            int Di, bool bf16, cudaStream_t st);
 cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float eps, bool bf16,
                            cudaStream_t st);
 // Pre-norm of a residual stream kept in fp32: y = bf16(gain * x / sqrt(mean(x^2) + eps)) per
@@ -180,6 +202,10 @@ cudaError_t launch_prenorm_f32_out_f32(const float* x, const float* gain, float*
 // h[b, t, :] = float([meta; x_b][t, :]) for a bf16 stack input (h fp32 [batch, L + M, d]).
 cudaError_t launch_prepend_f32(const void* x, const void* meta, float* h, int batch, int L, int M, int d,
                                cudaStream_t st);
+// dst + b * dst_stride = src for b in [0, batch): one block of `bytes` (a multiple of 16,
+// 16-byte aligned addresses and stride) copied to every sequence.
+cudaError_t launch_broadcast(const void* src, size_t bytes, void* dst, size_t dst_stride, int batch,
+                             cudaStream_t st);
 // dst[c, r] = src[r, c] for a bf16 matrix src [rows, cols] with row stride src_ld.
 cudaError_t launch_transpose_bf16(const void* src, long long src_ld, void* dst, int rows, int cols,
                                   cudaStream_t st);
@@ -188,7 +214,7 @@ cudaError_t launch_transpose_bf16(const void* src, long long src_ld, void* dst, 
 // beta2[k - w_attn]) for a [N, w_attn + w_ssm] weight.
 cudaError_t launch_row_ssq(const void* z, long long rows, int w_attn, int w_ssm, float2* ssq, cudaStream_t st);
 cudaError_t launch_scale_cols(const void* w, void* w_out, int N, int w_attn, int w_ssm, const float* beta1,
-                              const float* beta2, cudaStream_t st);
+                              const float* beta2, cudaStream_t st, float s2 = 1.f);
 
 int num_sms();
 

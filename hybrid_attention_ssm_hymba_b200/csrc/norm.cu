@@ -98,7 +98,8 @@ __device__ __forceinline__ void scale_row(const T* src, T* dst, int w, float r, 
 
 template <typename T>
 __global__ void __launch_bounds__(NT) branch_norm_kernel(T* z, const float* __restrict__ beta1,
-                                                         const float* __restrict__ beta2, int wa, int ws, float eps) {
+                                                         const float* __restrict__ beta2, int wa, int ws, float eps,
+                                                         float s2) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[NT / 32 + 1];
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(NT) branch_norm_kernel(T* z, const float* __re
   const float ss = block_sum(sumsq(row + wa, ws), red);
   const float ra = rsqrtf(sa / wa + eps), rs = rsqrtf(ss / ws + eps);
   scale_row(row, row, wa, ra, beta1);
-  scale_row(row + wa, row + wa, ws, rs, beta2);
+  scale_row(row + wa, row + wa, ws, rs * s2, beta2);
 }
 
 template <typename T>
@@ -128,7 +129,7 @@ template <int MAXV>
 __global__ void __launch_bounds__(256) rownorm_warp_kernel(const __nv_bfloat16* x,  // x and y may alias
                                                            __nv_bfloat16* y, long long rows, int wa,
                                                            int ws, const float* __restrict__ beta1,
-                                                           const float* __restrict__ beta2, float eps) {
+                                                           const float* __restrict__ beta2, float eps, float s2) {
   pdl_trigger();
   pdl_wait();
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -168,7 +169,7 @@ __global__ void __launch_bounds__(256) rownorm_warp_kernel(const __nv_bfloat16* 
     if (vi < nv) {
       const int col = vi * 8;
       const bool first = col < wa;
-      const float r = first ? ra : rs;
+      const float r = first ? ra : rs * s2;
       const float* beta = first ? beta1 + col : (beta2 ? beta2 + (col - wa) : nullptr);
       const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
       float f[8];
@@ -189,21 +190,21 @@ __global__ void __launch_bounds__(256) rownorm_warp_kernel(const __nv_bfloat16* 
 
 template <int MAXV>
 void launch_rownorm(const void* x, void* y, long long rows, int wa, int ws, const float* b1, const float* b2,
-                    float eps, cudaStream_t st) {
+                    float eps, float s2, cudaStream_t st) {
   launch(rownorm_warp_kernel<MAXV>, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, st,
-         static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), rows, wa, ws, b1, b2, eps);
+         static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), rows, wa, ws, b1, b2, eps, s2);
 }
 
 // picks the smallest register footprint that holds a row; false if the row is too wide
 bool rownorm_bf16(const void* x, void* y, long long rows, int wa, int ws, const float* b1, const float* b2, float eps,
-                  cudaStream_t st) {
+                  cudaStream_t st, float s2 = 1.f) {
   const int nv = (wa + ws) / 8;
   const int per_lane = (nv + 31) / 32;
-  if (per_lane <= 4) launch_rownorm<4>(x, y, rows, wa, ws, b1, b2, eps, st);
-  else if (per_lane <= 8) launch_rownorm<8>(x, y, rows, wa, ws, b1, b2, eps, st);
-  else if (per_lane <= 12) launch_rownorm<12>(x, y, rows, wa, ws, b1, b2, eps, st);
-  else if (per_lane <= 16) launch_rownorm<16>(x, y, rows, wa, ws, b1, b2, eps, st);
-  else if (per_lane <= 24) launch_rownorm<24>(x, y, rows, wa, ws, b1, b2, eps, st);
+  if (per_lane <= 4) launch_rownorm<4>(x, y, rows, wa, ws, b1, b2, eps, s2, st);
+  else if (per_lane <= 8) launch_rownorm<8>(x, y, rows, wa, ws, b1, b2, eps, s2, st);
+  else if (per_lane <= 12) launch_rownorm<12>(x, y, rows, wa, ws, b1, b2, eps, s2, st);
+  else if (per_lane <= 16) launch_rownorm<16>(x, y, rows, wa, ws, b1, b2, eps, s2, st);
+  else if (per_lane <= 24) launch_rownorm<24>(x, y, rows, wa, ws, b1, b2, eps, s2, st);
   else return false;
   return true;
 }
@@ -250,14 +251,17 @@ __global__ void __launch_bounds__(256) row_ssq_kernel(const __nv_bfloat16* __res
 __global__ void __launch_bounds__(256) scale_cols_kernel(const uint4* __restrict__ w, uint4* __restrict__ w_out,
                                                          long long n_vec, int row_vecs, int wa,
                                                          const float* __restrict__ beta1,
-                                                         const float* __restrict__ beta2) {
+                                                         const float* __restrict__ beta2, float s2) {
   pdl_trigger();
   pdl_wait();
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n_vec;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int k0 = static_cast<int>(i % row_vecs) * 8;
     const float* bb = k0 < wa ? beta1 + k0 : beta2 + (k0 - wa);
-    const float4 b0 = __ldg(reinterpret_cast<const float4*>(bb)), b1 = __ldg(reinterpret_cast<const float4*>(bb + 4));
+    const float sg = k0 < wa ? 1.f : s2;
+    float4 b0 = __ldg(reinterpret_cast<const float4*>(bb)), b1 = __ldg(reinterpret_cast<const float4*>(bb + 4));
+    b0 = make_float4(b0.x * sg, b0.y * sg, b0.z * sg, b0.w * sg);
+    b1 = make_float4(b1.x * sg, b1.y * sg, b1.z * sg, b1.w * sg);
     const uint4 q = w[i];
     w_out[i] = make_uint4(pack_bf16(bf16lo(q.x) * b0.x, bf16hi(q.x) * b0.y), pack_bf16(bf16lo(q.y) * b0.z, bf16hi(q.y) * b0.w),
                           pack_bf16(bf16lo(q.z) * b1.x, bf16hi(q.z) * b1.y), pack_bf16(bf16lo(q.w) * b1.z, bf16hi(q.w) * b1.w));
@@ -281,25 +285,25 @@ cudaError_t launch_row_ssq(const void* z, long long rows, int w_attn, int w_ssm,
 }
 
 cudaError_t launch_scale_cols(const void* w, void* w_out, int N, int w_attn, int w_ssm, const float* beta1,
-                              const float* beta2, cudaStream_t st) {
+                              const float* beta2, cudaStream_t st, float s2) {
   const int row_vecs = (w_attn + w_ssm) / 8;
   const long long n_vec = static_cast<long long>(N) * row_vecs;
   if (n_vec <= 0) return cudaSuccess;
   const long long blocks = (n_vec + 255) / 256;
   return launch(scale_cols_kernel, dim3(static_cast<unsigned>(blocks < 4 * num_sms() ? blocks : 4 * num_sms())),
                 dim3(256), 0, st, static_cast<const uint4*>(w), static_cast<uint4*>(w_out), n_vec, row_vecs, w_attn,
-                beta1, beta2);
+                beta1, beta2, s2);
 }
 
 cudaError_t launch_branch_norm(void* z, const float* beta1, const float* beta2, long long rows, int w_attn, int w_ssm,
-                               float eps, bool bf16, cudaStream_t st) {
+                               float eps, bool bf16, cudaStream_t st, float s2) {
   if (rows <= 0) return cudaSuccess;
-  if (bf16 && rownorm_bf16(z, z, rows, w_attn, w_ssm, beta1, beta2, eps, st)) return cudaGetLastError();
+  if (bf16 && rownorm_bf16(z, z, rows, w_attn, w_ssm, beta1, beta2, eps, st, s2)) return cudaGetLastError();
   if (bf16)
     return launch(branch_norm_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(rows)), dim3(NT), 0, st,
-                  static_cast<__nv_bfloat16*>(z), beta1, beta2, w_attn, w_ssm, eps);
+                  static_cast<__nv_bfloat16*>(z), beta1, beta2, w_attn, w_ssm, eps, s2);
   return launch(branch_norm_kernel<float>, dim3(static_cast<unsigned>(rows)), dim3(NT), 0, st, static_cast<float*>(z),
-                beta1, beta2, w_attn, w_ssm, eps);
+                beta1, beta2, w_attn, w_ssm, eps, s2);
 }
 
 cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float eps, bool bf16, cudaStream_t st) {
@@ -404,7 +408,32 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16
   }
 }
 
+// dst + b * stride = src (16-byte units), grid-stride over batch x units.
+__global__ void __launch_bounds__(256) broadcast_kernel(const uint4* __restrict__ src, long long units,
+                                                        uint8_t* __restrict__ dst, long long stride, int batch) {
+  pdl_trigger();
+  pdl_wait();
+  const long long total = units * batch;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long b = i / units, u = i - b * units;
+    reinterpret_cast<uint4*>(dst + b * stride)[u] = src[u];
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_broadcast(const void* src, size_t bytes, void* dst, size_t dst_stride, int batch,
+                             cudaStream_t st) {
+  if (bytes == 0 || batch <= 0) return cudaSuccess;
+  if (bytes % 16 || dst_stride % 16 || (reinterpret_cast<uintptr_t>(src) & 15) || (reinterpret_cast<uintptr_t>(dst) & 15))
+    return cudaErrorInvalidValue;
+  const long long units = static_cast<long long>(bytes / 16), total = units * batch;
+  const long long blocks = (total + 255) / 256;
+  return launch(broadcast_kernel, dim3(static_cast<unsigned>(blocks < 4 * num_sms() ? blocks : 4 * num_sms())),
+                dim3(256), 0, st, static_cast<const uint4*>(src), units, static_cast<uint8_t*>(dst),
+                static_cast<long long>(dst_stride), batch);
+}
 
 cudaError_t launch_prenorm_f32(const float* x, const float* gain, void* y, void* y_lo, long long rows, int d,
                                float eps, cudaStream_t st) {

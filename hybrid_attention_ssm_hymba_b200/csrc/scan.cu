@@ -48,7 +48,15 @@ struct ScanParams {
   long long y_ld;
   int T, Di, N;
   float* h_out;  // [batch, Di, N] state after the last row, or nullptr
+  int t0;                 // first row scanned
+  const float* h0;        // [Di, N] state entering row t0 (sequence b at h0 + b * h0_bstride), or nullptr
+  long long h0_bstride;
 };
+
+// The state entering row t0 for NS components [n0, n0 + NS) of channel c of sequence b.
+HY_DEV void load_h0(const ScanParams& p, int b, int c, int n0, int NS, float* h) {
+  for (int n = 0; n < NS; ++n) h[n] = p.h0 ? p.h0[b * p.h0_bstride + static_cast<long long>(c) * p.N + n0 + n] : 0.f;
+}
 
 template <typename TI, int NS, int TPC, int NWT>
 __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
@@ -67,8 +75,8 @@ __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
   const int b = blockIdx.y;
   const bool valid = c < p.Di;
   const int cc = valid ? c : 0;
-  const int Lc = (p.T + NWT - 1) / NWT;
-  const int t0 = min(p.T, warp * Lc), t1 = min(p.T, t0 + Lc);
+  const int Lc = (p.T - p.t0 + NWT - 1) / NWT;
+  const int t0 = min(p.T, p.t0 + warp * Lc), t1 = min(p.T, t0 + Lc);
   const int n0 = slice * NS;
   const long long row0 = static_cast<long long>(b) * p.T + t0;
 
@@ -138,9 +146,13 @@ __global__ void __launch_bounds__(32 * NWT) scan_kernel(const ScanParams p) {
   if (slice == 0) s_logdec[warp * CPW + ch] = logdec;
   __syncthreads();
 
-  // ---------------- combine: state entering this warp's chunk
+  // ---------------- combine: state entering this warp's chunk (from the state entering row t0)
+  {
+    float hz[NS];
+    load_h0(p, b, cc, n0, NS, hz);
 #pragma unroll
-  for (int i = 0; i < NP; ++i) h[i] = make_float2(0.f, 0.f);
+    for (int i = 0; i < NP; ++i) h[i] = make_float2(hz[2 * i], hz[2 * i + 1]);
+  }
   for (int k = 0; k < warp; ++k) {
     const float dec = ex2_approx(s_logdec[k * CPW + ch]);
     const float2 dec2 = make_float2(dec, dec);
@@ -318,7 +330,7 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
   const int grp = warp / sp.S, chunk = warp % sp.S;
   const int wcol = (blockIdx.x * sp.G + grp) * CPW;  // first channel of this warp
   const bool active = wcol < p.Di;                   // inactive warps still meet the CTA barriers
-  const int n_tiles = (p.T + C::ROWS - 1) / C::ROWS;
+  const int n_tiles = (p.T - p.t0 + C::ROWS - 1) / C::ROWS;   // tiles of rows [t0, T)
   const int k_begin = min(n_tiles, chunk * sp.ctiles), k_end = min(n_tiles, k_begin + sp.ctiles);
 
   uint8_t* wsm = smem_raw + warp * C::WARP_B;
@@ -340,7 +352,7 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
     const int slot = issued % C::STAGES;
     uint8_t* st = wsm + slot * C::STAGE_B;
     mbar_arrive_expect_tx(&full[slot], (with_gate ? 3 : 2) * C::XB + C::BCB);
-    const int t = k * C::ROWS;
+    const int t = p.t0 + k * C::ROWS;
     tma_load_3d(st, &tmX, &full[slot], wcol, t, b);
     tma_load_3d(st + C::XB, &tmDT, &full[slot], wcol, t, b);
     if (with_gate) tma_load_3d(st + 2 * C::XB, &tmG, &full[slot], wcol, t, b);
@@ -373,6 +385,22 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
     ncl[q] = 0.f;
   }
   const bool ywriter = slice == 0;
+  // the state entering row t0: the entry state of a single chunk, or the start of the
+  // chunk combine below
+  float2 g0[CPL][NP];
+#pragma unroll
+  for (int q = 0; q < CPL; ++q) {
+    float hz[NS];
+    load_h0(p, b, (active && c0 + q < p.Di) ? c0 + q : 0, n0, NS, hz);
+#pragma unroll
+    for (int i = 0; i < NP; ++i) g0[q][i] = make_float2(hz[2 * i], hz[2 * i + 1]);
+  }
+  if (sp.S == 1) {
+#pragma unroll
+    for (int q = 0; q < CPL; ++q)
+#pragma unroll
+      for (int i = 0; i < NP; ++i) g[q][i] = g0[q][i];
+  }
 
   auto load_b = [&](uint32_t row_addr, float4 (&bq)[NQ]) {
 #pragma unroll
@@ -558,7 +586,7 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
 #pragma unroll
     for (int q = 0; q < CPL; ++q) {
 #pragma unroll
-      for (int i = 0; i < NP; ++i) g[q][i] = make_float2(0.f, 0.f);
+      for (int i = 0; i < NP; ++i) g[q][i] = g0[q][i];
       ncl[q] = 0.f;
     }
     for (int j = 0; j < chunk; ++j) {  // c_{j+1} = D_j c_j + h_end_j
@@ -692,7 +720,7 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
       __syncwarp();
       if (lane == 0) {
         if (k + C::STAGES < k_end) issue(k + C::STAGES, true);
-        tma_store_3d(&tmY, yt, wcol, k * C::ROWS, b);
+        tma_store_3d(&tmY, yt, wcol, p.t0 + k * C::ROWS, b);
         bulk_commit();
       }
     }
@@ -743,10 +771,9 @@ __global__ void __launch_bounds__(128) scan_ps_kernel(const ScanParams p) {
   const int n0 = slice * NS;
   float A2[NS], h[NS];
 #pragma unroll
-  for (int n = 0; n < NS; ++n) {
-    A2[n] = -expf(p.a_log[static_cast<long long>(cc) * N + n0 + n]) * 1.4426950408889634f;
-    h[n] = 0.f;
-  }
+  load_h0(p, b, cc, n0, NS, h);
+#pragma unroll
+  for (int n = 0; n < NS; ++n) A2[n] = -expf(p.a_log[static_cast<long long>(cc) * N + n0 + n]) * 1.4426950408889634f;
   const long long row0 = static_cast<long long>(b) * p.T;
   const TI* xp = static_cast<const TI*>(p.x) + row0 * p.Di + cc;
   const TI* dp = static_cast<const TI*>(p.dt) + row0 * p.Di + cc;
@@ -754,7 +781,7 @@ __global__ void __launch_bounds__(128) scan_ps_kernel(const ScanParams p) {
   const float* bp = p.bc + row0 * 2 * N + n0;
   TI* yp = static_cast<TI*>(p.y) + row0 * p.y_ld + cc;
 #pragma unroll 1
-  for (int t = 0; t < p.T; ++t) {
+  for (int t = p.t0; t < p.T; ++t) {
     const float d = to_f<TI>(dp[static_cast<long long>(t) * p.Di]);
     const float u = d * to_f<TI>(xp[static_cast<long long>(t) * p.Di]);
     const float* brow = bp + static_cast<long long>(t) * 2 * N;
@@ -786,7 +813,8 @@ template <typename TI, int N>
 cudaError_t launch_ps(const ScanDesc& s, cudaStream_t st) {
   constexpr int NS = N < 8 ? N : 8;
   constexpr int CPB = 4 * (32 / (N / NS));  // channels per block
-  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state, s.h_out};
+  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state, s.h_out, s.t0, s.h0,
+               s.h0_bstride};
   dim3 grid((s.d_inner + CPB - 1) / CPB, s.batch);
   return launch(scan_ps_kernel<TI, N>, grid, dim3(128), 0, st, p);
 }
@@ -847,7 +875,7 @@ cudaError_t launch_w(const ScanDesc& s, cudaStream_t st) {
       !map3d(&ty, s.y, f32, s.batch, s.T, s.d_inner, s.y_ld, C::CPW, C::ROWS))
     return cudaErrorInvalidValue;
   const int groups = (s.d_inner + C::CPW - 1) / C::CPW;
-  const int n_tiles = (s.T + C::ROWS - 1) / C::ROWS;
+  const int n_tiles = (s.T - s.t0 + C::ROWS - 1) / C::ROWS;
   const int max_warps = (227 * 1024 - 128) / C::WARP_B < C::MAX_WARPS ? (227 * 1024 - 128) / C::WARP_B : C::MAX_WARPS;
   static std::atomic<uint64_t> attr_done{0};
   if (cudaError_t e = smem_attr_once(scan_w_kernel<TI, N, TPC, CPL>, max_warps * C::WARP_B + 128, attr_done))
@@ -869,7 +897,8 @@ cudaError_t launch_w(const ScanDesc& s, cudaStream_t st) {
   }
   const int warps = sp.G * sp.S;
   const int smem = warps * C::WARP_B + 128;
-  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state, s.h_out};
+  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state, s.h_out, s.t0, s.h0,
+               s.h0_bstride};
   dim3 grid((groups + sp.G - 1) / sp.G, s.batch);
   return launch(scan_w_kernel<TI, N, TPC, CPL>, grid, dim3(32 * warps), smem, st, tx, td, tg, tb, ty, p, sp, s.status);
 }
@@ -877,7 +906,8 @@ cudaError_t launch_w(const ScanDesc& s, cudaStream_t st) {
 template <typename TI, int NS, int TPC, int NWT>
 cudaError_t launch_one(const ScanDesc& s, cudaStream_t st) {
   constexpr int CPW = 32 / TPC;
-  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state, s.h_out};
+  ScanParams p{s.x, s.dt, s.bc, s.gate, s.a_log, s.y, s.y_ld, s.T, s.d_inner, s.d_state, s.h_out, s.t0, s.h0,
+               s.h0_bstride};
   dim3 grid((s.d_inner + CPW - 1) / CPW, s.batch);
   return launch(scan_kernel<TI, NS, TPC, NWT>, grid, dim3(32 * NWT), 0, st, p);
 }

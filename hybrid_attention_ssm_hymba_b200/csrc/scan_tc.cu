@@ -123,7 +123,8 @@ __global__ void __launch_bounds__(NTHR, 1)
                    const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmBC,
                    const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmWD,
                    const float* __restrict__ a_log, const float* __restrict__ b_dt, int T, int Di,
-                   float* __restrict__ h_out, unsigned* status) {
+                   float* __restrict__ h_out, int t0, const float* __restrict__ h0, long long h0_bstride,
+                   unsigned* status) {
   using L = Lay<FUSED>;
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(NTHR, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c0 = blockIdx.x * CH, b = blockIdx.y;
-  const int nblk = (T + Q - 1) / Q;
+  const int nblk = (T - t0 + Q - 1) / Q;   // blocks of rows [t0, T)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -193,10 +194,10 @@ __global__ void __launch_bounds__(NTHR, 1)
         if (k >= STAGES && !mbar_wait(&empty[s], ((k / STAGES) - 1) & 1u, status, abort_flag)) break;
         mbar_arrive_expect_tx(&full[s], 2 * TILE_B + L::D_B + BC_B + (FUSED && k == 0 ? WD_B : 0));
         if (FUSED && k == 0) tma_load_2d(sm + L::OFF_WD, &tmWD, &full[s], 0, c0);
-        tma_load_3d(sm + L::OFF_X + s * TILE_B, &tmX, &full[s], c0, k * Q, b);
-        tma_load_3d(sm + L::OFF_D + s * L::D_B, &tmD, &full[s], FUSED ? 0 : c0, k * Q, b);
-        tma_load_3d(sm + L::OFF_G + s * TILE_B, &tmG, &full[s], c0, k * Q, b);
-        tma_load_3d(sm + L::OFF_BC + s * BC_B, &tmBC, &full[s], 0, k * Q, b);
+        tma_load_3d(sm + L::OFF_X + s * TILE_B, &tmX, &full[s], c0, t0 + k * Q, b);
+        tma_load_3d(sm + L::OFF_D + s * L::D_B, &tmD, &full[s], FUSED ? 0 : c0, t0 + k * Q, b);
+        tma_load_3d(sm + L::OFF_G + s * TILE_B, &tmG, &full[s], c0, t0 + k * Q, b);
+        tma_load_3d(sm + L::OFF_BC + s * BC_B, &tmBC, &full[s], 0, t0 + k * Q, b);
       }
       if (k < nblk) {  // aborted: let the copies already issued land before smem goes away
         int never = 0;
@@ -315,9 +316,17 @@ __global__ void __launch_bounds__(NTHR, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const float A2 = c < Di ? expf(a_log[c]) * 1.4426950408889634f : 0.f;  // |A| / ln 2
     const float bdt = FUSED && c < Di ? b_dt[c] : 0.f;
-    float h[NST];
+    float h[NST];   // the state entering the current block (half 1), from h0 at row t0
 #pragma unroll
     for (int n = 0; n < NST; ++n) h[n] = 0.f;
+    if (h0 && c < Di) {
+      const float4* hi = reinterpret_cast<const float4*>(h0 + b * h0_bstride + static_cast<long long>(c) * NST);
+#pragma unroll
+      for (int j = 0; j < NST / 4; ++j) {
+        const float4 v = hi[j];
+        h[4 * j] = v.x; h[4 * j + 1] = v.y; h[4 * j + 2] = v.z; h[4 * j + 3] = v.w;
+      }
+    }
     float pS0 = 0.f, pS1 = 0.f;  // previous block's half sums (chain)
     bool prev_any = false;
     for (int k = 0; k <= nblk; ++k) {
@@ -343,7 +352,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             for (int j = 0; j < 32; ++j) z[j] = 0u;
           }
           // steps past T (zero-filled dt_low) get dt = 0, so they leave the state alone
-          const int t_end = T - (k * Q + 32 * half);
+          const int t_end = T - (t0 + k * Q + 32 * half);
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
             float2 d = softplus2(make_float2(__uint_as_float(z[j]) + bdt, __uint_as_float(z[j + 1]) + bdt));
@@ -496,7 +505,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         fence_proxy_async_smem();
         if (bar_red_or(1, NCHT, fail || *abort_flag)) break;
         if (threadIdx.x == 0) {
-          tma_store_3d(&tmY, sm + L::OFF_Y + i * TILE_B, c0, jb * Q, b);
+          tma_store_3d(&tmY, sm + L::OFF_Y + i * TILE_B, c0, t0 + jb * Q, b);
           bulk_commit();
           bulk_wait_read1();  // the store before it has read its tile: that tile may be rewritten
         }
@@ -601,7 +610,7 @@ cudaError_t launch_tc(const ScanDesc& s, cudaStream_t st) {
   if (cudaError_t e = smem_attr_once(scan_tc_kernel<FUSED>, L::SMEM_TOTAL, attr_done)) return e;
   dim3 grid((s.d_inner + CH - 1) / CH, s.batch);
   return launch(scan_tc_kernel<FUSED>, grid, dim3(NTHR), L::SMEM_TOTAL, st, tx, td, tg, tb, ty, tw, s.a_log, s.b_dt,
-                s.T, s.d_inner, s.h_out, s.status);
+                s.T, s.d_inner, s.h_out, s.t0, s.h0, s.h0_bstride, s.status);
 }
 
 }  // namespace

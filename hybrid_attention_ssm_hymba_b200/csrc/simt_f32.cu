@@ -27,6 +27,7 @@ struct F32GemmParams {
   float* out;
   long long out_ld;
   int swiglu_F;
+  int remap_L, remap_T, remap_M;   // segment rows: r -> (r / L) T + M + r % L when remap_L > 0
 };
 
 __device__ __forceinline__ const float* a_row(const F32GemmParams& p, long long r) {
@@ -110,7 +111,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const __grid_constant__ F
         if (p.epi == EPI_RESIDUAL)
           p.out[row * p.out_ld + col] = p.resid[row * p.resid_ld + col] + acc[i][j];
         else
-          store_elem(p, row, col, acc[i][j]);
+          store_elem(p, p.remap_L ? (row / p.remap_L) * p.remap_T + p.remap_M + row % p.remap_L : row, col,
+                     acc[i][j]);
       }
     }
   }
@@ -196,6 +198,9 @@ cudaError_t launch_gemm_f32(const GemmDesc& g, cudaStream_t st) {
   p.out = static_cast<float*>(g.out);
   p.out_ld = g.out_ld;
   p.swiglu_F = g.swiglu_F;
+  p.remap_L = g.remap_L;
+  p.remap_T = g.remap_T;
+  p.remap_M = g.remap_M;
   if (p.rows <= 0) return cudaSuccess;
   const int ncols = g.epi == EPI_SWIGLU ? g.swiglu_F : g.N;
   dim3 grid((ncols + TB - 1) / TB, static_cast<unsigned>((p.rows + TB - 1) / TB));

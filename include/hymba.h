@@ -85,6 +85,14 @@ typedef struct {
   int ffn_dim;      /* F: SwiGLU FFN width for hymba_stack_fwd; 0 = no FFN */
   float rms_eps;    /* RMSNorm epsilon (1e-6) */
   hymba_dtype_t dtype;
+  /* Options beyond the pages' formula (0 = off; the five workloads use none):           */
+  int conv_width;   /* 1..4: Mamba's causal depthwise conv + SiLU on X_ssm before x_proj
+                       and the scan (weights w_conv, b_conv); prefill/decode and the
+                       meta-prefix calls return HYMBA_ERR_UNSUPPORTED with it */
+  int norm_group;   /* 64, 128 or 256: the branch norm per group of this many features
+                       (per head); 0 = over each branch's full width */
+  int fusion;       /* 0: out = W_out,a(b1 n(Y_a)) + W_out,s(b2 n(Y_s)); 1: difference, the SSM
+                       branch subtracted (the intra-layer hybrid study, gist.science page) */
 } hymba_cfg_t;
 
 /* Weights of one layer; device pointers, nn.Linear layout [out_features, in_features]. */
@@ -103,6 +111,9 @@ typedef struct {
   const float* norm1;     /* [d] fp32 gain of the block's pre-norm before the mixer (stack only);
                              NULL = unit gain; ignored by the single-layer entry points */
   const float* norm2;     /* [d] fp32 gain of the pre-norm before the FFN (stack only); NULL = unit gain */
+  const void* w_conv;     /* [Di, conv_width] dtype: the causal conv taps (tap conv_width-1 = current row) */
+  const float* b_conv;    /* [Di] fp32 conv bias (required with conv_width) */
+  const float* d_skip;    /* [Di] fp32: Mamba's D, Y_ssm = gate * (y + D x); NULL = no skip */
 } hymba_weights_t;
 
 /* Human-readable name of a status code (static string). */
@@ -251,6 +262,45 @@ HYMBA_API hymba_status_t hymba_layer_prefill(const void* x, const void* meta, co
 HYMBA_API hymba_status_t hymba_layer_decode(const void* x_t, const hymba_weights_t* w, const hymba_cfg_t* cfg,
                                   void* kv_cache, int cache_rows, int pos, float* ssm_state,
                                   void* out_t, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------- meta-prefix precompute ----------------
+ * The meta tokens are the same learned rows in front of every sequence (the review,
+ * "Meta Tokens"; the networkstorageforum page, "Key Components of Hymba": a learned
+ * initialisation of the caches).  Under the causal mask a meta row sees only meta rows,
+ * so everything the layer computes for them -- their K/V, the SSM state after them, their
+ * output rows -- is the same for every sequence and every call with the same weights.
+ * hymba_meta_prefix computes that once into a record; hymba_layer_fwd_prefixed then runs
+ * only the user rows.
+ *
+ * Record (caller-owned device memory of hymba_meta_prefix_size(cfg) bytes, 256-byte
+ * aligned): the M meta rows' outputs [M, d] (dtype), their K then V [2, M, Hkv*dh]
+ * (dtype; absent for a HYMBA_KV_CONSUME layer), the SSM state after them [Di, N] fp32.
+ */
+HYMBA_API size_t hymba_meta_prefix_size(const hymba_cfg_t* cfg);  /* 0 if cfg invalid or n_meta = 0 */
+
+/*
+ * Fills `prefix` for the layer of `cfg` (n_meta >= 1; batch and seq_len are not used).
+ *   meta_in       [M, d] dtype: the layer's input meta rows -- the meta tokens for the first
+ *                 layer, or the previous layer's prefix output rows (the first M rows of the
+ *                 record) for a layer that takes another layer's output
+ *   kv_prefix_in  the producer's record, for a HYMBA_KV_CONSUME layer; else NULL
+ *   workspace     >= hymba_workspace_size(cfg) bytes (the full layer's; 256-byte aligned)
+ */
+HYMBA_API hymba_status_t hymba_meta_prefix(const void* meta_in, const hymba_weights_t* w, const hymba_cfg_t* cfg,
+                                 const void* kv_prefix_in, void* prefix, void* workspace, size_t ws_bytes,
+                                 void* stream);
+
+/*
+ * hymba_layer_fwd with the meta rows taken from a record of hymba_meta_prefix: x holds
+ * the user rows only, [B, L, d]; the input projection, attention queries and scan run on
+ * rows [M, T) of each sequence (the scan from the record's state), the meta rows' K/V are
+ * copied into each sequence's K/V (kv_out for a producing layer), and out [B, T, d]
+ * receives the record's meta rows and the computed user rows.  Other arguments as in
+ * hymba_layer_fwd (kv_in for a consuming layer: the producer's kv_out of its prefixed call).
+ */
+HYMBA_API hymba_status_t hymba_layer_fwd_prefixed(const void* x, const void* prefix, const hymba_weights_t* w,
+                                        const hymba_cfg_t* cfg, const void* kv_in, void* kv_out, void* out,
+                                        void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Check of the failure-detection path (no counterpart in the pages).  Every kernel of this

@@ -57,6 +57,11 @@ def _cfg(**kw):
     (dict(a_per_state=2), H.HYMBA_ERR_INVALID_ARG),
     (dict(dt_rank=40), H.HYMBA_ERR_UNSUPPORTED),
     (dict(dtype=7), H.HYMBA_ERR_INVALID_ARG),
+    (dict(conv_width=5), H.HYMBA_ERR_INVALID_ARG),
+    (dict(conv_width=-1), H.HYMBA_ERR_INVALID_ARG),
+    (dict(fusion=2), H.HYMBA_ERR_INVALID_ARG),
+    (dict(norm_group=96), H.HYMBA_ERR_UNSUPPORTED),
+    (dict(norm_group=512), H.HYMBA_ERR_UNSUPPORTED),
 ])
 def test_layer_validation_rejects_before_launch(kw, expect):
     """Bad configs return their status without any CUDA call (this runs on a CPU machine)."""
@@ -161,3 +166,29 @@ def test_per_state_decay_layer_is_accepted():
     c = H.make_cfg(dataclasses.replace(synth.workload("hymba350m_layer").first, a_per_state=1))
     assert H.hymba_workspace_size(c) > 0
     assert not H.hymba_layer_fuses_dt_proj(c)
+
+
+def test_generation_and_prefix_entry_points_validate_on_the_host():
+    """Bad arguments of the generation and meta-prefix calls return before any CUDA call."""
+    c = _cfg()
+    full = H.make_weights({k: 1 << 20 for k in ("w_in", "w_x", "w_dt", "w_out", "a_log", "b_dt", "beta1", "beta2")})
+    P = 1 << 20
+    need = H.hymba_decode_workspace_size(c)
+    assert need >= H.hymba_workspace_size(c) > 0
+    # cache smaller than the prompt; pos outside the cache; missing state
+    assert H.load().hymba_layer_prefill(P, P, full, c, P, c.seq_len, P, P, P, need, None) == H.HYMBA_ERR_INVALID_ARG
+    T = c.seq_len + c.n_meta
+    assert H.load().hymba_layer_decode(P, full, c, P, T, T, P, P, P, need, None) == H.HYMBA_ERR_INVALID_ARG
+    assert H.load().hymba_layer_decode(P, full, c, P, T, -1, P, P, P, need, None) == H.HYMBA_ERR_INVALID_ARG
+    assert H.load().hymba_layer_decode(P, full, c, P, T + 1, T, None, P, P, need, None) == H.HYMBA_ERR_INVALID_ARG
+    assert H.load().hymba_layer_decode(P, full, c, P, T + 1, T, P, P, P, need - 1, None) == H.HYMBA_ERR_WORKSPACE
+    # more than 8 query heads per KV head, or a head_dim that is not a multiple of 32: unsupported
+    assert H.hymba_decode_workspace_size(_cfg(n_q_heads=16, n_kv_heads=1)) == 0
+    # meta prefix: needs meta rows; record and workspace checked
+    assert H.hymba_meta_prefix_size(_cfg(n_meta=0)) == 0
+    rec = H.hymba_meta_prefix_size(c)
+    assert rec > 0 and rec % 256 == 0
+    assert H.load().hymba_meta_prefix(P, full, c, None, P + 8, P, 1 << 40, None) == H.HYMBA_ERR_INVALID_ARG
+    assert H.load().hymba_meta_prefix(P, full, _cfg(kv_mode=H.HYMBA_KV_CONSUME), None, P, P, 1 << 40,
+                                      None) == H.HYMBA_ERR_INVALID_ARG
+    assert H.load().hymba_layer_fwd_prefixed(P, P, full, c, None, None, P, P, 16, None) == H.HYMBA_ERR_WORKSPACE

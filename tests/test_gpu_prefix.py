@@ -1,0 +1,101 @@
+"""Meta-prefix precompute on the GPU through the C ABI.
+
+hymba_meta_prefix computes what the layer does for the M meta rows -- identical for every
+sequence under the causal mask -- once into a record; hymba_layer_fwd_prefixed then runs
+only the user rows.  Checked: with d_state 16 and M a multiple of the scan's 64-row block
+the prefixed layer is bit-identical to hymba_layer_fwd (the same kernels see the same
+values in the same order); a KV-sharing pair with SWA and d_state 128 (the consumer's
+record built from the producer's) and the fp32 path match the oracle."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import hybrid_attention_ssm_hymba_b200 as H
+import oracle as O
+from hybrid_attention_ssm_hymba_b200 import host, synth
+from gpu_util import assert_close, dev, requires_cuda, status_ok, to_np
+
+pytestmark = [pytest.mark.gpu, requires_cuda]
+
+
+def _prefixed_chain(wl, x, meta, dps):
+    """Every layer of the workload through records + prefixed calls (a pair: the consumer's
+    record from the producer's record rows and K/V)."""
+    layers = wl.layers
+    s0 = layers[0]
+    dt = s0.dtype
+    cfgs = [H.make_cfg(s) for s in layers]
+    ws = host.workspace(max(H.hymba_workspace_size(c) for c in cfgs))
+    recs = [host.workspace(H.hymba_meta_prefix_size(c)) for c in cfgs]
+    tm = dev(meta, dt)
+    meta_in = tm
+    for i, c in enumerate(cfgs):
+        H.check(H.hymba_meta_prefix(meta_in, H.make_weights(dps[i]), c, recs[0] if i > 0 else None, recs[i], ws),
+                f"prefix {i}")
+        # the next layer's meta rows are this layer's meta output rows (the record's first M rows)
+        meta_in = recs[i][:s0.n_meta * s0.d_model * (2 if dt == "bf16" else 4)].view(
+            host.torch_dtype(dt)).view(s0.n_meta, s0.d_model)
+    kv = host.empty((2, s0.batch * s0.T, s0.kv_width), dt) if len(layers) > 1 else None
+    out = host.empty((s0.batch, s0.T, s0.d_model), dt)
+    H.check(H.hymba_layer_fwd_prefixed(dev(x, dt), recs[0], H.make_weights(dps[0]), cfgs[0], None, kv, out, ws),
+            "prefixed 0")
+    outs = [out]
+    for i in range(1, len(layers)):
+        # the consumer takes the producer's user rows; its meta rows come from its record
+        o2 = host.empty((s0.batch, s0.T, s0.d_model), dt)
+        H.check(H.hymba_layer_fwd_prefixed(outs[-1][:, s0.n_meta:].contiguous(), recs[i], H.make_weights(dps[i]),
+                                           cfgs[i], kv, None, o2, ws), f"prefixed {i}")
+        outs.append(o2)
+    status_ok(ws)
+    return to_np(outs[-1])
+
+
+def _plain_chain(wl, x, meta, dps):
+    layers = wl.layers
+    s0 = layers[0]
+    dt = s0.dtype
+    cfgs = [H.make_cfg(s) for s in layers]
+    ws = host.workspace(max(H.hymba_workspace_size(c) for c in cfgs))
+    kv = host.empty((2, s0.batch * s0.T, s0.kv_width), dt) if len(layers) > 1 else None
+    out = host.empty((s0.batch, s0.T, s0.d_model), dt)
+    H.check(H.hymba_layer_fwd(dev(x, dt), dev(meta, dt), H.make_weights(dps[0]), cfgs[0], None, kv, out, ws), "0")
+    outs = [out]
+    for i in range(1, len(layers)):
+        o2 = host.empty((s0.batch, s0.T, s0.d_model), dt)
+        H.check(H.hymba_layer_fwd(outs[-1], None, H.make_weights(dps[i]), cfgs[i], kv, None, o2, ws), f"{i}")
+        outs.append(o2)
+    status_ok(ws)
+    return to_np(outs[-1])
+
+
+def _setup(wl):
+    x, meta = synth.layer_inputs(wl)
+    ps = [synth.layer_params(wl, i) for i in range(len(wl.layers))]
+    return x, meta, ps, [host.params_to_device(p, wl.first.dtype) for p in ps]
+
+
+def test_prefixed_layer_is_bit_identical_to_the_full_layer():
+    wl = synth.workload("hymba350m_layer", batch=3, seq_len=333, n_meta=128)
+    x, meta, ps, dps = _setup(wl)
+    np.testing.assert_array_equal(_prefixed_chain(wl, x, meta, dps), _plain_chain(wl, x, meta, dps))
+
+
+def test_prefixed_kv_pair_swa_dstate128_matches_oracle_and_full_path():
+    wl = synth.workload("hymba1p5b_kvpair", batch=2, seq_len=400, window=96, d_model=512, n_q_heads=8,
+                        n_kv_heads=2, d_inner=512, dt_rank=32)
+    x, meta, ps, dps = _setup(wl)
+    g = _prefixed_chain(wl, x, meta, dps)
+    full = _plain_chain(wl, x, meta, dps)
+    h, kv = O.layer_forward(x, meta, ps[0], wl.layers[0])
+    ref, _ = O.layer_forward(h, None, ps[1], wl.layers[1], kv_in=kv)
+    assert_close(g, ref, "bf16", "prefixed pair vs oracle")
+    assert_close(g, full, "bf16", "prefixed pair vs the full path", tol=2e-3)
+
+
+@pytest.mark.parametrize("a_per_state", [0, 1])
+def test_prefixed_fp32(a_per_state):
+    wl = synth.workload("tiny_fp32", batch=2, a_per_state=a_per_state)
+    x, meta, ps, dps = _setup(wl)
+    ref, _ = O.layer_forward(x, meta, ps[0], wl.first)
+    assert_close(_prefixed_chain(wl, x, meta, dps), ref, "f32", "prefixed fp32 layer")
