@@ -737,7 +737,7 @@ def run_native(args, rank, world, local_rank):
     ranks = Ranks(world, local_rank, "nccl", dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    bench = Workbench(args.workload, dev)
+    bench = Workbench(args.workload, dev, **({"batch": args.batch} if args.batch else {}))
     K = args.steps
     rec, total_ms = measure(bench, K, args.warmup, ranks, dev, flush, stages=True, e2e=not args.no_e2e)
     value = weak_scaling_rate(world, K, bench.tokens, total_ms)
@@ -817,11 +817,17 @@ def main():
     ap.add_argument("--workload", default="hymba1p5b_kvpair", choices=synth.WORKLOAD_ORDER)
     ap.add_argument("--no-per-workload", action="store_true", help="skip the other workloads' lines")
     ap.add_argument("--no-decode", action="store_true", help="skip the generation-step measurement")
+    ap.add_argument("--only-headline", action="store_true",
+                    help="the headline workload only: no other workloads, decode, options, e2e or CPU baseline "
+                         "(profiling runs)")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         print("note: fewer than 3 warm-up steps requested", file=sys.stderr)
+    if args.only_headline:
+        args.no_per_workload = args.no_decode = args.no_e2e = args.no_cpu_baseline = True
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

@@ -20,6 +20,10 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller; row-major;
  *     the library allocates no memory.  Calls are asynchronous on `stream`
  *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - Per device the library keeps a few handles it makes on first use (kernel
+ *     attributes, the second streams of hymba_layer_fwd, the address of the
+ *     hymba_layer_fwd_noalloc block); none of them survives a reset of the device or of
+ *     its primary context, so no call may follow cudaDeviceReset in the same process.
  *   - "dtype" tensors (activations and projection weights) are bf16 when
  *     cfg.dtype == HYMBA_BF16 (fp32 accumulation, fp32 scan state) and fp32
  *     when cfg.dtype == HYMBA_F32.  a_log, b_dt, beta1, beta2 are always fp32.
@@ -126,7 +130,14 @@ HYMBA_API size_t hymba_workspace_size(const hymba_cfg_t* cfg);
 HYMBA_API size_t hymba_stack_workspace_size(const hymba_cfg_t* cfgs, int n_layers);
 
 /*
- * One hybrid-head layer, forward (prefill).
+ * One hybrid-head layer, forward (prefill): the fused hybrid-head module of the
+ * blog.outta.ai review, section "Design formulation" -- X~ = [meta; X], the one input
+ * projection W_in_proj = [W_Q, W_K, W_V, W_SSM, W_G], attention heads and SSM heads in
+ * parallel (the SSM head's mixing matrix alpha_ij = C_i (prod_{k=j+1..i} exp(A dt_k)) B_j dt_j,
+ * gated by G), each branch normalised and scaled by beta1 / beta2, summed through W_out
+ * ("total fusion formulation"); sliding-window attention with the meta tokens always
+ * visible ("Combine global and local attention", "Meta Tokens"); cross-layer KV sharing
+ * through kv_out / kv_in ("Cross-layer KV sharing").
  *   x       [B, L, d] dtype when meta != NULL; [B, T, d] (rows already X~) when meta == NULL
  *   meta    [M, d] dtype, the learnable meta tokens shared by the batch, or NULL
  *   kv_in   [2, B, T, Hkv*dh] dtype (K then V, token-major, head h at columns
@@ -136,11 +147,14 @@ HYMBA_API size_t hymba_stack_workspace_size(const hymba_cfg_t* cfgs, int n_layer
  *   workspace >= hymba_workspace_size(cfg) bytes, 256-byte aligned; its first 256
  *           bytes hold the status word (reset by this call)
  * Streams: all work is ordered on `stream`.  The attention heads run on a second,
- * non-blocking stream the library creates on its first call on each device (forked
- * from `stream` after the input projection with an event and joined back before the
- * branch norm), so the call behaves as one stream-ordered operation and can be
- * captured into a CUDA graph once the first call on the device has been made
- * outside the capture.
+ * non-blocking stream of the library's (forked from `stream` after the input projection
+ * with an event and joined back before the branch norm), so the call behaves as one
+ * stream-ordered operation.  There is one such second stream (and its two events) per
+ * host thread, device and stream priority, made on that thread's first call with the
+ * caller stream's priority: calls from different threads never share one; calls one
+ * thread makes on several streams do (their attention launches are then ordered among
+ * themselves).  The call can be captured into a CUDA graph once the calling thread has
+ * made one call on the device outside the capture.
  */
 HYMBA_API hymba_status_t hymba_layer_fwd(const void* x, const void* meta, const hymba_weights_t* w,
                                const hymba_cfg_t* cfg, const void* kv_in, void* kv_out,
