@@ -5,6 +5,7 @@ algorithmic FLOPs and HBM bytes of one launch.  These checks pin that accounting
 shapes: the visible-pair count against brute-force enumeration of the attention mask,
 the contraction FLOPs against 2·K·N per row, and the dt projection moving into the scan
 (its FLOPs move, its bytes change by exactly the dt round trip it saves)."""
+import dataclasses
 import os
 import sys
 
@@ -52,3 +53,38 @@ def test_dt_projection_moves_into_the_scan():
     total_plain = sum(b for _, b in plain.values())
     total_fused = sum(b for _, b in fused.values())
     assert total_plain - total_fused == 2 * saved   # dt written once and read once
+
+
+def test_stage_rooflines_sum_layers_and_pick_the_binding_resource():
+    """The layer pair's stages add over both layers; the CUDA-core scan (d_state 128) is
+    held to the fp32 FMA peak, the tensor-core one (d_state 16) to HBM; the workload's
+    roofline time is the sum over stages and layers of the slowest term."""
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    wl = synth.workload("hymba1p5b_kvpair")
+    fused = [False, False]
+    names = list(bench.stage_work(wl.layers[0]).keys())
+    us = {k: 100.0 for k in names}
+    roof, t_us = bench.stage_rooflines(wl.layers, us, peaks, fused, 1965)
+    assert roof["scan"]["bound"] == "alu" and roof["attention"]["bound"] == "tensor"
+    fl0, _ = bench.stage_work(wl.layers[0])["in_proj"]
+    fl1, _ = bench.stage_work(wl.layers[1])["in_proj"]
+    assert roof["in_proj"]["work"] == fl0 + fl1 and fl1 < fl0   # the consumer has no K/V rows
+    alu = 148 * 128 * 2 * 1965e6
+    exp = 0.0
+    for s in wl.layers:
+        for k, (fl, by) in bench.stage_work(s).items():
+            b = bench.stage_bound(k, s)
+            exp += max(fl / 1600e12 if b == "tensor" else 0.0, by / 6000e9, fl / alu if b == "alu" else 0.0)
+    assert abs(t_us - exp * 1e6) < 1e-6 * t_us
+    s16 = synth.workload("hymba350m_layer").first
+    assert bench.stage_bound("scan", s16) == "hbm" and bench.scan_kernel_name(s16).startswith("scan_tc")
+
+
+def test_stack_roofline_counts_the_ffn():
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    wl = synth.workload("hymba1p5b_stack24", n_layers=2)
+    with_ffn = bench.stack_roofline_us(wl.layers, peaks, [False, False])
+    no_ffn = bench.stack_roofline_us([dataclasses.replace(s, ffn_dim=0) for s in wl.layers], peaks, [False, False])
+    fl, _ = bench.ffn_work(wl.layers[0])
+    assert fl == 6.0 * 2048 * 5632 * wl.first.batch * wl.first.T
+    assert with_ffn - no_ffn >= 2 * fl / 1600e12 * 1e6 * 0.999
