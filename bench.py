@@ -758,19 +758,29 @@ def run_native(args, rank, world, local_rank):
             if k in rec:
                 line[k] = rec[k]
         line["device_status"] = bench.H.hymba_status_string(status)
-        pre = measure_prefixed(bench, K, args.warmup, dev, flush)
-        if pre is not None:
-            pre["saving_frac"] = round(1.0 - pre["ms_per_step"] / line["ms_per_step"], 4)
-            line["meta_prefix"] = pre
+        try:
+            pre = measure_prefixed(bench, K, args.warmup, dev, flush)
+            if pre is not None:
+                pre["saving_frac"] = round(1.0 - pre["ms_per_step"] / line["ms_per_step"], 4)
+                line["meta_prefix"] = pre
+        except Exception as ex:  # noqa: BLE001 -- reported in the line, the headline stands
+            line["meta_prefix"] = {"error": f"{type(ex).__name__}: {ex}"}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, bench.x_np, bench.meta_np, bench.ps_np)
     del bench
     torch.cuda.empty_cache()
+    # The secondary records (single GPU only): a failure in one of them is recorded in the
+    # line and does not drop the headline.
+    def secondary(fn):
+        try:
+            return fn()
+        except Exception as ex:  # noqa: BLE001 -- reported, not hidden
+            return {"error": f"{type(ex).__name__}: {ex}"}
+
     if world == 1 and not args.no_per_workload:
         per = {}
-        for name in synth.WORKLOAD_ORDER:
-            if name == args.workload:
-                continue
+
+        def one(name):
             b = Workbench(name, dev)
             k = min(K, 10 if not b.stack else 3)
             r, t_ms = measure(b, k, 3, ranks, dev, flush, stages=True, e2e=False)
@@ -780,27 +790,32 @@ def run_native(args, rank, world, local_rank):
             r["config"] = _workload_config(b.wl)
             if rank == 0 and not args.no_cpu_baseline:
                 r["cpu_baseline"] = cpu_baseline(b.wl, b.x_np, b.meta_np, b.ps_np, budget_s=6.0)
-            per[name] = r
-            del b
-            torch.cuda.empty_cache()
+            return r
+
+        for name in synth.WORKLOAD_ORDER:
+            if name != args.workload:
+                per[name] = secondary(lambda: one(name))
+                torch.cuda.empty_cache()
         if line is not None:
             line["per_workload"] = per
     if world == 1 and not args.no_decode and line is not None:
-        line["decode"] = measure_decode("hymba1p5b_kvpair", dev, flush)
+        line["decode"] = secondary(lambda: measure_decode("hymba1p5b_kvpair", dev, flush))
+        torch.cuda.empty_cache()
     if world == 1 and not args.no_per_workload and line is not None:
         # the option paths (Mamba conv + D skip, per-group branch norm, difference fusion) on
         # the 350M-shaped layer, against the same layer without them
-        opts = dict(conv_width=4, d_skip=1, norm_group=128, fusion=1)
-        b = Workbench("hymba350m_layer", dev, **opts)
-        r, t_ms = measure(b, min(K, 10), 3, ranks, dev, flush, stages=True, e2e=False)
-        r["value"] = weak_scaling_rate(1, min(K, 10), b.tokens, t_ms)
-        r["unit"] = UNIT
-        r["options"] = opts
-        base = line.get("per_workload", {}).get("hymba350m_layer")
-        if base:
-            r["overhead_frac"] = round(r["ms_per_step"] / base["ms_per_step"] - 1.0, 4)
-        line["options"] = r
-        del b
+        def options():
+            opts = dict(conv_width=4, d_skip=1, norm_group=128, fusion=1)
+            b = Workbench("hymba350m_layer", dev, **opts)
+            r, t_ms = measure(b, min(K, 10), 3, ranks, dev, flush, stages=True, e2e=False)
+            r["value"] = weak_scaling_rate(1, min(K, 10), b.tokens, t_ms)
+            r["unit"] = UNIT
+            r["options"] = opts
+            base = line.get("per_workload", {}).get("hymba350m_layer")
+            if base and "ms_per_step" in base:
+                r["overhead_frac"] = round(r["ms_per_step"] / base["ms_per_step"] - 1.0, 4)
+            return r
+        line["options"] = secondary(options)
         torch.cuda.empty_cache()
     if line is not None:
         print(json.dumps(line), flush=True)

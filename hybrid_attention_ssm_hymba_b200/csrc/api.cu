@@ -832,7 +832,6 @@ hymba_status_t hymba_layer_prefill(const void* x, const void* meta, const hymba_
   const int T = cfg->seq_len + cfg->n_meta;
   if (!x || !out || !kv_cache || !ssm_state || !weights_ok(w, *cfg, false) || cache_rows < T)
     return HYMBA_ERR_INVALID_ARG;
-  if (cfg->n_meta > 0 && !meta) return HYMBA_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < hymba_decode_workspace_size(cfg)) return HYMBA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255) return HYMBA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -844,7 +843,8 @@ hymba_status_t hymba_layer_prefill(const void* x, const void* meta, const hymba_
   lo.out = out;
   lo.h_out = ssm_state;
   lo.kv_rows = cache_rows;
-  s = run_layer(x, meta, *w, p, cfg->kv_mode == HYMBA_KV_CONSUME ? kv_cache : nullptr, nullptr, lo, ws, status, st);
+  s = run_layer(x, cfg->n_meta > 0 ? meta : nullptr, *w, p, cfg->kv_mode == HYMBA_KV_CONSUME ? kv_cache : nullptr,
+                nullptr, lo, ws, status, st);
   if (s != HYMBA_OK || cfg->kv_mode == HYMBA_KV_CONSUME) return s;
   // K, V [2][B*T][wkv] in the workspace -> the cache [2][B][cache_rows][wkv]
   const size_t es = esize(cfg->dtype), wkv = static_cast<size_t>(cfg->n_kv_heads) * cfg->head_dim;

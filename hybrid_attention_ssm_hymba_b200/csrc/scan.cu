@@ -387,13 +387,19 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
   const bool ywriter = slice == 0;
   // the state entering row t0: the entry state of a single chunk, or the start of the
   // chunk combine below
+  // g[q][2j], g[q][2j + 1] hold state components n0 + ((j + rot) % NQ) * 4 + {0, 1}, {2, 3}
+  // (the lane's 16-byte chunks are visited in a rotated order, see load_b)
   float2 g0[CPL][NP];
 #pragma unroll
   for (int q = 0; q < CPL; ++q) {
     float hz[NS];
     load_h0(p, b, (active && c0 + q < p.Di) ? c0 + q : 0, n0, NS, hz);
 #pragma unroll
-    for (int i = 0; i < NP; ++i) g0[q][i] = make_float2(hz[2 * i], hz[2 * i + 1]);
+    for (int j = 0; j < NQ; ++j) {
+      const int e = ((j + rot) & (NQ - 1)) * 4;
+      g0[q][2 * j] = make_float2(hz[e], hz[e + 1]);
+      g0[q][2 * j + 1] = make_float2(hz[e + 2], hz[e + 3]);
+    }
   }
   if (sp.S == 1) {
 #pragma unroll
@@ -734,9 +740,12 @@ __global__ void __launch_bounds__(256) scan_w_kernel(const __grid_constant__ CUt
         const float P = ex2_approx(-ncl[q]);
         float* ho = p.h_out + (static_cast<long long>(b) * p.Di + c0 + q) * N + n0;
 #pragma unroll
-        for (int i = 0; i < NP; ++i) {
-          ho[2 * i] = g[q][i].x * P;
-          ho[2 * i + 1] = g[q][i].y * P;
+        for (int j = 0; j < NQ; ++j) {   // undo the rotated chunk order (see g0 above)
+          const int e = ((j + rot) & (NQ - 1)) * 4;
+          ho[e] = g[q][2 * j].x * P;
+          ho[e + 1] = g[q][2 * j].y * P;
+          ho[e + 2] = g[q][2 * j + 1].x * P;
+          ho[e + 3] = g[q][2 * j + 1].y * P;
         }
       }
     }

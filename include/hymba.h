@@ -256,7 +256,8 @@ HYMBA_API size_t hymba_decode_workspace_size(const hymba_cfg_t* cfg);
  * hymba_layer_fwd over the T = L + M prompt rows (cfg.seq_len = L) that also leaves what
  * the next token needs: rows [0, T) of each sequence's K/V in kv_cache (cache_rows >= T;
  * for a HYMBA_KV_CONSUME layer kv_cache is the producer's cache, read only) and the SSM
- * state after row T - 1 in ssm_state.  x, meta, out as in hymba_layer_fwd.
+ * state after row T - 1 in ssm_state.  x, meta, out as in hymba_layer_fwd (meta NULL: x
+ * already holds the T rows of X~, e.g. the previous layer's output).
  */
 HYMBA_API hymba_status_t hymba_layer_prefill(const void* x, const void* meta, const hymba_weights_t* w,
                                    const hymba_cfg_t* cfg, void* kv_cache, int cache_rows,

@@ -99,3 +99,18 @@ def test_prefixed_fp32(a_per_state):
     x, meta, ps, dps = _setup(wl)
     ref, _ = O.layer_forward(x, meta, ps[0], wl.first)
     assert_close(_prefixed_chain(wl, x, meta, dps), ref, "f32", "prefixed fp32 layer")
+
+
+@pytest.mark.parametrize("window,d_state", [(-1, 16), (96, 16), (-1, 128), (96, 128)])
+def test_prefixed_single_layer_window_and_state_size(window, d_state):
+    """One layer with its own K/V, global or windowed, tensor-core (d_state 16) or CUDA-core
+    (d_state 128) scan: the prefixed call against the full path and the oracle."""
+    wl = synth.workload("hymba1p5b_kvpair", n_layers=1, batch=2, seq_len=400, window=window, d_model=512,
+                        n_q_heads=8, n_kv_heads=2, d_inner=512, dt_rank=32, d_state=d_state, kv_mode=H.HYMBA_KV_OWN)
+    x, meta, ps, dps = _setup(wl)
+    g = _prefixed_chain(wl, x, meta, dps)
+    full = _plain_chain(wl, x, meta, dps)
+    ref, _ = O.layer_forward(x, meta, ps[0], wl.first)
+    assert_close(full, ref, "bf16", "full path vs oracle")
+    assert_close(g, full, "bf16", "prefixed vs the full path", tol=2e-3)
+    assert_close(g, ref, "bf16", "prefixed vs oracle")
