@@ -71,7 +71,7 @@ LayerWs layer_ws(const hymba_cfg_t& c, size_t base) {
 // xlo and the fp32 residual stream h; K/V of the current pair; the FFN activation; for
 // bf16 the transposed W_SSM and W_eff = W_x W_SSM of the current block.
 struct StackWs {
-  size_t layer, xn, xlo, h, kv, act, wssm_t, weff, total;
+  size_t layer, xn, h, kv, act, wssm_t, weff, whi, wlohi, total;
 };
 
 StackWs stack_ws(const hymba_cfg_t* cfgs, int n) {
@@ -94,13 +94,14 @@ StackWs stack_ws(const hymba_cfg_t* cfgs, int n) {
   StackWs w;
   size_t o = 0;
   w.layer = o; o = al256(o + layer_max);
-  w.xn = o; o = al256(o + rows * d * es);
-  w.xlo = o; o = al256(o + (bf16 ? rows * d * 2 : 0));
+  w.xn = o; o = al256(o + rows * d * es * (bf16 ? 2 : 1));   // bf16: [x_hi | x_lo] per row
   w.h = o; o = al256(o + (bf16 ? rows * d * 4 : 0));
   w.kv = o; o = al256(o + 2 * rows * kvw * es);
   w.act = o; o = al256(o + rows * ffn * es);
   w.wssm_t = o; o = al256(o + (bf16 ? d * di * 2 : 0));
-  w.weff = o; o = al256(o + (bf16 ? xw * d * 2 : 0));
+  w.weff = o; o = al256(o + (bf16 ? xw * d * 4 : 0));        // W_x W_SSM, fp32
+  w.whi = o; o = al256(o + (bf16 ? xw * d * 2 : 0));
+  w.wlohi = o; o = al256(o + (bf16 ? xw * d * 4 : 0));       // [W_lo | W_hi]
   w.total = o;
   return w;
 }
@@ -211,16 +212,20 @@ struct SideJoin {
 
 // Where a layer's out_proj writes: out = Z W_out^T, or out = resid + Z W_out^T (resid may
 // alias out), each in the layer's dtype or in fp32 (a stack's fp32 residual stream).
-// xlo / weff: the x_proj of a stacked block adds xlo W_eff^T (xlo the bf16 rounding
-// remainder of the block's normalised input, W_eff = W_x W_SSM) to [dt_low | B | C].
+// a_ld: row stride of the layer input x (plain mode; 0 = d_model).
+// w_hi / w_lohi: a stacked block's x_proj straight from its input: [dt_low | B | C] =
+// X_ssm W_x^T = x (W_x W_SSM)^T, evaluated as x_hi W_hi^T + [x_hi | x_lo] [W_lo | W_hi]^T with
+// x_hi the bf16 normalised input, x_lo its bf16 rounding remainder (the columns of x after
+// x_hi: x is [rows, 2 d] with row stride a_ld), W_hi + W_lo = W_x W_SSM to ~16 bits.
 // h_out: the SSM heads' state after the last row [B, Di, N] fp32 (a prefill that a
 // generation step continues); kv_rows: rows per sequence of a consumed K/V buffer (a cache).
 struct LayerOut {
   void* out = nullptr;
   const void* resid = nullptr;
   bool resid_f32 = false, out_f32 = false;
-  const void* xlo = nullptr;
-  const void* weff = nullptr;
+  long long a_ld = 0;
+  const void* w_hi = nullptr;
+  const void* w_lohi = nullptr;
   float* h_out = nullptr;
   long long kv_rows = 0;
   // Meta-prefix record (hymba_meta_prefix): x holds the user rows [B, L, d] only; the meta
@@ -335,6 +340,7 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   } else {
     gi.a = x;
     gi.a_rows = rows;
+    gi.a_ld = lo.a_ld;
   }
   gi.K = c.d_model;
   gi.w = w.w_in;
@@ -408,18 +414,23 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
                                                c.dtype == HYMBA_BF16, st) != cudaSuccess)
     return HYMBA_ERR_CUDA;
   GemmDesc gx;
-  gx.a = xin_ssm;
   gx.a_rows = rows;
-  gx.K = di;
-  gx.w = w.w_x;
   gx.N = c.dt_rank + 2 * c.d_state;
+  if (lo.w_hi && c.dtype == HYMBA_BF16) {   // from the layer input, compensated (see LayerOut)
+    gx.a = x;
+    gx.a_ld = lo.a_ld;
+    gx.K = c.d_model;
+    gx.w = lo.w_hi;
+    gx.a2 = x;
+    gx.K2 = 2 * c.d_model;
+    gx.w2 = lo.w_lohi;
+  } else {
+    gx.a = xin_ssm;
+    gx.K = di;
+    gx.w = w.w_x;
+  }
   gx.seg[gx.nseg++] = seg(0, c.dt_rank, dtlow, c.dt_rank, f32out, hy::SEG_STORE);
   gx.seg[gx.nseg++] = seg(c.dt_rank, gx.N, bc, 2 * c.d_state, 1, hy::SEG_STORE);
-  if (lo.xlo && c.dtype == HYMBA_BF16) {
-    gx.a2 = lo.xlo;
-    gx.w2 = lo.weff;
-    gx.K2 = c.d_model;
-  }
   gx.status = status;
   if ((e = gemm(gx, c.dtype, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
 
@@ -715,14 +726,16 @@ hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weig
   const long long rows = static_cast<long long>(c0.batch) * T;
   const int d = c0.d_model;
   uint8_t* lws = base + S.layer;
-  void* xn = base + S.xn;
-  void* xlo = bf16 ? base + S.xlo : nullptr;
+  void* xn = base + S.xn;   // bf16: row r = [x_hi (d) | x_lo (d)], row stride 2 d
+  const long long xn_ld = bf16 ? 2LL * d : d;
   void* kv = base + S.kv;
   void* act = base + S.act;
   // the residual stream h: fp32 in the workspace (bf16), or `out` itself (fp32)
   float* h = bf16 ? reinterpret_cast<float*>(base + S.h) : static_cast<float*>(out);
   void* wssm_t = base + S.wssm_t;
-  void* weff = base + S.weff;
+  float* weff = reinterpret_cast<float*>(base + S.weff);
+  void* whi = base + S.whi;
+  void* wlohi = base + S.wlohi;
 
   cudaError_t e;
   if (bf16) {
@@ -748,31 +761,33 @@ hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weig
     const bool mixer_last = last && c.ffn_dim == 0;
     lo.out = (bf16 && mixer_last) ? out : static_cast<void*>(h);
     lo.out_f32 = !(bf16 && mixer_last);
-    // the B|C compensation is linear in the normalised input: not with the conv option
+    // x_proj straight from the block input (linear in it): not with the conv option
     const bool compensate = bf16 && c.conv_width == 0;
+    lo.a_ld = xn_ld;
     if (bf16) {
-      if ((e = hy::launch_prenorm_f32(h, w[i].norm1, xn, compensate ? xlo : nullptr, rows, d, c.rms_eps, st)) !=
-          cudaSuccess)
+      if ((e = hy::launch_prenorm_f32(h, w[i].norm1, xn, compensate ? static_cast<uint8_t*>(xn) + d * 2 : nullptr,
+                                      rows, d, c.rms_eps, st, xn_ld)) != cudaSuccess)
         return HYMBA_ERR_CUDA;
     }
     if (compensate) {
-      // W_eff = W_x W_SSM [R + 2N, d]: x_proj adds xlo W_eff^T, the part of [dt_low | B | C]
-      // that the bf16 rounding of the normalised input dropped
+      // W_eff = W_x W_SSM [R + 2N, d] in fp32, split into bf16 W_hi + W_lo
       const int wa = c.n_q_heads * c.head_dim, wkv = c.n_kv_heads * c.head_dim;
       const int ssm_row0 = wa + (c.kv_mode == HYMBA_KV_CONSUME ? 0 : 2 * wkv);
+      const int xw = c.dt_rank + 2 * c.d_state;
       const uint8_t* wssm = static_cast<const uint8_t*>(w[i].w_in) + static_cast<size_t>(ssm_row0) * d * 2;
       if ((e = hy::launch_transpose_bf16(wssm, d, wssm_t, c.d_inner, d, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
       GemmDesc ge;
       ge.a = w[i].w_x;
-      ge.a_rows = c.dt_rank + 2 * c.d_state;
+      ge.a_rows = xw;
       ge.K = c.d_inner;
       ge.w = wssm_t;
       ge.N = d;
-      ge.seg[ge.nseg++] = seg(0, d, weff, d, 0, hy::SEG_STORE);
+      ge.seg[ge.nseg++] = seg(0, d, weff, d, 1, hy::SEG_STORE);
       ge.status = status;
       if (gemm(ge, c.dtype, st) != cudaSuccess) return HYMBA_ERR_CUDA;
-      lo.xlo = xlo;
-      lo.weff = weff;
+      if ((e = hy::launch_split_hi_lo(weff, whi, wlohi, xw, d, st)) != cudaSuccess) return HYMBA_ERR_CUDA;
+      lo.w_hi = whi;
+      lo.w_lohi = wlohi;
     } else if (!bf16 && (e = hy::launch_prenorm_f32_out_f32(h, w[i].norm1, static_cast<float*>(xn), rows, d,
                                                             c.rms_eps, st)) != cudaSuccess) {
       return HYMBA_ERR_CUDA;
@@ -780,11 +795,12 @@ hymba_status_t hymba_stack_fwd(const void* x, const void* meta, const hymba_weig
     hymba_status_t s = run_layer(xn, nullptr, w[i], c, kv, kv, lo, lws, status, st);
     if (s != HYMBA_OK) return s;
     if (c.ffn_dim > 0) {
-      e = bf16 ? hy::launch_prenorm_f32(h, w[i].norm2, xn, nullptr, rows, d, c.rms_eps, st)
+      e = bf16 ? hy::launch_prenorm_f32(h, w[i].norm2, xn, nullptr, rows, d, c.rms_eps, st, xn_ld)
                : hy::launch_prenorm_f32_out_f32(h, w[i].norm2, static_cast<float*>(xn), rows, d, c.rms_eps, st);
       if (e != cudaSuccess) return HYMBA_ERR_CUDA;
       GemmDesc gu;
       gu.a = xn;
+      gu.a_ld = xn_ld;
       gu.a_rows = rows;
       gu.K = d;
       gu.w = w[i].w_gate_up;

@@ -818,7 +818,7 @@ cudaError_t prepare(const GemmDesc& g, int b_rows, int m_rows, int n_cols, CUten
     p.a_rows = static_cast<long long>(g.batch) * p.T;
   } else {
     uint64_t da[2] = {K, static_cast<uint64_t>(g.a_rows)};
-    uint64_t sa[1] = {K * 2};
+    uint64_t sa[1] = {static_cast<uint64_t>(g.a_ld > 0 ? g.a_ld : g.K) * 2};
     uint32_t ba[2] = {BK, BM};
     if (!make_map(&tmA, g.a, 2, da, sa, ba)) return cudaErrorInvalidValue;
     tmAx2 = tmA;

@@ -68,6 +68,7 @@ struct GemmDesc {
   bool meta_mode = false;
   const void* a = nullptr;
   long long a_rows = 0;
+  long long a_ld = 0;   // plain mode: row stride of A in elements (0: K)
   const void* x = nullptr;
   const void* meta = nullptr;
   int batch = 0, L = 0, n_meta = 0;
@@ -196,7 +197,10 @@ cudaError_t launch_rmsnorm(const void* x, void* y, long long rows, int d, float 
 // row of x [rows, d] fp32 (gain [d] fp32, or NULL for unit gain); when y_lo is given it also
 // receives the part of the fp32 result that the bf16 rounding dropped, bf16(v - float(y)).
 cudaError_t launch_prenorm_f32(const float* x, const float* gain, void* y, void* y_lo, long long rows, int d,
-                               float eps, cudaStream_t st);
+                               float eps, cudaStream_t st, long long y_ld = 0);
+// hi = bf16(src), lohi = [bf16(src - hi) | hi] per row: src [rows, cols] fp32, hi [rows, cols],
+// lohi [rows, 2 cols] (bf16).
+cudaError_t launch_split_hi_lo(const float* src, void* hi, void* lohi, int rows, int cols, cudaStream_t st);
 cudaError_t launch_prenorm_f32_out_f32(const float* x, const float* gain, float* y, long long rows, int d, float eps,
                                        cudaStream_t st);
 // h[b, t, :] = float([meta; x_b][t, :]) for a bf16 stack input (h fp32 [batch, L + M, d]).

@@ -330,7 +330,7 @@ namespace {
 template <typename TO>
 __global__ void __launch_bounds__(256) prenorm_f32_kernel(const float* __restrict__ x, const float* __restrict__ gain,
                                                           TO* __restrict__ y, __nv_bfloat16* __restrict__ y_lo,
-                                                          long long rows, int d, float eps) {
+                                                          long long rows, int d, float eps, long long y_ld) {
   pdl_trigger();
   pdl_wait();
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -359,12 +359,12 @@ __global__ void __launch_bounds__(256) prenorm_f32_kernel(const float* __restric
 #pragma unroll
       for (int j = 0; j < 8; ++j) f[j] *= r;
     }
-    Vec8<TO>::store(y + row * d + i, f);
+    Vec8<TO>::store(y + row * y_ld + i, f);
     if (y_lo) {
       float lo[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) lo[j] = f[j] - __bfloat162float(__float2bfloat16_rn(f[j]));
-      Vec8<__nv_bfloat16>::store(y_lo + row * d + i, lo);
+      Vec8<__nv_bfloat16>::store(y_lo + row * y_ld + i, lo);
     }
   }
 }
@@ -436,12 +436,38 @@ cudaError_t launch_broadcast(const void* src, size_t bytes, void* dst, size_t ds
 }
 
 cudaError_t launch_prenorm_f32(const float* x, const float* gain, void* y, void* y_lo, long long rows, int d,
-                               float eps, cudaStream_t st) {
+                               float eps, cudaStream_t st, long long y_ld) {
   if (rows <= 0) return cudaSuccess;
-  if (d % 8) return cudaErrorInvalidValue;
+  if (d % 8 || (y_ld && (y_ld < d || y_ld % 8))) return cudaErrorInvalidValue;
   const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
   return launch(prenorm_f32_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, x, gain,
-                static_cast<__nv_bfloat16*>(y), static_cast<__nv_bfloat16*>(y_lo), rows, d, eps);
+                static_cast<__nv_bfloat16*>(y), static_cast<__nv_bfloat16*>(y_lo), rows, d, eps, y_ld ? y_ld : d);
+}
+
+namespace {
+__global__ void __launch_bounds__(256) split_hi_lo_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ hi,
+                                                          __nv_bfloat16* __restrict__ lohi, int rows, int cols) {
+  pdl_trigger();
+  pdl_wait();
+  const long long n = static_cast<long long>(rows) * cols;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / cols, c = i - r * cols;
+    const float v = src[i];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lohi[r * 2 * cols + c] = __float2bfloat16_rn(v - __bfloat162float(h));
+    lohi[r * 2 * cols + cols + c] = h;
+  }
+}
+}  // namespace
+
+cudaError_t launch_split_hi_lo(const float* src, void* hi, void* lohi, int rows, int cols, cudaStream_t st) {
+  const long long n = static_cast<long long>(rows) * cols;
+  if (n <= 0) return cudaSuccess;
+  const long long blocks = (n + 255) / 256;
+  return launch(split_hi_lo_kernel, dim3(static_cast<unsigned>(blocks < 4 * num_sms() ? blocks : 4 * num_sms())),
+                dim3(256), 0, st, src, static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lohi), rows, cols);
 }
 
 cudaError_t launch_prenorm_f32_out_f32(const float* x, const float* gain, float* y, long long rows, int d, float eps,
@@ -450,7 +476,7 @@ cudaError_t launch_prenorm_f32_out_f32(const float* x, const float* gain, float*
   if (d % 8) return cudaErrorInvalidValue;
   const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
   return launch(prenorm_f32_kernel<float>, dim3(grid), dim3(256), 0, st, x, gain, y,
-                static_cast<__nv_bfloat16*>(nullptr), rows, d, eps);
+                static_cast<__nv_bfloat16*>(nullptr), rows, d, eps, static_cast<long long>(d));
 }
 
 cudaError_t launch_prepend_f32(const void* x, const void* meta, float* h, int batch, int L, int M, int d,
