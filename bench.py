@@ -302,8 +302,12 @@ def _oracle_sample(wl: synth.Workload, x, meta, ps, b: int, L: int):
 
 
 def _sample_len(wl: synth.Workload) -> int:
+    """User tokens of one oracle sample: about half a second of fp64 work on a host core
+    set for every workload (its cost per token grows with width, state size and depth)."""
     s = wl.first
     if s.ffn_dim:
+        return min(s.seq_len, 64)
+    if s.d_state >= 128 or s.d_model >= 2048:
         return min(s.seq_len, 256)
     return min(s.seq_len, 2048)
 
