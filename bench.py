@@ -444,9 +444,10 @@ class Workbench:
         # the options add the conv and the D skip
         per_layer = [(8 if bf16 and not s.norm_group else 7) - int(f) + int(s.conv_width > 0) + int(bool(s.d_skip))
                      for f, s in zip(self.dt_in_scan, wl.layers)]
-        if self.stack:   # the prepend; per block: the mixer's pre-norm (bf16: + W_SSM transpose and the
-            # W_eff GEMM), the layer, and with an FFN its pre-norm and two GEMMs
-            self.launches = 1 + sum(n + (3 if bf16 else 1) + (3 if s.ffn_dim else 0)
+        if self.stack:   # the prepend; per block: the mixer's pre-norm (bf16 without the conv: + the
+            # W_SSM transpose, the W_x W_SSM GEMM and its hi/lo split), the layer, and with an FFN
+            # its pre-norm and two GEMMs
+            self.launches = 1 + sum(n + (4 if bf16 and not s.conv_width else 1) + (3 if s.ffn_dim else 0)
                                     for n, s in zip(per_layer, wl.layers))
         else:
             self.launches = sum(per_layer)
