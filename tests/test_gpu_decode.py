@@ -54,16 +54,23 @@ def _run(wl, norm_tol=None):
         outs.append(out)
         inp, inp_meta = out, None
     status_ok(ws)
-    # the oracle's prefill chain
+    # the oracle layer by layer, each on the input the GPU layer saw: X and meta for the
+    # first, the previous GPU layer's output after that, and for a consumer the K/V the
+    # GPU cache holds (a chained fp64 comparison would measure how much the layer pair
+    # amplifies bf16 rounding of its input, ~1e-2 here, not the layer)
     refs, kv_ref, h_ref = [], None, []
     xin, min_ = x, meta
     for i, s in enumerate(layers):
-        o, kv_l, h = O.layer_prefill_state(xin, min_, ps[i], s, kv_in=kv_ref if s.kv_mode == O.KV_CONSUME else None)
+        kv_in = None
+        if s.kv_mode == O.KV_CONSUME:
+            kc = to_np(cache[:, :, :T])
+            kv_in = (kc[0], kc[1])
+        o, kv_l, h = O.layer_prefill_state(xin, min_, ps[i], s, kv_in=kv_in)
         if s.kv_mode != O.KV_CONSUME:
             kv_ref = kv_l
         refs.append(o)
         h_ref.append(h)
-        xin, min_ = o, None
+        xin, min_ = to_np(outs[i]), None
     for i in range(len(layers)):
         assert_close(to_np(outs[i]), refs[i], dtype, f"prefill out, layer {i}")
         assert_close(to_np(states[i]), h_ref[i], dtype, f"SSM state after the prefill, layer {i}")
@@ -81,11 +88,18 @@ def _run(wl, norm_tol=None):
             out_t = host.empty((s0.batch, s0.d_model), dtype)
             H.check(H.hymba_layer_decode(g_in, H.make_weights(dps[i]), c, cache, cap, pos, states[i], out_t, ws),
                     f"decode layer {i} step {step}")
-            r_out, kv_new, hs[i] = O.layer_decode_step(r_in, ps[i], s, kv_ref, hs[i], pos)
+            kv_step = kv_ref
+            if s.kv_mode == O.KV_CONSUME:
+                kc = to_np(cache[:, :, :pos + 1])
+                kv_step = (kc[0], kc[1])
+            r_out, kv_new, hs[i] = O.layer_decode_step(r_in, ps[i], s, kv_step, hs[i], pos)
             if s.kv_mode != O.KV_CONSUME:
                 kv_ref = kv_new
+                kc = to_np(cache[:, :, pos])
+                assert_close(kc[0], kv_new[0][:, pos], dtype, f"cached K row {pos}, layer {i}")
+                assert_close(kc[1], kv_new[1][:, pos], dtype, f"cached V row {pos}, layer {i}")
             assert_close(to_np(out_t), r_out, dtype, f"decode step {step}, layer {i}")
-            g_in, r_in = out_t, r_out
+            g_in, r_in = out_t, to_np(out_t)
         status_ok(ws)
     for i in range(len(layers)):
         assert_close(to_np(states[i]), hs[i], dtype, f"SSM state after {STEPS} steps, layer {i}")

@@ -51,7 +51,9 @@ def _prefixed_chain(wl, x, meta, dps):
     return to_np(outs[-1])
 
 
-def _plain_chain(wl, x, meta, dps):
+def _plain_chain(wl, x, meta, dps, every_layer=False):
+    """hymba_layer_fwd over every layer: the last layer's output, or (every_layer) each
+    layer's output and the shared K/V."""
     layers = wl.layers
     s0 = layers[0]
     dt = s0.dtype
@@ -66,6 +68,8 @@ def _plain_chain(wl, x, meta, dps):
         H.check(H.hymba_layer_fwd(outs[-1], None, H.make_weights(dps[i]), cfgs[i], kv, None, o2, ws), f"{i}")
         outs.append(o2)
     status_ok(ws)
+    if every_layer:
+        return [to_np(o) for o in outs], (None if kv is None else to_np(kv))
     return to_np(outs[-1])
 
 
@@ -82,13 +86,22 @@ def test_prefixed_layer_is_bit_identical_to_the_full_layer():
 
 
 def test_prefixed_kv_pair_swa_dstate128_matches_oracle_and_full_path():
+    """Each layer of the pair against the oracle on the inputs that layer saw: the producer
+    on X and meta, the consumer on the producer's GPU output rows and K/V.  (Fed the
+    oracle's own fp64 producer output instead, the consumer differs by ~1e-2 from
+    bf16-rounding that input alone: the pair amplifies input rounding, so a chained
+    comparison would test the conditioning, not the consumer.)"""
     wl = synth.workload("hymba1p5b_kvpair", batch=2, seq_len=400, window=96, d_model=512, n_q_heads=8,
                         n_kv_heads=2, d_inner=512, dt_rank=32)
     x, meta, ps, dps = _setup(wl)
+    s0 = wl.first
     g = _prefixed_chain(wl, x, meta, dps)
-    full = _plain_chain(wl, x, meta, dps)
-    h, kv = O.layer_forward(x, meta, ps[0], wl.layers[0])
-    ref, _ = O.layer_forward(h, None, ps[1], wl.layers[1], kv_in=kv)
+    (h_gpu, full), kv_gpu = _plain_chain(wl, x, meta, dps, every_layer=True)
+    h, _ = O.layer_forward(x, meta, ps[0], s0)
+    assert_close(h_gpu, h, "bf16", "producer vs oracle")
+    kv_b = kv_gpu.reshape(2, s0.batch, s0.T, s0.kv_width)
+    ref, _ = O.layer_forward(h_gpu, None, ps[1], wl.layers[1], kv_in=(kv_b[0], kv_b[1]))
+    assert_close(full, ref, "bf16", "consumer (full path) vs oracle")
     assert_close(g, ref, "bf16", "prefixed pair vs oracle")
     assert_close(g, full, "bf16", "prefixed pair vs the full path", tol=2e-3)
 
