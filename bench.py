@@ -115,8 +115,12 @@ def ffn_work(s: synth.LayerShape):
 
 
 def scan_kernel_name(s: synth.LayerShape) -> str:
-    if s.dtype == "bf16" and s.d_state == 16 and not s.a_per_state:
-        return "scan_tc_kernel, tcgen05 tf32"
+    """The scan kernel the library selects for a layer (mirrors the C++ choice)."""
+    if s.dtype == "bf16" and not s.a_per_state:
+        if s.d_state == 16:
+            return "scan_tc_kernel, tcgen05 tf32"
+        if s.d_state == 128 and s.dt_rank % 8 == 0 and 8 <= s.dt_rank <= 128:
+            return "scan_tc128_kernel, tcgen05 tf32, state in TMEM"
     return "scan_w_kernel, fp32 FMA"
 
 

@@ -14,6 +14,7 @@ from ._abi import (ENTRY_POINTS, HYMBA_BF16, HYMBA_ERR_CUDA, HYMBA_ERR_INVALID_A
                    hymba_layer_decode, hymba_layer_prefill, hymba_meta_prefix_size, hymba_meta_prefix,
                    hymba_layer_fwd_prefixed, hymba_branch_norm, hymba_cfg_t, hymba_gemm,
                    hymba_layer_fuses_dt_proj, hymba_layer_fwd, hymba_layer_fwd_events, hymba_layer_fwd_noalloc,
-                   HYMBA_NOALLOC_SCRATCH_BYTES, hymba_rmsnorm, hymba_selective_scan, hymba_stack_fwd,
+                   HYMBA_NOALLOC_SCRATCH_BYTES, hymba_rmsnorm, hymba_selective_scan, hymba_selective_scan_dtproj,
+                   hymba_selective_scan_dtproj_workspace_size, hymba_stack_fwd,
                    hymba_stack_workspace_size, hymba_status_string, hymba_weights_t,
                    hymba_workspace_size, hymba_workspace_status, load, make_cfg, make_weights, STAGES)

@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhymba.so
 ENTRY_POINTS = (
     "hymba_status_string", "hymba_workspace_size", "hymba_stack_workspace_size", "hymba_layer_fwd",
     "hymba_stack_fwd", "hymba_workspace_status", "hymba_layer_fwd_events", "hymba_gemm", "hymba_selective_scan",
+    "hymba_selective_scan_dtproj_workspace_size", "hymba_selective_scan_dtproj",
     "hymba_attention", "hymba_branch_norm", "hymba_rmsnorm", "hymba_layer_fwd_noalloc", "hymba_layer_fuses_dt_proj",
     "hymba_check_wait_timeout", "hymba_decode_workspace_size", "hymba_layer_prefill", "hymba_layer_decode",
     "hymba_meta_prefix_size", "hymba_meta_prefix", "hymba_layer_fwd_prefixed",
@@ -70,6 +71,9 @@ _SIGS = {
     "hymba_workspace_status": (_I, [_VP, _VP]),
     "hymba_gemm": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "hymba_selective_scan": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
+    "hymba_selective_scan_dtproj_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "hymba_selective_scan_dtproj": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP,
+                                         _SZ, _VP]),
     "hymba_attention": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "hymba_branch_norm": (_I, [_VP, _VP, _VP, _I, _I, _I, _F, _I, _VP]),
     "hymba_rmsnorm": (_I, [_VP, _VP, _I, _I, _F, _I, _VP]),
@@ -226,6 +230,18 @@ def hymba_selective_scan(x, dt, bc, gate, a_log, y, y_ld: int, batch: int, T: in
     return load().hymba_selective_scan(_ptr(x), _ptr(dt), _ptr(bc), _ptr(gate), _ptr(a_log), _ptr(y),
                                        y_ld, batch, T, d_inner, d_state, int(a_per_state), dtype,
                                        _ptr(workspace), _nbytes(workspace), _stream(stream))
+
+
+def hymba_selective_scan_dtproj_workspace_size(batch: int, T: int, d_inner: int, d_state: int, dt_rank: int,
+                                               dtype: int) -> int:
+    return load().hymba_selective_scan_dtproj_workspace_size(batch, T, d_inner, d_state, dt_rank, dtype)
+
+
+def hymba_selective_scan_dtproj(x, dt_low, w_dt, b_dt, dt_rank: int, bc, gate, a_log, y, y_ld: int, batch: int,
+                                T: int, d_inner: int, d_state: int, dtype: int, workspace, stream=None) -> int:
+    return load().hymba_selective_scan_dtproj(_ptr(x), _ptr(dt_low), _ptr(w_dt), _ptr(b_dt), dt_rank, _ptr(bc),
+                                              _ptr(gate), _ptr(a_log), _ptr(y), y_ld, batch, T, d_inner, d_state,
+                                              dtype, _ptr(workspace), _nbytes(workspace), _stream(stream))
 
 
 def hymba_attention(q, kv, out, out_ld: int, batch: int, T: int, n_q_heads: int, n_kv_heads: int,

@@ -1120,6 +1120,73 @@ hymba_status_t hymba_selective_scan(const void* x, const void* dt, const float* 
   return cuda_status(hy::launch_scan(s, static_cast<cudaStream_t>(stream)));
 }
 
+size_t hymba_selective_scan_dtproj_workspace_size(int batch, int T, int d_inner, int d_state, int dt_rank,
+                                                  hymba_dtype_t dtype) {
+  if (batch < 1 || T < 1 || d_inner < 1 || dt_rank < 1) return 0;
+  hy::ScanDesc f;
+  f.x = f.gate = f.dt_low = f.w_dt = reinterpret_cast<const void*>(256);
+  f.y = reinterpret_cast<void*>(256);
+  f.bc = reinterpret_cast<const float*>(256);
+  f.b_dt = reinterpret_cast<const float*>(256);
+  f.y_ld = d_inner;
+  f.d_inner = d_inner;
+  f.d_state = d_state;
+  f.dt_rank = dt_rank;
+  f.bf16 = dtype == HYMBA_BF16;
+  if (hy::scan_tc_fuses_dt(f)) return 256;
+  const size_t es = dtype == HYMBA_BF16 ? 2 : 4;
+  return 256 + (static_cast<size_t>(batch) * T * d_inner * es + 255) / 256 * 256;
+}
+
+hymba_status_t hymba_selective_scan_dtproj(const void* x, const void* dt_low, const void* w_dt, const float* b_dt,
+                                           int dt_rank, const float* bc, const void* gate, const float* a_log,
+                                           void* y, int y_ld, int batch, int T, int d_inner, int d_state,
+                                           hymba_dtype_t dtype, void* workspace, size_t ws_bytes, void* stream) {
+  if (!x || !dt_low || !w_dt || !b_dt || !bc || !gate || !a_log || !y || batch < 1 || T < 1 || d_inner < 1 ||
+      dt_rank < 1 || y_ld < d_inner)
+    return HYMBA_ERR_INVALID_ARG;
+  if (dtype != HYMBA_BF16 && dtype != HYMBA_F32) return HYMBA_ERR_INVALID_ARG;
+  if (!valid_state(d_state)) return HYMBA_ERR_UNSUPPORTED;
+  const size_t need = hymba_selective_scan_dtproj_workspace_size(batch, T, d_inner, d_state, dt_rank, dtype);
+  if (!workspace || ws_bytes < need) return HYMBA_ERR_WORKSPACE;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  hy::ScanDesc s;
+  s.x = x;
+  s.bc = bc;
+  s.gate = gate;
+  s.a_log = a_log;
+  s.y = y;
+  s.y_ld = y_ld;
+  s.batch = batch;
+  s.T = T;
+  s.d_inner = d_inner;
+  s.d_state = d_state;
+  s.bf16 = dtype == HYMBA_BF16;
+  s.status = static_cast<unsigned*>(workspace);
+  hy::ScanDesc f = s;
+  f.dt = ws;  // unread when fused
+  f.dt_low = dt_low;
+  f.w_dt = w_dt;
+  f.b_dt = b_dt;
+  f.dt_rank = dt_rank;
+  if (hy::scan_tc_fuses_dt(f)) return cuda_status(hy::launch_scan(f, st));
+  // otherwise dt = softplus(dt_low W_dt^T + b_dt) through the GEMM into the workspace first
+  void* dt = ws + 256;
+  GemmDesc gd;
+  gd.a = dt_low;
+  gd.a_rows = static_cast<long long>(batch) * T;
+  gd.K = dt_rank;
+  gd.w = w_dt;
+  gd.N = d_inner;
+  gd.seg[gd.nseg++] = seg(0, d_inner, dt, d_inner, 0, hy::SEG_SOFTPLUS_BIAS, b_dt);
+  gd.status = s.status;
+  cudaError_t e = gemm(gd, dtype, st);
+  if (e != cudaSuccess) return HYMBA_ERR_CUDA;
+  s.dt = dt;
+  return cuda_status(hy::launch_scan(s, st));
+}
+
 hymba_status_t hymba_attention(const void* q, const void* kv, void* out, int out_ld, int batch, int T,
                                int n_q_heads, int n_kv_heads, int head_dim, int n_meta, int window,
                                hymba_dtype_t dtype, void* workspace, size_t ws_bytes, void* stream) {

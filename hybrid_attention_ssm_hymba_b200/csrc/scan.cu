@@ -929,6 +929,8 @@ cudaError_t launch_t(const ScanDesc& s, cudaStream_t st) {
   const long long es = static_cast<long long>(sizeof(TI));
   const bool tma_ok = (s.d_inner * es) % 16 == 0 && (s.y_ld * es) % 16 == 0 && a16(s.x) && a16(s.dt) &&
                      a16(s.gate) && a16(s.bc) && a16(s.y);
+  // a fused dt projection (dt_low set) exists only in the tensor-core kernels
+  if (s.dt_low) return tma_ok && sizeof(TI) == 2 ? launch_scan_tc(s, st) : cudaErrorInvalidValue;
   if (tma_ok) {
 #if HY_SCAN_TC
     if (sizeof(TI) == 2 && s.d_state == 16) {

@@ -42,7 +42,7 @@ _STREAM = {
     "w_conv": 22, "b_conv": 23, "d_skip": 24,
     # free-standing stage inputs used by the per-kernel tests
     "s_x": 40, "s_dt": 41, "s_bc": 42, "s_g": 43, "s_q": 44, "s_kv": 45,
-    "s_z": 46, "s_a": 47, "s_w": 48,
+    "s_z": 46, "s_a": 47, "s_w": 48, "s_dl": 49, "s_wd": 50, "s_bd": 51,
 }
 
 # kv_mode values (match hymba_kv_mode_t in include/hymba.h)
@@ -303,6 +303,18 @@ def scan_inputs(seed: int, B: int, T: int, Di: int, N: int, dt_min=1e-3, dtype="
     a_shape = (Di, N) if a_per_state else (Di,)
     a_log = uniform(seed, 0, "s_a", a_shape, 0.0, math.log(16.0))
     return dict(x=x, dt=dt, bc=bc, g=gate, a_log=a_log)
+
+
+def scan_dtproj_inputs(seed: int, B: int, T: int, Di: int, N: int, R: int, dt_min=1e-3, dtype="bf16"):
+    """scan_inputs with dt given through its low-rank projection, as the layer forms it:
+    dt_low [B*T, R] ~ N(0, 0.5) (dtype), w_dt [Di, R] ~ N(0, 0.02) (dtype), b_dt [Di] fp32
+    the inverse softplus of dt0 ~ U(dt_min, 0.1).  No dt entry."""
+    d = scan_inputs(seed, B, T, Di, N, dt_min=dt_min, dtype=dtype)
+    del d["dt"]
+    d["dt_low"] = normal(seed, 0, "s_dl", (B * T, R), 0.5, dtype)
+    d["w_dt"] = normal(seed, 0, "s_wd", (Di, R), 0.02, dtype)
+    d["b_dt"] = inverse_softplus(uniform(seed, 0, "s_bd", (Di,), dt_min, 0.1)).astype(np.float32)
+    return d
 
 
 def attention_inputs(seed: int, B: int, T: int, Hq: int, Hkv: int, dh: int, dtype="bf16",

@@ -356,6 +356,28 @@ HYMBA_API hymba_status_t hymba_selective_scan(const void* x, const void* dt, con
                                     void* stream);
 
 /*
+ * The selective scan with the SSM heads' dt projection in front of it: the same scan
+ * as hymba_selective_scan with
+ *   dt = softplus(dt_low W_dt^T + b_dt)          (Mamba's discretisation step, per row and channel)
+ *   dt_low [batch*T, dt_rank] dtype (row stride dt_rank);  w_dt [d_inner, dt_rank] dtype;
+ *   b_dt [d_inner] fp32;  one decay rate per channel (a_log [d_inner]).
+ * Where a tensor-core kernel takes the configuration (bf16; d_state 16 with dt_rank 64,
+ * or d_state 128 with dt_rank a multiple of 8 up to 128; 16-byte aligned operands and
+ * row strides) dt is formed block by block inside the scan and never stored; otherwise
+ * it is computed into the workspace first.
+ * hymba_selective_scan_dtproj_workspace_size gives the bytes needed (256 for the fused
+ * kernels: the status word); HYMBA_ERR_WORKSPACE when ws_bytes is smaller.
+ */
+HYMBA_API size_t hymba_selective_scan_dtproj_workspace_size(int batch, int T, int d_inner, int d_state,
+                                                            int dt_rank, hymba_dtype_t dtype);
+HYMBA_API hymba_status_t hymba_selective_scan_dtproj(const void* x, const void* dt_low, const void* w_dt,
+                                           const float* b_dt, int dt_rank, const float* bc,
+                                           const void* gate, const float* a_log, void* y, int y_ld,
+                                           int batch, int T, int d_inner, int d_state,
+                                           hymba_dtype_t dtype, void* workspace, size_t ws_bytes,
+                                           void* stream);
+
+/*
  * Attention heads ("Design formulation", attention head; "Combine global and local
  * attention"): per sequence and query head h (KV head h / (Hq/Hkv)),
  *   out_i = sum_j softmax_j(q_i . k_j / sqrt(dh)) v_j  over visible j (see hymba_cfg_t.window)

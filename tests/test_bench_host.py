@@ -56,11 +56,12 @@ def test_dt_projection_moves_into_the_scan():
 
 
 def test_stage_rooflines_sum_layers_and_pick_the_binding_resource():
-    """The layer pair's stages add over both layers; the CUDA-core scan (d_state 128) is
-    held to the fp32 FMA peak, the tensor-core one (d_state 16) to HBM; the workload's
-    roofline time is the sum over stages and layers of the slowest term."""
+    """The layer pair's stages add over both layers; the CUDA-core scan (here d_state 128
+    with one decay per state, which has no tensor-core form) is held to the fp32 FMA peak,
+    the tensor-core ones (d_state 16, and 128 with one decay per channel) to HBM; the
+    workload's roofline time is the sum over stages and layers of the slowest term."""
     peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
-    wl = synth.workload("hymba1p5b_kvpair")
+    wl = synth.workload("hymba1p5b_kvpair", a_per_state=True)
     fused = [False, False]
     names = list(bench.stage_work(wl.layers[0]).keys())
     us = {k: 100.0 for k in names}
@@ -77,7 +78,10 @@ def test_stage_rooflines_sum_layers_and_pick_the_binding_resource():
             exp += max(fl / 1600e12 if b == "tensor" else 0.0, by / 6000e9, fl / alu if b == "alu" else 0.0)
     assert abs(t_us - exp * 1e6) < 1e-6 * t_us
     s16 = synth.workload("hymba350m_layer").first
-    assert bench.stage_bound("scan", s16) == "hbm" and bench.scan_kernel_name(s16).startswith("scan_tc")
+    assert bench.stage_bound("scan", s16) == "hbm" and bench.scan_kernel_name(s16).startswith("scan_tc_kernel")
+    s128 = synth.workload("hymba1p5b_kvpair").first
+    assert bench.stage_bound("scan", s128) == "hbm" and bench.scan_kernel_name(s128).startswith("scan_tc128")
+    assert bench.scan_kernel_name(dataclasses.replace(s128, dt_rank=136)).startswith("scan_w")
 
 
 def test_stack_roofline_counts_the_ffn():

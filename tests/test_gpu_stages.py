@@ -215,3 +215,88 @@ def test_rmsnorm_parity(dtype):
     y = host.empty(x.shape, dtype)
     H.check(H.hymba_rmsnorm(tx, y, 513, 2048, 1e-6, DT[dtype]), "rmsnorm")
     assert_close(to_np(y), O.rms_normalize(x, 1e-6), dtype, "rmsnorm")
+
+
+# ------------------------------------------------------------------ scan with the dt projection
+
+def _dtproj_ref(inp, B, T, Di, N, chans=None):
+    chans = np.arange(Di) if chans is None else np.asarray(chans)
+    dt = O.softplus(O.linear(inp["dt_low"], inp["w_dt"][chans]) + inp["b_dt"][chans].astype(np.float64))
+    x = inp["x"].reshape(B, T, Di)[:, :, chans]
+    g = inp["g"].reshape(B, T, Di)[:, :, chans]
+    bc = inp["bc"].reshape(B, T, 2 * N)
+    y = O.selective_scan(x, dt.reshape(B, T, len(chans)), O.ssm_decay_rate(inp["a_log"][chans]), bc[..., :N],
+                         bc[..., N:])
+    return (g * y).reshape(B * T, len(chans))
+
+
+def _run_dtproj(inp, B, T, Di, N, dtype, y_ld=None):
+    R = inp["dt_low"].shape[1]
+    y_ld = Di if y_ld is None else y_ld
+    y = host.empty((B * T, y_ld), dtype)
+    y.zero_()   # columns past Di are not written
+    ws = host.workspace(H.hymba_selective_scan_dtproj_workspace_size(B, T, Di, N, R, DT[dtype]))
+    H.check(H.hymba_selective_scan_dtproj(dev(inp["x"], dtype), dev(inp["dt_low"], dtype), dev(inp["w_dt"], dtype),
+                                          fp32(inp["b_dt"]), R, fp32(inp["bc"]), dev(inp["g"], dtype),
+                                          fp32(inp["a_log"]), y, y_ld, B, T, Di, N, DT[dtype], ws), "scan dtproj")
+    status_ok(ws)
+    return to_np(y)[:, :Di]
+
+
+@pytest.mark.parametrize("dtype,B,T,Di,N,R", [
+    ("bf16", 2, 300, 256, 128, 128),   # tensor-core form, d_state 128: two dt atoms, ragged last block
+    ("bf16", 1, 517, 200, 128, 96),    # second channel tile partial, dt_rank 96 (zero-filled atom tail)
+    ("bf16", 3, 65, 128, 128, 64),     # one dt atom, three sequences
+    ("bf16", 1, 31, 136, 128, 8),      # a single partial block, 8-wide dt projection
+    ("bf16", 2, 333, 192, 16, 64),     # d_state 16 tensor-core form
+    ("bf16", 1, 100, 64, 64, 32),      # no tensor-core form: dt through the GEMM, then the scan
+    ("f32", 2, 90, 48, 128, 40),
+])
+def test_scan_dtproj_parity(dtype, B, T, Di, N, R):
+    inp = synth.scan_dtproj_inputs(31, B, T, Di, N, R, dtype=dtype)
+    assert_close(_run_dtproj(inp, B, T, Di, N, dtype), _dtproj_ref(inp, B, T, Di, N), dtype, "scan dtproj")
+
+
+def test_scan_dtproj_d128_output_row_stride():
+    """y written into the SSM columns of a wider row (the layer's Z layout)."""
+    B, T, Di, N, R = 2, 150, 256, 128, 128
+    inp = synth.scan_dtproj_inputs(32, B, T, Di, N, R)
+    assert_close(_run_dtproj(inp, B, T, Di, N, "bf16", y_ld=Di + 64), _dtproj_ref(inp, B, T, Di, N), "bf16",
+                 "scan dtproj y_ld")
+
+
+def test_scan_dtproj_d128_hands_large_decay_blocks_to_the_recurrence():
+    """d_state 128 tensor-core form: a 32-step block where some channel's half-block decay
+    sum leaves the factored form's range runs the plain recurrence on the state held in
+    TMEM, and the block products resume after it.  dt is pushed up (to ~10) for one channel
+    per case by a run of large dt_low rows times a positive W_dt row: in the first and in the
+    second half of a block, in the second (partial) channel tile, in the ragged last block,
+    and over a run spanning two blocks."""
+    B, T, Di, N, R = 2, 300, 200, 128, 128
+    inp = synth.scan_dtproj_inputs(33, B, T, Di, N, R)
+    dl = inp["dt_low"].reshape(B, T, R).copy()
+    wd = inp["w_dt"].copy()
+    for c in (7, 150, 100, 60):
+        wd[c] = np.abs(wd[c]) + 0.05
+    # dt_low runs: rows are shared by all channels, so every channel with a positive-leaning
+    # W_dt row sees them, the four above most strongly
+    dl[0, 36:44] = 2.0     # block 1, first half
+    dl[0, 120:124] = 2.0   # block 3, second half
+    dl[1, 290:298] = 2.0   # block 9 (12 steps), ragged
+    dl[1, 60:70] = 2.0     # across blocks 1 and 2
+    inp["dt_low"] = synth.round_bf16(dl.reshape(B * T, R))
+    inp["w_dt"] = synth.round_bf16(wd)
+    dt = O.softplus(O.linear(inp["dt_low"], inp["w_dt"]) + inp["b_dt"].astype(np.float64))
+    assert dt.max() > 5.0, "the runs must produce large dt"
+    assert_close(_run_dtproj(inp, B, T, Di, N, "bf16"), _dtproj_ref(inp, B, T, Di, N), "bf16",
+                 "scan dtproj mixed blocks")
+
+
+@pytest.mark.parametrize("B,T,Di,N,R,dt_min", [(4, 8320, 4096, 128, 128, 1e-3), (1, 32896, 3072, 128, 96, 1e-4)])
+def test_scan_dtproj_full_size_sampled_channels(B, T, Di, N, R, dt_min):
+    """The 1.5B-shaped pair's and the 32K layer's scan shapes in the layer's launch
+    configuration; channels from both ends of several 128-channel tiles checked exactly."""
+    inp = synth.scan_dtproj_inputs(34, B, T, Di, N, R, dt_min=dt_min)
+    y = _run_dtproj(inp, B, T, Di, N, "bf16")
+    chans = np.array([0, 1, 127, 128, 777, Di - 1])
+    assert_close(y[:, chans], _dtproj_ref(inp, B, T, Di, N, chans), "bf16", "scan dtproj sampled channels")
