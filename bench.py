@@ -124,11 +124,22 @@ def scan_kernel_name(s: synth.LayerShape) -> str:
     return "scan_w_kernel, fp32 FMA"
 
 
-def stage_bound(stage: str, s: synth.LayerShape) -> str:
+GEMM_STAGES = ("in_proj", "x_proj", "dt_proj", "out_proj")
+
+
+def stage_bound(stage: str, s: synth.LayerShape, work=None, peaks=None) -> str:
     """The bound that binds each stage: a dense contraction on the tensor cores, HBM
-    traffic, or (the CUDA-core scan at d_state > 16) the fp32 FMA rate."""
-    if stage in ("in_proj", "out_proj", "attention"):
+    traffic, or (the CUDA-core scan) the fp32 FMA rate.  A GEMM stage is held to whichever
+    of its FLOP time and its byte time is longer (x_proj's N = dt_rank + 2 d_state is
+    narrow: byte-bound on some shapes, FLOP-bound on others); given no work and peaks it
+    counts as a contraction."""
+    if stage == "attention":
         return "tensor"
+    if stage in GEMM_STAGES:
+        if work is None or peaks is None:
+            return "tensor"
+        fl, by = work
+        return "tensor" if fl / (peaks["bf16_tflops"] * 1e12) >= by / (peaks["hbm_gbs"] * 1e9) else "hbm"
     if stage == "scan" and not scan_kernel_name(s).startswith("scan_tc"):
         return "alu"
     return "hbm"
@@ -190,7 +201,7 @@ def stage_rooflines(layers, stage_us, peaks, dt_in_scan, sm_max_mhz=None):
     t_roof = 0.0
     for s, fused in zip(layers, dt_in_scan):
         for name, (fl, by) in stage_work(s, fused).items():
-            b = stage_bound(name, s)
+            b = stage_bound(name, s, (fl, by), peaks)
             t_roof += max(fl / tc if b == "tensor" else 0.0, by / hbm, fl / alu if b == "alu" else 0.0)
             f0, b0, _ = tot.get(name, (0.0, 0.0, b))
             tot[name] = (f0 + fl, b0 + by, b)
@@ -223,7 +234,7 @@ def stack_roofline_us(layers, peaks, dt_in_scan):
     t = 0.0
     for s, fused in zip(layers, dt_in_scan):
         for name, (fl, by) in stage_work(s, fused).items():
-            b = stage_bound(name, s)
+            b = stage_bound(name, s, (fl, by), peaks)
             t += max(fl / tc if b == "tensor" else 0.0, by / hbm, fl / alu if b == "alu" else 0.0)
         if s.ffn_dim:
             fl, by = ffn_work(s)

@@ -63,6 +63,43 @@ __device__ __forceinline__ bool visible(int i, int j, int n_meta, int window) {
   return j <= i && (window < 0 || i - j <= window || j < n_meta);
 }
 
+// Three-input fp32 maximum (sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Maximum of a 128-value row (fp32 bit patterns): eight independent chains of
+// three-input maxima, so the reduction is 9 dependent steps deep instead of 128.
+__device__ __forceinline__ float row_max128(const uint32_t (&sv)[128]) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(__uint_as_float(sv[i]), __uint_as_float(sv[i + 8]));
+#pragma unroll
+  for (int e = 16; e < 128; e += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = max3f(m[i], __uint_as_float(sv[e + i]), __uint_as_float(sv[e + 8 + i]));
+  return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+// P = 2^(S scale - m_ref) for a 128-value row, packed in place as bf16 pairs
+// (sv[q] <- (p[2q], p[2q+1]); reads index >= q first); returns the row sum of the fp32
+// values.  Paired scale-and-subtract, four independent partial sums.
+__device__ __forceinline__ float row_exp128(uint32_t (&sv)[128], float scale_log2, float m_ref) {
+  const float2 sc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
+  float2 acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int q = 0; q < 64; ++q) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1])), sc, nm);
+    const float2 pq = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    acc[q & 3] = __fadd2_rn(acc[q & 3], pq);
+    sv[q] = pack_bf16(pq.x, pq.y);
+  }
+  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return t.x + t.y;
+}
+
 __global__ void __launch_bounds__(192, 1)
     attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnParams p) {
@@ -534,10 +571,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int e = 0; e < 128; ++e)
           if (!visible(i, k0 + e, p.n_meta, p.window)) sv[e] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
-      const float m_cand = mx * p.scale_log2;
+      const float m_cand = row_max128(sv) * p.scale_log2;
       const bool need = m_cand > m_used + kRescaleLog2;
       float alpha = 1.f;
       if (need) {
@@ -545,15 +579,8 @@ __global__ void __launch_bounds__(320, 1)
         m_used = m_cand;
       }
       const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
-      float sum = 0.f;
-      // P in bf16, packed in place: sv[q] <- (p[2q], p[2q+1]) (reads index >= q first)
-#pragma unroll
-      for (int q = 0; q < 64; ++q) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * q]), p.scale_log2, -m_ref));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * q + 1]), p.scale_log2, -m_ref));
-        sum += p0 + p1;
-        sv[q] = pack_bf16(p0, p1);
-      }
+      // P in bf16, packed in place over the first 64 words
+      const float sum = row_exp128(sv, p.scale_log2, m_ref);
       tmem_st32(tSx, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_st32(tSx + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       if (j > 0 && __any_sync(0xffffffffu, need)) {

@@ -618,30 +618,40 @@ cudaError_t launch_tc(const ScanDesc& s, cudaStream_t st) {
 
 
 // ---------------------------------------------------------------------------------
-// d_state = 128.  The same block form, re-balanced for a state eight times larger:
+// d_state = 128.  The same block form, re-balanced for a state eight times larger.
 //
 // * The state lives in TMEM as G' (fp32, 128 columns), and the tensor core advances it
 //   itself.  With r = S0 (the decay sum of a block's first half, log2 units) and S1 that
 //   of its second half, the state leaving block k is h_{k+1} = 2^-S1 (G'_k + V_k B_k),
 //   so G'_{k+1} = 2^-S0_{k+1} 2^-S1_k (G'_k + V_k B_k): the product dG = V B accumulates
-//   straight into G' after Y += G' C^T has read it (tcgen05.mma of one thread execute in
+//   straight into G' after Y = G' C^T has read it (tcgen05.mma of one thread execute in
 //   issue order), and the CUDA cores rescale G' once per block, one multiply per element
 //   (two factors, each at most 2^100, applied one after the other).
 // * Blocks of Q = 32 steps (halves of 16): a B|C row is 1 KB, and two stages of 32 rows
-//   of x, gate, dt_low and B|C (56 KB each) fit beside the other tiles.
-// * B|C arrive as eight 32-column boxes ([32 t][128 B] each, 128-byte swizzle): chunks
-//   0-3 are B (n in [32 q, 32 q + 32)), 4-7 are C, each one K atom of the tf32 products.
-// * M and B^T are double-buffered, so the mask/transpose warps prepare block k while
-//   block k - 1's products run; V, W and Y are double-buffered in TMEM.
+//   of x, gate, dt_low and B|C (56 KB each) fit beside the other tiles.  B|C arrive as
+//   eight 32-column boxes ([32 t][128 B] each, 128-byte swizzle): chunks 0-3 are B (n in
+//   [32 q, 32 q + 32)), 4-7 are C, each one K atom of the tf32 products.
+// * The per-block dependency chain is only: the state products of block k -> the CUDA
+//   cores rescale G' -> the state products of block k + 1.  Everything else is kept off
+//   it: the copy warps turn each stage's B into B^T and copy C (both tf32, double-
+//   buffered) as soon as it lands, so the stage is released long before the state
+//   products read B and C; the channel warps form V and W of block k + 1 while block k's
+//   products run (V, W triple-buffered in TMEM); the part of Y that does not depend on
+//   the state (V M^T) is added after the state products; and the MMA thread issues
+//   whichever of its four tasks is ready (state products, a landed stage's dt projection
+//   and C B^T, V M^T, stage release) instead of waiting in a fixed order.
 // * The dt projection is always fused (dt_rank <= 128: one or two 64-column atoms of
 //   dt_low and W_dt, columns past dt_rank zero-filled by TMA).
 // * A block where some channel's half-block decay sum exceeds kRange runs the plain
-//   recurrence on the CUDA cores (half-1 warps, 32 state columns at a time from TMEM),
-//   with G' holding the raw state on entry and on exit and V = 0.
+//   recurrence on the CUDA cores (half-1 warps, 32 state columns at a time from TMEM,
+//   B and C from the tf32 copies), with G' holding the raw state on entry and on exit;
+//   its V, W columns then carry dt x and the gate, and the MMA thread skips its products.
+// * y goes straight from registers to global memory (a warp writes 32 adjacent channels
+//   of a row).
 //
 // CTA = 128 channels of one sequence, 384 threads: warps 0-7 channels (TMEM quadrant
-// w % 4, half w / 4 of the block's steps and of G''s columns), warp 8 the mask M and half
-// of B^T, warp 9 the other half of B^T, warp 10 TMA, warp 11 TMEM and MMA.
+// w % 4, half w / 4 of the block's steps and of G''s columns), warps 8-9 B^T and the C
+// copy (warp 8 also the mask M, from TMEM lanes 0-31), warp 10 TMA, warp 11 TMEM and MMA.
 namespace t128 {
 constexpr int Q = 32;
 constexpr int HQ = 16;
@@ -655,57 +665,73 @@ constexpr int DL_B = 2 * DLC_B;
 constexpr int WDC_B = CH * 128;         // one W_dt atom [128 c][64 r] bf16
 constexpr int MT_B = Q * Q * 4;         // M [t][s] tf32
 constexpr int BT_B = NS * Q * 4;        // B^T [n][s] tf32
+constexpr int CC_B = 4 * BCC_B;         // C [t][n] tf32, four chunks
 constexpr int ST = 2;                   // stages
 constexpr int OFF_BC = 0;               // first: C B^T reads 96 rows past a C chunk
 constexpr int OFF_DL = OFF_BC + ST * BC_B;
 constexpr int OFF_WD = OFF_DL + ST * DL_B;
 constexpr int OFF_MT = OFF_WD + 2 * WDC_B;
 constexpr int OFF_BT = OFF_MT + 2 * MT_B;
-constexpr int OFF_X = OFF_BT + 2 * BT_B;
+constexpr int OFF_CC = OFF_BT + 2 * BT_B;
+constexpr int OFF_X = OFF_CC + 2 * CC_B;
 constexpr int OFF_G = OFF_X + ST * TILE_B;
-constexpr int OFF_Y = OFF_G + ST * TILE_B;
-constexpr int OFF_S = OFF_Y + 2 * TILE_B;
-constexpr int OFF_BAR = OFF_S + 2 * CH * 4;
-constexpr int NBAR = 2 * ST + 2 + 2 + 5;
+constexpr int OFF_S = OFF_G + ST * TILE_B;   // float [2 blocks][2 halves][128]: half-block decay sums
+constexpr int OFF_ANY = OFF_S + 2 * 2 * CH * 4;  // int [3]: the block runs the plain recurrence
+constexpr int OFF_BAR = OFF_ANY + 16;
+// full[ST] empty[ST] dtready[2] mraw[2] vready[3] btready[2] mready[2] gready dgready[2] yready[2] mma_done
+constexpr int NBAR = 2 * ST + 2 + 2 + 3 + 2 + 2 + 1 + 2 + 2 + 1;
 constexpr int SMEM_TOTAL = OFF_BAR + NBAR * 8 + 16 + 1024;
-static_assert(OFF_DL % 1024 == 0 && OFF_WD % 1024 == 0 && OFF_MT % 1024 == 0 && OFF_BT % 1024 == 0,
+static_assert(OFF_DL % 1024 == 0 && OFF_WD % 1024 == 0 && OFF_MT % 1024 == 0 && OFF_BT % 1024 == 0 &&
+                  OFF_CC % 1024 == 0,
               "swizzled tiles 1024-aligned");
 static_assert(OFF_BC + (ST - 1) * BC_B + 7 * BCC_B + 128 * 128 <= OFF_BAR, "C B^T's A rows stay in the allocation");
 static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
 
 constexpr uint32_t COL_Y = 0;     // [2][32]
-constexpr uint32_t COL_W = 64;    // [2][32]; dt in a block that runs the plain recurrence
-constexpr uint32_t COL_V = 128;   // [2][32]
-constexpr uint32_t COL_DT = 192;  // [32] W_dt dt_low^T
-constexpr uint32_t COL_MR = 224;  // [32] C B^T (lanes 0-31)
-constexpr uint32_t COL_GP = 256;  // [128] G'
+constexpr uint32_t COL_W = 64;    // [3][32]
+constexpr uint32_t COL_V = 160;   // [3][32]
+constexpr uint32_t COL_DT = 256;  // [2][32] W_dt dt_low^T
+constexpr uint32_t COL_MR = 320;  // [2][32] C B^T (lanes 0-31)
+constexpr uint32_t COL_GP = 384;  // [128] G'
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_Q = idesc_tf32(128, Q);
 constexpr uint32_t IDESC_N = idesc_tf32(128, NS);
 constexpr uint32_t IDESC_DT = idesc_bf16(128, Q, false, false);
 
+// Offsets of element (n, s) in B^T [n][s] and (t, n) in the C copy [t][n] (K-major,
+// 128-byte swizzle; B^T one 128-row atom, C four 32-column chunks).
+HY_DEV uint32_t bt_off(int n, int s) {
+  return (n >> 3) * 1024 + (n & 7) * 128 + (((s >> 2) ^ (n & 7)) << 4) + (s & 3) * 4;
+}
+HY_DEV uint32_t cc_off(int t, int n) {
+  return (n >> 5) * BCC_B + (t >> 3) * 1024 + (t & 7) * 128 + ((((n & 31) >> 2) ^ (t & 7)) << 4) + (n & 3) * 4;
+}
+
 __global__ void __launch_bounds__(NTHR, 1)
     scan_tc128_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDL,
                       const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmBC,
-                      const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmWD,
-                      const float* __restrict__ a_log, const float* __restrict__ b_dt, int T, int Di, int ka,
-                      float* __restrict__ h_out, int t0, const float* __restrict__ h0, long long h0_bstride,
+                      const __grid_constant__ CUtensorMap tmWD, const float* __restrict__ a_log,
+                      const float* __restrict__ b_dt, __nv_bfloat16* __restrict__ y, long long y_ld, int T, int Di,
+                      int ka, float* __restrict__ h_out, int t0, const float* __restrict__ h0, long long h0_bstride,
                       unsigned* status) {
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);  // [ST] TMA landed
   uint64_t* empty = full + ST;         // [ST] the stage's last reader done
-  uint64_t* vready = empty + ST;       // [2] V, W of the block in TMEM (256 arrivals)
-  uint64_t* dgready = vready + 2;      // [2] the block's products done: Y complete, G' advanced
-  uint64_t* gready = dgready + 2;      // G' rescaled for the block (256 arrivals)
-  uint64_t* mraw = gready + 1;         // C B^T in TMEM
-  uint64_t* mready = mraw + 1;         // M and B^T in shared memory (64 arrivals)
-  uint64_t* dtready = mready + 1;      // W_dt dt_low^T in TMEM
-  uint64_t* mma_done = dtready + 1;
+  uint64_t* dtready = empty + ST;      // [2] W_dt dt_low^T of the block in TMEM
+  uint64_t* mraw = dtready + 2;        // [2] C B^T of the block in TMEM
+  uint64_t* vready = mraw + 2;         // [3] V, W of the block in TMEM (256 arrivals)
+  uint64_t* btready = vready + 3;      // [2] B^T and the C copy in shared memory (64 arrivals)
+  uint64_t* mready = btready + 2;      // [2] M in shared memory (32 arrivals)
+  uint64_t* gready = mready + 2;       // G' rescaled for the block (256 arrivals)
+  uint64_t* dgready = gready + 1;      // [2] the block's state products done (G' advanced)
+  uint64_t* yready = dgready + 2;      // [2] the block's Y complete
+  uint64_t* mma_done = yready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sS = reinterpret_cast<float*>(sm + OFF_S);
+  volatile int* sAny = reinterpret_cast<volatile int*>(sm + OFF_ANY);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c0 = blockIdx.x * CH, b = blockIdx.y;
@@ -717,13 +743,15 @@ __global__ void __launch_bounds__(NTHR, 1)
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&vready[i], NCHT);
+      mbar_init(&dtready[i], 1);
+      mbar_init(&mraw[i], 1);
+      mbar_init(&btready[i], 64);
+      mbar_init(&mready[i], 32);
       mbar_init(&dgready[i], 1);
+      mbar_init(&yready[i], 1);
     }
+    for (int i = 0; i < 3; ++i) mbar_init(&vready[i], NCHT);
     mbar_init(gready, NCHT);
-    mbar_init(mraw, 1);
-    mbar_init(mready, 64);
-    mbar_init(dtready, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -738,7 +766,6 @@ __global__ void __launch_bounds__(NTHR, 1)
     tma_prefetch(&tmDL);
     tma_prefetch(&tmG);
     tma_prefetch(&tmBC);
-    tma_prefetch(&tmY);
     tma_prefetch(&tmWD);
   }
   tc_fence_before();
@@ -770,73 +797,142 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
     }
   } else if (warp == 11) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer: a small
+    // dataflow scheduler over four tasks, each issued as soon as its inputs are ready
+    //   stage(ks):   dt projection and C B^T of a landed stage
+    //   chain(kc):   Y = G' C^T, G' += V B (the state products; releases the stage first)
+    //   vm(kv):      Y += V M^T, then Y is complete
+    // Buffer reuse: DT / MR buffer ks & 1 held block ks - 2, consumed before gready /
+    // mready of that block (chain(ks - 2), vm(ks - 2) issued); the stage of block kc holds
+    // nothing the state products read (B^T and the C copy are separate).
     if (lane == 0) {
-      // block k's stage has landed: W_dt dt_low^T and C B^T
-      auto issue_stage = [&](int k) -> bool {
-        const int s = k % ST;
-        if (!mbar_wait(&full[s], (k / ST) & 1u, status, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t dl = sbase + OFF_DL + s * DL_B, wd = sbase + OFF_WD;
-        for (int a = 0; a < ka; ++a)
-          for (int j = 0; j < KA / 16; ++j)
-            umma_bf16_ss(tmem + COL_DT, sdesc_sw128(wd + a * WDC_B + 32 * j, 16, 1024),
-                         sdesc_sw128(dl + a * DLC_B + 32 * j, 16, 1024), IDESC_DT, (a | j) != 0);
-        umma_commit(dtready);
-        // C B^T: A = a C chunk (128 rows read, rows 32..127 land in TMEM lanes nobody
-        // reads), B = the B chunk of the same columns; K = n = 128 = 16 tf32 steps
-        const uint32_t bc = sbase + OFF_BC + s * BC_B;
-        for (int q = 0; q < 4; ++q)
-          for (int j = 0; j < 4; ++j)
-            umma_tf32_ss(tmem + COL_MR, sdesc_sw128(bc + (4 + q) * BCC_B + 32 * j, 16, 1024),
-                         sdesc_sw128(bc + q * BCC_B + 32 * j, 16, 1024), IDESC_Q, (q | j) != 0);
-        umma_commit(mraw);
-        return true;
-      };
-      bool ok = nblk > 0 && issue_stage(0);
-      for (int k = 0; ok && k < nblk; ++k) {
-        const int i = k & 1, s = k % ST;
-        if (!mbar_wait(&vready[i], (k >> 1) & 1u, status, abort_flag) || !mbar_wait(mready, k & 1u, status, abort_flag))
-          break;
-        tc_fence_after();
-        const uint32_t mt = sbase + OFF_MT + i * MT_B, bt = sbase + OFF_BT + i * BT_B;
-        // Y = V M^T (K = s = 32)
-        for (int j = 0; j < 4; ++j)
-          umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_V + 32 * i + 8 * j, sdesc_sw128(mt + 32 * j, 16, 1024),
-                       IDESC_Q, j);
-        // the next block's dt projection and C B^T (their TMEM was read before vready / mready)
-        if (k + 1 < nblk && !issue_stage(k + 1)) break;
-        if (!mbar_wait(gready, k & 1u, status, abort_flag)) break;
-        tc_fence_after();
-        // Y += G' C^T (K = n = 128), then G' += V B (K = s = 32, B^T rows n)
-        const uint32_t bc = sbase + OFF_BC + s * BC_B;
-        for (int q = 0; q < 4; ++q)
-          for (int j = 0; j < 4; ++j)
-            umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_GP + 32 * q + 8 * j,
-                         sdesc_sw128(bc + (4 + q) * BCC_B + 32 * j, 16, 1024), IDESC_Q, 1);
-        for (int j = 0; j < 4; ++j)
-          umma_tf32_ts(tmem + COL_GP, tmem + COL_V + 32 * i + 8 * j, sdesc_sw128(bt + 32 * j, 16, 1024), IDESC_N, 1);
-        umma_commit(&dgready[i]);
-        umma_commit(&empty[s]);
+      int ks = 0, kc = 0, kv = 0;
+      unsigned long long t_last = 0;
+      uint32_t idle = 0;
+      while (kv < nblk) {
+        if (ks < nblk && ks <= kc + 1 && ks <= kv + 1 && mbar_try_wait(&full[ks % ST], (ks / ST) & 1u)) {
+          tc_fence_after();
+          const int s = ks % ST, i = ks & 1;
+          const uint32_t dl = sbase + OFF_DL + s * DL_B, wd = sbase + OFF_WD;
+          for (int a = 0; a < ka; ++a)
+            for (int j = 0; j < KA / 16; ++j)
+              umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_sw128(wd + a * WDC_B + 32 * j, 16, 1024),
+                           sdesc_sw128(dl + a * DLC_B + 32 * j, 16, 1024), IDESC_DT, (a | j) != 0);
+          umma_commit(&dtready[i]);
+          // C B^T: A = a C chunk (128 rows read, rows 32..127 land in TMEM lanes nobody
+          // reads), B = the B chunk of the same columns; K = n = 128 = 16 tf32 steps
+          const uint32_t bc = sbase + OFF_BC + s * BC_B;
+          for (int q = 0; q < 4; ++q)
+            for (int j = 0; j < 4; ++j)
+              umma_tf32_ss(tmem + COL_MR + 32 * i, sdesc_sw128(bc + (4 + q) * BCC_B + 32 * j, 16, 1024),
+                           sdesc_sw128(bc + q * BCC_B + 32 * j, 16, 1024), IDESC_Q, (q | j) != 0);
+          umma_commit(&mraw[i]);
+          ++ks;
+          idle = 0;
+          continue;
+        }
+        if (kc < ks && mbar_try_wait(&vready[kc % 3], (kc / 3) & 1u) &&
+            mbar_try_wait(&btready[kc & 1], (kc >> 1) & 1u) && mbar_try_wait(gready, kc & 1u)) {
+          tc_fence_after();
+          // the stage of block kc: its dt projection and C B^T were issued before (their
+          // completion is what the commit tracks), x and gate were read before vready,
+          // B and C copied before btready
+          umma_commit(&empty[kc % ST]);
+          if (!sAny[kc % 3]) {
+            const int i = kc & 1, vb = kc % 3;
+            const uint32_t cc = sbase + OFF_CC + i * CC_B, bt = sbase + OFF_BT + i * BT_B;
+            // Y = G' C^T (K = n = 128), then G' += V B (K = s = 32, B^T rows n)
+            for (int q = 0; q < 4; ++q)
+              for (int j = 0; j < 4; ++j)
+                umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_GP + 32 * q + 8 * j,
+                             sdesc_sw128(cc + q * BCC_B + 32 * j, 16, 1024), IDESC_Q, (q | j) != 0);
+            for (int j = 0; j < 4; ++j)
+              umma_tf32_ts(tmem + COL_GP, tmem + COL_V + 32 * vb + 8 * j, sdesc_sw128(bt + 32 * j, 16, 1024), IDESC_N,
+                           1);
+          }
+          umma_commit(&dgready[kc & 1]);
+          ++kc;
+          idle = 0;
+          continue;
+        }
+        if (kv < kc && mbar_try_wait(&mready[kv & 1], (kv >> 1) & 1u)) {
+          tc_fence_after();
+          if (!sAny[kv % 3]) {  // Y += V M^T (K = s = 32)
+            const int i = kv & 1, vb = kv % 3;
+            const uint32_t mt = sbase + OFF_MT + i * MT_B;
+            for (int j = 0; j < 4; ++j)
+              umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_V + 32 * vb + 8 * j, sdesc_sw128(mt + 32 * j, 16, 1024),
+                           IDESC_Q, 1);
+          }
+          umma_commit(&yready[kv & 1]);
+          ++kv;
+          idle = 0;
+          continue;
+        }
+        // nothing ready: back off briefly, give up after kWaitLimitNs without progress
+        ++idle;
+        if (idle > 8u) __nanosleep(32);
+        if ((idle & 63u) == 0u) {
+          if (*abort_flag) break;
+          const unsigned long long now = globaltimer();
+          if (idle == 64u) {
+            t_last = now;
+          } else if (now - t_last > kWaitLimitNs) {
+            atomicExch(status, kStatusTimeout);
+            *abort_flag = 1;
+            break;
+          }
+        }
       }
       umma_commit(mma_done);
       int never = 0;
       mbar_wait(mma_done, 0, nullptr, &never, 100000000ull);
     }
   } else if (warp >= 8) {
-    // ------------------------------------------------------------ M = mask(C B^T), B^T
+    // ------------------------------------------------------------ B^T, the C copy, M
     const int wq = warp - 8;
     for (int k = 0; k < nblk; ++k) {
       const int s = k % ST, i = k & 1;
-      bool ok = mbar_wait(mraw, k & 1u, status, abort_flag) && mbar_wait(&full[s], (k / ST) & 1u, status, abort_flag);
-      // this buffer of M and B^T was last read by block k - 2's products
+      bool ok = mbar_wait(&full[s], (k / ST) & 1u, status, abort_flag);
+      // B^T / C copy buffer i was last read by block k - 2's state products
       if (ok && k >= 2) ok = mbar_wait(&dgready[i], ((k - 2) >> 1) & 1u, status, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
+      const uint8_t* stg = sm + OFF_BC + s * BC_B;
+      {  // B^T [n][s] for n in [64 wq, 64 wq + 64), s = lane
+        const int sr = lane;
+        const uint8_t* src = stg + (sr >> 3) * 1024 + (sr & 7) * 128;
+        uint8_t* bt = sm + OFF_BT + i * BT_B;
+#pragma unroll 4
+        for (int nn = 0; nn < 64; nn += 4) {
+          const int n = 64 * wq + nn;
+          const float4 v = *reinterpret_cast<const float4*>(src + (n >> 5) * BCC_B + ((((n & 31) >> 2) ^ (sr & 7)) << 4));
+          const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) *reinterpret_cast<uint32_t*>(bt + bt_off(n + e, sr)) = tf32_round(vv[e]);
+        }
+      }
+      {  // C chunks 2 wq, 2 wq + 1 (same layout), rounded to tf32
+        const uint4* src = reinterpret_cast<const uint4*>(stg + (4 + 2 * wq) * BCC_B);
+        uint4* dst = reinterpret_cast<uint4*>(sm + OFF_CC + i * CC_B + 2 * wq * BCC_B);
+#pragma unroll 4
+        for (int j = lane; j < 2 * BCC_B / 16; j += 32) {
+          const uint4 v = src[j];
+          dst[j] = make_uint4(tf32_round(__uint_as_float(v.x)), tf32_round(__uint_as_float(v.y)),
+                              tf32_round(__uint_as_float(v.z)), tf32_round(__uint_as_float(v.w)));
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&btready[i]);
       if (wq == 0) {  // row t = lane of M (K-major, 128-byte swizzle), from TMEM lanes 0-31
+        ok = mbar_wait(&mraw[i], (k >> 1) & 1u, status, abort_flag);
+        // M buffer i was last read by block k - 2's V M^T
+        if (ok && k >= 2) ok = mbar_wait(&yready[i], ((k - 2) >> 1) & 1u, status, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
         const int t = lane;
         uint32_t r[32];
-        tmem_ld32(tmem + COL_MR, r);
+        tmem_ld32(tmem + COL_MR + 32 * i, r);
         tmem_wait_ld();
         uint8_t* row = sm + OFF_MT + i * MT_B + (t >> 3) * 1024 + (t & 7) * 128;
 #pragma unroll
@@ -846,28 +942,10 @@ __global__ void __launch_bounds__(NTHR, 1)
           for (int e = 0; e < 4; ++e) v[e] = 4 * j + e <= t ? tf32_round(__uint_as_float(r[4 * j + e])) : 0u;
           *reinterpret_cast<uint4*>(row + ((j ^ (t & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&mready[i]);
       }
-      // B^T [n][s] for n in [64 wq, 64 wq + 64), s = lane
-      {
-        const int sr = lane;
-        const uint8_t* src = sm + OFF_BC + s * BC_B + (sr >> 3) * 1024 + (sr & 7) * 128;
-        uint8_t* bt = sm + OFF_BT + i * BT_B;
-#pragma unroll 4
-        for (int nn = 0; nn < 64; nn += 4) {
-          const int n = 64 * wq + nn;
-          const float4 v = *reinterpret_cast<const float4*>(src + (n >> 5) * BCC_B + ((((n & 31) >> 2) ^ (sr & 7)) << 4));
-          const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int ne = n + e;
-            *reinterpret_cast<uint32_t*>(bt + (ne >> 3) * 1024 + (ne & 7) * 128 + (((sr >> 2) ^ (ne & 7)) << 4) +
-                                         (sr & 3) * 4) = tf32_round(vv[e]);
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(mready);
     }
   } else {
     // ------------------------------------------------------------ channel warps
@@ -876,6 +954,8 @@ __global__ void __launch_bounds__(NTHR, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const float A2 = c < Di ? expf(a_log[c]) * 1.4426950408889634f : 0.f;  // |A| / ln 2
     const float bdt = c < Di ? b_dt[c] : 0.f;
+    __nv_bfloat16* ycol = y + static_cast<long long>(b) * T * y_ld + c;
+    bool fail = false;
     // the state entering row t0 (raw: the first block applies only its own scale)
 #pragma unroll 1
     for (int part = 0; part < 2; ++part) {
@@ -898,204 +978,243 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     tmem_wait_st();
     tc_fence_before();
+
+    // dt of block k's half (steps past T: dt = 0, the state stays), from W_dt dt_low^T
+    auto load_dt = [&](int k, float (&dtv)[HQ]) {
+      uint32_t z[HQ];
+      tmem_ld16(tl + COL_DT + 32 * (k & 1) + HQ * half, z);
+      tmem_wait_ld();
+      const int t_end = T - (t0 + k * Q + HQ * half);
+#pragma unroll
+      for (int j = 0; j < HQ; j += 2) {
+        float2 d = softplus2(make_float2(__uint_as_float(z[j]) + bdt, __uint_as_float(z[j + 1]) + bdt));
+        if (j >= t_end) d.x = 0.f;
+        if (j + 1 >= t_end) d.y = 0.f;
+        dtv[j] = d.x;
+        dtv[j + 1] = d.y;
+      }
+    };
+    // V and W of block k into TMEM buffer k % 3: V = dt x 2^(lambda - r), W = gate
+    // 2^(r - lambda), or for a block that runs the plain recurrence V = dt x, W = gate.
+    // Returns the block's flag and this channel's two half-block decay sums.
+    auto form_vw = [&](int k, float& S0, float& S1) -> bool {
+      const int s = k % ST, vb = k % 3;
+      fail = fail || !__all_sync(0xffffffffu, mbar_wait(&full[s], (k / ST) & 1u, status, abort_flag) &&
+                                                  mbar_wait(&dtready[k & 1], (k >> 1) & 1u, status, abort_flag));
+      float dtv[HQ];
+      if (!fail) {
+        tc_fence_after();
+        load_dt(k, dtv);
+      } else {
+#pragma unroll
+        for (int j = 0; j < HQ; ++j) dtv[j] = 0.f;
+      }
+      float2 S2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < HQ; j += 2) S2 = __ffma2_rn(make_float2(A2, A2), make_float2(dtv[j], dtv[j + 1]), S2);
+      const float S = S2.x + S2.y;
+      float* ss = sS + (k & 1) * 2 * CH;
+      ss[half * CH + cl] = S;
+      const bool any = bar_red_or(1, NCHT, fail || !(S <= kRange));
+      S0 = ss[cl];
+      S1 = ss[CH + cl];
+      if (!fail) {
+        const uint8_t* xt = sm + OFF_X + s * TILE_B + cl * 2 + HQ * half * 256;
+        const uint8_t* gt = sm + OFF_G + s * TILE_B + cl * 2 + HQ * half * 256;
+        uint32_t vr[HQ], wr[HQ];
+        float mu = half ? 0.f : -S;  // lambda - r
+#pragma unroll
+        for (int j = 0; j < HQ; j += 2) {
+          const float2 xv = make_float2(bf2f(*reinterpret_cast<const uint16_t*>(xt + j * 256)),
+                                        bf2f(*reinterpret_cast<const uint16_t*>(xt + (j + 1) * 256)));
+          const float2 gv = make_float2(bf2f(*reinterpret_cast<const uint16_t*>(gt + j * 256)),
+                                        bf2f(*reinterpret_cast<const uint16_t*>(gt + (j + 1) * 256)));
+          const float2 u = __fmul2_rn(make_float2(dtv[j], dtv[j + 1]), xv);
+          if (!any) {
+            const float mu0 = fmaf(A2, dtv[j], mu);
+            mu = fmaf(A2, dtv[j + 1], mu0);
+            const float2 v = __fmul2_rn(u, make_float2(ex2_approx(mu0), ex2_approx(mu)));
+            const float2 w = __fmul2_rn(gv, make_float2(ex2_approx(-mu0), ex2_approx(-mu)));
+            vr[j] = tf32_round(v.x);
+            vr[j + 1] = tf32_round(v.y);
+            wr[j] = __float_as_uint(w.x);
+            wr[j + 1] = __float_as_uint(w.y);
+          } else {
+            vr[j] = __float_as_uint(u.x);
+            vr[j + 1] = __float_as_uint(u.y);
+            wr[j] = __float_as_uint(gv.x);
+            wr[j + 1] = __float_as_uint(gv.y);
+          }
+        }
+        tmem_st16(tl + COL_V + 32 * vb + HQ * half, vr);
+        tmem_st16(tl + COL_W + 32 * vb + HQ * half, wr);
+        tmem_wait_st();
+      }
+      if (threadIdx.x == 0) sAny[vb] = any ? 1 : 0;
+      tc_fence_before();
+      mbar_arrive(&vready[vb]);
+      return any;
+    };
+
+    float cS0 = 0.f, cS1 = 0.f;
+    bool c_any = nblk > 0 ? form_vw(0, cS0, cS1) : false;
     float pS1 = 0.f;        // the previous block's second-half decay sum
     bool prev_any = true;   // the previous block left the raw state in G' (so does the start)
-    for (int k = 0; k <= nblk; ++k) {
-      bool fail = false, any = false;
-      if (k < nblk) {
-        const int s = k % ST, i = k & 1;
-        const uint8_t* xt = sm + OFF_X + s * TILE_B + cl * 2;
-        const uint8_t* gt = sm + OFF_G + s * TILE_B + cl * 2;
-        fail = !__all_sync(0xffffffffu, mbar_wait(&full[s], (k / ST) & 1u, status, abort_flag));
-        if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(dtready, k & 1u, status, abort_flag));
-        // ---- dt of this half block (steps past T: dt = 0, the state stays) and its decay sum
-        uint32_t z[16];
-        if (!fail) {
-          tc_fence_after();
-          tmem_ld16(tl + COL_DT + 16 * half, z);
+    for (int k = 0; k < nblk; ++k) {
+      // ---- G' for block k: block k - 1's state products are done
+      if (k > 0 && !fail)
+        fail = !__all_sync(0xffffffffu, mbar_wait(&dgready[(k - 1) & 1], ((k - 1) >> 1) & 1u, status, abort_flag));
+      if (!fail) {
+        // G' <- 2^-e_in 2^-e_out G'; one multiply while 2^-(e_in + e_out) is a normal float
+        const float e_in = prev_any ? 0.f : pS1, e_out = c_any ? 0.f : cS0;
+        const bool one = __all_sync(0xffffffffu, e_in + e_out < 120.f);
+        const float f1 = ex2_approx(one ? -(e_in + e_out) : -e_in), f2 = one ? 1.f : ex2_approx(-e_out);
+        const float2 fa = make_float2(f1, f1), fb = make_float2(f2, f2);
+        tc_fence_after();
+#pragma unroll 1
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t col = tl + COL_GP + 64 * half + 32 * part;
+          uint32_t g[32];
+          tmem_ld32(col, g);
           tmem_wait_ld();
-        } else {
+          if (one) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) z[j] = 0u;
-        }
-        const int t_end = T - (t0 + k * Q + HQ * half);
-        float dtv[16];
-        float2 S2 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          float2 d = softplus2(make_float2(__uint_as_float(z[j]) + bdt, __uint_as_float(z[j + 1]) + bdt));
-          if (j >= t_end) d.x = 0.f;
-          if (j + 1 >= t_end) d.y = 0.f;
-          dtv[j] = d.x;
-          dtv[j + 1] = d.y;
-          S2 = __ffma2_rn(make_float2(A2, A2), d, S2);
-        }
-        const float S = S2.x + S2.y;
-        sS[half * CH + cl] = S;
-        any = bar_red_or(1, NCHT, fail || !(S <= kRange));
-        const float S0 = sS[cl], S1 = sS[CH + cl];
-        // ---- V = dt x 2^(lambda - r), W = gate 2^(r - lambda); a plain block: V = 0, W = dt.
-        // Their buffer was last read by block k - 2, complete (dgready) before iteration k - 1 ended.
-        if (!fail) {
-          uint32_t vr[16], wr[16];
-          if (!any) {
-            float mu = half ? 0.f : -S;  // lambda - r
-#pragma unroll
-            for (int j = 0; j < 16; j += 2) {
-              const float mu0 = fmaf(A2, dtv[j], mu);
-              mu = fmaf(A2, dtv[j + 1], mu0);
-              const int row = (HQ * half + j) * 256;
-              const float2 xv = make_float2(bf2f(*reinterpret_cast<const uint16_t*>(xt + row)),
-                                            bf2f(*reinterpret_cast<const uint16_t*>(xt + row + 256)));
-              const float2 gv = make_float2(bf2f(*reinterpret_cast<const uint16_t*>(gt + row)),
-                                            bf2f(*reinterpret_cast<const uint16_t*>(gt + row + 256)));
-              const float2 e = make_float2(ex2_approx(mu0), ex2_approx(mu));
-              const float2 v = __fmul2_rn(__fmul2_rn(make_float2(dtv[j], dtv[j + 1]), xv), e);
-              const float2 w = __fmul2_rn(gv, make_float2(ex2_approx(-mu0), ex2_approx(-mu)));
-              vr[j] = tf32_round(v.x);
-              vr[j + 1] = tf32_round(v.y);
-              wr[j] = __float_as_uint(w.x);
-              wr[j + 1] = __float_as_uint(w.y);
+            for (int j = 0; j < 32; j += 2) {
+              const float2 v = __fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa);
+              g[j] = __float_as_uint(v.x);
+              g[j + 1] = __float_as_uint(v.y);
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              vr[j] = 0u;
-              wr[j] = __float_as_uint(dtv[j]);
+            for (int j = 0; j < 32; j += 2) {
+              const float2 v =
+                  __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa), fb);
+              g[j] = __float_as_uint(v.x);
+              g[j + 1] = __float_as_uint(v.y);
             }
           }
-          tc_fence_after();
-          tmem_st16(tl + COL_V + 32 * i + HQ * half, vr);
-          tmem_st16(tl + COL_W + 32 * i + HQ * half, wr);
-          tmem_wait_st();
-          tc_fence_before();
+          tmem_st32(col, g);
         }
-        mbar_arrive(&vready[i]);
-        // ---- G' for block k: block k - 1's products are done (G' advanced, Y complete)
-        if (k > 0 && !fail)
-          fail = !__all_sync(0xffffffffu, mbar_wait(&dgready[(k - 1) & 1], ((k - 1) >> 1) & 1u, status, abort_flag));
-        if (!fail) {
-          const float f_in = prev_any ? 1.f : ex2_approx(-pS1), f_out = any ? 1.f : ex2_approx(-S0);
+        tmem_wait_st();
+      }
+      // ---- large decays: the plain recurrence over block k on the raw state in G'
+      if (c_any) {
+        tc_fence_before();
+        bar_sync_n(1, NCHT);  // both halves' G' columns are stored
+        const int i = k & 1, vb = k % 3;
+        if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(&btready[i], (k >> 1) & 1u, status, abort_flag));
+        if (half == 1 && !fail) {
           tc_fence_after();
+          const uint8_t* bt = sm + OFF_BT + i * BT_B;
+          const uint8_t* cc = sm + OFF_CC + i * CC_B;
 #pragma unroll 1
-          for (int part = 0; part < 2; ++part) {
-            const uint32_t col = tl + COL_GP + 64 * half + 32 * part;
-            uint32_t g[32];
-            tmem_ld32(col, g);
+          for (int th = 0; th < Q; th += HQ) {
+            uint32_t zq[HQ], uq[HQ], gq[HQ];
+            tmem_ld16(tl + COL_DT + 32 * i + th, zq);
+            tmem_ld16(tl + COL_V + 32 * vb + th, uq);
+            tmem_ld16(tl + COL_W + 32 * vb + th, gq);
             tmem_wait_ld();
+            const int t_end = T - (t0 + k * Q + th);
+            float a[HQ], y16[HQ];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) g[j] = __float_as_uint((__uint_as_float(g[j]) * f_in) * f_out);
-            tmem_st32(col, g);
-          }
-          tmem_wait_st();
-          tc_fence_before();
-        }
-        // ---- large decays: the plain recurrence over the block on the raw state in G',
-        // y straight into the y tile.  G' is announced only after it.
-        if (any) {
-          if (threadIdx.x == 0) bulk_wait_all();  // the store that last read this y tile is done
-          bar_sync_n(1, NCHT);                    // both halves' dt and G' columns are in TMEM
-          if (half == 1 && !fail) {
-            tc_fence_after();
-            const uint8_t* bct = sm + OFF_BC + s * BC_B;
-            uint8_t* yt = sm + OFF_Y + i * TILE_B + cl * 2;
-            // 16 steps at a time over the four 32-column pieces of the state
+            for (int j = 0; j < HQ; ++j) {
+              const float dt = j < t_end ? softplus_f(__uint_as_float(zq[j]) + bdt) : 0.f;
+              a[j] = ex2_approx(-A2 * dt);
+              y16[j] = 0.f;
+            }
 #pragma unroll 1
-            for (int th = 0; th < Q; th += HQ) {
-              uint32_t dq[HQ];
-              tmem_ld16(tl + COL_W + 32 * i + th, dq);
+            for (int q = 0; q < 4; ++q) {
+              uint32_t hr[32];
+              tmem_ld32(tl + COL_GP + 32 * q, hr);
               tmem_wait_ld();
-              float y[HQ];
+              float h[32];
 #pragma unroll
-              for (int t = 0; t < HQ; ++t) y[t] = 0.f;
+              for (int j = 0; j < 32; ++j) h[j] = __uint_as_float(hr[j]);
 #pragma unroll 1
-              for (int q = 0; q < 4; ++q) {
-                uint32_t hr[32];
-                tmem_ld32(tl + COL_GP + 32 * q, hr);
-                tmem_wait_ld();
-                float h[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) h[j] = __uint_as_float(hr[j]);
-#pragma unroll
-                for (int tt = 0; tt < HQ; ++tt) {
-                  const int t = th + tt;
-                  const float dt = __uint_as_float(dq[tt]);
-                  const float xv = bf2f(*reinterpret_cast<const uint16_t*>(xt + t * 256));
-                  const float a = ex2_approx(-A2 * dt), u = dt * xv;
-                  const uint8_t* brow = bct + q * BCC_B + (t >> 3) * 1024 + (t & 7) * 128;
-                  const uint8_t* crow = brow + 4 * BCC_B;
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) {
-                    const float4 bq = *reinterpret_cast<const float4*>(brow + ((j ^ (t & 7)) << 4));
-                    const float4 cq = *reinterpret_cast<const float4*>(crow + ((j ^ (t & 7)) << 4));
-                    h[4 * j + 0] = fmaf(a, h[4 * j + 0], u * bq.x);
-                    h[4 * j + 1] = fmaf(a, h[4 * j + 1], u * bq.y);
-                    h[4 * j + 2] = fmaf(a, h[4 * j + 2], u * bq.z);
-                    h[4 * j + 3] = fmaf(a, h[4 * j + 3], u * bq.w);
-                    y[tt] = fmaf(cq.x, h[4 * j + 0], y[tt]);
-                    y[tt] = fmaf(cq.y, h[4 * j + 1], y[tt]);
-                    y[tt] = fmaf(cq.z, h[4 * j + 2], y[tt]);
-                    y[tt] = fmaf(cq.w, h[4 * j + 3], y[tt]);
-                  }
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) hr[j] = __float_as_uint(h[j]);
-                tmem_st32(tl + COL_GP + 32 * q, hr);
-                tmem_wait_st();
-              }
-#pragma unroll
               for (int tt = 0; tt < HQ; ++tt) {
                 const int t = th + tt;
-                const float gv = bf2f(*reinterpret_cast<const uint16_t*>(gt + t * 256));
-                *reinterpret_cast<uint16_t*>(yt + t * 256) = bf16_bits(gv * y[tt]);
+                const float u = __uint_as_float(uq[tt]);
+                float acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                  const float4 cv = *reinterpret_cast<const float4*>(cc + cc_off(t, 32 * q + j));
+                  const float cq[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const float bn = *reinterpret_cast<const float*>(bt + bt_off(32 * q + j + e, t));
+                    h[j + e] = fmaf(a[tt], h[j + e], u * bn);
+                    acc = fmaf(cq[e], h[j + e], acc);
+                  }
+                }
+                y16[tt] += acc;
+              }
+#pragma unroll
+              for (int j = 0; j < 32; ++j) hr[j] = __float_as_uint(h[j]);
+              tmem_st32(tl + COL_GP + 32 * q, hr);
+              tmem_wait_st();
+            }
+            if (c < Di) {
+#pragma unroll
+              for (int j = 0; j < HQ; ++j) {
+                const int t = t0 + k * Q + th + j;
+                if (t < T) ycol[static_cast<long long>(t) * y_ld] = __float2bfloat16_rn(__uint_as_float(gq[j]) * y16[j]);
               }
             }
-            tc_fence_before();
           }
         }
-        mbar_arrive(gready);
-        pS1 = S1;
       }
-      // ---- output of block k - 1: y = W * Y into the y tile, TMA store
-      if (k > 0) {
+      tc_fence_before();
+      mbar_arrive(gready);
+      // ---- output of block k - 1: y = W * Y
+      if (k > 0 && !prev_any) {
         const int jb = k - 1, i = jb & 1;
-        // after the last block no barrier has followed thread 0's wait for the store that
-        // last read this y tile: meet one
-        if (k == nblk) bar_sync_n(1, NCHT);
-        if (k == nblk && !fail)
-          fail = !__all_sync(0xffffffffu, mbar_wait(&dgready[i], (jb >> 1) & 1u, status, abort_flag));
-        if (!fail && !prev_any) {
+        if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(&yready[i], (jb >> 1) & 1u, status, abort_flag));
+        if (!fail) {
           tc_fence_after();
-          uint32_t yv[16], wv[16];
+          uint32_t yv[HQ], wv[HQ];
           tmem_ld16(tl + COL_Y + 32 * i + HQ * half, yv);
-          tmem_ld16(tl + COL_W + 32 * i + HQ * half, wv);
+          tmem_ld16(tl + COL_W + 32 * (jb % 3) + HQ * half, wv);
           tmem_wait_ld();
-          uint8_t* yt = sm + OFF_Y + i * TILE_B + cl * 2 + HQ * half * 256;
+          if (c < Di) {
+            const int tb = t0 + jb * Q + HQ * half;
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const float2 o = __fmul2_rn(make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])),
-                                        make_float2(__uint_as_float(wv[j]), __uint_as_float(wv[j + 1])));
-            const uint32_t p2 = pack_bf16(o.x, o.y);
-            *reinterpret_cast<uint16_t*>(yt + j * 256) = static_cast<uint16_t>(p2);
-            *reinterpret_cast<uint16_t*>(yt + (j + 1) * 256) = static_cast<uint16_t>(p2 >> 16);
+            for (int j = 0; j < HQ; ++j)
+              if (tb + j < T)
+                ycol[static_cast<long long>(tb + j) * y_ld] =
+                    __float2bfloat16_rn(__uint_as_float(yv[j]) * __uint_as_float(wv[j]));
           }
         }
-        fence_proxy_async_smem();
-        if (bar_red_or(1, NCHT, fail || *abort_flag)) break;
-        if (threadIdx.x == 0) {
-          tma_store_3d(&tmY, sm + OFF_Y + i * TILE_B, c0, t0 + jb * Q, b);
-          bulk_commit();
-          bulk_wait_read1();  // the store before it has read its tile: that tile may be rewritten
-        }
-      } else if (fail) {
-        if (bar_red_or(1, NCHT, true)) break;
-      } else {
-        if (bar_red_or(1, NCHT, *abort_flag != 0)) break;
       }
-      if (k < nblk) prev_any = any;
-      if (k == nblk && h_out) {  // warp-uniform (tcgen05.ld is warp-collective)
-        // the state after the last row: 2^-S1 (G' + dG) after a product-form block, the
-        // raw state after a plain one (its products added V = 0)
+      pS1 = cS1;
+      prev_any = c_any;
+      // ---- V and W of block k + 1 (their buffer's last reader, block k - 2's V M^T,
+      // completed before the output of block k - 2 above, an iteration ago)
+      if (k + 1 < nblk) c_any = form_vw(k + 1, cS0, cS1);
+      if (bar_red_or(1, NCHT, fail || *abort_flag)) break;
+    }
+    // ---- output of the last block and the state after the last row
+    if (__all_sync(0xffffffffu, !fail && nblk > 0 && !*abort_flag)) {
+      const int jb = nblk - 1, i = jb & 1;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&dgready[i], (jb >> 1) & 1u, status, abort_flag));
+      if (got && !prev_any) {
+        if (__all_sync(0xffffffffu, mbar_wait(&yready[i], (jb >> 1) & 1u, status, abort_flag))) {
+          tc_fence_after();
+          uint32_t yv[HQ], wv[HQ];
+          tmem_ld16(tl + COL_Y + 32 * i + HQ * half, yv);
+          tmem_ld16(tl + COL_W + 32 * (jb % 3) + HQ * half, wv);
+          tmem_wait_ld();
+          if (c < Di) {
+            const int tb = t0 + jb * Q + HQ * half;
+#pragma unroll
+            for (int j = 0; j < HQ; ++j)
+              if (tb + j < T)
+                ycol[static_cast<long long>(tb + j) * y_ld] =
+                    __float2bfloat16_rn(__uint_as_float(yv[j]) * __uint_as_float(wv[j]));
+          }
+        }
+      }
+      if (got && h_out) {
+        // 2^-S1 (G' + dG) after a product-form block, the raw state after a plain one
         const float f = prev_any ? 1.f : ex2_approx(-pS1);
         tc_fence_after();
 #pragma unroll 1
@@ -1113,8 +1232,12 @@ __global__ void __launch_bounds__(NTHR, 1)
           }
         }
       }
+    } else if (nblk == 0 && h_out && c < Di && h0) {
+      // no rows to scan: the state passes through
+      const float* hp = h0 + b * h0_bstride + static_cast<long long>(c) * NS + 64 * half;
+      float* ho = h_out + (static_cast<long long>(b) * Di + c) * NS + 64 * half;
+      for (int j = 0; j < 64; ++j) ho[j] = hp[j];
     }
-    if (threadIdx.x == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -1125,12 +1248,11 @@ __global__ void __launch_bounds__(NTHR, 1)
 }
 
 cudaError_t launch_tc128(const ScanDesc& s, cudaStream_t st) {
-  CUtensorMap tx, td, tg, tb, ty, tw;
+  CUtensorMap tx, td, tg, tb, tw;
   const bool ok =
       map3d(&tx, s.x, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
       map3d(&tg, s.gate, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
       map3d(&tb, s.bc, true, s.batch, s.T, 2 * NS, 2 * NS, 32, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
-      map3d(&ty, s.y, false, s.batch, s.T, s.d_inner, s.y_ld, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
       map3d(&td, s.dt_low, false, s.batch, s.T, s.dt_rank, s.dt_rank, KA, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
       map2d_sw128(&tw, s.w_dt, s.d_inner, s.dt_rank, s.dt_rank, KA, CH);
   if (!ok) return cudaErrorNotSupported;
@@ -1138,8 +1260,9 @@ cudaError_t launch_tc128(const ScanDesc& s, cudaStream_t st) {
   if (cudaError_t e = smem_attr_once(scan_tc128_kernel, SMEM_TOTAL, attr_done)) return e;
   const int ka = (s.dt_rank + KA - 1) / KA;
   dim3 grid((s.d_inner + CH - 1) / CH, s.batch);
-  return launch(scan_tc128_kernel, grid, dim3(NTHR), SMEM_TOTAL, st, tx, td, tg, tb, ty, tw, s.a_log, s.b_dt, s.T,
-                s.d_inner, ka, s.h_out, s.t0, s.h0, s.h0_bstride, s.status);
+  return launch(scan_tc128_kernel, grid, dim3(NTHR), SMEM_TOTAL, st, tx, td, tg, tb, tw, s.a_log, s.b_dt,
+                static_cast<__nv_bfloat16*>(s.y), s.y_ld, s.T, s.d_inner, ka, s.h_out, s.t0, s.h0, s.h0_bstride,
+                s.status);
 }
 }  // namespace t128
 

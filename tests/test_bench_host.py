@@ -74,7 +74,7 @@ def test_stage_rooflines_sum_layers_and_pick_the_binding_resource():
     exp = 0.0
     for s in wl.layers:
         for k, (fl, by) in bench.stage_work(s).items():
-            b = bench.stage_bound(k, s)
+            b = bench.stage_bound(k, s, (fl, by), peaks)
             exp += max(fl / 1600e12 if b == "tensor" else 0.0, by / 6000e9, fl / alu if b == "alu" else 0.0)
     assert abs(t_us - exp * 1e6) < 1e-6 * t_us
     s16 = synth.workload("hymba350m_layer").first
@@ -92,3 +92,15 @@ def test_stack_roofline_counts_the_ffn():
     fl, _ = bench.ffn_work(wl.layers[0])
     assert fl == 6.0 * 2048 * 5632 * wl.first.batch * wl.first.T
     assert with_ffn - no_ffn >= 2 * fl / 1600e12 * 1e6 * 0.999
+
+
+def test_gemm_stage_bound_is_the_longer_of_flop_and_byte_time():
+    """x_proj of the 1.5B pair (N = 128 + 2 x 128) is FLOP-bound at these peaks; a GEMM
+    whose bytes dominate is held to HBM; with no work given a GEMM counts as tensor."""
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0}
+    s = synth.workload("hymba1p5b_kvpair").first
+    fl, by = bench.stage_work(s)["x_proj"]
+    assert fl / 1600e12 > by / 6000e9
+    assert bench.stage_bound("x_proj", s, (fl, by), peaks) == "tensor"
+    assert bench.stage_bound("x_proj", s, (fl, 1e3 * by), peaks) == "hbm"
+    assert bench.stage_bound("out_proj", s) == "tensor"

@@ -19,9 +19,10 @@ from gpu_util import assert_close, dev, requires_cuda, status_ok, to_np
 pytestmark = [pytest.mark.gpu, requires_cuda]
 
 
-def _prefixed_chain(wl, x, meta, dps):
+def _prefixed_chain(wl, x, meta, dps, every_layer=False):
     """Every layer of the workload through records + prefixed calls (a pair: the consumer's
-    record from the producer's record rows and K/V)."""
+    record from the producer's record rows and K/V).  The last layer's output, or
+    (every_layer) each layer's output and the shared K/V."""
     layers = wl.layers
     s0 = layers[0]
     dt = s0.dtype
@@ -48,6 +49,8 @@ def _prefixed_chain(wl, x, meta, dps):
                                            cfgs[i], kv, None, o2, ws), f"prefixed {i}")
         outs.append(o2)
     status_ok(ws)
+    if every_layer:
+        return [to_np(o) for o in outs], (None if kv is None else to_np(kv))
     return to_np(outs[-1])
 
 
@@ -86,24 +89,32 @@ def test_prefixed_layer_is_bit_identical_to_the_full_layer():
 
 
 def test_prefixed_kv_pair_swa_dstate128_matches_oracle_and_full_path():
-    """Each layer of the pair against the oracle on the inputs that layer saw: the producer
-    on X and meta, the consumer on the producer's GPU output rows and K/V.  (Fed the
+    """Each layer of the pair on the inputs that layer saw.  Against the oracle (2e-2): the
+    producer on X and meta, the consumer on the producer's GPU output rows and K/V (fed the
     oracle's own fp64 producer output instead, the consumer differs by ~1e-2 from
-    bf16-rounding that input alone: the pair amplifies input rounding, so a chained
-    comparison would test the conditioning, not the consumer.)"""
+    bf16-rounding that input alone: the pair amplifies input rounding).  Against the full
+    path (2e-3): the prefixed producer with hymba_layer_fwd on the same X, the prefixed
+    consumer with hymba_layer_fwd on the prefixed producer's output and K/V."""
     wl = synth.workload("hymba1p5b_kvpair", batch=2, seq_len=400, window=96, d_model=512, n_q_heads=8,
                         n_kv_heads=2, d_inner=512, dt_rank=32)
     x, meta, ps, dps = _setup(wl)
-    s0 = wl.first
-    g = _prefixed_chain(wl, x, meta, dps)
-    (h_gpu, full), kv_gpu = _plain_chain(wl, x, meta, dps, every_layer=True)
+    s0, s1 = wl.layers
+    (p0, p1), kv_p = _prefixed_chain(wl, x, meta, dps, every_layer=True)
+    (h_gpu, _), _ = _plain_chain(wl, x, meta, dps, every_layer=True)
     h, _ = O.layer_forward(x, meta, ps[0], s0)
-    assert_close(h_gpu, h, "bf16", "producer vs oracle")
-    kv_b = kv_gpu.reshape(2, s0.batch, s0.T, s0.kv_width)
-    ref, _ = O.layer_forward(h_gpu, None, ps[1], wl.layers[1], kv_in=(kv_b[0], kv_b[1]))
-    assert_close(full, ref, "bf16", "consumer (full path) vs oracle")
-    assert_close(g, ref, "bf16", "prefixed pair vs oracle")
-    assert_close(g, full, "bf16", "prefixed pair vs the full path", tol=2e-3)
+    assert_close(h_gpu, h, "bf16", "producer (full path) vs oracle")
+    assert_close(p0, h, "bf16", "prefixed producer vs oracle")
+    assert_close(p0, h_gpu, "bf16", "prefixed producer vs the full path", tol=2e-3)
+    kv_b = kv_p.reshape(2, s0.batch, s0.T, s0.kv_width)
+    ref, _ = O.layer_forward(p0, None, ps[1], s1, kv_in=(kv_b[0], kv_b[1]))
+    assert_close(p1, ref, "bf16", "prefixed consumer vs oracle")
+    cfg1 = H.make_cfg(s1)
+    ws = host.workspace(H.hymba_workspace_size(cfg1))
+    full1 = host.empty((s0.batch, s0.T, s0.d_model), "bf16")
+    H.check(H.hymba_layer_fwd(dev(p0, "bf16"), None, H.make_weights(dps[1]), cfg1, dev(kv_p, "bf16"), None, full1, ws),
+            "consumer full path")
+    status_ok(ws)
+    assert_close(p1, to_np(full1), "bf16", "prefixed consumer vs the full path on the same input", tol=2e-3)
 
 
 @pytest.mark.parametrize("a_per_state", [0, 1])
