@@ -203,19 +203,20 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       // ---------------------------------------------------------------- UMMA issuer
       bool ok = mbar_wait(q_full, 0, p.status, abort_flag);
-      const uint32_t q_addr = smem_u32(sQ);
+      // descriptors of the Q tile and the first K, P and V tiles; the rest are fixed offsets
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024), dK = sdesc_sw128(smem_u32(sK), 16, 1024),
+                     dP = sdesc_sw128(smem_u32(sP), 16, 1024), dV = sdesc_sw128(smem_u32(sV), HALF, 1024);
       auto issue_s = [&](int j) -> bool {
         const int s = j & 1;
         const uint32_t par = (j >> 1) & 1;
         if (!mbar_wait(&k_full[s], par, p.status, abort_flag)) return false;
         if (!mbar_wait(&s_free[s], par ^ 1u, p.status, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + s * TILE_BYTES);
+        const uint64_t kd = sdesc_add(dK, s * TILE_BYTES);
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
           const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
-          umma_bf16_ss(tS + s * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
-                       IDESC_QK, k != 0 ? 1u : 0u);
+          umma_bf16_ss(tS + s * 128, sdesc_add(dQ, off), sdesc_add(kd, off), IDESC_QK, k != 0 ? 1u : 0u);
         }
         umma_commit(&s_full[s]);
         umma_commit(&k_empty[s]);
@@ -229,14 +230,12 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait(&p_full[s], par, p.status, abort_flag)) break;
         if (!mbar_wait(&v_full[s], par, p.status, abort_flag)) break;
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(sP + s * TILE_BYTES);
-        const uint32_t v_addr = smem_u32(sV + s * TILE_BYTES);
+        const uint64_t pd = sdesc_add(dP, s * TILE_BYTES), vd = sdesc_add(dV, s * TILE_BYTES);
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k) {
           const uint32_t a_off = (k >> 2) * HALF + (k & 3) * 32;  // P: K-major, keys 16k..16k+15
           const uint32_t b_off = k * 16 * 128;                      // V: MN-major, key rows 16k..
-          umma_bf16_ss(tO, sdesc_sw128(p_addr + a_off, 16, 1024), sdesc_sw128(v_addr + b_off, HALF, 1024), IDESC_PV,
-                       (j | k) != 0 ? 1u : 0u);
+          umma_bf16_ss(tO, sdesc_add(pd, a_off), sdesc_add(vd, b_off), IDESC_PV, (j | k) != 0 ? 1u : 0u);
         }
         umma_commit(o_done);
         umma_commit(&p_free[s]);
@@ -482,22 +481,24 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       // ---------------------------------------------------------------- UMMA issuer
       bool ok = mbar_wait(q_full, 0, p.status, abort_flag);
+      // descriptors of the first Q, K and V tiles; every other one is a fixed offset away
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024), dK = sdesc_sw128(smem_u32(sK), 16, 1024),
+                     dV = sdesc_sw128(smem_u32(sV), HALF, 1024);
       auto issue_s = [&](int x, int j) {  // S_x(j) = Q_x K_j^T into TMEM columns [128 x, 128 x + 128)
-        const uint32_t q_addr = smem_u32(sQ + x * TILE_BYTES), k_addr = smem_u32(sK + (j & 1) * TILE_BYTES);
+        const uint64_t qd = sdesc_add(dQ, x * TILE_BYTES), kd = sdesc_add(dK, (j & 1) * TILE_BYTES);
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
           const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
-          umma_bf16_ss(tmem_base + x * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
-                       IDESC_QK, k != 0 ? 1u : 0u);
+          umma_bf16_ss(tmem_base + x * 128, sdesc_add(qd, off), sdesc_add(kd, off), IDESC_QK, k != 0 ? 1u : 0u);
         }
         umma_commit(&s_full[x]);
       };
       auto issue_pv = [&](int x, int j) {  // O_x (+)= P_x(j) V_j, P_x from TMEM over S_x
-        const uint32_t v_addr = smem_u32(sV + (j & 1) * TILE_BYTES);
+        const uint64_t vd = sdesc_add(dV, (j & 1) * TILE_BYTES);
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k)
-          umma_bf16_ts(tmem_base + 256 + x * 128, tmem_base + x * 128 + k * 8,
-                       sdesc_sw128(v_addr + k * 16 * 128, HALF, 1024), IDESC_PV, (j | k) != 0 ? 1u : 0u);
+          umma_bf16_ts(tmem_base + 256 + x * 128, tmem_base + x * 128 + k * 8, sdesc_add(vd, k * 16 * 128), IDESC_PV,
+                       (j | k) != 0 ? 1u : 0u);
         umma_commit(&o_done[x]);
       };
       if (ok && n > 0) {
@@ -518,8 +519,9 @@ __global__ void __launch_bounds__(320, 1)
           issue_pv(x, j);
           if (x == 1) umma_commit(&v_empty[j & 1]);
           if (j + 1 < n) {
-            // S_x(j+1) overwrites the TMEM columns P_x(j) V_j reads: wait for that MMA
-            if (!mbar_wait(&o_done[x], par, p.status, abort_flag)) { ok = false; break; }
+            // S_x(j+1) overwrites the TMEM columns P_x(j) V_j reads.  tcgen05.mma issued by
+            // one thread execute in issue order, so it is issued right behind P_x(j) V_j
+            // (the scan's state update relies on the same order)
             if (x == 0 && !mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, p.status, abort_flag)) {
               ok = false;
               break;

@@ -269,6 +269,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ UMMA issuer
+      // stage descriptors are fixed offsets from the first stage's (one add per MMA)
+      const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024), dB = sdesc_sw128(smem_u32(sB), 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -288,11 +290,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
-          const uint32_t b0 = smem_u32(sB + stage * C::B_STAGE);
+          const uint64_t ad = sdesc_add(dA, stage * A_STAGE), bd = sdesc_add(dB, stage * C::B_STAGE);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_bf16_ss(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024), sdesc_sw128(b0 + k * 32, 16, 1024), C::IDESC,
+            umma_bf16_ss(d_tmem, sdesc_add(ad, k * 32), sdesc_add(bd, k * 32), C::IDESC,
                          (kb != kfirst || k != 0) ? 1u : 0u);
           umma_commit(&empty[stage]);
           if (++stage == C::STAGES) {
@@ -574,6 +575,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ------------------------------------------------ UMMA issuer (first CTA of the pair)
+      const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024), dB = sdesc_sw128(smem_u32(sB), 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -592,12 +594,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
-          const uint32_t b0 = smem_u32(sB + stage * PAIR_B_STAGE);
+          const uint64_t ad = sdesc_add(dA, stage * A_STAGE), bd = sdesc_add(dB, stage * PAIR_B_STAGE);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_bf16_ss_pair(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024), sdesc_sw128(b0 + k * 32, 16, 1024),
-                              PAIR_IDESC, (kb != kfirst || k != 0) ? 1u : 0u);
+            umma_bf16_ss_pair(d_tmem, sdesc_add(ad, k * 32), sdesc_add(bd, k * 32), PAIR_IDESC,
+                              (kb != kfirst || k != 0) ? 1u : 0u);
           umma_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == PAIR_STAGES) {
             stage = 0;

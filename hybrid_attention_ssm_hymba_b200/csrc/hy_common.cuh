@@ -285,6 +285,12 @@ HY_DEV uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_byt
   return d;
 }
 
+// The descriptor of the same layout `bytes` further on: the start-address field is the
+// low 14 bits (address >> 4) and shared-memory addresses stay below 2^18, so the sum
+// never carries out of it.  One add per MMA instead of rebuilding the descriptor: the
+// issuing thread is otherwise slower than the tensor core on MMAs of N <= 128.
+HY_DEV uint64_t sdesc_add(uint64_t desc, uint32_t bytes) { return desc + static_cast<uint64_t>(bytes >> 4); }
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                    // D format: f32

@@ -208,25 +208,28 @@ __global__ void __launch_bounds__(NTHR, 1)
   } else if (warp == 11) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t mt = sbase + L::OFF_MT, bt = sbase + L::OFF_BT;
+      // descriptors of the first stage's tiles; every other tile is a fixed offset away
+      const uint64_t dMT = sdesc_sw128(sbase + L::OFF_MT, 16, 1024), dBT = sdesc_sw128(sbase + L::OFF_BT, 16, 1024),
+                     dBC = sdesc_sw128(sbase + L::OFF_BC, 16, 1024), dD = sdesc_sw128(sbase + L::OFF_D, 16, 1024),
+                     dWD = sdesc_sw128(sbase + L::OFF_WD, 16, 1024);
       // Block k's stage has landed: W_dt dt_low^T (FUSED) and C B^T.
       auto issue_stage = [&](int k) -> bool {
         const int s = k % STAGES;
         if (!mbar_wait(&full[s], (k / STAGES) & 1u, status, abort_flag)) return false;
         tc_fence_after();
         if (FUSED) {
-          const uint32_t dl = sbase + L::OFF_D + s * L::D_B, wd = sbase + L::OFF_WD;
+          const uint64_t dl = sdesc_add(dD, s * L::D_B);
+#pragma unroll
           for (int j = 0; j < KR / 16; ++j)
-            umma_bf16_ss(tmem + COL_DT, sdesc_sw128(wd + 32 * j, 16, 1024), sdesc_sw128(dl + 32 * j, 16, 1024),
-                         IDESC_DT, j);
+            umma_bf16_ss(tmem + COL_DT, sdesc_add(dWD, 32 * j), sdesc_add(dl, 32 * j), IDESC_DT, j);
           umma_commit(dtready);
         }
-        const uint32_t bc = sbase + L::OFF_BC + s * BC_B;
+        const uint64_t bc = sdesc_add(dBC, s * BC_B);
         // C B^T: A = C rows (128 rows read; rows 64..127 are whatever follows the tile and
         // land in TMEM lanes nobody reads), B = B rows; K = 16 = two tf32 steps.
+#pragma unroll
         for (int j = 0; j < 2; ++j)
-          umma_tf32_ss(tmem + COL_MR, sdesc_sw128(bc + 64 + 32 * j, 16, 1024), sdesc_sw128(bc + 32 * j, 16, 1024),
-                       IDESC_N64, j);
+          umma_tf32_ss(tmem + COL_MR, sdesc_add(bc, 64 + 32 * j), sdesc_add(bc, 32 * j), IDESC_N64, j);
         umma_commit(mraw);
         return true;
       };
@@ -237,22 +240,24 @@ __global__ void __launch_bounds__(NTHR, 1)
         if (!mbar_wait(&vready[i], par, status, abort_flag) || !mbar_wait(mready, k & 1u, status, abort_flag)) break;
         tc_fence_after();
         // Y = V M^T (K = s, 64 = 8 steps) and dG = V B (B^T tile)
+#pragma unroll
         for (int j = 0; j < 8; ++j)
-          umma_tf32_ts(tmem + COL_Y + 64 * i, tmem + COL_V + 8 * j,
-                       sdesc_sw128(mt + (j >> 2) * 8192 + (j & 3) * 32, 16, 1024), IDESC_N64, j);
+          umma_tf32_ts(tmem + COL_Y + 64 * i, tmem + COL_V + 8 * j, sdesc_add(dMT, (j >> 2) * 8192 + (j & 3) * 32),
+                       IDESC_N64, j);
+#pragma unroll
         for (int j = 0; j < 8; ++j)
-          umma_tf32_ts(tmem + COL_DG + 16 * i, tmem + COL_V + 8 * j,
-                       sdesc_sw128(bt + (j >> 2) * 2048 + (j & 3) * 32, 16, 1024), IDESC_N16, j);
+          umma_tf32_ts(tmem + COL_DG + 16 * i, tmem + COL_V + 8 * j, sdesc_add(dBT, (j >> 2) * 2048 + (j & 3) * 32),
+                       IDESC_N16, j);
         umma_commit(&dgready[i]);
         // the next block's dt projection and C B^T (their TMEM was read before vready / mready)
         if (k + 1 < nblk && !issue_stage(k + 1)) break;
         if (!mbar_wait(&gready[i], par, status, abort_flag)) break;
         tc_fence_after();
         // Y += G' C^T (K = n = 16)
-        const uint32_t bc = sbase + L::OFF_BC + s * BC_B;
+        const uint64_t bc = sdesc_add(dBC, s * BC_B);
+#pragma unroll
         for (int j = 0; j < 2; ++j)
-          umma_tf32_ts(tmem + COL_Y + 64 * i, tmem + COL_GP + 16 * i + 8 * j, sdesc_sw128(bc + 64 + 32 * j, 16, 1024),
-                       IDESC_N64, 1);
+          umma_tf32_ts(tmem + COL_Y + 64 * i, tmem + COL_GP + 16 * i + 8 * j, sdesc_add(bc, 64 + 32 * j), IDESC_N64, 1);
         umma_commit(&yready[i]);
         umma_commit(&empty[s]);
       }
@@ -800,55 +805,76 @@ __global__ void __launch_bounds__(NTHR, 1)
     // ------------------------------------------------------------ MMA issuer: a small
     // dataflow scheduler over four tasks, each issued as soon as its inputs are ready
     //   stage(ks):   dt projection and C B^T of a landed stage
-    //   chain(kc):   Y = G' C^T, G' += V B (the state products; releases the stage first)
+    //   release(kr): the stage of block kr back to the producer
+    //   chain(kc):   Y = G' C^T, G' += V B (the state products)
     //   vm(kv):      Y += V M^T, then Y is complete
     // Buffer reuse: DT / MR buffer ks & 1 held block ks - 2, consumed before gready /
-    // mready of that block (chain(ks - 2), vm(ks - 2) issued); the stage of block kc holds
-    // nothing the state products read (B^T and the C copy are separate).
+    // mready of that block (chain(ks - 2), vm(ks - 2) issued); the stage holds nothing the
+    // state products read (B^T and the C copy are separate).  Releases run in block order,
+    // so a vready / btready phase is never tested after the next phase of the same
+    // barrier completed (that needs the stage of block kr + 2, or kr + 3, loaded).
     if (lane == 0) {
-      int ks = 0, kc = 0, kv = 0;
+      // descriptors of the first stage's tiles; every other tile is a fixed offset away
+      const uint64_t dBC = sdesc_sw128(sbase + OFF_BC, 16, 1024), dDL = sdesc_sw128(sbase + OFF_DL, 16, 1024),
+                     dWD = sdesc_sw128(sbase + OFF_WD, 16, 1024), dCC = sdesc_sw128(sbase + OFF_CC, 16, 1024),
+                     dBT = sdesc_sw128(sbase + OFF_BT, 16, 1024), dMT = sdesc_sw128(sbase + OFF_MT, 16, 1024);
+      int ks = 0, kc = 0, kv = 0, kr = 0;
       unsigned long long t_last = 0;
       uint32_t idle = 0;
       while (kv < nblk) {
         if (ks < nblk && ks <= kc + 1 && ks <= kv + 1 && mbar_try_wait(&full[ks % ST], (ks / ST) & 1u)) {
           tc_fence_after();
           const int s = ks % ST, i = ks & 1;
-          const uint32_t dl = sbase + OFF_DL + s * DL_B, wd = sbase + OFF_WD;
-          for (int a = 0; a < ka; ++a)
+          const uint64_t dl = sdesc_add(dDL, s * DL_B);
+#pragma unroll
+          for (int j = 0; j < KA / 16; ++j)
+            umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_add(dWD, 32 * j), sdesc_add(dl, 32 * j), IDESC_DT, j != 0);
+          if (ka > 1) {
+#pragma unroll
             for (int j = 0; j < KA / 16; ++j)
-              umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_sw128(wd + a * WDC_B + 32 * j, 16, 1024),
-                           sdesc_sw128(dl + a * DLC_B + 32 * j, 16, 1024), IDESC_DT, (a | j) != 0);
+              umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_add(dWD, WDC_B + 32 * j), sdesc_add(dl, DLC_B + 32 * j),
+                           IDESC_DT, 1u);
+          }
           umma_commit(&dtready[i]);
           // C B^T: A = a C chunk (128 rows read, rows 32..127 land in TMEM lanes nobody
           // reads), B = the B chunk of the same columns; K = n = 128 = 16 tf32 steps
-          const uint32_t bc = sbase + OFF_BC + s * BC_B;
+          const uint64_t bc = sdesc_add(dBC, s * BC_B);
+#pragma unroll
           for (int q = 0; q < 4; ++q)
+#pragma unroll
             for (int j = 0; j < 4; ++j)
-              umma_tf32_ss(tmem + COL_MR + 32 * i, sdesc_sw128(bc + (4 + q) * BCC_B + 32 * j, 16, 1024),
-                           sdesc_sw128(bc + q * BCC_B + 32 * j, 16, 1024), IDESC_Q, (q | j) != 0);
+              umma_tf32_ss(tmem + COL_MR + 32 * i, sdesc_add(bc, (4 + q) * BCC_B + 32 * j), sdesc_add(bc, q * BCC_B + 32 * j),
+                           IDESC_Q, (q | j) != 0);
           umma_commit(&mraw[i]);
           ++ks;
           idle = 0;
           continue;
         }
-        if (kc < ks && mbar_try_wait(&vready[kc % 3], (kc / 3) & 1u) &&
-            mbar_try_wait(&btready[kc & 1], (kc >> 1) & 1u) && mbar_try_wait(gready, kc & 1u)) {
+        // release(kr): block kr's stage is free once its dt projection and C B^T are done
+        // (what the commit tracks), x and gate were read (vready) and B, C copied (btready)
+        // -- a period before its state products, so the next load has two periods to land
+        if (kr < ks && mbar_try_wait(&vready[kr % 3], (kr / 3) & 1u) &&
+            mbar_try_wait(&btready[kr & 1], (kr >> 1) & 1u)) {
+          umma_commit(&empty[kr % ST]);
+          ++kr;
+          idle = 0;
+          continue;
+        }
+        if (kc < kr && mbar_try_wait(gready, kc & 1u)) {
           tc_fence_after();
-          // the stage of block kc: its dt projection and C B^T were issued before (their
-          // completion is what the commit tracks), x and gate were read before vready,
-          // B and C copied before btready
-          umma_commit(&empty[kc % ST]);
           if (!sAny[kc % 3]) {
             const int i = kc & 1, vb = kc % 3;
-            const uint32_t cc = sbase + OFF_CC + i * CC_B, bt = sbase + OFF_BT + i * BT_B;
+            const uint64_t cc = sdesc_add(dCC, i * CC_B), bt = sdesc_add(dBT, i * BT_B);
             // Y = G' C^T (K = n = 128), then G' += V B (K = s = 32, B^T rows n)
+#pragma unroll
             for (int q = 0; q < 4; ++q)
+#pragma unroll
               for (int j = 0; j < 4; ++j)
-                umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_GP + 32 * q + 8 * j,
-                             sdesc_sw128(cc + q * BCC_B + 32 * j, 16, 1024), IDESC_Q, (q | j) != 0);
+                umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_GP + 32 * q + 8 * j, sdesc_add(cc, q * BCC_B + 32 * j),
+                             IDESC_Q, (q | j) != 0);
+#pragma unroll
             for (int j = 0; j < 4; ++j)
-              umma_tf32_ts(tmem + COL_GP, tmem + COL_V + 32 * vb + 8 * j, sdesc_sw128(bt + 32 * j, 16, 1024), IDESC_N,
-                           1);
+              umma_tf32_ts(tmem + COL_GP, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(bt, 32 * j), IDESC_N, 1);
           }
           umma_commit(&dgready[kc & 1]);
           ++kc;
@@ -859,10 +885,10 @@ __global__ void __launch_bounds__(NTHR, 1)
           tc_fence_after();
           if (!sAny[kv % 3]) {  // Y += V M^T (K = s = 32)
             const int i = kv & 1, vb = kv % 3;
-            const uint32_t mt = sbase + OFF_MT + i * MT_B;
+            const uint64_t mt = sdesc_add(dMT, i * MT_B);
+#pragma unroll
             for (int j = 0; j < 4; ++j)
-              umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_V + 32 * vb + 8 * j, sdesc_sw128(mt + 32 * j, 16, 1024),
-                           IDESC_Q, 1);
+              umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(mt, 32 * j), IDESC_Q, 1);
           }
           umma_commit(&yready[kv & 1]);
           ++kv;
