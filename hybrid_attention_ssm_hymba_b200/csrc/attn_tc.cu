@@ -519,9 +519,10 @@ __global__ void __launch_bounds__(320, 1)
           issue_pv(x, j);
           if (x == 1) umma_commit(&v_empty[j & 1]);
           if (j + 1 < n) {
-            // S_x(j+1) overwrites the TMEM columns P_x(j) V_j reads.  tcgen05.mma issued by
-            // one thread execute in issue order, so it is issued right behind P_x(j) V_j
-            // (the scan's state update relies on the same order)
+            // S_x(j+1) overwrites the TMEM columns P_x(j) V_j reads: wait for that MMA (an
+            // MMA issued behind another is not held back from writing TMEM the earlier one
+            // still reads)
+            if (!mbar_wait(&o_done[x], par, p.status, abort_flag)) { ok = false; break; }
             if (x == 0 && !mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, p.status, abort_flag)) {
               ok = false;
               break;

@@ -683,8 +683,9 @@ constexpr int OFF_G = OFF_X + ST * TILE_B;
 constexpr int OFF_S = OFF_G + ST * TILE_B;   // float [2 blocks][2 halves][128]: half-block decay sums
 constexpr int OFF_ANY = OFF_S + 2 * 2 * CH * 4;  // int [3]: the block runs the plain recurrence
 constexpr int OFF_BAR = OFF_ANY + 16;
-// full[ST] empty[ST] dtready[2] mraw[2] vready[3] btready[2] mready[2] gready dgready[2] yready[2] mma_done
-constexpr int NBAR = 2 * ST + 2 + 2 + 3 + 2 + 2 + 1 + 2 + 2 + 1;
+// full[ST] empty[ST] dtready[2] mraw[2] vready[3] btready[2] mready[2] gready dgready[2] yready[2] yidone
+// mma_done
+constexpr int NBAR = 2 * ST + 2 + 2 + 3 + 2 + 2 + 1 + 2 + 2 + 1 + 1;
 constexpr int SMEM_TOTAL = OFF_BAR + NBAR * 8 + 16 + 1024;
 static_assert(OFF_DL % 1024 == 0 && OFF_WD % 1024 == 0 && OFF_MT % 1024 == 0 && OFF_BT % 1024 == 0 &&
                   OFF_CC % 1024 == 0,
@@ -732,7 +733,8 @@ __global__ void __launch_bounds__(NTHR, 1)
   uint64_t* gready = mready + 2;       // G' rescaled for the block (256 arrivals)
   uint64_t* dgready = gready + 1;      // [2] the block's state products done (G' advanced)
   uint64_t* yready = dgready + 2;      // [2] the block's Y complete
-  uint64_t* mma_done = yready + 2;
+  uint64_t* yidone = yready + 2;       // Y = G' C^T done reading G' (once per block)
+  uint64_t* mma_done = yidone + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sS = reinterpret_cast<float*>(sm + OFF_S);
@@ -757,6 +759,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     for (int i = 0; i < 3; ++i) mbar_init(&vready[i], NCHT);
     mbar_init(gready, NCHT);
+    mbar_init(yidone, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -819,6 +822,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                      dWD = sdesc_sw128(sbase + OFF_WD, 16, 1024), dCC = sdesc_sw128(sbase + OFF_CC, 16, 1024),
                      dBT = sdesc_sw128(sbase + OFF_BT, 16, 1024), dMT = sdesc_sw128(sbase + OFF_MT, 16, 1024);
       int ks = 0, kc = 0, kv = 0, kr = 0;
+      uint32_t n_yi = 0;   // completed phases of yidone (product-form blocks only)
       unsigned long long t_last = 0;
       uint32_t idle = 0;
       while (kv < nblk) {
@@ -865,13 +869,19 @@ __global__ void __launch_bounds__(NTHR, 1)
           if (!sAny[kc % 3]) {
             const int i = kc & 1, vb = kc % 3;
             const uint64_t cc = sdesc_add(dCC, i * CC_B), bt = sdesc_add(dBT, i * BT_B);
-            // Y = G' C^T (K = n = 128), then G' += V B (K = s = 32, B^T rows n)
+            // Y = G' C^T (K = n = 128), then G' += V B (K = s = 32, B^T rows n).  The update
+            // writes the TMEM G' the first product reads as its A operand: it is issued only
+            // once that product has completed (an MMA issued behind another is not held back
+            // from writing TMEM the earlier one still reads)
 #pragma unroll
             for (int q = 0; q < 4; ++q)
 #pragma unroll
               for (int j = 0; j < 4; ++j)
                 umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_GP + 32 * q + 8 * j, sdesc_add(cc, q * BCC_B + 32 * j),
                              IDESC_Q, (q | j) != 0);
+            umma_commit(yidone);
+            if (!mbar_wait(yidone, n_yi & 1u, status, abort_flag)) break;
+            ++n_yi;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               umma_tf32_ts(tmem + COL_GP, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(bt, 32 * j), IDESC_N, 1);

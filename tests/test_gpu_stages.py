@@ -300,3 +300,32 @@ def test_scan_dtproj_full_size_sampled_channels(B, T, Di, N, R, dt_min):
     y = _run_dtproj(inp, B, T, Di, N, "bf16")
     chans = np.array([0, 1, 127, 128, 777, Di - 1])
     assert_close(y[:, chans], _dtproj_ref(inp, B, T, Di, N, chans), "bf16", "scan dtproj sampled channels")
+
+
+# ------------------------------------------------------------------ run-to-run repeatability
+
+@pytest.mark.parametrize("N,R", [(128, 128), (16, 64)])
+def test_scan_dtproj_is_repeatable_bit_for_bit(N, R):
+    """The tensor-core scans are deterministic: the same inputs give the same bits on every
+    call (a race between the state products and the state's rescale, or between an MMA
+    reading TMEM and a later one writing it, shows up here first)."""
+    B, T, Di = 3, 1200, 384
+    inp = synth.scan_dtproj_inputs(42, B, T, Di, N, R)
+    first = _run_dtproj(inp, B, T, Di, N, "bf16")
+    for _ in range(4):
+        np.testing.assert_array_equal(_run_dtproj(inp, B, T, Di, N, "bf16"), first)
+
+
+def test_attention_is_repeatable_bit_for_bit():
+    B, T, Hq, Hkv, M, W = 2, 1500, 8, 2, 64, 300
+    q, kv = synth.attention_inputs(43, B, T, Hq, Hkv, 128)
+    runs = []
+    for _ in range(4):
+        out = host.empty((B * T, Hq * 128), "bf16")
+        ws = host.workspace(256)
+        H.check(H.hymba_attention(dev(q, "bf16"), dev(kv, "bf16"), out, Hq * 128, B, T, Hq, Hkv, 128, M, W,
+                                  H.HYMBA_BF16, ws), "attention")
+        status_ok(ws)
+        runs.append(to_np(out))
+    for r in runs[1:]:
+        np.testing.assert_array_equal(r, runs[0])
