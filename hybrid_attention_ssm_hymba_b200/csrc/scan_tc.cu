@@ -713,6 +713,31 @@ HY_DEV uint32_t cc_off(int t, int n) {
   return (n >> 5) * BCC_B + (t >> 3) * 1024 + (t & 7) * 128 + ((((n & 31) >> 2) ^ (t & 7)) << 4) + (n & 3) * 4;
 }
 
+// 16 consecutive rows (tb, tb + 1, ...) of y for this lane's channel, written as 8-byte
+// stores of 4 adjacent channels: two shuffle rounds hand each lane 4 rows of its 4-lane
+// group's channels (lane 4h + 2p + e ends with rows 4m + 2p + e, m < 4, channels 4h..4h+3),
+// so a warp writes 4 x 8 rows x 64 bytes instead of 16 x 64-byte row pieces per thread.
+// ybase: row 0, channel 0 of the sequence; c4: the group's first channel (a multiple of 4;
+// d_inner is a multiple of 8, so a group is inside or outside d_inner as a whole).
+HY_DEV void store_y16(__nv_bfloat16* ybase, long long y_ld, int tb, int T, int c4, bool c_ok, const float (&v)[16]) {
+  const int lane = threadIdx.x & 31, e = lane & 1, p = (lane >> 1) & 1;
+  uint32_t w[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {  // rows 2m + e of channels (2 (lane >> 1), + 1)
+    const float send = e ? v[2 * m] : v[2 * m + 1];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    w[m] = e ? pack_bf16(recv, v[2 * m + 1]) : pack_bf16(v[2 * m], recv);
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {  // rows 4m + 2p + e of channels c4 .. c4 + 3
+    const uint32_t send = p ? w[2 * m] : w[2 * m + 1];
+    const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 2);
+    const uint2 q = p ? make_uint2(recv, w[2 * m + 1]) : make_uint2(w[2 * m], recv);
+    const int t = tb + 4 * m + 2 * p + e;
+    if (c_ok && t < T) *reinterpret_cast<uint2*>(ybase + static_cast<long long>(t) * y_ld + c4) = q;
+  }
+}
+
 __global__ void __launch_bounds__(NTHR, 1)
     scan_tc128_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDL,
                       const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmBC,
@@ -991,6 +1016,8 @@ __global__ void __launch_bounds__(NTHR, 1)
     const float A2 = c < Di ? expf(a_log[c]) * 1.4426950408889634f : 0.f;  // |A| / ln 2
     const float bdt = c < Di ? b_dt[c] : 0.f;
     __nv_bfloat16* ycol = y + static_cast<long long>(b) * T * y_ld + c;
+    __nv_bfloat16* ybase = y + static_cast<long long>(b) * T * y_ld;
+    const int c4 = c0 + qd * 32 + (lane & ~3);   // this lane's 4-channel store group
     bool fail = false;
     // the state entering row t0 (raw: the first block applies only its own scale)
 #pragma unroll 1
@@ -1107,30 +1134,30 @@ __global__ void __launch_bounds__(NTHR, 1)
         const float f1 = ex2_approx(one ? -(e_in + e_out) : -e_in), f2 = one ? 1.f : ex2_approx(-e_out);
         const float2 fa = make_float2(f1, f1), fb = make_float2(f2, f2);
         tc_fence_after();
-#pragma unroll 1
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t col = tl + COL_GP + 64 * half + 32 * part;
-          uint32_t g[32];
-          tmem_ld32(col, g);
-          tmem_wait_ld();
-          if (one) {
+        // both 32-column pieces of this half in flight at once: one load wait, one store wait
+        const uint32_t col = tl + COL_GP + 64 * half;
+        uint32_t g[64];
+        tmem_ld32(col, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+        tmem_ld32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
+        tmem_wait_ld();
+        if (one) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float2 v = __fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa);
-              g[j] = __float_as_uint(v.x);
-              g[j + 1] = __float_as_uint(v.y);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float2 v =
-                  __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa), fb);
-              g[j] = __float_as_uint(v.x);
-              g[j + 1] = __float_as_uint(v.y);
-            }
+          for (int j = 0; j < 64; j += 2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa);
+            g[j] = __float_as_uint(v.x);
+            g[j + 1] = __float_as_uint(v.y);
           }
-          tmem_st32(col, g);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            const float2 v =
+                __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa), fb);
+            g[j] = __float_as_uint(v.x);
+            g[j + 1] = __float_as_uint(v.y);
+          }
         }
+        tmem_st32(col, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+        tmem_st32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
         tmem_wait_st();
       }
       // ---- large decays: the plain recurrence over block k on the raw state in G'
@@ -1201,24 +1228,22 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
       tc_fence_before();
       mbar_arrive(gready);
-      // ---- output of block k - 1: y = W * Y
-      if (k > 0 && !prev_any) {
+      // ---- output of block k - 1: y = W * Y.  Every phase of yready is waited for, even
+      // after a plain block (whose y went out already): a skipped phase would let the parity
+      // test of the next wait on the same barrier pass a phase early
+      if (k > 0) {
         const int jb = k - 1, i = jb & 1;
         if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(&yready[i], (jb >> 1) & 1u, status, abort_flag));
-        if (!fail) {
+        if (!fail && !prev_any) {
           tc_fence_after();
           uint32_t yv[HQ], wv[HQ];
           tmem_ld16(tl + COL_Y + 32 * i + HQ * half, yv);
           tmem_ld16(tl + COL_W + 32 * (jb % 3) + HQ * half, wv);
           tmem_wait_ld();
-          if (c < Di) {
-            const int tb = t0 + jb * Q + HQ * half;
+          float o[HQ];
 #pragma unroll
-            for (int j = 0; j < HQ; ++j)
-              if (tb + j < T)
-                ycol[static_cast<long long>(tb + j) * y_ld] =
-                    __float2bfloat16_rn(__uint_as_float(yv[j]) * __uint_as_float(wv[j]));
-          }
+          for (int j = 0; j < HQ; ++j) o[j] = __uint_as_float(yv[j]) * __uint_as_float(wv[j]);
+          store_y16(ybase, y_ld, t0 + jb * Q + HQ * half, T, c4, c4 < Di, o);
         }
       }
       pS1 = cS1;
@@ -1239,14 +1264,10 @@ __global__ void __launch_bounds__(NTHR, 1)
           tmem_ld16(tl + COL_Y + 32 * i + HQ * half, yv);
           tmem_ld16(tl + COL_W + 32 * (jb % 3) + HQ * half, wv);
           tmem_wait_ld();
-          if (c < Di) {
-            const int tb = t0 + jb * Q + HQ * half;
+          float o[HQ];
 #pragma unroll
-            for (int j = 0; j < HQ; ++j)
-              if (tb + j < T)
-                ycol[static_cast<long long>(tb + j) * y_ld] =
-                    __float2bfloat16_rn(__uint_as_float(yv[j]) * __uint_as_float(wv[j]));
-          }
+          for (int j = 0; j < HQ; ++j) o[j] = __uint_as_float(yv[j]) * __uint_as_float(wv[j]);
+          store_y16(ybase, y_ld, t0 + jb * Q + HQ * half, T, c4, c4 < Di, o);
         }
       }
       if (got && h_out) {
