@@ -1017,6 +1017,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     const float bdt = c < Di ? b_dt[c] : 0.f;
     __nv_bfloat16* ycol = y + static_cast<long long>(b) * T * y_ld + c;
     __nv_bfloat16* ybase = y + static_cast<long long>(b) * T * y_ld;
+    bool stop = false;   // uniform over the channel threads: leave the block loop
     const int c4 = c0 + qd * 32 + (lane & ~3);   // this lane's 4-channel store group
     bool fail = false;
     // the state entering row t0 (raw: the first block applies only its own scale)
@@ -1078,35 +1079,48 @@ __global__ void __launch_bounds__(NTHR, 1)
       const float S = S2.x + S2.y;
       float* ss = sS + (k & 1) * 2 * CH;
       ss[half * CH + cl] = S;
-      const bool any = bar_red_or(1, NCHT, fail || !(S <= kRange));
+      // one reduction in the common case: "some channel needs the plain recurrence or some
+      // thread failed"; only when it is set, a second one tells the two apart
+      bool any = bar_red_or(1, NCHT, fail || !(S <= kRange));
+      if (any && bar_red_or(1, NCHT, fail)) stop = true;   // uniform
       S0 = ss[cl];
       S1 = ss[CH + cl];
       if (!fail) {
-        const uint8_t* xt = sm + OFF_X + s * TILE_B + cl * 2 + HQ * half * 256;
-        const uint8_t* gt = sm + OFF_G + s * TILE_B + cl * 2 + HQ * half * 256;
-        uint32_t vr[HQ], wr[HQ];
-        float mu = half ? 0.f : -S;  // lambda - r
+        // x and gate of this half (explicit shared loads, all issued first), the running
+        // decay mu = lambda - r (one dependent FMA per step), then the exponentials, which
+        // are independent of one another; the block-uniform branch stays outside the loops
+        const uint32_t xa = sbase + OFF_X + s * TILE_B + cl * 2 + HQ * half * 256;
+        const uint32_t ga = sbase + OFF_G + s * TILE_B + cl * 2 + HQ * half * 256;
+        float xv[HQ], gv[HQ], mu[HQ];
 #pragma unroll
-        for (int j = 0; j < HQ; j += 2) {
-          const float2 xv = make_float2(bf2f(*reinterpret_cast<const uint16_t*>(xt + j * 256)),
-                                        bf2f(*reinterpret_cast<const uint16_t*>(xt + (j + 1) * 256)));
-          const float2 gv = make_float2(bf2f(*reinterpret_cast<const uint16_t*>(gt + j * 256)),
-                                        bf2f(*reinterpret_cast<const uint16_t*>(gt + (j + 1) * 256)));
-          const float2 u = __fmul2_rn(make_float2(dtv[j], dtv[j + 1]), xv);
-          if (!any) {
-            const float mu0 = fmaf(A2, dtv[j], mu);
-            mu = fmaf(A2, dtv[j + 1], mu0);
-            const float2 v = __fmul2_rn(u, make_float2(ex2_approx(mu0), ex2_approx(mu)));
-            const float2 w = __fmul2_rn(gv, make_float2(ex2_approx(-mu0), ex2_approx(-mu)));
+        for (int j = 0; j < HQ; ++j) {
+          xv[j] = bf2f(static_cast<uint16_t>(lds_u16(xa + j * 256)));
+          gv[j] = bf2f(static_cast<uint16_t>(lds_u16(ga + j * 256)));
+        }
+        uint32_t vr[HQ], wr[HQ];
+        if (!any) {
+          float m = half ? 0.f : -S;
+#pragma unroll
+          for (int j = 0; j < HQ; ++j) {
+            m = fmaf(A2, dtv[j], m);
+            mu[j] = m;
+          }
+#pragma unroll
+          for (int j = 0; j < HQ; j += 2) {
+            const float2 u = __fmul2_rn(make_float2(dtv[j], dtv[j + 1]), make_float2(xv[j], xv[j + 1]));
+            const float2 v = __fmul2_rn(u, make_float2(ex2_approx(mu[j]), ex2_approx(mu[j + 1])));
+            const float2 w =
+                __fmul2_rn(make_float2(gv[j], gv[j + 1]), make_float2(ex2_approx(-mu[j]), ex2_approx(-mu[j + 1])));
             vr[j] = tf32_round(v.x);
             vr[j + 1] = tf32_round(v.y);
             wr[j] = __float_as_uint(w.x);
             wr[j + 1] = __float_as_uint(w.y);
-          } else {
-            vr[j] = __float_as_uint(u.x);
-            vr[j + 1] = __float_as_uint(u.y);
-            wr[j] = __float_as_uint(gv.x);
-            wr[j + 1] = __float_as_uint(gv.y);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < HQ; ++j) {
+            vr[j] = __float_as_uint(dtv[j] * xv[j]);
+            wr[j] = __float_as_uint(gv[j]);
           }
         }
         tmem_st16(tl + COL_V + 32 * vb + HQ * half, vr);
@@ -1121,9 +1135,10 @@ __global__ void __launch_bounds__(NTHR, 1)
 
     float cS0 = 0.f, cS1 = 0.f;
     bool c_any = nblk > 0 ? form_vw(0, cS0, cS1) : false;
+    if (stop) fail = true;
     float pS1 = 0.f;        // the previous block's second-half decay sum
     bool prev_any = true;   // the previous block left the raw state in G' (so does the start)
-    for (int k = 0; k < nblk; ++k) {
+    for (int k = 0; k < nblk && !stop; ++k) {
       // ---- G' for block k: block k - 1's state products are done
       if (k > 0 && !fail)
         fail = !__all_sync(0xffffffffu, mbar_wait(&dgready[(k - 1) & 1], ((k - 1) >> 1) & 1u, status, abort_flag));
@@ -1250,8 +1265,13 @@ __global__ void __launch_bounds__(NTHR, 1)
       prev_any = c_any;
       // ---- V and W of block k + 1 (their buffer's last reader, block k - 2's V M^T,
       // completed before the output of block k - 2 above, an iteration ago)
+      // a failure anywhere in this iteration (or another role's abort, seen by the waits)
+      // reaches every channel thread through form_vw's reduction
       if (k + 1 < nblk) c_any = form_vw(k + 1, cS0, cS1);
-      if (bar_red_or(1, NCHT, fail || *abort_flag)) break;
+      if (stop) {
+        fail = true;
+        break;
+      }
     }
     // ---- output of the last block and the state after the last row
     if (__all_sync(0xffffffffu, !fail && nblk > 0 && !*abort_flag)) {
