@@ -54,7 +54,10 @@ LayerWs layer_ws(const hymba_cfg_t& c, size_t base) {
   w.g = o; o = al256(o + rows * c.d_inner * es);
   w.dtlow = o; o = al256(o + rows * c.dt_rank * es);
   w.bc = o; o = al256(o + rows * 2 * c.d_state * 4);
-  w.dt = o; o = al256(o + rows * c.d_inner * es);
+  // dt, or (d_state 128 with dt_proj fused into the scan, which stores no dt) the
+  // blocks' shared operands, 36 KB per 32 rows (C B^T, B^T and C, fp32)
+  const size_t dt_bytes = rows * c.d_inner * es, mgram = c.d_state == 128 ? (rows + 31 * c.batch) / 32 * 36864 : 0;
+  w.dt = o; o = al256(o + (dt_bytes > mgram ? dt_bytes : mgram));
   w.z = o; o = al256(o + rows * (wa + c.d_inner) * es);
   // fused branch norm (bf16): per row, the sums of squares of Y_attn and Y_ssm; and
   // W_out with beta1 | beta2 folded into its columns
@@ -299,14 +302,16 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
     sd.h0 = reinterpret_cast<const float*>(lo.prefix + PL.h);
     sd.h0_bstride = 0;
   }
-  // bf16 with d_state 16 and dt_rank 64: dt_proj runs inside the tensor-core scan
-  // (dt = softplus(dt_low W_dt^T + b_dt) per block, never stored)
+  // bf16 with d_state 16 (dt_rank 64) or 128 (dt_rank 8..128, a multiple of 8): dt_proj
+  // runs inside the tensor-core scan (dt = softplus(dt_low W_dt^T + b_dt) per block,
+  // never stored)
   {
     hy::ScanDesc f = sd;
     f.dt_low = dtlow;
     f.w_dt = w.w_dt;
     f.b_dt = w.b_dt;
     f.dt_rank = c.dt_rank;
+    f.mgram = dt;   // unused as dt when fused
     if (hy::scan_tc_fuses_dt(f)) sd = f;
   }
   const bool fused_dt = sd.dt_low != nullptr;
@@ -1133,7 +1138,9 @@ size_t hymba_selective_scan_dtproj_workspace_size(int batch, int T, int d_inner,
   f.d_state = d_state;
   f.dt_rank = dt_rank;
   f.bf16 = dtype == HYMBA_BF16;
-  if (hy::scan_tc_fuses_dt(f)) return 256;
+  f.batch = batch;
+  f.T = T;
+  if (hy::scan_tc_fuses_dt(f)) return 256 + (hy::scan_mgram_bytes(f) + 255) / 256 * 256;
   const size_t es = dtype == HYMBA_BF16 ? 2 : 4;
   return 256 + (static_cast<size_t>(batch) * T * d_inner * es + 255) / 256 * 256;
 }
@@ -1170,6 +1177,7 @@ hymba_status_t hymba_selective_scan_dtproj(const void* x, const void* dt_low, co
   f.w_dt = w_dt;
   f.b_dt = b_dt;
   f.dt_rank = dt_rank;
+  f.mgram = ws + 256;
   if (hy::scan_tc_fuses_dt(f)) return cuda_status(hy::launch_scan(f, st));
   // otherwise dt = softplus(dt_low W_dt^T + b_dt) through the GEMM into the workspace first
   void* dt = ws + 256;

@@ -53,6 +53,21 @@ HY_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same phase (mbarrier.try_wait may suspend the thread for a
+// while when the phase is not complete; a thread that polls several barriers in turn
+// must not be held on one of them).
+HY_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase of parity `parity` to complete.  Bounded: gives up after
 // kWaitLimitNs (records a timeout) or as soon as another role raised `abort`.
 HY_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status, volatile int* abort_flag,

@@ -131,8 +131,13 @@ struct ScanDesc {
   int t0 = 0;
   const float* h0 = nullptr;
   long long h0_bstride = 0;
+  // d_state 128 with the dt projection fused: scratch for the blocks' C B^T,
+  // scan_mgram_bytes(s) bytes, 16-byte aligned (written and read within the call).
+  void* mgram = nullptr;
 };
 cudaError_t launch_scan(const ScanDesc& s, cudaStream_t st);
+// Bytes of ScanDesc::mgram the scan needs (0 when it needs none).
+size_t scan_mgram_bytes(const ScanDesc& s);
 // The tensor-core form of the scan (bf16, d_state = 16, 16-byte aligned operands);
 // cudaErrorNotSupported for any other configuration.
 cudaError_t launch_scan_tc(const ScanDesc& s, cudaStream_t st);

@@ -597,6 +597,20 @@ bool map2d_sw128(CUtensorMap* m, const void* base, long long rows, long long col
 
 bool a16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
 
+// 3-D fp32 map over nrec records of rec_bytes, each [rows][cols] with row stride
+// row_bytes; box = bc x br x 1, 128-byte swizzle.
+bool map_rec_f32(CUtensorMap* m, const void* base, long long cols, long long rows, long long row_bytes, long long nrec,
+                 long long rec_bytes, int bc, int br) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(nrec)};
+  cuuint64_t gs[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rec_bytes)};
+  cuuint32_t bx[3] = {static_cast<cuuint32_t>(bc), static_cast<cuuint32_t>(br), 1}, el[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), gd, gs, bx, el,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool FUSED>
 cudaError_t launch_tc(const ScanDesc& s, cudaStream_t st) {
   using L = Lay<FUSED>;
@@ -636,44 +650,50 @@ cudaError_t launch_tc(const ScanDesc& s, cudaStream_t st) {
 //   of x, gate, dt_low and B|C (56 KB each) fit beside the other tiles.  B|C arrive as
 //   eight 32-column boxes ([32 t][128 B] each, 128-byte swizzle): chunks 0-3 are B (n in
 //   [32 q, 32 q + 32)), 4-7 are C, each one K atom of the tf32 products.
-// * The per-block dependency chain is only: the state products of block k -> the CUDA
-//   cores rescale G' -> the state products of block k + 1.  Everything else is kept off
+// * The per-block dependency chain is only: the state products of block k -> the state
+//   warps rescale G' -> the state products of block k + 1.  Everything else is kept off
 //   it: the copy warps turn each stage's B into B^T and copy C (both tf32, double-
 //   buffered) as soon as it lands, so the stage is released long before the state
-//   products read B and C; the channel warps form V and W of block k + 1 while block k's
-//   products run (V, W triple-buffered in TMEM); the part of Y that does not depend on
-//   the state (V M^T) is added after the state products; and the MMA thread issues
-//   whichever of its four tasks is ready (state products, a landed stage's dt projection
-//   and C B^T, V M^T, stage release) instead of waiting in a fixed order.
+//   products read B and C; separate V/W warps form dt, the decay sums, V and W of the
+//   blocks ahead (V, W triple-buffered in TMEM), so that the state warps only rescale G'
+//   and write y; the part of Y that does not depend on the state (V M^T) is added after
+//   the state products; and the MMA thread issues whichever of its four tasks is ready
+//   (state products, a landed stage's dt projection and C B^T, V M^T, stage release)
+//   instead of waiting in a fixed order.
 // * The dt projection is always fused (dt_rank <= 128: one or two 64-column atoms of
 //   dt_low and W_dt, columns past dt_rank zero-filled by TMA).
 // * A block where some channel's half-block decay sum exceeds kRange runs the plain
-//   recurrence on the CUDA cores (half-1 warps, 32 state columns at a time from TMEM,
-//   B and C from the tf32 copies), with G' holding the raw state on entry and on exit;
-//   its V, W columns then carry dt x and the gate, and the MMA thread skips its products.
-// * y goes straight from registers to global memory (a warp writes 32 adjacent channels
-//   of a row).
+//   recurrence on the CUDA cores (the half-1 state warps, 8 state columns at a time from
+//   TMEM, B and C from the tf32 copies), with G' holding the raw state on exit; its V, W
+//   columns then carry dt x and the gate, and the MMA thread skips its products.
+// * y goes straight from registers to global memory (8-byte stores of 4 adjacent
+//   channels after two shuffle rounds).
 //
-// CTA = 128 channels of one sequence, 384 threads: warps 0-7 channels (TMEM quadrant
-// w % 4, half w / 4 of the block's steps and of G''s columns), warps 8-9 B^T and the C
-// copy (warp 8 also the mask M, from TMEM lanes 0-31), warp 10 TMA, warp 11 TMEM and MMA.
+// CTA = 128 channels of one sequence, 640 threads: warps 0-7 state warps (TMEM quadrant
+// w % 4, half w / 4 of G''s columns and of each block's output rows), warps 8-15 V/W
+// warps (quadrant w % 4, half (w - 8) / 4 of each block's steps), warps 16-17 B^T and the
+// C copy (warp 16 also the mask M, from TMEM lanes 0-31), warp 18 TMA, warp 19 TMEM and
+// MMA.
 namespace t128 {
 constexpr int Q = 32;
-constexpr int HQ = 16;
 constexpr int NS = 128;
+constexpr int HQ = 16;                  // steps per V/W thread and block (a half)
+constexpr int QQ = 8;                   // steps per pass of the plain recurrence
+constexpr int NTHR2 = 608;
+constexpr int NRT = 256;                // state threads
+constexpr int NVT = 256;                // V/W threads (named barrier 1)
 constexpr int KA = 64;                  // dt_rank per K atom of the dt projection
 constexpr int TILE_B = Q * CH * 2;      // [32 t][128 c] bf16
-constexpr int BCC_B = Q * 128;          // one 32-column B|C chunk [32 t][32] fp32
-constexpr int BC_B = 8 * BCC_B;
+constexpr int BCC_B = Q * 128;          // one 32-column chunk of C [32 t][32] fp32
 constexpr int DLC_B = Q * 128;          // one dt_low atom [32 t][64 r] bf16
 constexpr int DL_B = 2 * DLC_B;
 constexpr int WDC_B = CH * 128;         // one W_dt atom [128 c][64 r] bf16
 constexpr int MT_B = Q * Q * 4;         // M [t][s] tf32
 constexpr int BT_B = NS * Q * 4;        // B^T [n][s] tf32
 constexpr int CC_B = 4 * BCC_B;         // C [t][n] tf32, four chunks
-constexpr int ST = 2;                   // stages
-constexpr int OFF_BC = 0;               // first: C B^T reads 96 rows past a C chunk
-constexpr int OFF_DL = OFF_BC + ST * BC_B;
+constexpr int GREC_B = MT_B + BT_B + CC_B;  // a block's record from bc_gram_kernel
+constexpr int ST = 4;                   // stages (x, gate, dt_low)
+constexpr int OFF_DL = 0;
 constexpr int OFF_WD = OFF_DL + ST * DL_B;
 constexpr int OFF_MT = OFF_WD + 2 * WDC_B;
 constexpr int OFF_BT = OFF_MT + 2 * MT_B;
@@ -683,21 +703,19 @@ constexpr int OFF_G = OFF_X + ST * TILE_B;
 constexpr int OFF_S = OFF_G + ST * TILE_B;   // float [2 blocks][2 halves][128]: half-block decay sums
 constexpr int OFF_ANY = OFF_S + 2 * 2 * CH * 4;  // int [3]: the block runs the plain recurrence
 constexpr int OFF_BAR = OFF_ANY + 16;
-// full[ST] empty[ST] dtready[2] mraw[2] vready[3] btready[2] mready[2] gready dgready[2] yready[2] yidone
+// full[ST] empty[ST] dtready[2] vready[3] btready[2] mready[2] gready dgready[2] yready[2] yidone wdone[3]
 // mma_done
-constexpr int NBAR = 2 * ST + 2 + 2 + 3 + 2 + 2 + 1 + 2 + 2 + 1 + 1;
+constexpr int NBAR = 2 * ST + 2 + 3 + 2 + 2 + 1 + 2 + 2 + 1 + 3 + 1;
 constexpr int SMEM_TOTAL = OFF_BAR + NBAR * 8 + 16 + 1024;
 static_assert(OFF_DL % 1024 == 0 && OFF_WD % 1024 == 0 && OFF_MT % 1024 == 0 && OFF_BT % 1024 == 0 &&
                   OFF_CC % 1024 == 0,
               "swizzled tiles 1024-aligned");
-static_assert(OFF_BC + (ST - 1) * BC_B + 7 * BCC_B + 128 * 128 <= OFF_BAR, "C B^T's A rows stay in the allocation");
 static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
 
 constexpr uint32_t COL_Y = 0;     // [2][32]
 constexpr uint32_t COL_W = 64;    // [3][32]
 constexpr uint32_t COL_V = 160;   // [3][32]
 constexpr uint32_t COL_DT = 256;  // [2][32] W_dt dt_low^T
-constexpr uint32_t COL_MR = 320;  // [2][32] C B^T (lanes 0-31)
 constexpr uint32_t COL_GP = 384;  // [128] G'
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_Q = idesc_tf32(128, Q);
@@ -711,6 +729,18 @@ HY_DEV uint32_t bt_off(int n, int s) {
 }
 HY_DEV uint32_t cc_off(int t, int n) {
   return (n >> 5) * BCC_B + (t >> 3) * 1024 + (t & 7) * 128 + ((((n & 31) >> 2) ^ (t & 7)) << 4) + (n & 3) * 4;
+}
+
+// 8-column variants of the TMEM load and store (32 lanes x 8 consecutive 32-bit columns).
+HY_DEV void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+HY_DEV void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 
 // 16 consecutive rows (tb, tb + 1, ...) of y for this lane's channel, written as 8-byte
@@ -738,28 +768,98 @@ HY_DEV void store_y16(__nv_bfloat16* ybase, long long y_ld, int tb, int T, int c
   }
 }
 
-__global__ void __launch_bounds__(NTHR, 1)
+// The operands every channel shares, once per block k (rows t0 + 32 k + t) of sequence
+// b, into record b * nblk + k of GREC_B bytes (rows past T read as zero):
+//   M   [t][s] = (C_t . B_s) [s <= t]: fp32 sums over n, rounded to tf32
+//   B^T [n][s] = B_s[n], rounded to tf32
+//   C   [t][n] = C_t[n], rounded to tf32
+// each row-major, so that a 128-byte-swizzled TMA box lands in shared memory as the
+// K-major operand of V M^T (M), of G' += V B (B^T) and of Y = G' C^T (C, four boxes of
+// 32 columns).  One CTA per block.
+__global__ void __launch_bounds__(256) bc_gram_kernel(const float* __restrict__ bc, int T, int t0, int nblk,
+                                                      uint8_t* __restrict__ rec) {
+  // no early trigger: the scan's CTAs (whose shared memory leaves no room for these)
+  // start once every record is written
+  __shared__ __align__(16) float sB[Q][NS + 4];   // rows padded by 16 bytes: conflict-free
+  __shared__ __align__(16) float sC[Q][NS + 4];
+  const int k = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int r0 = t0 + k * Q;
+  pdl_wait();
+  for (int i = tid; i < Q * 2 * NS / 4; i += blockDim.x) {  // a row: B 32 float4, C 32 float4
+    const int r = i / (2 * NS / 4), q = i % (2 * NS / 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < T) v = reinterpret_cast<const float4*>(bc + (static_cast<long long>(b) * T + r0 + r) * 2 * NS)[q];
+    float* dst = q < NS / 4 ? &sB[r][4 * q] : &sC[r][4 * q - NS];
+    *reinterpret_cast<float4*>(dst) = v;
+  }
+  __syncthreads();
+  uint8_t* out = rec + (static_cast<long long>(b) * nblk + k) * GREC_B;
+  {  // M: thread = row t, columns s4 .. s4 + 3
+    const int t = tid >> 3, s4 = (tid & 7) * 4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int n = 0; n < NS; n += 4) {
+      const float4 cv = *reinterpret_cast<const float4*>(&sC[t][n]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 bv = *reinterpret_cast<const float4*>(&sB[s4 + e][n]);
+        acc[e] = fmaf(cv.x, bv.x, acc[e]);
+        acc[e] = fmaf(cv.y, bv.y, acc[e]);
+        acc[e] = fmaf(cv.z, bv.z, acc[e]);
+        acc[e] = fmaf(cv.w, bv.w, acc[e]);
+      }
+    }
+    uint4 o;
+    o.x = s4 <= t ? tf32_round(acc[0]) : 0u;
+    o.y = s4 + 1 <= t ? tf32_round(acc[1]) : 0u;
+    o.z = s4 + 2 <= t ? tf32_round(acc[2]) : 0u;
+    o.w = s4 + 3 <= t ? tf32_round(acc[3]) : 0u;
+    reinterpret_cast<uint4*>(out)[t * (Q / 4) + s4 / 4] = o;
+  }
+  {  // B^T: thread = row n, columns 16 h .. 16 h + 15
+    const int n = tid >> 1, h = tid & 1;
+    uint4* dst = reinterpret_cast<uint4*>(out + MT_B + n * Q * 4 + h * 64);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int s0 = 16 * h + 4 * j;
+      dst[j] = make_uint4(tf32_round(sB[s0][n]), tf32_round(sB[s0 + 1][n]), tf32_round(sB[s0 + 2][n]),
+                          tf32_round(sB[s0 + 3][n]));
+    }
+  }
+  {  // C: thread = row t, columns 16 h .. 16 h + 15
+    const int t = tid >> 3, h = tid & 7;
+    uint4* dst = reinterpret_cast<uint4*>(out + MT_B + BT_B + t * NS * 4 + h * 64);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 v = *reinterpret_cast<const float4*>(&sC[t][16 * h + 4 * j]);
+      dst[j] = make_uint4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z), tf32_round(v.w));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(NTHR2, 1)
     scan_tc128_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDL,
-                      const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmBC,
-                      const __grid_constant__ CUtensorMap tmWD, const float* __restrict__ a_log,
-                      const float* __restrict__ b_dt, __nv_bfloat16* __restrict__ y, long long y_ld, int T, int Di,
-                      int ka, float* __restrict__ h_out, int t0, const float* __restrict__ h0, long long h0_bstride,
-                      unsigned* status) {
+                      const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmWD,
+                      const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmBT,
+                      const __grid_constant__ CUtensorMap tmC,
+                      const float* __restrict__ a_log, const float* __restrict__ b_dt, __nv_bfloat16* __restrict__ y,
+                      long long y_ld, int T, int Di, int ka, float* __restrict__ h_out, int t0,
+                      const float* __restrict__ h0, long long h0_bstride, unsigned* status) {
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);  // [ST] TMA landed
   uint64_t* empty = full + ST;         // [ST] the stage's last reader done
   uint64_t* dtready = empty + ST;      // [2] W_dt dt_low^T of the block in TMEM
-  uint64_t* mraw = dtready + 2;        // [2] C B^T of the block in TMEM
-  uint64_t* vready = mraw + 2;         // [3] V, W of the block in TMEM (256 arrivals)
-  uint64_t* btready = vready + 3;      // [2] B^T and the C copy in shared memory (64 arrivals)
-  uint64_t* mready = btready + 2;      // [2] M in shared memory (32 arrivals)
+  uint64_t* vready = dtready + 2;         // [3] V, W and the decay sums of the block ready (256 arrivals)
+  uint64_t* btready = vready + 3;      // [2] B^T and C of the block in shared memory (TMA)
+  uint64_t* mready = btready + 2;      // [2] M of the block in shared memory (TMA)
   uint64_t* gready = mready + 2;       // G' rescaled for the block (256 arrivals)
   uint64_t* dgready = gready + 1;      // [2] the block's state products done (G' advanced)
   uint64_t* yready = dgready + 2;      // [2] the block's Y complete
   uint64_t* yidone = yready + 2;       // Y = G' C^T done reading G' (once per block)
-  uint64_t* mma_done = yidone + 1;
+  uint64_t* wdone = yidone + 1;        // [3] the block's output written: V, W buffer free (256 arrivals)
+  uint64_t* mma_done = wdone + 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sS = reinterpret_cast<float*>(sm + OFF_S);
@@ -776,30 +876,35 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&dtready[i], 1);
-      mbar_init(&mraw[i], 1);
-      mbar_init(&btready[i], 64);
-      mbar_init(&mready[i], 32);
+      mbar_init(&btready[i], 1);
+      mbar_init(&mready[i], 1);
       mbar_init(&dgready[i], 1);
       mbar_init(&yready[i], 1);
     }
-    for (int i = 0; i < 3; ++i) mbar_init(&vready[i], NCHT);
-    mbar_init(gready, NCHT);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&vready[i], NVT);
+      mbar_init(&wdone[i], NRT);
+    }
+    mbar_init(gready, NRT);
     mbar_init(yidone, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 11) {
+  if (warp == 18) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   pdl_wait();
-  if (threadIdx.x == 320) {
+  if (threadIdx.x == 16 * 32) {
     tma_prefetch(&tmX);
     tma_prefetch(&tmDL);
     tma_prefetch(&tmG);
-    tma_prefetch(&tmBC);
     tma_prefetch(&tmWD);
+  } else if (threadIdx.x == 17 * 32) {
+    tma_prefetch(&tmM);
+    tma_prefetch(&tmBT);
+    tma_prefetch(&tmC);
   }
   tc_fence_before();
   __syncthreads();
@@ -807,21 +912,20 @@ __global__ void __launch_bounds__(NTHR, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(sm);
 
-  if (warp == 10) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 16) {
+    // ------------------------------------------------------------ TMA: x, gate, dt_low
     if (lane == 0) {
       int k = 0;
       for (; k < nblk; ++k) {
         const int s = k % ST;
         if (k >= ST && !mbar_wait(&empty[s], ((k / ST) - 1) & 1u, status, abort_flag)) break;
-        mbar_arrive_expect_tx(&full[s], 2 * TILE_B + ka * DLC_B + BC_B + (k == 0 ? ka * WDC_B : 0));
+        mbar_arrive_expect_tx(&full[s], 2 * TILE_B + ka * DLC_B + (k == 0 ? ka * WDC_B : 0));
         const int t = t0 + k * Q;
         if (k == 0)
           for (int a = 0; a < ka; ++a) tma_load_2d(sm + OFF_WD + a * WDC_B, &tmWD, &full[s], a * KA, c0);
         tma_load_3d(sm + OFF_X + s * TILE_B, &tmX, &full[s], c0, t, b);
         tma_load_3d(sm + OFF_G + s * TILE_B, &tmG, &full[s], c0, t, b);
         for (int a = 0; a < ka; ++a) tma_load_3d(sm + OFF_DL + s * DL_B + a * DLC_B, &tmDL, &full[s], a * KA, t, b);
-        for (int q = 0; q < 8; ++q) tma_load_3d(sm + OFF_BC + s * BC_B + q * BCC_B, &tmBC, &full[s], 32 * q, t, b);
       }
       if (k < nblk) {  // aborted: let the copies already issued land before smem goes away
         int never = 0;
@@ -829,246 +933,157 @@ __global__ void __launch_bounds__(NTHR, 1)
           mbar_wait(&full[j % ST], (j / ST) & 1u, nullptr, &never, 100000000ull);
       }
     }
-  } else if (warp == 11) {
-    // ------------------------------------------------------------ MMA issuer: a small
-    // dataflow scheduler over four tasks, each issued as soon as its inputs are ready
-    //   stage(ks):   dt projection and C B^T of a landed stage
-    //   release(kr): the stage of block kr back to the producer
-    //   chain(kc):   Y = G' C^T, G' += V B (the state products)
-    //   vm(kv):      Y += V M^T, then Y is complete
-    // Buffer reuse: DT / MR buffer ks & 1 held block ks - 2, consumed before gready /
-    // mready of that block (chain(ks - 2), vm(ks - 2) issued); the stage holds nothing the
-    // state products read (B^T and the C copy are separate).  Releases run in block order,
-    // so a vready / btready phase is never tested after the next phase of the same
-    // barrier completed (that needs the stage of block kr + 2, or kr + 3, loaded).
+  } else if (warp == 17) {
+    // ------------------------------------------------------------ TMA: B^T, C, M of each
+    // block (written beforehand by bc_gram_kernel) into double buffers
+    if (lane == 0) {
+      int nbt = 0, nm = 0;   // copies issued
+      for (int k = 0; k < nblk; ++k) {
+        const int i = k & 1, rec = b * nblk + k;
+        // B^T / C buffer i was last read by block k - 2's state products
+        if (k >= 2 && !mbar_wait(&dgready[i], ((k - 2) >> 1) & 1u, status, abort_flag)) break;
+        mbar_arrive_expect_tx(&btready[i], BT_B + CC_B);
+        tma_load_3d(sm + OFF_BT + i * BT_B, &tmBT, &btready[i], 0, 0, rec);
+        for (int q = 0; q < 4; ++q) tma_load_3d(sm + OFF_CC + i * CC_B + q * BCC_B, &tmC, &btready[i], 32 * q, 0, rec);
+        ++nbt;
+        // M buffer i was last read by block k - 2's V M^T
+        if (k >= 2 && !mbar_wait(&yready[i], ((k - 2) >> 1) & 1u, status, abort_flag)) break;
+        mbar_arrive_expect_tx(&mready[i], MT_B);
+        tma_load_3d(sm + OFF_MT + i * MT_B, &tmM, &mready[i], 0, 0, rec);
+        ++nm;
+      }
+      // let the last copies land before shared memory goes away
+      int never = 0;
+      for (int j = (nbt > 2 ? nbt - 2 : 0); j < nbt; ++j)
+        mbar_wait(&btready[j & 1], (j >> 1) & 1u, nullptr, &never, 100000000ull);
+      for (int j = (nm > 2 ? nm - 2 : 0); j < nm; ++j)
+        mbar_wait(&mready[j & 1], (j >> 1) & 1u, nullptr, &never, 100000000ull);
+    }
+  } else if (warp == 18) {
+    // ------------------------------------------------------------ MMA issuer, in a fixed
+    // order per block k (its inputs are ready, in the steady state, before it gets to them):
+    //   chain(k):     Y = G' C^T, G' += V B (the state products) -> dgready
+    //   vm(k):        Y += V M^T -> yready
+    //   stage(k + 2): the dt projection of block k + 2 -> dtready
+    //   release(k + 1): block k + 1's stage back to the producer
+    // so that while the state warps rescale G' for block k + 1 the tensor pipe works on
+    // vm(k) and the dt projection, and chain(k + 1) follows as soon as G' is ready.
+    // Buffer reuse: DT buffer k & 1 is rewritten by stage(k + 2) after chain(k) (the V/W
+    // warps read it before vready(k), the plain recurrence before gready(k)); the stage of
+    // block k + 1 holds only x, gate (read before vready(k + 1)) and dt_low (read by the dt
+    // projection, which the release commit tracks).
     if (lane == 0) {
       // descriptors of the first stage's tiles; every other tile is a fixed offset away
-      const uint64_t dBC = sdesc_sw128(sbase + OFF_BC, 16, 1024), dDL = sdesc_sw128(sbase + OFF_DL, 16, 1024),
-                     dWD = sdesc_sw128(sbase + OFF_WD, 16, 1024), dCC = sdesc_sw128(sbase + OFF_CC, 16, 1024),
-                     dBT = sdesc_sw128(sbase + OFF_BT, 16, 1024), dMT = sdesc_sw128(sbase + OFF_MT, 16, 1024);
-      int ks = 0, kc = 0, kv = 0, kr = 0;
+      const uint64_t dDL = sdesc_sw128(sbase + OFF_DL, 16, 1024), dWD = sdesc_sw128(sbase + OFF_WD, 16, 1024),
+                     dCC = sdesc_sw128(sbase + OFF_CC, 16, 1024), dBT = sdesc_sw128(sbase + OFF_BT, 16, 1024),
+                     dMT = sdesc_sw128(sbase + OFF_MT, 16, 1024);
       uint32_t n_yi = 0;   // completed phases of yidone (product-form blocks only)
-      unsigned long long t_last = 0;
-      uint32_t idle = 0;
-      while (kv < nblk) {
-        if (ks < nblk && ks <= kc + 1 && ks <= kv + 1 && mbar_try_wait(&full[ks % ST], (ks / ST) & 1u)) {
-          tc_fence_after();
-          const int s = ks % ST, i = ks & 1;
-          const uint64_t dl = sdesc_add(dDL, s * DL_B);
+      auto stage = [&](int ks) -> bool {   // dt = W_dt dt_low^T of block ks into DT buffer ks & 1
+        if (!mbar_wait(&full[ks % ST], (ks / ST) & 1u, status, abort_flag)) return false;
+        tc_fence_after();
+        const int i = ks & 1;
+        const uint64_t dl = sdesc_add(dDL, (ks % ST) * DL_B);
+#pragma unroll
+        for (int j = 0; j < KA / 16; ++j)
+          umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_add(dWD, 32 * j), sdesc_add(dl, 32 * j), IDESC_DT, j != 0);
+        if (ka > 1) {
 #pragma unroll
           for (int j = 0; j < KA / 16; ++j)
-            umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_add(dWD, 32 * j), sdesc_add(dl, 32 * j), IDESC_DT, j != 0);
-          if (ka > 1) {
-#pragma unroll
-            for (int j = 0; j < KA / 16; ++j)
-              umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_add(dWD, WDC_B + 32 * j), sdesc_add(dl, DLC_B + 32 * j),
-                           IDESC_DT, 1u);
-          }
-          umma_commit(&dtready[i]);
-          // C B^T: A = a C chunk (128 rows read, rows 32..127 land in TMEM lanes nobody
-          // reads), B = the B chunk of the same columns; K = n = 128 = 16 tf32 steps
-          const uint64_t bc = sdesc_add(dBC, s * BC_B);
+            umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_add(dWD, WDC_B + 32 * j), sdesc_add(dl, DLC_B + 32 * j),
+                         IDESC_DT, 1u);
+        }
+        umma_commit(&dtready[i]);
+        return true;
+      };
+      auto release = [&](int kr) -> bool {   // x and gate read (vready); the dt projection tracked
+        if (!mbar_wait(&vready[kr % 3], (kr / 3) & 1u, status, abort_flag)) return false;
+        umma_commit(&empty[kr % ST]);
+        return true;
+      };
+      bool ok = true;
+      for (int k = 0; k < 2 && k < nblk && ok; ++k) ok = stage(k);
+      if (ok && nblk > 0) ok = release(0);
+      for (int k = 0; k < nblk && ok; ++k) {
+        const int i = k & 1, vb = k % 3;
+        // ---- chain(k)
+        if (!mbar_wait(gready, k & 1u, status, abort_flag) ||
+            !mbar_wait(&btready[i], (k >> 1) & 1u, status, abort_flag))
+          break;
+        tc_fence_after();
+        const bool plain = sAny[vb] != 0;
+        if (!plain) {
+          const uint64_t cc = sdesc_add(dCC, i * CC_B), bt = sdesc_add(dBT, i * BT_B);
+          // Y = G' C^T (K = n = 128), then G' += V B (K = s = 32, B^T rows n).  The update
+          // writes the TMEM G' the first product reads as its A operand: it is issued only
+          // once that product has completed (an MMA issued behind another is not held back
+          // from writing TMEM the earlier one still reads)
 #pragma unroll
           for (int q = 0; q < 4; ++q)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              umma_tf32_ss(tmem + COL_MR + 32 * i, sdesc_add(bc, (4 + q) * BCC_B + 32 * j), sdesc_add(bc, q * BCC_B + 32 * j),
+              umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_GP + 32 * q + 8 * j, sdesc_add(cc, q * BCC_B + 32 * j),
                            IDESC_Q, (q | j) != 0);
-          umma_commit(&mraw[i]);
-          ++ks;
-          idle = 0;
-          continue;
-        }
-        // release(kr): block kr's stage is free once its dt projection and C B^T are done
-        // (what the commit tracks), x and gate were read (vready) and B, C copied (btready)
-        // -- a period before its state products, so the next load has two periods to land
-        if (kr < ks && mbar_try_wait(&vready[kr % 3], (kr / 3) & 1u) &&
-            mbar_try_wait(&btready[kr & 1], (kr >> 1) & 1u)) {
-          umma_commit(&empty[kr % ST]);
-          ++kr;
-          idle = 0;
-          continue;
-        }
-        if (kc < kr && mbar_try_wait(gready, kc & 1u)) {
-          tc_fence_after();
-          if (!sAny[kc % 3]) {
-            const int i = kc & 1, vb = kc % 3;
-            const uint64_t cc = sdesc_add(dCC, i * CC_B), bt = sdesc_add(dBT, i * BT_B);
-            // Y = G' C^T (K = n = 128), then G' += V B (K = s = 32, B^T rows n).  The update
-            // writes the TMEM G' the first product reads as its A operand: it is issued only
-            // once that product has completed (an MMA issued behind another is not held back
-            // from writing TMEM the earlier one still reads)
+          umma_commit(yidone);
+          if (!mbar_wait(yidone, n_yi & 1u, status, abort_flag)) break;
+          ++n_yi;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_GP + 32 * q + 8 * j, sdesc_add(cc, q * BCC_B + 32 * j),
-                             IDESC_Q, (q | j) != 0);
-            umma_commit(yidone);
-            if (!mbar_wait(yidone, n_yi & 1u, status, abort_flag)) break;
-            ++n_yi;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              umma_tf32_ts(tmem + COL_GP, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(bt, 32 * j), IDESC_N, 1);
-          }
-          umma_commit(&dgready[kc & 1]);
-          ++kc;
-          idle = 0;
-          continue;
+          for (int j = 0; j < 4; ++j)
+            umma_tf32_ts(tmem + COL_GP, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(bt, 32 * j), IDESC_N, 1);
         }
-        if (kv < kc && mbar_try_wait(&mready[kv & 1], (kv >> 1) & 1u)) {
-          tc_fence_after();
-          if (!sAny[kv % 3]) {  // Y += V M^T (K = s = 32)
-            const int i = kv & 1, vb = kv % 3;
-            const uint64_t mt = sdesc_add(dMT, i * MT_B);
+        umma_commit(&dgready[i]);
+        // ---- vm(k): Y += V M^T (K = s = 32), then Y is complete
+        if (!mbar_wait(&mready[i], (k >> 1) & 1u, status, abort_flag)) break;
+        tc_fence_after();
+        if (!plain) {
+          const uint64_t mt = sdesc_add(dMT, i * MT_B);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(mt, 32 * j), IDESC_Q, 1);
-          }
-          umma_commit(&yready[kv & 1]);
-          ++kv;
-          idle = 0;
-          continue;
+          for (int j = 0; j < 4; ++j)
+            umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(mt, 32 * j), IDESC_Q, 1);
         }
-        // nothing ready: back off briefly, give up after kWaitLimitNs without progress
-        ++idle;
-        if (idle > 8u) __nanosleep(32);
-        if ((idle & 63u) == 0u) {
-          if (*abort_flag) break;
-          const unsigned long long now = globaltimer();
-          if (idle == 64u) {
-            t_last = now;
-          } else if (now - t_last > kWaitLimitNs) {
-            atomicExch(status, kStatusTimeout);
-            *abort_flag = 1;
-            break;
-          }
-        }
+        umma_commit(&yready[i]);
+        // ---- the dt projection two blocks ahead, then the next stage's release
+        if (k + 2 < nblk && !stage(k + 2)) break;
+        if (k + 1 < nblk && !release(k + 1)) break;
       }
       umma_commit(mma_done);
       int never = 0;
       mbar_wait(mma_done, 0, nullptr, &never, 100000000ull);
     }
   } else if (warp >= 8) {
-    // ------------------------------------------------------------ B^T, the C copy, M
-    const int wq = warp - 8;
-    for (int k = 0; k < nblk; ++k) {
-      const int s = k % ST, i = k & 1;
-      bool ok = mbar_wait(&full[s], (k / ST) & 1u, status, abort_flag);
-      // B^T / C copy buffer i was last read by block k - 2's state products
-      if (ok && k >= 2) ok = mbar_wait(&dgready[i], ((k - 2) >> 1) & 1u, status, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      const uint8_t* stg = sm + OFF_BC + s * BC_B;
-      {  // B^T [n][s] for n in [64 wq, 64 wq + 64), s = lane
-        const int sr = lane;
-        const uint8_t* src = stg + (sr >> 3) * 1024 + (sr & 7) * 128;
-        uint8_t* bt = sm + OFF_BT + i * BT_B;
-#pragma unroll 4
-        for (int nn = 0; nn < 64; nn += 4) {
-          const int n = 64 * wq + nn;
-          const float4 v = *reinterpret_cast<const float4*>(src + (n >> 5) * BCC_B + ((((n & 31) >> 2) ^ (sr & 7)) << 4));
-          const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) *reinterpret_cast<uint32_t*>(bt + bt_off(n + e, sr)) = tf32_round(vv[e]);
-        }
-      }
-      {  // C chunks 2 wq, 2 wq + 1 (same layout), rounded to tf32
-        const uint4* src = reinterpret_cast<const uint4*>(stg + (4 + 2 * wq) * BCC_B);
-        uint4* dst = reinterpret_cast<uint4*>(sm + OFF_CC + i * CC_B + 2 * wq * BCC_B);
-#pragma unroll 4
-        for (int j = lane; j < 2 * BCC_B / 16; j += 32) {
-          const uint4 v = src[j];
-          dst[j] = make_uint4(tf32_round(__uint_as_float(v.x)), tf32_round(__uint_as_float(v.y)),
-                              tf32_round(__uint_as_float(v.z)), tf32_round(__uint_as_float(v.w)));
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&btready[i]);
-      if (wq == 0) {  // row t = lane of M (K-major, 128-byte swizzle), from TMEM lanes 0-31
-        ok = mbar_wait(&mraw[i], (k >> 1) & 1u, status, abort_flag);
-        // M buffer i was last read by block k - 2's V M^T
-        if (ok && k >= 2) ok = mbar_wait(&yready[i], ((k - 2) >> 1) & 1u, status, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after();
-        const int t = lane;
-        uint32_t r[32];
-        tmem_ld32(tmem + COL_MR + 32 * i, r);
-        tmem_wait_ld();
-        uint8_t* row = sm + OFF_MT + i * MT_B + (t >> 3) * 1024 + (t & 7) * 128;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint32_t v[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) v[e] = 4 * j + e <= t ? tf32_round(__uint_as_float(r[4 * j + e])) : 0u;
-          *reinterpret_cast<uint4*>(row + ((j ^ (t & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&mready[i]);
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ channel warps
-    const int qd = warp & 3, half = warp >> 2;
+    // ------------------------------------------------------------ V/W warps: for every
+    // block, dt (softplus of W_dt dt_low^T + b_dt), the half-block decay sums, and V, W
+    // into TMEM buffer k % 3: V = dt x 2^(lambda - r), W = gate 2^(r - lambda) (r: lambda
+    // after the first half), or for a block that runs the plain recurrence V = dt x,
+    // W = gate.  Warp 8 + w: TMEM quadrant w % 4, half w / 4 of the block's steps.
+    const int qd = warp & 3, half = (warp - 8) >> 2;
     const int cl = qd * 32 + lane, c = c0 + cl;
     const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const float A2 = c < Di ? expf(a_log[c]) * 1.4426950408889634f : 0.f;  // |A| / ln 2
     const float bdt = c < Di ? b_dt[c] : 0.f;
-    __nv_bfloat16* ycol = y + static_cast<long long>(b) * T * y_ld + c;
-    __nv_bfloat16* ybase = y + static_cast<long long>(b) * T * y_ld;
-    bool stop = false;   // uniform over the channel threads: leave the block loop
-    const int c4 = c0 + qd * 32 + (lane & ~3);   // this lane's 4-channel store group
     bool fail = false;
-    // the state entering row t0 (raw: the first block applies only its own scale)
 #pragma unroll 1
-    for (int part = 0; part < 2; ++part) {
-      const int n0 = 64 * half + 32 * part;
-      uint32_t hz[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) hz[j] = 0u;
-      if (h0 && c < Di) {
-        const float4* hp = reinterpret_cast<const float4*>(h0 + b * h0_bstride + static_cast<long long>(c) * NS + n0);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 v = hp[j];
-          hz[4 * j] = __float_as_uint(v.x);
-          hz[4 * j + 1] = __float_as_uint(v.y);
-          hz[4 * j + 2] = __float_as_uint(v.z);
-          hz[4 * j + 3] = __float_as_uint(v.w);
-        }
-      }
-      tmem_st32(tl + COL_GP + n0, hz);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-
-    // dt of block k's half (steps past T: dt = 0, the state stays), from W_dt dt_low^T
-    auto load_dt = [&](int k, float (&dtv)[HQ]) {
-      uint32_t z[HQ];
-      tmem_ld16(tl + COL_DT + 32 * (k & 1) + HQ * half, z);
-      tmem_wait_ld();
-      const int t_end = T - (t0 + k * Q + HQ * half);
-#pragma unroll
-      for (int j = 0; j < HQ; j += 2) {
-        float2 d = softplus2(make_float2(__uint_as_float(z[j]) + bdt, __uint_as_float(z[j + 1]) + bdt));
-        if (j >= t_end) d.x = 0.f;
-        if (j + 1 >= t_end) d.y = 0.f;
-        dtv[j] = d.x;
-        dtv[j + 1] = d.y;
-      }
-    };
-    // V and W of block k into TMEM buffer k % 3: V = dt x 2^(lambda - r), W = gate
-    // 2^(r - lambda), or for a block that runs the plain recurrence V = dt x, W = gate.
-    // Returns the block's flag and this channel's two half-block decay sums.
-    auto form_vw = [&](int k, float& S0, float& S1) -> bool {
+    for (int k = 0; k < nblk; ++k) {
       const int s = k % ST, vb = k % 3;
+      // buffer vb was last read by the output of block k - 3 (after that block's products)
       fail = fail || !__all_sync(0xffffffffu, mbar_wait(&full[s], (k / ST) & 1u, status, abort_flag) &&
-                                                  mbar_wait(&dtready[k & 1], (k >> 1) & 1u, status, abort_flag));
+                                                  mbar_wait(&dtready[k & 1], (k >> 1) & 1u, status, abort_flag) &&
+                                                  (k < 3 || mbar_wait(&wdone[vb], ((k - 3) / 3) & 1u, status, abort_flag)));
+      // dt of this half (steps past T: dt = 0, the state stays)
       float dtv[HQ];
       if (!fail) {
         tc_fence_after();
-        load_dt(k, dtv);
+        uint32_t z[HQ];
+        tmem_ld16(tl + COL_DT + 32 * (k & 1) + HQ * half, z);
+        tmem_wait_ld();
+        const int t_end = T - (t0 + k * Q + HQ * half);
+#pragma unroll
+        for (int j = 0; j < HQ; j += 2) {
+          float2 d = softplus2(make_float2(__uint_as_float(z[j]) + bdt, __uint_as_float(z[j + 1]) + bdt));
+          if (j >= t_end) d.x = 0.f;
+          if (j + 1 >= t_end) d.y = 0.f;
+          dtv[j] = d.x;
+          dtv[j + 1] = d.y;
+        }
       } else {
 #pragma unroll
         for (int j = 0; j < HQ; ++j) dtv[j] = 0.f;
@@ -1080,18 +1095,18 @@ __global__ void __launch_bounds__(NTHR, 1)
       float* ss = sS + (k & 1) * 2 * CH;
       ss[half * CH + cl] = S;
       // one reduction in the common case: "some channel needs the plain recurrence or some
-      // thread failed"; only when it is set, a second one tells the two apart
-      bool any = bar_red_or(1, NCHT, fail || !(S <= kRange));
-      if (any && bar_red_or(1, NCHT, fail)) stop = true;   // uniform
-      S0 = ss[cl];
-      S1 = ss[CH + cl];
+      // thread failed"; only when it is set, a second one tells the two apart (both
+      // uniform over the V/W threads, which therefore leave the loop together)
+      const bool any = bar_red_or(1, NVT, fail || !(S <= kRange));
+      const bool stop = any && bar_red_or(1, NVT, fail);
+      const float S0 = ss[cl];
       if (!fail) {
-        // x and gate of this half (explicit shared loads, all issued first), the running
-        // decay mu = lambda - r (one dependent FMA per step), then the exponentials, which
-        // are independent of one another; the block-uniform branch stays outside the loops
+        // x and gate of this half (shared loads issued first), the running decay
+        // mu = lambda - r (one dependent FMA per step), then the exponentials, which are
+        // independent of one another; the block-uniform branch stays outside the loops
         const uint32_t xa = sbase + OFF_X + s * TILE_B + cl * 2 + HQ * half * 256;
         const uint32_t ga = sbase + OFF_G + s * TILE_B + cl * 2 + HQ * half * 256;
-        float xv[HQ], gv[HQ], mu[HQ];
+        float xv[HQ], gv[HQ];
 #pragma unroll
         for (int j = 0; j < HQ; ++j) {
           xv[j] = bf2f(static_cast<uint16_t>(lds_u16(xa + j * 256)));
@@ -1099,7 +1114,8 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
         uint32_t vr[HQ], wr[HQ];
         if (!any) {
-          float m = half ? 0.f : -S;
+          float mu[HQ];
+          float m = half ? 0.f : -S0;
 #pragma unroll
           for (int j = 0; j < HQ; ++j) {
             m = fmaf(A2, dtv[j], m);
@@ -1127,115 +1143,167 @@ __global__ void __launch_bounds__(NTHR, 1)
         tmem_st16(tl + COL_W + 32 * vb + HQ * half, wr);
         tmem_wait_st();
       }
-      if (threadIdx.x == 0) sAny[vb] = any ? 1 : 0;
+      if (warp == 8 && lane == 0) sAny[vb] = any ? 1 : 0;
       tc_fence_before();
       mbar_arrive(&vready[vb]);
-      return any;
+      if (stop) break;
+    }
+  } else {
+    // ------------------------------------------------------------ state warps: per block,
+    // rescale G' (or run the plain recurrence), hand the block to the MMA thread, then
+    // write the previous block's y.  Warp w: TMEM quadrant w % 4, half w / 4 of G''s
+    // columns and of the block's output rows.
+    const int qd = warp & 3, half = warp >> 2;
+    const int cl = qd * 32 + lane, c = c0 + cl;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const float A2 = c < Di ? expf(a_log[c]) * 1.4426950408889634f : 0.f;  // |A| / ln 2
+    const float bdt = c < Di ? b_dt[c] : 0.f;
+    __nv_bfloat16* ycol = y + static_cast<long long>(b) * T * y_ld + c;
+    __nv_bfloat16* ybase = y + static_cast<long long>(b) * T * y_ld;
+    const int c4 = c0 + qd * 32 + (lane & ~3);   // this lane's 4-channel store group
+    bool fail = false;
+    // the state entering row t0, columns [64 half, 64 half + 64) (raw: the first block
+    // applies only its own scale)
+#pragma unroll 1
+    for (int part = 0; part < 2; ++part) {
+      const int n0 = 64 * half + 32 * part;
+      uint32_t hz[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) hz[j] = 0u;
+      if (h0 && c < Di) {
+        const float4* hp = reinterpret_cast<const float4*>(h0 + b * h0_bstride + static_cast<long long>(c) * NS + n0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 v = hp[j];
+          hz[4 * j] = __float_as_uint(v.x);
+          hz[4 * j + 1] = __float_as_uint(v.y);
+          hz[4 * j + 2] = __float_as_uint(v.z);
+          hz[4 * j + 3] = __float_as_uint(v.w);
+        }
+      }
+      tmem_st32(tl + COL_GP + n0, hz);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    // y = W * Y over this half's 16 rows of block jb
+    auto out_block = [&](int jb) {
+      const int i = jb & 1;
+      tc_fence_after();
+      uint32_t yv[HQ], wv[HQ];
+      tmem_ld16(tl + COL_Y + 32 * i + HQ * half, yv);
+      tmem_ld16(tl + COL_W + 32 * (jb % 3) + HQ * half, wv);
+      tmem_wait_ld();
+      float o[HQ];
+#pragma unroll
+      for (int j = 0; j < HQ; ++j) o[j] = __uint_as_float(yv[j]) * __uint_as_float(wv[j]);
+      store_y16(ybase, y_ld, t0 + jb * Q + HQ * half, T, c4, c4 < Di, o);
     };
 
-    float cS0 = 0.f, cS1 = 0.f;
-    bool c_any = nblk > 0 ? form_vw(0, cS0, cS1) : false;
-    if (stop) fail = true;
     float pS1 = 0.f;        // the previous block's second-half decay sum
     bool prev_any = true;   // the previous block left the raw state in G' (so does the start)
-    for (int k = 0; k < nblk && !stop; ++k) {
-      // ---- G' for block k: block k - 1's state products are done
-      if (k > 0 && !fail)
-        fail = !__all_sync(0xffffffffu, mbar_wait(&dgready[(k - 1) & 1], ((k - 1) >> 1) & 1u, status, abort_flag));
-      if (!fail) {
+#pragma unroll 1
+    for (int k = 0; k < nblk; ++k) {
+      // ---- block k's sums and flag (V/W done) and G' (block k - 1's products done)
+      if (k > 0)
+        fail = fail || !__all_sync(0xffffffffu, mbar_wait(&dgready[(k - 1) & 1], ((k - 1) >> 1) & 1u, status, abort_flag));
+      fail = fail || !__all_sync(0xffffffffu, mbar_wait(&vready[k % 3], (k / 3) & 1u, status, abort_flag));
+      if (fail) break;
+      const float* ss = sS + (k & 1) * 2 * CH;
+      const float cS0 = ss[cl], cS1 = ss[CH + cl];
+      const bool c_any = sAny[k % 3] != 0;
+      tc_fence_after();
+      if (!c_any) {
         // G' <- 2^-e_in 2^-e_out G'; one multiply while 2^-(e_in + e_out) is a normal float
-        const float e_in = prev_any ? 0.f : pS1, e_out = c_any ? 0.f : cS0;
+        const float e_in = prev_any ? 0.f : pS1, e_out = cS0;
         const bool one = __all_sync(0xffffffffu, e_in + e_out < 120.f);
         const float f1 = ex2_approx(one ? -(e_in + e_out) : -e_in), f2 = one ? 1.f : ex2_approx(-e_out);
         const float2 fa = make_float2(f1, f1), fb = make_float2(f2, f2);
-        tc_fence_after();
-        // both 32-column pieces of this half in flight at once: one load wait, one store wait
-        const uint32_t col = tl + COL_GP + 64 * half;
-        uint32_t g[64];
-        tmem_ld32(col, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
-        tmem_ld32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
-        tmem_wait_ld();
-        if (one) {
 #pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const float2 v = __fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa);
-            g[j] = __float_as_uint(v.x);
-            g[j + 1] = __float_as_uint(v.y);
-          }
-        } else {
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t col = tl + COL_GP + 64 * half + 32 * part;
+          uint32_t g[32];
+          tmem_ld32(col, g);
+          tmem_wait_ld();
+          if (one) {
 #pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const float2 v =
-                __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa), fb);
-            g[j] = __float_as_uint(v.x);
-            g[j + 1] = __float_as_uint(v.y);
+            for (int j = 0; j < 32; j += 2) {
+              const float2 v = __fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa);
+              g[j] = __float_as_uint(v.x);
+              g[j + 1] = __float_as_uint(v.y);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float2 v =
+                  __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa), fb);
+              g[j] = __float_as_uint(v.x);
+              g[j + 1] = __float_as_uint(v.y);
+            }
           }
+          tmem_st32(col, g);
         }
-        tmem_st32(col, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
-        tmem_st32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
         tmem_wait_st();
-      }
-      // ---- large decays: the plain recurrence over block k on the raw state in G'
-      if (c_any) {
-        tc_fence_before();
-        bar_sync_n(1, NCHT);  // both halves' G' columns are stored
+      } else if (half == 1) {
+        // ---- large decays: the plain recurrence over block k by the half-1 warps (one
+        // thread per channel, all 128 state columns, 8 at a time).  G' holds 2^S1 times
+        // the state after a product-form block: that factor is taken out as it is loaded.
+        const float f_in = prev_any ? 1.f : ex2_approx(-pS1);
         const int i = k & 1, vb = k % 3;
-        if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(&btready[i], (k >> 1) & 1u, status, abort_flag));
-        if (half == 1 && !fail) {
+        fail = !__all_sync(0xffffffffu, mbar_wait(&btready[i], (k >> 1) & 1u, status, abort_flag));
+        if (!fail) {
           tc_fence_after();
           const uint8_t* bt = sm + OFF_BT + i * BT_B;
           const uint8_t* cc = sm + OFF_CC + i * CC_B;
 #pragma unroll 1
-          for (int th = 0; th < Q; th += HQ) {
-            uint32_t zq[HQ], uq[HQ], gq[HQ];
-            tmem_ld16(tl + COL_DT + 32 * i + th, zq);
-            tmem_ld16(tl + COL_V + 32 * vb + th, uq);
-            tmem_ld16(tl + COL_W + 32 * vb + th, gq);
+          for (int th = 0; th < Q; th += QQ) {
+            uint32_t zq[QQ], uq[QQ], gq[QQ];
+            tmem_ld8(tl + COL_DT + 32 * i + th, zq);
+            tmem_ld8(tl + COL_V + 32 * vb + th, uq);
+            tmem_ld8(tl + COL_W + 32 * vb + th, gq);
             tmem_wait_ld();
             const int t_end = T - (t0 + k * Q + th);
-            float a[HQ], y16[HQ];
+            float a[QQ], yq[QQ];
 #pragma unroll
-            for (int j = 0; j < HQ; ++j) {
+            for (int j = 0; j < QQ; ++j) {
               const float dt = j < t_end ? softplus_f(__uint_as_float(zq[j]) + bdt) : 0.f;
               a[j] = ex2_approx(-A2 * dt);
-              y16[j] = 0.f;
+              yq[j] = 0.f;
             }
+            const float fq = th == 0 ? f_in : 1.f;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-              uint32_t hr[32];
-              tmem_ld32(tl + COL_GP + 32 * q, hr);
+            for (int q = 0; q < NS / 8; ++q) {
+              uint32_t hr[8];
+              tmem_ld8(tl + COL_GP + 8 * q, hr);
               tmem_wait_ld();
-              float h[32];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) h[j] = __uint_as_float(hr[j]);
-#pragma unroll 1
-              for (int tt = 0; tt < HQ; ++tt) {
+              for (int j = 0; j < 8; ++j) hr[j] = __float_as_uint(__uint_as_float(hr[j]) * fq);
+#pragma unroll
+              for (int tt = 0; tt < QQ; ++tt) {
                 const int t = th + tt;
                 const float u = __uint_as_float(uq[tt]);
                 float acc = 0.f;
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                  const float4 cv = *reinterpret_cast<const float4*>(cc + cc_off(t, 32 * q + j));
+                for (int j = 0; j < 8; j += 4) {
+                  const float4 cv = *reinterpret_cast<const float4*>(cc + cc_off(t, 8 * q + j));
                   const float cq[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
                   for (int e = 0; e < 4; ++e) {
-                    const float bn = *reinterpret_cast<const float*>(bt + bt_off(32 * q + j + e, t));
-                    h[j + e] = fmaf(a[tt], h[j + e], u * bn);
-                    acc = fmaf(cq[e], h[j + e], acc);
+                    const float bn = *reinterpret_cast<const float*>(bt + bt_off(8 * q + j + e, t));
+                    const float h = fmaf(a[tt], __uint_as_float(hr[j + e]), u * bn);
+                    hr[j + e] = __float_as_uint(h);
+                    acc = fmaf(cq[e], h, acc);
                   }
                 }
-                y16[tt] += acc;
+                yq[tt] += acc;
               }
-#pragma unroll
-              for (int j = 0; j < 32; ++j) hr[j] = __float_as_uint(h[j]);
-              tmem_st32(tl + COL_GP + 32 * q, hr);
+              tmem_st8(tl + COL_GP + 8 * q, hr);
               tmem_wait_st();
             }
             if (c < Di) {
 #pragma unroll
-              for (int j = 0; j < HQ; ++j) {
+              for (int j = 0; j < QQ; ++j) {
                 const int t = t0 + k * Q + th + j;
-                if (t < T) ycol[static_cast<long long>(t) * y_ld] = __float2bfloat16_rn(__uint_as_float(gq[j]) * y16[j]);
+                if (t < T) ycol[static_cast<long long>(t) * y_ld] = __float2bfloat16_rn(__uint_as_float(gq[j]) * yq[j]);
               }
             }
           }
@@ -1243,53 +1311,26 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
       tc_fence_before();
       mbar_arrive(gready);
-      // ---- output of block k - 1: y = W * Y.  Every phase of yready is waited for, even
-      // after a plain block (whose y went out already): a skipped phase would let the parity
-      // test of the next wait on the same barrier pass a phase early
+      if (fail) break;
+      // ---- output of block k - 1.  Every phase of yready is waited for, even after a
+      // plain block (whose y went out already): a skipped phase would let the parity test
+      // of the next wait on the same barrier pass a phase early
       if (k > 0) {
-        const int jb = k - 1, i = jb & 1;
-        if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(&yready[i], (jb >> 1) & 1u, status, abort_flag));
-        if (!fail && !prev_any) {
-          tc_fence_after();
-          uint32_t yv[HQ], wv[HQ];
-          tmem_ld16(tl + COL_Y + 32 * i + HQ * half, yv);
-          tmem_ld16(tl + COL_W + 32 * (jb % 3) + HQ * half, wv);
-          tmem_wait_ld();
-          float o[HQ];
-#pragma unroll
-          for (int j = 0; j < HQ; ++j) o[j] = __uint_as_float(yv[j]) * __uint_as_float(wv[j]);
-          store_y16(ybase, y_ld, t0 + jb * Q + HQ * half, T, c4, c4 < Di, o);
-        }
+        const int jb = k - 1;
+        fail = !__all_sync(0xffffffffu, mbar_wait(&yready[jb & 1], (jb >> 1) & 1u, status, abort_flag));
+        if (fail) break;
+        if (!prev_any) out_block(jb);
+        mbar_arrive(&wdone[jb % 3]);   // W and V of block k - 1 are free
       }
       pS1 = cS1;
       prev_any = c_any;
-      // ---- V and W of block k + 1 (their buffer's last reader, block k - 2's V M^T,
-      // completed before the output of block k - 2 above, an iteration ago)
-      // a failure anywhere in this iteration (or another role's abort, seen by the waits)
-      // reaches every channel thread through form_vw's reduction
-      if (k + 1 < nblk) c_any = form_vw(k + 1, cS0, cS1);
-      if (stop) {
-        fail = true;
-        break;
-      }
     }
     // ---- output of the last block and the state after the last row
     if (__all_sync(0xffffffffu, !fail && nblk > 0 && !*abort_flag)) {
       const int jb = nblk - 1, i = jb & 1;
       const bool got = __all_sync(0xffffffffu, mbar_wait(&dgready[i], (jb >> 1) & 1u, status, abort_flag));
-      if (got && !prev_any) {
-        if (__all_sync(0xffffffffu, mbar_wait(&yready[i], (jb >> 1) & 1u, status, abort_flag))) {
-          tc_fence_after();
-          uint32_t yv[HQ], wv[HQ];
-          tmem_ld16(tl + COL_Y + 32 * i + HQ * half, yv);
-          tmem_ld16(tl + COL_W + 32 * (jb % 3) + HQ * half, wv);
-          tmem_wait_ld();
-          float o[HQ];
-#pragma unroll
-          for (int j = 0; j < HQ; ++j) o[j] = __uint_as_float(yv[j]) * __uint_as_float(wv[j]);
-          store_y16(ybase, y_ld, t0 + jb * Q + HQ * half, T, c4, c4 < Di, o);
-        }
-      }
+      if (got && !prev_any && __all_sync(0xffffffffu, mbar_wait(&yready[i], (jb >> 1) & 1u, status, abort_flag)))
+        out_block(jb);
       if (got && h_out) {
         // 2^-S1 (G' + dG) after a product-form block, the raw state after a plain one
         const float f = prev_any ? 1.f : ex2_approx(-pS1);
@@ -1318,26 +1359,36 @@ __global__ void __launch_bounds__(NTHR, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 11) {
+  if (warp == 18) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
 cudaError_t launch_tc128(const ScanDesc& s, cudaStream_t st) {
-  CUtensorMap tx, td, tg, tb, tw;
+  if (!s.mgram || !a16(s.mgram)) return cudaErrorInvalidValue;
+  const int nblk = (s.T - s.t0 + Q - 1) / Q;
+  const long long nrec = static_cast<long long>(s.batch) * (nblk > 0 ? nblk : 1);
+  uint8_t* rec = static_cast<uint8_t*>(s.mgram);
+  CUtensorMap tx, td, tg, tw, tm, tbt, tc;
   const bool ok =
+      map_rec_f32(&tm, rec, Q, Q, Q * 4, nrec, GREC_B, Q, Q) &&
+      map_rec_f32(&tbt, rec + MT_B, Q, NS, Q * 4, nrec, GREC_B, Q, NS) &&
+      map_rec_f32(&tc, rec + MT_B + BT_B, NS, Q, NS * 4, nrec, GREC_B, 32, Q) &&
       map3d(&tx, s.x, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
       map3d(&tg, s.gate, false, s.batch, s.T, s.d_inner, s.d_inner, CH, Q, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      map3d(&tb, s.bc, true, s.batch, s.T, 2 * NS, 2 * NS, 32, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
       map3d(&td, s.dt_low, false, s.batch, s.T, s.dt_rank, s.dt_rank, KA, Q, CU_TENSOR_MAP_SWIZZLE_128B) &&
       map2d_sw128(&tw, s.w_dt, s.d_inner, s.dt_rank, s.dt_rank, KA, CH);
   if (!ok) return cudaErrorNotSupported;
   static std::atomic<uint64_t> attr_done{0};
   if (cudaError_t e = smem_attr_once(scan_tc128_kernel, SMEM_TOTAL, attr_done)) return e;
   const int ka = (s.dt_rank + KA - 1) / KA;
+  if (nblk > 0) {
+    if (cudaError_t e = launch(bc_gram_kernel, dim3(nblk, s.batch), dim3(256), 0, st, s.bc, s.T, s.t0, nblk, rec))
+      return e;
+  }
   dim3 grid((s.d_inner + CH - 1) / CH, s.batch);
-  return launch(scan_tc128_kernel, grid, dim3(NTHR), SMEM_TOTAL, st, tx, td, tg, tb, tw, s.a_log, s.b_dt,
+  return launch(scan_tc128_kernel, grid, dim3(NTHR2), SMEM_TOTAL, st, tx, td, tg, tw, tm, tbt, tc, s.a_log, s.b_dt,
                 static_cast<__nv_bfloat16*>(s.y), s.y_ld, s.T, s.d_inner, ka, s.h_out, s.t0, s.h0, s.h0_bstride,
                 s.status);
 }
@@ -1352,6 +1403,12 @@ bool scan_tc_fuses_dt(const ScanDesc& s) {
   return s.bf16 && rank_ok && !s.a_per_state && (s.d_inner * 2) % 16 == 0 && (s.y_ld * 2) % 16 == 0 && a16(s.x) &&
          a16(s.gate) && a16(s.bc) && a16(s.y) && a16(s.dt_low) && a16(s.w_dt) && s.b_dt != nullptr &&
          (s.h0 == nullptr || a16(s.h0)) && (s.h_out == nullptr || a16(s.h_out));
+}
+
+size_t scan_mgram_bytes(const ScanDesc& s) {
+  if (s.d_state != t128::NS || !s.dt_low || s.T <= s.t0) return 0;
+  const size_t nblk = static_cast<size_t>(s.T - s.t0 + t128::Q - 1) / t128::Q;
+  return static_cast<size_t>(s.batch) * nblk * t128::GREC_B;
 }
 
 // bf16, d_state 16 or 128, 16-byte aligned operands and row strides (checked by the

@@ -365,8 +365,10 @@ HYMBA_API hymba_status_t hymba_selective_scan(const void* x, const void* dt, con
  * or d_state 128 with dt_rank a multiple of 8 up to 128; 16-byte aligned operands and
  * row strides) dt is formed block by block inside the scan and never stored; otherwise
  * it is computed into the workspace first.
- * hymba_selective_scan_dtproj_workspace_size gives the bytes needed (256 for the fused
- * kernels: the status word); HYMBA_ERR_WORKSPACE when ws_bytes is smaller.
+ * hymba_selective_scan_dtproj_workspace_size gives the bytes needed (for the fused
+ * kernels the 256-byte status word, plus for d_state 128 36 KB per sequence and 32 rows
+ * for the operands every channel shares: C B^T, B^T and C of each block); HYMBA_ERR_WORKSPACE
+ * when ws_bytes is smaller.
  */
 HYMBA_API size_t hymba_selective_scan_dtproj_workspace_size(int batch, int T, int d_inner, int d_state,
                                                             int dt_rank, hymba_dtype_t dtype);

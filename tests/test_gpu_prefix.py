@@ -18,6 +18,11 @@ from gpu_util import assert_close, dev, requires_cuda, status_ok, to_np
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
 
+# Two GPU paths over the same input (prefixed call vs the full layer) agree to fp32 rounding
+# before the bf16 stores; the largest output can still land one bf16 unit apart, 2^-7 of
+# its magnitude.
+PATH_TOL = 2.0 ** -7
+
 
 def _prefixed_chain(wl, x, meta, dps, every_layer=False):
     """Every layer of the workload through records + prefixed calls (a pair: the consumer's
@@ -93,7 +98,7 @@ def test_prefixed_kv_pair_swa_dstate128_matches_oracle_and_full_path():
     producer on X and meta, the consumer on the producer's GPU output rows and K/V (fed the
     oracle's own fp64 producer output instead, the consumer differs by ~1e-2 from
     bf16-rounding that input alone: the pair amplifies input rounding).  Against the full
-    path (2e-3): the prefixed producer with hymba_layer_fwd on the same X, the prefixed
+    path (one bf16 unit of the largest output): the prefixed producer with hymba_layer_fwd on the same X, the prefixed
     consumer with hymba_layer_fwd on the prefixed producer's output and K/V."""
     wl = synth.workload("hymba1p5b_kvpair", batch=2, seq_len=400, window=96, d_model=512, n_q_heads=8,
                         n_kv_heads=2, d_inner=512, dt_rank=32)
@@ -104,7 +109,7 @@ def test_prefixed_kv_pair_swa_dstate128_matches_oracle_and_full_path():
     h, _ = O.layer_forward(x, meta, ps[0], s0)
     assert_close(h_gpu, h, "bf16", "producer (full path) vs oracle")
     assert_close(p0, h, "bf16", "prefixed producer vs oracle")
-    assert_close(p0, h_gpu, "bf16", "prefixed producer vs the full path", tol=2e-3)
+    assert_close(p0, h_gpu, "bf16", "prefixed producer vs the full path", tol=PATH_TOL)
     kv_b = kv_p.reshape(2, s0.batch, s0.T, s0.kv_width)
     ref, _ = O.layer_forward(p0, None, ps[1], s1, kv_in=(kv_b[0], kv_b[1]))
     assert_close(p1, ref, "bf16", "prefixed consumer vs oracle")
@@ -114,7 +119,7 @@ def test_prefixed_kv_pair_swa_dstate128_matches_oracle_and_full_path():
     H.check(H.hymba_layer_fwd(dev(p0, "bf16"), None, H.make_weights(dps[1]), cfg1, dev(kv_p, "bf16"), None, full1, ws),
             "consumer full path")
     status_ok(ws)
-    assert_close(p1, to_np(full1), "bf16", "prefixed consumer vs the full path on the same input", tol=2e-3)
+    assert_close(p1, to_np(full1), "bf16", "prefixed consumer vs the full path on the same input", tol=PATH_TOL)
 
 
 @pytest.mark.parametrize("a_per_state", [0, 1])
@@ -136,5 +141,5 @@ def test_prefixed_single_layer_window_and_state_size(window, d_state):
     full = _plain_chain(wl, x, meta, dps)
     ref, _ = O.layer_forward(x, meta, ps[0], wl.first)
     assert_close(full, ref, "bf16", "full path vs oracle")
-    assert_close(g, full, "bf16", "prefixed vs the full path", tol=2e-3)
+    assert_close(g, full, "bf16", "prefixed vs the full path", tol=PATH_TOL)
     assert_close(g, ref, "bf16", "prefixed vs oracle")
