@@ -685,8 +685,7 @@ constexpr int NVT = 256;                // V/W threads (named barrier 1)
 constexpr int KA = 64;                  // dt_rank per K atom of the dt projection
 constexpr int TILE_B = Q * CH * 2;      // [32 t][128 c] bf16
 constexpr int BCC_B = Q * 128;          // one 32-column chunk of C [32 t][32] fp32
-constexpr int DLC_B = Q * 128;          // one dt_low atom [32 t][64 r] bf16
-constexpr int DL_B = 2 * DLC_B;
+constexpr int DLC_B = Q * 128;          // one dt_low atom [32 t][64 r] bf16 (of one stage)
 constexpr int WDC_B = CH * 128;         // one W_dt atom [128 c][64 r] bf16
 constexpr int MT_B = Q * Q * 4;         // M [t][s] tf32
 constexpr int BT_B = NS * Q * 4;        // B^T [n][s] tf32
@@ -694,7 +693,7 @@ constexpr int CC_B = 4 * BCC_B;         // C [t][n] tf32, four chunks
 constexpr int GREC_B = MT_B + BT_B + CC_B;  // a block's record from bc_gram_kernel
 constexpr int ST = 4;                   // stages (x, gate, dt_low)
 constexpr int OFF_DL = 0;
-constexpr int OFF_WD = OFF_DL + ST * DL_B;
+constexpr int OFF_WD = OFF_DL + 2 * ST * DLC_B;   // dt_low [atom][stage][32 t]: stages 2j, 2j + 1 adjacent
 constexpr int OFF_MT = OFF_WD + 2 * WDC_B;
 constexpr int OFF_BT = OFF_MT + 2 * MT_B;
 constexpr int OFF_CC = OFF_BT + 2 * BT_B;
@@ -715,12 +714,12 @@ static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
 constexpr uint32_t COL_Y = 0;     // [2][32]
 constexpr uint32_t COL_W = 64;    // [3][32]
 constexpr uint32_t COL_V = 160;   // [3][32]
-constexpr uint32_t COL_DT = 256;  // [2][32] W_dt dt_low^T
+constexpr uint32_t COL_DT = 256;  // [4][32] W_dt dt_low^T (block k in slot k % 4)
 constexpr uint32_t COL_GP = 384;  // [128] G'
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_Q = idesc_tf32(128, Q);
 constexpr uint32_t IDESC_N = idesc_tf32(128, NS);
-constexpr uint32_t IDESC_DT = idesc_bf16(128, Q, false, false);
+constexpr uint32_t IDESC_DT = idesc_bf16(128, 2 * Q, false, false);   // two blocks at once
 
 // Offsets of element (n, s) in B^T [n][s] and (t, n) in the C copy [t][n] (K-major,
 // 128-byte swizzle; B^T one 128-row atom, C four 32-column chunks).
@@ -850,7 +849,7 @@ __global__ void __launch_bounds__(NTHR2, 1)
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);  // [ST] TMA landed
   uint64_t* empty = full + ST;         // [ST] the stage's last reader done
-  uint64_t* dtready = empty + ST;      // [2] W_dt dt_low^T of the block in TMEM
+  uint64_t* dtready = empty + ST;      // [2] W_dt dt_low^T of a block pair in TMEM (pair p: p & 1)
   uint64_t* vready = dtready + 2;         // [3] V, W and the decay sums of the block ready (256 arrivals)
   uint64_t* btready = vready + 3;      // [2] B^T and C of the block in shared memory (TMA)
   uint64_t* mready = btready + 2;      // [2] M of the block in shared memory (TMA)
@@ -925,7 +924,8 @@ __global__ void __launch_bounds__(NTHR2, 1)
           for (int a = 0; a < ka; ++a) tma_load_2d(sm + OFF_WD + a * WDC_B, &tmWD, &full[s], a * KA, c0);
         tma_load_3d(sm + OFF_X + s * TILE_B, &tmX, &full[s], c0, t, b);
         tma_load_3d(sm + OFF_G + s * TILE_B, &tmG, &full[s], c0, t, b);
-        for (int a = 0; a < ka; ++a) tma_load_3d(sm + OFF_DL + s * DL_B + a * DLC_B, &tmDL, &full[s], a * KA, t, b);
+        for (int a = 0; a < ka; ++a)
+          tma_load_3d(sm + OFF_DL + (a * ST + s) * DLC_B, &tmDL, &full[s], a * KA, t, b);
       }
       if (k < nblk) {  // aborted: let the copies already issued land before smem goes away
         int never = 0;
@@ -964,35 +964,39 @@ __global__ void __launch_bounds__(NTHR2, 1)
     // order per block k (its inputs are ready, in the steady state, before it gets to them):
     //   chain(k):     Y = G' C^T, G' += V B (the state products) -> dgready
     //   vm(k):        Y += V M^T -> yready
-    //   stage(k + 2): the dt projection of block k + 2 -> dtready
+    //   pair(k + 2):  for even k, the dt projection of blocks k + 2 and k + 3 (one N = 64
+    //                 product over both stages' dt_low rows) -> dtready
     //   release(k + 1): block k + 1's stage back to the producer
     // so that while the state warps rescale G' for block k + 1 the tensor pipe works on
     // vm(k) and the dt projection, and chain(k + 1) follows as soon as G' is ready.
-    // Buffer reuse: DT buffer k & 1 is rewritten by stage(k + 2) after chain(k) (the V/W
-    // warps read it before vready(k), the plain recurrence before gready(k)); the stage of
-    // block k + 1 holds only x, gate (read before vready(k + 1)) and dt_low (read by the dt
-    // projection, which the release commit tracks).
+    // Buffer reuse: DT slots (k + 2) % 4, (k + 3) % 4 held blocks k - 2, k - 1, done with
+    // by chain(k - 1) (the V/W warps read a slot before vready, the plain recurrence before
+    // gready); the stage of block k + 1 holds only x, gate (read before vready(k + 1)) and
+    // dt_low (read by the dt projection, issued earlier and tracked by the release commit).
     if (lane == 0) {
       // descriptors of the first stage's tiles; every other tile is a fixed offset away
       const uint64_t dDL = sdesc_sw128(sbase + OFF_DL, 16, 1024), dWD = sdesc_sw128(sbase + OFF_WD, 16, 1024),
                      dCC = sdesc_sw128(sbase + OFF_CC, 16, 1024), dBT = sdesc_sw128(sbase + OFF_BT, 16, 1024),
                      dMT = sdesc_sw128(sbase + OFF_MT, 16, 1024);
       uint32_t n_yi = 0;   // completed phases of yidone (product-form blocks only)
-      auto stage = [&](int ks) -> bool {   // dt = W_dt dt_low^T of block ks into DT buffer ks & 1
+      // dt = W_dt dt_low^T of blocks ks, ks + 1 (ks even) into DT slots ks % 4, ks % 4 + 1:
+      // the two stages' dt_low rows are adjacent (64 rows of each atom).  Without a block
+      // ks + 1 the product's second half reads a stale stage into a slot nobody reads.
+      auto pair = [&](int ks) -> bool {
         if (!mbar_wait(&full[ks % ST], (ks / ST) & 1u, status, abort_flag)) return false;
+        if (ks + 1 < nblk && !mbar_wait(&full[(ks + 1) % ST], ((ks + 1) / ST) & 1u, status, abort_flag)) return false;
         tc_fence_after();
-        const int i = ks & 1;
-        const uint64_t dl = sdesc_add(dDL, (ks % ST) * DL_B);
+        const uint64_t dl = sdesc_add(dDL, (ks % ST) * DLC_B);
+        const uint32_t d = tmem + COL_DT + 32 * (ks & 3);
 #pragma unroll
         for (int j = 0; j < KA / 16; ++j)
-          umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_add(dWD, 32 * j), sdesc_add(dl, 32 * j), IDESC_DT, j != 0);
+          umma_bf16_ss(d, sdesc_add(dWD, 32 * j), sdesc_add(dl, 32 * j), IDESC_DT, j != 0);
         if (ka > 1) {
 #pragma unroll
           for (int j = 0; j < KA / 16; ++j)
-            umma_bf16_ss(tmem + COL_DT + 32 * i, sdesc_add(dWD, WDC_B + 32 * j), sdesc_add(dl, DLC_B + 32 * j),
-                         IDESC_DT, 1u);
+            umma_bf16_ss(d, sdesc_add(dWD, WDC_B + 32 * j), sdesc_add(dl, ST * DLC_B + 32 * j), IDESC_DT, 1u);
         }
-        umma_commit(&dtready[i]);
+        umma_commit(&dtready[(ks >> 1) & 1]);
         return true;
       };
       auto release = [&](int kr) -> bool {   // x and gate read (vready); the dt projection tracked
@@ -1001,8 +1005,7 @@ __global__ void __launch_bounds__(NTHR2, 1)
         return true;
       };
       bool ok = true;
-      for (int k = 0; k < 2 && k < nblk && ok; ++k) ok = stage(k);
-      if (ok && nblk > 0) ok = release(0);
+      if (nblk > 0) ok = pair(0) && release(0);
       for (int k = 0; k < nblk && ok; ++k) {
         const int i = k & 1, vb = k % 3;
         // ---- chain(k)
@@ -1041,8 +1044,8 @@ __global__ void __launch_bounds__(NTHR2, 1)
             umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(mt, 32 * j), IDESC_Q, 1);
         }
         umma_commit(&yready[i]);
-        // ---- the dt projection two blocks ahead, then the next stage's release
-        if (k + 2 < nblk && !stage(k + 2)) break;
+        // ---- the dt projection of the next pair, then the next stage's release
+        if ((k & 1) == 0 && k + 2 < nblk && !pair(k + 2)) break;
         if (k + 1 < nblk && !release(k + 1)) break;
       }
       umma_commit(mma_done);
@@ -1066,14 +1069,14 @@ __global__ void __launch_bounds__(NTHR2, 1)
       const int s = k % ST, vb = k % 3;
       // buffer vb was last read by the output of block k - 3 (after that block's products)
       fail = fail || !__all_sync(0xffffffffu, mbar_wait(&full[s], (k / ST) & 1u, status, abort_flag) &&
-                                                  mbar_wait(&dtready[k & 1], (k >> 1) & 1u, status, abort_flag) &&
+                                                  mbar_wait(&dtready[(k >> 1) & 1], (k >> 2) & 1u, status, abort_flag) &&
                                                   (k < 3 || mbar_wait(&wdone[vb], ((k - 3) / 3) & 1u, status, abort_flag)));
       // dt of this half (steps past T: dt = 0, the state stays)
       float dtv[HQ];
       if (!fail) {
         tc_fence_after();
         uint32_t z[HQ];
-        tmem_ld16(tl + COL_DT + 32 * (k & 1) + HQ * half, z);
+        tmem_ld16(tl + COL_DT + 32 * (k & 3) + HQ * half, z);
         tmem_wait_ld();
         const int t_end = T - (t0 + k * Q + HQ * half);
 #pragma unroll
@@ -1218,30 +1221,30 @@ __global__ void __launch_bounds__(NTHR2, 1)
         const bool one = __all_sync(0xffffffffu, e_in + e_out < 120.f);
         const float f1 = ex2_approx(one ? -(e_in + e_out) : -e_in), f2 = one ? 1.f : ex2_approx(-e_out);
         const float2 fa = make_float2(f1, f1), fb = make_float2(f2, f2);
+        // both 32-column pieces in flight at once: one load wait, one store wait
+        const uint32_t col = tl + COL_GP + 64 * half;
+        uint32_t g[64];
+        tmem_ld32(col, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+        tmem_ld32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
+        tmem_wait_ld();
+        if (one) {
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t col = tl + COL_GP + 64 * half + 32 * part;
-          uint32_t g[32];
-          tmem_ld32(col, g);
-          tmem_wait_ld();
-          if (one) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float2 v = __fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa);
-              g[j] = __float_as_uint(v.x);
-              g[j + 1] = __float_as_uint(v.y);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float2 v =
-                  __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa), fb);
-              g[j] = __float_as_uint(v.x);
-              g[j + 1] = __float_as_uint(v.y);
-            }
+          for (int j = 0; j < 64; j += 2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa);
+            g[j] = __float_as_uint(v.x);
+            g[j + 1] = __float_as_uint(v.y);
           }
-          tmem_st32(col, g);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            const float2 v =
+                __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])), fa), fb);
+            g[j] = __float_as_uint(v.x);
+            g[j + 1] = __float_as_uint(v.y);
+          }
         }
+        tmem_st32(col, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+        tmem_st32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
         tmem_wait_st();
       } else if (half == 1) {
         // ---- large decays: the plain recurrence over block k by the half-1 warps (one
@@ -1257,7 +1260,7 @@ __global__ void __launch_bounds__(NTHR2, 1)
 #pragma unroll 1
           for (int th = 0; th < Q; th += QQ) {
             uint32_t zq[QQ], uq[QQ], gq[QQ];
-            tmem_ld8(tl + COL_DT + 32 * i + th, zq);
+            tmem_ld8(tl + COL_DT + 32 * (k & 3) + th, zq);
             tmem_ld8(tl + COL_V + 32 * vb + th, uq);
             tmem_ld8(tl + COL_W + 32 * vb + th, gq);
             tmem_wait_ld();
