@@ -793,45 +793,65 @@ __global__ void __launch_bounds__(256) bc_gram_kernel(const float* __restrict__ 
   }
   __syncthreads();
   uint8_t* out = rec + (static_cast<long long>(b) * nblk + k) * GREC_B;
-  {  // M: thread = row t, columns s4 .. s4 + 3
-    const int t = tid >> 3, s4 = (tid & 7) * 4;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int n = 0; n < NS; n += 4) {
-      const float4 cv = *reinterpret_cast<const float4*>(&sC[t][n]);
+  if (tid < 64) {
+    // M: thread = a 4 x 4 tile (rows t0..t0+3, columns s0..s0+3), paired FMAs along s
+    const int t0 = (tid >> 3) * 4, s0 = (tid & 7) * 4;
+    float2 acc[4][2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float4 bv = *reinterpret_cast<const float4*>(&sB[s4 + e][n]);
-        acc[e] = fmaf(cv.x, bv.x, acc[e]);
-        acc[e] = fmaf(cv.y, bv.y, acc[e]);
-        acc[e] = fmaf(cv.z, bv.z, acc[e]);
-        acc[e] = fmaf(cv.w, bv.w, acc[e]);
+    for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
+#pragma unroll 2
+    for (int n = 0; n < NS; n += 4) {
+      float4 cv[4], bv[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        cv[r] = *reinterpret_cast<const float4*>(&sC[t0 + r][n]);
+        bv[r] = *reinterpret_cast<const float4*>(&sB[s0 + r][n]);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float c4[4] = {cv[r].x, cv[r].y, cv[r].z, cv[r].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 cc = make_float2(c4[e], c4[e]);
+          const float b0 = e == 0 ? bv[0].x : e == 1 ? bv[0].y : e == 2 ? bv[0].z : bv[0].w;
+          const float b1 = e == 0 ? bv[1].x : e == 1 ? bv[1].y : e == 2 ? bv[1].z : bv[1].w;
+          const float b2 = e == 0 ? bv[2].x : e == 1 ? bv[2].y : e == 2 ? bv[2].z : bv[2].w;
+          const float b3 = e == 0 ? bv[3].x : e == 1 ? bv[3].y : e == 2 ? bv[3].z : bv[3].w;
+          acc[r][0] = __ffma2_rn(cc, make_float2(b0, b1), acc[r][0]);
+          acc[r][1] = __ffma2_rn(cc, make_float2(b2, b3), acc[r][1]);
+        }
       }
     }
-    uint4 o;
-    o.x = s4 <= t ? tf32_round(acc[0]) : 0u;
-    o.y = s4 + 1 <= t ? tf32_round(acc[1]) : 0u;
-    o.z = s4 + 2 <= t ? tf32_round(acc[2]) : 0u;
-    o.w = s4 + 3 <= t ? tf32_round(acc[3]) : 0u;
-    reinterpret_cast<uint4*>(out)[t * (Q / 4) + s4 / 4] = o;
-  }
-  {  // B^T: thread = row n, columns 16 h .. 16 h + 15
-    const int n = tid >> 1, h = tid & 1;
-    uint4* dst = reinterpret_cast<uint4*>(out + MT_B + n * Q * 4 + h * 64);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int s0 = 16 * h + 4 * j;
-      dst[j] = make_uint4(tf32_round(sB[s0][n]), tf32_round(sB[s0 + 1][n]), tf32_round(sB[s0 + 2][n]),
-                          tf32_round(sB[s0 + 3][n]));
+    for (int r = 0; r < 4; ++r) {
+      const int t = t0 + r;
+      uint4 o;
+      o.x = s0 <= t ? tf32_round(acc[r][0].x) : 0u;
+      o.y = s0 + 1 <= t ? tf32_round(acc[r][0].y) : 0u;
+      o.z = s0 + 2 <= t ? tf32_round(acc[r][1].x) : 0u;
+      o.w = s0 + 3 <= t ? tf32_round(acc[r][1].y) : 0u;
+      reinterpret_cast<uint4*>(out)[t * (Q / 4) + s0 / 4] = o;
     }
-  }
-  {  // C: thread = row t, columns 16 h .. 16 h + 15
-    const int t = tid >> 3, h = tid & 7;
-    uint4* dst = reinterpret_cast<uint4*>(out + MT_B + BT_B + t * NS * 4 + h * 64);
+  } else {
+    // B^T (row n, columns 16 h .. 16 h + 15) and C (row t, columns 16 h .. 16 h + 15)
+    for (int u = tid - 64; u < 2 * NS; u += 192) {
+      const int n = u >> 1, h = u & 1;
+      uint4* dst = reinterpret_cast<uint4*>(out + MT_B + n * Q * 4 + h * 64);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 v = *reinterpret_cast<const float4*>(&sC[t][16 * h + 4 * j]);
-      dst[j] = make_uint4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z), tf32_round(v.w));
+      for (int j = 0; j < 4; ++j) {
+        const int s0 = 16 * h + 4 * j;
+        dst[j] = make_uint4(tf32_round(sB[s0][n]), tf32_round(sB[s0 + 1][n]), tf32_round(sB[s0 + 2][n]),
+                            tf32_round(sB[s0 + 3][n]));
+      }
+    }
+    for (int u = tid - 64; u < Q * 8; u += 192) {
+      const int t = u >> 3, h = u & 7;
+      uint4* dst = reinterpret_cast<uint4*>(out + MT_B + BT_B + t * NS * 4 + h * 64);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 v = *reinterpret_cast<const float4*>(&sC[t][16 * h + 4 * j]);
+        dst[j] = make_uint4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z), tf32_round(v.w));
+      }
     }
   }
 }
@@ -963,9 +983,9 @@ __global__ void __launch_bounds__(NTHR2, 1)
     // ------------------------------------------------------------ MMA issuer, in a fixed
     // order per block k (its inputs are ready, in the steady state, before it gets to them):
     //   chain(k):     Y = G' C^T, G' += V B (the state products) -> dgready
-    //   vm(k):        Y += V M^T -> yready
     //   pair(k + 2):  for even k, the dt projection of blocks k + 2 and k + 3 (one N = 64
     //                 product over both stages' dt_low rows) -> dtready
+    //   vm(k):        Y += V M^T -> yready
     //   release(k + 1): block k + 1's stage back to the producer
     // so that while the state warps rescale G' for block k + 1 the tensor pipe works on
     // vm(k) and the dt projection, and chain(k + 1) follows as soon as G' is ready.
@@ -1034,6 +1054,9 @@ __global__ void __launch_bounds__(NTHR2, 1)
             umma_tf32_ts(tmem + COL_GP, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(bt, 32 * j), IDESC_N, 1);
         }
         umma_commit(&dgready[i]);
+        // ---- the dt projection of the next pair first: the V/W warps need it as soon as
+        // they are done with block k + 1, while Y(k) is wanted only after G' is rescaled
+        if ((k & 1) == 0 && k + 2 < nblk && !pair(k + 2)) break;
         // ---- vm(k): Y += V M^T (K = s = 32), then Y is complete
         if (!mbar_wait(&mready[i], (k >> 1) & 1u, status, abort_flag)) break;
         tc_fence_after();
@@ -1044,8 +1067,7 @@ __global__ void __launch_bounds__(NTHR2, 1)
             umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(mt, 32 * j), IDESC_Q, 1);
         }
         umma_commit(&yready[i]);
-        // ---- the dt projection of the next pair, then the next stage's release
-        if ((k & 1) == 0 && k + 2 < nblk && !pair(k + 2)) break;
+        // ---- the next stage's release
         if (k + 1 < nblk && !release(k + 1)) break;
       }
       umma_commit(mma_done);
