@@ -69,28 +69,28 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// Maximum of a 128-value row (fp32 bit patterns): eight independent chains of
-// three-input maxima, so the reduction is 9 dependent steps deep instead of 128.
-__device__ __forceinline__ float row_max128(const uint32_t (&sv)[128]) {
+// Maximum of a 64-value half row (fp32 bit patterns): eight independent chains of
+// three-input maxima, so the reduction is 5 dependent steps deep instead of 64.
+__device__ __forceinline__ float row_max64(const uint32_t (&sv)[64]) {
   float m[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = fmaxf(__uint_as_float(sv[i]), __uint_as_float(sv[i + 8]));
 #pragma unroll
-  for (int e = 16; e < 128; e += 16)
+  for (int e = 16; e < 64; e += 16)
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = max3f(m[i], __uint_as_float(sv[e + i]), __uint_as_float(sv[e + 8 + i]));
   return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
-// P = 2^(S scale - m_ref) for a 128-value row, packed in place as bf16 pairs
-// (sv[q] <- (p[2q], p[2q+1]); reads index >= q first); returns the row sum of the fp32
+// P = 2^(S scale - m_ref) for a 64-value half row, packed in place as bf16 pairs
+// (sv[q] <- (p[2q], p[2q+1]); reads index >= q first); returns the sum of the fp32
 // values.  Paired scale-and-subtract, four independent partial sums.
-__device__ __forceinline__ float row_exp128(uint32_t (&sv)[128], float scale_log2, float m_ref) {
+__device__ __forceinline__ float row_exp64(uint32_t (&sv)[64], float scale_log2, float m_ref) {
   const float2 sc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
   float2 acc[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int q = 0; q < 64; ++q) {
+  for (int q = 0; q < 32; ++q) {
     const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1])), sc, nm);
     const float2 pq = make_float2(ex2_approx(x.x), ex2_approx(x.y));
     acc[q & 3] = __fadd2_rn(acc[q & 3], pq);
@@ -374,18 +374,21 @@ __global__ void __launch_bounds__(192, 1)
 
 // ---------------------------------------------------------------------------------
 // Two query heads of one KV head per CTA (GQA groups of even size): the two softmax
-// warpgroups ping-pong against the tensor core and share every K/V tile.
+// groups ping-pong against the tensor core and share every K/V tile.
 //   warp 0      TMA producer: Q of both heads once, then K_j / V_j (2-deep rings)
 //   warp 1      UMMA issuer, per block j: P_a V_j, S_a(j+1), P_b V_j, S_b(j+1)
-//   warps 2..5  softmax of head a, warps 6..9 softmax of head b (one row per thread)
+//   warps 2..9  softmax of head a, warps 10..17 softmax of head b: two threads per query
+//               row (warps w and w + 4 share a TMEM lane quadrant), each over 64 of the
+//               block's 128 keys and 64 of O's columns; the row maximum is exchanged
+//               through shared memory once per block, the row sum once at the end
 // TMEM (512 columns): S_a | S_b | O_a | O_b, 128 fp32 columns each.  P_x(j) (bf16,
 // two keys per 32-bit column) is written over the consumed S_x(j) columns and read
 // by the P V instruction straight from TMEM, so P never touches shared memory; S_x(j+1)
 // is issued only after P_x V_j has completed.  O accumulates in TMEM with the same
 // lazy rescale as the one-head kernel.
-constexpr int SMEM2_BYTES = 6 * TILE_BYTES + 1024 + 256;
+constexpr int SMEM2_BYTES = 6 * TILE_BYTES + 1024 + 256 + 2 * 2 * 2 * 128 * 4 + 2 * 2 * 128 * 4;
 
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
     attn_fwd_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -405,6 +408,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* mma_done = bars + 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* smax = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // [2 j][2 head][2 half][128 row]
+  float* slsum = smax + 2 * 2 * 2 * 128;                                           // [2 head][2 half][128 row]
 
   pdl_trigger();
   pdl_wait();
@@ -424,7 +429,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], 256);
       mbar_init(&o_done[s], 1);
     }
     mbar_init(mma_done, 1);
@@ -538,13 +543,14 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait(mma_done, 0, nullptr, &never, 100000000ull);
     }
   } else {
-    // ------------------------------------------------------------------ softmax (two warpgroups)
-    const int x = (warp - 2) >> 2;  // head of this warpgroup
+    // ------------------------------------------------------------------ softmax (two groups of 8 warps)
+    const int x = (warp - 2) >> 3;        // head of this group
+    const int kh = ((warp - 2) >> 2) & 1;  // half of the keys and of O's columns
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int i = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tSx = tmem_base + x * 128 + lane_off, tOx = tmem_base + 256 + x * 128 + lane_off;
+    const uint32_t tSx = tmem_base + x * 128 + lane_off, tOx = tmem_base + 256 + x * 128 + lane_off + kh * 64;
     constexpr float kRescaleLog2 = 8.0f;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -552,64 +558,72 @@ __global__ void __launch_bounds__(320, 1)
       const int k0 = bl.block(j) * BKV;
       const bool need_mask =
           !((k0 + BKV - 1 <= q0) && (p.window < 0 || q0 + BQ - 1 - k0 <= p.window || k0 + BKV - 1 < p.n_meta));
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1, p.status, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sv[128];
-      {
-        uint32_t (&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
-        uint32_t (&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-        uint32_t (&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[64]);
-        uint32_t (&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[96]);
-        tmem_ld32(tSx, c0);
-        tmem_ld32(tSx + 32, c1);
-        tmem_ld32(tSx + 64, c2);
-        tmem_ld32(tSx + 96, c3);
+      // every thread of the group takes the same steps, so the group barrier below is
+      // reached by all of them (a failed wait only skips the work)
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1, p.status, abort_flag));
+      uint32_t sv[64];
+      float m_half = -INFINITY;
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tSx + kh * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tSx + kh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_wait_ld();
-      }
-      if (need_mask) {
+        if (need_mask) {
 #pragma unroll
-        for (int e = 0; e < 128; ++e)
-          if (!visible(i, k0 + e, p.n_meta, p.window)) sv[e] = __float_as_uint(-INFINITY);
-      }
-      const float m_cand = row_max128(sv) * p.scale_log2;
-      const bool need = m_cand > m_used + kRescaleLog2;
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2_approx(m_used - m_cand);  // 0 when m_used is -inf
-        m_used = m_cand;
-      }
-      const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
-      // P in bf16, packed in place over the first 64 words
-      const float sum = row_exp128(sv, p.scale_log2, m_ref);
-      tmem_st32(tSx, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_st32(tSx + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // rescale O (every earlier P V of this head has completed: S_x(j) was issued
-        // after it, and P_x V_j cannot start before p_full below)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tOx + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tOx + c * 32, o);
+          for (int e = 0; e < 64; ++e)
+            if (!visible(i, k0 + kh * 64 + e, p.n_meta, p.window)) sv[e] = __float_as_uint(-INFINITY);
         }
+        m_half = row_max64(sv) * p.scale_log2;
       }
-      tmem_wait_st();
-      l = fmaf(l, alpha, sum);
+      // the row maximum over both halves; the barrier also orders this half's reads of
+      // S before the other half's P stores (P of keys 64..127 lands in S columns 32..63)
+      float* sm_j = smax + (j & 1) * 512 + x * 256;
+      sm_j[kh * 128 + r] = m_half;
+      tc_fence_before();
+      bar_sync_n(1 + x, 256);
+      tc_fence_after();
+      const float m_cand = fmaxf(sm_j[r], sm_j[128 + r]);
+      if (ok) {
+        const bool need = m_cand > m_used + kRescaleLog2;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2_approx(m_used - m_cand);  // 0 when m_used is -inf
+          m_used = m_cand;
+        }
+        const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
+        // P in bf16, packed in place over the first 32 words: keys 64 kh .. 64 kh + 63
+        // into P columns 32 kh .. 32 kh + 31
+        const float sum = row_exp64(sv, p.scale_log2, m_ref);
+        tmem_st32(tSx + kh * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // rescale this half of O (every earlier P V of this head has completed: S_x(j)
+          // was issued after it, and P_x V_j cannot start before p_full below)
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tOx + c * 16, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(tOx + c * 16, o);
+          }
+        }
+        tmem_wait_st();
+        l = fmaf(l, alpha, sum);
+      }
       tc_fence_before();
       mbar_arrive(&p_full[x]);
     }
-    if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(&o_done[x], (n - 1) & 1, p.status, abort_flag))) {
+    ok = ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(&o_done[x], (n - 1) & 1, p.status, abort_flag));
+    // the row sum over both halves (every thread of the group reaches this barrier)
+    slsum[x * 256 + kh * 128 + r] = l;
+    bar_sync_n(1 + x, 256);
+    if (ok) {
       tc_fence_after();
-      const float inv = 1.f / l;
-      __nv_bfloat16* orow = p.out + (static_cast<long long>(b) * p.T + i) * p.out_ld + (h0 + x) * DH;
+      const float inv = 1.f / (slsum[x * 256 + r] + slsum[x * 256 + 128 + r]);
+      __nv_bfloat16* orow = p.out + (static_cast<long long>(b) * p.T + i) * p.out_ld + (h0 + x) * DH + kh * 64;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
         tmem_ld32(tOx + c * 32, o);
         tmem_wait_ld();
@@ -694,7 +708,7 @@ cudaError_t launch_attention(const AttnDesc& a, cudaStream_t st) {
   if ((a.n_q_heads / a.n_kv_heads) % 2 == 0) {  // pairs of query heads share each K/V tile
     if (cudaError_t e = smem_attr_once(attn_fwd_tc2, SMEM2_BYTES, attr2_done)) return e;
     dim3 grid(p.q_tiles - a.q_row0 / BQ, a.n_q_heads / 2, a.batch);
-    return launch(attn_fwd_tc2, grid, dim3(320), SMEM2_BYTES, st, tq, tk, tv, p);
+    return launch(attn_fwd_tc2, grid, dim3(576), SMEM2_BYTES, st, tq, tk, tv, p);
   }
   dim3 grid(p.q_tiles - a.q_row0 / BQ, a.n_q_heads, a.batch);
   return launch(attn_fwd_tc, grid, dim3(192), SMEM_BYTES, st, tq, tk, tv, p);
