@@ -22,6 +22,11 @@
 #include "hy_kernels.h"
 #include "hymba.h"
 
+namespace hy {  // gemv.cu
+bool gemv_bf16_takes(const GemmDesc& g);
+cudaError_t launch_gemv_bf16(const GemmDesc& g, cudaStream_t st);
+}  // namespace hy
+
 namespace {
 
 using hy::GemmDesc;
@@ -142,7 +147,10 @@ hymba_status_t validate_cfg(const hymba_cfg_t* c) {
 
 hymba_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? HYMBA_OK : HYMBA_ERR_CUDA; }
 
+// A product with a handful of rows (a generation step) streams W on the CUDA cores
+// (gemv.cu); every other one runs on the tensor-core GEMM.
 cudaError_t gemm(const GemmDesc& g, hymba_dtype_t t, cudaStream_t st) {
+  if (t == HYMBA_BF16 && hy::gemv_bf16_takes(g)) return hy::launch_gemv_bf16(g, st);
   return t == HYMBA_BF16 ? hy::launch_gemm_bf16(g, st) : hy::launch_gemm_f32(g, st);
 }
 

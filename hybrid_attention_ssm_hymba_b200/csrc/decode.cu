@@ -13,7 +13,8 @@
 //                        in fp32 (exp2 with the log2(e)/sqrt(dh) scale folded into q).
 //   attn_decode_combine  merges the splits' (max, sum, unnormalised output) per row.
 //   scan_step_kernel     h <- exp(A dt) h + dt x B, y = gate * (C . h) for one row, the
-//                        state read and written in place; 8 lanes per channel.
+//                        state read and written in place; 8 lanes per channel, each with
+//                        every eighth 16-byte chunk of the state.
 #include "hy_common.cuh"
 #include "hy_kernels.h"
 
@@ -101,14 +102,40 @@ __global__ void __launch_bounds__(32 * kDecWarps) attn_decode_kernel(const Decod
     for (int g = 0; g < kMaxG; ++g) s[g] = 0.f;
     if (valid) {
       const T* kr = kb + static_cast<long long>(vk.key(idx)) * p.kv_ld;
-      for (int e0 = 0; e0 < dh; e0 += 8) {
-        float kf[8];
-        load_row_f<T>(kr + e0, 8, kf);
+      if constexpr (sizeof(T) == 2) {
+        // the whole K row (dh <= 128: at most 16 vectors) in flight before any is used
+        uint4 kv[16];
 #pragma unroll
-        for (int g = 0; g < kMaxG; ++g) {
-          if (g < G) {
+        for (int j = 0; j < 16; ++j)
+          if (8 * j < dh) kv[j] = *reinterpret_cast<const uint4*>(kr + 8 * j);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s[g] = fmaf(sq[g][e0 + e], kf[e], s[g]);
+        for (int j = 0; j < 16; ++j) {
+          if (8 * j >= dh) continue;
+          const uint32_t u[4] = {kv[j].x, kv[j].y, kv[j].z, kv[j].w};
+          float kf[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            kf[2 * q] = bf16lo(u[q]);
+            kf[2 * q + 1] = bf16hi(u[q]);
+          }
+#pragma unroll
+          for (int g = 0; g < kMaxG; ++g) {
+            if (g < G) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) s[g] = fmaf(sq[g][8 * j + e], kf[e], s[g]);
+            }
+          }
+        }
+      } else {
+        for (int e0 = 0; e0 < dh; e0 += 8) {
+          float kf[8];
+          load_row_f<T>(kr + e0, 8, kf);
+#pragma unroll
+          for (int g = 0; g < kMaxG; ++g) {
+            if (g < G) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) s[g] = fmaf(sq[g][e0 + e], kf[e], s[g]);
+            }
           }
         }
       }
@@ -134,17 +161,28 @@ __global__ void __launch_bounds__(32 * kDecWarps) attn_decode_kernel(const Decod
     }
     // P V: lane = head-dim slice [lane * epl, lane * epl + epl)
     const int nk = min(32, k1 - c0);
-    for (int kk = 0; kk < nk; ++kk) {
-      const T* vr = vb + static_cast<long long>(vk.key(c0 + kk)) * p.kv_ld + lane * epl;
-      float vf[kMaxEPL];
+    for (int kk0 = 0; kk0 < nk; kk0 += 8) {
+      // eight V rows' slices in flight at once
+      float vf[8][kMaxEPL];
 #pragma unroll
-      for (int e = 0; e < kMaxEPL; ++e) vf[e] = e < epl ? to_f<T>(vr[e]) : 0.f;
+      for (int u8 = 0; u8 < 8; ++u8) {
+        const int kk = kk0 + u8;
+        const T* vr = vb + static_cast<long long>(vk.key(c0 + min(kk, nk - 1))) * p.kv_ld + lane * epl;
 #pragma unroll
-      for (int g = 0; g < kMaxG; ++g) {
-        if (g >= G) continue;
-        const float pk = __shfl_sync(0xffffffffu, pr[g], kk);
+        for (int e = 0; e < kMaxEPL; ++e) vf[u8][e] = e < epl ? to_f<T>(vr[e]) : 0.f;
+      }
 #pragma unroll
-        for (int e = 0; e < kMaxEPL; ++e) o[g][e] = fmaf(pk, vf[e], o[g][e]);
+      for (int u8 = 0; u8 < 8; ++u8) {
+        const int kk = kk0 + u8;
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) {
+          if (g >= G) continue;
+          const float pk = __shfl_sync(0xffffffffu, pr[g], kk & 31);
+          if (kk < nk) {
+#pragma unroll
+            for (int e = 0; e < kMaxEPL; ++e) o[g][e] = fmaf(pk, vf[u8][e], o[g][e]);
+          }
+        }
       }
     }
   }
@@ -222,19 +260,48 @@ __global__ void __launch_bounds__(256) scan_step_kernel(const T* __restrict__ x,
   const int b = valid ? static_cast<int>(ch / Di) : 0, c = valid ? static_cast<int>(ch % Di) : 0;
   float yv = 0.f;
   if (valid) {
+    // lane sl owns the 16-byte chunks sl, sl + 8, ... of the channel's state (and of B, C):
+    // the 8 lanes of a channel read 128 contiguous bytes per step, every load issued first
     const long long r = static_cast<long long>(b) * Di + c;
     const float d = to_f<T>(dt[r]), u = d * to_f<T>(x[r]);
-    const float* Bb = bc + static_cast<long long>(b) * 2 * N;
-    const float* Cb = Bb + N;
-    float* hp = h + r * N;
+    const float4* B4 = reinterpret_cast<const float4*>(bc + static_cast<long long>(b) * 2 * N);
+    const float4* C4 = B4 + N / 4;
+    float4* h4 = reinterpret_cast<float4*>(h + r * N);
+    const float4* al4 = reinterpret_cast<const float4*>(a_log + static_cast<long long>(c) * N);
     const float A1 = a_per_state ? 0.f : -expf(a_log[c]) * 1.4426950408889634f;
     const float a1 = ex2_approx(A1 * d);
-    for (int n = sl * ns; n < sl * ns + ns; ++n) {
-      const float a = a_per_state ? ex2_approx(-expf(a_log[static_cast<long long>(c) * N + n]) * 1.4426950408889634f * d)
-                                  : a1;
-      const float hn = fmaf(a, hp[n], u * Bb[n]);
-      hp[n] = hn;
-      yv = fmaf(Cb[n], hn, yv);
+    const int nq = N / 4;
+    for (int base = 0; base < nq; base += 32) {   // 128 states per pass (one pass for N <= 128)
+      float4 hv[4], bv[4], cv[4], av[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = base + sl + 8 * i;
+        if (q < nq) {
+          hv[i] = h4[q];
+          bv[i] = B4[q];
+          cv[i] = C4[q];
+          av[i] = a_per_state ? al4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = base + sl + 8 * i;
+        if (q < nq) {
+          float a[4] = {a1, a1, a1, a1};
+          if (a_per_state) {
+            const float al[4] = {av[i].x, av[i].y, av[i].z, av[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) a[e] = ex2_approx(-expf(al[e]) * 1.4426950408889634f * d);
+          }
+          float4 hn;
+          hn.x = fmaf(a[0], hv[i].x, u * bv[i].x);
+          hn.y = fmaf(a[1], hv[i].y, u * bv[i].y);
+          hn.z = fmaf(a[2], hv[i].z, u * bv[i].z);
+          hn.w = fmaf(a[3], hv[i].w, u * bv[i].w);
+          h4[q] = hn;
+          yv = fmaf(cv[i].x, hn.x, fmaf(cv[i].y, hn.y, fmaf(cv[i].z, hn.z, fmaf(cv[i].w, hn.w, yv))));
+        }
+      }
     }
   }
 #pragma unroll

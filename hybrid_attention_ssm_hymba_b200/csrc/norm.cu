@@ -140,11 +140,17 @@ __global__ void __launch_bounds__(256) rownorm_warp_kernel(const __nv_bfloat16* 
   const uint4* src = reinterpret_cast<const uint4*>(x + row * W);
   uint4 v[MAXV];
   float sa = 0.f, ss = 0.f;
+  // every load of the row issued before any is used (a short grid has no other warps to
+  // hide their latency behind)
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int vi = lane + 32 * k;
+    v[k] = vi < nv ? src[vi] : make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll
   for (int k = 0; k < MAXV; ++k) {
     const int vi = lane + 32 * k;
     if (vi < nv) {
-      v[k] = src[vi];
       const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
       float acc = 0.f;
 #pragma unroll
@@ -188,6 +194,87 @@ __global__ void __launch_bounds__(256) rownorm_warp_kernel(const __nv_bfloat16* 
   }
 }
 
+// The same norm for a few rows (a generation step): a CTA per row, 256 threads with at
+// most MAXV 16-byte vectors each, the row and its beta values loaded before any use.
+template <int MAXV>
+__global__ void __launch_bounds__(256) rownorm_cta_kernel(const __nv_bfloat16* x,  // x and y may alias
+                                                          __nv_bfloat16* y, int wa, int ws,
+                                                          const float* __restrict__ beta1,
+                                                          const float* __restrict__ beta2, float eps, float s2) {
+  __shared__ float red[8][2];
+  pdl_trigger();
+  pdl_wait();
+  const long long row = blockIdx.x;
+  const int W = wa + ws, nv = W / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(x + row * W);
+  uint4 v[MAXV];
+  float4 bl[MAXV], bh[MAXV];
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int vi = threadIdx.x + 256 * k;
+    v[k] = make_uint4(0u, 0u, 0u, 0u);
+    bl[k] = bh[k] = make_float4(1.f, 1.f, 1.f, 1.f);
+    if (vi < nv) {
+      v[k] = src[vi];
+      const int col = vi * 8;
+      const float* beta = col < wa ? beta1 + col : (beta2 ? beta2 + (col - wa) : nullptr);
+      if (beta) {
+        bl[k] = *reinterpret_cast<const float4*>(beta);
+        bh[k] = *reinterpret_cast<const float4*>(beta + 4);
+      }
+    }
+  }
+  float sa = 0.f, ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int vi = threadIdx.x + 256 * k;
+    const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+    float acc = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float a = bf16lo(u[q]), bb = bf16hi(u[q]);
+      acc = fmaf(a, a, fmaf(bb, bb, acc));
+    }
+    if (vi * 8 < wa) sa += acc;
+    else ss += acc;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sa += __shfl_xor_sync(0xffffffffu, sa, o);
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red[warp][0] = sa;
+    red[warp][1] = ss;
+  }
+  __syncthreads();
+  sa = ss = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    sa += red[w][0];
+    ss += red[w][1];
+  }
+  const float ra = wa > 0 ? rsqrtf(sa / wa + eps) : 0.f, rs = rsqrtf(ss / ws + eps);
+  uint4* dst = reinterpret_cast<uint4*>(y + row * W);
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int vi = threadIdx.x + 256 * k;
+    if (vi < nv) {
+      const float r = vi * 8 < wa ? ra : rs * s2;
+      const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+      const float b[8] = {bl[k].x, bl[k].y, bl[k].z, bl[k].w, bh[k].x, bh[k].y, bh[k].z, bh[k].w};
+      float f[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        f[2 * q] = bf16lo(u[q]) * r * b[2 * q];
+        f[2 * q + 1] = bf16hi(u[q]) * r * b[2 * q + 1];
+      }
+      dst[vi] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
+    }
+  }
+}
+
 template <int MAXV>
 void launch_rownorm(const void* x, void* y, long long rows, int wa, int ws, const float* b1, const float* b2,
                     float eps, float s2, cudaStream_t st) {
@@ -199,6 +286,17 @@ void launch_rownorm(const void* x, void* y, long long rows, int wa, int ws, cons
 bool rownorm_bf16(const void* x, void* y, long long rows, int wa, int ws, const float* b1, const float* b2, float eps,
                   cudaStream_t st, float s2 = 1.f) {
   const int nv = (wa + ws) / 8;
+  if (rows < 512 && nv <= 4 * 256) {   // too few rows to fill the GPU one warp each
+    const auto args = [&](auto kern) {
+      launch(kern, dim3(static_cast<unsigned>(rows)), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x),
+             static_cast<__nv_bfloat16*>(y), wa, ws, b1, b2, eps, s2);
+    };
+    if (nv <= 256) args(rownorm_cta_kernel<1>);
+    else if (nv <= 512) args(rownorm_cta_kernel<2>);
+    else if (nv <= 768) args(rownorm_cta_kernel<3>);
+    else args(rownorm_cta_kernel<4>);
+    return true;
+  }
   const int per_lane = (nv + 31) / 32;
   if (per_lane <= 4) launch_rownorm<4>(x, y, rows, wa, ws, b1, b2, eps, s2, st);
   else if (per_lane <= 8) launch_rownorm<8>(x, y, rows, wa, ws, b1, b2, eps, s2, st);

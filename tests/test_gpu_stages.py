@@ -248,6 +248,8 @@ def _run_dtproj(inp, B, T, Di, N, dtype, y_ld=None):
     ("bf16", 1, 517, 200, 128, 96),    # second channel tile partial, dt_rank 96 (zero-filled atom tail)
     ("bf16", 3, 65, 128, 128, 64),     # one dt atom, three sequences
     ("bf16", 1, 31, 136, 128, 8),      # a single partial block, 8-wide dt projection
+    ("bf16", 2, 64, 128, 128, 128),    # exactly one dt pair (two full blocks)
+    ("bf16", 1, 33, 128, 128, 128),    # two blocks, the second a single step
     ("bf16", 2, 333, 192, 16, 64),     # d_state 16 tensor-core form
     ("bf16", 1, 100, 64, 64, 32),      # no tensor-core form: dt through the GEMM, then the scan
     ("f32", 2, 90, 48, 128, 40),
