@@ -332,7 +332,8 @@ HYMBA_API hymba_status_t hymba_check_wait_timeout(void* workspace, size_t ws_byt
 /* ---------------- stage entry points (each one kernel family) ---------------- */
 
 /* C[M, N] = A[M, K] W[N, K]^T (dtype in and out, fp32 accumulation); bf16 runs on the
- * tcgen05 tensor-core GEMM.  workspace: >= 256 bytes (status word). */
+ * tcgen05 tensor-core GEMM, or for M <= 8 (K a multiple of 8, 16-byte aligned A and W) on
+ * the CUDA cores as a stream over W.  workspace: >= 256 bytes (status word). */
 HYMBA_API hymba_status_t hymba_gemm(const void* a, const void* w, void* c, int M, int N, int K,
                           hymba_dtype_t dtype, void* workspace, size_t ws_bytes, void* stream);
 
