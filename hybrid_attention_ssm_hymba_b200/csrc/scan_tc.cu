@@ -868,7 +868,7 @@ __global__ void __launch_bounds__(NTHR2, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);  // [ST] TMA landed
-  uint64_t* empty = full + ST;         // [ST] the stage's last reader done
+  uint64_t* empty = full + ST;         // [ST] the stage's x and gate read by the V/W warps (256 arrivals)
   uint64_t* dtready = empty + ST;      // [2] W_dt dt_low^T of a block pair in TMEM (pair p: p & 1)
   uint64_t* vready = dtready + 2;         // [3] V, W and the decay sums of the block ready (256 arrivals)
   uint64_t* btready = vready + 3;      // [2] B^T and C of the block in shared memory (TMA)
@@ -891,7 +891,7 @@ __global__ void __launch_bounds__(NTHR2, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], NVT);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&dtready[i], 1);
@@ -986,13 +986,12 @@ __global__ void __launch_bounds__(NTHR2, 1)
     //   pair(k + 2):  for even k, the dt projection of blocks k + 2 and k + 3 (one N = 64
     //                 product over both stages' dt_low rows) -> dtready
     //   vm(k):        Y += V M^T -> yready
-    //   release(k + 1): block k + 1's stage back to the producer
     // so that while the state warps rescale G' for block k + 1 the tensor pipe works on
     // vm(k) and the dt projection, and chain(k + 1) follows as soon as G' is ready.
     // Buffer reuse: DT slots (k + 2) % 4, (k + 3) % 4 held blocks k - 2, k - 1, done with
     // by chain(k - 1) (the V/W warps read a slot before vready, the plain recurrence before
-    // gready); the stage of block k + 1 holds only x, gate (read before vready(k + 1)) and
-    // dt_low (read by the dt projection, issued earlier and tracked by the release commit).
+    // gready).  The V/W warps free a stage themselves once they have read its x and gate:
+    // they read them only after the dt projection over its dt_low rows has completed.
     if (lane == 0) {
       // descriptors of the first stage's tiles; every other tile is a fixed offset away
       const uint64_t dDL = sdesc_sw128(sbase + OFF_DL, 16, 1024), dWD = sdesc_sw128(sbase + OFF_WD, 16, 1024),
@@ -1019,13 +1018,8 @@ __global__ void __launch_bounds__(NTHR2, 1)
         umma_commit(&dtready[(ks >> 1) & 1]);
         return true;
       };
-      auto release = [&](int kr) -> bool {   // x and gate read (vready); the dt projection tracked
-        if (!mbar_wait(&vready[kr % 3], (kr / 3) & 1u, status, abort_flag)) return false;
-        umma_commit(&empty[kr % ST]);
-        return true;
-      };
       bool ok = true;
-      if (nblk > 0) ok = pair(0) && release(0);
+      if (nblk > 0) ok = pair(0);
       for (int k = 0; k < nblk && ok; ++k) {
         const int i = k & 1, vb = k % 3;
         // ---- chain(k)
@@ -1067,8 +1061,6 @@ __global__ void __launch_bounds__(NTHR2, 1)
             umma_tf32_ts(tmem + COL_Y + 32 * i, tmem + COL_V + 32 * vb + 8 * j, sdesc_add(mt, 32 * j), IDESC_Q, 1);
         }
         umma_commit(&yready[i]);
-        // ---- the next stage's release
-        if (k + 1 < nblk && !release(k + 1)) break;
       }
       umma_commit(mma_done);
       int never = 0;
@@ -1137,6 +1129,7 @@ __global__ void __launch_bounds__(NTHR2, 1)
           xv[j] = bf2f(static_cast<uint16_t>(lds_u16(xa + j * 256)));
           gv[j] = bf2f(static_cast<uint16_t>(lds_u16(ga + j * 256)));
         }
+        mbar_arrive(&empty[s]);   // x and gate are in registers: the stage can be refilled
         uint32_t vr[HQ], wr[HQ];
         if (!any) {
           float mu[HQ];
@@ -1168,6 +1161,7 @@ __global__ void __launch_bounds__(NTHR2, 1)
         tmem_st16(tl + COL_W + 32 * vb + HQ * half, wr);
         tmem_wait_st();
       }
+      if (fail) mbar_arrive(&empty[s]);   // (skipped above)
       if (warp == 8 && lane == 0) sAny[vb] = any ? 1 : 0;
       tc_fence_before();
       mbar_arrive(&vready[vb]);
