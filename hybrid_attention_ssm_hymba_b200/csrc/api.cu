@@ -477,7 +477,7 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
   if (fused_norm) {
     if ((e = hy::launch_scale_cols(w.w_out, w_out_scaled, c.d_model, wa, di, w.beta1, w.beta2, st, s2)) !=
             cudaSuccess ||
-        (e = hy::launch_row_ssq(z, rows, wa, di, ssq, st)) != cudaSuccess)
+        (e = hy::launch_row_ssq(z, rows, wa, di, ssq, st, status)) != cudaSuccess)
       return HYMBA_ERR_CUDA;
   } else if (c.norm_group) {
     if ((e = hy::launch_group_norm(z, rows, wa, di, c.norm_group, w.beta1, w.beta2, s2, c.rms_eps,

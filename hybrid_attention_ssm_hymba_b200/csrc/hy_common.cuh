@@ -174,6 +174,15 @@ HY_DEV void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
       : "memory");
 }
 
+// Untiled bulk copy global -> shared of `bytes` contiguous bytes (both addresses 16-byte
+// aligned, bytes a multiple of 16), completing on `bar` as transaction bytes.
+HY_DEV void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // TMA store smem -> global (bulk async group), and its completion waits
 HY_DEV void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(

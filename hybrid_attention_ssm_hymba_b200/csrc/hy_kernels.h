@@ -221,7 +221,8 @@ cudaError_t launch_transpose_bf16(const void* src, long long src_ld, void* dst, 
 // Fused branch norm (bf16).  row_ssq: ssq[row] = (sum of z[row, :w_attn]^2, sum of
 // z[row, w_attn:]^2).  scale_cols: w_out[n, k] = w[n, k] * (k < w_attn ? beta1[k] :
 // beta2[k - w_attn]) for a [N, w_attn + w_ssm] weight.
-cudaError_t launch_row_ssq(const void* z, long long rows, int w_attn, int w_ssm, float2* ssq, cudaStream_t st);
+cudaError_t launch_row_ssq(const void* z, long long rows, int w_attn, int w_ssm, float2* ssq, cudaStream_t st,
+                           unsigned* status = nullptr);
 cudaError_t launch_scale_cols(const void* w, void* w_out, int N, int w_attn, int w_ssm, const float* beta1,
                               const float* beta2, cudaStream_t st, float s2 = 1.f);
 

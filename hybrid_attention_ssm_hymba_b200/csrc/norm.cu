@@ -11,7 +11,10 @@
 //     columns.
 // bf16 rows up to 6144 elements: one warp per row with the row held in registers
 // (one HBM read, one write).  Wider rows and fp32: one CTA per row (the second read
-// of the row hits L1/L2).  fp32 sums; 16-byte vector loads and stores.
+// of the row hits L1/L2).  fp32 sums; 16-byte vector loads and stores.  row_ssq, a pure
+// read of Z, streams Z through shared memory with bulk copies (one CTA per SM).
+#include <algorithm>
+
 #include "hy_common.cuh"
 #include "hy_kernels.h"
 
@@ -345,6 +348,87 @@ __global__ void __launch_bounds__(256) row_ssq_kernel(const __nv_bfloat16* __res
   if (lane == 0) ssq[row] = make_float2(sa, ss);
 }
 
+// The same sums with Z streamed through shared memory by bulk copies.  Z's rows are
+// contiguous, so a chunk of rpc rows is one copy; one CTA per SM walks chunks blockIdx.x,
+// blockIdx.x + gridDim.x, ... through a ring of nst chunks: warp 8 (one thread) issues the
+// copies, warps 0..7 take the chunk's rows (row w, w + 8, ...) and reduce them from shared
+// memory.  The copy engine keeps more bytes in flight per SM than the warps' own 16-byte
+// loads can, which a stream over HBM needs.
+constexpr int SSQ_WARPS = 8;
+constexpr int SSQ_RING = 200 * 1024;   // bytes of the ring at most
+
+__global__ void __launch_bounds__((SSQ_WARPS + 1) * 32, 1)
+    row_ssq_bulk_kernel(const __nv_bfloat16* __restrict__ z, long long rows, int wa, int ws, int rpc, int nst,
+                        float2* __restrict__ ssq, unsigned* status) {
+  extern __shared__ __align__(16) uint8_t ring[];  // [nst][rpc rows], then full[nst], empty[nst], abort flag
+  const uint32_t row_bytes = static_cast<uint32_t>(wa + ws) * 2u, chunk_bytes = row_bytes * rpc;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + static_cast<size_t>(nst) * chunk_bytes);
+  uint64_t* empty = full + nst;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + nst);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long nchunk = (rows + rpc - 1) / rpc;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < nst; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], SSQ_WARPS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();
+  if (warp == SSQ_WARPS) {
+    if (lane == 0) {
+      long long i = 0;  // chunks issued
+      for (long long q = blockIdx.x; q < nchunk; q += gridDim.x, ++i) {
+        const int s = static_cast<int>(i % nst);
+        if (i >= nst && !mbar_wait(&empty[s], static_cast<uint32_t>((i / nst) - 1) & 1u, status, abort_flag)) break;
+        const long long r0 = q * rpc;
+        const uint32_t bytes = static_cast<uint32_t>(rows - r0 < rpc ? rows - r0 : rpc) * row_bytes;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        bulk_load_1d(ring + static_cast<size_t>(s) * chunk_bytes, reinterpret_cast<const uint8_t*>(z) + r0 * row_bytes,
+                     bytes, &full[s]);
+      }
+      // the copies still in flight land before shared memory goes away
+      int never = 0;
+      for (long long j = (i > nst ? i - nst : 0); j < i; ++j)
+        mbar_wait(&full[j % nst], static_cast<uint32_t>(j / nst) & 1u, nullptr, &never, 100000000ull);
+    }
+  } else {
+    const int nva = wa / 8, nv = (wa + ws) / 8;
+    long long i = 0;
+    for (long long q = blockIdx.x; q < nchunk; q += gridDim.x, ++i) {
+      const int s = static_cast<int>(i % nst);
+      if (!mbar_wait(&full[s], static_cast<uint32_t>(i / nst) & 1u, status, abort_flag)) break;
+      const long long r0 = q * rpc;
+      const int nr = static_cast<int>(rows - r0 < rpc ? rows - r0 : rpc);
+      for (int r = warp; r < nr; r += SSQ_WARPS) {
+        const uint32_t base = smem_u32(ring + static_cast<size_t>(s) * chunk_bytes + static_cast<size_t>(r) * row_bytes);
+        float sa = 0.f, ss = 0.f;
+#pragma unroll 4
+        for (int v = lane; v < nv; v += 32) {
+          const float4 f = lds_f4(base + 16u * v);
+          const uint32_t u[4] = {__float_as_uint(f.x), __float_as_uint(f.y), __float_as_uint(f.z), __float_as_uint(f.w)};
+          float acc = 0.f;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc = fmaf(bf16lo(u[k]), bf16lo(u[k]), fmaf(bf16hi(u[k]), bf16hi(u[k]), acc));
+          if (v < nva) sa += acc;
+          else ss += acc;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          sa += __shfl_xor_sync(0xffffffffu, sa, o);
+          ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        }
+        if (lane == 0) ssq[r0 + r] = make_float2(sa, ss);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+  }
+}
+
 // w_out[n, k] = w[n, k] * beta(k), 8 bf16 per thread, grid-stride.
 __global__ void __launch_bounds__(256) scale_cols_kernel(const uint4* __restrict__ w, uint4* __restrict__ w_out,
                                                          long long n_vec, int row_vecs, int wa,
@@ -368,8 +452,22 @@ __global__ void __launch_bounds__(256) scale_cols_kernel(const uint4* __restrict
 
 }  // namespace
 
-cudaError_t launch_row_ssq(const void* z, long long rows, int w_attn, int w_ssm, float2* ssq, cudaStream_t st) {
+cudaError_t launch_row_ssq(const void* z, long long rows, int w_attn, int w_ssm, float2* ssq, cudaStream_t st,
+                           unsigned* status) {
   if (rows <= 0) return cudaSuccess;
+  const long long row_bytes = static_cast<long long>(w_attn + w_ssm) * 2;
+  if ((reinterpret_cast<uintptr_t>(z) & 15) == 0 && row_bytes % 16 == 0 && row_bytes <= SSQ_RING / 2) {
+    // chunks of up to 48 KB (at most 8 rows, one per reducing warp), as many as the ring holds
+    const int rpc = static_cast<int>(std::max<long long>(1, std::min<long long>(SSQ_WARPS, 49152 / row_bytes)));
+    const int nst = static_cast<int>(std::min<long long>(8, SSQ_RING / (rpc * row_bytes)));
+    const size_t smem = static_cast<size_t>(nst) * rpc * row_bytes + 2 * nst * 8 + 16;
+    static std::atomic<uint64_t> attr_done{0};
+    if (cudaError_t e = smem_attr_once(row_ssq_bulk_kernel, SSQ_RING + 2 * 8 * 8 + 16, attr_done)) return e;
+    const long long nchunk = (rows + rpc - 1) / rpc;
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(nchunk, num_sms()));
+    return launch(row_ssq_bulk_kernel, dim3(grid), dim3((SSQ_WARPS + 1) * 32), smem, st,
+                  static_cast<const __nv_bfloat16*>(z), rows, w_attn, w_ssm, rpc, nst, ssq, status);
+  }
   const int per_lane = ((w_attn + w_ssm) / 8 + 31) / 32;
   const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
   const __nv_bfloat16* zz = static_cast<const __nv_bfloat16*>(z);
