@@ -320,7 +320,11 @@ hymba_status_t run_layer(const void* x, const void* meta, const hymba_weights_t&
     f.b_dt = w.b_dt;
     f.dt_rank = c.dt_rank;
     f.mgram = dt;   // unused as dt when fused
-    if (hy::scan_tc_fuses_dt(f)) sd = f;
+    // Not for a prefixed call with d_state 128: the tensor-core scan started after the meta
+    // rows from a stored state gave wrong outputs in a few rows of its first block,
+    // intermittently, which shows a premature read that is not yet found; such a call takes
+    // dt_proj as a GEMM and the CUDA-core scan instead.
+    if (!(lo.prefix && c.d_state == 128) && hy::scan_tc_fuses_dt(f)) sd = f;
   }
   const bool fused_dt = sd.dt_low != nullptr;
   // bf16: the branch norm is fused into out_proj -- the rows of Z are not rewritten;
