@@ -147,7 +147,7 @@ def stage_bound(stage: str, s: synth.LayerShape, work=None, peaks=None) -> str:
 
 KERNEL_NAMES = {"in_proj": "gemm_bf16_tc, tcgen05", "x_proj": "gemm_bf16_tc, tcgen05",
                 "dt_proj": "gemm_bf16_tc, tcgen05", "attention": "attn_fwd_tc2, tcgen05",
-                "branch_norm": "row_ssq_kernel + scale_cols_kernel",
+                "branch_norm": "row_ssq_bulk_kernel + scale_cols_kernel",
                 "out_proj": "gemm_bf16_tc, tcgen05, two accumulators"}
 
 PROFILE_COMMON = ("hybrid_attention_ssm_hymba_b200/csrc/hy_common.cuh",
