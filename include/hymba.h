@@ -312,6 +312,9 @@ HYMBA_API hymba_status_t hymba_meta_prefix(const void* meta_in, const hymba_weig
  * copied into each sequence's K/V (kv_out for a producing layer), and out [B, T, d]
  * receives the record's meta rows and the computed user rows.  Other arguments as in
  * hymba_layer_fwd (kv_in for a consuming layer: the producer's kv_out of its prefixed call).
+ * With d_state 128 the scan of such a call runs on the CUDA cores after a separate dt_proj
+ * GEMM, not in the tensor-core scan with the fused dt projection (that kernel, started from
+ * a stored state, was seen to write a few wrong rows of its first block intermittently).
  */
 HYMBA_API hymba_status_t hymba_layer_fwd_prefixed(const void* x, const void* prefix, const hymba_weights_t* w,
                                         const hymba_cfg_t* cfg, const void* kv_in, void* kv_out, void* out,
